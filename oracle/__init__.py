@@ -1,0 +1,10 @@
+"""Float64 CPU oracle for the gain-weighted residual memory scan.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and
+bench.py's CPU baseline, never by the product package.  See ``oracle.scan``
+for what it computes, the readings it takes and the pins that hold it.
+"""
+
+from .scan import decode_step, diag_update, kalman_update, scan_delta, scan_kalman_diag, scan_kalman_full
+
+__all__ = ["scan_delta", "scan_kalman_full", "scan_kalman_diag", "decode_step", "kalman_update", "diag_update"]
