@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Throughput of the gain-weighted residual memory scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kdn|reference]
+
+One step = one pass of the scan (every stage of the path: staging, gates,
+gains, intra-chunk solves, output, state write-back) over one batch of
+synthetic input resident in HBM.  The headline workload is the diagonal-Kalman
+language-model layer (B=8, H=16, L=8192, d_k=d_v=128, bf16 inputs, fp32
+state): the largest d=128 scan configuration.  The same line also reports the
+other layer workloads (delta rule at d=128 and d=64, full Kalman at d=128) and
+the decode step in ``also``.
+
+Metric: scan tokens/s per layer (B*H*L / time).  Time is measured on the
+device with CUDA events on the launching stream, after W warm-up steps, as the
+max over ranks.  Inputs (about 1.1 GB per step) are larger than the 126 MB L2,
+so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own batch of the same shape (heads
+are independent: weak scaling, no collective on the data path); the value is
+the tokens all ranks processed divided by the slowest rank's time.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only) and prints the same line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_decode_inputs, make_scan_inputs  # noqa: E402
+
+HEADLINE = "kalman_diag_d128"
+SECONDARY = ["gdn_d128", "kalman_full_d128", "gdn_d64"]
+DECODE = ["decode_delta", "decode_diag"]
+METRIC = "scan tokens/s per layer (B*H*L/time) at d=128"
+
+
+# ----------------------------------------------------------------------------- roofline bookkeeping
+
+
+def algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
+    """Bytes one scan must move: q, k, v in, o out, per-token scalars, m out, state in and out."""
+    tok = w.B * w.H * w.L
+    io = tok * ((2 * w.dk + w.dv) * in_bytes + w.dv * out_bytes + 4)  # + m
+    scalars = {"delta": 8, "kalman_diag": 8, "kalman_full": 8}[w.variant]  # beta|r and a
+    state = w.B * w.H * w.dk * w.dv * 4 * 2
+    if w.variant == "kalman_full":
+        state += w.B * w.H * w.dk * w.dk * 4 * 2
+    elif w.variant == "kalman_diag":
+        state += w.B * w.H * w.dk * 4 * 2
+    return io + tok * scalars + state
+
+
+def decode_bytes(w, in_bytes=2, out_bytes=2) -> int:
+    n = w.B * w.H
+    per = (2 * w.dk + w.dv) * in_bytes + w.dv * out_bytes + 4 + 8 + w.dk * w.dv * 4 * 2
+    if w.variant == "kalman_diag":
+        per += w.dk * 4 * 2
+    return n * per
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, max_mhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                max_mhz = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- device timing
+
+
+def _barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_device(fn, steps, warmup, dist_on, clocks=None):
+    """Mean ms per call of ``fn`` on the current stream, max over ranks."""
+    for _ in range(warmup):
+        fn()
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    ctx = clocks if clocks is not None else _NullCtx()
+    with ctx:
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+    _barrier(dist_on)
+    return _max_over_ranks(start.elapsed_time(end) / steps, dist_on)
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+# ----------------------------------------------------------------------------- workloads
+
+
+def scan_closure(w, x, kdn):
+    """A zero-argument step for workload ``w`` on resident inputs ``x``; returns (fn, outputs)."""
+    B, H, dk, dv = w.B, w.H, w.dk, w.dv
+    dev = x["q"].device
+    S = torch.zeros(B, H, dk, dv, device=dev)
+    o = torch.empty(B, H, w.L, dv, dtype=x["q"].dtype, device=dev)
+    m = torch.empty(B, H, w.L, device=dev)
+    ws = torch.empty(kdn.workspace_bytes(w.variant, B, H, w.L, dk, dv), dtype=torch.uint8, device=dev)
+    outs = {"o": o, "m": m}
+    if w.variant == "delta":
+        def fn():
+            kdn.scan_delta(x["q"], x["k"], x["v"], x["beta"], a=x["a"], S=S, o=o, m=m, workspace=ws)
+        return fn, outs
+    if w.variant == "kalman_full":
+        P = torch.eye(dk, device=dev).repeat(B, H, 1, 1)
+
+        def fn():
+            kdn.scan_kalman_full(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, P=P, o=o, m=m,
+                                 workspace=ws)
+        return fn, outs
+    p = torch.ones(B, H, dk, device=dev)
+
+    def fn():
+        kdn.scan_kalman_diag(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, p=p, o=o, m=m, workspace=ws)
+    return fn, outs
+
+
+def scan_plan(w):
+    from delta_rule_recurrent_scan_b200 import kdn
+    return kdn.plan(w.variant, w.B, w.H, w.L, w.dk, w.dv,
+                    in_dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+
+
+def bench_scan(w, steps, warmup, dist_on, rank, world, clocks=None):
+    from delta_rule_recurrent_scan_b200 import kdn
+    x = make_scan_inputs(w, seed=rank, device="cuda")
+    fn, _ = scan_closure(w, x, kdn)
+    ms = time_device(fn, steps, warmup, dist_on, clocks)
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": scan_plan(w)["launches"] * steps}
+
+
+def bench_e2e(w, steps, warmup, dist_on, rank, world):
+    """Through the public API with host buffers: pinned host inputs -> device, scan, outputs -> host."""
+    from delta_rule_recurrent_scan_b200 import kdn
+    xd = make_scan_inputs(w, seed=rank, device="cuda")
+    host = {k: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
+    dev = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
+    del xd
+    fn_dev, outs = scan_closure(w, dev, kdn)
+    o_host = torch.empty(outs["o"].shape, dtype=outs["o"].dtype).pin_memory()
+    m_host = torch.empty(outs["m"].shape).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if isinstance(v, torch.Tensor))
+    d2h = o_host.numel() * o_host.element_size() + m_host.numel() * 4
+
+    def step():
+        for k, v in host.items():
+            if isinstance(v, torch.Tensor):
+                dev[k].copy_(v, non_blocking=True)
+        fn_dev()
+        o_host.copy_(outs["o"], non_blocking=True)
+        m_host.copy_(outs["m"], non_blocking=True)
+
+    ms = time_device(step, steps, warmup, dist_on)
+    return {"value": w.tokens * world / (ms * 1e-3), "ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def bench_decode(w, steps, warmup, dist_on, rank, world):
+    from delta_rule_recurrent_scan_b200 import kdn
+    n_inputs = 8  # distinct token batches cycled through (inputs are per call; the 512 MB state dominates)
+    x = make_decode_inputs(w, steps=n_inputs, seed=rank, device="cuda")
+    S = torch.zeros(w.B, w.H, w.dk, w.dv, device="cuda")
+    p = torch.ones(w.B, w.H, w.dk, device="cuda")
+    o = torch.empty(w.B, w.H, w.dv, dtype=x["q"].dtype, device="cuda")
+    m = torch.empty(w.B, w.H, device="cuda")
+    it = [0]
+
+    def fn():
+        t = it[0] % n_inputs
+        it[0] += 1
+        kdn.decode_step(w.variant, x["q"][t], x["k"][t], x["v"][t], S, beta=x["beta"][t], a=x["a"][t], r=x["r"][t],
+                        qn=x["qn"], p=p if w.variant == "kalman_diag" else None, o=o, m=m)
+    ms = time_device(fn, steps, warmup, dist_on)
+    return {"ms": ms, "value": w.B * w.H * world / (ms * 1e-3), "launches": steps}
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+
+
+def cpu_baseline(w, heads=16, seconds_hint=None):
+    """The float64 oracle, as it stands, on a bounded sample: ``heads`` heads over the full sequence."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import oracle
+
+    B = max(1, heads // w.H)
+    H = min(w.H, heads)
+    x = make_scan_inputs(w, seed=0, device="cpu", B=B, H=H)
+    np_ = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    t0 = time.perf_counter()
+    if w.variant == "delta":
+        oracle.scan_delta(np_["q"], np_["k"], np_["v"], np_["beta"], a=np_["a"])
+    elif w.variant == "kalman_full":
+        oracle.scan_kalman_full(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+    else:
+        oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+    dt = time.perf_counter() - t0
+    tokens = B * H * w.L
+    del np
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{B * H} of {w.B * w.H} heads x full L={w.L} ({tokens} tokens, {dt:.1f} s, float64 NumPy, "
+                      f"one thread)"}
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="kdn", choices=["kdn", "reference"])
+    ap.add_argument("--no-also", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return reference_arm(args, w, rank, world)
+
+    torch.cuda.set_device(local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+
+    from delta_rule_recurrent_scan_b200 import kdn
+
+    kdn.lib()  # fail loudly if the library is missing
+    peak, peak_kind = measured_peaks()
+    clocks = ClockSampler(local)
+    head = bench_scan(w, args.steps, args.warmup, dist_on, rank, world, clocks=clocks)
+    ms = head["ms"]
+    alg = algorithmic_bytes(w)
+    achieved = alg / (ms * 1e-3) / 1e9
+    plan = scan_plan(w)
+    torch.cuda.empty_cache()
+
+    e2e = bench_e2e(w, min(args.steps, 5), 3, dist_on, rank, world)
+    torch.cuda.empty_cache()
+
+    also = []
+    if not args.no_also:
+        for name in SECONDARY:
+            if name == args.workload:
+                continue
+            sw = WORKLOADS[name]
+            r = bench_scan(sw, max(3, args.steps // 4), 3, dist_on, rank, world)
+            ab = algorithmic_bytes(sw)
+            also.append({"workload": name, "variant": sw.variant, "value": r["value"], "unit": "tokens/s",
+                         "ms_per_step": r["ms"], "gpu_launches": r["launches"],
+                         "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
+            del r
+            torch.cuda.empty_cache()
+        for name in DECODE:
+            dw = WORKLOADS[name]
+            r = bench_decode(dw, 64, 8, dist_on, rank, world)
+            ab = decode_bytes(dw)
+            also.append({"workload": name, "variant": dw.variant, "value": r["value"], "unit": "states/s",
+                         "ms_per_step": r["ms"], "gpu_launches": r["launches"],
+                         "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
+            torch.cuda.empty_cache()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": head["value"],
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if plan["arith"] == "bf16-tc" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "variant": w.variant, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk,
+                       "dv": w.dv, "in_dtype": w.dtype, "state": "fp32", "seed": "rank",
+                       "l2": f"inputs larger than L2 ({alg / 1e9:.2f} GB per step), no flush",
+                       "parallelism": f"dp{world} (independent heads, no collective)",
+                       "kernel_path": plan},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                         "algorithmic_bytes_per_launch": alg, "kernel": plan["kernel"],
+                         "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events"},
+            "e2e": {"value": e2e["value"], "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                    "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"]},
+            "gpu_launches": head["launches"],
+            "clocks": clocks.summary(),
+            "also": also,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def reference_arm(args, w, rank, world):
+    """The float64 CPU oracle as the reference arm: rank 0 only, bounded sample per step."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+
+    heads, Ls = 2, w.L
+    B, H = 1, heads
+    x = make_scan_inputs(w, seed=0, device="cpu", B=B, H=H, L=Ls)
+    np_ = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+    def step():
+        if w.variant == "delta":
+            oracle.scan_delta(np_["q"], np_["k"], np_["v"], np_["beta"], a=np_["a"])
+        elif w.variant == "kalman_full":
+            oracle.scan_kalman_full(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+        else:
+            oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+
+    for _ in range(min(args.warmup, 1)):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    tokens = B * H * Ls
+    value = tokens / dt
+    sample = f"{B * H} of {w.B * w.H} heads x full L={Ls} per step ({tokens} tokens), float64 NumPy, one thread"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "variant": w.variant, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del np
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

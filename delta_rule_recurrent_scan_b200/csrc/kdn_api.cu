@@ -1,0 +1,281 @@
+// C-ABI layer of libkdn: argument validation, workspace layout, dispatch.
+//
+// Declared in include/kdn.h.  Every entry point validates its arguments on the
+// host (enqueuing nothing on failure), clears the device status word in the
+// caller's workspace, and enqueues its kernels on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <string>
+
+#include "../../include/kdn.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "chunk.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kdn_status fail(kdn_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+kdn_status ok() {
+  g_last_error.clear();
+  return KDN_OK;
+}
+
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// A device-accessible pointer: device or managed memory.
+kdn_status check_ptr(const void* p, const char* name, size_t align, bool allow_null) {
+  if (p == nullptr) {
+    if (allow_null) return KDN_OK;
+    return fail(KDN_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  }
+  if (reinterpret_cast<uintptr_t>(p) % align != 0)
+    return fail(KDN_ERR_INVALID_ARG, std::string(name) + " is not " + std::to_string(align) + "-byte aligned");
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(KDN_ERR_INVALID_ARG, std::string(name) + ": cudaPointerGetAttributes failed (" +
+                                         cudaGetErrorString(e) + ")");
+  }
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(KDN_ERR_INVALID_ARG, std::string(name) + " is not a device pointer");
+  return KDN_OK;
+}
+
+// Launch on the device that owns the state buffer (the library links its own
+// CUDA runtime, whose current device need not be the caller's).
+kdn_status use_device_of(const void* p) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(KDN_ERR_INVALID_ARG, "cannot query the device of the state buffer");
+  }
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != attr.device) {
+    cudaError_t e = cudaSetDevice(attr.device);
+    if (e != cudaSuccess) return fail(KDN_ERR_CUDA, std::string("cudaSetDevice: ") + cudaGetErrorString(e));
+  }
+  return KDN_OK;
+}
+
+#define KDN_TRY(expr)                 \
+  do {                                \
+    kdn_status _s = (expr);           \
+    if (_s != KDN_OK) return _s;      \
+  } while (0)
+
+kdn_status check_dims(const kdn_dims* d) {
+  if (d == nullptr) return fail(KDN_ERR_INVALID_ARG, "dims is NULL");
+  if (d->B < 1 || d->H < 1 || d->L < 0)
+    return fail(KDN_ERR_INVALID_ARG, "B and H must be >= 1 and L >= 0");
+  if ((long long)d->B * d->H * (long long)(d->L > 0 ? d->L : 1) > (1LL << 40))
+    return fail(KDN_ERR_INVALID_ARG, "B*H*L too large");
+  if (d->in_dtype != KDN_F32 && d->in_dtype != KDN_BF16) return fail(KDN_ERR_INVALID_ARG, "bad in_dtype");
+  if (d->out_dtype != KDN_F32 && d->out_dtype != KDN_BF16) return fail(KDN_ERR_INVALID_ARG, "bad out_dtype");
+  if (!supported_dim(d->dk) || !supported_dim(d->dv))
+    return fail(KDN_ERR_UNSUPPORTED, "dk and dv must be 16, 32, 64 or 128");
+  if (d->chunk != 0 && d->chunk != 16 && d->chunk != 32 && d->chunk != 64)
+    return fail(KDN_ERR_UNSUPPORTED, "chunk must be 0, 16, 32 or 64");
+  return KDN_OK;
+}
+
+constexpr size_t kStatusBytes = 256;
+
+size_t gains_bytes(const kdn_dims* d) { return (size_t)d->B * d->H * (size_t)d->L * d->dk * sizeof(float); }
+
+kdn_status common_checks(kdn_variant var, const kdn_dims* d, const void* q, const void* k, const void* v,
+                         const float* S, const void* o, const float* m, const void* ws, size_t ws_bytes) {
+  KDN_TRY(check_dims(d));
+  const bool any = d->L > 0;
+  KDN_TRY(check_ptr(S, "S", 16, false));
+  KDN_TRY(check_ptr(q, "q", 16, !any));
+  KDN_TRY(check_ptr(k, "k", 16, !any));
+  KDN_TRY(check_ptr(v, "v", 16, !any));
+  KDN_TRY(check_ptr(o, "o", 16, !any));
+  KDN_TRY(check_ptr(m, "m", 4, true));
+  KDN_TRY(check_ptr(ws, "workspace", 256, false));
+  const size_t need = kdn_workspace_bytes(var, d);
+  if (ws_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(ws_bytes) + " < required " +
+                                         std::to_string(need));
+  return use_device_of(S);
+}
+
+kdn_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(KDN_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+int kdn_api_version(void) { return KDN_API_VERSION; }
+
+const char* kdn_status_string(kdn_status s) {
+  switch (s) {
+    case KDN_OK: return "KDN_OK";
+    case KDN_ERR_INVALID_ARG: return "KDN_ERR_INVALID_ARG";
+    case KDN_ERR_UNSUPPORTED: return "KDN_ERR_UNSUPPORTED";
+    case KDN_ERR_CUDA: return "KDN_ERR_CUDA";
+    case KDN_ERR_NUMERIC: return "KDN_ERR_NUMERIC";
+    case KDN_ERR_TIMEOUT: return "KDN_ERR_TIMEOUT";
+  }
+  return "KDN_UNKNOWN_STATUS";
+}
+
+const char* kdn_last_error(void) { return g_last_error.c_str(); }
+
+size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
+  if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
+  if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
+  size_t n = kStatusBytes;
+  switch (variant) {
+    case KDN_DELTA: break;
+    case KDN_KALMAN_DIAG:
+    case KDN_KALMAN_FULL: n += gains_bytes(dims); break;
+    default: return 0;
+  }
+  return (n + 255) / 256 * 256;
+}
+
+kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, const char** kernel,
+                    const char** arith) {
+  KDN_TRY(check_dims(dims));
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_FULL)
+    return fail(KDN_ERR_INVALID_ARG, "bad variant");
+  int n = 0;
+  const char* name = "";
+  const char* ar = "f32";
+  if (dims->L == 0) {
+    n = 0, name = "none";
+  } else if (kdn::chunk_supported(variant, *dims)) {
+    kdn::chunk_plan(variant, *dims, &n, &name, &ar);
+  } else if (variant == KDN_DELTA) {
+    n = 1, name = "seq_scan_kernel";
+  } else {
+    n = 2, name = "seq_scan_kernel";
+  }
+  if (launches) *launches = n;
+  if (kernel) *kernel = name;
+  if (arith) *arith = ar;
+  return ok();
+}
+
+kdn_status kdn_read_device_status(const void* workspace, int* status_out, void* stream) {
+  if (status_out == nullptr) return fail(KDN_ERR_INVALID_ARG, "status_out is NULL");
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  KDN_TRY(use_device_of(workspace));
+  unsigned word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "reading the device status");
+  *status_out = (word & kdn::kStatusNumeric) ? KDN_ERR_NUMERIC : (word & kdn::kStatusTimeout) ? KDN_ERR_TIMEOUT : KDN_OK;
+  return ok();
+}
+
+kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
+                          const float* a, float* S, void* o, float* m, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  KDN_TRY(common_checks(KDN_DELTA, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(beta, "beta", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "clearing the status word");
+  if (!any) return ok();
+  const int BH = dims->B * dims->H;
+  if (kdn::chunk_supported(KDN_DELTA, *dims)) {
+    kdn::ChunkArgs c{};
+    c.q = q, c.k = k, c.v = v, c.beta = beta, c.a = a, c.S = S, c.o = o, c.m = m;
+    c.out_dtype = dims->out_dtype, c.BH = BH, c.L = dims->L;
+    c.status = reinterpret_cast<unsigned*>(workspace);
+    return cuda_status(kdn::launch_chunk(KDN_DELTA, *dims, c, st), "chunked delta scan launch");
+  }
+  kdn::SeqScanArgs s{q, k, v, dims->in_dtype, dims->out_dtype, beta, a, nullptr, S, o, m, BH, dims->L};
+  return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, s, st), "delta scan launch");
+}
+
+static kdn_status kalman_scan(kdn_variant var, const kdn_dims* dims, const void* q, const void* k, const void* v,
+                              const float* a, const float* r, const float* qn, float qn_scalar, float* S, float* P,
+                              void* o, float* m, void* workspace, size_t workspace_bytes, void* stream) {
+  KDN_TRY(common_checks(var, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(P, var == KDN_KALMAN_FULL ? "P" : "p", var == KDN_KALMAN_FULL ? 16 : 4, false));
+  KDN_TRY(check_ptr(r, "r", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(qn, "qn", 4, true));
+  if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "clearing the status word");
+  if (!any) return ok();
+  const int BH = dims->B * dims->H;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  if (kdn::chunk_supported(var, *dims)) {
+    kdn::ChunkArgs c{};
+    c.q = q, c.k = k, c.v = v, c.a = a, c.r = r, c.qn = qn, c.qn_scalar = qn_scalar, c.S = S, c.o = o, c.m = m;
+    c.P = P, c.out_dtype = dims->out_dtype, c.BH = BH, c.L = dims->L, c.status = status;
+    c.workspace = reinterpret_cast<char*>(workspace) + kStatusBytes;
+    return cuda_status(kdn::launch_chunk(var, *dims, c, st), "chunked Kalman scan launch");
+  }
+  float* gains = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + kStatusBytes);
+  kdn::GainArgs g{k, dims->in_dtype, a, r, qn, qn_scalar, var == KDN_KALMAN_FULL ? P : nullptr,
+                  var == KDN_KALMAN_DIAG ? P : nullptr, gains, status, BH, dims->L};
+  e = var == KDN_KALMAN_FULL ? kdn::launch_kalman_full_gains(dims->dk, g, st)
+                             : kdn::launch_kalman_diag_gains(dims->dk, g, st);
+  if (e != cudaSuccess) return cuda_status(e, "Kalman gain launch");
+  kdn::SeqScanArgs s{q, k, v, dims->in_dtype, dims->out_dtype, nullptr, a, gains, S, o, m, BH, dims->L};
+  return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, s, st), "Kalman scan launch");
+}
+
+kdn_status kdn_scan_kalman_full(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* a,
+                                const float* r, const float* qn, float qn_scalar, float* S, float* P, void* o,
+                                float* m, void* workspace, size_t workspace_bytes, void* stream) {
+  return kalman_scan(KDN_KALMAN_FULL, dims, q, k, v, a, r, qn, qn_scalar, S, P, o, m, workspace, workspace_bytes,
+                     stream);
+}
+
+kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* a,
+                                const float* r, const float* qn, float qn_scalar, float* S, float* p, void* o,
+                                float* m, void* workspace, size_t workspace_bytes, void* stream) {
+  return kalman_scan(KDN_KALMAN_DIAG, dims, q, k, v, a, r, qn, qn_scalar, S, p, o, m, workspace, workspace_bytes,
+                     stream);
+}
+
+kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype, kdn_dtype out_dtype,
+                           const void* q, const void* k, const void* v, const float* beta, const float* a,
+                           const float* r, float qn_scalar, float* S, float* p, void* o, float* m, void* stream) {
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG)
+    return fail(KDN_ERR_UNSUPPORTED, "decode supports KDN_DELTA and KDN_KALMAN_DIAG");
+  kdn_dims d{B, H, 1, dk, dv, 0, in_dtype, out_dtype};
+  KDN_TRY(check_dims(&d));
+  KDN_TRY(check_ptr(q, "q", 16, false));
+  KDN_TRY(check_ptr(k, "k", 16, false));
+  KDN_TRY(check_ptr(v, "v", 16, false));
+  KDN_TRY(check_ptr(S, "S", 16, false));
+  KDN_TRY(check_ptr(o, "o", 16, false));
+  KDN_TRY(check_ptr(m, "m", 4, true));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  if (variant == KDN_DELTA) {
+    KDN_TRY(check_ptr(beta, "beta", 4, false));
+  } else {
+    KDN_TRY(check_ptr(r, "r", 4, false));
+    KDN_TRY(check_ptr(p, "p", 4, false));
+    if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  }
+  KDN_TRY(use_device_of(S));
+  kdn::DecodeArgs args{q, k, v, in_dtype, out_dtype, beta, a, r, qn_scalar, S, p, o, m, B * H};
+  return cuda_status(kdn::launch_decode(dk, dv, variant == KDN_KALMAN_DIAG, args, (cudaStream_t)stream),
+                     "decode launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// Internal launch interface between the C-ABI layer (kdn_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kdn {
+
+// Per-token S-side scan: o, m and the final S for gains g_t given either as
+// beta_t k_t (delta rule) or read from a precomputed fp32 gain array.
+struct SeqScanArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_dtype;
+  int out_dtype;
+  const float* beta;   // delta: [BH, L]
+  const float* a;      // [BH, L] or nullptr
+  const float* gains;  // Kalman: [BH, L, dk] fp32, or nullptr for the delta rule
+  float* S;            // [BH, dk, dv]
+  void* o;             // [BH, L, dv]
+  float* m;            // [BH, L] or nullptr
+  int BH;
+  int L;
+};
+
+// Per-token Kalman gain recursions (covariance side; independent of v and S).
+struct GainArgs {
+  const void* k;
+  int in_dtype;
+  const float* a;   // [BH, L] or nullptr
+  const float* r;   // [BH, L]
+  const float* qn;  // [BH, L] or nullptr
+  float qn_scalar;
+  float* P;         // full: [BH, dk, dk]
+  float* p;         // diagonal: [BH, dk]
+  float* gains;     // out: [BH, L, dk]
+  unsigned* status;
+  int BH;
+  int L;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_dtype;
+  int out_dtype;
+  const float* beta;  // delta: [BH]
+  const float* a;     // [BH] or nullptr
+  const float* r;     // diagonal: [BH]
+  float qn_scalar;
+  float* S;           // [BH, dk, dv]
+  float* p;           // diagonal: [BH, dk]
+  void* o;            // [BH, dv]
+  float* m;           // [BH] or nullptr
+  int BH;
+};
+
+cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream);
+cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream);
+cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream);
+cudaError_t launch_decode(int dk, int dv, bool diag, const DecodeArgs& args, cudaStream_t stream);
+
+}  // namespace kdn

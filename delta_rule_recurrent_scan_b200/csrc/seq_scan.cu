@@ -1,0 +1,311 @@
+// Per-token (sequential) scan kernels on the fp32 CUDA cores.
+//
+// These are the exact token-by-token recurrences, one CTA per head with the
+// state held in registers; they serve every shape the library accepts and are
+// the reference the chunked tensor-core kernels are tested against.
+//
+// S-side (all variants), per token t with gain g_t
+//   (A Hippocampus for Linear Attention, section 3.3 Eq. (5)-(6), section 3.5):
+//     y_k = S^T k_t, y_q = S^T q_t                 (one reduction round)
+//     e_t = v_t - a_t y_k
+//     o_t = S_t^T q_t = a_t y_q + (g_t . q_t) e_t
+//     S  <- a_t S + g_t e_t^T
+//     m_t = ||g_t|| ||e_t||
+// Covariance side (Kalman Delta Networks, Abstract; DeltaNet-PC Eq. (7)):
+//     full  P^- = a^2 P + Qn I, u = P^- k, s = k.u + r, g = u / s,
+//           P <- P^- - u u^T / s
+//     diag  p^- = a^2 p + Qn, s = sum p^- k^2 + r, g = p^- k / s,
+//           p <- p^- r / (r + p^- k^2)
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kdn {
+
+constexpr int kTokBlock = 16;  // tokens staged in shared memory at a time
+
+template <int DK, int DV, bool kGainsFromWs>
+__global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_kernel(SeqScanArgs args) {
+  using Lay = RowBlockLayout<DK, DV>;
+  constexpr int NT = Lay::kThreads, CG = Lay::kColGroups, RG = Lay::kRowGroups, RPT = Lay::kRowsPerThread;
+  constexpr int NW = NT / 32;
+  constexpr int DVW = (DV + 31) / 32 * 32;
+  static_assert(NT >= DVW, "phase B needs whole warps over d_v");
+
+  __shared__ float k_s[kTokBlock][DK], q_s[kTokBlock][DK], g_s[kTokBlock][DK];
+  __shared__ float v_s[kTokBlock][DV];
+  __shared__ float a_s[kTokBlock], b_s[kTokBlock], gq_s[kTokBlock], gn_s[kTokBlock];
+  __shared__ __align__(16) float red[RG][2][DV];
+  __shared__ float e_s[DV];
+  __shared__ float ered[DVW / 32];
+
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid % CG, rg = tid / CG;
+  const int L = args.L;
+  const size_t tok0 = (size_t)bh * L;
+
+  float S[RPT][4];
+  float* Sg = args.S + (size_t)bh * DK * DV;
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float4 x = *reinterpret_cast<const float4*>(Sg + (size_t)(rg + i * RG) * DV + cg * 4);
+    S[i][0] = x.x, S[i][1] = x.y, S[i][2] = x.z, S[i][3] = x.w;
+  }
+
+  for (int t0 = 0; t0 < L; t0 += kTokBlock) {
+    const int nt = min(kTokBlock, L - t0);
+    __syncthreads();
+    for (int idx = tid; idx < nt * DK; idx += NT) {
+      const int j = idx / DK, i = idx % DK;
+      const size_t off = (tok0 + t0 + j) * DK + i;
+      k_s[j][i] = load_elem(args.k, off, args.in_dtype);
+      q_s[j][i] = load_elem(args.q, off, args.in_dtype);
+      if constexpr (kGainsFromWs) g_s[j][i] = args.gains[off];
+    }
+    for (int idx = tid; idx < nt * DV; idx += NT) {
+      const int j = idx / DV, i = idx % DV;
+      v_s[j][i] = load_elem(args.v, (tok0 + t0 + j) * DV + i, args.in_dtype);
+    }
+    for (int j = tid; j < nt; j += NT) {
+      a_s[j] = args.a ? args.a[tok0 + t0 + j] : 1.f;
+      b_s[j] = kGainsFromWs ? 0.f : args.beta[tok0 + t0 + j];
+    }
+    __syncthreads();
+    for (int j = warp; j < nt; j += NW) {
+      float sq = 0.f, sn = 0.f;
+      for (int i = lane; i < DK; i += 32) {
+        const float g = kGainsFromWs ? g_s[j][i] : b_s[j] * k_s[j][i];
+        sq = fmaf(g, q_s[j][i], sq);
+        sn = fmaf(g, g, sn);
+      }
+      sq = warp_sum(sq);
+      sn = warp_sum(sn);
+      if (lane == 0) gq_s[j] = sq, gn_s[j] = sn;
+    }
+    __syncthreads();
+
+    for (int j = 0; j < nt; ++j) {
+      const float a = a_s[j];
+      // phase A: partial S^T k and S^T q over this thread's rows
+      float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int row = rg + i * RG;
+        const float kr = k_s[j][row], qr = q_s[j][row];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          pk[c] = fmaf(S[i][c], kr, pk[c]);
+          pq[c] = fmaf(S[i][c], qr, pq[c]);
+        }
+      }
+      *reinterpret_cast<float4*>(&red[rg][0][cg * 4]) = make_float4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<float4*>(&red[rg][1][cg * 4]) = make_float4(pq[0], pq[1], pq[2], pq[3]);
+      __syncthreads();
+      // phase B: residual, output, residual norm
+      if (tid < DVW) {
+        float e = 0.f;
+        if (tid < DV) {
+          float yk = 0.f, yq = 0.f;
+#pragma unroll
+          for (int r = 0; r < RG; ++r) yk += red[r][0][tid], yq += red[r][1][tid];
+          e = v_s[j][tid] - a * yk;
+          store_elem(args.o, (tok0 + t0 + j) * DV + tid, fmaf(a, yq, gq_s[j] * e), args.out_dtype);
+          e_s[tid] = e;
+        }
+        const float es = warp_sum(e * e);
+        if (lane == 0) ered[warp] = es;
+      }
+      __syncthreads();
+      // phase C: rank-1 write
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int row = rg + i * RG;
+        const float gr = kGainsFromWs ? g_s[j][row] : b_s[j] * k_s[j][row];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) S[i][c] = fmaf(a, S[i][c], gr * e_s[cg * 4 + c]);
+      }
+      if (tid == 0 && args.m != nullptr) {
+        float es = 0.f;
+#pragma unroll
+        for (int w = 0; w < DVW / 32; ++w) es += ered[w];
+        args.m[tok0 + t0 + j] = sqrtf(gn_s[j]) * sqrtf(es);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+    *reinterpret_cast<float4*>(Sg + (size_t)(rg + i * RG) * DV + cg * 4) = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+}
+
+template <int DK>
+__global__ void __launch_bounds__(RowBlockLayout<DK, DK>::kThreads) kalman_full_gains_kernel(GainArgs args) {
+  using Lay = RowBlockLayout<DK, DK>;
+  constexpr int NT = Lay::kThreads, CG = Lay::kColGroups, RG = Lay::kRowGroups, RPT = Lay::kRowsPerThread;
+  constexpr int DKW = (DK + 31) / 32 * 32;
+  static_assert(NT >= DKW, "reduction needs whole warps over d_k");
+
+  __shared__ float k_s[kTokBlock][DK];
+  __shared__ float a_s[kTokBlock], qn_s[kTokBlock], r_s[kTokBlock];
+  __shared__ __align__(16) float red[RG][DK];
+  __shared__ float u_s[DK];
+  __shared__ float ured[DKW / 32];
+
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid % CG, rg = tid / CG;
+  const int L = args.L;
+  const size_t tok0 = (size_t)bh * L;
+
+  float P[RPT][4];
+  float* Pg = args.P + (size_t)bh * DK * DK;
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float4 x = *reinterpret_cast<const float4*>(Pg + (size_t)(rg + i * RG) * DK + cg * 4);
+    P[i][0] = x.x, P[i][1] = x.y, P[i][2] = x.z, P[i][3] = x.w;
+  }
+
+  for (int t0 = 0; t0 < L; t0 += kTokBlock) {
+    const int nt = min(kTokBlock, L - t0);
+    __syncthreads();
+    for (int idx = tid; idx < nt * DK; idx += NT) {
+      const int j = idx / DK, i = idx % DK;
+      k_s[j][i] = load_elem(args.k, (tok0 + t0 + j) * DK + i, args.in_dtype);
+    }
+    for (int j = tid; j < nt; j += NT) {
+      const size_t tk = tok0 + t0 + j;
+      a_s[j] = args.a ? args.a[tk] : 1.f;
+      qn_s[j] = args.qn ? args.qn[tk] : args.qn_scalar;
+      r_s[j] = args.r[tk];
+    }
+    __syncthreads();
+    for (int j = 0; j < nt; ++j) {
+      const float a2 = a_s[j] * a_s[j], qn = qn_s[j];
+      float pu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int row = rg + i * RG;
+        const float kr = k_s[j][row];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float x = fmaf(a2, P[i][c], (row == cg * 4 + c) ? qn : 0.f);
+          P[i][c] = x;
+          pu[c] = fmaf(x, kr, pu[c]);
+        }
+      }
+      *reinterpret_cast<float4*>(&red[rg][cg * 4]) = make_float4(pu[0], pu[1], pu[2], pu[3]);
+      __syncthreads();
+      if (tid < DKW) {
+        float ku = 0.f;
+        if (tid < DK) {
+          float u = 0.f;
+#pragma unroll
+          for (int r = 0; r < RG; ++r) u += red[r][tid];
+          u_s[tid] = u;
+          ku = k_s[j][tid] * u;
+        }
+        ku = warp_sum(ku);
+        if (lane == 0) ured[warp] = ku;
+      }
+      __syncthreads();
+      float s = r_s[j];
+#pragma unroll
+      for (int w = 0; w < DKW / 32; ++w) s += ured[w];
+      if (tid == 0 && !(s > 0.f && isfinite(s))) raise_status(args.status, kStatusNumeric);
+      const float inv_s = 1.f / s;
+      if (tid < DK) args.gains[(tok0 + t0 + j) * DK + tid] = u_s[tid] * inv_s;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const float ur = u_s[rg + i * RG];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) P[i][c] -= (ur * u_s[cg * 4 + c]) * inv_s;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+    *reinterpret_cast<float4*>(Pg + (size_t)(rg + i * RG) * DK + cg * 4) = make_float4(P[i][0], P[i][1], P[i][2], P[i][3]);
+}
+
+// One warp per head; the p recursion is sequential in t and cheap.
+template <int DK>
+__global__ void __launch_bounds__(128) kalman_diag_gains_kernel(GainArgs args) {
+  constexpr int PER = (DK + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (bh >= args.BH) return;
+  const int L = args.L;
+  const size_t tok0 = (size_t)bh * L;
+  float p[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = lane + 32 * i;
+    p[i] = c < DK ? args.p[(size_t)bh * DK + c] : 0.f;
+  }
+  for (int t = 0; t < L; ++t) {
+    const size_t tk = tok0 + t;
+    const float a = args.a ? args.a[tk] : 1.f;
+    const float qn = args.qn ? args.qn[tk] : args.qn_scalar;
+    const float r = args.r[tk];
+    float kk[PER], pp[PER], part = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int c = lane + 32 * i;
+      kk[i] = c < DK ? load_elem(args.k, tk * DK + c, args.in_dtype) : 0.f;
+      pp[i] = c < DK ? fmaf(a * a, p[i], qn) : 0.f;
+      part = fmaf(pp[i] * kk[i], kk[i], part);
+    }
+    const float s = warp_sum(part) + r;
+    if (lane == 0 && !(s > 0.f && isfinite(s))) raise_status(args.status, kStatusNumeric);
+    const float inv_s = 1.f / s;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int c = lane + 32 * i;
+      if (c < DK) {
+        args.gains[tk * DK + c] = pp[i] * kk[i] * inv_s;
+        p[i] = pp[i] * r / fmaf(pp[i] * kk[i], kk[i], r);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = lane + 32 * i;
+    if (c < DK) args.p[(size_t)bh * DK + c] = p[i];
+  }
+}
+
+#define KDN_DIMS_SWITCH(D, NAME, ...)         \
+  switch (D) {                                \
+    case 16: { constexpr int NAME = 16; __VA_ARGS__; } break;   \
+    case 32: { constexpr int NAME = 32; __VA_ARGS__; } break;   \
+    case 64: { constexpr int NAME = 64; __VA_ARGS__; } break;   \
+    case 128: { constexpr int NAME = 128; __VA_ARGS__; } break; \
+    default: return cudaErrorInvalidValue;    \
+  }
+
+cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream) {
+  if (args.BH <= 0 || args.L <= 0) return cudaSuccess;
+  KDN_DIMS_SWITCH(dk, DK, KDN_DIMS_SWITCH(dv, DV, {
+    constexpr int NT = RowBlockLayout<DK, DV>::kThreads;
+    if (args.gains != nullptr)
+      seq_scan_kernel<DK, DV, true><<<args.BH, NT, 0, stream>>>(args);
+    else
+      seq_scan_kernel<DK, DV, false><<<args.BH, NT, 0, stream>>>(args);
+  }));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream) {
+  if (args.BH <= 0 || args.L <= 0) return cudaSuccess;
+  KDN_DIMS_SWITCH(dk, DK, {
+    kalman_full_gains_kernel<DK><<<args.BH, RowBlockLayout<DK, DK>::kThreads, 0, stream>>>(args);
+  });
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream) {
+  if (args.BH <= 0 || args.L <= 0) return cudaSuccess;
+  KDN_DIMS_SWITCH(dk, DK, { kalman_diag_gains_kernel<DK><<<(args.BH + 3) / 4, 128, 0, stream>>>(args); });
+  return cudaGetLastError();
+}
+
+}  // namespace kdn

@@ -1,0 +1,165 @@
+/*
+ * kdn.h - C ABI of the B200 (sm_100a) forward scan of a recurrent
+ * associative memory written by a gain-weighted residual.
+ *
+ * Per head (b, h) the memory is a matrix S (d_k x d_v, fp32) read as
+ * o_t = S_t^T q_t.  Every entry point writes it token by token with
+ *
+ *     S_t = a_t S_{t-1} + g_t e_t^T,     e_t = v_t - (a_t S_{t-1})^T k_t,
+ *
+ * and emits the surprise score m_t = ||g_t|| ||e_t||, the Frobenius norm of
+ * the write (A Hippocampus for Linear Attention, section 3.3, Eq. (5)-(6);
+ * the decay gate and the residual against the decayed state: same page,
+ * section 3.5 "Instantiation (GDN)").  The entry points differ in the gain:
+ *
+ *   kdn_scan_delta        g_t = beta_t k_t                    (gated delta rule)
+ *   kdn_scan_kalman_full  g_t = P^- k_t / (k_t^T P^- k_t + r_t), with
+ *                         P^- = a_t^2 P + Qn_t I and P <- P^- - s_t g_t g_t^T
+ *                         (Kalman Delta Networks, Abstract; Memory by Design,
+ *                         Abstract; DeltaNet-PC, "How it works", Eq. (5)-(7))
+ *   kdn_scan_kalman_diag  the same with P = diag(p), p_i <- p^-_i r /
+ *                         (r + p^-_i k_i^2): the one-step posterior projected on
+ *                         diagonal Gaussians by mean-field VI (Kalman Delta
+ *                         Networks, Abstract)
+ *   kdn_decode_step       one token against a resident state (delta or diag)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every array argument is a DEVICE pointer (cudaMalloc, a CUDA
+ *   caching allocator, or managed memory) to a dense row-major array.  q, k,
+ *   v, o, S and P must be 16-byte aligned, the workspace 256-byte aligned, and
+ *   the fp32 per-token arrays (beta, a, r, qn, m) and p 4-byte aligned.  Host
+ *   pointers are rejected with KDN_ERR_INVALID_ARG.
+ * Ownership.  The caller owns every buffer; the library allocates nothing and
+ *   keeps no pointer after the call returns.  Scratch space is the caller's
+ *   workspace, sized by kdn_workspace_bytes().
+ * Layouts (B batch, H heads, L tokens):
+ *   q, k      [B, H, L, d_k]   in_dtype (bf16 or fp32); keys are expected
+ *                               unit-L2 (HOLA section 3.4) but not required
+ *   v         [B, H, L, d_v]   in_dtype
+ *   o         [B, H, L, d_v]   out_dtype
+ *   m         [B, H, L]        fp32, may be NULL (not written)
+ *   beta, a, r, qn [B, H, L]   fp32; a == NULL means a_t = 1; qn == NULL means
+ *                               Qn_t = qn_scalar for every token
+ *   S         [B, H, d_k, d_v] fp32, in: initial state, out: state after token L
+ *   P         [B, H, d_k, d_k] fp32 symmetric PD, in: P_0, out: P_L
+ *   p         [B, H, d_k]      fp32 positive, in: p_0, out: p_L
+ *   States are updated in place, so consecutive calls continue one scan.
+ * Streams.  ``stream`` is a cudaStream_t (NULL = legacy default stream).
+ *   Every call only enqueues work on it and returns; nothing synchronises.
+ * Errors.  Argument errors return synchronously and enqueue nothing.  A failed
+ *   launch returns KDN_ERR_CUDA.  Numeric failures found on the device (a
+ *   non-positive or non-finite innovation variance) set the status word in
+ *   the workspace, read back with kdn_read_device_status().  Nothing in the
+ *   library aborts, exits or traps.  kdn_last_error() gives a message for the
+ *   last failing call on the calling thread.
+ * Supported sizes.  d_k, d_v in {16, 32, 64, 128}; any L >= 0 (L = 0 is a
+ *   no-op); chunk 0 (library choice) or 16/32/64.
+ * Precision.  State, gains and accumulation are fp32.  Where a product runs
+ *   on the tensor cores, bf16 inputs enter it exactly and every fp32 operand
+ *   (the state, the gains, the chunk solves) is split into two bf16 terms
+ *   (hi + lo), keeping about 16 mantissa bits.
+ */
+#ifndef KDN_H_
+#define KDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDN_API_VERSION 1
+
+#if defined(__GNUC__)
+#define KDN_EXPORT __attribute__((visibility("default")))
+#else
+#define KDN_EXPORT
+#endif
+
+typedef enum kdn_status {
+  KDN_OK = 0,
+  KDN_ERR_INVALID_ARG = 1,  /* null / host / misaligned pointer, bad size or dtype */
+  KDN_ERR_UNSUPPORTED = 2,  /* valid request outside the supported sizes */
+  KDN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  KDN_ERR_NUMERIC = 4,      /* device status: non-positive / non-finite innovation variance */
+  KDN_ERR_TIMEOUT = 5       /* device status: a bounded wait gave up */
+} kdn_status;
+
+typedef enum kdn_dtype { KDN_F32 = 0, KDN_BF16 = 1 } kdn_dtype;
+
+typedef enum kdn_variant { KDN_DELTA = 0, KDN_KALMAN_DIAG = 1, KDN_KALMAN_FULL = 2 } kdn_variant;
+
+typedef struct kdn_dims {
+  int B, H, L;          /* batch, heads, tokens */
+  int dk, dv;           /* key and value head dimensions */
+  int chunk;            /* 0 = library choice; else 16, 32 or 64 tokens per chunk */
+  kdn_dtype in_dtype;   /* dtype of q, k, v */
+  kdn_dtype out_dtype;  /* dtype of o */
+} kdn_dims;
+
+/* Gated delta rule scan (A Hippocampus for Linear Attention, section 3.3
+ * Eq. (5)-(6), section 3.5).  beta: write strengths, required.  a: decay gates
+ * in (0, 1] or NULL.  S: state in/out.  o, m: outputs. */
+KDN_EXPORT kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                          const float* beta, const float* a, float* S, void* o, float* m,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Full-covariance Kalman / RLS scan (Kalman Delta Networks, Abstract; Memory
+ * by Design, Abstract; DeltaNet-PC, Eq. (5)-(7)).  Per token: propagate
+ * S^- = a S, P^- = a^2 P + Qn I, then update with the Kalman gain.  r: observation
+ * noise variances (> 0), required.  P: covariance in/out, symmetric PD. */
+KDN_EXPORT kdn_status kdn_scan_kalman_full(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                const float* a, const float* r, const float* qn, float qn_scalar,
+                                float* S, float* P, void* o, float* m,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Diagonal-covariance Kalman scan (Kalman Delta Networks, Abstract: mean-field
+ * projection on diagonal Gaussians).  p: diagonal of P in/out, positive. */
+KDN_EXPORT kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                const float* a, const float* r, const float* qn, float qn_scalar,
+                                float* S, float* p, void* o, float* m,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* One recurrent token per head against a resident state (constant-memory
+ * decoding: Kalman Delta Networks, Abstract).  variant: KDN_DELTA (beta
+ * required, p ignored) or KDN_KALMAN_DIAG (r and p required).  q, k [B,H,d_k],
+ * v [B,H,d_v], scalars [B,H], o [B,H,d_v], m [B,H] or NULL; S [B,H,d_k,d_v]
+ * and p [B,H,d_k] in/out.  Needs no workspace. */
+KDN_EXPORT kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype,
+                           kdn_dtype out_dtype, const void* q, const void* k, const void* v,
+                           const float* beta, const float* a, const float* r, float qn_scalar,
+                           float* S, float* p, void* o, float* m, void* stream);
+
+/* Bytes of device workspace a scan with these dims needs (always >= 256: the
+ * first 256 bytes hold the device status word).  Returns 0 for invalid dims. */
+KDN_EXPORT size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims);
+
+/* Synchronises ``stream``, then reads the device status word of ``workspace``
+ * into *status_out (a kdn_status value: KDN_OK, KDN_ERR_NUMERIC or
+ * KDN_ERR_TIMEOUT).  Each scan clears the word when it is enqueued. */
+KDN_EXPORT kdn_status kdn_read_device_status(const void* workspace, int* status_out, void* stream);
+
+/* Which kernels a scan with these dims runs: *launches = kernel launches per
+ * call (the status-word clear, a 256-byte memset, not counted), *kernel = name
+ * of the kernel that takes most of the time, *arith = arithmetic of that
+ * kernel ("bf16-tc" for tensor-core products with fp32 accumulation, "f32"
+ * for fp32 CUDA-core arithmetic).  Strings are static.  Pure host call. */
+KDN_EXPORT kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, const char** kernel,
+                               const char** arith);
+
+/* Static string for a status code. */
+KDN_EXPORT const char* kdn_status_string(kdn_status status);
+
+/* Message for the last failing call on the calling thread ("" if none). */
+KDN_EXPORT const char* kdn_last_error(void);
+
+/* KDN_API_VERSION of the loaded library. */
+KDN_EXPORT int kdn_api_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDN_H_ */

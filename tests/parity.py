@@ -1,0 +1,86 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path and the oracle on
+the same seeded inputs and compare them with the normwise per-head metric.
+
+Error metric (one reading of "max relative error"): for each head (b, h),
+max |x - y| / max |y| over that head's elements; the test takes the max over
+heads.  Elementwise relative error is undefined near the zeros of o.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+from delta_rule_recurrent_scan_b200 import kdn
+
+TOL = {"f32": 1e-4, "bf16": 3e-3}
+
+
+def normwise_err(x, y, lead=2):
+    x = torch.as_tensor(x).double().cpu()
+    y = torch.as_tensor(y).double().cpu()
+    n = int(np.prod(x.shape[:lead]))
+    x, y = x.reshape(n, -1), y.reshape(n, -1)
+    den = y.abs().amax(dim=1).clamp_min(1e-30)
+    return float(((x - y).abs().amax(dim=1) / den).max())
+
+
+def initial_state(variant, B, H, dk, dv, device):
+    S = torch.zeros(B, H, dk, dv, dtype=torch.float32, device=device)
+    if variant == "kalman_full":
+        return S, torch.eye(dk, dtype=torch.float32, device=device).repeat(B, H, 1, 1)
+    if variant == "kalman_diag":
+        return S, torch.ones(B, H, dk, dtype=torch.float32, device=device)
+    return S, None
+
+
+def run_gpu(variant, x, S=None, C=None, chunk=0, out_dtype=None):
+    q, k, v = x["q"], x["k"], x["v"]
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if S is None:
+        S, C = initial_state(variant, B, H, dk, dv, q.device)
+    if variant == "delta":
+        o, m, S = kdn.scan_delta(q, k, v, x["beta"], a=x["a"], S=S, chunk=chunk, out_dtype=out_dtype)
+        return {"o": o, "m": m, "S": S}
+    fn = kdn.scan_kalman_full if variant == "kalman_full" else kdn.scan_kalman_diag
+    key = "P" if variant == "kalman_full" else "p"
+    kw = {key: C}
+    o, m, S, C = fn(q, k, v, x["r"], a=x["a"], qn=x["qn"], S=S, chunk=chunk, out_dtype=out_dtype, **kw)
+    return {"o": o, "m": m, "S": S, key: C}
+
+
+def _np(t):
+    return None if t is None else t.detach().double().cpu().numpy()
+
+
+def run_oracle(variant, x, S0=None, C0=None, heads=None):
+    """Oracle on the same inputs; ``heads`` = list of (b, h) to restrict to."""
+    def pick(t):
+        if t is None:
+            return None
+        if heads is None:
+            return _np(t)
+        return np.stack([_np(t[b, h]) for b, h in heads])[None]
+
+    q, k, v = pick(x["q"]), pick(x["k"]), pick(x["v"])
+    a = pick(x["a"])
+    if variant == "delta":
+        return oracle.scan_delta(q, k, v, pick(x["beta"]), a=a, S0=pick(S0))
+    if variant == "kalman_full":
+        return oracle.scan_kalman_full(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), P0=pick(C0))
+    return oracle.scan_kalman_diag(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), p0=pick(C0))
+
+
+def compare(got, ref, tol, heads=None):
+    """Max normwise error over the outputs; returns a dict key -> error."""
+    errs = {}
+    for key, val in ref.items():
+        if key not in got:
+            continue
+        g = got[key]
+        if heads is not None:
+            g = torch.stack([g[b, h] for b, h in heads])[None]
+        errs[key] = normwise_err(g, val)
+    bad = {k_: e for k_, e in errs.items() if not (e <= tol)}
+    assert not bad, f"errors above {tol}: {errs}"
+    return errs

@@ -1,0 +1,71 @@
+"""The C-ABI library builds, loads and exports every entry point include/kdn.h
+declares; host-side validation answers without touching a GPU."""
+
+import ctypes
+
+import pytest
+
+from delta_rule_recurrent_scan_b200 import build, kdn
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kdn.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = kdn.exported_names()
+    assert {"kdn_scan_delta", "kdn_scan_kalman_full", "kdn_scan_kalman_diag", "kdn_decode_step",
+            "kdn_workspace_bytes", "kdn_read_device_status", "kdn_status_string", "kdn_last_error",
+            "kdn_api_version"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert L.kdn_api_version() == 1
+    for code, name in enumerate(["KDN_OK", "KDN_ERR_INVALID_ARG", "KDN_ERR_UNSUPPORTED", "KDN_ERR_CUDA",
+                                 "KDN_ERR_NUMERIC", "KDN_ERR_TIMEOUT"]):
+        assert L.kdn_status_string(code).decode() == name
+
+
+def test_workspace_bytes(L):
+    d = kdn.Dims(2, 3, 100, 64, 64, 0, kdn.KDN_BF16, kdn.KDN_BF16)
+    for v in (0, 1, 2):
+        n = L.kdn_workspace_bytes(v, ctypes.byref(d))
+        assert n >= 256 and n % 256 == 0
+    bad = kdn.Dims(2, 3, 100, 48, 64, 0, kdn.KDN_BF16, kdn.KDN_BF16)
+    assert L.kdn_workspace_bytes(0, ctypes.byref(bad)) == 0
+    assert L.kdn_workspace_bytes(0, None) == 0
+
+
+def _delta(L, dims, S=None, ws=None, ws_bytes=0):
+    return L.kdn_scan_delta(ctypes.byref(dims) if dims is not None else None, None, None, None, None, None, S, None,
+                            None, ws, ws_bytes, None)
+
+
+def test_host_validation_without_gpu(L):
+    # null dims, bad sizes and bad dtypes are rejected before any CUDA call
+    assert _delta(L, None) == kdn.KDN_ERR_INVALID_ARG
+    assert b"dims" in L.kdn_last_error()
+    assert _delta(L, kdn.Dims(0, 1, 4, 64, 64, 0, 1, 1)) == kdn.KDN_ERR_INVALID_ARG
+    assert _delta(L, kdn.Dims(1, 1, -1, 64, 64, 0, 1, 1)) == kdn.KDN_ERR_INVALID_ARG
+    assert _delta(L, kdn.Dims(1, 1, 4, 96, 64, 0, 1, 1)) == kdn.KDN_ERR_UNSUPPORTED
+    assert _delta(L, kdn.Dims(1, 1, 4, 64, 64, 48, 1, 1)) == kdn.KDN_ERR_UNSUPPORTED
+    assert _delta(L, kdn.Dims(1, 1, 4, 64, 64, 0, 7, 1)) == kdn.KDN_ERR_INVALID_ARG
+    # a NULL or misaligned state pointer is caught before its memory type is asked
+    assert _delta(L, kdn.Dims(1, 1, 4, 64, 64, 0, 1, 1)) == kdn.KDN_ERR_INVALID_ARG
+    assert b"S" in L.kdn_last_error()
+    assert _delta(L, kdn.Dims(1, 1, 4, 64, 64, 0, 1, 1), S=ctypes.c_void_p(0x1004)) == kdn.KDN_ERR_INVALID_ARG
+    assert b"aligned" in L.kdn_last_error()
+    assert L.kdn_decode_step(5, 1, 1, 64, 64, 1, 1, *([None] * 6), 0.0, *([None] * 5)) == kdn.KDN_ERR_UNSUPPORTED
+    out = ctypes.c_int(0)
+    assert L.kdn_read_device_status(None, ctypes.byref(out), None) == kdn.KDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 1, 4, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        kdn.scan_delta(q, q, q, torch.zeros(1, 1, 4))
