@@ -51,7 +51,7 @@ METRIC = "scan tokens/s per layer (B*H*L/time) at d=128"
 # ----------------------------------------------------------------------------- roofline bookkeeping
 
 
-def algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
+def algorithmic_bytes(w, in_bytes=2, out_bytes=4) -> int:
     """Bytes one scan must move: q, k, v in, o out, per-token scalars, m out, state in and out."""
     tok = w.B * w.H * w.L
     io = tok * ((2 * w.dk + w.dv) * in_bytes + w.dv * out_bytes + 4)  # + m
@@ -64,7 +64,7 @@ def algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
     return io + tok * scalars + state
 
 
-def decode_bytes(w, in_bytes=2, out_bytes=2) -> int:
+def decode_bytes(w, in_bytes=2, out_bytes=4) -> int:
     n = w.B * w.H
     per = (2 * w.dk + w.dv) * in_bytes + w.dv * out_bytes + 4 + 8 + w.dk * w.dv * 4 * 2
     if w.variant == "kalman_diag":
@@ -190,7 +190,7 @@ def scan_closure(w, x, kdn):
     B, H, dk, dv = w.B, w.H, w.dk, w.dv
     dev = x["q"].device
     S = torch.zeros(B, H, dk, dv, device=dev)
-    o = torch.empty(B, H, w.L, dv, dtype=x["q"].dtype, device=dev)
+    o = torch.empty(B, H, w.L, dv, dtype=torch.float32, device=dev)
     m = torch.empty(B, H, w.L, device=dev)
     ws = torch.empty(kdn.workspace_bytes(w.variant, B, H, w.L, dk, dv), dtype=torch.uint8, device=dev)
     outs = {"o": o, "m": m}
@@ -257,7 +257,7 @@ def bench_decode(w, steps, warmup, dist_on, rank, world):
     x = make_decode_inputs(w, steps=n_inputs, seed=rank, device="cuda")
     S = torch.zeros(w.B, w.H, w.dk, w.dv, device="cuda")
     p = torch.ones(w.B, w.H, w.dk, device="cuda")
-    o = torch.empty(w.B, w.H, w.dv, dtype=x["q"].dtype, device="cuda")
+    o = torch.empty(w.B, w.H, w.dv, dtype=torch.float32, device="cuda")
     m = torch.empty(w.B, w.H, device="cuda")
     it = [0]
 
@@ -382,7 +382,7 @@ def main():
             "dtype": "bf16" if plan["arith"] == "bf16-tc" else "f32",
             "data": "synthetic",
             "config": {"workload": w.name, "variant": w.variant, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk,
-                       "dv": w.dv, "in_dtype": w.dtype, "state": "fp32", "seed": "rank",
+                       "dv": w.dv, "in_dtype": w.dtype, "out_dtype": "f32", "state": "fp32", "seed": "rank",
                        "l2": f"inputs larger than L2 ({alg / 1e9:.2f} GB per step), no flush",
                        "parallelism": f"dp{world} (independent heads, no collective)",
                        "kernel_path": plan},

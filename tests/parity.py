@@ -71,8 +71,24 @@ def run_oracle(variant, x, S0=None, C0=None, heads=None):
     return oracle.scan_kalman_diag(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), p0=pick(C0))
 
 
+BF16_HALF_ULP = 2.0 ** -8  # bf16 keeps 8 significand bits: round-to-nearest costs up to 2^-8 relative
+
+
+def normwise_err_rounded(x, y, lead=2):
+    """Normwise error after removing what rounding y to bf16 alone may cost:
+    max over heads of max(|x - y| - 2^-8 |y|, 0) / max |y|."""
+    x = torch.as_tensor(x).double().cpu()
+    y = torch.as_tensor(y).double().cpu()
+    n = int(np.prod(x.shape[:lead]))
+    x, y = x.reshape(n, -1), y.reshape(n, -1)
+    den = y.abs().amax(dim=1).clamp_min(1e-30)
+    excess = ((x - y).abs() - BF16_HALF_ULP * y.abs()).clamp_min(0.0)
+    return float((excess.amax(dim=1) / den).max())
+
+
 def compare(got, ref, tol, heads=None):
-    """Max normwise error over the outputs; returns a dict key -> error."""
+    """Max normwise error over the outputs; returns a dict key -> error.  A bf16
+    output is held to the tolerance beyond its own rounding (2^-8 of each element)."""
     errs = {}
     for key, val in ref.items():
         if key not in got:
@@ -80,7 +96,10 @@ def compare(got, ref, tol, heads=None):
         g = got[key]
         if heads is not None:
             g = torch.stack([g[b, h] for b, h in heads])[None]
-        errs[key] = normwise_err(g, val)
+        if g.dtype == torch.bfloat16:
+            errs[key] = normwise_err_rounded(g, val)
+        else:
+            errs[key] = normwise_err(g, val)
     bad = {k_: e for k_, e in errs.items() if not (e <= tol)}
     assert not bad, f"errors above {tol}: {errs}"
     return errs

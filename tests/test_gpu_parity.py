@@ -3,8 +3,9 @@
 Sizes here span several 64-token chunks and a ragged tail; the layer-scale
 workloads run at full size in the launch configuration the benchmark times and
 are checked on sampled heads over the whole sequence.  Tolerances (normwise per
-head): 1e-4 for fp32 inputs, 3e-3 for bf16 inputs (bf16 output rounding
-included).
+head): 1e-4 for fp32 inputs, 3e-3 for bf16 inputs.  The read-out o is fp32 by
+default; a bf16 o is held to the same tolerance beyond its own rounding (bf16
+keeps 8 significand bits, so rounding alone may cost 2^-8 > 3e-3).
 """
 
 import ctypes
@@ -67,10 +68,19 @@ def test_layer_shapes_reduced(name, B, H, L):
 
 @pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
 @pytest.mark.parametrize("dk,dv", [(64, 32), (32, 128), (16, 64), (128, 16)])
-def test_unequal_head_dims_and_fp32_output(variant, dk, dv):
+def test_unequal_head_dims(variant, dk, dv):
     w = WORKLOADS["gdn_d64"].with_(variant=variant, dk=dk, dv=dv, qn=1e-3)
     x = make_scan_inputs(w, seed=2, device=DEV, B=1, H=2, L=130)
-    got = run_gpu(variant, x, out_dtype=torch.float32)
+    got = run_gpu(variant, x)
+    compare(got, run_oracle(variant, x), TOL["bf16"])
+
+
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+def test_bf16_output_within_tolerance_beyond_its_rounding(variant):
+    w = WORKLOADS["gdn_d128"].with_(variant=variant, qn=1e-3)
+    x = make_scan_inputs(w, seed=13, device=DEV, B=1, H=2, L=200)
+    got = run_gpu(variant, x, out_dtype=torch.bfloat16)
+    assert got["o"].dtype == torch.bfloat16
     compare(got, run_oracle(variant, x), TOL["bf16"])
 
 
