@@ -49,15 +49,17 @@ enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
 template <int D, int VAR>
 struct Layout {
   static constexpr int NP = D / 64;                 // 64-wide panels across d
-  static constexpr int KQ_PANEL = 128 * 128;        // [K; Q] rows 0..63 K, 64..127 Q
+  static constexpr int KQ_PANEL = 128 * 128;        // [K; Q]: rows 0..63 K, 64..127 Q
   static constexpr int V_PANEL = 64 * 128;
   static constexpr int G_PANEL = 64 * 128;
   static constexpr int S_PANEL = D * 128;           // d_k rows
   static constexpr int RE_PANEL = 64 * 128;
   static constexpr int TAT_BYTES = 128 * 128;       // one panel of 128 rows x 64
+  static constexpr int KQ_BUFS = (VAR == kDelta) ? 2 : 1;  // the delta rule reads K until the last MMA
 
   static constexpr int OFF_KQ = 0;
-  static constexpr int OFF_V = OFF_KQ + NP * KQ_PANEL;
+  static constexpr int KQ_BYTES = NP * KQ_PANEL;
+  static constexpr int OFF_V = OFF_KQ + KQ_BUFS * KQ_BYTES;
   static constexpr int OFF_GHI = OFF_V + NP * V_PANEL;
   static constexpr int G_BYTES = (VAR == kDelta) ? 0 : NP * G_PANEL;
   static constexpr int OFF_GLO = OFF_GHI + G_BYTES;
@@ -68,24 +70,23 @@ struct Layout {
   static constexpr int OFF_RHI = OFF_TLO + TAT_BYTES;
   static constexpr int OFF_RLO = OFF_RHI + NP * RE_PANEL;
   static constexpr int END = OFF_RLO + NP * RE_PANEL;
-  // fp32 [64][64] scratch for N and T; alias dead buffers when they are large enough
-  static constexpr int NF_BYTES = 64 * 64 * 4;
-  static constexpr bool NF_IN_V = NP * V_PANEL >= NF_BYTES;
-  static constexpr bool TF_IN_S = NP * S_PANEL >= NF_BYTES;
-  static constexpr int OFF_NF = NF_IN_V ? OFF_V : END;
-  static constexpr int OFF_TF = TF_IN_S ? OFF_SHI : (NF_IN_V ? END : END + NF_BYTES);
-  static constexpr int TOTAL = END + (NF_IN_V ? 0 : NF_BYTES) + (TF_IN_S ? 0 : NF_BYTES);
+  // fp32 [64][68] scratch for N and T: inside the state panels (dead between the
+  // [K;Q] S0 product and the state write-back) when they are large enough
+  static constexpr int SCR_LD = 68;
+  static constexpr int SCR_BYTES = 64 * SCR_LD * 4;
+  static constexpr bool SCR_IN_S = NP * S_PANEL >= SCR_BYTES;
+  static constexpr int OFF_NF = SCR_IN_S ? OFF_SLO : END;
+  static constexpr int OFF_TF = SCR_IN_S ? OFF_SHI : END + SCR_BYTES;
+  static constexpr int TOTAL = END + (SCR_IN_S ? 0 : 2 * SCR_BYTES);
   static constexpr int SMEM = TOTAL + 1024;         // + alignment slack
-  // fp32 [64][D] gain scratch (diag / full) in the R/E area: 2 * NP * 8 KB = 256 * D bytes
+  // fp32 [64][D] gain scratch in the R/E area (2 * NP * 8 KB = 256 * D bytes)
   static constexpr int OFF_GF = OFF_RHI;
   // TMEM columns
   static constexpr uint32_t T_D1 = 0, T_D2 = 64, T_DT = 64 + D, T_D3 = 128 + D, T_D4 = 128 + 2 * D;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(128 + 3 * D <= 512, "TMEM budget");
-  static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+  static_assert(TOTAL <= 224 * 1024, "shared memory budget");
 };
-
-__device__ __forceinline__ int fidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }  // [64][64] fp32, bank-spread
 
 __device__ __forceinline__ void store8_split(uint8_t* hi, uint8_t* lo, uint32_t off, const float (&x)[8]) {
   __align__(16) __nv_bfloat16 h[8], l[8];
@@ -95,8 +96,28 @@ __device__ __forceinline__ void store8_split(uint8_t* hi, uint8_t* lo, uint32_t 
   *reinterpret_cast<uint4*>(lo + off) = *reinterpret_cast<const uint4*>(l);
 }
 
-__device__ __forceinline__ float ld_bf16(const uint8_t* base, uint32_t off) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
+// 8 consecutive bf16 of a swizzled panel (one 16-byte chunk) as floats.
+__device__ __forceinline__ void load8_bf16(const uint8_t* base, uint32_t off, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(base + off);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    x[2 * e] = f.x, x[2 * e + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
 }
 
 struct Params {
@@ -121,11 +142,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, Params P) {
   using Lay = Layout<D, VAR>;
   constexpr int NP = Lay::NP;
-  constexpr int HALF = D / 2;  // columns of d_v per column half
+  constexpr int HALF = D / 2;  // d_v columns per column half
+  constexpr int LD = Lay::SCR_LD;
+  constexpr int QD = D / 4;    // coordinates per thread in the per-token reductions
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* KQ = sm + Lay::OFF_KQ;
   uint8_t* Vs = sm + Lay::OFF_V;
   uint8_t* Ghi = sm + Lay::OFF_GHI;
   uint8_t* Glo = sm + Lay::OFF_GLO;
@@ -139,8 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* Tf = reinterpret_cast<float*>(sm + Lay::OFF_TF);
   float* Gf = reinterpret_cast<float*>(sm + Lay::OFF_GF);
 
-  __shared__ float ell[kC], Aex[kC], sc1[kC], sc2[kC], sc3[kC], gn[kC], en[2][kC];
-  __shared__ uint64_t bar_load, bar_mma;
+  __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];  // a, beta|r, Qn of this chunk and the next
+  __shared__ float ell[kC], Aex[kC], Arat[kC], gn[kC], en[2][kC];
+  __shared__ uint64_t bar_kq[2], bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -150,20 +173,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int L = P.L;
   const int nchunks = (L + kC - 1) / kC;
 
+  // per-token scalars of chunk cc: read into registers early, stored into shared memory late,
+  // so that the global-load latency hides behind a whole chunk
+  float ra = 1.f, rb = 0.f, rq = 0.f;
+  auto fetch_scalars = [&](int cc) {
+    if (tid < kC) {
+      const int tok = cc * kC + tid;
+      const bool valid = tok < L;
+      const size_t ti = (size_t)bh * L + tok;
+      ra = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;
+      if (VAR == kDelta) rb = valid ? P.beta[ti] : 0.f;
+      else rb = valid ? P.r[ti] : 1.f;
+      rq = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;
+    }
+  };
+  auto store_scalars = [&](int buf) {
+    if (tid < kC) sA[buf][tid] = ra, sB[buf][tid] = rb, sQ[buf][tid] = rq;
+  };
+  auto issue_kq = [&](int cc, int buf) {
+    uint8_t* dst = sm + Lay::OFF_KQ + buf * Lay::KQ_BYTES;
+    sm100::mbar_arrive_expect_tx(&bar_kq[buf], 2 * NP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) {
+      sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL, &tm_k, &bar_kq[buf], 64 * pn, cc * kC, bh);
+      sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL + 64 * 128, &tm_q, &bar_kq[buf], 64 * pn, cc * kC, bh);
+    }
+  };
+  auto issue_v = [&](int cc) {
+    sm100::mbar_arrive_expect_tx(&bar_v, NP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) sm100::tma_load_3d(Vs + pn * Lay::V_PANEL, &tm_v, &bar_v, 64 * pn, cc * kC, bh);
+  };
+
   if (tid == 0) {
     sm100::prefetch_tmap(&tm_q);
     sm100::prefetch_tmap(&tm_k);
     sm100::prefetch_tmap(&tm_v);
-    sm100::mbar_init(&bar_load, 1);
+    sm100::mbar_init(&bar_kq[0], 1);
+    sm100::mbar_init(&bar_kq[1], 1);
+    sm100::mbar_init(&bar_v, 1);
     sm100::mbar_init(&bar_mma, 1);
     sm100::fence_mbar_init();
+    issue_kq(0, 0);  // chunk c issues chunk c + 1
+    issue_v(0);
   }
   if (warp == 0) {
     sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
     sm100::tmem_relinquish();
   }
+  fetch_scalars(0);
+  store_scalars(0);
 
-  // ---- initial state: fp32 master in registers, bf16 hi/lo panels for the MMAs
+  // ---- state: fp32 master in registers (thread = d_k row, one column half), bf16 hi/lo panels for the MMAs
   float Sr[HALF];
   const bool s_owner = row < D;
   float* Sg = P.S + (size_t)bh * D * D;
@@ -174,10 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       Sr[c] = x.x, Sr[c + 1] = x.y, Sr[c + 2] = x.z, Sr[c + 3] = x.w;
     }
   }
-  // per-coordinate diagonal covariance, owned by threads 128 + i
+  // diagonal covariance: coordinate tid (threads 0 .. D-1)
   float pcur = 1.f;
-  const int pi = tid - 128;
-  if (VAR == kDiag && pi >= 0 && pi < D) pcur = P.p[(size_t)bh * D + pi];
+  if (VAR == kDiag && tid < D) pcur = P.p[(size_t)bh * D + tid];
 
   auto write_state_panels = [&]() {
     if (!s_owner) return;
@@ -200,45 +260,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t mma_phase = 0;
   bool aborted = false;
-  // single-thread wait on an mbarrier, then a CTA-wide vote
-  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+  // one thread waits on the mbarriers, then a CTA-wide vote
+  auto wait_all = [&](uint64_t* b1, uint32_t par1, uint64_t* b2, uint32_t par2) -> bool {
     int bad = 0;
-    if (tid == 0) bad = !sm100::mbar_wait_bounded(bar, parity, kWaitCycles);
+    if (tid == 0) {
+      bad = !sm100::mbar_wait_bounded(b1, par1, kWaitCycles);
+      if (!bad && b2 != nullptr) bad = !sm100::mbar_wait_bounded(b2, par2, kWaitCycles);
+    }
     bad = __syncthreads_or(bad);
     if (bad && tid == 0) raise_status(P.status, kStatusTimeout);
     sm100::tc_fence_after();
     return !bad;
   };
 
-  const uint32_t kq0 = sm100::smem_u32(KQ);
+  const uint32_t shi = sm100::smem_u32(Shi), slo = sm100::smem_u32(Slo);
+  const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
+  const uint32_t thi = sm100::smem_u32(Thi), tlo = sm100::smem_u32(Tlo);
+  const uint32_t rhi = sm100::smem_u32(Rhi), rlo = sm100::smem_u32(Rlo);
 
-  for (int c = 0; c < nchunks && !aborted; ++c) {
+  for (int c = 0; c < nchunks; ++c) {
     const int t0 = c * kC;
-    // ---------------------------------------------------------------- stage inputs
-    if (tid == 0) {
-      sm100::mbar_arrive_expect_tx(&bar_load, 3 * NP * 64 * 128);
-#pragma unroll
-      for (int pn = 0; pn < NP; ++pn) {
-        sm100::tma_load_3d(KQ + pn * Lay::KQ_PANEL, &tm_k, &bar_load, 64 * pn, t0, bh);
-        sm100::tma_load_3d(KQ + pn * Lay::KQ_PANEL + 64 * 128, &tm_q, &bar_load, 64 * pn, t0, bh);
-        sm100::tma_load_3d(Vs + pn * Lay::V_PANEL, &tm_v, &bar_load, 64 * pn, t0, bh);
-      }
-    }
-    if (tid < kC) {
-      const int tok = t0 + tid;
-      const bool valid = tok < L;
-      const size_t ti = (size_t)bh * L + tok;
-      sc1[tid] = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;                          // a
-      if (VAR == kDelta) sc2[tid] = valid ? P.beta[ti] : 0.f;                  // beta
-      else sc2[tid] = valid ? P.r[ti] : 1.f;                                   // r
-      sc3[tid] = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;                // Qn
-    }
-    if (!wait_all(&bar_load, c & 1)) { aborted = true; break; }
+    const int kb = (Lay::KQ_BUFS == 2) ? (c & 1) : 0;
+    const int sb = c & 1;
+    uint8_t* KQ = sm + Lay::OFF_KQ + kb * Lay::KQ_BYTES;
+    const uint32_t kq0 = sm100::smem_u32(KQ);
+    const float* a_c = sA[sb];
+    const float* b_c = sB[sb];
+    const float* q_c = sQ[sb];
 
-    // ---------------------------------------------------------------- gates and gains
-    if (warp == 0) {
+    // ---------------------------------------------------------------- K, Q of this chunk; start [K;Q] S0
+    if (!wait_all(&bar_kq[kb], (Lay::KQ_BUFS == 2) ? ((c >> 1) & 1) : (c & 1), nullptr, 0)) { aborted = true; break; }
+    if (tid == 0) {
+      if (Lay::KQ_BUFS == 2 && c + 1 < nchunks) issue_kq(c + 1, kb ^ 1);
+      constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id2 = sm100::idesc_bf16(128, D, false, true);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
+        const uint64_t a = sm100::smem_desc(kq0 + koff, 16, 1024);
+        sm100::mma_bf16(tmem + Lay::T_D2, a, sm100::smem_desc(shi + ks * 2048, Lay::S_PANEL, 1024), id2, ks > 0);
+        sm100::mma_bf16(tmem + Lay::T_D2, a, sm100::smem_desc(slo + ks * 2048, Lay::S_PANEL, 1024), id2, true);
+        if (VAR == kDelta)  // G = K: [K;Q] K^T now
+          sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(kq0 + koff, 16, 1024), id1, ks > 0);
+      }
+      if (VAR == kDelta) sm100::mma_commit(&bar_mma);
+    }
+
+    if (c + 1 < nchunks) fetch_scalars(c + 1);
+
+    // ---------------------------------------------------------------- gates
+    if (warp == 1) {
       // inclusive prefix sums of log a over the chunk (a gate of 0 enters as exp(-60))
-      float x0 = sc1[lane], x1 = sc1[32 + lane];
+      float x0 = a_c[lane], x1 = a_c[32 + lane];
       x0 = x0 > 0.f ? fmaxf(__logf(x0), -60.f) : -60.f;
       x1 = x1 > 0.f ? fmaxf(__logf(x1), -60.f) : -60.f;
 #pragma unroll
@@ -247,69 +320,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane >= o) x0 += y0, x1 += y1;
       }
       x1 += __shfl_sync(0xffffffffu, x0, 31);
+      const float lC = __shfl_sync(0xffffffffu, x1, 31);
       ell[lane] = x0, ell[32 + lane] = x1;
-      Aex[lane] = expf(x0), Aex[32 + lane] = expf(x1);
+      Aex[lane] = __expf(x0), Aex[32 + lane] = __expf(x1);
+      Arat[lane] = __expf(lC - x0), Arat[32 + lane] = __expf(lC - x1);  // A_C / A_i without a division
     }
-    if (VAR == kDiag && pi >= 0 && pi < D) {
-      // per-coordinate variance recursion (independent of v and S):
-      // p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + p^- k^2)
-      const uint8_t* Kp = KQ + (pi / 64) * Lay::KQ_PANEL;
+    // ---------------------------------------------------------------- diagonal variances
+    if (VAR == kDiag && tid < D) {
+      // Per coordinate i (independent of v and S) each token maps the variance by the Moebius map
+      // p -> (r a^2 p + r Qn) / (k^2 a^2 p + k^2 Qn + r)  (Kalman Delta Networks, Abstract: the
+      // uncertainty recurrences are Moebius maps).  The 2x2 prefix product from the chunk start is
+      // the only serial chain; each p_{t-1} = P_{t-1}(p_0) and p^-_t k_t follow off the chain.
+      const uint8_t* Kp = KQ + (tid / 64) * Lay::KQ_PANEL;
+      float m00 = 1.f, m01 = 0.f, m10 = 0.f, m11 = 1.f;
+      const float p0 = pcur;
+#pragma unroll 8
       for (int t = 0; t < kC; ++t) {
-        const float at = sc1[t], rt = sc2[t];
-        const float kt = ld_bf16(Kp, sm100::sw128(t, pi % 64));
-        const float pp = fmaf(at * at, pcur, sc3[t]);
-        const float pk = pp * kt;
-        Gf[t * D + pi] = pk;
-        pcur = pp * rt / fmaf(pk, kt, rt);
+        const float at = a_c[t], rt = b_c[t], qt = q_c[t];
+        const float kt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t, tid % 64)));
+        const float pprev = __fdividef(fmaf(m00, p0, m01), fmaf(m10, p0, m11));
+        const float a2 = at * at, k2 = kt * kt;
+        Gf[t * D + tid] = fmaf(a2, pprev, qt) * kt;  // p^-_t k_t
+        const float e00 = rt * a2, e01 = rt * qt, e10 = k2 * a2, e11 = fmaf(k2, qt, rt);
+        const float n00 = fmaf(e00, m00, e01 * m10), n01 = fmaf(e00, m01, e01 * m11);
+        const float n10 = fmaf(e10, m00, e11 * m10), n11 = fmaf(e10, m01, e11 * m11);
+        m00 = n00, m01 = n01, m10 = n10, m11 = n11;
+        if ((t & 7) == 7) {  // maps are scale free: renormalise against under/overflow
+          const float sc = __fdividef(1.f, m11);
+          m00 *= sc, m01 *= sc, m10 *= sc, m11 = 1.f;
+        }
       }
-    }
-    if (VAR == kFull) {
-      for (int idx = tid; idx < kC * D / 4; idx += kThreads) {
-        const int t = idx / (D / 4), i4 = idx % (D / 4);
-        float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t0 + t < L) g = *reinterpret_cast<const float4*>(P.gains + ((size_t)bh * L + t0 + t) * D + 4 * i4);
-        *reinterpret_cast<float4*>(Gf + t * D + 4 * i4) = g;
-      }
+      pcur = __fdividef(fmaf(m00, p0, m01), fmaf(m10, p0, m11));
     }
     __syncthreads();
-    // gains: normalise (diag), squared norms, bf16 hi/lo panels of G
-    for (int t = warp; t < kC; t += kThreads / 32) {
+
+    // ---------------------------------------------------------------- gains: norms, hi/lo panels (4 threads per token)
+    {
+      const int t = tid >> 2, part = tid & 3;
+      const int i0 = part * QD;  // first coordinate of this thread
+      float kv[QD];
+#pragma unroll
+      for (int u = 0; u < QD / 8; ++u) {
+        float x[8];
+        const int i = i0 + 8 * u;
+        load8_bf16(KQ + (i / 64) * Lay::KQ_PANEL, sm100::sw128_chunk(t, (i % 64) / 8), x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kv[8 * u + e] = x[e];
+      }
       if (VAR == kDelta) {
         float s = 0.f;
-        for (int i = lane; i < D; i += 32) {
-          const float kv = ld_bf16(KQ + (i / 64) * Lay::KQ_PANEL, sm100::sw128(t, i % 64));
-          s = fmaf(kv, kv, s);
-        }
-        s = warp_sum(s);
-        if (lane == 0) gn[t] = sc2[t] * sc2[t] * s;
+#pragma unroll
+        for (int e = 0; e < QD; ++e) s = fmaf(kv[e], kv[e], s);
+        s = quad_sum(s);
+        if (part == 0) gn[t] = b_c[t] * b_c[t] * s;
       } else {
-        float inv_s = 1.f;
+        float g[QD];
         if (VAR == kDiag) {
+#pragma unroll
+          for (int e = 0; e < QD; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(Gf + t * D + i0 + e);
+            g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
+          }
           float s = 0.f;
-          for (int i = lane; i < D; i += 32)
-            s = fmaf(Gf[t * D + i], ld_bf16(KQ + (i / 64) * Lay::KQ_PANEL, sm100::sw128(t, i % 64)), s);
-          s = warp_sum(s) + sc2[t];
-          if (lane == 0 && !(s > 0.f && isfinite(s))) raise_status(P.status, kStatusNumeric);
-          inv_s = 1.f / s;
+#pragma unroll
+          for (int e = 0; e < QD; ++e) s = fmaf(g[e], kv[e], s);
+          s = quad_sum(s) + b_c[t];
+          if (part == 0 && !(s > 0.f && isfinite(s))) raise_status(P.status, kStatusNumeric);
+          const float inv_s = 1.f / s;
+#pragma unroll
+          for (int e = 0; e < QD; ++e) g[e] *= inv_s;
+        } else {
+          const bool valid = t0 + t < L;
+#pragma unroll
+          for (int e = 0; e < QD; e += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (valid) x = *reinterpret_cast<const float4*>(P.gains + ((size_t)bh * L + t0 + t) * D + i0 + e);
+            g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
+          }
         }
         float n2 = 0.f;
-        for (int i = lane; i < D; i += 32) {
-          const float g = Gf[t * D + i] * inv_s;
-          Gf[t * D + i] = g;
-          n2 = fmaf(g, g, n2);
-        }
-        n2 = warp_sum(n2);
-        if (lane == 0) gn[t] = n2;
-      }
-    }
-    if (VAR != kDelta) {
-      __syncthreads();
-      for (int idx = tid; idx < kC * D / 8; idx += kThreads) {
-        const int t = idx / (D / 8), c8 = idx % (D / 8);
-        float x[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = Gf[t * D + 8 * c8 + e];
-        store8_split(Ghi, Glo, (c8 / 8) * Lay::G_PANEL + sm100::sw128_chunk(t, c8 % 8), x);
+        for (int e = 0; e < QD; ++e) n2 = fmaf(g[e], g[e], n2);
+        n2 = quad_sum(n2);
+        if (part == 0) gn[t] = n2;
+#pragma unroll
+        for (int u = 0; u < QD / 8; ++u) {
+          const int i = i0 + 8 * u;
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = g[8 * u + e];
+          store8_split(Ghi, Glo, (i / 64) * Lay::G_PANEL + sm100::sw128_chunk(t, (i % 64) / 8), x);
+        }
       }
     }
     sm100::fence_async_smem();
@@ -317,34 +418,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     sm100::tc_fence_after();
 
-    // ---------------------------------------------------------------- D1 = [K;Q] G^T, D2 = [K;Q] S0
-    if (tid == 0) {
+    // ---------------------------------------------------------------- D1 = [K;Q] G^T (Kalman gains)
+    if (tid == 0 && VAR != kDelta) {
       constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
-      constexpr uint32_t id2 = sm100::idesc_bf16(128, D, false, true);
-      const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
-      const uint32_t shi = sm100::smem_u32(Shi), slo = sm100::smem_u32(Slo);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
+        const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
         const uint64_t a = sm100::smem_desc(kq0 + koff, 16, 1024);
-        if (VAR == kDelta) {
-          sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(kq0 + koff, 16, 1024), id1, ks > 0);
-        } else {
-          const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
-          sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + goff, 16, 1024), id1, ks > 0);
-          sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(glo + goff, 16, 1024), id1, true);
-        }
-        sm100::mma_bf16(tmem + Lay::T_D2, a, sm100::smem_desc(shi + ks * 2048, Lay::S_PANEL, 1024), id2, ks > 0);
-        sm100::mma_bf16(tmem + Lay::T_D2, a, sm100::smem_desc(slo + ks * 2048, Lay::S_PANEL, 1024), id2, true);
+        sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + goff, 16, 1024), id1, ks > 0);
+        sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(glo + goff, 16, 1024), id1, true);
       }
       sm100::mma_commit(&bar_mma);
     }
-    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    if (!wait_all(&bar_mma, mma_phase, &bar_v, c & 1)) { aborted = true; break; }
     mma_phase ^= 1;
+    if (tid == 0 && Lay::KQ_BUFS == 1 && c + 1 < nchunks) issue_kq(c + 1, 0);  // K, Q of this chunk are dead
 
-    // ---------------------------------------------------------------- R = V - diag(A) K S0
+    // ---------------------------------------------------------------- N, R (lanes 0..63) | Attn, T (lanes 64..127)
+    // The warps that own TMEM lanes 0..63 ([K;Q] rows of K) build N, hand it over through a named
+    // barrier and then build R; the warps that own lanes 64..127 build Attn and then invert I + N.
     if (qw < 2) {
       const int i = row;  // token in chunk
+      {
+        // N_ij = (K G^T)_ij Gam_ij for j < i
+        float Y[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * ch, Y);
+        sm100::tmem_wait_ld();
+        const float li = ell[i];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float v4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 32 * ch + e + u;
+            v4[u] = (j < i) ? Y[e + u] * __expf(li - ell[j]) * (VAR == kDelta ? b_c[j] : 1.f) : 0.f;
+          }
+          *reinterpret_cast<float4*>(Nf + i * LD + 32 * ch + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+        }
+      }
+      named_arrive(1, 256);  // N is ready
       const float Ai = Aex[i];
 #pragma unroll
       for (int cc = 0; cc < HALF; cc += 32) {
@@ -355,93 +468,102 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           const int cb = c0 + 8 * c8;
-          float x[8];
+          const uint32_t off = (cb / 64) * Lay::V_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8);
+          float vv[8], x[8];
+          load8_bf16(Vs, off, vv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            x[e] = ld_bf16(Vs + (cb / 64) * Lay::V_PANEL, sm100::sw128(i, (cb % 64) + e)) - Ai * X[8 * c8 + e];
-          store8_split(Rhi, Rlo, (cb / 64) * Lay::RE_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8), x);
+          for (int e = 0; e < 8; ++e) x[e] = fmaf(-Ai, X[8 * c8 + e], vv[e]);
+          store8_split(Rhi, Rlo, off, x);
         }
       }
-    }
-    __syncthreads();  // V is dead from here (Nf may alias it)
-
-    // ---------------------------------------------------------------- N and Attn from D1
-    {
-      const int i = row & 63;
-      const float li = ell[i];
-      float X[32];
-      sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * ch, X);
-      sm100::tmem_wait_ld();
-      if (qw < 2) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = 32 * ch + e;
-          float v = 0.f;
-          if (j < i) v = X[e] * __expf(li - ell[j]) * (VAR == kDelta ? sc2[j] : 1.f);
-          Nf[fidx(i, j)] = v;
-        }
-      } else {
+    } else {
+      const int gt = (qw - 2) * 32 + lane + 64 * ch;  // 0..127 within this group
+      {
+        // Attn_ij = (Q G^T)_ij Gam_ij for j <= i, into rows 64.. of the [T; AT] panel
+        const int i = row - 64;
+        float Y[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * ch, Y);
+        sm100::tmem_wait_ld();
+        const float li = ell[i];
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int j = 32 * ch + 8 * c8 + e;
-            x[e] = (j <= i) ? X[8 * c8 + e] * __expf(li - ell[j]) * (VAR == kDelta ? sc2[j] : 1.f) : 0.f;
+            x[e] = (j <= i) ? Y[8 * c8 + e] * __expf(li - ell[j]) * (VAR == kDelta ? b_c[j] : 1.f) : 0.f;
           }
           store8_split(Thi, Tlo, sm100::sw128_chunk(64 + i, 4 * ch + c8), x);
         }
       }
-    }
-    __syncthreads();
-
-    // ---------------------------------------------------------------- T = (I + N)^-1, blocked by 16
-    if (tid < 64) {
-      const int b = tid >> 4, cc = tid & 15;
-      float t[16];
+      named_sync(1, 256);  // wait for N
+      // ---- T = (I + N)^-1, blocked by 16: diagonal blocks right-looking (column cc of block b)
+      if (gt < 64) {
+        const int b = gt >> 4, cc = gt & 15;
+        const float* Nb = Nf + (16 * b) * LD + 16 * b;
+        float acc[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float acc = (i == cc) ? 1.f : 0.f;
+        for (int i = 0; i < 16; ++i) acc[i] = (i == cc) ? 1.f : 0.f;
 #pragma unroll
-        for (int j = 0; j < i; ++j) acc = fmaf(-Nf[fidx(16 * b + i, 16 * b + j)], t[j], acc);
-        t[i] = acc;
+        for (int j = 0; j < 16; ++j) {
+          const float tj = acc[j];
+#pragma unroll
+          for (int i = j + 1; i < 16; ++i) acc[i] = fmaf(-Nb[i * LD + j], tj, acc[i]);
+        }
+        float* Tb = Tf + (16 * b) * LD + 16 * b;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = acc[i];
       }
+      named_sync(2, 128);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Tf[fidx(16 * b + i, 16 * b + cc)] = t[i];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-      // M_ab = sum_{k=b}^{a-1} N_ak T_kb, kept in the (unused) upper block (b, a)
-      for (int e = tid; e < (4 - d) * 256; e += kThreads) {
-        const int b = e >> 8, a = b + d, ii = (e >> 4) & 15, jj = e & 15;
-        float acc = 0.f;
-        for (int k = b; k < a; ++k)
+      for (int d = 1; d < 4; ++d) {
+        // off-diagonal blocks at distance d: T_ab = -T_aa sum_{k=b}^{a-1} N_ak T_kb (a = b + d)
+        for (int e = gt; e < (4 - d) * 64; e += 128) {
+          const int b = e >> 6, a = b + d, ii = (e >> 2) & 15, jq = e & 3;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int l = 0; l < 16; ++l) acc = fmaf(Nf[fidx(16 * a + ii, 16 * k + l)], Tf[fidx(16 * k + l, 16 * b + jj)], acc);
-        Tf[fidx(16 * b + ii, 16 * a + jj)] = acc;
+          for (int k = 0; k < d; ++k) {
+            const float* nrow = Nf + (16 * a + ii) * LD + 16 * (b + k);
+#pragma unroll
+            for (int l = 0; l < 16; ++l) {
+              const float n = nrow[l];
+              const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * (b + k) + l) * LD + 16 * b + 4 * jq);
+              acc.x = fmaf(n, t4.x, acc.x), acc.y = fmaf(n, t4.y, acc.y);
+              acc.z = fmaf(n, t4.z, acc.z), acc.w = fmaf(n, t4.w, acc.w);
+            }
+          }
+          // M_ab parked in the unused upper block (b, a)
+          *reinterpret_cast<float4*>(Tf + (16 * b + ii) * LD + 16 * a + 4 * jq) = acc;
+        }
+        named_sync(2, 128);
+        for (int e = gt; e < (4 - d) * 64; e += 128) {
+          const int b = e >> 6, a = b + d, ii = (e >> 2) & 15, jq = e & 3;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          const float* trow = Tf + (16 * a + ii) * LD + 16 * a;
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            const float tv = trow[l];
+            const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + l) * LD + 16 * a + 4 * jq);
+            acc.x = fmaf(tv, m4.x, acc.x), acc.y = fmaf(tv, m4.y, acc.y);
+            acc.z = fmaf(tv, m4.z, acc.z), acc.w = fmaf(tv, m4.w, acc.w);
+          }
+          *reinterpret_cast<float4*>(Tf + (16 * a + ii) * LD + 16 * b + 4 * jq) =
+              make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        }
+        named_sync(2, 128);
       }
-      __syncthreads();
-      // T_ab = -T_aa M_ab
-      for (int e = tid; e < (4 - d) * 256; e += kThreads) {
-        const int b = e >> 8, a = b + d, ii = (e >> 4) & 15, jj = e & 15;
-        float acc = 0.f;
+      // T (unit diagonal, zero above) as bf16 hi/lo into rows 0..63 of the [T; AT] panel
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(Tf[fidx(16 * a + ii, 16 * a + l)], Tf[fidx(16 * b + l, 16 * a + jj)], acc);
-        Tf[fidx(16 * a + ii, 16 * b + jj)] = -acc;
-      }
-      __syncthreads();
-    }
-    {
-      const int i = tid >> 2, q4 = tid & 3;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int c8 = 2 * q4 + h;
+      for (int h = 0; h < 4; ++h) {
+        const int i = (gt >> 1) & 63, c8 = 4 * (gt & 1) + h;
+        const float4 lo4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8);
+        const float4 hi4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8 + 4);
+        const float tv[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
         float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int j = 8 * c8 + e;
-          x[e] = (j < i) ? Tf[fidx(i, j)] : (j == i ? 1.f : 0.f);
+          x[e] = (j < i) ? tv[e] : (j == i ? 1.f : 0.f);
         }
         store8_split(Thi, Tlo, sm100::sw128_chunk(i, c8), x);
       }
@@ -450,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
+    if (tid == 0 && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
 
-    const uint32_t thi = sm100::smem_u32(Thi), tlo = sm100::smem_u32(Tlo);
     // ---------------------------------------------------------------- DT = [T; Attn] T  (rows 64..127: AT)
     if (tid == 0) {
       constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, true);
@@ -465,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sm100::mma_commit(&bar_mma);
     }
-    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    if (!wait_all(&bar_mma, mma_phase, nullptr, 0)) { aborted = true; break; }
     mma_phase ^= 1;
     if (qw >= 2) {
       const int i = row - 64;
@@ -486,7 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_after();
 
     // ---------------------------------------------------------------- D3 = [T; AT] R
-    const uint32_t rhi = sm100::smem_u32(Rhi), rlo = sm100::smem_u32(Rlo);
     if (tid == 0) {
       constexpr uint32_t id = sm100::idesc_bf16(128, D, false, true);
 #pragma unroll
@@ -500,14 +621,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sm100::mma_commit(&bar_mma);
     }
-    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    if (!wait_all(&bar_mma, mma_phase, nullptr, 0)) { aborted = true; break; }
     mma_phase ^= 1;
 
-    // ---------------------------------------------------------------- E -> scaled E panels, O out
+    // ---------------------------------------------------------------- E -> scaled E panels; O out
     const float AC = Aex[kC - 1];
     if (qw < 2) {
       const int i = row;
-      const float sc = __expf(ell[kC - 1] - ell[i]) * (VAR == kDelta ? sc2[i] : 1.f);  // A_C / A_i, no division
+      const float sc = Arat[i] * (VAR == kDelta ? b_c[i] : 1.f);
       float es = 0.f;
 #pragma unroll
       for (int cc = 0; cc < HALF; cc += 32) {
@@ -564,8 +685,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
-    if (tid < kC && P.m != nullptr && t0 + tid < L)
-      P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[tid]) * sqrtf(en[0][tid] + en[1][tid]);
 
     // ---------------------------------------------------------------- D4 = G^T Et
     if (tid == 0) {
@@ -579,8 +698,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm100::mma_bf16(tmem + Lay::T_D4, ak, bh_, id, ks > 0);
           sm100::mma_bf16(tmem + Lay::T_D4, ak, bl, id, true);
         } else {
-          const uint64_t ah = sm100::smem_desc(sm100::smem_u32(Ghi) + ks * 2048, Lay::G_PANEL, 1024);
-          const uint64_t al = sm100::smem_desc(sm100::smem_u32(Glo) + ks * 2048, Lay::G_PANEL, 1024);
+          const uint64_t ah = sm100::smem_desc(ghi + ks * 2048, Lay::G_PANEL, 1024);
+          const uint64_t al = sm100::smem_desc(glo + ks * 2048, Lay::G_PANEL, 1024);
           sm100::mma_bf16(tmem + Lay::T_D4, ah, bh_, id, ks > 0);
           sm100::mma_bf16(tmem + Lay::T_D4, al, bh_, id, true);
           sm100::mma_bf16(tmem + Lay::T_D4, ah, bl, id, true);
@@ -588,7 +707,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sm100::mma_commit(&bar_mma);
     }
-    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    if (tid < kC && P.m != nullptr && t0 + tid < L)
+      P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[tid]) * sqrtf(en[0][tid] + en[1][tid]);
+    if (!wait_all(&bar_mma, mma_phase, nullptr, 0)) { aborted = true; break; }
     mma_phase ^= 1;
 
     // ---------------------------------------------------------------- S <- A_C S + D4
@@ -603,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     write_state_panels();
+    if (c + 1 < nchunks) store_scalars(sb ^ 1);
     sm100::fence_async_smem();
     sm100::tc_fence_before();
     __syncthreads();
@@ -617,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<float4*>(Sg + (size_t)row * D + ch * HALF + c) =
             make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
     }
-    if (VAR == kDiag && pi >= 0 && pi < D) P.p[(size_t)bh * D + pi] = pcur;
+    if (VAR == kDiag && tid < D) P.p[(size_t)bh * D + tid] = pcur;
   }
   sm100::tc_fence_before();
   __syncthreads();
