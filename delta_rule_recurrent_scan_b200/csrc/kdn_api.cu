@@ -9,11 +9,13 @@
 #include <string>
 
 #include "../../include/kdn.h"
+#include "api_internal.h"
+#include "chunk.h"
 #include "common.cuh"
 #include "kernels.h"
-#include "chunk.h"
 
-namespace {
+namespace kdn {
+namespace api {
 
 thread_local std::string g_last_error;
 
@@ -86,7 +88,7 @@ kdn_status check_dims(const kdn_dims* d) {
   return KDN_OK;
 }
 
-constexpr size_t kStatusBytes = 256;
+
 
 size_t gains_bytes(const kdn_dims* d) { return (size_t)d->B * d->H * (size_t)d->L * d->dk * sizeof(float); }
 
@@ -113,7 +115,10 @@ kdn_status cuda_status(cudaError_t e, const char* what) {
   return fail(KDN_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
-}  // namespace
+}  // namespace api
+}  // namespace kdn
+
+using namespace kdn::api;
 
 extern "C" {
 
@@ -204,7 +209,9 @@ kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, co
   return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, s, st), "delta scan launch");
 }
 
-static kdn_status kalman_scan(kdn_variant var, const kdn_dims* dims, const void* q, const void* k, const void* v,
+}  // extern "C"
+
+kdn_status kdn::api::kalman_scan(kdn_variant var, const kdn_dims* dims, const void* q, const void* k, const void* v,
                               const float* a, const float* r, const float* qn, float qn_scalar, float* S, float* P,
                               void* o, float* m, void* workspace, size_t workspace_bytes, void* stream) {
   KDN_TRY(common_checks(var, dims, q, k, v, S, o, m, workspace, workspace_bytes));
@@ -236,6 +243,8 @@ static kdn_status kalman_scan(kdn_variant var, const kdn_dims* dims, const void*
   kdn::SeqScanArgs s{q, k, v, dims->in_dtype, dims->out_dtype, nullptr, a, gains, S, o, m, BH, dims->L};
   return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, s, st), "Kalman scan launch");
 }
+
+extern "C" {
 
 kdn_status kdn_scan_kalman_full(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* a,
                                 const float* r, const float* qn, float qn_scalar, float* S, float* P, void* o,

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_kalman_full.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_diag.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_decode_step.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
+    L.kdn_scan_kalman_full_noalloc.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
+    L.kdn_scan_kalman_full_noalloc.restype = ctypes.c_int
     L.kdn_workspace_bytes.argtypes = [i, dims]
     L.kdn_workspace_bytes.restype = sz
     L.kdn_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
@@ -203,6 +205,26 @@ def scan_kalman_full(q, k, v, r, a=None, qn=None, S=None, P=None, o=None, m=None
                                     _ptr(S), _ptr(P), _ptr(o), _ptr(m), _ptr(workspace), workspace.numel(),
                                     _stream(stream))
     _check(st, "kdn_scan_kalman_full")
+    return o, m, S, P
+
+
+def scan_kalman_full_noalloc(q, k, v, r, a=None, qn=None, S=None, P=None, o=None, m=None, chunk=0,
+                             out_dtype=None, stream=None):
+    """Full-Kalman scan without a workspace, for callers that cannot allocate one: the library uses a static
+    device array (B*H*L*d_k <= 4,194,304; overlapping calls race on it).  Returns (o, m, S, P)."""
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    B, H, L, dk = q.shape
+    tok = (B, H, L)
+    _need(r, "r", tok, torch.float32, q.device)
+    if a is not None:
+        _need(a, "a", tok, torch.float32, q.device)
+    qn_t, qn_s = _qn_args(qn, tok, q.device)
+    if P is None:
+        P = torch.eye(dk, dtype=torch.float32, device=q.device).repeat(B, H, 1, 1)
+    _need(P, "P", (B, H, dk, dk), torch.float32, q.device)
+    st = lib().kdn_scan_kalman_full_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(r),
+                                            _ptr(qn_t), qn_s, _ptr(S), _ptr(P), _ptr(o), _ptr(m), _stream(stream))
+    _check(st, "kdn_scan_kalman_full_noalloc")
     return o, m, S, P
 
 

@@ -122,6 +122,29 @@ KDN_EXPORT kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, 
                                 float* S, float* p, void* o, float* m,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* kdn_scan_kalman_full for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is a deployment variant.  Callers that must
+ * not call cudaMalloc while running (a server that reserves all device memory
+ * at start-up, a plugin whose host framework owns the device allocator, a
+ * real-time loop that forbids allocation) and have no buffer to spare for
+ * the workspace use this instead.  Same arguments, layouts and results as
+ * kdn_scan_kalman_full, minus the workspace; the library allocates nothing.
+ *   Scratch: a static device array inside the library (256-byte status word
+ *   plus 16 MiB of per-token gains), which every GPU that loads the library
+ *   holds until the process exits.  Limit: B*H*L*d_k <= 4,194,304; larger
+ *   requests return KDN_ERR_UNSUPPORTED (kdn_last_error() says why) and
+ *   enqueue nothing.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Sharing: every call, on every stream, uses the same array and leaves its
+ *   last contents behind (the status word is cleared at the start of each
+ *   call).  Calls whose GPU work overlaps race on it: serialise them.  The
+ *   device status word is not readable through this entry point. */
+KDN_EXPORT kdn_status kdn_scan_kalman_full_noalloc(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                                   const float* a, const float* r, const float* qn, float qn_scalar,
+                                                   float* S, float* P, void* o, float* m, void* stream);
+
 /* One recurrent token per head against a resident state (constant-memory
  * decoding: Kalman Delta Networks, Abstract).  variant: KDN_DELTA (beta
  * required, p ignored) or KDN_KALMAN_DIAG (r and p required).  q, k [B,H,d_k],
