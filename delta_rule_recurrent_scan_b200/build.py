@@ -23,11 +23,13 @@ LIB = os.path.join(LIB_DIR, "libkdn.so")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
     "-Xcompiler", "-fPIC,-O3,-fvisibility=hidden",
-    "-shared", "-cudart", "static",
     "--expt-relaxed-constexpr",
 ]
+# IEEE single precision everywhere except the chunked tensor-core kernel, whose operands are
+# well-scaled (no denormals matter) and whose reciprocals and divisions sit on serial chains.
+IEEE_FLAGS = ["-ftz=false", "-prec-div=true", "-prec-sqrt=true"]
+PER_FILE_FLAGS = {"chunk_scan.cu": ["-ftz=true", "-prec-div=false", "-prec-sqrt=false"]}
 
 
 def _nvcc() -> str:
@@ -54,11 +56,23 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(LIB_DIR, exist_ok=True)
+    obj_dir = os.path.join(LIB_DIR, "obj")
+    os.makedirs(obj_dir, exist_ok=True)
+    objs = []
+    for src in sources():
+        name = os.path.basename(src)
+        obj = os.path.join(obj_dir, name + ".o")
+        cmd = [_nvcc(), *NVCC_FLAGS, *PER_FILE_FLAGS.get(name, IEEE_FLAGS), "-I", INCLUDE, "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.run(cmd, check=True)
+        objs.append(obj)
     tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
+    link = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
+            "-Xcompiler", "-fPIC", "-o", tmp, *objs]
     if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.run(cmd, check=True)
+        print(" ".join(link), flush=True)
+    subprocess.run(link, check=True)
     os.replace(tmp, LIB)
     return LIB
 

@@ -41,7 +41,7 @@ namespace kdn {
 namespace {
 
 constexpr int kC = 64;          // tokens per chunk
-constexpr int kThreads = 256;   // 8 warps: warp w reads TMEM lanes 32*(w%4).., column half w/4
+constexpr int kThreads = 512;   // 16 warps: warp w reads TMEM lanes 32*(w%4).., column quarter w/4
 constexpr long long kWaitCycles = 2000000000LL;  // bounded waits: about one second
 
 enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
@@ -81,8 +81,8 @@ struct Layout {
   static constexpr int SMEM = TOTAL + 1024;         // + alignment slack
   // fp32 [64][D] gain scratch in the R/E area (2 * NP * 8 KB = 256 * D bytes)
   static constexpr int OFF_GF = OFF_RHI;
-  // TMEM columns
-  static constexpr uint32_t T_D1 = 0, T_D2 = 64, T_DT = 64 + D, T_D3 = 128 + D, T_D4 = 128 + 2 * D;
+  // TMEM columns; T_SM holds the fp32 state master, which D4 = G^T Et accumulates onto
+  static constexpr uint32_t T_D1 = 0, T_D2 = 64, T_DT = 64 + D, T_D3 = 128 + D, T_SM = 128 + 2 * D;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(128 + 3 * D <= 512, "TMEM budget");
   static_assert(TOTAL <= 224 * 1024, "shared memory budget");
@@ -114,9 +114,11 @@ __device__ __forceinline__ void named_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ float quad_sum(float x) {
+// Sum over the 8 consecutive lanes that share a token.
+__device__ __forceinline__ float oct_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);
   x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
   return x;
 }
 
@@ -142,9 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, Params P) {
   using Lay = Layout<D, VAR>;
   constexpr int NP = Lay::NP;
-  constexpr int HALF = D / 2;  // d_v columns per column half
+  constexpr int QC = D / 4;    // d_v columns per column quarter
   constexpr int LD = Lay::SCR_LD;
-  constexpr int QD = D / 4;    // coordinates per thread in the per-token reductions
+  constexpr int GD = D / 8;    // coordinates per thread in the per-token reductions (8 threads per token)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -162,13 +164,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* Gf = reinterpret_cast<float*>(sm + Lay::OFF_GF);
 
   __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];  // a, beta|r, Qn of this chunk and the next
-  __shared__ float ell[kC], Aex[kC], Arat[kC], gn[kC], en[2][kC];
+  __shared__ float ell[kC], Aex[kC], Arat[kC], gn[kC], en[4][kC];
   __shared__ uint64_t bar_kq[2], bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int qw = warp & 3, ch = warp >> 2;
-  const int row = 32 * qw + lane;  // TMEM lane of this thread
+  const int qw = warp & 3, cq = warp >> 2;  // TMEM lane quarter, column quarter
+  const int row = 32 * qw + lane;           // TMEM lane of this thread
   const int bh = blockIdx.x;
   const int L = P.L;
   const int nchunks = (L + kC - 1) / kC;
@@ -223,40 +225,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   fetch_scalars(0);
   store_scalars(0);
-
-  // ---- state: fp32 master in registers (thread = d_k row, one column half), bf16 hi/lo panels for the MMAs
-  float Sr[HALF];
-  const bool s_owner = row < D;
-  float* Sg = P.S + (size_t)bh * D * D;
-  if (s_owner) {
-#pragma unroll
-    for (int c = 0; c < HALF; c += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(Sg + (size_t)row * D + ch * HALF + c);
-      Sr[c] = x.x, Sr[c + 1] = x.y, Sr[c + 2] = x.z, Sr[c + 3] = x.w;
-    }
-  }
-  // diagonal covariance: coordinate tid (threads 0 .. D-1)
-  float pcur = 1.f;
-  if (VAR == kDiag && tid < D) pcur = P.p[(size_t)bh * D + tid];
-
-  auto write_state_panels = [&]() {
-    if (!s_owner) return;
-#pragma unroll
-    for (int c8 = 0; c8 < HALF / 8; ++c8) {
-      const int c = ch * HALF + c8 * 8;  // d_v column
-      float x[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = Sr[c8 * 8 + e];
-      store8_split(Shi, Slo, (c / 64) * Lay::S_PANEL + sm100::sw128_chunk(row, (c % 64) / 8), x);
-    }
-  };
-  write_state_panels();
-  sm100::fence_async_smem();
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = tmem_base;
   const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+
+  // ---- state: thread (lane row, column quarter) owns S[row][cq*QC .. +QC); fp32 master in TMEM,
+  //      bf16 hi/lo panels in shared memory for the [K;Q] S0 product
+  const bool s_owner = row < D;
+  float* Sg = P.S + (size_t)bh * D * D;
+  auto write_state_panels = [&](const float (&x)[QC]) {
+#pragma unroll
+    for (int u = 0; u < QC / 8; ++u) {
+      const int c = cq * QC + 8 * u;  // d_v column
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = x[8 * u + e];
+      store8_split(Shi, Slo, (c / 64) * Lay::S_PANEL + sm100::sw128_chunk(row, (c % 64) / 8), y);
+    }
+  };
+  if (s_owner) {  // warp-uniform: D is 64 or 128
+    float x[QC];
+#pragma unroll
+    for (int c = 0; c < QC; c += 4) {
+      const float4 v4 = *reinterpret_cast<const float4*>(Sg + (size_t)row * D + cq * QC + c);
+      x[c] = v4.x, x[c + 1] = v4.y, x[c + 2] = v4.z, x[c + 3] = v4.w;
+    }
+    sm100::tmem_st<QC>(tmem + t_lane + Lay::T_SM + cq * QC, x);
+    write_state_panels(x);
+    sm100::tmem_wait_st();
+  }
+  // diagonal covariance: coordinate tid (threads 0 .. D-1)
+  float pcur = 1.f;
+  if (VAR == kDiag && tid < D) pcur = P.p[(size_t)bh * D + tid];
+  sm100::fence_async_smem();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
 
   uint32_t mma_phase = 0;
   bool aborted = false;
@@ -305,7 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (VAR == kDelta) sm100::mma_commit(&bar_mma);
     }
-
     if (c + 1 < nchunks) fetch_scalars(c + 1);
 
     // ---------------------------------------------------------------- gates
@@ -354,13 +359,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // ---------------------------------------------------------------- gains: norms, hi/lo panels (4 threads per token)
+    // ---------------------------------------------------------------- gains: norms, hi/lo panels (8 threads per token)
     {
-      const int t = tid >> 2, part = tid & 3;
-      const int i0 = part * QD;  // first coordinate of this thread
-      float kv[QD];
+      const int t = tid >> 3, part = tid & 7;
+      const int i0 = part * GD;  // first coordinate of this thread
+      float kv[GD];
 #pragma unroll
-      for (int u = 0; u < QD / 8; ++u) {
+      for (int u = 0; u < GD / 8; ++u) {
         float x[8];
         const int i = i0 + 8 * u;
         load8_bf16(KQ + (i / 64) * Lay::KQ_PANEL, sm100::sw128_chunk(t, (i % 64) / 8), x);
@@ -370,29 +375,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (VAR == kDelta) {
         float s = 0.f;
 #pragma unroll
-        for (int e = 0; e < QD; ++e) s = fmaf(kv[e], kv[e], s);
-        s = quad_sum(s);
+        for (int e = 0; e < GD; ++e) s = fmaf(kv[e], kv[e], s);
+        s = oct_sum(s);
         if (part == 0) gn[t] = b_c[t] * b_c[t] * s;
       } else {
-        float g[QD];
+        float g[GD];
         if (VAR == kDiag) {
 #pragma unroll
-          for (int e = 0; e < QD; e += 4) {
+          for (int e = 0; e < GD; e += 4) {
             const float4 x = *reinterpret_cast<const float4*>(Gf + t * D + i0 + e);
             g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
           }
           float s = 0.f;
 #pragma unroll
-          for (int e = 0; e < QD; ++e) s = fmaf(g[e], kv[e], s);
-          s = quad_sum(s) + b_c[t];
+          for (int e = 0; e < GD; ++e) s = fmaf(g[e], kv[e], s);
+          s = oct_sum(s) + b_c[t];
           if (part == 0 && !(s > 0.f && isfinite(s))) raise_status(P.status, kStatusNumeric);
           const float inv_s = 1.f / s;
 #pragma unroll
-          for (int e = 0; e < QD; ++e) g[e] *= inv_s;
+          for (int e = 0; e < GD; ++e) g[e] *= inv_s;
         } else {
           const bool valid = t0 + t < L;
 #pragma unroll
-          for (int e = 0; e < QD; e += 4) {
+          for (int e = 0; e < GD; e += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (valid) x = *reinterpret_cast<const float4*>(P.gains + ((size_t)bh * L + t0 + t) * D + i0 + e);
             g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
@@ -400,11 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float n2 = 0.f;
 #pragma unroll
-        for (int e = 0; e < QD; ++e) n2 = fmaf(g[e], g[e], n2);
-        n2 = quad_sum(n2);
+        for (int e = 0; e < GD; ++e) n2 = fmaf(g[e], g[e], n2);
+        n2 = oct_sum(n2);
         if (part == 0) gn[t] = n2;
 #pragma unroll
-        for (int u = 0; u < QD / 8; ++u) {
+        for (int u = 0; u < GD / 8; ++u) {
           const int i = i0 + 8 * u;
           float x[8];
 #pragma unroll
@@ -441,62 +446,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (qw < 2) {
       const int i = row;  // token in chunk
       {
-        // N_ij = (K G^T)_ij Gam_ij for j < i
-        float Y[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * ch, Y);
+        // N_ij = (K G^T)_ij Gam_ij for j < i, columns 16 cq .. 16 cq + 15
+        float Y[16];
+        sm100::tmem_ld16(tmem + t_lane + Lay::T_D1 + 16 * cq, Y);
         sm100::tmem_wait_ld();
         const float li = ell[i];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
+        for (int e = 0; e < 16; e += 4) {
           float v4[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int j = 32 * ch + e + u;
+            const int j = 16 * cq + e + u;
             v4[u] = (j < i) ? Y[e + u] * __expf(li - ell[j]) * (VAR == kDelta ? b_c[j] : 1.f) : 0.f;
           }
-          *reinterpret_cast<float4*>(Nf + i * LD + 32 * ch + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+          *reinterpret_cast<float4*>(Nf + i * LD + 16 * cq + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
         }
       }
-      named_arrive(1, 256);  // N is ready
+      named_arrive(1, kThreads);  // N is ready
       const float Ai = Aex[i];
+      float X[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_D2 + cq * QC, X);
+      sm100::tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < HALF; cc += 32) {
-        const int c0 = ch * HALF + cc;
-        float X[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + c0, X);
-        sm100::tmem_wait_ld();
+      for (int u = 0; u < QC / 8; ++u) {
+        const int cb = cq * QC + 8 * u;
+        const uint32_t off = (cb / 64) * Lay::V_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8);
+        float vv[8], x[8];
+        load8_bf16(Vs, off, vv);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          const int cb = c0 + 8 * c8;
-          const uint32_t off = (cb / 64) * Lay::V_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8);
-          float vv[8], x[8];
-          load8_bf16(Vs, off, vv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = fmaf(-Ai, X[8 * c8 + e], vv[e]);
-          store8_split(Rhi, Rlo, off, x);
-        }
+        for (int e = 0; e < 8; ++e) x[e] = fmaf(-Ai, X[8 * u + e], vv[e]);
+        store8_split(Rhi, Rlo, off, x);
       }
     } else {
-      const int gt = (qw - 2) * 32 + lane + 64 * ch;  // 0..127 within this group
+      const int gt = (qw - 2) * 32 + lane + 64 * cq;  // 0..255 within this group
       {
         // Attn_ij = (Q G^T)_ij Gam_ij for j <= i, into rows 64.. of the [T; AT] panel
         const int i = row - 64;
-        float Y[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * ch, Y);
+        float Y[16];
+        sm100::tmem_ld16(tmem + t_lane + Lay::T_D1 + 16 * cq, Y);
         sm100::tmem_wait_ld();
         const float li = ell[i];
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
+        for (int h = 0; h < 2; ++h) {
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int j = 32 * ch + 8 * c8 + e;
-            x[e] = (j <= i) ? Y[8 * c8 + e] * __expf(li - ell[j]) * (VAR == kDelta ? b_c[j] : 1.f) : 0.f;
+            const int j = 16 * cq + 8 * h + e;
+            x[e] = (j <= i) ? Y[8 * h + e] * __expf(li - ell[j]) * (VAR == kDelta ? b_c[j] : 1.f) : 0.f;
           }
-          store8_split(Thi, Tlo, sm100::sw128_chunk(64 + i, 4 * ch + c8), x);
+          store8_split(Thi, Tlo, sm100::sw128_chunk(64 + i, 2 * cq + h), x);
         }
       }
-      named_sync(1, 256);  // wait for N
+      named_sync(1, kThreads);  // wait for N
       // ---- T = (I + N)^-1, blocked by 16: diagonal blocks right-looking (column cc of block b)
       if (gt < 64) {
         const int b = gt >> 4, cc = gt & 15;
@@ -514,56 +515,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = acc[i];
       }
-      named_sync(2, 128);
+      named_sync(2, kThreads / 2);
 #pragma unroll
       for (int d = 1; d < 4; ++d) {
         // off-diagonal blocks at distance d: T_ab = -T_aa sum_{k=b}^{a-1} N_ak T_kb (a = b + d)
-        for (int e = gt; e < (4 - d) * 64; e += 128) {
-          const int b = e >> 6, a = b + d, ii = (e >> 2) & 15, jq = e & 3;
+        const bool act = gt < (4 - d) * 64;
+        const int b = gt >> 6, a = b + d, ii = (gt >> 2) & 15, jq = gt & 3;
+        if (act) {
+          float nv[16 * 3];
+#pragma unroll
+          for (int k = 0; k < d; ++k)
+#pragma unroll
+            for (int l = 0; l < 16; l += 4) {
+              const float4 n4 = *reinterpret_cast<const float4*>(Nf + (16 * a + ii) * LD + 16 * (b + k) + l);
+              nv[16 * k + l] = n4.x, nv[16 * k + l + 1] = n4.y, nv[16 * k + l + 2] = n4.z, nv[16 * k + l + 3] = n4.w;
+            }
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int k = 0; k < d; ++k) {
-            const float* nrow = Nf + (16 * a + ii) * LD + 16 * (b + k);
+          for (int k = 0; k < d; ++k)
 #pragma unroll
             for (int l = 0; l < 16; ++l) {
-              const float n = nrow[l];
+              const float n = nv[16 * k + l];
               const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * (b + k) + l) * LD + 16 * b + 4 * jq);
               acc.x = fmaf(n, t4.x, acc.x), acc.y = fmaf(n, t4.y, acc.y);
               acc.z = fmaf(n, t4.z, acc.z), acc.w = fmaf(n, t4.w, acc.w);
             }
-          }
           // M_ab parked in the unused upper block (b, a)
           *reinterpret_cast<float4*>(Tf + (16 * b + ii) * LD + 16 * a + 4 * jq) = acc;
         }
-        named_sync(2, 128);
-        for (int e = gt; e < (4 - d) * 64; e += 128) {
-          const int b = e >> 6, a = b + d, ii = (e >> 2) & 15, jq = e & 3;
+        named_sync(2, kThreads / 2);
+        if (act) {
+          float tv[16];
+#pragma unroll
+          for (int l = 0; l < 16; l += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * a + ii) * LD + 16 * a + l);
+            tv[l] = t4.x, tv[l + 1] = t4.y, tv[l + 2] = t4.z, tv[l + 3] = t4.w;
+          }
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          const float* trow = Tf + (16 * a + ii) * LD + 16 * a;
 #pragma unroll
           for (int l = 0; l < 16; ++l) {
-            const float tv = trow[l];
             const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + l) * LD + 16 * a + 4 * jq);
-            acc.x = fmaf(tv, m4.x, acc.x), acc.y = fmaf(tv, m4.y, acc.y);
-            acc.z = fmaf(tv, m4.z, acc.z), acc.w = fmaf(tv, m4.w, acc.w);
+            acc.x = fmaf(tv[l], m4.x, acc.x), acc.y = fmaf(tv[l], m4.y, acc.y);
+            acc.z = fmaf(tv[l], m4.z, acc.z), acc.w = fmaf(tv[l], m4.w, acc.w);
           }
           *reinterpret_cast<float4*>(Tf + (16 * a + ii) * LD + 16 * b + 4 * jq) =
               make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         }
-        named_sync(2, 128);
+        named_sync(2, kThreads / 2);
       }
       // T (unit diagonal, zero above) as bf16 hi/lo into rows 0..63 of the [T; AT] panel
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int i = (gt >> 1) & 63, c8 = 4 * (gt & 1) + h;
+      for (int h = 0; h < 2; ++h) {
+        const int e = gt + 256 * h;
+        const int i = e >> 3, c8 = e & 7;
         const float4 lo4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8);
         const float4 hi4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8 + 4);
         const float tv[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
         float x[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = 8 * c8 + e;
-          x[e] = (j < i) ? tv[e] : (j == i ? 1.f : 0.f);
+        for (int u = 0; u < 8; ++u) {
+          const int j = 8 * c8 + u;
+          x[u] = (j < i) ? tv[u] : (j == i ? 1.f : 0.f);
         }
         store8_split(Thi, Tlo, sm100::sw128_chunk(i, c8), x);
       }
@@ -591,15 +603,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_phase ^= 1;
     if (qw >= 2) {
       const int i = row - 64;
-      float X[32];
-      sm100::tmem_ld32(tmem + t_lane + Lay::T_DT + 32 * ch, X);
+      float X[16];
+      sm100::tmem_ld16(tmem + t_lane + Lay::T_DT + 16 * cq, X);
       sm100::tmem_wait_ld();
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
+      for (int h = 0; h < 2; ++h) {
         float x[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = X[8 * c8 + e];
-        store8_split(Thi, Tlo, sm100::sw128_chunk(64 + i, 4 * ch + c8), x);
+        for (int e = 0; e < 8; ++e) x[e] = X[8 * h + e];
+        store8_split(Thi, Tlo, sm100::sw128_chunk(64 + i, 2 * cq + h), x);
       }
     }
     sm100::fence_async_smem();
@@ -624,69 +636,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(&bar_mma, mma_phase, nullptr, 0)) { aborted = true; break; }
     mma_phase ^= 1;
 
-    // ---------------------------------------------------------------- E -> scaled E panels; O out
+    // ---------------------------------------------------------------- E -> scaled E panels; O out; S master *= A_C
     const float AC = Aex[kC - 1];
     if (qw < 2) {
       const int i = row;
       const float sc = Arat[i] * (VAR == kDelta ? b_c[i] : 1.f);
+      float X[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_D3 + cq * QC, X);
+      sm100::tmem_wait_ld();
       float es = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < HALF; cc += 32) {
-        const int c0 = ch * HALF + cc;
-        float X[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D3 + c0, X);
-        sm100::tmem_wait_ld();
+      for (int u = 0; u < QC / 8; ++u) {
+        const int cb = cq * QC + 8 * u;
+        float x[8];
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          const int cb = c0 + 8 * c8;
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            es = fmaf(X[8 * c8 + e], X[8 * c8 + e], es);
-            x[e] = X[8 * c8 + e] * sc;
-          }
-          store8_split(Rhi, Rlo, (cb / 64) * Lay::RE_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8), x);
+        for (int e = 0; e < 8; ++e) {
+          es = fmaf(X[8 * u + e], X[8 * u + e], es);
+          x[e] = X[8 * u + e] * sc;
         }
+        store8_split(Rhi, Rlo, (cb / 64) * Lay::RE_PANEL + sm100::sw128_chunk(i, (cb % 64) / 8), x);
       }
-      en[ch][i] = es;
+      en[cq][i] = es;
     } else {
       const int i = row - 64;
       const int tok = t0 + i;
       const float Ai = Aex[i];
+      float Y[QC], Oi[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_D2 + cq * QC, Y);
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_D3 + cq * QC, Oi);
+      sm100::tmem_wait_ld();
+      if (tok < L) {
+        const size_t off = ((size_t)bh * L + tok) * D + cq * QC;
+        if (P.out_dtype == kF32) {
+          float* op = reinterpret_cast<float*>(P.o) + off;
 #pragma unroll
-      for (int cc = 0; cc < HALF; cc += 32) {
-        const int c0 = ch * HALF + cc;
-        float Y[32], Oi[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + c0, Y);
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D3 + c0, Oi);
-        sm100::tmem_wait_ld();
-        if (tok < L) {
-          const size_t off = ((size_t)bh * L + tok) * D + c0;
-          if (P.out_dtype == kF32) {
-            float* op = reinterpret_cast<float*>(P.o) + off;
+          for (int e = 0; e < QC; e += 4)
+            *reinterpret_cast<float4*>(op + e) = make_float4(fmaf(Ai, Y[e], Oi[e]), fmaf(Ai, Y[e + 1], Oi[e + 1]),
+                                                             fmaf(Ai, Y[e + 2], Oi[e + 2]), fmaf(Ai, Y[e + 3], Oi[e + 3]));
+        } else {
+          __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(P.o) + off;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(op + e) = make_float4(fmaf(Ai, Y[e], Oi[e]), fmaf(Ai, Y[e + 1], Oi[e + 1]),
-                                                               fmaf(Ai, Y[e + 2], Oi[e + 2]), fmaf(Ai, Y[e + 3], Oi[e + 3]));
-          } else {
-            __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(P.o) + off;
+          for (int e = 0; e < QC; e += 8) {
+            __align__(16) __nv_bfloat16 h[8];
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              __align__(16) __nv_bfloat16 h[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) h[u] = __float2bfloat16_rn(fmaf(Ai, Y[e + u], Oi[e + u]));
-              *reinterpret_cast<uint4*>(op + e) = *reinterpret_cast<const uint4*>(h);
-            }
+            for (int u = 0; u < 8; ++u) h[u] = __float2bfloat16_rn(fmaf(Ai, Y[e + u], Oi[e + u]));
+            *reinterpret_cast<uint4*>(op + e) = *reinterpret_cast<const uint4*>(h);
           }
         }
       }
+    }
+    if (s_owner) {  // the product Gm^T Et accumulates onto A_C S0
+      float x[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_SM + cq * QC, x);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < QC; ++e) x[e] *= AC;
+      sm100::tmem_st<QC>(tmem + t_lane + Lay::T_SM + cq * QC, x);
+      sm100::tmem_wait_st();
     }
     sm100::fence_async_smem();
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
 
-    // ---------------------------------------------------------------- D4 = G^T Et
+    // ---------------------------------------------------------------- S master += G^T Et
     if (tid == 0) {
       constexpr uint32_t id = sm100::idesc_bf16(128, D, true, true);
 #pragma unroll
@@ -695,35 +708,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bl = sm100::smem_desc(rlo + ks * 2048, Lay::RE_PANEL, 1024);
         if (VAR == kDelta) {
           const uint64_t ak = sm100::smem_desc(kq0 + ks * 2048, Lay::KQ_PANEL, 1024);
-          sm100::mma_bf16(tmem + Lay::T_D4, ak, bh_, id, ks > 0);
-          sm100::mma_bf16(tmem + Lay::T_D4, ak, bl, id, true);
+          sm100::mma_bf16(tmem + Lay::T_SM, ak, bh_, id, true);
+          sm100::mma_bf16(tmem + Lay::T_SM, ak, bl, id, true);
         } else {
           const uint64_t ah = sm100::smem_desc(ghi + ks * 2048, Lay::G_PANEL, 1024);
           const uint64_t al = sm100::smem_desc(glo + ks * 2048, Lay::G_PANEL, 1024);
-          sm100::mma_bf16(tmem + Lay::T_D4, ah, bh_, id, ks > 0);
-          sm100::mma_bf16(tmem + Lay::T_D4, al, bh_, id, true);
-          sm100::mma_bf16(tmem + Lay::T_D4, ah, bl, id, true);
+          sm100::mma_bf16(tmem + Lay::T_SM, ah, bh_, id, true);
+          sm100::mma_bf16(tmem + Lay::T_SM, al, bh_, id, true);
+          sm100::mma_bf16(tmem + Lay::T_SM, ah, bl, id, true);
         }
       }
       sm100::mma_commit(&bar_mma);
     }
     if (tid < kC && P.m != nullptr && t0 + tid < L)
-      P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[tid]) * sqrtf(en[0][tid] + en[1][tid]);
+      P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[tid]) * sqrtf(en[0][tid] + en[1][tid] + en[2][tid] + en[3][tid]);
     if (!wait_all(&bar_mma, mma_phase, nullptr, 0)) { aborted = true; break; }
     mma_phase ^= 1;
 
-    // ---------------------------------------------------------------- S <- A_C S + D4
+    // ---------------------------------------------------------------- state panels for the next chunk
     if (s_owner) {
-#pragma unroll
-      for (int cc = 0; cc < HALF; cc += 32) {
-        float X[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_D4 + ch * HALF + cc, X);
-        sm100::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) Sr[cc + e] = fmaf(AC, Sr[cc + e], X[e]);
-      }
+      float x[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_SM + cq * QC, x);
+      sm100::tmem_wait_ld();
+      write_state_panels(x);
     }
-    write_state_panels();
     if (c + 1 < nchunks) store_scalars(sb ^ 1);
     sm100::fence_async_smem();
     sm100::tc_fence_before();
@@ -734,10 +742,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- write back the state (and the diagonal covariance)
   if (!aborted) {
     if (s_owner) {
+      float x[QC];
+      sm100::tmem_ld<QC>(tmem + t_lane + Lay::T_SM + cq * QC, x);
+      sm100::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < HALF; c += 4)
-        *reinterpret_cast<float4*>(Sg + (size_t)row * D + ch * HALF + c) =
-            make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
+      for (int e = 0; e < QC; e += 4)
+        *reinterpret_cast<float4*>(Sg + (size_t)row * D + cq * QC + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
     }
     if (VAR == kDiag && tid < D) P.p[(size_t)bh * D + tid] = pcur;
   }
