@@ -72,6 +72,36 @@ def decode_bytes(w, in_bytes=2, out_bytes=4) -> int:
     return n * per
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel from one ncu
+# capture, per token (it scales with the tokens of a launch).  Valid only for the kernel source it was
+# taken on: a different source hash reports null.
+NCU_TRAFFIC = {
+    "kalman_diag_d128": {"source": "delta_rule_recurrent_scan_b200/csrc/chunk_scan.cu",
+                         "sha1": "a4d45e21606002d911e4dc1a1f754a7982defd1b",
+                         "bytes_per_token": (205.815296e6 + 100.244480e6) / (2 * 16 * 8192),
+                         "capture": "profiles/chunk_scan_kernel_kalman_diag_d128.md (B=2 case, scaled)"},
+    "gdn_d128": {"source": "delta_rule_recurrent_scan_b200/csrc/chunk_scan.cu",
+                 "sha1": "a4d45e21606002d911e4dc1a1f754a7982defd1b",
+                 "bytes_per_token": (205.605376e6 + 100.905472e6) / (2 * 16 * 8192),
+                 "capture": "profiles/chunk_scan_kernel_delta_d128.md (B=2 case, scaled)"},
+}
+
+
+def ncu_traffic(w):
+    import hashlib
+
+    rec = NCU_TRAFFIC.get(w.name)
+    if rec is None:
+        return None
+    try:
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != rec["sha1"]:
+                return None
+    except OSError:
+        return None
+    return rec["bytes_per_token"] * w.tokens
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -391,7 +421,7 @@ def main():
                        "parallelism": f"dp{world} (independent heads, no collective)",
                        "kernel_path": plan},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                         "frac": achieved / peak, "traffic": ncu_traffic(w), "peak_source": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "kernel": plan["kernel"],
                          "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events"},
             "e2e": None if e2e is None else {"value": e2e["value"], "unit": "tokens/s",
