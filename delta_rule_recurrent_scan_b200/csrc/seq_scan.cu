@@ -137,39 +137,48 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
     *reinterpret_cast<float4*>(Sg + (size_t)(rg + i * RG) * DV + cg * 4) = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
 }
 
-template <int DK>
-__global__ void __launch_bounds__(RowBlockLayout<DK, DK>::kThreads) kalman_full_gains_kernel(GainArgs args) {
-  using Lay = RowBlockLayout<DK, DK>;
-  constexpr int NT = Lay::kThreads, CG = Lay::kColGroups, RG = Lay::kRowGroups, RPT = Lay::kRowsPerThread;
-  constexpr int DKW = (DK + 31) / 32 * 32;
-  static_assert(NT >= DKW, "reduction needs whole warps over d_k");
+// Full-covariance Riccati recursion, one token at a time, one CTA per head.  Four
+// consecutive threads share column c of P (symmetric, so P^- k is a column dot
+// product); each holds d_k/4 of its rows in registers.  The accumulated process
+// noise is kept as a scalar offset, P = Pt + c I with c <- a^2 c + Qn, so the
+// diagonal is never touched: u = P^- k = a^2 Pt k + c k, Pt <- a^2 Pt - u u^T / s.
+// One block barrier per token (u and the pieces of s = k.u + r go through
+// double-buffered shared slots).  Shared vectors are stored with a 4-float skew
+// per 32 floats so that the four row segments of a column sit in distinct banks.
+__device__ __forceinline__ int skew32(int x) { return x + ((x >> 5) << 2); }
 
-  __shared__ float k_s[kTokBlock][DK];
+template <int DK>
+__global__ void __launch_bounds__(4 * DK) kalman_full_gains_kernel(GainArgs args) {
+  constexpr int NT = 4 * DK, RP = DK / 4, NW = NT / 32;
+  constexpr int DKS = (DK + DK / 8 + 3) / 4 * 4;  // skewed width, rows 16-byte aligned
+  __shared__ __align__(16) float k_s[kTokBlock][DKS];
   __shared__ float a_s[kTokBlock], qn_s[kTokBlock], r_s[kTokBlock];
-  __shared__ __align__(16) float red[RG][DK];
-  __shared__ float u_s[DK];
-  __shared__ float ured[DKW / 32];
+  __shared__ __align__(16) float u_s[2][DKS];
+  __shared__ float red[2][NW];
 
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int cg = tid % CG, rg = tid / CG;
+  const int col = tid >> 2, part = tid & 3, r0 = part * RP;
   const int L = args.L;
   const size_t tok0 = (size_t)bh * L;
 
-  float P[RPT][4];
-  float* Pg = args.P + (size_t)bh * DK * DK;
+  float Pc[RP];  // Pt[r0 + i][col]
+  const float* Prow = args.P + (size_t)bh * DK * DK + (size_t)col * DK + r0;
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const float4 x = *reinterpret_cast<const float4*>(Pg + (size_t)(rg + i * RG) * DK + cg * 4);
-    P[i][0] = x.x, P[i][1] = x.y, P[i][2] = x.z, P[i][3] = x.w;
+  for (int i = 0; i < RP; i += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(Prow + i);
+    Pc[i] = x.x, Pc[i + 1] = x.y, Pc[i + 2] = x.z, Pc[i + 3] = x.w;
   }
+  float cI = 0.f;  // P = Pt + cI * I
+  const int sr0 = skew32(r0), scol = skew32(col);
 
+  int par = 0;
   for (int t0 = 0; t0 < L; t0 += kTokBlock) {
     const int nt = min(kTokBlock, L - t0);
     __syncthreads();
     for (int idx = tid; idx < nt * DK; idx += NT) {
       const int j = idx / DK, i = idx % DK;
-      k_s[j][i] = load_elem(args.k, (tok0 + t0 + j) * DK + i, args.in_dtype);
+      k_s[j][skew32(i)] = load_elem(args.k, (tok0 + t0 + j) * DK + i, args.in_dtype);
     }
     for (int j = tid; j < nt; j += NT) {
       const size_t tk = tok0 + t0 + j;
@@ -179,51 +188,52 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DK>::kThreads) kalman_full_
     }
     __syncthreads();
     for (int j = 0; j < nt; ++j) {
-      const float a2 = a_s[j] * a_s[j], qn = qn_s[j];
-      float pu[4] = {0.f, 0.f, 0.f, 0.f};
+      const float a2 = a_s[j] * a_s[j];
+      cI = fmaf(a2, cI, qn_s[j]);
+      float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) {
-        const int row = rg + i * RG;
-        const float kr = k_s[j][row];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float x = fmaf(a2, P[i][c], (row == cg * 4 + c) ? qn : 0.f);
-          P[i][c] = x;
-          pu[c] = fmaf(x, kr, pu[c]);
-        }
+      for (int i = 0; i < RP; i += 4) {  // RP is a multiple of 4 and a segment never crosses a skew boundary
+        const float4 k4 = *reinterpret_cast<const float4*>(&k_s[j][sr0 + i]);
+        v0 = fmaf(Pc[i], k4.x, v0);
+        v1 = fmaf(Pc[i + 1], k4.y, v1);
+        v2 = fmaf(Pc[i + 2], k4.z, v2);
+        v3 = fmaf(Pc[i + 3], k4.w, v3);
       }
-      *reinterpret_cast<float4*>(&red[rg][cg * 4]) = make_float4(pu[0], pu[1], pu[2], pu[3]);
-      __syncthreads();
-      if (tid < DKW) {
-        float ku = 0.f;
-        if (tid < DK) {
-          float u = 0.f;
-#pragma unroll
-          for (int r = 0; r < RG; ++r) u += red[r][tid];
-          u_s[tid] = u;
-          ku = k_s[j][tid] * u;
-        }
-        ku = warp_sum(ku);
-        if (lane == 0) ured[warp] = ku;
-      }
+      float v = (v0 + v1) + (v2 + v3);
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      const float kc = k_s[j][scol];
+      v = fmaf(a2, v, cI * kc);  // u_col
+      float sp = (part == 0) ? kc * v : 0.f;
+      sp = warp_sum(sp);
+      if (part == 0) u_s[par][scol] = v;
+      if (lane == 0) red[par][warp] = sp;
       __syncthreads();
       float s = r_s[j];
 #pragma unroll
-      for (int w = 0; w < DKW / 32; ++w) s += ured[w];
+      for (int w = 0; w < NW; ++w) s += red[par][w];
       if (tid == 0 && !(s > 0.f && isfinite(s))) raise_status(args.status, kStatusNumeric);
-      const float inv_s = 1.f / s;
-      if (tid < DK) args.gains[(tok0 + t0 + j) * DK + tid] = u_s[tid] * inv_s;
+      const float gcol = v / s;
+      if (part == 0) args.gains[(tok0 + t0 + j) * DK + col] = gcol;
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) {
-        const float ur = u_s[rg + i * RG];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) P[i][c] -= (ur * u_s[cg * 4 + c]) * inv_s;
+      for (int i = 0; i < RP; i += 4) {
+        const float4 u4 = *reinterpret_cast<const float4*>(&u_s[par][sr0 + i]);
+        Pc[i] = fmaf(-u4.x, gcol, a2 * Pc[i]);
+        Pc[i + 1] = fmaf(-u4.y, gcol, a2 * Pc[i + 1]);
+        Pc[i + 2] = fmaf(-u4.z, gcol, a2 * Pc[i + 2]);
+        Pc[i + 3] = fmaf(-u4.w, gcol, a2 * Pc[i + 3]);
       }
+      par ^= 1;
     }
   }
+  if (col >= r0 && col < r0 + RP) {
 #pragma unroll
-  for (int i = 0; i < RPT; ++i)
-    *reinterpret_cast<float4*>(Pg + (size_t)(rg + i * RG) * DK + cg * 4) = make_float4(P[i][0], P[i][1], P[i][2], P[i][3]);
+    for (int i = 0; i < RP; ++i)
+      if (r0 + i == col) Pc[i] += cI;
+  }
+  float* Pw = args.P + (size_t)bh * DK * DK + (size_t)col * DK + r0;
+#pragma unroll
+  for (int i = 0; i < RP; i += 4) *reinterpret_cast<float4*>(Pw + i) = make_float4(Pc[i], Pc[i + 1], Pc[i + 2], Pc[i + 3]);
 }
 
 // One warp per head; the p recursion is sequential in t and cheap.
@@ -296,9 +306,7 @@ cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_
 
 cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream) {
   if (args.BH <= 0 || args.L <= 0) return cudaSuccess;
-  KDN_DIMS_SWITCH(dk, DK, {
-    kalman_full_gains_kernel<DK><<<args.BH, RowBlockLayout<DK, DK>::kThreads, 0, stream>>>(args);
-  });
+  KDN_DIMS_SWITCH(dk, DK, { kalman_full_gains_kernel<DK><<<args.BH, 4 * DK, 0, stream>>>(args); });
   return cudaGetLastError();
 }
 
