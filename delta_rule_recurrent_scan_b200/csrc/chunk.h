@@ -1,6 +1,7 @@
 // Internal interface of the chunked (tensor-core) scan kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/kdn.h"
@@ -26,6 +27,15 @@ struct ChunkArgs {
   unsigned* status;
   void* workspace;    // past the status word
 };
+
+// [BH][L][d] bf16 viewed as a 3-D tensor map with 64 x 64 boxes and the 128-byte swizzle.
+bool make_bf16_tmap(CUtensorMap* tm, const void* base, int BH, int L, int d);
+
+// Covariance side of the full-Kalman scan, chunked (Woodbury / LDL): per-token gains into ``gains``
+// ([BH, L, d] fp32) and P updated in place.  d in {64, 128}, bf16 keys.
+cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const float* r, const float* qn,
+                                float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
+                                cudaStream_t stream);
 
 // True when the chunked tensor-core kernel serves this request.
 bool chunk_supported(kdn_variant variant, const kdn_dims& dims);

@@ -34,15 +34,21 @@
 #include "chunk.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "chunk_common.cuh"
 #include "sm100.cuh"
 
 namespace kdn {
 
 namespace {
 
-constexpr int kC = 64;          // tokens per chunk
+using chunk::kC;
+using chunk::kWaitCycles;
+using chunk::load8_bf16;
+using chunk::named_arrive;
+using chunk::named_sync;
+using chunk::oct_sum;
+using chunk::store8_split;
 constexpr int kThreads = 512;   // 16 warps: warp w reads TMEM lanes 32*(w%4).., column quarter w/4
-constexpr long long kWaitCycles = 2000000000LL;  // bounded waits: about one second
 
 enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
 
@@ -88,39 +94,9 @@ struct Layout {
   static_assert(TOTAL <= 224 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ void store8_split(uint8_t* hi, uint8_t* lo, uint32_t off, const float (&x)[8]) {
-  __align__(16) __nv_bfloat16 h[8], l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) sm100::split_bf16(x[e], h[e], l[e]);
-  *reinterpret_cast<uint4*>(hi + off) = *reinterpret_cast<const uint4*>(h);
-  *reinterpret_cast<uint4*>(lo + off) = *reinterpret_cast<const uint4*>(l);
-}
 
-// 8 consecutive bf16 of a swizzled panel (one 16-byte chunk) as floats.
-__device__ __forceinline__ void load8_bf16(const uint8_t* base, uint32_t off, float (&x)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(base + off);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(h[e]);
-    x[2 * e] = f.x, x[2 * e + 1] = f.y;
-  }
-}
 
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void named_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
-// Sum over the 8 consecutive lanes that share a token.
-__device__ __forceinline__ float oct_sum(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  x += __shfl_xor_sync(0xffffffffu, x, 4);
-  return x;
-}
 
 struct Params {
   const float* beta;
@@ -498,71 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       named_sync(1, kThreads);  // wait for N
-      // ---- T = (I + N)^-1, blocked by 16: diagonal blocks right-looking (column cc of block b)
-      if (gt < 64) {
-        const int b = gt >> 4, cc = gt & 15;
-        const float* Nb = Nf + (16 * b) * LD + 16 * b;
-        float acc[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = (i == cc) ? 1.f : 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float tj = acc[j];
-#pragma unroll
-          for (int i = j + 1; i < 16; ++i) acc[i] = fmaf(-Nb[i * LD + j], tj, acc[i]);
-        }
-        float* Tb = Tf + (16 * b) * LD + 16 * b;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = acc[i];
-      }
-      named_sync(2, kThreads / 2);
-#pragma unroll
-      for (int d = 1; d < 4; ++d) {
-        // off-diagonal blocks at distance d: T_ab = -T_aa sum_{k=b}^{a-1} N_ak T_kb (a = b + d)
-        const bool act = gt < (4 - d) * 64;
-        const int b = gt >> 6, a = b + d, ii = (gt >> 2) & 15, jq = gt & 3;
-        if (act) {
-          float nv[16 * 3];
-#pragma unroll
-          for (int k = 0; k < d; ++k)
-#pragma unroll
-            for (int l = 0; l < 16; l += 4) {
-              const float4 n4 = *reinterpret_cast<const float4*>(Nf + (16 * a + ii) * LD + 16 * (b + k) + l);
-              nv[16 * k + l] = n4.x, nv[16 * k + l + 1] = n4.y, nv[16 * k + l + 2] = n4.z, nv[16 * k + l + 3] = n4.w;
-            }
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int k = 0; k < d; ++k)
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-              const float n = nv[16 * k + l];
-              const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * (b + k) + l) * LD + 16 * b + 4 * jq);
-              acc.x = fmaf(n, t4.x, acc.x), acc.y = fmaf(n, t4.y, acc.y);
-              acc.z = fmaf(n, t4.z, acc.z), acc.w = fmaf(n, t4.w, acc.w);
-            }
-          // M_ab parked in the unused upper block (b, a)
-          *reinterpret_cast<float4*>(Tf + (16 * b + ii) * LD + 16 * a + 4 * jq) = acc;
-        }
-        named_sync(2, kThreads / 2);
-        if (act) {
-          float tv[16];
-#pragma unroll
-          for (int l = 0; l < 16; l += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * a + ii) * LD + 16 * a + l);
-            tv[l] = t4.x, tv[l + 1] = t4.y, tv[l + 2] = t4.z, tv[l + 3] = t4.w;
-          }
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int l = 0; l < 16; ++l) {
-            const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + l) * LD + 16 * a + 4 * jq);
-            acc.x = fmaf(tv[l], m4.x, acc.x), acc.y = fmaf(tv[l], m4.y, acc.y);
-            acc.z = fmaf(tv[l], m4.z, acc.z), acc.w = fmaf(tv[l], m4.w, acc.w);
-          }
-          *reinterpret_cast<float4*>(Tf + (16 * a + ii) * LD + 16 * b + 4 * jq) =
-              make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        }
-        named_sync(2, kThreads / 2);
-      }
+      // ---- T = (I + N)^-1 (group of the 256 threads that own lanes 64..127)
+      chunk::invert_unit_lower_64(Nf, Tf, gt, [] { named_sync(2, kThreads / 2); });
       // T (unit diagonal, zero above) as bf16 hi/lo into rows 0..63 of the [T; AT] panel
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -776,7 +689,7 @@ EncodeTiledFn encode_fn() {
 }
 
 // [BH][L][d] bf16 viewed as a 3-D tensor; 64 x 64 boxes with the 128-byte swizzle.
-bool make_tmap(CUtensorMap* tm, const void* base, int BH, int L, int d) {
+bool make_tmap_impl(CUtensorMap* tm, const void* base, int BH, int L, int d) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
@@ -801,6 +714,8 @@ cudaError_t launch_typed(const CUtensorMap& q, const CUtensorMap& k, const CUten
 
 }  // namespace
 
+bool make_bf16_tmap(CUtensorMap* tm, const void* base, int BH, int L, int d) { return make_tmap_impl(tm, base, BH, L, d); }
+
 bool chunk_supported(kdn_variant variant, const kdn_dims& d) {
   (void)variant;
   return d.in_dtype == KDN_BF16 && d.dk == d.dv && (d.dk == 64 || d.dk == 128) && (d.chunk == 0 || d.chunk == 64) &&
@@ -809,23 +724,23 @@ bool chunk_supported(kdn_variant variant, const kdn_dims& d) {
 
 void chunk_plan(kdn_variant variant, const kdn_dims&, int* launches, const char** kernel, const char** arith) {
   *launches = variant == KDN_KALMAN_FULL ? 2 : 1;
-  *kernel = variant == KDN_KALMAN_FULL ? "kalman_full_gains_kernel" : "chunk_scan_kernel";
+  *kernel = variant == KDN_KALMAN_FULL ? "kalman_pside_kernel" : "chunk_scan_kernel";
   *arith = "bf16-tc";
 }
 
 cudaError_t launch_chunk(kdn_variant variant, const kdn_dims& d, const ChunkArgs& a, cudaStream_t stream) {
   const int BH = a.BH;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, a.q, BH, a.L, d.dk) || !make_tmap(&tk, a.k, BH, a.L, d.dk) || !make_tmap(&tv, a.v, BH, a.L, d.dv))
+  if (!make_tmap_impl(&tq, a.q, BH, a.L, d.dk) || !make_tmap_impl(&tk, a.k, BH, a.L, d.dk) ||
+      !make_tmap_impl(&tv, a.v, BH, a.L, d.dv))
     return cudaErrorInvalidValue;
   Params p{};
   p.beta = a.beta, p.a = a.a, p.r = a.r, p.qn = a.qn, p.qn_scalar = a.qn_scalar;
   p.S = a.S, p.o = a.o, p.m = a.m, p.out_dtype = a.out_dtype, p.L = a.L, p.status = a.status;
   if (variant == KDN_KALMAN_FULL) {
-    // covariance side first: per-token gains into the workspace, then the chunked S side
+    // covariance side first (chunked Woodbury / LDL): per-token gains into the workspace, then the S side
     float* gains = reinterpret_cast<float*>(a.workspace);
-    GainArgs g{a.k, KDN_BF16, a.a, a.r, a.qn, a.qn_scalar, a.P, nullptr, gains, a.status, BH, a.L};
-    cudaError_t e = launch_kalman_full_gains(d.dk, g, stream);
+    cudaError_t e = launch_kalman_pside(d.dk, a.k, a.a, a.r, a.qn, a.qn_scalar, a.P, gains, a.status, BH, a.L, stream);
     if (e != cudaSuccess) return e;
     p.gains = gains;
     return d.dk == 64 ? launch_typed<64, kFull>(tq, tk, tv, p, BH, stream)

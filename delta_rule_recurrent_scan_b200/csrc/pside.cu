@@ -1,0 +1,565 @@
+// Covariance side of the full-Kalman scan, chunked: the Woodbury form with an LDL of the innovation Gram.
+//
+// Kalman Delta Networks, Abstract (the Kalman gain weights each residual write; exact tracking is a dense,
+// state-dependent Riccati recursion) and Memory by Design, Abstract (exact Bayesian filtering of mean and
+// covariance).  For a chunk of C = 64 tokens with prior covariance P0, the joint Gaussian of the chunk's
+// observations gives every per-token gain without the 64 rank-1 Riccati steps:
+//
+//   gamma_j = a_j^2 gamma_{j-1} + Qn_j,  A_j = prod_{m<=j} a_m,  Gam_ij = A_i / A_j
+//   U = K P0,  Bt_j = A_j^2 U_j + gamma_j k_j                    (Bt_j = Pi_j k_j, Pi_j = A_j^2 P0 + gamma_j I)
+//   G_ij = Gam_ij k_i . Bt_j (i >= j, symmetric) + r_i [i = j]   (innovation Gram)  =  L D L^T
+//   Z = (L^-1 o Gam) Bt,  g_t = Z_t / D_t,  s_t = D_t
+//   P_C = A_C^2 P0 + gamma_C I - sum_j (A_C/A_j)^2 D_j g_j g_j^T
+//
+// U, the Gram, Z and the rank-64 covariance update run on the tcgen05 tensor cores (fp32 operands as
+// bf16 hi + lo); the LDL (blocked by 16) and the unit-lower-triangular inverse run on the CUDA cores.
+// One CTA per head walks the chunks; P lives in TMEM (fp32) with bf16 hi/lo panels for the next chunk's
+// U = K P0.  The gains go to the workspace for the state-side kernel.
+#include <cuda.h>
+
+#include "chunk.h"
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace kdn {
+
+namespace {
+
+using chunk::kC;
+using chunk::kLD;
+using chunk::kWaitCycles;
+using chunk::load8_bf16;
+using chunk::store8_split;
+
+constexpr int kPThreads = 256;  // 8 warps: warp w reads TMEM lanes 32*(w%4).., column half w/4
+
+template <int D>
+struct PLayout {
+  static constexpr int NP = D / 64;
+  static constexpr int K_PANEL = 128 * 128;   // K in rows 0..63; rows 64..127 are read (M = 128) but unused
+  static constexpr int P_PANEL = D * 128;     // d_k rows
+  static constexpr int B_PANEL = 64 * 128;
+  static constexpr int GL_BYTES = (NP * 64 * 128 > 128 * 128) ? NP * 64 * 128 : 128 * 128;
+  static constexpr int SCR = 64 * kLD * 4;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_PHI = OFF_K + NP * K_PANEL;
+  static constexpr int OFF_PLO = OFF_PHI + NP * P_PANEL;
+  static constexpr int OFF_BHI = OFF_PLO + NP * P_PANEL;  // Bt, later the weighted gains W G
+  static constexpr int OFF_BLO = OFF_BHI + NP * B_PANEL;
+  static constexpr int OFF_GHI = OFF_BLO + NP * B_PANEL;  // L^-1 o Gam (A of Z), later the gains G
+  static constexpr int OFF_GLO = OFF_GHI + GL_BYTES;
+  static constexpr int OFF_GF = OFF_GLO + GL_BYTES;       // fp32 Gram -> LDL (D on the diagonal, L below)
+  static constexpr int OFF_LF = OFF_GF + SCR;             // fp32 panel scratch, then L^-1
+  static constexpr int TOTAL = OFF_LF + SCR;
+  static constexpr int SMEM = TOTAL + 1024;
+  static constexpr uint32_t T_P = 0, T_U = D, T_W = 2 * D, T_Z = 2 * D + 64;
+  static constexpr uint32_t TMEM_COLS = (3 * D + 64 <= 256) ? 256 : 512;
+  static_assert(3 * D + 64 <= 512, "TMEM budget");
+  static_assert(TOTAL <= 224 * 1024, "shared memory budget");
+};
+
+struct PParams {
+  const float* a;
+  const float* r;
+  const float* qn;
+  float qn_scalar;
+  float* P;      // [BH, D, D] in: P_0, out: P_L
+  float* gains;  // [BH, L, D] out
+  int L;
+  unsigned* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPThreads, 1)
+    kalman_pside_kernel(const __grid_constant__ CUtensorMap tm_k, PParams P) {
+  using Lay = PLayout<D>;
+  constexpr int NP = Lay::NP;
+  constexpr int HALF = D / 2;
+  constexpr int LD = kLD;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Ks = sm + Lay::OFF_K;
+  uint8_t* Phi = sm + Lay::OFF_PHI;
+  uint8_t* Plo = sm + Lay::OFF_PLO;
+  uint8_t* Bhi = sm + Lay::OFF_BHI;
+  uint8_t* Blo = sm + Lay::OFF_BLO;
+  uint8_t* Ghi = sm + Lay::OFF_GHI;
+  uint8_t* Glo = sm + Lay::OFF_GLO;
+  float* Gf = reinterpret_cast<float*>(sm + Lay::OFF_GF);
+  float* Lf = reinterpret_cast<float*>(sm + Lay::OFF_LF);
+
+  __shared__ float sA[2][kC], sR[2][kC], sQ[2][kC];
+  __shared__ float ell[kC], Aex[kC], gam[kC];
+  __shared__ uint64_t bar_k, bar_mma;
+  __shared__ uint32_t tmem_base;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qw = warp & 3, ch = warp >> 2;
+  const int row = 32 * qw + lane;
+  const int bh = blockIdx.x;
+  const int L = P.L;
+  const int nchunks = (L + kC - 1) / kC;
+
+  float ra = 1.f, rr = 1.f, rq = 0.f;
+  auto fetch_scalars = [&](int cc) {
+    if (tid < kC) {
+      const int tok = cc * kC + tid;
+      const bool valid = tok < L;
+      const size_t ti = (size_t)bh * L + tok;
+      ra = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;
+      rr = valid ? P.r[ti] : 1.f;
+      rq = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;
+    }
+  };
+  auto store_scalars = [&](int buf) {
+    if (tid < kC) sA[buf][tid] = ra, sR[buf][tid] = rr, sQ[buf][tid] = rq;
+  };
+  auto issue_k = [&](int cc) {
+    sm100::mbar_arrive_expect_tx(&bar_k, NP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) sm100::tma_load_3d(Ks + pn * Lay::K_PANEL, &tm_k, &bar_k, 64 * pn, cc * kC, bh);
+  };
+
+  if (tid == 0) {
+    sm100::prefetch_tmap(&tm_k);
+    sm100::mbar_init(&bar_k, 1);
+    sm100::mbar_init(&bar_mma, 1);
+    sm100::fence_mbar_init();
+    issue_k(0);
+  }
+  if (warp == 0) {
+    sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
+    sm100::tmem_relinquish();
+  }
+  fetch_scalars(0);
+  store_scalars(0);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+
+  // ---- covariance: thread (lane row, column half) owns P[row][ch*HALF ..); fp32 master in TMEM
+  const bool p_owner = row < D;
+  float* Pg = P.P + (size_t)bh * D * D;
+  auto write_p_panels = [&](const float* x) {
+#pragma unroll
+    for (int u = 0; u < HALF / 8; ++u) {
+      const int c = ch * HALF + 8 * u;
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = x[8 * u + e];
+      store8_split(Phi, Plo, (c / 64) * Lay::P_PANEL + sm100::sw128_chunk(row, (c % 64) / 8), y);
+    }
+  };
+  if (p_owner) {
+#pragma unroll
+    for (int cc = 0; cc < HALF; cc += 32) {
+      float x[32];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(Pg + (size_t)row * D + ch * HALF + cc + e);
+        x[e] = v4.x, x[e + 1] = v4.y, x[e + 2] = v4.z, x[e + 3] = v4.w;
+      }
+      sm100::tmem_st32(tmem + t_lane + Lay::T_P + ch * HALF + cc, x);
+      const int c0 = ch * HALF + cc;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = x[8 * u + e];
+        store8_split(Phi, Plo, ((c0 + 8 * u) / 64) * Lay::P_PANEL + sm100::sw128_chunk(row, ((c0 + 8 * u) % 64) / 8), y);
+      }
+    }
+    sm100::tmem_wait_st();
+  }
+  sm100::fence_async_smem();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+
+  uint32_t mma_phase = 0;
+  bool aborted = false;
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int bad = 0;
+    if (tid == 0) bad = !sm100::mbar_wait_bounded(bar, parity, kWaitCycles);
+    bad = __syncthreads_or(bad);
+    if (bad && tid == 0) raise_status(P.status, kStatusTimeout);
+    sm100::tc_fence_after();
+    return !bad;
+  };
+  auto sync_all = [] { __syncthreads(); };
+
+  const uint32_t k0 = sm100::smem_u32(Ks);
+  const uint32_t phi = sm100::smem_u32(Phi), plo = sm100::smem_u32(Plo);
+  const uint32_t bhi = sm100::smem_u32(Bhi), blo = sm100::smem_u32(Blo);
+  const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int t0 = c * kC;
+    const int sb = c & 1;
+    const float* a_c = sA[sb];
+    const float* r_c = sR[sb];
+    const float* q_c = sQ[sb];
+
+    // ---------------------------------------------------------------- U = K P0
+    if (!wait_all(&bar_k, c & 1)) { aborted = true; break; }
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, D, false, true);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t a = sm100::smem_desc(k0 + (ks / 4) * Lay::K_PANEL + (ks % 4) * 32, 16, 1024);
+        sm100::mma_bf16(tmem + Lay::T_U, a, sm100::smem_desc(phi + ks * 2048, Lay::P_PANEL, 1024), id, ks > 0);
+        sm100::mma_bf16(tmem + Lay::T_U, a, sm100::smem_desc(plo + ks * 2048, Lay::P_PANEL, 1024), id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    if (c + 1 < nchunks) fetch_scalars(c + 1);
+    // ---------------------------------------------------------------- gates and the process-noise prefix
+    if (warp == 1) {
+      float x0 = a_c[lane], x1 = a_c[32 + lane];
+      // gamma_j = a_j^2 gamma_{j-1} + Qn_j: inclusive scan of the affine maps x -> a^2 x + Qn
+      float m0 = x0 * x0, b0 = q_c[lane], m1 = x1 * x1, b1 = q_c[32 + lane];
+      x0 = x0 > 0.f ? fmaxf(__logf(x0), -60.f) : -60.f;
+      x1 = x1 > 0.f ? fmaxf(__logf(x1), -60.f) : -60.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+        const float pm0 = __shfl_up_sync(0xffffffffu, m0, o), pb0 = __shfl_up_sync(0xffffffffu, b0, o);
+        const float pm1 = __shfl_up_sync(0xffffffffu, m1, o), pb1 = __shfl_up_sync(0xffffffffu, b1, o);
+        if (lane >= o) {
+          x0 += y0, x1 += y1;
+          b0 = fmaf(m0, pb0, b0), m0 *= pm0;  // (m, b) o (pm, pb) = (m pm, m pb + b)
+          b1 = fmaf(m1, pb1, b1), m1 *= pm1;
+        }
+      }
+      x1 += __shfl_sync(0xffffffffu, x0, 31);
+      const float g31 = __shfl_sync(0xffffffffu, b0, 31);
+      b1 = fmaf(m1, g31, b1);
+      ell[lane] = x0, ell[32 + lane] = x1;
+      Aex[lane] = __expf(x0), Aex[32 + lane] = __expf(x1);
+      gam[lane] = b0, gam[32 + lane] = b1;
+    }
+    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    mma_phase ^= 1;
+
+    // ---------------------------------------------------------------- Bt_j = A_j^2 U_j + gamma_j k_j
+    if (qw < 2) {
+      const int j = row;
+      const float A2 = Aex[j] * Aex[j], gj = gam[j];
+#pragma unroll
+      for (int cc = 0; cc < HALF; cc += 32) {
+        const int c0 = ch * HALF + cc;
+        float X[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_U + c0, X);
+        sm100::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int cb = c0 + 8 * u;
+          float kk[8], y[8];
+          load8_bf16(Ks + (cb / 64) * Lay::K_PANEL, sm100::sw128_chunk(j, (cb % 64) / 8), kk);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = fmaf(A2, X[8 * u + e], gj * kk[e]);
+          store8_split(Bhi, Blo, (cb / 64) * Lay::B_PANEL + sm100::sw128_chunk(j, (cb % 64) / 8), y);
+        }
+      }
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- W = K Bt^T
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t a = sm100::smem_desc(k0 + (ks / 4) * Lay::K_PANEL + (ks % 4) * 32, 16, 1024);
+        const uint32_t boff = (ks / 4) * Lay::B_PANEL + (ks % 4) * 32;
+        sm100::mma_bf16(tmem + Lay::T_W, a, sm100::smem_desc(bhi + boff, 16, 1024), id, ks > 0);
+        sm100::mma_bf16(tmem + Lay::T_W, a, sm100::smem_desc(blo + boff, 16, 1024), id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    mma_phase ^= 1;
+    if (tid == 0 && c + 1 < nchunks) issue_k(c + 1);  // K of this chunk is dead
+
+    // ---------------------------------------------------------------- innovation Gram (lower part)
+    if (qw < 2) {
+      const int i = row;
+      float X[32];
+      sm100::tmem_ld32(tmem + t_lane + Lay::T_W + 32 * ch, X);
+      sm100::tmem_wait_ld();
+      const float li = ell[i];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        float v4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 32 * ch + e + u;
+          v4[u] = (j <= i) ? X[e + u] * __expf(li - ell[j]) + (j == i ? r_c[i] : 0.f) : 0.f;
+        }
+        *reinterpret_cast<float4*>(Gf + i * LD + 32 * ch + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+      }
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- LDL of the Gram, blocked by 16
+    // In place on the lower part of Gf: D on the diagonal, the unit lower factor below it.  Scratch in
+    // Lf: the panel rows y = l D (rows 16..63, columns 0..15) and the panel transposed (rows 0..15).
+#pragma unroll 1
+    for (int kb = 0; kb < 4; ++kb) {
+      const int s0 = 16 * kb, s1 = s0 + 16;
+      if (warp == 0) {
+        // diagonal block in registers: lane i < 16 holds row s0 + i; right-looking with shuffles
+        float av[16];
+        const int li = lane & 15;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(Gf + (s0 + li) * LD + s0 + j);
+          av[j] = v4.x, av[j + 1] = v4.y, av[j + 2] = v4.z, av[j + 3] = v4.w;
+        }
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float dp = __shfl_sync(0xffffffffu, av[p], p);
+          const float lp = av[p] * (1.f / dp);
+#pragma unroll
+          for (int j = 1; j < 16; ++j) {  // fixed bounds: every register index is a constant
+            const float cj = __shfl_sync(0xffffffffu, av[p], j);  // A[s0+j][s0+p], not yet scaled
+            if (j > p && li > p && j <= li) av[j] = fmaf(-lp, cj, av[j]);
+          }
+          if (li > p) av[p] = lp;
+        }
+        if (lane < 16) {
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(Gf + (s0 + li) * LD + s0 + j) = make_float4(av[j], av[j + 1], av[j + 2], av[j + 3]);
+          float dpiv = 0.f;  // av[li] without a dynamic register index
+#pragma unroll
+          for (int j = 0; j < 16; ++j) dpiv = (j == li) ? av[j] : dpiv;
+          if (!(dpiv > 0.f && isfinite(dpiv))) raise_status(P.status, kStatusNumeric);
+        }
+      }
+      __syncthreads();
+      if (kb < 3) {
+        // panel rows i >= s1: solve y L_kk^T = x, l = y / D
+        const int nr = 64 - s1;
+        if (tid < nr) {
+          const int i = s1 + tid;
+          float y[16];
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            float v = Gf[i * LD + s0 + cc];
+#pragma unroll
+            for (int m = 0; m < 15; ++m)  // fixed bounds: every register index is a constant
+              if (m < cc) v = fmaf(-y[m], Gf[(s0 + cc) * LD + s0 + m], v);
+            y[cc] = v;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            const float l = y[cc] / Gf[(s0 + cc) * LD + s0 + cc];
+            Lf[i * LD + cc] = y[cc];
+            Lf[cc * LD + i] = l;  // transposed panel (rows 0..15)
+            Gf[i * LD + s0 + cc] = l;
+          }
+        }
+        __syncthreads();
+        // trailing update, strips of 4 columns: A[i][j..j+3] -= y_i . l_{j..j+3}
+        for (int idx = tid; idx < nr * (nr / 4); idx += kPThreads) {
+          const int i = s1 + idx / (nr / 4), j = s1 + 4 * (idx % (nr / 4));
+          if (j > i) continue;
+          float4 acc = *reinterpret_cast<const float4*>(Gf + i * LD + j);
+#pragma unroll
+          for (int cc = 0; cc < 16; cc += 4) {
+            const float4 y4 = *reinterpret_cast<const float4*>(Lf + i * LD + cc);
+            const float yv[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 l4 = *reinterpret_cast<const float4*>(Lf + (cc + u) * LD + j);
+              acc.x = fmaf(-yv[u], l4.x, acc.x), acc.y = fmaf(-yv[u], l4.y, acc.y);
+              acc.z = fmaf(-yv[u], l4.z, acc.z), acc.w = fmaf(-yv[u], l4.w, acc.w);
+            }
+          }
+          *reinterpret_cast<float4*>(Gf + i * LD + j) = acc;
+        }
+        __syncthreads();
+      }
+    }
+
+    // ---------------------------------------------------------------- L^-1, then (L^-1 o Gam) as bf16 hi/lo
+    chunk::invert_unit_lower_64(Gf, Lf, tid, sync_all);
+    {
+      const int t = tid >> 2, q4 = tid & 3;
+      const float lt = ell[t];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c8 = 2 * q4 + h;
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int m = 8 * c8 + e;
+          x[e] = (m < t) ? Lf[t * LD + m] * __expf(lt - ell[m]) : (m == t ? 1.f : 0.f);
+        }
+        store8_split(Ghi, Glo, sm100::sw128_chunk(t, c8), x);
+      }
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- Z = (L^-1 o Gam) Bt
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, D, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t ah = sm100::smem_desc(ghi + ks * 32, 16, 1024), al = sm100::smem_desc(glo + ks * 32, 16, 1024);
+        const uint64_t bh_ = sm100::smem_desc(bhi + ks * 2048, Lay::B_PANEL, 1024);
+        const uint64_t bl = sm100::smem_desc(blo + ks * 2048, Lay::B_PANEL, 1024);
+        sm100::mma_bf16(tmem + Lay::T_Z, ah, bh_, id, ks > 0);
+        sm100::mma_bf16(tmem + Lay::T_Z, al, bh_, id, true);
+        sm100::mma_bf16(tmem + Lay::T_Z, ah, bl, id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    mma_phase ^= 1;
+
+    // ---------------------------------------------------------------- gains, weighted gains; P <- A_C^2 P + gamma_C I
+    const float AC = Aex[kC - 1];
+    if (qw < 2) {
+      const int t = row;
+      const float Dt = Gf[t * LD + t];
+      const float inv_d = 1.f / Dt;
+      const float ratio = __expf(ell[kC - 1] - ell[t]);  // A_C / A_t
+      const float w = -ratio * ratio * Dt;
+      const bool valid = t0 + t < L;
+#pragma unroll
+      for (int cc = 0; cc < HALF; cc += 32) {
+        const int c0 = ch * HALF + cc;
+        float X[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_Z + c0, X);
+        sm100::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) X[e] *= inv_d;
+        if (valid) {
+          float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + c0;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(gp + e) = make_float4(X[e], X[e + 1], X[e + 2], X[e + 3]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int cb = c0 + 8 * u;
+          float g8[8], w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) g8[e] = X[8 * u + e], w8[e] = w * X[8 * u + e];
+          const uint32_t off = (cb / 64) * (64 * 128) + sm100::sw128_chunk(t, (cb % 64) / 8);
+          store8_split(Ghi, Glo, off, g8);
+          store8_split(Bhi, Blo, off, w8);
+        }
+      }
+    }
+    if (p_owner) {
+      const float AC2 = AC * AC, gC = gam[kC - 1];
+#pragma unroll
+      for (int cc = 0; cc < HALF; cc += 32) {
+        const int c0 = ch * HALF + cc;
+        float x[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_P + c0, x);
+        sm100::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = fmaf(AC2, x[e], (c0 + e == row) ? gC : 0.f);
+        sm100::tmem_st32(tmem + t_lane + Lay::T_P + c0, x);
+      }
+      sm100::tmem_wait_st();
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- P += G^T (w G)
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, D, true, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t ah = sm100::smem_desc(ghi + ks * 2048, 64 * 128, 1024);
+        const uint64_t al = sm100::smem_desc(glo + ks * 2048, 64 * 128, 1024);
+        const uint64_t bh_ = sm100::smem_desc(bhi + ks * 2048, Lay::B_PANEL, 1024);
+        const uint64_t bl = sm100::smem_desc(blo + ks * 2048, Lay::B_PANEL, 1024);
+        sm100::mma_bf16(tmem + Lay::T_P, ah, bh_, id, true);
+        sm100::mma_bf16(tmem + Lay::T_P, al, bh_, id, true);
+        sm100::mma_bf16(tmem + Lay::T_P, ah, bl, id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
+    mma_phase ^= 1;
+
+    // ---------------------------------------------------------------- P panels for the next chunk
+    if (p_owner) {
+#pragma unroll
+      for (int cc = 0; cc < HALF; cc += 32) {
+        float x[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_P + ch * HALF + cc, x);
+        sm100::tmem_wait_ld();
+        const int c0 = ch * HALF + cc;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = x[8 * u + e];
+          store8_split(Phi, Plo, ((c0 + 8 * u) / 64) * Lay::P_PANEL + sm100::sw128_chunk(row, ((c0 + 8 * u) % 64) / 8), y);
+        }
+      }
+    }
+    if (c + 1 < nchunks) store_scalars(sb ^ 1);
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+  }
+
+  if (!aborted && p_owner) {
+#pragma unroll
+    for (int cc = 0; cc < HALF; cc += 32) {
+      float x[32];
+      sm100::tmem_ld32(tmem + t_lane + Lay::T_P + ch * HALF + cc, x);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(Pg + (size_t)row * D + ch * HALF + cc + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) sm100::tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+template <int D>
+cudaError_t launch_pside_typed(const CUtensorMap& tk, const PParams& p, int BH, cudaStream_t stream) {
+  using Lay = PLayout<D>;
+  cudaError_t e = cudaFuncSetAttribute(kalman_pside_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+  if (e != cudaSuccess) return e;
+  kalman_pside_kernel<D><<<BH, kPThreads, Lay::SMEM, stream>>>(tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const float* r, const float* qn,
+                                float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
+                                cudaStream_t stream) {
+  CUtensorMap tk;
+  if (!make_bf16_tmap(&tk, k, BH, L, d)) return cudaErrorInvalidValue;
+  PParams p{a, r, qn, qn_scalar, P, gains, L, status};
+  if (d == 64) return launch_pside_typed<64>(tk, p, BH, stream);
+  if (d == 128) return launch_pside_typed<128>(tk, p, BH, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kdn
