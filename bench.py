@@ -178,11 +178,19 @@ def _barrier(dist_on):
 
 
 def _max_over_ranks(x: float, dist_on: bool) -> float:
+    """The slowest rank's value (NCCL groups reduce on the GPU, gloo groups on the CPU)."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, ms_per_step: float, world: int) -> float:
+    """Whole-job throughput: every rank runs its own batch of the same shape (independent heads);
+    the job's time is the slowest rank's."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
 
 
 def time_device(fn, steps, warmup, dist_on, clocks=None):
@@ -253,7 +261,7 @@ def bench_scan(w, steps, warmup, dist_on, rank, world, clocks=None):
     x = make_scan_inputs(w, seed=rank, device="cuda")
     fn, _ = scan_closure(w, x, kdn)
     ms = time_device(fn, steps, warmup, dist_on, clocks)
-    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": scan_plan(w)["launches"] * steps}
+    return {"ms": ms, "value": weak_scaling_value(w.tokens, ms, world), "launches": scan_plan(w)["launches"] * steps}
 
 
 def bench_e2e(w, steps, warmup, dist_on, rank, world):

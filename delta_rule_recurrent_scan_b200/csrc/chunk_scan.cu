@@ -308,30 +308,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------------------------------------------------------- diagonal variances
     if (VAR == kDiag && tid < D) {
-      // Per coordinate i (independent of v and S) each token maps the variance by the Moebius map
-      // p -> (r a^2 p + r Qn) / (k^2 a^2 p + k^2 Qn + r)  (Kalman Delta Networks, Abstract: the
-      // uncertainty recurrences are Moebius maps).  The 2x2 prefix product from the chunk start is
-      // the only serial chain; each p_{t-1} = P_{t-1}(p_0) and p^-_t k_t follow off the chain.
+      // Per coordinate i (independent of v and S): p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k).
+      // Eight tokens of keys and scalars are read ahead of the serial chain.
       const uint8_t* Kp = KQ + (tid / 64) * Lay::KQ_PANEL;
-      float m00 = 1.f, m01 = 0.f, m10 = 0.f, m11 = 1.f;
-      const float p0 = pcur;
-#pragma unroll 8
-      for (int t = 0; t < kC; ++t) {
-        const float at = a_c[t], rt = b_c[t], qt = q_c[t];
-        const float kt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t, tid % 64)));
-        const float pprev = __fdividef(fmaf(m00, p0, m01), fmaf(m10, p0, m11));
-        const float a2 = at * at, k2 = kt * kt;
-        Gf[t * D + tid] = fmaf(a2, pprev, qt) * kt;  // p^-_t k_t
-        const float e00 = rt * a2, e01 = rt * qt, e10 = k2 * a2, e11 = fmaf(k2, qt, rt);
-        const float n00 = fmaf(e00, m00, e01 * m10), n01 = fmaf(e00, m01, e01 * m11);
-        const float n10 = fmaf(e10, m00, e11 * m10), n11 = fmaf(e10, m01, e11 * m11);
-        m00 = n00, m01 = n01, m10 = n10, m11 = n11;
-        if ((t & 7) == 7) {  // maps are scale free: renormalise against under/overflow
-          const float sc = __fdividef(1.f, m11);
-          m00 *= sc, m01 *= sc, m10 *= sc, m11 = 1.f;
+#pragma unroll 1
+      for (int t8 = 0; t8 < kC; t8 += 8) {
+        float kk[8], aa[8], rr8[8], qq[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, tid % 64)));
+          aa[u] = a_c[t8 + u], rr8[u] = b_c[t8 + u], qq[u] = q_c[t8 + u];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float pp = fmaf(aa[u] * aa[u], pcur, qq[u]);
+          const float pk = pp * kk[u];
+          Gf[(t8 + u) * D + tid] = pk;
+          pcur = __fdividef(pp * rr8[u], fmaf(pk, kk[u], rr8[u]));
         }
       }
-      pcur = __fdividef(fmaf(m00, p0, m01), fmaf(m10, p0, m11));
     }
     __syncthreads();
 
