@@ -49,6 +49,9 @@ using chunk::named_sync;
 using chunk::oct_sum;
 using chunk::store8_split;
 constexpr int kThreads = 512;   // 16 warps: warp w reads TMEM lanes 32*(w%4).., column quarter w/4
+// One thread issues every tcgen05.mma and commit (a commit tracks only its own thread's products): the
+// first lane of the last warp, which has no part in the diagonal-variance recursion at a chunk's start.
+constexpr int kIssuer = kThreads - 32;
 
 enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
 
@@ -272,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- K, Q of this chunk; start [K;Q] S0
     if (!wait_all(&bar_kq[kb], (Lay::KQ_BUFS == 2) ? ((c >> 1) & 1) : (c & 1), nullptr, 0)) { aborted = true; break; }
-    if (tid == 0) {
-      if (Lay::KQ_BUFS == 2 && c + 1 < nchunks) issue_kq(c + 1, kb ^ 1);
+    if (tid == 0 && Lay::KQ_BUFS == 2 && c + 1 < nchunks) issue_kq(c + 1, kb ^ 1);
+    if (tid == kIssuer) {
       constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
       constexpr uint32_t id2 = sm100::idesc_bf16(128, D, false, true);
 #pragma unroll
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_after();
 
     // ---------------------------------------------------------------- D1 = [K;Q] G^T (Kalman gains)
-    if (tid == 0 && VAR != kDelta) {
+    if (tid == kIssuer && VAR != kDelta) {
       constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -495,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
 
     // ---------------------------------------------------------------- DT = [T; Attn] T  (rows 64..127: AT)
-    if (tid == 0) {
+    if (tid == kIssuer) {
       constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_after();
 
     // ---------------------------------------------------------------- D3 = [T; AT] R
-    if (tid == 0) {
+    if (tid == kIssuer) {
       constexpr uint32_t id = sm100::idesc_bf16(128, D, false, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
@@ -608,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_after();
 
     // ---------------------------------------------------------------- S master += G^T Et
-    if (tid == 0) {
+    if (tid == kIssuer) {
       constexpr uint32_t id = sm100::idesc_bf16(128, D, true, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
