@@ -37,6 +37,11 @@ cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const floa
                                 float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
                                 cudaStream_t stream);
 
+// Warp-specialised chunk kernel for d_k = d_v = 128 (preparation of chunk c + 1 beside the state chain
+// of chunk c).  ``gains``: full-Kalman per-token gains [BH, L, 128] fp32, else unused.
+cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& dims, const ChunkArgs& args, const float* gains,
+                            cudaStream_t stream);
+
 // True when the chunked tensor-core kernel serves this request.
 bool chunk_supported(kdn_variant variant, const kdn_dims& dims);
 void chunk_plan(kdn_variant variant, const kdn_dims& dims, int* launches, const char** kernel, const char** arith);

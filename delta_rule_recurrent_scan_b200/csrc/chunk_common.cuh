@@ -15,11 +15,13 @@ constexpr int kLD = 68;                           // row stride of the fp32 [64]
 
 // fp32 -> bf16 hi + lo for 8 consecutive values, stored as two 16-byte chunks.
 __device__ __forceinline__ void store8_split(uint8_t* hi, uint8_t* lo, uint32_t off, const float (&x)[8]) {
-  __align__(16) __nv_bfloat16 h[8], l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) sm100::split_bf16(x[e], h[e], l[e]);
-  *reinterpret_cast<uint4*>(hi + off) = *reinterpret_cast<const uint4*>(h);
-  *reinterpret_cast<uint4*>(lo + off) = *reinterpret_cast<const uint4*>(l);
+  uint4 h, l;
+  sm100::split2_bf16(x[0], x[1], h.x, l.x);
+  sm100::split2_bf16(x[2], x[3], h.y, l.y);
+  sm100::split2_bf16(x[4], x[5], h.z, l.z);
+  sm100::split2_bf16(x[6], x[7], h.w, l.w);
+  *reinterpret_cast<uint4*>(hi + off) = h;
+  *reinterpret_cast<uint4*>(lo + off) = l;
 }
 
 // 8 consecutive bf16 of a swizzled panel (one 16-byte chunk) as floats.
@@ -41,6 +43,20 @@ __device__ __forceinline__ void named_arrive(int id, int count) {
 }
 
 // Sum over the 8 consecutive lanes that share a token.
+// Named barrier over ``count`` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ float oct_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);
   x += __shfl_xor_sync(0xffffffffu, x, 2);
@@ -48,75 +64,119 @@ __device__ __forceinline__ float oct_sum(float x) {
   return x;
 }
 
-// T = (I + N)^-1 for a 64 x 64 strictly lower N (fp32, row stride kLD, only the strict lower part is
-// read).  T's lower part (the unit diagonal excluded) is written to Tf; its upper blocks are used as
-// scratch.  Run by the 256 threads gt = 0..255 of a group that synchronises with ``sync()``.
-// Blocked by 16: diagonal blocks right-looking (one thread per column), then the off-diagonal blocks by
-// distance d = 1..3, T_ab = -T_aa sum_{k=b}^{a-1} N_ak T_kb.
+// T = (I + N)^-1 for a 64 x 64 strictly lower N (fp32, row stride kLD; only the strict lower part of N
+// is read).  T's lower part is written to Tf (its unit diagonal and the zeros above it inside the 16 x 16
+// diagonal blocks too); the other upper blocks of Tf are scratch.  Run by the 256 threads gt = 0..255 of
+// a group that synchronises with ``sync()``.
+//   (1) diagonal blocks T_bb = (I + N_bb)^-1 by forward substitution, one thread per column;
+//   (2) 16 -> 32: T_{b+1,b} = -T_{b+1,b+1} (N_{b+1,b} T_bb) for b = 0, 2;
+//   (3) 32 -> 64: T_{[23],[01]} = -T_{[23],[23]} (N_{[23],[01]} T_{[01],[01]}),
+// the block form of the inverse of [[X, 0], [Y, Z]] at each doubling.
 template <class Sync>
 __device__ __forceinline__ void invert_unit_lower_64(const float* Nf, float* Tf, int gt, Sync sync) {
   constexpr int LD = kLD;
   if (gt < 64) {
     const int b = gt >> 4, cc = gt & 15;
     const float* Nb = Nf + (16 * b) * LD + 16 * b;
-    float acc[16];
+    float t[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = (i == cc) ? 1.f : 0.f;
+    for (int i = 0; i < 16; ++i) t[i] = (i == cc) ? 1.f : 0.f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float tj = acc[j];
+    for (int i = 1; i < 16; ++i) {
+      float acc = 0.f;
 #pragma unroll
-      for (int i = 1; i < 16; ++i)  // fixed bounds: every register index is a constant
-        if (i > j) acc[i] = fmaf(-Nb[i * LD + j], tj, acc[i]);
+      for (int q = 0; q < (i + 3) / 4; ++q) {
+        const float4 n4 = *reinterpret_cast<const float4*>(Nb + i * LD + 4 * q);
+        const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * q + e < i) acc = fmaf(nv[e], t[4 * q + e], acc);  // compile-time bounds: strict lower only
+      }
+      if (i > cc) t[i] = -acc;
     }
     float* Tb = Tf + (16 * b) * LD + 16 * b;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = acc[i];
+    for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = t[i];
   }
   sync();
+  // (2) pairs (a, b) = (1, 0), (3, 2): M = N_ab T_bb parked in the upper block (b, a), then T_ab = -T_aa M
+  {
+    const int pr = gt >> 6, i = (gt >> 2) & 15, jq = gt & 3;
+    const int a = 2 * pr + 1, b = 2 * pr;
+    if (gt < 128) {
+      float nv[16];
 #pragma unroll
-  for (int d = 1; d < 4; ++d) {
-    const bool act = gt < (4 - d) * 64;
-    const int b = gt >> 6, a = b + d, ii = (gt >> 2) & 15, jq = gt & 3;
-    if (act) {
-      float nv[16 * 3];
-#pragma unroll
-      for (int k = 0; k < d; ++k)
-#pragma unroll
-        for (int l = 0; l < 16; l += 4) {
-          const float4 n4 = *reinterpret_cast<const float4*>(Nf + (16 * a + ii) * LD + 16 * (b + k) + l);
-          nv[16 * k + l] = n4.x, nv[16 * k + l + 1] = n4.y, nv[16 * k + l + 2] = n4.z, nv[16 * k + l + 3] = n4.w;
-        }
+      for (int l = 0; l < 16; l += 4) {
+        const float4 n4 = *reinterpret_cast<const float4*>(Nf + (16 * a + i) * LD + 16 * b + l);
+        nv[l] = n4.x, nv[l + 1] = n4.y, nv[l + 2] = n4.z, nv[l + 3] = n4.w;
+      }
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < d; ++k)
-#pragma unroll
-        for (int l = 0; l < 16; ++l) {
-          const float n = nv[16 * k + l];
-          const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * (b + k) + l) * LD + 16 * b + 4 * jq);
-          acc.x = fmaf(n, t4.x, acc.x), acc.y = fmaf(n, t4.y, acc.y);
-          acc.z = fmaf(n, t4.z, acc.z), acc.w = fmaf(n, t4.w, acc.w);
-        }
-      // M_ab parked in the unused upper block (b, a)
-      *reinterpret_cast<float4*>(Tf + (16 * b + ii) * LD + 16 * a + 4 * jq) = acc;
+      for (int k = 0; k < 16; ++k) {
+        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * b + k) * LD + 16 * b + 4 * jq);
+        acc.x = fmaf(nv[k], t4.x, acc.x), acc.y = fmaf(nv[k], t4.y, acc.y);
+        acc.z = fmaf(nv[k], t4.z, acc.z), acc.w = fmaf(nv[k], t4.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(Tf + (16 * b + i) * LD + 16 * a + 4 * jq) = acc;
     }
     sync();
-    if (act) {
+    if (gt < 128) {
       float tv[16];
 #pragma unroll
       for (int l = 0; l < 16; l += 4) {
-        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * a + ii) * LD + 16 * a + l);
+        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * a + i) * LD + 16 * a + l);
         tv[l] = t4.x, tv[l + 1] = t4.y, tv[l + 2] = t4.z, tv[l + 3] = t4.w;
       }
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int l = 0; l < 16; ++l) {
-        const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + l) * LD + 16 * a + 4 * jq);
-        acc.x = fmaf(tv[l], m4.x, acc.x), acc.y = fmaf(tv[l], m4.y, acc.y);
-        acc.z = fmaf(tv[l], m4.z, acc.z), acc.w = fmaf(tv[l], m4.w, acc.w);
+      for (int k = 0; k < 16; ++k) {
+        const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + k) * LD + 16 * a + 4 * jq);
+        acc.x = fmaf(tv[k], m4.x, acc.x), acc.y = fmaf(tv[k], m4.y, acc.y);
+        acc.z = fmaf(tv[k], m4.z, acc.z), acc.w = fmaf(tv[k], m4.w, acc.w);
       }
-      *reinterpret_cast<float4*>(Tf + (16 * a + ii) * LD + 16 * b + 4 * jq) =
+      *reinterpret_cast<float4*>(Tf + (16 * a + i) * LD + 16 * b + 4 * jq) =
           make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    sync();
+  }
+  // (3) X = N_{[23],[01]} T_{[01],[01]} parked in rows 0..31, columns 32..63; then the lower-left 32 x 32
+  // block of T = -T_{[23],[23]} X.  Warps take uniform ranges: jh (columns 16 jh ..) and the row octet.
+  {
+    const int jh = gt >> 7, ii = (gt >> 2) & 31, jq = gt & 3;
+    const int j0 = 16 * jh + 4 * jq;
+    {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int kb = 0; kb < 32; kb += 4) {
+        if (kb < 16 * jh) continue;  // T_{[01],[01]}[k][j] = 0 for k < 16 <= j
+        const float4 n4 = *reinterpret_cast<const float4*>(Nf + (32 + ii) * LD + kb);
+        const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 t4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + j0);
+          acc.x = fmaf(nv[e], t4.x, acc.x), acc.y = fmaf(nv[e], t4.y, acc.y);
+          acc.z = fmaf(nv[e], t4.z, acc.z), acc.w = fmaf(nv[e], t4.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4*>(Tf + ii * LD + 32 + j0) = acc;
+    }
+    sync();
+    {
+      const int kend = ii < 16 ? 16 : 32;  // T_{[23],[23]}[i][k] = 0 for i < 16 <= k
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int kb = 0; kb < 32; kb += 4) {
+        if (kb >= kend) continue;
+        const float4 t4r = *reinterpret_cast<const float4*>(Tf + (32 + ii) * LD + 32 + kb);
+        const float tv[4] = {t4r.x, t4r.y, t4r.z, t4r.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 x4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + 32 + j0);
+          acc.x = fmaf(tv[e], x4.x, acc.x), acc.y = fmaf(tv[e], x4.y, acc.y);
+          acc.z = fmaf(tv[e], x4.z, acc.z), acc.w = fmaf(tv[e], x4.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4*>(Tf + (32 + ii) * LD + j0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
     sync();
   }

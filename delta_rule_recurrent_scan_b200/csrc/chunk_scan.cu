@@ -1,4 +1,5 @@
-// Chunked scan on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// Chunked scan on the sm_100a tensor cores (tcgen05 + TMEM + TMA), d_k = d_v = 64.  (d = 128 runs the
+// warp-specialised kernel of chunk_scan_ws.cu; the host entry below dispatches both.)
 //
 // One CTA per head walks the sequence in chunks of C = 64 tokens.  Within a
 // chunk, with A_i = prod_{m<=i} a_m and Gam_ij = A_i / A_j (i >= j), the
@@ -26,7 +27,7 @@
 // K, Q and V enter exactly (bf16); every fp32 operand (S0, G, T, AT, R, the
 // scaled E) is split into two bf16 terms hi + lo and its products take two or
 // three MMAs, which keeps about 16 significand bits.  T comes from a blocked
-// triangular inversion on the CUDA cores.  The state S is fp32 in registers.
+// triangular inversion on the CUDA cores.  The fp32 state master lives in TMEM.
 #include <cuda.h>
 
 #include <mutex>
@@ -116,6 +117,15 @@ struct Params {
   int L;
   unsigned* status;
 };
+
+// Position of coordinate i within a row of the fp32 gain scratch. Within each 64-wide block the
+// 4-float quads are permuted, (i % 64) = 8 p + 4 h + e  ->  32 h + 4 (p ^ 4 h) + e, so that a warp
+// writing 32 consecutive coordinates, and eight lanes reading the quads h of chunks p = 0..7, each
+// touch 32 distinct banks.
+__device__ __forceinline__ int gf_pos(int i) {
+  const int h = (i >> 2) & 1;
+  return (i & ~63) | (h << 5) | ((((i >> 3) & 7) ^ (h << 2)) << 2) | (i & 3);
+}
 
 template <int D, int VAR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -312,8 +322,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- diagonal variances
     if (VAR == kDiag && tid < D) {
       // Per coordinate i (independent of v and S): p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k).
-      // Eight tokens of keys and scalars are read ahead of the serial chain.
+      // The step is a linear-fractional map of p, so it runs on the homogeneous pair p = x / y:
+      //   x^- = a^2 x + Qn y,  x <- r x^-,  y <- r y + k^2 x^-,
+      // which keeps the division out of the serial chain (three multiply-adds per token); pk = x^- k / y
+      // hangs off it. Every four tokens the pair is rescaled by a power of two, so y stays in [1, 2).
       const uint8_t* Kp = KQ + (tid / 64) * Lay::KQ_PANEL;
+      const int gpos = gf_pos(tid);
+      float x = pcur, y = 1.f;
 #pragma unroll 1
       for (int t8 = 0; t8 < kC; t8 += 8) {
         float kk[8], aa[8], rr8[8], qq[8];
@@ -324,27 +339,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float pp = fmaf(aa[u] * aa[u], pcur, qq[u]);
-          const float pk = pp * kk[u];
-          Gf[(t8 + u) * D + tid] = pk;
-          pcur = __fdividef(pp * rr8[u], fmaf(pk, kk[u], rr8[u]));
+          const float xm = fmaf(aa[u] * aa[u], x, qq[u] * y);
+          Gf[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
+          x = rr8[u] * xm;
+          y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
+          if (u % 4 == 3) {
+            const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
+            const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
+            x *= sc, y *= sc;
+          }
         }
       }
+      pcur = __fdividef(x, y);
     }
     __syncthreads();
 
     // ---------------------------------------------------------------- gains: norms, hi/lo panels (8 threads per token)
     {
+      // Thread `part` of token t takes the 16-byte chunk `part` of every 64-wide panel: coordinates
+      // 64 pn + 8 part .. + 7, so each group of eight lanes reads and writes one whole 128-byte row.
       const int t = tid >> 3, part = tid & 7;
-      const int i0 = part * GD;  // first coordinate of this thread
       float kv[GD];
 #pragma unroll
-      for (int u = 0; u < GD / 8; ++u) {
+      for (int pn = 0; pn < NP; ++pn) {
         float x[8];
-        const int i = i0 + 8 * u;
-        load8_bf16(KQ + (i / 64) * Lay::KQ_PANEL, sm100::sw128_chunk(t, (i % 64) / 8), x);
+        load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kv[8 * u + e] = x[e];
+        for (int e = 0; e < 8; ++e) kv[8 * pn + e] = x[e];
       }
       if (VAR == kDelta) {
         float s = 0.f;
@@ -356,10 +377,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float g[GD];
         if (VAR == kDiag) {
 #pragma unroll
-          for (int e = 0; e < GD; e += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(Gf + t * D + i0 + e);
-            g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
-          }
+          for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 x = *reinterpret_cast<const float4*>(Gf + t * D + gf_pos(64 * pn + 8 * part + 4 * h));
+              g[8 * pn + 4 * h] = x.x, g[8 * pn + 4 * h + 1] = x.y, g[8 * pn + 4 * h + 2] = x.z, g[8 * pn + 4 * h + 3] = x.w;
+            }
           float s = 0.f;
 #pragma unroll
           for (int e = 0; e < GD; ++e) s = fmaf(g[e], kv[e], s);
@@ -370,12 +393,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < GD; ++e) g[e] *= inv_s;
         } else {
           const bool valid = t0 + t < L;
+          const float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + 8 * part;
 #pragma unroll
-          for (int e = 0; e < GD; e += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (valid) x = *reinterpret_cast<const float4*>(P.gains + ((size_t)bh * L + t0 + t) * D + i0 + e);
-            g[e] = x.x, g[e + 1] = x.y, g[e + 2] = x.z, g[e + 3] = x.w;
-          }
+          for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (valid) x = *reinterpret_cast<const float4*>(gp + 64 * pn + 4 * h);
+              g[8 * pn + 4 * h] = x.x, g[8 * pn + 4 * h + 1] = x.y, g[8 * pn + 4 * h + 2] = x.z, g[8 * pn + 4 * h + 3] = x.w;
+            }
         }
         float n2 = 0.f;
 #pragma unroll
@@ -383,12 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         n2 = oct_sum(n2);
         if (part == 0) gn[t] = n2;
 #pragma unroll
-        for (int u = 0; u < GD / 8; ++u) {
-          const int i = i0 + 8 * u;
+        for (int pn = 0; pn < NP; ++pn) {
           float x[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = g[8 * u + e];
-          store8_split(Ghi, Glo, (i / 64) * Lay::G_PANEL + sm100::sw128_chunk(t, (i % 64) / 8), x);
+          for (int e = 0; e < 8; ++e) x[e] = g[8 * pn + e];
+          store8_split(Ghi, Glo, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), x);
         }
       }
     }
@@ -720,9 +745,10 @@ bool chunk_supported(kdn_variant variant, const kdn_dims& d) {
          d.L > 0 && encode_fn() != nullptr;
 }
 
-void chunk_plan(kdn_variant variant, const kdn_dims&, int* launches, const char** kernel, const char** arith) {
+void chunk_plan(kdn_variant variant, const kdn_dims& d, int* launches, const char** kernel, const char** arith) {
   *launches = variant == KDN_KALMAN_FULL ? 2 : 1;
-  *kernel = variant == KDN_KALMAN_FULL ? "kalman_pside_kernel" : "chunk_scan_kernel";
+  *kernel = variant == KDN_KALMAN_FULL ? "kalman_pside_kernel"
+                                       : (d.dk == 128 ? "chunk_scan_ws_kernel" : "chunk_scan_kernel");
   *arith = "bf16-tc";
 }
 
@@ -740,17 +766,16 @@ cudaError_t launch_chunk(kdn_variant variant, const kdn_dims& d, const ChunkArgs
     float* gains = reinterpret_cast<float*>(a.workspace);
     cudaError_t e = launch_kalman_pside(d.dk, a.k, a.a, a.r, a.qn, a.qn_scalar, a.P, gains, a.status, BH, a.L, stream);
     if (e != cudaSuccess) return e;
+    if (d.dk == 128) return launch_chunk_ws(variant, d, a, gains, stream);
     p.gains = gains;
-    return d.dk == 64 ? launch_typed<64, kFull>(tq, tk, tv, p, BH, stream)
-                      : launch_typed<128, kFull>(tq, tk, tv, p, BH, stream);
+    return launch_typed<64, kFull>(tq, tk, tv, p, BH, stream);
   }
+  if (d.dk == 128) return launch_chunk_ws(variant, d, a, nullptr, stream);
   if (variant == KDN_KALMAN_DIAG) {
     p.p = a.P;
-    return d.dk == 64 ? launch_typed<64, kDiag>(tq, tk, tv, p, BH, stream)
-                      : launch_typed<128, kDiag>(tq, tk, tv, p, BH, stream);
+    return launch_typed<64, kDiag>(tq, tk, tv, p, BH, stream);
   }
-  return d.dk == 64 ? launch_typed<64, kDelta>(tq, tk, tv, p, BH, stream)
-                    : launch_typed<128, kDelta>(tq, tk, tv, p, BH, stream);
+  return launch_typed<64, kDelta>(tq, tk, tv, p, BH, stream);
 }
 
 }  // namespace kdn

@@ -1,0 +1,815 @@
+// Warp-specialised chunked scan for d_k = d_v = 128 on the sm_100a tensor cores.
+//
+// The chunk algebra is the generalised WY / UT form of the token recurrence
+// S_t = a_t S_{t-1} + g_t e_t^T, e_t = v_t - a_t S_{t-1}^T k_t (A Hippocampus for
+// Linear Attention, section 3.3 Eq. (5) and section 3.5; Kalman Delta Networks,
+// Abstract, for the Kalman gains): with A_i = prod_{m<=i} a_m and Gam_ij = A_i / A_j,
+//
+//   (I + N) E = R,   N = strict_lower((K G^T) o Gam),   R = V - diag(A) K S0,
+//   O = diag(A) Q S0 + AT R,   AT = ((Q G^T) o Gam o lower) T,   T = (I + N)^-1,
+//   S_C = A_C S0 + G^T diag(A_C / A_j) E.
+//
+// Everything that does not involve the state (gates, diagonal variances, gains,
+// N, T, AT) is the "preparation" of a chunk; what does (S0 products, R, E, O,
+// the state update) is its "chain".  The CTA runs two groups of 8 warps at once:
+// the preparation group works on chunk c + 1 while the chain group works on
+// chunk c, so the serial part of each chunk is the chain alone.
+//
+// The chain runs transposed, with the d_v index on the TMEM lanes, so that every
+// state-dependent operand lives in tensor memory and enters the products as the
+// A operand (bf16 hi/lo pairs, 2-3 MMAs per product):
+//
+//   D2^T = S0^T [K; Q]^T         A = S0^T (TMEM)      B = [K; Q] tile    -> (K S0)^T | (Q S0)^T
+//   R^T  = V^T - (K S0)^T diag(A)                      (in place, TMEM)
+//   D3^T = R^T [T; AT]^T         A = R^T (TMEM)       B = [T; AT]         -> E^T | (AT R)^T
+//   S_C^T = A_C S0^T + E'^T G    A = E'^T (TMEM)      B = G (or K)        accumulated onto the fp32 master
+//
+// and the preparation keeps the row-major products [K; Q] G^T and [T; Attn] T.
+// fp32 state master and accumulators in TMEM; K, Q, V enter exactly as bf16.
+#include <cuda.h>
+
+#include "chunk.h"
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace kdn {
+
+namespace {
+
+using chunk::kC;
+using chunk::kWaitCycles;
+using chunk::load8_bf16;
+using chunk::named_sync;
+using chunk::named_sync_or;
+using chunk::oct_sum;
+using chunk::store8_split;
+
+enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
+
+constexpr int D = 128;
+constexpr int NP = D / 64;                 // 64-wide panels across d
+constexpr int kThreads = 512;
+constexpr int kGroup = 256;                // threads per group; group 0 = chain, group 1 = preparation
+constexpr int kBarChain = 1, kBarPrep = 2;  // named barriers of the two groups (0 is __syncthreads)
+constexpr int kGD = D / 8;                 // coordinates per thread in the per-token reductions
+
+template <int VAR>
+struct WsLayout {
+  static constexpr int KQ_PANEL = 128 * 128;             // [K; Q]: 128 rows x 64 bf16
+  static constexpr int KQ_BYTES = NP * KQ_PANEL;
+  static constexpr int NKQ = (VAR == kDelta) ? 3 : 2;    // [K; Q] tiles in flight
+  static constexpr int V_PANEL = 64 * 128;
+  static constexpr int V_BYTES = NP * V_PANEL;
+  static constexpr int G_PANEL = 64 * 128;
+  static constexpr int G_HALF = (VAR == kDelta) ? 0 : NP * G_PANEL;  // hi or lo of one gain slot
+  static constexpr int TAT_HALF = 128 * 128;             // [T; AT]: 128 rows x 64 bf16, hi or lo
+  static constexpr int SCR_BYTES = 64 * chunk::kLD * 4;  // fp32 [64][68]
+
+  static constexpr int OFF_KQ = 0;
+  static constexpr int OFF_V = OFF_KQ + NKQ * KQ_BYTES;
+  static constexpr int OFF_G = OFF_V + V_BYTES;          // slot s: hi at 2 s G_HALF, lo at (2 s + 1) G_HALF
+  static constexpr int OFF_TAT = OFF_G + 4 * G_HALF;     // hi, then lo
+  static constexpr int OFF_NF = OFF_TAT + 2 * TAT_HALF;
+  static constexpr int OFF_TF = OFF_NF + SCR_BYTES;
+  static constexpr int OFF_GF = OFF_NF;                  // fp32 [64][D] gain scratch, dead before N is built
+  static constexpr int TOTAL = OFF_TF + SCR_BYTES;
+  static constexpr int SMEM = TOTAL + 1024;              // + alignment slack
+  static_assert(64 * D * 4 <= 2 * SCR_BYTES, "gain scratch");
+  static_assert(TOTAL <= 216 * 1024, "shared memory budget");
+
+  // TMEM columns
+  static constexpr uint32_t T_SM = 0;    // fp32 S^T master: lane j (d_v), column i (d_k)
+  static constexpr uint32_t T_SA = 128;  // S0^T as bf16 pairs: hi 0..63, lo 64..127; later D3^T = E^T | (AT R)^T
+  static constexpr uint32_t T_D2 = 256;  // 0..63: (K S0)^T, then R^T, then E'^T as pairs; 64..127: (Q S0)^T
+  static constexpr uint32_t T_D1 = 384;  // [K; Q] G^T
+  static constexpr uint32_t T_DT = 448;  // [T; Attn] T
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+struct Params {
+  const float* beta;
+  const float* a;
+  const float* r;
+  const float* qn;
+  float qn_scalar;
+  const float* gains;  // full Kalman: [BH, L, D] fp32
+  float* S;
+  float* p;            // diag: [BH, D]
+  void* o;
+  float* m;
+  int out_dtype;
+  int L;
+  unsigned* status;
+};
+
+// Position of coordinate i in a row of the fp32 gain scratch: within each 64-wide block,
+// (i % 64) = 8 p + 4 h + e -> 32 h + 4 (p ^ 4 h) + e, so that 32 consecutive coordinates and the
+// quads h of chunks p = 0..7 each fall on 32 distinct banks.
+__device__ __forceinline__ int gf_pos(int i) {
+  const int h = (i >> 2) & 1;
+  return (i & ~63) | (h << 5) | ((((i >> 3) & 7) ^ (h << 2)) << 2) | (i & 3);
+}
+
+// Token column u of a 16-token block of bf16 pairs (hi or lo): TMEM column offset.
+// Thread half h holds tokens 32 h .. 32 h + 31 as 16 hi pair columns at 32 h and 16 lo at 32 h + 16.
+__device__ __forceinline__ uint32_t tok_pair_col(int ks, bool lo) {
+  return 32u * (ks >> 1) + (lo ? 16u : 0u) + 8u * (ks & 1);
+}
+
+template <int VAR>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_scan_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, Params P) {
+  using Lay = WsLayout<VAR>;
+  constexpr int NKQ = Lay::NKQ;
+  constexpr int LD = chunk::kLD;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Vs = sm + Lay::OFF_V;
+  uint8_t* TAThi = sm + Lay::OFF_TAT;
+  uint8_t* TATlo = TAThi + Lay::TAT_HALF;
+  float* Nf = reinterpret_cast<float*>(sm + Lay::OFF_NF);
+  float* Tf = reinterpret_cast<float*>(sm + Lay::OFF_TF);
+  float* Gf = reinterpret_cast<float*>(sm + Lay::OFF_GF);
+
+  // per-chunk scalars, two slots (chunk c uses slot c & 1)
+  __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];         // a, beta | r, Qn
+  __shared__ float ell[2][kC], gn[2][kC];
+  __shared__ __align__(16) float Aex[2][kC];                // A_t
+  __shared__ __align__(16) float esc[2][kC];                // scale of row t of E in the state update:
+                                                            // A_C / A_t (times beta_t for the delta rule)
+  __shared__ float en[4][kC];                               // ||e_t||^2 partials per lane quarter
+  __shared__ uint64_t kq_full[NKQ], v_full, bar_c, bar_p, tat_free;
+  __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2];
+  __shared__ uint32_t tmem_base;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qw = warp & 3;                   // TMEM lane quarter of this warp
+  const int gw = (warp & 7);                 // warp within its group
+  const int half = gw >> 2;                  // 0 / 1: which half of the columns this thread takes
+  const int row = 32 * qw + lane;            // TMEM lane
+  const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+  const int bh = blockIdx.x;
+  const int L = P.L;
+  const int nchunks = (L + kC - 1) / kC;
+
+  auto issue_kq = [&](int cc) {
+    const int slot = cc % NKQ;
+    uint8_t* dst = sm + Lay::OFF_KQ + slot * Lay::KQ_BYTES;
+    sm100::mbar_arrive_expect_tx(&kq_full[slot], 2 * NP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) {
+      sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL, &tm_k, &kq_full[slot], 64 * pn, cc * kC, bh);
+      sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL + 64 * 128, &tm_q, &kq_full[slot], 64 * pn, cc * kC, bh);
+    }
+  };
+  auto issue_v = [&](int cc) {
+    sm100::mbar_arrive_expect_tx(&v_full, NP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) sm100::tma_load_3d(Vs + pn * Lay::V_PANEL, &tm_v, &v_full, 64 * pn, cc * kC, bh);
+  };
+
+  if (tid == 0) {
+    sm100::prefetch_tmap(&tm_q);
+    sm100::prefetch_tmap(&tm_k);
+    sm100::prefetch_tmap(&tm_v);
+#pragma unroll
+    for (int i = 0; i < NKQ; ++i) sm100::mbar_init(&kq_full[i], 1);
+    sm100::mbar_init(&v_full, 1);
+    sm100::mbar_init(&bar_c, 1);
+    sm100::mbar_init(&bar_p, 1);
+    sm100::mbar_init(&tat_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&gates_ready[i], 1);
+      sm100::mbar_init(&prep_done[i], 1);
+      sm100::mbar_init(&chain_done[i], 1);
+    }
+    sm100::fence_mbar_init();
+    for (int cc = 0; cc < NKQ && cc < nchunks; ++cc) issue_kq(cc);
+    issue_v(0);
+  }
+  if (warp == 0) {
+    sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (tid < kGroup) {
+    // =============================================================================== chain group
+    const int j = row;                       // d_v index
+    const bool leader = tid == 0;            // issues the chain's products and every TMA load
+    bool aborted = false;
+    uint32_t ph_c = 0;
+    auto gwait = [&](uint64_t* b, uint32_t parity) -> bool {
+      bool bad = false;
+      if (leader) bad = !sm100::mbar_wait_bounded(b, parity, kWaitCycles);
+      bad = named_sync_or(kBarChain, kGroup, bad);
+      if (bad && leader) raise_status(P.status, kStatusTimeout);
+      sm100::tc_fence_after();
+      return !bad;
+    };
+    // S0^T pairs for the next [K; Q] product and the master pre-scaled by the next chunk's A_C:
+    // x = S[64 half + 32 v .. + 31][j]
+    auto emit_state = [&](float (&x)[32], int v, float scale) {
+      float hw[16], lw[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        uint32_t hu, lu;
+        sm100::split2_bf16(x[2 * e], x[2 * e + 1], hu, lu);
+        hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
+      }
+      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 32 * half + 16 * v, hw);
+      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 64 + 32 * half + 16 * v, lw);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= scale;
+      sm100::tmem_st32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
+    };
+
+    float* Sg = P.S + (size_t)bh * D * D;
+    if (!gwait(&gates_ready[0], 0)) {
+      aborted = true;
+    } else {
+      const float AC0 = Aex[0][kC - 1];
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        float x[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) x[u] = Sg[(size_t)(64 * half + 32 * v + u) * D + j];
+        emit_state(x, v, AC0);
+      }
+      sm100::tmem_wait_st();
+    }
+    sm100::tc_fence_before();
+    named_sync(kBarChain, kGroup);
+    sm100::tc_fence_after();
+
+    const uint32_t tat_hi = sm100::smem_u32(TAThi), tat_lo = sm100::smem_u32(TATlo);
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+      const int s = c & 1, kslot = c % NKQ;
+      const int t0 = c * kC;
+      const uint32_t kq0 = sm100::smem_u32(sm + Lay::OFF_KQ + kslot * Lay::KQ_BYTES);
+
+      // ---------------------------------------------------------------- D2^T = S0^T [K; Q]^T
+      if (!gwait(&kq_full[kslot], (c / NKQ) & 1)) { aborted = true; break; }
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t b = sm100::smem_desc(kq0 + (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32, 16, 1024);
+          sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 8 * ks, b, id, ks > 0);
+          sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 64 + 8 * ks, b, id, true);
+        }
+        sm100::mma_commit(&bar_c);
+      }
+
+      // ---------------------------------------------------------------- R^T = V^T - (K S0)^T diag(A), in place
+      {
+        bool bad = false;
+        if (leader) {
+          bad = !sm100::mbar_wait_bounded(&bar_c, ph_c, kWaitCycles) ||
+                !sm100::mbar_wait_bounded(&v_full, c & 1, kWaitCycles) ||
+                !sm100::mbar_wait_bounded(&gates_ready[s], (c >> 1) & 1, kWaitCycles);
+        }
+        bad = named_sync_or(kBarChain, kGroup, bad);
+        if (bad) {
+          if (leader) raise_status(P.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
+        sm100::tc_fence_after();
+        ph_c ^= 1;
+      }
+      {
+        float X[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + 32 * half, X);
+        sm100::tmem_wait_ld();
+        const uint8_t* vp = Vs + (j / 64) * Lay::V_PANEL;
+        const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
+        float hw[16], lw[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 av = A4[e4];
+          const float aa[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int e = 2 * e4 + e2;
+            const int t = 32 * half + 2 * e;
+            const float v0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vp + sm100::sw128(t, j % 64)));
+            const float v1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vp + sm100::sw128(t + 1, j % 64)));
+            uint32_t hu, lu;
+            sm100::split2_bf16(fmaf(-aa[2 * e2], X[2 * e], v0), fmaf(-aa[2 * e2 + 1], X[2 * e + 1], v1), hu, lu);
+            hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
+          }
+        }
+        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);
+        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half + 16, lw);
+        sm100::tmem_wait_st();
+      }
+      sm100::tc_fence_before();
+      named_sync(kBarChain, kGroup);
+      sm100::tc_fence_after();
+      if (leader && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
+
+      // ---------------------------------------------------------------- D3^T = R^T [T; AT]^T
+      if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bh_ = sm100::smem_desc(tat_hi + ks * 32, 16, 1024);
+          const uint64_t bl = sm100::smem_desc(tat_lo + ks * 32, 16, 1024);
+          const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks, false);
+          const uint32_t al = tmem + Lay::T_D2 + tok_pair_col(ks, true);
+          sm100::mma_bf16_ts(tmem + Lay::T_SA, ah, bh_, id, ks > 0);
+          sm100::mma_bf16_ts(tmem + Lay::T_SA, al, bh_, id, true);
+          sm100::mma_bf16_ts(tmem + Lay::T_SA, ah, bl, id, true);
+        }
+        sm100::mma_commit(&bar_c);
+        sm100::mma_commit(&tat_free);
+      }
+      if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
+      ph_c ^= 1;
+
+      // ---------------------------------------------------------------- E' pairs, ||e||^2, O
+      {
+        float E[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_SA + 32 * half, E);
+        sm100::tmem_wait_ld();
+        const float4* S4 = reinterpret_cast<const float4*>(&esc[s][32 * half]);
+        float hw[16], lw[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 sv = S4[e4];
+          uint32_t hu, lu;
+          sm100::split2_bf16(E[4 * e4] * sv.x, E[4 * e4 + 1] * sv.y, hu, lu);
+          hw[2 * e4] = __uint_as_float(hu), lw[2 * e4] = __uint_as_float(lu);
+          sm100::split2_bf16(E[4 * e4 + 2] * sv.z, E[4 * e4 + 3] * sv.w, hu, lu);
+          hw[2 * e4 + 1] = __uint_as_float(hu), lw[2 * e4 + 1] = __uint_as_float(lu);
+        }
+        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);
+        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half + 16, lw);
+        // sum of E^2 over this warp's 32 lanes for each of the 32 tokens: after the butterfly,
+        // lane l holds token 32 half + l
+#pragma unroll
+        for (int u = 0; u < 32; ++u) E[u] *= E[u];
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1) {
+          const bool up = (lane & k) != 0;
+#pragma unroll
+          for (int i = 0; i < k; ++i) {
+            const float send = up ? E[i] : E[i + k];
+            const float keep = up ? E[i + k] : E[i];
+            E[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+          }
+        }
+        en[qw][32 * half + lane] = E[0];
+      }
+      sm100::tmem_wait_st();
+      sm100::tc_fence_before();
+      named_sync(kBarChain, kGroup);
+      sm100::tc_fence_after();
+
+      // ---------------------------------------------------------------- S^T master += E'^T G
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks, false);
+          const uint32_t al = tmem + Lay::T_D2 + tok_pair_col(ks, true);
+          if (VAR == kDelta) {
+            const uint64_t bk = sm100::smem_desc(kq0 + ks * 2048, Lay::KQ_PANEL, 1024);
+            sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bk, id, true);
+            sm100::mma_bf16_ts(tmem + Lay::T_SM, al, bk, id, true);
+          } else {
+            const uint32_t g0 = sm100::smem_u32(sm + Lay::OFF_G + 2 * s * Lay::G_HALF);
+            const uint64_t bgh = sm100::smem_desc(g0 + ks * 2048, Lay::G_PANEL, 1024);
+            const uint64_t bgl = sm100::smem_desc(g0 + Lay::G_HALF + ks * 2048, Lay::G_PANEL, 1024);
+            sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bgh, id, true);
+            sm100::mma_bf16_ts(tmem + Lay::T_SM, al, bgh, id, true);
+            sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bgl, id, true);
+          }
+        }
+        sm100::mma_commit(&bar_c);
+      }
+      // O = diag(A) Q S0 + AT R, while the state product runs (it touches neither column range)
+      {
+        const bool full = t0 + kC <= L;
+        const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
+        const size_t base = ((size_t)bh * L + t0 + 32 * half) * D + j;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float Y[16], Oi[16];
+          sm100::tmem_ld16(tmem + t_lane + Lay::T_D2 + 64 + 32 * half + 16 * hh, Y);
+          sm100::tmem_ld16(tmem + t_lane + Lay::T_SA + 64 + 32 * half + 16 * hh, Oi);
+          sm100::tmem_wait_ld();
+          float ov[16];
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const float4 av = A4[4 * hh + u4];
+            ov[4 * u4] = fmaf(av.x, Y[4 * u4], Oi[4 * u4]);
+            ov[4 * u4 + 1] = fmaf(av.y, Y[4 * u4 + 1], Oi[4 * u4 + 1]);
+            ov[4 * u4 + 2] = fmaf(av.z, Y[4 * u4 + 2], Oi[4 * u4 + 2]);
+            ov[4 * u4 + 3] = fmaf(av.w, Y[4 * u4 + 3], Oi[4 * u4 + 3]);
+          }
+          if (P.out_dtype == kF32) {
+            float* op = reinterpret_cast<float*>(P.o) + base + (size_t)(16 * hh) * D;
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * D] = ov[u];
+          } else {
+            __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(P.o) + base + (size_t)(16 * hh) * D;
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * D] = __float2bfloat16_rn(ov[u]);
+          }
+        }
+      }
+      if (tid < kC && P.m != nullptr && t0 + tid < L)
+        P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[s][tid]) * sqrtf(en[0][tid] + en[1][tid] + en[2][tid] + en[3][tid]);
+      if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
+      ph_c ^= 1;
+
+      // ---------------------------------------------------------------- state operands of the next chunk
+      if (c + 1 < nchunks) {
+        if (!gwait(&gates_ready[s ^ 1], ((c + 1) >> 1) & 1)) { aborted = true; break; }
+        const float ACn = Aex[s ^ 1][kC - 1];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          float x[32];
+          sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
+          sm100::tmem_wait_ld();
+          emit_state(x, v, ACn);
+        }
+        sm100::tmem_wait_st();
+      }
+      sm100::tc_fence_before();
+      named_sync(kBarChain, kGroup);
+      sm100::tc_fence_after();
+      if (leader) {
+        sm100::mbar_arrive(&chain_done[s]);
+        if (c + NKQ < nchunks) issue_kq(c + NKQ);  // this slot's K, Q are dead
+      }
+    }
+    if (!aborted) {
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        float x[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
+        sm100::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) Sg[(size_t)(64 * half + 32 * v + u) * D + j] = x[u];
+      }
+    }
+  } else {
+    // =============================================================================== preparation group
+    const int pt = tid - kGroup;
+    const bool leader = pt == 0;             // issues the preparation's products
+    bool aborted = false;
+    uint32_t ph_p = 0;
+    float ra = 1.f, rb = 0.f, rq = 0.f;
+    auto fetch_scalars = [&](int cc) {
+      if (pt < kC) {
+        const int tok = cc * kC + pt;
+        const bool valid = tok < L;
+        const size_t ti = (size_t)bh * L + tok;
+        ra = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;
+        if (VAR == kDelta) rb = valid ? P.beta[ti] : 0.f;
+        else rb = valid ? P.r[ti] : 1.f;
+        rq = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;
+      }
+    };
+    float pcur = 1.f;
+    if (VAR == kDiag && pt < D) pcur = P.p[(size_t)bh * D + pt];
+    fetch_scalars(0);
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1, kslot = c % NKQ;
+      const int t0 = c * kC;
+      uint8_t* KQ = sm + Lay::OFF_KQ + kslot * Lay::KQ_BYTES;
+      const uint32_t kq0 = sm100::smem_u32(KQ);
+      uint8_t* Ghi = sm + Lay::OFF_G + 2 * s * Lay::G_HALF;
+      uint8_t* Glo = Ghi + Lay::G_HALF;
+
+      // ---------------------------------------------------------------- slot s free (chain of c - 2), K, Q of c
+      {
+        bool bad = false;
+        if (leader) {
+          if (c >= 2) bad = !sm100::mbar_wait_bounded(&chain_done[s], ((c - 2) >> 1) & 1, kWaitCycles);
+          if (!bad) bad = !sm100::mbar_wait_bounded(&kq_full[kslot], (c / NKQ) & 1, kWaitCycles);
+        }
+        bad = named_sync_or(kBarPrep, kGroup, bad);
+        if (bad) {
+          if (leader) raise_status(P.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
+      }
+      if (pt < kC) sA[s][pt] = ra, sB[s][pt] = rb, sQ[s][pt] = rq;
+      if (c + 1 < nchunks) fetch_scalars(c + 1);
+      named_sync(kBarPrep, kGroup);
+
+      // ---------------------------------------------------------------- gates | diagonal variances
+      if (gw == 4) {
+        // inclusive prefix sums of log a over the chunk (a gate of 0 enters as exp(-60))
+        float x0 = sA[s][lane], x1 = sA[s][32 + lane];
+        x0 = x0 > 0.f ? fmaxf(__logf(x0), -60.f) : -60.f;
+        x1 = x1 > 0.f ? fmaxf(__logf(x1), -60.f) : -60.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+          if (lane >= o) x0 += y0, x1 += y1;
+        }
+        x1 += __shfl_sync(0xffffffffu, x0, 31);
+        const float lC = __shfl_sync(0xffffffffu, x1, 31);
+        ell[s][lane] = x0, ell[s][32 + lane] = x1;
+        Aex[s][lane] = __expf(x0), Aex[s][32 + lane] = __expf(x1);
+        // A_C / A_i without a division
+        const float r0 = __expf(lC - x0), r1 = __expf(lC - x1);
+        esc[s][lane] = VAR == kDelta ? r0 * sB[s][lane] : r0;
+        esc[s][32 + lane] = VAR == kDelta ? r1 * sB[s][32 + lane] : r1;
+      }
+      if (VAR == kDiag && pt < D) {
+        // Per coordinate i: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the homogeneous
+        // pair p = x / y (x^- = a^2 x + Qn y, x <- r x^-, y <- r y + k^2 x^-): three multiply-adds of
+        // serial chain per token, the division that recovers p^- off the chain, and a power-of-two
+        // rescale every four tokens that keeps y in [1, 2).
+        const uint8_t* Kp = KQ + (pt / 64) * Lay::KQ_PANEL;
+        const int gpos = gf_pos(pt);
+        float x = pcur, y = 1.f;
+#pragma unroll 1
+        for (int t8 = 0; t8 < kC; t8 += 8) {
+          float kk[8], aa[8], rr8[8], qq[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, pt % 64)));
+            aa[u] = sA[s][t8 + u], rr8[u] = sB[s][t8 + u], qq[u] = sQ[s][t8 + u];
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float xm = fmaf(aa[u] * aa[u], x, qq[u] * y);
+            Gf[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
+            x = rr8[u] * xm;
+            y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
+            if (u % 4 == 3) {
+              const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
+              const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
+              x *= sc, y *= sc;
+            }
+          }
+        }
+        pcur = __fdividef(x, y);
+      }
+      named_sync(kBarPrep, kGroup);
+      if (leader) sm100::mbar_arrive(&gates_ready[s]);
+
+      // ---------------------------------------------------------------- gains: norms, hi/lo panels (8 threads per token)
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        // Thread `part` of token t takes the 16-byte chunk `part` of every 64-wide panel: coordinates
+        // 64 pn + 8 part .. + 7, so each group of eight lanes reads and writes one whole 128-byte row.
+        const int t = 32 * pass + (pt >> 3), part = pt & 7;
+        float kv[kGD];
+#pragma unroll
+        for (int pn = 0; pn < NP; ++pn) {
+          float xk[8];
+          load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[8 * pn + e] = xk[e];
+        }
+        if (VAR == kDelta) {
+          float sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < kGD; ++e) sq = fmaf(kv[e], kv[e], sq);
+          sq = oct_sum(sq);
+          if (part == 0) gn[s][t] = sB[s][t] * sB[s][t] * sq;
+        } else {
+          float g[kGD];
+          if (VAR == kDiag) {
+#pragma unroll
+            for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+              for (int hq = 0; hq < 2; ++hq) {
+                const float4 x4 = *reinterpret_cast<const float4*>(Gf + t * D + gf_pos(64 * pn + 8 * part + 4 * hq));
+                g[8 * pn + 4 * hq] = x4.x, g[8 * pn + 4 * hq + 1] = x4.y;
+                g[8 * pn + 4 * hq + 2] = x4.z, g[8 * pn + 4 * hq + 3] = x4.w;
+              }
+            float sd = 0.f;
+#pragma unroll
+            for (int e = 0; e < kGD; ++e) sd = fmaf(g[e], kv[e], sd);
+            sd = oct_sum(sd) + sB[s][t];
+            if (part == 0 && !(sd > 0.f && isfinite(sd))) raise_status(P.status, kStatusNumeric);
+            const float inv_s = 1.f / sd;
+#pragma unroll
+            for (int e = 0; e < kGD; ++e) g[e] *= inv_s;
+          } else {
+            const bool valid = t0 + t < L;
+            const float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + 8 * part;
+#pragma unroll
+            for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+              for (int hq = 0; hq < 2; ++hq) {
+                float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (valid) x4 = *reinterpret_cast<const float4*>(gp + 64 * pn + 4 * hq);
+                g[8 * pn + 4 * hq] = x4.x, g[8 * pn + 4 * hq + 1] = x4.y;
+                g[8 * pn + 4 * hq + 2] = x4.z, g[8 * pn + 4 * hq + 3] = x4.w;
+              }
+          }
+          float n2 = 0.f;
+#pragma unroll
+          for (int e = 0; e < kGD; ++e) n2 = fmaf(g[e], g[e], n2);
+          n2 = oct_sum(n2);
+          if (part == 0) gn[s][t] = n2;
+#pragma unroll
+          for (int pn = 0; pn < NP; ++pn) {
+            float xg[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xg[e] = g[8 * pn + e];
+            store8_split(Ghi, Glo, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
+          }
+        }
+      }
+      sm100::fence_async_smem();
+      sm100::tc_fence_before();
+      named_sync(kBarPrep, kGroup);
+      sm100::tc_fence_after();
+
+      // ---------------------------------------------------------------- D1 = [K; Q] G^T
+      if (leader) {
+        constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
+        const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
+          const uint64_t a = sm100::smem_desc(kq0 + koff, 16, 1024);
+          if (VAR == kDelta) {
+            sm100::mma_bf16(tmem + Lay::T_D1, a, a, id1, ks > 0);  // G = K (beta enters with Gam)
+          } else {
+            const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
+            sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + goff, 16, 1024), id1, ks > 0);
+            sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(glo + goff, 16, 1024), id1, true);
+          }
+        }
+        sm100::mma_commit(&bar_p);
+      }
+      {
+        bool bad = false;
+        if (leader) {
+          bad = !sm100::mbar_wait_bounded(&bar_p, ph_p, kWaitCycles);
+          if (!bad && c >= 1) bad = !sm100::mbar_wait_bounded(&tat_free, (c - 1) & 1, kWaitCycles);
+        }
+        bad = named_sync_or(kBarPrep, kGroup, bad);
+        if (bad) {
+          if (leader) raise_status(P.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
+        sm100::tc_fence_after();
+        ph_p ^= 1;
+      }
+
+      // ---------------------------------------------------------------- N (lanes 0..63) | Attn (lanes 64..127)
+      {
+        float Y[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * half, Y);
+        sm100::tmem_wait_ld();
+        if (qw < 2) {
+          const int i = row;
+          const float li = ell[s][i];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float v4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int jj = 32 * half + e + u;
+              v4[u] = (jj < i) ? Y[e + u] * __expf(li - ell[s][jj]) * (VAR == kDelta ? sB[s][jj] : 1.f) : 0.f;
+            }
+            *reinterpret_cast<float4*>(Nf + i * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+          }
+        } else {
+          const int i = row - 64;
+          const float li = ell[s][i];
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float xa[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int jj = 32 * half + 8 * q8 + e;
+              xa[e] = (jj <= i) ? Y[8 * q8 + e] * __expf(li - ell[s][jj]) * (VAR == kDelta ? sB[s][jj] : 1.f) : 0.f;
+            }
+            store8_split(TAThi, TATlo, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
+          }
+        }
+      }
+      named_sync(kBarPrep, kGroup);
+
+      // ---------------------------------------------------------------- T = (I + N)^-1 into rows 0..63 of [T; AT]
+      chunk::invert_unit_lower_64(Nf, Tf, pt, [] { named_sync(kBarPrep, kGroup); });
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int e = pt + 256 * hh;
+        const int i = e >> 3, c8 = e & 7;
+        const float4 lo4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8);
+        const float4 hi4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8 + 4);
+        const float tv[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
+        float xt[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int jj = 8 * c8 + u;
+          xt[u] = (jj < i) ? tv[u] : (jj == i ? 1.f : 0.f);
+        }
+        store8_split(TAThi, TATlo, sm100::sw128_chunk(i, c8), xt);
+      }
+      sm100::fence_async_smem();
+      sm100::tc_fence_before();
+      named_sync(kBarPrep, kGroup);
+      sm100::tc_fence_after();
+
+      // ---------------------------------------------------------------- DT = [T; Attn] T  (rows 64..127: AT)
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, true);
+        const uint32_t thi = sm100::smem_u32(TAThi), tlo = sm100::smem_u32(TATlo);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ah = sm100::smem_desc(thi + ks * 32, 16, 1024), al = sm100::smem_desc(tlo + ks * 32, 16, 1024);
+          const uint64_t bh_ = sm100::smem_desc(thi + ks * 2048, 16, 1024), bl = sm100::smem_desc(tlo + ks * 2048, 16, 1024);
+          sm100::mma_bf16(tmem + Lay::T_DT, ah, bh_, id, ks > 0);
+          sm100::mma_bf16(tmem + Lay::T_DT, al, bh_, id, true);
+          sm100::mma_bf16(tmem + Lay::T_DT, ah, bl, id, true);
+        }
+        sm100::mma_commit(&bar_p);
+      }
+      {
+        bool bad = false;
+        if (leader) bad = !sm100::mbar_wait_bounded(&bar_p, ph_p, kWaitCycles);
+        bad = named_sync_or(kBarPrep, kGroup, bad);
+        if (bad) {
+          if (leader) raise_status(P.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
+        sm100::tc_fence_after();
+        ph_p ^= 1;
+      }
+      if (qw >= 2) {
+        const int i = row - 64;
+        float X[32];
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_DT + 32 * half, X);
+        sm100::tmem_wait_ld();
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float xa[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xa[e] = X[8 * q8 + e];
+          store8_split(TAThi, TATlo, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
+        }
+      }
+      sm100::fence_async_smem();
+      sm100::tc_fence_before();
+      named_sync(kBarPrep, kGroup);
+      sm100::tc_fence_after();
+      if (leader) sm100::mbar_arrive(&prep_done[s]);
+    }
+    if (!aborted && VAR == kDiag && pt < D) P.p[(size_t)bh * D + pt] = pcur;
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) sm100::tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+template <int VAR>
+cudaError_t launch_ws_typed(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const Params& p, int BH,
+                            cudaStream_t stream) {
+  using Lay = WsLayout<VAR>;
+  cudaError_t e = cudaFuncSetAttribute(chunk_scan_ws_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+  if (e != cudaSuccess) return e;
+  chunk_scan_ws_kernel<VAR><<<BH, kThreads, Lay::SMEM, stream>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& d, const ChunkArgs& a, const float* gains,
+                            cudaStream_t stream) {
+  if (d.dk != D || d.dv != D) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_bf16_tmap(&tq, a.q, a.BH, a.L, D) || !make_bf16_tmap(&tk, a.k, a.BH, a.L, D) ||
+      !make_bf16_tmap(&tv, a.v, a.BH, a.L, D))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.beta = a.beta, p.a = a.a, p.r = a.r, p.qn = a.qn, p.qn_scalar = a.qn_scalar, p.gains = gains;
+  p.S = a.S, p.o = a.o, p.m = a.m, p.out_dtype = a.out_dtype, p.L = a.L, p.status = a.status;
+  if (variant == KDN_KALMAN_FULL) return launch_ws_typed<kFull>(tq, tk, tv, p, a.BH, stream);
+  if (variant == KDN_KALMAN_DIAG) {
+    p.p = a.P;
+    return launch_ws_typed<kDiag>(tq, tk, tv, p, a.BH, stream);
+  }
+  return launch_ws_typed<kDelta>(tq, tk, tv, p, a.BH, stream);
+}
+
+}  // namespace kdn
