@@ -72,10 +72,9 @@ struct WsLayout {
   static constexpr int OFF_TAT = OFF_G + 4 * G_HALF;     // hi, then lo
   static constexpr int OFF_NF = OFF_TAT + 2 * TAT_HALF;
   static constexpr int OFF_TF = OFF_NF + SCR_BYTES;
-  static constexpr int OFF_GF = OFF_NF;                  // fp32 [64][D] gain scratch, dead before N is built
   static constexpr int TOTAL = OFF_TF + SCR_BYTES;
   static constexpr int SMEM = TOTAL + 1024;              // + alignment slack
-  static_assert(64 * D * 4 <= 2 * SCR_BYTES, "gain scratch");
+  static_assert(VAR == kDelta || 64 * D * 4 == 2 * G_HALF, "a gain slot holds the fp32 gains before their split");
   static_assert(TOTAL <= 216 * 1024, "shared memory budget");
 
   // TMEM columns
@@ -123,6 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_v, Params P) {
   using Lay = WsLayout<VAR>;
   constexpr int NKQ = Lay::NKQ;
+  // The diagonal variant's chain runs the gates and variances of chunk c + 1 while it waits for the
+  // preparation of chunk c; the other variants' preparation runs its own gates.
+  constexpr bool kChainGates = VAR == kDiag;
   constexpr int LD = chunk::kLD;
 
   extern __shared__ uint8_t smem_raw[];
@@ -132,7 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* TATlo = TAThi + Lay::TAT_HALF;
   float* Nf = reinterpret_cast<float*>(sm + Lay::OFF_NF);
   float* Tf = reinterpret_cast<float*>(sm + Lay::OFF_TF);
-  float* Gf = reinterpret_cast<float*>(sm + Lay::OFF_GF);
 
   // per-chunk scalars, two slots (chunk c uses slot c & 1)
   __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];         // a, beta | r, Qn
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                             // A_C / A_t (times beta_t for the delta rule)
   __shared__ float en[4][kC];                               // ||e_t||^2 partials per lane quarter
   __shared__ uint64_t kq_full[NKQ], v_full, bar_c, bar_p, tat_free;
-  __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2];
+  __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2], var_done[2];
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -183,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::mbar_init(&tat_free, 1);
     for (int i = 0; i < 2; ++i) {
       sm100::mbar_init(&gates_ready[i], 1);
+      sm100::mbar_init(&var_done[i], 1);
       sm100::mbar_init(&prep_done[i], 1);
       sm100::mbar_init(&chain_done[i], 1);
     }
@@ -194,6 +196,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
     sm100::tmem_relinquish();
   }
+  // raw per-token scalars of chunk cc into registers (threads 0..63 of the preparation group); chunk 0's
+  // go to slot 0 before the groups part, chunk c + 1's are stored by the preparation of chunk c
+  float ra = 1.f, rb = 0.f, rq = 0.f;
+  auto fetch_scalars = [&](int cc) {
+    const int u = tid - kGroup;
+    if (u >= 0 && u < kC) {
+      const int tok = cc * kC + u;
+      const bool valid = tok < L;
+      const size_t ti = (size_t)bh * L + tok;
+      ra = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;
+      if (VAR == kDelta) rb = valid ? P.beta[ti] : 0.f;
+      else rb = valid ? P.r[ti] : 1.f;
+      rq = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;
+    }
+  };
+  auto store_scalars = [&](int slot) {
+    const int u = tid - kGroup;
+    if (u >= 0 && u < kC) sA[slot][u] = ra, sB[slot][u] = rb, sQ[slot][u] = rq;
+  };
+  // gates of chunk cc into its slot, by one warp: inclusive prefix sums of log a over the chunk (a gate of 0
+  // enters as exp(-60)), A_t, and the state-update row scale A_C / A_t (times beta_t for the delta rule)
+  auto run_gates = [&](int cc) {
+    const int sl = cc & 1;
+    float x0 = sA[sl][lane], x1 = sA[sl][32 + lane];
+    x0 = x0 > 0.f ? fmaxf(__logf(x0), -60.f) : -60.f;
+    x1 = x1 > 0.f ? fmaxf(__logf(x1), -60.f) : -60.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+      if (lane >= o) x0 += y0, x1 += y1;
+    }
+    x1 += __shfl_sync(0xffffffffu, x0, 31);
+    const float lC = __shfl_sync(0xffffffffu, x1, 31);
+    ell[sl][lane] = x0, ell[sl][32 + lane] = x1;
+    Aex[sl][lane] = __expf(x0), Aex[sl][32 + lane] = __expf(x1);
+    const float r0 = __expf(lC - x0), r1 = __expf(lC - x1);  // A_C / A_t without a division
+    esc[sl][lane] = VAR == kDelta ? r0 * sB[sl][lane] : r0;
+    esc[sl][32 + lane] = VAR == kDelta ? r1 * sB[sl][32 + lane] : r1;
+  };
+  fetch_scalars(0);
+  store_scalars(0);
+  if (nchunks > 1) fetch_scalars(1);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -230,8 +274,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::tmem_st32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
     };
 
+    // Diagonal variances of chunk cc (threads 0..D-1, coordinate i = tid; independent of v and S), run one
+    // chunk ahead while the chain waits for the preparation.  Per coordinate: p^- = a^2 p + Qn,
+    // pk = p^- k, p <- p^- r / (r + pk k), on the homogeneous pair p = x / y (x^- = a^2 x + Qn y,
+    // x <- r x^-, y <- r y + k^2 x^-): three multiply-adds of serial chain per token, the division that
+    // recovers p^- off the chain, and a power-of-two rescale every four tokens that keeps y in [1, 2).
+    // The unnormalised gains pk go, fp32, into the gain slot of chunk cc.
+    float pcur = 1.f;
+    if (VAR == kDiag && tid < D) pcur = P.p[(size_t)bh * D + tid];
+    auto run_variances = [&](int cc) {
+      if (VAR == kDiag && tid < D) {
+        const int sl = cc & 1;
+        const uint8_t* Kp = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES + (tid / 64) * Lay::KQ_PANEL;
+        float* Gw = reinterpret_cast<float*>(sm + Lay::OFF_G + 2 * sl * Lay::G_HALF);
+        const int gpos = gf_pos(tid);
+        float x = pcur, y = 1.f;
+#pragma unroll 1
+        for (int t8 = 0; t8 < kC; t8 += 8) {
+          float kk[8], aa[8], rr8[8], qq[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, tid % 64)));
+            aa[u] = sA[sl][t8 + u], rr8[u] = sB[sl][t8 + u], qq[u] = sQ[sl][t8 + u];
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float xm = fmaf(aa[u] * aa[u], x, qq[u] * y);
+            Gw[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
+            x = rr8[u] * xm;
+            y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
+            if (u % 4 == 3) {
+              const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
+              const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
+              x *= sc, y *= sc;
+            }
+          }
+        }
+        pcur = __fdividef(x, y);
+      }
+    };
+
     float* Sg = P.S + (size_t)bh * D * D;
-    if (!gwait(&gates_ready[0], 0)) {
+    if (kChainGates) {  // gates and variances of chunk 0 (its scalars are in slot 0 already)
+      if (!gwait(&kq_full[0], 0)) {
+        aborted = true;
+      } else {
+        run_variances(0);
+        if (gw == 4) run_gates(0);
+        named_sync(kBarChain, kGroup);
+        if (leader) sm100::mbar_arrive(&var_done[0]);
+      }
+    }
+    if (aborted || (!kChainGates && !gwait(&gates_ready[0], 0))) {
       aborted = true;
     } else {
       const float AC0 = Aex[0][kC - 1];
@@ -314,6 +408,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_sync(kBarChain, kGroup);
       sm100::tc_fence_after();
       if (leader && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
+
+      // ---------------------------------------------------------------- variances of chunk c + 1
+      if (kChainGates && c + 1 < nchunks) {
+        // its scalars were stored before gates_ready of chunk c, its K before the slot's load completed
+        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
+        run_variances(c + 1);
+        if (gw == 4) run_gates(c + 1);
+        named_sync(kBarChain, kGroup);
+        if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
+      }
 
       // ---------------------------------------------------------------- D3^T = R^T [T; AT]^T
       if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
@@ -436,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---------------------------------------------------------------- state operands of the next chunk
       if (c + 1 < nchunks) {
-        if (!gwait(&gates_ready[s ^ 1], ((c + 1) >> 1) & 1)) { aborted = true; break; }
+        if (!kChainGates && !gwait(&gates_ready[s ^ 1], ((c + 1) >> 1) & 1)) { aborted = true; break; }
         const float ACn = Aex[s ^ 1][kC - 1];
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
@@ -464,6 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 32; ++u) Sg[(size_t)(64 * half + 32 * v + u) * D + j] = x[u];
       }
+      if (VAR == kDiag && tid < D) P.p[(size_t)bh * D + tid] = pcur;
     }
   } else {
     // =============================================================================== preparation group
@@ -471,21 +576,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = pt == 0;             // issues the preparation's products
     bool aborted = false;
     uint32_t ph_p = 0;
-    float ra = 1.f, rb = 0.f, rq = 0.f;
-    auto fetch_scalars = [&](int cc) {
-      if (pt < kC) {
-        const int tok = cc * kC + pt;
-        const bool valid = tok < L;
-        const size_t ti = (size_t)bh * L + tok;
-        ra = valid ? (P.a ? P.a[ti] : 1.f) : 1.f;
-        if (VAR == kDelta) rb = valid ? P.beta[ti] : 0.f;
-        else rb = valid ? P.r[ti] : 1.f;
-        rq = valid ? (P.qn ? P.qn[ti] : P.qn_scalar) : 0.f;
-      }
-    };
-    float pcur = 1.f;
-    if (VAR == kDiag && pt < D) pcur = P.p[(size_t)bh * D + pt];
-    fetch_scalars(0);
 
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1, kslot = c % NKQ;
@@ -509,127 +599,102 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
       }
-      if (pt < kC) sA[s][pt] = ra, sB[s][pt] = rb, sQ[s][pt] = rq;
-      if (c + 1 < nchunks) fetch_scalars(c + 1);
-      named_sync(kBarPrep, kGroup);
-
       // ---------------------------------------------------------------- gates | diagonal variances
-      if (gw == 4) {
-        // inclusive prefix sums of log a over the chunk (a gate of 0 enters as exp(-60))
-        float x0 = sA[s][lane], x1 = sA[s][32 + lane];
-        x0 = x0 > 0.f ? fmaxf(__logf(x0), -60.f) : -60.f;
-        x1 = x1 > 0.f ? fmaxf(__logf(x1), -60.f) : -60.f;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
-          if (lane >= o) x0 += y0, x1 += y1;
-        }
-        x1 += __shfl_sync(0xffffffffu, x0, 31);
-        const float lC = __shfl_sync(0xffffffffu, x1, 31);
-        ell[s][lane] = x0, ell[s][32 + lane] = x1;
-        Aex[s][lane] = __expf(x0), Aex[s][32 + lane] = __expf(x1);
-        // A_C / A_i without a division
-        const float r0 = __expf(lC - x0), r1 = __expf(lC - x1);
-        esc[s][lane] = VAR == kDelta ? r0 * sB[s][lane] : r0;
-        esc[s][32 + lane] = VAR == kDelta ? r1 * sB[s][32 + lane] : r1;
-      }
-      if (VAR == kDiag && pt < D) {
-        // Per coordinate i: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the homogeneous
-        // pair p = x / y (x^- = a^2 x + Qn y, x <- r x^-, y <- r y + k^2 x^-): three multiply-adds of
-        // serial chain per token, the division that recovers p^- off the chain, and a power-of-two
-        // rescale every four tokens that keeps y in [1, 2).
-        const uint8_t* Kp = KQ + (pt / 64) * Lay::KQ_PANEL;
-        const int gpos = gf_pos(pt);
-        float x = pcur, y = 1.f;
-#pragma unroll 1
-        for (int t8 = 0; t8 < kC; t8 += 8) {
-          float kk[8], aa[8], rr8[8], qq[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, pt % 64)));
-            aa[u] = sA[s][t8 + u], rr8[u] = sB[s][t8 + u], qq[u] = sQ[s][t8 + u];
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float xm = fmaf(aa[u] * aa[u], x, qq[u] * y);
-            Gf[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
-            x = rr8[u] * xm;
-            y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
-            if (u % 4 == 3) {
-              const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
-              const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
-              x *= sc, y *= sc;
-            }
-          }
-        }
-        pcur = __fdividef(x, y);
+      if (!kChainGates && gw == 4) run_gates(c);
+      if (c + 1 < nchunks) {  // raw scalars of the next chunk (its slot was last read by chunk c - 1)
+        store_scalars(s ^ 1);
+        if (c + 2 < nchunks) fetch_scalars(c + 2);
       }
       named_sync(kBarPrep, kGroup);
+      // gates_ready: this chunk's gates (unless the chain runs them) and the next chunk's raw scalars
       if (leader) sm100::mbar_arrive(&gates_ready[s]);
+      if (kChainGates) {  // the chain has run this chunk's gates and written its unnormalised gains into slot s
+        bool bad = false;
+        if (leader) bad = !sm100::mbar_wait_bounded(&var_done[s], (c >> 1) & 1, kWaitCycles);
+        bad = named_sync_or(kBarPrep, kGroup, bad);
+        if (bad) {
+          if (leader) raise_status(P.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
+      }
 
       // ---------------------------------------------------------------- gains: norms, hi/lo panels (8 threads per token)
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
+      {
         // Thread `part` of token t takes the 16-byte chunk `part` of every 64-wide panel: coordinates
         // 64 pn + 8 part .. + 7, so each group of eight lanes reads and writes one whole 128-byte row.
-        const int t = 32 * pass + (pt >> 3), part = pt & 7;
-        float kv[kGD];
+        // The diagonal variant normalises the fp32 gains that share the slot with their hi/lo split: all
+        // of them are read before any split is written.
+        const int part = pt & 7;
+        float g[2][kGD];
 #pragma unroll
-        for (int pn = 0; pn < NP; ++pn) {
-          float xk[8];
-          load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) kv[8 * pn + e] = xk[e];
-        }
-        if (VAR == kDelta) {
-          float sq = 0.f;
-#pragma unroll
-          for (int e = 0; e < kGD; ++e) sq = fmaf(kv[e], kv[e], sq);
-          sq = oct_sum(sq);
-          if (part == 0) gn[s][t] = sB[s][t] * sB[s][t] * sq;
-        } else {
-          float g[kGD];
-          if (VAR == kDiag) {
-#pragma unroll
-            for (int pn = 0; pn < NP; ++pn)
-#pragma unroll
-              for (int hq = 0; hq < 2; ++hq) {
-                const float4 x4 = *reinterpret_cast<const float4*>(Gf + t * D + gf_pos(64 * pn + 8 * part + 4 * hq));
-                g[8 * pn + 4 * hq] = x4.x, g[8 * pn + 4 * hq + 1] = x4.y;
-                g[8 * pn + 4 * hq + 2] = x4.z, g[8 * pn + 4 * hq + 3] = x4.w;
-              }
-            float sd = 0.f;
-#pragma unroll
-            for (int e = 0; e < kGD; ++e) sd = fmaf(g[e], kv[e], sd);
-            sd = oct_sum(sd) + sB[s][t];
-            if (part == 0 && !(sd > 0.f && isfinite(sd))) raise_status(P.status, kStatusNumeric);
-            const float inv_s = 1.f / sd;
-#pragma unroll
-            for (int e = 0; e < kGD; ++e) g[e] *= inv_s;
-          } else {
-            const bool valid = t0 + t < L;
-            const float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + 8 * part;
-#pragma unroll
-            for (int pn = 0; pn < NP; ++pn)
-#pragma unroll
-              for (int hq = 0; hq < 2; ++hq) {
-                float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (valid) x4 = *reinterpret_cast<const float4*>(gp + 64 * pn + 4 * hq);
-                g[8 * pn + 4 * hq] = x4.x, g[8 * pn + 4 * hq + 1] = x4.y;
-                g[8 * pn + 4 * hq + 2] = x4.z, g[8 * pn + 4 * hq + 3] = x4.w;
-              }
-          }
-          float n2 = 0.f;
-#pragma unroll
-          for (int e = 0; e < kGD; ++e) n2 = fmaf(g[e], g[e], n2);
-          n2 = oct_sum(n2);
-          if (part == 0) gn[s][t] = n2;
+        for (int pass = 0; pass < 2; ++pass) {
+          const int t = 32 * pass + (pt >> 3);
+          float kv[kGD];
 #pragma unroll
           for (int pn = 0; pn < NP; ++pn) {
-            float xg[8];
+            float xk[8];
+            load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xg[e] = g[8 * pn + e];
-            store8_split(Ghi, Glo, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
+            for (int e = 0; e < 8; ++e) kv[8 * pn + e] = xk[e];
+          }
+          if (VAR == kDelta) {
+            float sq = 0.f;
+#pragma unroll
+            for (int e = 0; e < kGD; ++e) sq = fmaf(kv[e], kv[e], sq);
+            sq = oct_sum(sq);
+            if (part == 0) gn[s][t] = sB[s][t] * sB[s][t] * sq;
+          } else {
+            if (VAR == kDiag) {
+              const float* Gw = reinterpret_cast<const float*>(Ghi);
+#pragma unroll
+              for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                  const float4 x4 = *reinterpret_cast<const float4*>(Gw + t * D + gf_pos(64 * pn + 8 * part + 4 * hq));
+                  g[pass][8 * pn + 4 * hq] = x4.x, g[pass][8 * pn + 4 * hq + 1] = x4.y;
+                  g[pass][8 * pn + 4 * hq + 2] = x4.z, g[pass][8 * pn + 4 * hq + 3] = x4.w;
+                }
+              float sd = 0.f;
+#pragma unroll
+              for (int e = 0; e < kGD; ++e) sd = fmaf(g[pass][e], kv[e], sd);
+              sd = oct_sum(sd) + sB[s][t];
+              if (part == 0 && !(sd > 0.f && isfinite(sd))) raise_status(P.status, kStatusNumeric);
+              const float inv_s = 1.f / sd;
+#pragma unroll
+              for (int e = 0; e < kGD; ++e) g[pass][e] *= inv_s;
+            } else {
+              const bool valid = t0 + t < L;
+              const float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + 8 * part;
+#pragma unroll
+              for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                  float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                  if (valid) x4 = *reinterpret_cast<const float4*>(gp + 64 * pn + 4 * hq);
+                  g[pass][8 * pn + 4 * hq] = x4.x, g[pass][8 * pn + 4 * hq + 1] = x4.y;
+                  g[pass][8 * pn + 4 * hq + 2] = x4.z, g[pass][8 * pn + 4 * hq + 3] = x4.w;
+                }
+            }
+            float n2 = 0.f;
+#pragma unroll
+            for (int e = 0; e < kGD; ++e) n2 = fmaf(g[pass][e], g[pass][e], n2);
+            n2 = oct_sum(n2);
+            if (part == 0) gn[s][t] = n2;
+          }
+        }
+        if (VAR != kDelta) {
+          if (VAR == kDiag) named_sync(kBarPrep, kGroup);
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {
+            const int t = 32 * pass + (pt >> 3);
+#pragma unroll
+            for (int pn = 0; pn < NP; ++pn) {
+              float xg[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) xg[e] = g[pass][8 * pn + e];
+              store8_split(Ghi, Glo, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
+            }
           }
         }
       }
@@ -774,7 +839,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::tc_fence_after();
       if (leader) sm100::mbar_arrive(&prep_done[s]);
     }
-    if (!aborted && VAR == kDiag && pt < D) P.p[(size_t)bh * D + pt] = pcur;
   }
 
   sm100::tc_fence_before();
