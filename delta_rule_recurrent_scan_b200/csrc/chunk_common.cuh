@@ -140,43 +140,58 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* Nf, float* Tf,
     sync();
   }
   // (3) X = N_{[23],[01]} T_{[01],[01]} parked in rows 0..31, columns 32..63; then the lower-left 32 x 32
-  // block of T = -T_{[23],[23]} X.  Warps take uniform ranges: jh (columns 16 jh ..) and the row octet.
+  // block of T = -T_{[23],[23]} X.  Threads 0..127 each take rows {r, r + 16} x four columns (register
+  // tiles halve the shared-memory reads of the broadcast operand); warps take uniform column ranges.
   {
-    const int jh = gt >> 7, ii = (gt >> 2) & 31, jq = gt & 3;
-    const int j0 = 16 * jh + 4 * jq;
-    {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int u = gt & 127;
+    if (gt < 128) {
+      const int jh = u >> 6, r = (u >> 2) & 15, j0 = 16 * jh + 4 * (u & 3);
+      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int kb = 0; kb < 32; kb += 4) {
         if (kb < 16 * jh) continue;  // T_{[01],[01]}[k][j] = 0 for k < 16 <= j
-        const float4 n4 = *reinterpret_cast<const float4*>(Nf + (32 + ii) * LD + kb);
-        const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+        const float4 na = *reinterpret_cast<const float4*>(Nf + (32 + r) * LD + kb);
+        const float4 nb = *reinterpret_cast<const float4*>(Nf + (48 + r) * LD + kb);
+        const float n0[4] = {na.x, na.y, na.z, na.w}, n1[4] = {nb.x, nb.y, nb.z, nb.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float4 t4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + j0);
-          acc.x = fmaf(nv[e], t4.x, acc.x), acc.y = fmaf(nv[e], t4.y, acc.y);
-          acc.z = fmaf(nv[e], t4.z, acc.z), acc.w = fmaf(nv[e], t4.w, acc.w);
+          acc0.x = fmaf(n0[e], t4.x, acc0.x), acc0.y = fmaf(n0[e], t4.y, acc0.y);
+          acc0.z = fmaf(n0[e], t4.z, acc0.z), acc0.w = fmaf(n0[e], t4.w, acc0.w);
+          acc1.x = fmaf(n1[e], t4.x, acc1.x), acc1.y = fmaf(n1[e], t4.y, acc1.y);
+          acc1.z = fmaf(n1[e], t4.z, acc1.z), acc1.w = fmaf(n1[e], t4.w, acc1.w);
         }
       }
-      *reinterpret_cast<float4*>(Tf + ii * LD + 32 + j0) = acc;
+      *reinterpret_cast<float4*>(Tf + r * LD + 32 + j0) = acc0;
+      *reinterpret_cast<float4*>(Tf + (16 + r) * LD + 32 + j0) = acc1;
     }
     sync();
-    {
-      const int kend = ii < 16 ? 16 : 32;  // T_{[23],[23]}[i][k] = 0 for i < 16 <= k
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (gt < 128) {
+      const int r = u >> 3, j0 = 4 * (u & 7);
+      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int kb = 0; kb < 32; kb += 4) {
-        if (kb >= kend) continue;
-        const float4 t4r = *reinterpret_cast<const float4*>(Tf + (32 + ii) * LD + 32 + kb);
-        const float tv[4] = {t4r.x, t4r.y, t4r.z, t4r.w};
+        // row r of T_{[23],[23]} is zero past column 15; row 16 + r runs to column 31
+        float t0v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (kb < 16) {
+          const float4 ta = *reinterpret_cast<const float4*>(Tf + (32 + r) * LD + 32 + kb);
+          t0v[0] = ta.x, t0v[1] = ta.y, t0v[2] = ta.z, t0v[3] = ta.w;
+        }
+        const float4 tb = *reinterpret_cast<const float4*>(Tf + (48 + r) * LD + 32 + kb);
+        const float t1v[4] = {tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float4 x4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + 32 + j0);
-          acc.x = fmaf(tv[e], x4.x, acc.x), acc.y = fmaf(tv[e], x4.y, acc.y);
-          acc.z = fmaf(tv[e], x4.z, acc.z), acc.w = fmaf(tv[e], x4.w, acc.w);
+          if (kb < 16) {
+            acc0.x = fmaf(t0v[e], x4.x, acc0.x), acc0.y = fmaf(t0v[e], x4.y, acc0.y);
+            acc0.z = fmaf(t0v[e], x4.z, acc0.z), acc0.w = fmaf(t0v[e], x4.w, acc0.w);
+          }
+          acc1.x = fmaf(t1v[e], x4.x, acc1.x), acc1.y = fmaf(t1v[e], x4.y, acc1.y);
+          acc1.z = fmaf(t1v[e], x4.z, acc1.z), acc1.w = fmaf(t1v[e], x4.w, acc1.w);
         }
       }
-      *reinterpret_cast<float4*>(Tf + (32 + ii) * LD + j0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+      *reinterpret_cast<float4*>(Tf + (32 + r) * LD + j0) = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
+      *reinterpret_cast<float4*>(Tf + (48 + r) * LD + j0) = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
     }
     sync();
   }
