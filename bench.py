@@ -73,17 +73,18 @@ def decode_bytes(w, in_bytes=2, out_bytes=4) -> int:
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel from one ncu
-# capture, per token (it scales with the tokens of a launch).  Valid only for the kernel source it was
-# taken on: a different source hash reports null.
+# capture, per token (it scales with the tokens of a launch).  Valid only for the kernel sources it was
+# taken on: a different hash of those files reports null.
+_WS_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/chunk_scan_ws.cu",
+               "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
+               "delta_rule_recurrent_scan_b200/csrc/sm100.cuh"]
 NCU_TRAFFIC = {
-    "kalman_diag_d128": {"source": "delta_rule_recurrent_scan_b200/csrc/chunk_scan.cu",
-                         "sha1": "a4d45e21606002d911e4dc1a1f754a7982defd1b",
-                         "bytes_per_token": (205.815296e6 + 100.244480e6) / (2 * 16 * 8192),
-                         "capture": "profiles/chunk_scan_kernel_kalman_diag_d128.md (B=2 case, scaled)"},
-    "gdn_d128": {"source": "delta_rule_recurrent_scan_b200/csrc/chunk_scan.cu",
-                 "sha1": "a4d45e21606002d911e4dc1a1f754a7982defd1b",
-                 "bytes_per_token": (205.605376e6 + 100.905472e6) / (2 * 16 * 8192),
-                 "capture": "profiles/chunk_scan_kernel_delta_d128.md (B=2 case, scaled)"},
+    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "39b1537fb07afebd68394982e597811441d83d3c",
+                         "bytes_per_token": (205.706496e6 + 103.683840e6) / (2 * 16 * 8192),
+                         "capture": "profiles/chunk_scan_ws_kernel_kalman_diag_d128.md (B=2 case, scaled)"},
+    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "39b1537fb07afebd68394982e597811441d83d3c",
+                 "bytes_per_token": (205.632256e6 + 104.837632e6) / (2 * 16 * 8192),
+                 "capture": "profiles/chunk_scan_ws_kernel_delta_d128.md (B=2 case, scaled)"},
 }
 
 
@@ -93,11 +94,14 @@ def ncu_traffic(w):
     rec = NCU_TRAFFIC.get(w.name)
     if rec is None:
         return None
+    h = hashlib.sha1()
     try:
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha1(f.read()).hexdigest() != rec["sha1"]:
-                return None
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
     except OSError:
+        return None
+    if h.hexdigest() != rec["sha1"]:
         return None
     return rec["bytes_per_token"] * w.tokens
 
