@@ -5,6 +5,8 @@ bench.py's CPU baseline, never by the product package.  See ``oracle.scan``
 for what it computes, the readings it takes and the pins that hold it.
 """
 
-from .scan import decode_step, diag_update, kalman_update, scan_delta, scan_kalman_diag, scan_kalman_full
+from .scan import (decode_step, diag_update, iso_update, kalman_update, scan_delta, scan_kalman_diag,
+                   scan_kalman_full, scan_kalman_iso)
 
-__all__ = ["scan_delta", "scan_kalman_full", "scan_kalman_diag", "decode_step", "kalman_update", "diag_update"]
+__all__ = ["scan_delta", "scan_kalman_full", "scan_kalman_diag", "scan_kalman_iso", "decode_step", "kalman_update",
+           "diag_update", "iso_update"]

@@ -57,6 +57,13 @@ R4  Surprise for every variant is the Frobenius norm of the write, excluding
 R5  The read uses the post-update state and no 1/sqrt(d) scale.
 R6  Orientation: S is d_k x d_v and the read is S^T q (HOLA and the GDN gate
     formula); the DeltaNet-PC page writes the transpose, S k.
+R12 Isotropic variant (one uncertainty scalar c per head; the KDN abstract
+    gives no formula): propagate c^- = a_t^2 c + Qn_t; the mean is the exact
+    posterior mean under the prior c^- I, so g_t = c^- k_t / (c^- ||k_t||^2 + r_t);
+    the variance is the isotropic mean-field optimum, KL(q || posterior) over
+    N(mu, c I), c = d_k / tr(posterior precision) = d_k c^- r / (d_k r + c^- ||k||^2).
+    Composed with the propagation this is again a Moebius map of c, and the
+    write is the delta rule's with beta_t = c^- / (c^- ||k_t||^2 + r_t).
 
 Pins (tests/test_oracle_pins.py): the ridge closed form for every prefix,
 brute-force joint-Gaussian conditioning on tiny inputs, the isotropic-surrogate
@@ -79,6 +86,8 @@ __all__ = [
     "decode_step",
     "kalman_update",
     "diag_update",
+    "scan_kalman_iso",
+    "iso_update",
 ]
 
 
@@ -284,6 +293,69 @@ def scan_kalman_diag(q, k, v, r, a=None, qn=None, S0=None, p0=None, return_state
     if return_states:
         out["S_hist"] = S_hist.reshape(*lead, L, dk, dv)
         out["p_hist"] = p_hist.reshape(*lead, L, dk)
+    return out
+
+
+# --------------------------------------------------------------------------- isotropic Kalman
+
+
+def iso_update(S_pred, c_pred, k, v, r):
+    """Measurement update with an isotropic prior covariance c_pred I (reading R12).
+
+    Kalman Delta Networks, Abstract: Isotropic KDN uses an isotropic
+    approximation with a single uncertainty scalar per head.  The posterior
+    mean is the exact conditional mean under the prior c_pred I; the projected
+    variance is d_k over the trace of the posterior precision
+    I / c_pred + k k^T / r, written without dividing by c_pred.
+
+    Returns (S, c, g, e, s).
+    """
+    dk = k.shape[-1]
+    e = v - _read(S_pred, k)
+    kk = np.einsum("ni,ni->n", k, k)
+    s = c_pred * kk + r
+    g = (c_pred / s)[:, None] * k
+    S = S_pred + g[:, :, None] * e[:, None, :]
+    c = dk * c_pred * r / (dk * r + c_pred * kk)
+    return S, c, g, e, s
+
+
+def scan_kalman_iso(q, k, v, r, a=None, qn=None, S0=None, c0=None, return_states=False):
+    """Isotropic-covariance Kalman memory, token by token.
+
+    Per token: S^- = a_t S, c^- = a_t^2 c + Qn_t, then ``iso_update``.
+    c0 [...] or None (=1).  Returns o, m, S, c and, with ``return_states``,
+    S_hist and c_hist.
+    """
+    lead, n, L, dk, dv, q, k, v = _flatten_inputs(q, k, v)
+    r = _per_token(r, n, L, 1.0)
+    a = _per_token(a, n, L, 1.0)
+    qn = _per_token(qn, n, L, 0.0)
+    S = np.zeros((n, dk, dv)) if S0 is None else _f64(S0).reshape(n, dk, dv).copy()
+    c = np.ones(n) if c0 is None else _f64(c0).reshape(n).copy()
+    o = np.zeros((n, L, dv))
+    m = np.zeros((n, L))
+    S_hist = np.zeros((n, L, dk, dv)) if return_states else None
+    c_hist = np.zeros((n, L)) if return_states else None
+    for t in range(L):
+        at = a[:, t]
+        S_pred = at[:, None, None] * S
+        c_pred = at * at * c + qn[:, t]
+        S, c, g, e, _ = iso_update(S_pred, c_pred, k[:, t], v[:, t], r[:, t])
+        o[:, t] = _read(S, q[:, t])
+        m[:, t] = np.linalg.norm(g, axis=-1) * np.linalg.norm(e, axis=-1)
+        if return_states:
+            S_hist[:, t] = S
+            c_hist[:, t] = c
+    out = {
+        "o": o.reshape(*lead, L, dv),
+        "m": m.reshape(*lead, L),
+        "S": S.reshape(*lead, dk, dv),
+        "c": c.reshape(lead),
+    }
+    if return_states:
+        out["S_hist"] = S_hist.reshape(*lead, L, dk, dv)
+        out["c_hist"] = c_hist.reshape(*lead, L)
     return out
 
 

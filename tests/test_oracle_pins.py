@@ -14,7 +14,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
-from oracle import decode_step, kalman_update, scan_delta, scan_kalman_diag, scan_kalman_full
+from oracle import decode_step, kalman_update, scan_delta, scan_kalman_diag, scan_kalman_full, scan_kalman_iso
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -254,7 +254,7 @@ def test_residual_reading_against_decayed_state():
 # ----------------------------------------------------------------------------- surprise
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_full", "kalman_diag"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_full", "kalman_diag", "kalman_iso"])
 def test_surprise_is_frobenius_norm_of_the_write(variant):
     """A Hippocampus for Linear Attention, section 3.3, Eq. (6): m_t = ||Delta_t||_F,
     Delta_t = S_t - a_t S_{t-1} (the write, without the decay)."""
@@ -268,8 +268,10 @@ def test_surprise_is_frobenius_norm_of_the_write(variant):
         res = scan_delta(q, k, v, beta[None], a=a[None], return_states=True)
     elif variant == "kalman_full":
         res = scan_kalman_full(q, k, v, r=r[None], a=a[None], qn=1e-3, return_states=True)
-    else:
+    elif variant == "kalman_diag":
         res = scan_kalman_diag(q, k, v, r=r[None], a=a[None], qn=1e-3, return_states=True)
+    else:
+        res = scan_kalman_iso(q, k, v, r=r[None], a=a[None], qn=1e-3, return_states=True)
     S_prev = np.zeros((6, 5))
     for t in range(L):
         S_t = res["S_hist"][0, t]
@@ -356,6 +358,102 @@ def test_diag_variances_minimise_reverse_kl():
                            p0=p_pred[None])
     np.testing.assert_allclose(res["p"][0], np.exp(opt.x), rtol=1e-6)
     assert S_pred.shape == (1, dk, 1)
+
+
+# ----------------------------------------------------------------------------- isotropic variant
+# Kalman Delta Networks, Abstract: Isotropic KDN keeps a single uncertainty scalar per head (reading R12).
+
+
+def test_iso_equals_full_kalman_in_one_dimension():
+    """With d_k = 1 every covariance is a scalar, so the isotropic projection is exact and
+    the variant is the full Kalman filter (and the diagonal one)."""
+    rng = np.random.default_rng(21)
+    L, dv, n = 50, 4, 3
+    q = rng.standard_normal((n, L, 1))
+    k = rng.standard_normal((n, L, 1))
+    v = rng.standard_normal((n, L, dv))
+    a = 0.4 + 0.6 * rng.random((n, L))
+    r = 0.1 + rng.random((n, L))
+    c0 = 0.3 + rng.random(n)
+    iso = scan_kalman_iso(q, k, v, r=r, a=a, qn=3e-2, c0=c0)
+    full = scan_kalman_full(q, k, v, r=r, a=a, qn=3e-2, P0=c0[:, None, None])
+    for key in ("o", "m", "S"):
+        np.testing.assert_allclose(iso[key], full[key], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(iso["c"], full["P"][:, 0, 0], rtol=1e-12)
+
+
+def test_iso_variance_closed_form_without_transition():
+    """a = 1, Q = 0: the trace of the precision grows by ||k_t||^2 / r_t per token, so
+    d_k / c_L = d_k / c0 + sum_t ||k_t||^2 / r_t (non-unit keys)."""
+    rng, q, k, v = _case(22, 60, 6, 3)
+    k = k * (0.3 + rng.random((1, 60, 1)))
+    r = 0.1 + rng.random(60)
+    c0 = 0.7
+    res = scan_kalman_iso(q, k, v, r=r[None], c0=np.array([c0]))
+    dk = 6
+    np.testing.assert_allclose(res["c"][0], dk / (dk / c0 + ((k[0] ** 2).sum(-1) / r).sum()), rtol=1e-12)
+
+
+def test_iso_mean_and_variance_are_conditioning_then_isotropic_projection():
+    """Each step: the mean is exact Gaussian conditioning under the isotropic prior
+    N(a S_{t-1}, c^- I) (explicit inverses), and the variance is d_k over the trace of the
+    posterior precision."""
+    rng, q, k, v = _case(23, 30, 5, 3)
+    L = 30
+    k = k * (0.5 + rng.random((1, L, 1)))
+    a = 0.5 + 0.5 * rng.random(L)
+    r = 0.1 + rng.random(L)
+    qn = 0.02
+    res = scan_kalman_iso(q, k, v, r=r[None], a=a[None], qn=qn, return_states=True)
+    S_prev, c_prev = np.zeros((5, 3)), 1.0
+    for t in range(L):
+        c_pred = a[t] ** 2 * c_prev + qn
+        kt = k[0, t]
+        prior_prec = np.eye(5) / c_pred
+        post_prec = prior_prec + np.outer(kt, kt) / r[t]
+        post_cov = np.linalg.inv(post_prec)
+        mean = post_cov @ (prior_prec @ (a[t] * S_prev) + np.outer(kt, v[0, t]) / r[t])
+        np.testing.assert_allclose(res["S_hist"][0, t], mean, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(res["c_hist"][0, t], 5.0 / np.trace(post_prec), rtol=1e-12)
+        S_prev, c_prev = res["S_hist"][0, t], res["c_hist"][0, t]
+
+
+def test_iso_variance_minimises_reverse_kl():
+    """The isotropic projection minimises KL(N(mu, c I) || posterior) over c; minimise it
+    numerically and compare."""
+    scipy_opt = pytest.importorskip("scipy.optimize")
+    rng = np.random.default_rng(24)
+    dk = 4
+    c_pred = 0.8
+    kt = rng.standard_normal(dk)
+    r = 0.3
+    prec = np.eye(dk) / c_pred + np.outer(kt, kt) / r
+
+    def kl(logc):  # KL(N(mu, exp(logc) I) || N(mu, prec^-1)), up to constants
+        return 0.5 * (np.exp(logc[0]) * np.trace(prec) - dk * logc[0])
+
+    opt = scipy_opt.minimize(kl, np.zeros(1), method="BFGS", options={"gtol": 1e-12})
+    res = scan_kalman_iso(np.zeros((1, 1, dk)), kt[None, None], np.zeros((1, 1, 1)), r=np.array([[r]]),
+                          c0=np.array([c_pred]))
+    np.testing.assert_allclose(res["c"][0], np.exp(opt.x[0]), rtol=1e-6)
+
+
+def test_iso_is_the_delta_rule_with_a_variance_driven_beta():
+    """The isotropic gain is c^- k / (c^- ||k||^2 + r): the delta rule's write with
+    beta_t = c^-_t / (c^-_t ||k_t||^2 + r_t)."""
+    rng, q, k, v = _case(25, 40, 6, 4)
+    L = 40
+    k = k * (0.5 + rng.random((1, L, 1)))
+    a = 0.5 + 0.5 * rng.random(L)
+    r = 0.1 + rng.random(L)
+    qn = 1e-2
+    iso = scan_kalman_iso(q, k, v, r=r[None], a=a[None], qn=qn, return_states=True)
+    c_prev = np.concatenate([[1.0], iso["c_hist"][0, :-1]])
+    c_pred = a * a * c_prev + qn
+    beta = c_pred / (c_pred * (k[0] ** 2).sum(-1) + r)
+    delta = scan_delta(q, k, v, beta[None], a=a[None])
+    for key in ("o", "m", "S"):
+        np.testing.assert_allclose(iso[key], delta[key], rtol=1e-12, atol=1e-13)
 
 
 # ----------------------------------------------------------------------------- decode
