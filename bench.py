@@ -43,7 +43,7 @@ sys.path.insert(0, ROOT)
 from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_decode_inputs, make_scan_inputs  # noqa: E402
 
 HEADLINE = "kalman_diag_d128"
-SECONDARY = ["gdn_d128", "kalman_full_d128", "gdn_d64"]
+SECONDARY = ["gdn_d128", "kalman_iso_d128", "kalman_full_d128", "gdn_d64"]
 DECODE = ["decode_delta", "decode_diag"]
 METRIC = "scan tokens/s per layer (B*H*L/time) at d=128"
 
@@ -55,12 +55,14 @@ def algorithmic_bytes(w, in_bytes=2, out_bytes=4) -> int:
     """Bytes one scan must move: q, k, v in, o out, per-token scalars, m out, state in and out."""
     tok = w.B * w.H * w.L
     io = tok * ((2 * w.dk + w.dv) * in_bytes + w.dv * out_bytes + 4)  # + m
-    scalars = {"delta": 8, "kalman_diag": 8, "kalman_full": 8}[w.variant]  # beta|r and a
+    scalars = {"delta": 8, "kalman_diag": 8, "kalman_full": 8, "kalman_iso": 8}[w.variant]  # beta|r and a
     state = w.B * w.H * w.dk * w.dv * 4 * 2
     if w.variant == "kalman_full":
         state += w.B * w.H * w.dk * w.dk * 4 * 2
     elif w.variant == "kalman_diag":
         state += w.B * w.H * w.dk * 4 * 2
+    elif w.variant == "kalman_iso":
+        state += w.B * w.H * 4 * 2
     return io + tok * scalars + state
 
 
@@ -247,6 +249,13 @@ def scan_closure(w, x, kdn):
             kdn.scan_kalman_full(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, P=P, o=o, m=m,
                                  workspace=ws)
         return fn, outs
+    if w.variant == "kalman_iso":
+        c = torch.ones(B, H, device=dev)
+
+        def fn():
+            kdn.scan_kalman_iso(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, c=c, o=o, m=m,
+                                workspace=ws)
+        return fn, outs
     p = torch.ones(B, H, dk, device=dev)
 
     def fn():
@@ -331,6 +340,8 @@ def cpu_baseline(w, heads=16, seconds_hint=None):
         oracle.scan_delta(np_["q"], np_["k"], np_["v"], np_["beta"], a=np_["a"])
     elif w.variant == "kalman_full":
         oracle.scan_kalman_full(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+    elif w.variant == "kalman_iso":
+        oracle.scan_kalman_iso(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
     else:
         oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
     dt = time.perf_counter() - t0
@@ -469,6 +480,8 @@ def reference_arm(args, w, rank, world):
             oracle.scan_delta(np_["q"], np_["k"], np_["v"], np_["beta"], a=np_["a"])
         elif w.variant == "kalman_full":
             oracle.scan_kalman_full(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
+        elif w.variant == "kalman_iso":
+            oracle.scan_kalman_iso(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
         else:
             oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
 

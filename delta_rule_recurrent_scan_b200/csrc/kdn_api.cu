@@ -146,6 +146,7 @@ size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
     case KDN_DELTA: break;
     case KDN_KALMAN_DIAG:
     case KDN_KALMAN_FULL: n += gains_bytes(dims); break;
+    case KDN_KALMAN_ISO: n += (size_t)dims->B * dims->H * (size_t)dims->L * sizeof(float); break;
     default: return 0;
   }
   return (n + 255) / 256 * 256;
@@ -154,20 +155,23 @@ size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
 kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, const char** kernel,
                     const char** arith) {
   KDN_TRY(check_dims(dims));
-  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_FULL)
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_FULL && variant != KDN_KALMAN_ISO)
     return fail(KDN_ERR_INVALID_ARG, "bad variant");
+  // the isotropic scan is the delta scan after its beta prologue (one more launch)
+  const kdn_variant body = variant == KDN_KALMAN_ISO ? KDN_DELTA : variant;
   int n = 0;
   const char* name = "";
   const char* ar = "f32";
   if (dims->L == 0) {
     n = 0, name = "none";
-  } else if (kdn::chunk_supported(variant, *dims)) {
-    kdn::chunk_plan(variant, *dims, &n, &name, &ar);
-  } else if (variant == KDN_DELTA) {
+  } else if (kdn::chunk_supported(body, *dims)) {
+    kdn::chunk_plan(body, *dims, &n, &name, &ar);
+  } else if (body == KDN_DELTA) {
     n = 1, name = "seq_scan_kernel";
   } else {
     n = 2, name = "seq_scan_kernel";
   }
+  if (variant == KDN_KALMAN_ISO && n > 0) n += 1;
   if (launches) *launches = n;
   if (kernel) *kernel = name;
   if (arith) *arith = ar;
@@ -258,6 +262,36 @@ kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, const void*
                                 float* m, void* workspace, size_t workspace_bytes, void* stream) {
   return kalman_scan(KDN_KALMAN_DIAG, dims, q, k, v, a, r, qn, qn_scalar, S, p, o, m, workspace, workspace_bytes,
                      stream);
+}
+
+kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* a,
+                               const float* r, const float* qn, float qn_scalar, float* S, float* c, void* o,
+                               float* m, void* workspace, size_t workspace_bytes, void* stream) {
+  KDN_TRY(common_checks(KDN_KALMAN_ISO, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(c, "c", 4, false));
+  KDN_TRY(check_ptr(r, "r", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(qn, "qn", 4, true));
+  if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "clearing the status word");
+  if (!any) return ok();
+  const int BH = dims->B * dims->H;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  float* beta = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + kStatusBytes);
+  kdn::IsoArgs ia{k, dims->in_dtype, a, r, qn, qn_scalar, c, beta, status, dims->L};
+  e = kdn::launch_iso_beta(dims->dk, ia, BH, st);
+  if (e != cudaSuccess) return cuda_status(e, "isotropic beta launch");
+  if (kdn::chunk_supported(KDN_DELTA, *dims)) {
+    kdn::ChunkArgs ch{};
+    ch.q = q, ch.k = k, ch.v = v, ch.beta = beta, ch.a = a, ch.S = S, ch.o = o, ch.m = m;
+    ch.out_dtype = dims->out_dtype, ch.BH = BH, ch.L = dims->L, ch.status = status;
+    return cuda_status(kdn::launch_chunk(KDN_DELTA, *dims, ch, st), "chunked isotropic scan launch");
+  }
+  kdn::SeqScanArgs sa{q, k, v, dims->in_dtype, dims->out_dtype, beta, a, nullptr, S, o, m, BH, dims->L};
+  return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, sa, st), "isotropic scan launch");
 }
 
 kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype, kdn_dtype out_dtype,

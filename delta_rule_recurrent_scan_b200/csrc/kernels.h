@@ -57,7 +57,22 @@ struct DecodeArgs {
   int BH;
 };
 
+// Isotropic-Kalman prologue: per-token write strengths beta_t from one uncertainty scalar per head.
+struct IsoArgs {
+  const void* k;     // [BH, L, dk]
+  int in_dtype;
+  const float* a;    // [BH, L] or nullptr
+  const float* r;    // [BH, L]
+  const float* qn;   // [BH, L] or nullptr
+  float qn_scalar;
+  float* c;          // [BH] in/out
+  float* beta;       // out: [BH, L]
+  unsigned* status;
+  int L;
+};
+
 cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream);
+cudaError_t launch_iso_beta(int dk, const IsoArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream);
 cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream);
 cudaError_t launch_decode(int dk, int dv, bool diag, const DecodeArgs& args, cudaStream_t stream);

@@ -24,7 +24,7 @@ HEADER = os.path.join(ROOT, "include", "kdn.h")
 
 KDN_OK, KDN_ERR_INVALID_ARG, KDN_ERR_UNSUPPORTED, KDN_ERR_CUDA, KDN_ERR_NUMERIC, KDN_ERR_TIMEOUT = range(6)
 KDN_F32, KDN_BF16 = 0, 1
-VARIANTS = {"delta": 0, "kalman_diag": 1, "kalman_full": 2}
+VARIANTS = {"delta": 0, "kalman_diag": 1, "kalman_full": 2, "kalman_iso": 3}
 _DTYPES = {torch.float32: KDN_F32, torch.bfloat16: KDN_BF16}
 
 
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_delta.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_full.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_diag.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
+    L.kdn_scan_kalman_iso.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_decode_step.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.restype = ctypes.c_int
@@ -247,6 +248,28 @@ def scan_kalman_diag(q, k, v, r, a=None, qn=None, S=None, p=None, o=None, m=None
                                     _stream(stream))
     _check(st, "kdn_scan_kalman_diag")
     return o, m, S, p
+
+
+def scan_kalman_iso(q, k, v, r, a=None, qn=None, S=None, c=None, o=None, m=None, workspace=None, chunk=0,
+                    out_dtype=None, stream=None):
+    """Isotropic-covariance Kalman scan (one uncertainty scalar per head).  Returns (o, m, S, c); S and c
+    are updated in place when given."""
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    B, H, L, dk = q.shape
+    tok = (B, H, L)
+    _need(r, "r", tok, torch.float32, q.device)
+    if a is not None:
+        _need(a, "a", tok, torch.float32, q.device)
+    qn_t, qn_s = _qn_args(qn, tok, q.device)
+    if c is None:
+        c = torch.ones(B, H, dtype=torch.float32, device=q.device)
+    _need(c, "c", (B, H), torch.float32, q.device)
+    workspace = _workspace("kalman_iso", dims, workspace, q.device)
+    st = lib().kdn_scan_kalman_iso(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(r), _ptr(qn_t), qn_s,
+                                   _ptr(S), _ptr(c), _ptr(o), _ptr(m), _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+    _check(st, "kdn_scan_kalman_iso")
+    return o, m, S, c
 
 
 def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=0.0, p=None, o=None, m=None, out_dtype=None,

@@ -31,7 +31,7 @@ __all__ = ["Workload", "WORKLOADS", "make_scan_inputs", "make_decode_inputs"]
 @dataclass(frozen=True)
 class Workload:
     name: str
-    variant: str  # "delta" | "kalman_full" | "kalman_diag"
+    variant: str  # "delta" | "kalman_full" | "kalman_diag" | "kalman_iso"
     B: int
     H: int
     L: int
@@ -65,6 +65,8 @@ WORKLOADS = {
     "kalman_full_d128": Workload("kalman_full_d128", "kalman_full", 2, 8, 4096, 128, 128, "bf16", a_shift=3.0, qn=1e-3),
     "kalman_diag_d128": Workload("kalman_diag_d128", "kalman_diag", 8, 16, 8192, 128, 128, "bf16", a_shift=2.0, qn=1e-3),
     "gdn_d128": Workload("gdn_d128", "delta", 8, 16, 8192, 128, 128, "bf16", a_shift=2.0),
+    # isotropic Kalman (one uncertainty scalar per head) at the diagonal layer's shape and distributions
+    "kalman_iso_d128": Workload("kalman_iso_d128", "kalman_iso", 8, 16, 8192, 128, 128, "bf16", a_shift=2.0, qn=1e-3),
     # decode: batch 256 x 32 heads, one token per call, 1024 calls
     "decode_delta": Workload("decode_delta", "delta", 256, 32, 1, 128, 128, "bf16", a_shift=2.0, steps=1024),
     "decode_diag": Workload("decode_diag", "kalman_diag", 256, 32, 1, 128, 128, "bf16", a_shift=2.0, qn=1e-3, steps=1024),
@@ -91,7 +93,7 @@ def make_scan_inputs(w: Workload, seed: int = 0, device="cpu", B: int | None = N
 
     Returns q, k [B,H,L,dk] and v [B,H,L,dv] in the workload dtype, and float32
     beta, a (or None), r [B,H,L], plus the scalar qn.  The initial state is
-    S0 = 0, P0 = I (full) or p0 = 1 (diagonal); the caller allocates it.
+    S0 = 0, P0 = I (full), p0 = 1 (diagonal) or c0 = 1 (isotropic); the caller allocates it.
     """
     B = w.B if B is None else B
     H = w.H if H is None else H

@@ -89,7 +89,7 @@ typedef enum kdn_status {
 
 typedef enum kdn_dtype { KDN_F32 = 0, KDN_BF16 = 1 } kdn_dtype;
 
-typedef enum kdn_variant { KDN_DELTA = 0, KDN_KALMAN_DIAG = 1, KDN_KALMAN_FULL = 2 } kdn_variant;
+typedef enum kdn_variant { KDN_DELTA = 0, KDN_KALMAN_DIAG = 1, KDN_KALMAN_FULL = 2, KDN_KALMAN_ISO = 3 } kdn_variant;
 
 typedef struct kdn_dims {
   int B, H, L;          /* batch, heads, tokens */
@@ -121,6 +121,19 @@ KDN_EXPORT kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, 
                                 const float* a, const float* r, const float* qn, float qn_scalar,
                                 float* S, float* p, void* o, float* m,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Isotropic-covariance Kalman scan (Kalman Delta Networks, Abstract: Isotropic
+ * KDN keeps a single uncertainty scalar per head; its recurrence is a Moebius
+ * map, scanned associatively).  Per token: c^- = a^2 c + Qn, gain
+ * c^- k / (c^- ||k||^2 + r) (the delta rule's write with that beta), and the
+ * isotropic mean-field variance c = d_k c^- r / (d_k r + c^- ||k||^2).
+ * c: [B,H] uncertainty in/out, positive.  Other arguments as for
+ * kdn_scan_kalman_diag.  The workspace also holds the per-token beta
+ * ([B,H,L] fp32 after the status word). */
+KDN_EXPORT kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                               const float* a, const float* r, const float* qn, float qn_scalar,
+                               float* S, float* c, void* o, float* m,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* kdn_scan_kalman_full for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a deployment variant.  Callers that must

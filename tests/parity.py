@@ -30,6 +30,8 @@ def initial_state(variant, B, H, dk, dv, device):
         return S, torch.eye(dk, dtype=torch.float32, device=device).repeat(B, H, 1, 1)
     if variant == "kalman_diag":
         return S, torch.ones(B, H, dk, dtype=torch.float32, device=device)
+    if variant == "kalman_iso":
+        return S, torch.ones(B, H, dtype=torch.float32, device=device)
     return S, None
 
 
@@ -42,8 +44,9 @@ def run_gpu(variant, x, S=None, C=None, chunk=0, out_dtype=None):
     if variant == "delta":
         o, m, S = kdn.scan_delta(q, k, v, x["beta"], a=x["a"], S=S, chunk=chunk, out_dtype=out_dtype)
         return {"o": o, "m": m, "S": S}
-    fn = kdn.scan_kalman_full if variant == "kalman_full" else kdn.scan_kalman_diag
-    key = "P" if variant == "kalman_full" else "p"
+    fn = {"kalman_full": kdn.scan_kalman_full, "kalman_diag": kdn.scan_kalman_diag,
+          "kalman_iso": kdn.scan_kalman_iso}[variant]
+    key = {"kalman_full": "P", "kalman_diag": "p", "kalman_iso": "c"}[variant]
     kw = {key: C}
     o, m, S, C = fn(q, k, v, x["r"], a=x["a"], qn=x["qn"], S=S, chunk=chunk, out_dtype=out_dtype, **kw)
     return {"o": o, "m": m, "S": S, key: C}
@@ -68,6 +71,8 @@ def run_oracle(variant, x, S0=None, C0=None, heads=None):
         return oracle.scan_delta(q, k, v, pick(x["beta"]), a=a, S0=pick(S0))
     if variant == "kalman_full":
         return oracle.scan_kalman_full(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), P0=pick(C0))
+    if variant == "kalman_iso":
+        return oracle.scan_kalman_iso(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), c0=pick(C0))
     return oracle.scan_kalman_diag(q, k, v, r=pick(x["r"]), a=a, qn=x["qn"], S0=pick(S0), p0=pick(C0))
 
 

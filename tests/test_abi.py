@@ -16,7 +16,7 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = kdn.exported_names()
-    assert {"kdn_scan_delta", "kdn_scan_kalman_full", "kdn_scan_kalman_diag", "kdn_decode_step",
+    assert {"kdn_scan_delta", "kdn_scan_kalman_full", "kdn_scan_kalman_diag", "kdn_scan_kalman_iso", "kdn_decode_step",
             "kdn_workspace_bytes", "kdn_read_device_status", "kdn_status_string", "kdn_last_error",
             "kdn_api_version"} <= set(names)
     for n in names:
@@ -32,9 +32,11 @@ def test_version_and_status_strings(L):
 
 def test_workspace_bytes(L):
     d = kdn.Dims(2, 3, 100, 64, 64, 0, kdn.KDN_BF16, kdn.KDN_BF16)
-    for v in (0, 1, 2):
+    for v in (0, 1, 2, 3):
         n = L.kdn_workspace_bytes(v, ctypes.byref(d))
         assert n >= 256 and n % 256 == 0
+    # the isotropic scan keeps one fp32 beta per token after the status word
+    assert L.kdn_workspace_bytes(3, ctypes.byref(d)) >= 256 + 2 * 3 * 100 * 4
     bad = kdn.Dims(2, 3, 100, 48, 64, 0, kdn.KDN_BF16, kdn.KDN_BF16)
     assert L.kdn_workspace_bytes(0, ctypes.byref(bad)) == 0
     assert L.kdn_workspace_bytes(0, None) == 0
@@ -62,6 +64,16 @@ def test_host_validation_without_gpu(L):
     assert L.kdn_decode_step(5, 1, 1, 64, 64, 1, 1, *([None] * 6), 0.0, *([None] * 5)) == kdn.KDN_ERR_UNSUPPORTED
     out = ctypes.c_int(0)
     assert L.kdn_read_device_status(None, ctypes.byref(out), None) == kdn.KDN_ERR_INVALID_ARG
+
+
+def test_plan_counts_the_isotropic_prologue(L):
+    for dims in (kdn.Dims(2, 3, 100, 128, 128, 0, kdn.KDN_BF16, kdn.KDN_F32),
+                 kdn.Dims(2, 3, 100, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32)):
+        n_delta, n_iso = ctypes.c_int(-1), ctypes.c_int(-1)
+        assert L.kdn_plan(0, ctypes.byref(dims), ctypes.byref(n_delta), None, None) == kdn.KDN_OK
+        assert L.kdn_plan(3, ctypes.byref(dims), ctypes.byref(n_iso), None, None) == kdn.KDN_OK
+        assert n_iso.value == n_delta.value + 1
+    assert L.kdn_plan(4, ctypes.byref(kdn.Dims(1, 1, 4, 64, 64, 0, 1, 1)), None, None, None) == kdn.KDN_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():

@@ -51,6 +51,17 @@ def test_tiny_kalman_fp32_matches_oracle_and_ridge():
     assert normwise_err(got["P"][0, 0][None, None], P_ridge[None, None]) < TOL["f32"]
 
 
+def test_tiny_isotropic_fp32_and_a_long_sequence():
+    """The isotropic prologue scans its per-head Moebius maps in tiles of 2048 tokens: a sequence of
+    several tiles (with a ragged last one) checks the carry between tiles."""
+    w = WORKLOADS["tiny_kalman"].with_(variant="kalman_iso", a_shift=2.0, qn=1e-3, r_const=None)
+    x = _to(make_scan_inputs(w, seed=0), DEV)
+    compare(run_gpu("kalman_iso", x), run_oracle("kalman_iso", x), TOL["f32"])
+    x = make_scan_inputs(w, seed=1, device=DEV, B=1, H=3, L=5000)
+    got = run_gpu("kalman_iso", x)
+    compare(got, run_oracle("kalman_iso", x), TOL["f32"])
+
+
 # ----------------------------------------------------------------------------- reduced layer shapes
 
 
@@ -59,6 +70,7 @@ def test_tiny_kalman_fp32_matches_oracle_and_ridge():
     ("gdn_d128", 1, 2, 300),
     ("kalman_diag_d128", 1, 2, 300),
     ("kalman_full_d128", 1, 2, 200),
+    ("kalman_iso_d128", 1, 2, 300),
 ])
 def test_layer_shapes_reduced(name, B, H, L):
     w = WORKLOADS[name]
@@ -67,7 +79,7 @@ def test_layer_shapes_reduced(name, B, H, L):
     compare(got, run_oracle(w.variant, x), TOL["bf16"])
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 @pytest.mark.parametrize("dk,dv", [(64, 32), (32, 128), (16, 64), (128, 16)])
 def test_unequal_head_dims(variant, dk, dv):
     w = WORKLOADS["gdn_d64"].with_(variant=variant, dk=dk, dv=dv, qn=1e-3)
@@ -76,7 +88,7 @@ def test_unequal_head_dims(variant, dk, dv):
     compare(got, run_oracle(variant, x), TOL["bf16"])
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 def test_bf16_output_within_tolerance_beyond_its_rounding(variant):
     w = WORKLOADS["gdn_d128"].with_(variant=variant, qn=1e-3)
     x = make_scan_inputs(w, seed=13, device=DEV, B=1, H=2, L=200)
@@ -85,14 +97,14 @@ def test_bf16_output_within_tolerance_beyond_its_rounding(variant):
     compare(got, run_oracle(variant, x), TOL["bf16"])
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 def test_fp32_inputs_d64(variant):
     w = WORKLOADS["gdn_d64"].with_(variant=variant, dtype="f32", qn=1e-3)
     x = make_scan_inputs(w, seed=3, device=DEV, B=1, H=2, L=150)
     compare(run_gpu(variant, x), run_oracle(variant, x), TOL["f32"])
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 @pytest.mark.parametrize("d", [64, 128])
 def test_tensor_core_path_matches_per_token_path(variant, d):
     """chunk=0 takes the chunked tcgen05 kernel for bf16 d in {64, 128}; chunk=32 the per-token kernels."""
@@ -110,7 +122,7 @@ def test_tensor_core_path_matches_per_token_path(variant, d):
 # ----------------------------------------------------------------------------- edge cases
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 def test_empty_sequence_is_a_no_op(variant):
     w = WORKLOADS["gdn_d64"].with_(variant=variant)
     x = make_scan_inputs(w, seed=4, device=DEV, B=2, H=2, L=0)
@@ -122,7 +134,7 @@ def test_empty_sequence_is_a_no_op(variant):
     assert torch.equal(got["S"], S0)
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 def test_single_token_and_degenerate_gates(variant):
     w = WORKLOADS["gdn_d64"].with_(variant=variant, qn=1e-3)
     x = make_scan_inputs(w, seed=5, device=DEV, B=2, H=2, L=97)
@@ -135,7 +147,7 @@ def test_single_token_and_degenerate_gates(variant):
     compare(run_gpu(variant, x1), run_oracle(variant, x1), TOL["bf16"])
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
 def test_split_invariance_and_resume(variant):
     """scan(x_1..L) equals scan(x_1..L1) then scan(x_L1+1..L) with the state passed through."""
     w = WORKLOADS["gdn_d64"].with_(variant=variant, qn=1e-3)
@@ -161,7 +173,7 @@ def _sample_heads(B, H, n=2, seed=0):
     return [(int(g.integers(B)), int(g.integers(H))) for _ in range(n)]
 
 
-@pytest.mark.parametrize("name", ["gdn_d64", "kalman_full_d128", "kalman_diag_d128", "gdn_d128"])
+@pytest.mark.parametrize("name", ["gdn_d64", "kalman_full_d128", "kalman_diag_d128", "gdn_d128", "kalman_iso_d128"])
 def test_full_size_sampled_heads(name):
     w = WORKLOADS[name]
     x = make_scan_inputs(w, seed=0, device=DEV)
@@ -239,6 +251,18 @@ def test_numeric_status_flag_for_non_positive_innovation_variance():
     assert kdn.read_device_status(ws) == kdn.KDN_ERR_NUMERIC
     x["r"][0, 0, 5] = 1.0
     kdn.scan_kalman_full(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=0.0, workspace=ws)
+    assert kdn.read_device_status(ws) == kdn.KDN_OK
+
+
+def test_isotropic_numeric_status_flag():
+    w = WORKLOADS["gdn_d64"].with_(variant="kalman_iso")
+    x = make_scan_inputs(w, seed=10, device=DEV, B=1, H=2, L=300)
+    x["r"][0, 1, 250] = -10.0
+    ws = torch.empty(kdn.workspace_bytes("kalman_iso", 1, 2, 300, 64, 64), dtype=torch.uint8, device=DEV)
+    kdn.scan_kalman_iso(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=0.0, workspace=ws)
+    assert kdn.read_device_status(ws) == kdn.KDN_ERR_NUMERIC
+    x["r"][0, 1, 250] = 1.0
+    kdn.scan_kalman_iso(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=0.0, workspace=ws)
     assert kdn.read_device_status(ws) == kdn.KDN_OK
 
 
