@@ -321,6 +321,30 @@ def bench_decode(w, steps, warmup, dist_on, rank, world):
     return {"ms": ms, "value": w.B * w.H * world / (ms * 1e-3), "launches": steps}
 
 
+def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
+    """Surprise-cache read over a layer (the scan's m as the surprise; random here)."""
+    from delta_rule_recurrent_scan_b200 import kdn
+    x = make_scan_inputs(w, seed=rank, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(rank)
+    m = torch.rand(w.B, w.H, w.L, device="cuda", generator=g)
+    gq = torch.ones(w.dk, device="cuda")
+    gk = torch.ones(w.dk, device="cuda")
+    sink = torch.zeros(w.H, device="cuda")
+    o = torch.empty(w.B, w.H, w.L, w.dv, device="cuda")
+    cache = torch.empty(w.B, w.H, cache_w, dtype=torch.int32, device="cuda")
+
+    def fn():
+        kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=cache_w, block=64, o=o, cache=cache)
+    ms = time_device(fn, steps, warmup, dist_on)
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": steps}
+
+
+def hola_bytes(w, in_bytes=2) -> int:
+    """q, k, v in, m in, o^cache out (fp32), the final cache indices."""
+    return w.tokens * ((2 * w.dk + w.dv) * in_bytes + 4 + w.dv * 4) + w.B * w.H * 64 * 4
+
+
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
 
@@ -415,6 +439,14 @@ def main():
                          "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
             del r
             torch.cuda.empty_cache()
+        hw = WORKLOADS["gdn_d128"]
+        r = bench_hola(hw, max(3, args.steps // 4), 3, dist_on, rank, world)
+        ab = hola_bytes(hw)
+        also.append({"workload": "hola_cache_read_d128", "variant": "surprise-cache read (w=64, block 64)",
+                     "value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"],
+                     "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
+        del r
+        torch.cuda.empty_cache()
         for name in DECODE:
             dw = WORKLOADS[name]
             r = bench_decode(dw, 64, 8, dist_on, rank, world)

@@ -294,6 +294,33 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
   return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, sa, st), "isotropic scan launch");
 }
 
+kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* m,
+                               const float* gamma_q, const float* gamma_k, const float* sink, int w, float* o_cache,
+                               int* cache_idx, void* stream) {
+  KDN_TRY(check_dims(dims));
+  if (w < 1 || w > 64) return fail(KDN_ERR_UNSUPPORTED, "w must be in 1..64");
+  const int block = dims->chunk == 0 ? 64 : dims->chunk;
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(q, "q", 16, !any));
+  KDN_TRY(check_ptr(k, "k", 16, !any));
+  KDN_TRY(check_ptr(v, "v", 16, !any));
+  KDN_TRY(check_ptr(m, "m", 4, !any));
+  KDN_TRY(check_ptr(o_cache, "o_cache", 16, !any));
+  KDN_TRY(check_ptr(gamma_q, "gamma_q", 4, false));
+  KDN_TRY(check_ptr(gamma_k, "gamma_k", 4, false));
+  KDN_TRY(check_ptr(sink, "sink", 4, false));
+  KDN_TRY(check_ptr(cache_idx, "cache_idx", 4, true));
+  KDN_TRY(use_device_of(gamma_q));
+  const int BH = dims->B * dims->H;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!any) {
+    if (cache_idx == nullptr) return ok();
+    return cuda_status(cudaMemsetAsync(cache_idx, 0xff, (size_t)BH * w * sizeof(int), st), "clearing cache_idx");
+  }
+  kdn::HolaArgs ha{q, k, v, dims->in_dtype, m, gamma_q, gamma_k, sink, o_cache, cache_idx, dims->H, dims->L, block, w};
+  return cuda_status(kdn::launch_hola_read(dims->dk, dims->dv, ha, BH, st), "surprise-cache read launch");
+}
+
 kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype, kdn_dtype out_dtype,
                            const void* q, const void* k, const void* v, const float* beta, const float* a,
                            const float* r, float qn_scalar, float* S, float* p, void* o, float* m, void* stream) {

@@ -71,7 +71,26 @@ struct IsoArgs {
   int L;
 };
 
+// Surprise-cache read: top-w exact cache by m, sharpened softmax over cache, causal block and a sink.
+struct HolaArgs {
+  const void* q;          // [BH, L, dk]
+  const void* k;          // [BH, L, dk]
+  const void* v;          // [BH, L, dv]
+  int in_dtype;
+  const float* m;         // [BH, L] surprise
+  const float* gamma_q;   // [dk]
+  const float* gamma_k;   // [dk]
+  const float* sink;      // [H]
+  float* o;               // [BH, L, dv] fp32
+  int* cache;             // [BH, w] final cache token indices, or nullptr
+  int H;
+  int L;
+  int block;              // 16, 32 or 64
+  int w;                  // 1..64
+};
+
 cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream);
+cudaError_t launch_hola_read(int dk, int dv, const HolaArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_iso_beta(int dk, const IsoArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream);
 cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream);

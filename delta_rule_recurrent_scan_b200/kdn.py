@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_kalman_full.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_diag.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_iso.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
+    L.kdn_hola_cache_read.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp]
     L.kdn_decode_step.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.restype = ctypes.c_int
@@ -270,6 +271,34 @@ def scan_kalman_iso(q, k, v, r, a=None, qn=None, S=None, c=None, o=None, m=None,
                                    _stream(stream))
     _check(st, "kdn_scan_kalman_iso")
     return o, m, S, c
+
+
+def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, cache=None, stream=None):
+    """Surprise-cache read: q, k [B,H,L,d_k], v [B,H,L,d_v] (bf16 or fp32), m [B,H,L], gamma_q/gamma_k [d_k],
+    sink [H].  Returns (o_cache [B,H,L,d_v] fp32, cache [B,H,w] int32 token indices, ascending, -1 empty)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, L, d_k]")
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _need(q, "q", (B, H, L, dk), q.dtype)
+    _need(k, "k", (B, H, L, dk), q.dtype, dev)
+    _need(v, "v", (B, H, L, dv), q.dtype, dev)
+    _need(m, "m", (B, H, L), torch.float32, dev)
+    _need(gamma_q, "gamma_q", (dk,), torch.float32, dev)
+    _need(gamma_k, "gamma_k", (dk,), torch.float32, dev)
+    _need(sink, "sink", (H,), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, L, dv, dtype=torch.float32, device=dev)
+    _need(o, "o", (B, H, L, dv), torch.float32, dev)
+    if cache is None:
+        cache = torch.empty(B, H, w, dtype=torch.int32, device=dev)
+    _need(cache, "cache", (B, H, w), torch.int32, dev)
+    dims = Dims(B, H, L, dk, dv, block, _DTYPES[q.dtype], KDN_F32)
+    st = lib().kdn_hola_cache_read(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(gamma_q),
+                                   _ptr(gamma_k), _ptr(sink), int(w), _ptr(o), _ptr(cache), _stream(stream))
+    _check(st, "kdn_hola_cache_read")
+    return o, cache
 
 
 def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=0.0, p=None, o=None, m=None, out_dtype=None,

@@ -135,6 +135,24 @@ KDN_EXPORT kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, c
                                float* S, float* c, void* o, float* m,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* Surprise-cache read (A Hippocampus for Linear Attention, sections 3.3-3.4,
+ * Eq. (6)-(7)).  Each head keeps the exact (k, v) of the w tokens with the
+ * largest surprise m seen so far (ties: the earlier token); token t of block b
+ * (dims->chunk tokens per block: 16, 32 or 64; 0 = 64) reads with a softmax,
+ * temperature 1, over the cache of blocks 0..b-1, the tokens of its own block
+ * up to t, and a null sink (logit sink[h], no value):
+ *   o_t = sum_j softmax_j(q~_t . k~_j / sqrt(d_k)) v_j,
+ *   q~ = RMSNorm(q) * gamma_q, k~ = RMSNorm(k) * gamma_k (eps 1e-6).
+ * q, k [B,H,L,d_k], v [B,H,L,d_v] (dims->in_dtype); m [B,H,L] fp32 (finite;
+ * the m of a scan); gamma_q, gamma_k [d_k] shared by the heads; sink [H];
+ * 1 <= w <= 64.  Out: o_cache [B,H,L,d_v] fp32; cache_idx [B,H,w] int32 token
+ * indices of the final cache, ascending, -1 for empty slots, or NULL.  The
+ * state-read gate that mixes o_cache into the layer output is the caller's.
+ * Needs no workspace. */
+KDN_EXPORT kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                               const float* m, const float* gamma_q, const float* gamma_k, const float* sink,
+                               int w, float* o_cache, int* cache_idx, void* stream);
+
 /* kdn_scan_kalman_full for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a deployment variant.  Callers that must
  * not call cudaMalloc while running (a server that reserves all device memory

@@ -51,10 +51,11 @@ def top_w_indices(m, upto, w):
     return sorted(order[:w])
 
 
-def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, eps=1e-6):
+def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, eps=1e-6, tokens=None):
     """Surprise-cache read for q, k [B, H, L, d_k], v [B, H, L, d_v], m [B, H, L], sink [H].
 
-    Token by token: the visible set, the sharpened logits, the softmax with the sink.
+    Token by token: the visible set, the sharpened logits, the softmax with the sink.  ``tokens``
+    restricts the read to those token positions (the other rows of o stay 0).
     Returns {"o": [B, H, L, d_v], "cache": [B, H, w] token indices of the final cache (-1 = empty)}.
     """
     q, k, v, m = (np.asarray(x, dtype=np.float64) for x in (q, k, v, m))
@@ -67,7 +68,7 @@ def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, eps=1e-6
     cache_out = -np.ones((B, H, w), dtype=np.int64)
     for b in range(B):
         for h in range(H):
-            for t in range(L):
+            for t in (range(L) if tokens is None else tokens):
                 b0 = (t // block) * block
                 vis = top_w_indices(m[b, h], b0, w) + list(range(b0, t + 1))
                 logits = np.array([qt[b, h, t] @ kt[b, h, j] for j in vis]) / np.sqrt(dk)
