@@ -29,7 +29,7 @@ NVCC_FLAGS = [
 # IEEE single precision everywhere except the chunked tensor-core kernel, whose operands are
 # well-scaled (no denormals matter) and whose reciprocals and divisions sit on serial chains.
 IEEE_FLAGS = ["-ftz=false", "-prec-div=true", "-prec-sqrt=true"]
-PER_FILE_FLAGS = {name: ["-ftz=true", "-prec-div=false", "-prec-sqrt=false"] for name in ("chunk_scan.cu", "chunk_scan_ws.cu", "pside.cu")}
+PER_FILE_FLAGS = {name: ["-ftz=true", "-prec-div=false", "-prec-sqrt=false"] for name in ("chunk_scan.cu", "chunk_scan_ws.cu", "pside.cu", "hola_tc.cu")}
 
 
 def _nvcc() -> str:

@@ -288,6 +288,7 @@ cudaError_t launch_dv(int dv, const HolaArgs& p, int BH, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_hola_read(int dk, int dv, const HolaArgs& p, int BH, cudaStream_t stream) {
+  if (hola_tc_supported(dk, dv, p.in_dtype, p.block)) return launch_hola_read_tc(p, BH, stream);
   switch (dk) {
     case 16: return launch_dv<16>(dv, p, BH, stream);
     case 32: return launch_dv<32>(dv, p, BH, stream);

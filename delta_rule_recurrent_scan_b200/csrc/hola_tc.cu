@@ -1,0 +1,351 @@
+// Surprise-cache read on the sm_100a tensor cores: bf16 q, k, v with d_k = d_v = 128, blocks of 64.
+//
+// The read of A Hippocampus for Linear Attention, section 3.4, Eq. (7): token t of block b takes a
+// softmax, temperature 1, over the top-w cache of blocks 0..b-1 (by surprise m, section 3.3), the causal
+// tokens of its own block and a null sink.  With q~ = q / rms(q) * gamma_q and k~ = k / rms(k) * gamma_k,
+//
+//   q~_t . k~_j = rq_t rk_j sum_d (q_td gamma_q,d gamma_k,d) k_jd,
+//
+// so the keys enter the product raw (exact bf16) and only the queries, scaled by gamma_q gamma_k, are
+// split into bf16 hi + lo.  Per block, with the 128 keys (64 cache rows, then 64 block rows) on the TMEM
+// lanes:
+//
+//   S^T = K [q o gamma]^T        M = 128 keys, N = 64 queries, K = 128      (2 MMAs per K step)
+//   softmax over the keys of each query column (warp butterflies, then the four lane quarters), sink
+//   O^T = V^T P                  M = 128 (d_v), N = 64 queries, K = 128 keys (P as bf16 hi + lo)
+//
+// The cache lives in two ping-pong buffers of 128 key / value rows: block b reads buffer b & 1 (cache in
+// rows 0..63, its own tokens in rows 64..127) and merges the best w candidates into rows 0..63 of the
+// other buffer (rank = number of candidates with a larger m, ties towards the earlier token).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace kdn {
+
+namespace {
+
+using chunk::kWaitCycles;
+using chunk::store8_split;
+
+constexpr int kTThreads = 256;
+constexpr int kD = 128;
+constexpr int kNP = kD / 64;                // 64-wide panels across d
+constexpr int kRows = 128;                  // key / value rows of a buffer: 64 cache + 64 block
+constexpr int kPanel = kRows * 128;         // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
+constexpr int kBuf = kNP * kPanel;          // 32 KB
+constexpr int kQPanel = 64 * 128;           // 8 KB: 64 query rows x 64 bf16
+constexpr int OFF_K = 0;                    // 2 x kBuf raw keys
+constexpr int OFF_V = OFF_K + 2 * kBuf;     // 2 x kBuf values
+constexpr int OFF_H = OFF_V + 2 * kBuf;     // scaled queries hi (kNP x kQPanel), then P hi (one kPanel)
+constexpr int OFF_L = OFF_H + kPanel;       // scaled queries lo, then P lo
+constexpr int kTotal = OFF_L + kPanel;
+constexpr int kSmem = kTotal + 1024;
+constexpr uint32_t T_S = 0, T_O = 64, kTmemCols = 128;
+static_assert(kNP * kQPanel == kPanel, "query panels and the P panel share a region");
+
+// Max (kind 0) or sum (kind 1) over the warp's 32 lanes for each of 32 values: afterwards lane l holds
+// the result for value index l.
+template <int KIND>
+__device__ __forceinline__ float butterfly(float (&x)[32], int lane) {
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = up ? x[i] : x[i + k];
+      const float keep = up ? x[i + k] : x[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, k);
+      x[i] = KIND == 0 ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return x[0];
+}
+
+__device__ __forceinline__ bool before(float mc, int ic, float md, int id) { return mc > md || (mc == md && ic < id); }
+
+__global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ float rk[2][kRows];     // 1 / rms(k) per buffer row
+  __shared__ float mcs[2][kRows];    // m per buffer row (-inf = empty)
+  __shared__ int ics[2][kRows];      // token index per buffer row (-1 = empty)
+  __shared__ float rq[64];
+  __shared__ float gqk[kD];          // gamma_q * gamma_k
+  __shared__ float red[4][64];
+  __shared__ float mxs[64], inv_den[64];
+  __shared__ int newpos[kRows];
+  __shared__ int ncache;
+  __shared__ uint64_t bar_mma;
+  __shared__ uint32_t tmem_base;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qw = warp & 3, half = warp >> 2;
+  const int bh = blockIdx.x, h = bh % p.H;
+  const int L = p.L, w = p.w;
+  const size_t tok0 = (size_t)bh * L;
+  const float sink = p.sink[h];
+  const float inv_sqrt_d = rsqrtf((float)kD);
+  const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+
+  for (int e = tid; e < 2 * kRows; e += kTThreads) {
+    mcs[e / kRows][e % kRows] = -INFINITY, ics[e / kRows][e % kRows] = -1, rk[e / kRows][e % kRows] = 0.f;
+  }
+  if (tid < kD) gqk[tid] = p.gamma_q[tid] * p.gamma_k[tid];
+  // both buffers start as zeros: empty cache rows meet probability 0 and must stay finite
+  for (int e = tid; e < (4 * kBuf) / 16; e += kTThreads) reinterpret_cast<uint4*>(sm + OFF_K)[e] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    ncache = 0;
+    sm100::mbar_init(&bar_mma, 1);
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0) {
+    sm100::tmem_alloc(&tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  uint32_t phase = 0;
+  bool aborted = false;
+  const uint32_t qh = sm100::smem_u32(sm + OFF_H), ql = sm100::smem_u32(sm + OFF_L);
+
+  int nblocks = 0;
+  for (int b0 = 0; b0 < L; b0 += 64, ++nblocks) {
+    const int X = nblocks & 1, Y = X ^ 1;
+    const int nb = min(64, L - b0);
+    uint8_t* KB = sm + OFF_K + X * kBuf;
+    uint8_t* VB = sm + OFF_V + X * kBuf;
+
+    // ---------------------------------------------------------------- block tokens: raw k, v rows; scaled q hi/lo
+    {
+      const int i = tid >> 2, part = tid & 3;   // token, quarter of its 16 chunks
+      const bool valid = i < nb;
+      const size_t t = tok0 + b0 + i;
+      const uint8_t* kg = reinterpret_cast<const uint8_t*>(p.k) + t * (kD * 2);
+      const uint8_t* vg = reinterpret_cast<const uint8_t*>(p.v) + t * (kD * 2);
+      const uint8_t* qg = reinterpret_cast<const uint8_t*>(p.q) + t * (kD * 2);
+      float kss = 0.f, qss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = 4 * part + u;             // chunk: elements 8 c .. 8 c + 7
+        uint4 kc = make_uint4(0, 0, 0, 0), vc = kc, qc = kc;
+        if (valid) {
+          kc = *reinterpret_cast<const uint4*>(kg + 16 * c);
+          vc = *reinterpret_cast<const uint4*>(vg + 16 * c);
+          qc = *reinterpret_cast<const uint4*>(qg + 16 * c);
+        }
+        const uint32_t off = (c / 8) * kPanel + sm100::sw128_chunk(64 + i, c % 8);
+        *reinterpret_cast<uint4*>(KB + off) = kc;
+        *reinterpret_cast<uint4*>(VB + off) = vc;
+        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kc);
+        const __nv_bfloat162* qh2 = reinterpret_cast<const __nv_bfloat162*>(&qc);
+        float qs[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __bfloat1622float2(kh[e]), qf = __bfloat1622float2(qh2[e]);
+          kss = fmaf(kf.x, kf.x, fmaf(kf.y, kf.y, kss));
+          qss = fmaf(qf.x, qf.x, fmaf(qf.y, qf.y, qss));
+          qs[2 * e] = qf.x * gqk[8 * c + 2 * e];
+          qs[2 * e + 1] = qf.y * gqk[8 * c + 2 * e + 1];
+        }
+        store8_split(sm + OFF_H, sm + OFF_L, (c / 8) * kQPanel + sm100::sw128_chunk(i, c % 8), qs);
+      }
+      kss += __shfl_xor_sync(0xffffffffu, kss, 1);
+      kss += __shfl_xor_sync(0xffffffffu, kss, 2);
+      qss += __shfl_xor_sync(0xffffffffu, qss, 1);
+      qss += __shfl_xor_sync(0xffffffffu, qss, 2);
+      if (part == 0) {
+        rk[X][64 + i] = valid ? rsqrtf(kss / kD + 1e-6f) : 0.f;
+        rq[i] = rsqrtf(qss / kD + 1e-6f);
+        mcs[X][64 + i] = valid ? p.m[t] : -INFINITY;
+        ics[X][64 + i] = valid ? b0 + i : -1;
+      }
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- S^T = K [q o gamma]^T
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, false);
+      const uint32_t kb = sm100::smem_u32(KB);
+#pragma unroll
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint64_t a = sm100::smem_desc(kb + (ks / 4) * kPanel + (ks % 4) * 32, 16, 1024);
+        const uint32_t boff = (ks / 4) * kQPanel + (ks % 4) * 32;
+        sm100::mma_bf16(tmem + T_S, a, sm100::smem_desc(qh + boff, 16, 1024), id, ks > 0);
+        sm100::mma_bf16(tmem + T_S, a, sm100::smem_desc(ql + boff, 16, 1024), id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    {
+      int bad = 0;
+      if (tid == 0) bad = !sm100::mbar_wait_bounded(&bar_mma, phase, kWaitCycles);
+      bad = __syncthreads_or(bad);
+      if (bad) {
+        if (tid == 0) raise_status(p.status, kStatusTimeout);
+        aborted = true;
+        break;
+      }
+      sm100::tc_fence_after();
+      phase ^= 1;
+    }
+
+    // ---------------------------------------------------------------- softmax over the keys (lanes) of each query
+    const int j = 32 * qw + lane;             // key row
+    float x[32];
+    {
+      float s[32];
+      sm100::tmem_ld32(tmem + t_lane + T_S + 32 * half, s);
+      sm100::tmem_wait_ld();
+      const float kscale = rk[X][j] * inv_sqrt_d;
+      const int nc = ncache;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int t = 32 * half + u;
+        const bool vis = j < 64 ? j < nc : (j - 64 <= t && j - 64 < nb);
+        x[u] = vis ? s[u] * kscale * rq[t] : -INFINITY;
+        s[u] = x[u];
+      }
+      red[qw][32 * half + lane] = butterfly<0>(s, lane);
+    }
+    __syncthreads();
+    if (tid < 64) mxs[tid] = fmaxf(fmaxf(fmaxf(red[0][tid], red[1][tid]), fmaxf(red[2][tid], red[3][tid])), sink);
+    __syncthreads();
+    {
+      float s[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        x[u] = __expf(x[u] - mxs[32 * half + u]);  // exp(-inf) = 0 for hidden keys
+        s[u] = x[u];
+      }
+      red[qw][32 * half + lane] = butterfly<1>(s, lane);
+    }
+    __syncthreads();
+    if (tid < 64) inv_den[tid] = 1.f / (red[0][tid] + red[1][tid] + red[2][tid] + red[3][tid] + __expf(sink - mxs[tid]));
+    __syncthreads();
+    // P (key rows, query columns) as bf16 hi / lo over the query panels, which the S product no longer reads
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8) {
+      float pv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pv[e] = x[8 * q8 + e] * inv_den[32 * half + 8 * q8 + e];
+      store8_split(sm + OFF_H, sm + OFF_L, sm100::sw128_chunk(j, 4 * half + q8), pv);
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- O^T = V^T P
+    if (tid == 0) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, 64, true, true);
+      const uint32_t vb = sm100::smem_u32(VB);
+#pragma unroll
+      for (int ks = 0; ks < kRows / 16; ++ks) {
+        const uint64_t a = sm100::smem_desc(vb + ks * 2048, kPanel, 1024);
+        sm100::mma_bf16(tmem + T_O, a, sm100::smem_desc(qh + ks * 2048, kPanel, 1024), id, ks > 0);
+        sm100::mma_bf16(tmem + T_O, a, sm100::smem_desc(ql + ks * 2048, kPanel, 1024), id, true);
+      }
+      sm100::mma_commit(&bar_mma);
+    }
+    // meanwhile: rank every candidate for the merged cache
+    if (tid < kRows) {
+      const float m0 = mcs[X][tid];
+      const int i0 = ics[X][tid];
+      int rank = 0;
+      for (int c = 0; c < kRows; ++c) rank += (ics[X][c] >= 0 && c != tid && before(mcs[X][c], ics[X][c], m0, i0)) ? 1 : 0;
+      newpos[tid] = (i0 >= 0 && rank < w) ? rank : -1;
+    }
+    {
+      int bad = 0;
+      if (tid == 0) bad = !sm100::mbar_wait_bounded(&bar_mma, phase, kWaitCycles);
+      bad = __syncthreads_or(bad);
+      if (bad) {
+        if (tid == 0) raise_status(p.status, kStatusTimeout);
+        aborted = true;
+        break;
+      }
+      sm100::tc_fence_after();
+      phase ^= 1;
+    }
+    {
+      float o[32];
+      sm100::tmem_ld32(tmem + t_lane + T_O + 32 * half, o);
+      sm100::tmem_wait_ld();
+      const int dv = j;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int t = 32 * half + u;
+        if (t < nb) p.o[(tok0 + b0 + t) * kD + dv] = o[u];
+      }
+    }
+
+    // ---------------------------------------------------------------- merge into rows 0..63 of the other buffer
+    if (tid < 64) mcs[Y][tid] = -INFINITY, ics[Y][tid] = -1;
+    {
+      uint8_t* KY = sm + OFF_K + Y * kBuf;
+      uint8_t* VY = sm + OFF_V + Y * kBuf;
+      for (int e = tid; e < kRows * 2 * 2 * kNP * 8 / 2; e += kTThreads) {   // rows x (key, value) x 16 chunks
+        const int c = e >> 5, q = e & 31;
+        const int np = newpos[c];
+        if (np < 0) continue;
+        const int which = q >> 4, cc = q & 15;
+        const uint8_t* src = (which ? VB : KB) + (cc / 8) * kPanel + sm100::sw128_chunk(c, cc % 8);
+        uint8_t* dst = (which ? VY : KY) + (cc / 8) * kPanel + sm100::sw128_chunk(np, cc % 8);
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      }
+    }
+    __syncthreads();
+    if (tid < kRows && newpos[tid] >= 0) {
+      const int np = newpos[tid];
+      mcs[Y][np] = mcs[X][tid], ics[Y][np] = ics[X][tid], rk[Y][np] = rk[X][tid];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int n = 0;
+      for (int c = 0; c < 64; ++c) n += ics[Y][c] >= 0 ? 1 : 0;
+      ncache = n;
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+  }
+
+  // ---------------------------------------------------------------- the final cache's token indices, ascending
+  if (!aborted && p.cache != nullptr && tid < w) {
+    const int F = nblocks & 1;
+    const int mine = tid < 64 ? ics[F][tid] : -1;
+    if (mine >= 0) {
+      int pos = 0;
+      for (int c = 0; c < 64; ++c) pos += (ics[F][c] >= 0 && ics[F][c] < mine) ? 1 : 0;
+      p.cache[(size_t)bh * w + pos] = mine;
+    }
+    if (tid >= ncache) p.cache[(size_t)bh * w + tid] = -1;
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) sm100::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+bool hola_tc_supported(int dk, int dv, int in_dtype, int block) {
+  return dk == kD && dv == kD && in_dtype == kBF16 && block == 64;
+}
+
+cudaError_t launch_hola_read_tc(const HolaArgs& p, int BH, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(hola_read_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  hola_read_tc_kernel<<<BH, kTThreads, kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kdn

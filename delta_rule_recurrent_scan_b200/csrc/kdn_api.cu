@@ -296,7 +296,7 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
 
 kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* m,
                                const float* gamma_q, const float* gamma_k, const float* sink, int w, float* o_cache,
-                               int* cache_idx, void* stream) {
+                               int* cache_idx, void* workspace, size_t workspace_bytes, void* stream) {
   KDN_TRY(check_dims(dims));
   if (w < 1 || w > 64) return fail(KDN_ERR_UNSUPPORTED, "w must be in 1..64");
   const int block = dims->chunk == 0 ? 64 : dims->chunk;
@@ -310,14 +310,19 @@ kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* 
   KDN_TRY(check_ptr(gamma_k, "gamma_k", 4, false));
   KDN_TRY(check_ptr(sink, "sink", 4, false));
   KDN_TRY(check_ptr(cache_idx, "cache_idx", 4, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  if (workspace_bytes < kStatusBytes) return fail(KDN_ERR_INVALID_ARG, "workspace_bytes < 256");
   KDN_TRY(use_device_of(gamma_q));
   const int BH = dims->B * dims->H;
   cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "clearing the status word");
   if (!any) {
     if (cache_idx == nullptr) return ok();
     return cuda_status(cudaMemsetAsync(cache_idx, 0xff, (size_t)BH * w * sizeof(int), st), "clearing cache_idx");
   }
-  kdn::HolaArgs ha{q, k, v, dims->in_dtype, m, gamma_q, gamma_k, sink, o_cache, cache_idx, dims->H, dims->L, block, w};
+  kdn::HolaArgs ha{q, k, v, dims->in_dtype, m, gamma_q, gamma_k, sink, o_cache, cache_idx, dims->H, dims->L, block, w,
+                   reinterpret_cast<unsigned*>(workspace)};
   return cuda_status(kdn::launch_hola_read(dims->dk, dims->dv, ha, BH, st), "surprise-cache read launch");
 }
 

@@ -87,10 +87,14 @@ struct HolaArgs {
   int L;
   int block;              // 16, 32 or 64
   int w;                  // 1..64
+  unsigned* status;       // device status word (bounded-wait timeouts)
 };
 
 cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream);
 cudaError_t launch_hola_read(int dk, int dv, const HolaArgs& args, int BH, cudaStream_t stream);
+// tensor-core variant (bf16, d_k = d_v = 128, blocks of 64); launch_hola_read picks it when it applies
+bool hola_tc_supported(int dk, int dv, int in_dtype, int block);
+cudaError_t launch_hola_read_tc(const HolaArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_iso_beta(int dk, const IsoArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream);
 cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream);

@@ -63,7 +63,7 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_kalman_full.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_diag.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
     L.kdn_scan_kalman_iso.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, sz, vp]
-    L.kdn_hola_cache_read.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp]
+    L.kdn_hola_cache_read.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.kdn_decode_step.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.argtypes = [dims, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
     L.kdn_scan_kalman_full_noalloc.restype = ctypes.c_int
@@ -273,7 +273,8 @@ def scan_kalman_iso(q, k, v, r, a=None, qn=None, S=None, c=None, o=None, m=None,
     return o, m, S, c
 
 
-def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, cache=None, stream=None):
+def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, cache=None, workspace=None,
+                    stream=None):
     """Surprise-cache read: q, k [B,H,L,d_k], v [B,H,L,d_v] (bf16 or fp32), m [B,H,L], gamma_q/gamma_k [d_k],
     sink [H].  Returns (o_cache [B,H,L,d_v] fp32, cache [B,H,w] int32 token indices, ascending, -1 empty)."""
     if q.dim() != 4:
@@ -294,9 +295,12 @@ def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, 
     if cache is None:
         cache = torch.empty(B, H, w, dtype=torch.int32, device=dev)
     _need(cache, "cache", (B, H, w), torch.int32, dev)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
     dims = Dims(B, H, L, dk, dv, block, _DTYPES[q.dtype], KDN_F32)
     st = lib().kdn_hola_cache_read(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(gamma_q),
-                                   _ptr(gamma_k), _ptr(sink), int(w), _ptr(o), _ptr(cache), _stream(stream))
+                                   _ptr(gamma_k), _ptr(sink), int(w), _ptr(o), _ptr(cache), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
     _check(st, "kdn_hola_cache_read")
     return o, cache
 

@@ -148,10 +148,12 @@ KDN_EXPORT kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, c
  * 1 <= w <= 64.  Out: o_cache [B,H,L,d_v] fp32; cache_idx [B,H,w] int32 token
  * indices of the final cache, ascending, -1 for empty slots, or NULL.  The
  * state-read gate that mixes o_cache into the layer output is the caller's.
- * Needs no workspace. */
+ * workspace: >= 256 bytes (the device status word, read with
+ * kdn_read_device_status). */
 KDN_EXPORT kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v,
                                const float* m, const float* gamma_q, const float* gamma_k, const float* sink,
-                               int w, float* o_cache, int* cache_idx, void* stream);
+                               int w, float* o_cache, int* cache_idx, void* workspace, size_t workspace_bytes,
+                               void* stream);
 
 /* kdn_scan_kalman_full for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a deployment variant.  Callers that must
