@@ -20,6 +20,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "chunk.h"
 #include "chunk_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -43,7 +44,8 @@ constexpr int OFF_K = 0;                    // 2 x kBuf raw keys
 constexpr int OFF_V = OFF_K + 2 * kBuf;     // 2 x kBuf values
 constexpr int OFF_H = OFF_V + 2 * kBuf;     // scaled queries hi (kNP x kQPanel), then P hi (one kPanel)
 constexpr int OFF_L = OFF_H + kPanel;       // scaled queries lo, then P lo
-constexpr int kTotal = OFF_L + kPanel;
+constexpr int OFF_QS = OFF_L + kPanel;      // raw queries of the next block (TMA staging), kNP x kQPanel
+constexpr int kTotal = OFF_QS + kNP * kQPanel;
 constexpr int kSmem = kTotal + 1024;
 constexpr uint32_t T_S = 0, T_O = 64, kTmemCols = 128;
 static_assert(kNP * kQPanel == kPanel, "query panels and the P panel share a region");
@@ -68,7 +70,9 @@ __device__ __forceinline__ float butterfly(float (&x)[32], int lane) {
 
 __device__ __forceinline__ bool before(float mc, int ic, float md, int id) { return mc > md || (mc == md && ic < id); }
 
-__global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) {
+__global__ void __launch_bounds__(kTThreads, 1)
+    hola_read_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, HolaArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ float rk[2][kRows];     // 1 / rms(k) per buffer row
@@ -79,8 +83,9 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
   __shared__ float red[4][64];
   __shared__ float mxs[64], inv_den[64];
   __shared__ int newpos[kRows];
+  __shared__ int rank_part[2][kRows];
   __shared__ int ncache;
-  __shared__ uint64_t bar_mma;
+  __shared__ uint64_t bar_mma, bar_load;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -98,9 +103,23 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
   if (tid < kD) gqk[tid] = p.gamma_q[tid] * p.gamma_k[tid];
   // both buffers start as zeros: empty cache rows meet probability 0 and must stay finite
   for (int e = tid; e < (4 * kBuf) / 16; e += kTThreads) reinterpret_cast<uint4*>(sm + OFF_K)[e] = make_uint4(0, 0, 0, 0);
+  // TMA of one block's raw k, v (rows 64..127 of a buffer) and q (staging): six 64 x 64 boxes
+  auto issue_block = [&](int bb, int buf) {
+    sm100::mbar_arrive_expect_tx(&bar_load, 3 * kNP * 64 * 128);
+#pragma unroll
+    for (int pn = 0; pn < kNP; ++pn) {
+      sm100::tma_load_3d(sm + OFF_K + buf * kBuf + pn * kPanel + 64 * 128, &tm_k, &bar_load, 64 * pn, bb, bh);
+      sm100::tma_load_3d(sm + OFF_V + buf * kBuf + pn * kPanel + 64 * 128, &tm_v, &bar_load, 64 * pn, bb, bh);
+      sm100::tma_load_3d(sm + OFF_QS + pn * kQPanel, &tm_q, &bar_load, 64 * pn, bb, bh);
+    }
+  };
   if (tid == 0) {
     ncache = 0;
+    sm100::prefetch_tmap(&tm_q);
+    sm100::prefetch_tmap(&tm_k);
+    sm100::prefetch_tmap(&tm_v);
     sm100::mbar_init(&bar_mma, 1);
+    sm100::mbar_init(&bar_load, 1);
     sm100::fence_mbar_init();
   }
   if (warp == 0) {
@@ -111,8 +130,12 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = tmem_base;
-  uint32_t phase = 0;
+  uint32_t phase = 0, lphase = 0;
   bool aborted = false;
+  if (tid == 0 && L > 0) {
+    sm100::fence_async_smem();  // the zeroed buffers precede the first copy in
+    issue_block(0, 0);
+  }
   const uint32_t qh = sm100::smem_u32(sm + OFF_H), ql = sm100::smem_u32(sm + OFF_L);
 
   int nblocks = 0;
@@ -122,27 +145,28 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
     uint8_t* KB = sm + OFF_K + X * kBuf;
     uint8_t* VB = sm + OFF_V + X * kBuf;
 
-    // ---------------------------------------------------------------- block tokens: raw k, v rows; scaled q hi/lo
+    // ---------------------------------------------------------------- block tokens: scales of k, scaled q hi/lo
+    {
+      int bad = 0;
+      if (tid == 0) bad = !sm100::mbar_wait_bounded(&bar_load, lphase, kWaitCycles);
+      bad = __syncthreads_or(bad);
+      if (bad) {
+        if (tid == 0) raise_status(p.status, kStatusTimeout);
+        aborted = true;
+        break;
+      }
+      lphase ^= 1;
+    }
     {
       const int i = tid >> 2, part = tid & 3;   // token, quarter of its 16 chunks
       const bool valid = i < nb;
-      const size_t t = tok0 + b0 + i;
-      const uint8_t* kg = reinterpret_cast<const uint8_t*>(p.k) + t * (kD * 2);
-      const uint8_t* vg = reinterpret_cast<const uint8_t*>(p.v) + t * (kD * 2);
-      const uint8_t* qg = reinterpret_cast<const uint8_t*>(p.q) + t * (kD * 2);
       float kss = 0.f, qss = 0.f;
+      const float mt = valid ? p.m[tok0 + b0 + i] : -INFINITY;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = 4 * part + u;             // chunk: elements 8 c .. 8 c + 7
-        uint4 kc = make_uint4(0, 0, 0, 0), vc = kc, qc = kc;
-        if (valid) {
-          kc = *reinterpret_cast<const uint4*>(kg + 16 * c);
-          vc = *reinterpret_cast<const uint4*>(vg + 16 * c);
-          qc = *reinterpret_cast<const uint4*>(qg + 16 * c);
-        }
-        const uint32_t off = (c / 8) * kPanel + sm100::sw128_chunk(64 + i, c % 8);
-        *reinterpret_cast<uint4*>(KB + off) = kc;
-        *reinterpret_cast<uint4*>(VB + off) = vc;
+        const uint4 kc = *reinterpret_cast<const uint4*>(KB + (c / 8) * kPanel + sm100::sw128_chunk(64 + i, c % 8));
+        const uint4 qc = *reinterpret_cast<const uint4*>(sm + OFF_QS + (c / 8) * kQPanel + sm100::sw128_chunk(i, c % 8));
         const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kc);
         const __nv_bfloat162* qh2 = reinterpret_cast<const __nv_bfloat162*>(&qc);
         float qs[8];
@@ -163,7 +187,7 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
       if (part == 0) {
         rk[X][64 + i] = valid ? rsqrtf(kss / kD + 1e-6f) : 0.f;
         rq[i] = rsqrtf(qss / kD + 1e-6f);
-        mcs[X][64 + i] = valid ? p.m[t] : -INFINITY;
+        mcs[X][64 + i] = mt;
         ics[X][64 + i] = valid ? b0 + i : -1;
       }
     }
@@ -173,6 +197,7 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
     sm100::tc_fence_after();
 
     // ---------------------------------------------------------------- S^T = K [q o gamma]^T
+    if (tid == 0 && b0 + 64 < L) issue_block(b0 + 64, Y);  // rows 64.. of the other buffer and the staging are free
     if (tid == 0) {
       constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, false);
       const uint32_t kb = sm100::smem_u32(KB);
@@ -256,13 +281,15 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
       }
       sm100::mma_commit(&bar_mma);
     }
-    // meanwhile: rank every candidate for the merged cache
-    if (tid < kRows) {
-      const float m0 = mcs[X][tid];
-      const int i0 = ics[X][tid];
+    // meanwhile: rank every candidate for the merged cache (two threads per candidate, half the others each)
+    {
+      const int cand = tid & (kRows - 1), hf = tid >> 7;
+      const float m0 = mcs[X][cand];
+      const int i0 = ics[X][cand];
       int rank = 0;
-      for (int c = 0; c < kRows; ++c) rank += (ics[X][c] >= 0 && c != tid && before(mcs[X][c], ics[X][c], m0, i0)) ? 1 : 0;
-      newpos[tid] = (i0 >= 0 && rank < w) ? rank : -1;
+      for (int c = 64 * hf; c < 64 * hf + 64; ++c)
+        rank += (ics[X][c] >= 0 && c != cand && before(mcs[X][c], ics[X][c], m0, i0)) ? 1 : 0;
+      rank_part[hf][cand] = rank;
     }
     {
       int bad = 0;
@@ -275,6 +302,10 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
       }
       sm100::tc_fence_after();
       phase ^= 1;
+    }
+    if (tid < kRows) {
+      const int rank = rank_part[0][tid] + rank_part[1][tid];
+      newpos[tid] = (ics[X][tid] >= 0 && rank < w) ? rank : -1;
     }
     {
       float o[32];
@@ -290,6 +321,7 @@ __global__ void __launch_bounds__(kTThreads, 1) hola_read_tc_kernel(HolaArgs p) 
 
     // ---------------------------------------------------------------- merge into rows 0..63 of the other buffer
     if (tid < 64) mcs[Y][tid] = -INFINITY, ics[Y][tid] = -1;
+    __syncthreads();  // newpos complete
     {
       uint8_t* KY = sm + OFF_K + Y * kBuf;
       uint8_t* VY = sm + OFF_V + Y * kBuf;
@@ -342,9 +374,13 @@ bool hola_tc_supported(int dk, int dv, int in_dtype, int block) {
 }
 
 cudaError_t launch_hola_read_tc(const HolaArgs& p, int BH, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_bf16_tmap(&tq, p.q, BH, p.L, kD) || !make_bf16_tmap(&tk, p.k, BH, p.L, kD) ||
+      !make_bf16_tmap(&tv, p.v, BH, p.L, kD))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(hola_read_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  hola_read_tc_kernel<<<BH, kTThreads, kSmem, stream>>>(p);
+  hola_read_tc_kernel<<<BH, kTThreads, kSmem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
