@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // S0^T pairs for the next [K; Q] product and the master pre-scaled by the next chunk's A_C:
     // x = S[64 half + 32 v .. + 31][j]
-    auto emit_state = [&](float (&x)[32], int v, float scale) {
+    // x = S[dk0 .. dk0 + 31][j]
+    auto emit_state = [&](float (&x)[32], int dk0, float scale) {
       float hw[16], lw[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -267,12 +268,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm100::split2_bf16(x[2 * e], x[2 * e + 1], hu, lu);
         hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
       }
-      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 32 * half + 16 * v, hw);
-      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 64 + 32 * half + 16 * v, lw);
+      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + dk0 / 2, hw);
+      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 64 + dk0 / 2, lw);
 #pragma unroll
       for (int e = 0; e < 32; ++e) x[e] *= scale;
-      sm100::tmem_st32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
+      sm100::tmem_st32(tmem + t_lane + Lay::T_SM + dk0, x);
     };
+    // D2^T = S0^T [K; Q]^T, K steps 4 part .. 4 part + 3 (d_k 64 part ..): issued as soon as that half of
+    // the S0^T pairs is in tensor memory; the second half commits
+    auto issue_d2 = [&](uint32_t kq_addr, int part) {
+      constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int ks = 4 * part + u;
+        const uint64_t b = sm100::smem_desc(kq_addr + (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32, 16, 1024);
+        sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 8 * ks, b, id, ks > 0);
+        sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 64 + 8 * ks, b, id, true);
+      }
+      if (part == 1) sm100::mma_commit(&bar_c);
+    };
+    auto kq_addr_of = [&](int cc) { return sm100::smem_u32(sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES); };
 
     // Diagonal variances of chunk cc (threads 0..D-1, coordinate i = tid; independent of v and S), run one
     // chunk ahead while the chain waits for the preparation.  Per coordinate: p^- = a^2 p + Qn,
@@ -325,22 +340,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) sm100::mbar_arrive(&var_done[0]);
       }
     }
-    if (aborted || (!kChainGates && !gwait(&gates_ready[0], 0))) {
+    if (aborted || (!kChainGates && !gwait(&gates_ready[0], 0)) || !gwait(&kq_full[0], 0)) {
       aborted = true;
     } else {
       const float AC0 = Aex[0][kC - 1];
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
         float x[32];
+        const int dk0 = 32 * half + 64 * v;
 #pragma unroll
-        for (int u = 0; u < 32; ++u) x[u] = Sg[(size_t)(64 * half + 32 * v + u) * D + j];
-        emit_state(x, v, AC0);
+        for (int u = 0; u < 32; ++u) x[u] = Sg[(size_t)(dk0 + u) * D + j];
+        emit_state(x, dk0, AC0);
+        sm100::tmem_wait_st();
+        sm100::tc_fence_before();
+        named_sync(kBarChain, kGroup);
+        sm100::tc_fence_after();
+        if (leader) issue_d2(kq_addr_of(0), v);
       }
-      sm100::tmem_wait_st();
     }
-    sm100::tc_fence_before();
-    named_sync(kBarChain, kGroup);
-    sm100::tc_fence_after();
 
     const uint32_t tat_hi = sm100::smem_u32(TAThi), tat_lo = sm100::smem_u32(TATlo);
     for (int c = 0; c < nchunks && !aborted; ++c) {
@@ -348,25 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t0 = c * kC;
       const uint32_t kq0 = sm100::smem_u32(sm + Lay::OFF_KQ + kslot * Lay::KQ_BYTES);
 
-      // ---------------------------------------------------------------- D2^T = S0^T [K; Q]^T
-      if (!gwait(&kq_full[kslot], (c / NKQ) & 1)) { aborted = true; break; }
-      if (leader) {
-        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t b = sm100::smem_desc(kq0 + (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32, 16, 1024);
-          sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 8 * ks, b, id, ks > 0);
-          sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 64 + 8 * ks, b, id, true);
-        }
-        sm100::mma_commit(&bar_c);
-      }
+      // D2^T = S0^T [K; Q]^T of this chunk was issued with its state operands (end of the previous chunk)
 
       // ---------------------------------------------------------------- R^T = V^T - (K S0)^T diag(A), in place
+      // V and the gates first: the column of V this thread needs is read while the S0 product runs
       {
         bool bad = false;
         if (leader) {
-          bad = !sm100::mbar_wait_bounded(&bar_c, ph_c, kWaitCycles) ||
-                !sm100::mbar_wait_bounded(&v_full, c & 1, kWaitCycles) ||
+          bad = !sm100::mbar_wait_bounded(&v_full, c & 1, kWaitCycles) ||
                 !sm100::mbar_wait_bounded(&gates_ready[s], (c >> 1) & 1, kWaitCycles);
         }
         bad = named_sync_or(kBarChain, kGroup, bad);
@@ -375,14 +381,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
-        sm100::tc_fence_after();
-        ph_c ^= 1;
       }
       {
+        const uint8_t* vp = Vs + (j / 64) * Lay::V_PANEL;
+        uint32_t vv[16];  // V[t][j] for the 32 tokens of this half, as bf16 pairs (t even in the low half)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int t = 32 * half + 2 * e;
+          const uint32_t v0 = *reinterpret_cast<const uint16_t*>(vp + sm100::sw128(t, j % 64));
+          const uint32_t v1 = *reinterpret_cast<const uint16_t*>(vp + sm100::sw128(t + 1, j % 64));
+          vv[e] = v0 | (v1 << 16);
+        }
+        if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
+        ph_c ^= 1;
         float X[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + 32 * half, X);
         sm100::tmem_wait_ld();
-        const uint8_t* vp = Vs + (j / 64) * Lay::V_PANEL;
         const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
         float hw[16], lw[16];
 #pragma unroll
@@ -392,9 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int e = 2 * e4 + e2;
-            const int t = 32 * half + 2 * e;
-            const float v0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vp + sm100::sw128(t, j % 64)));
-            const float v1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vp + sm100::sw128(t + 1, j % 64)));
+            const float v0 = __uint_as_float(vv[e] << 16), v1 = __uint_as_float(vv[e] & 0xffff0000u);
             uint32_t hu, lu;
             sm100::split2_bf16(fmaf(-aa[2 * e2], X[2 * e], v0), fmaf(-aa[2 * e2 + 1], X[2 * e + 1], v1), hu, lu);
             hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
@@ -439,9 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
       ph_c ^= 1;
 
-      // ---------------------------------------------------------------- E' pairs, ||e||^2, O
+      // ---------------------------------------------------------------- E' pairs; S^T master += E'^T G; ||e||^2
+      float E[32];
       {
-        float E[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_SA + 32 * half, E);
         sm100::tmem_wait_ld();
         const float4* S4 = reinterpret_cast<const float4*>(&esc[s][32 * half]);
@@ -457,28 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);
         sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half + 16, lw);
-        // sum of E^2 over this warp's 32 lanes for each of the 32 tokens: after the butterfly,
-        // lane l holds token 32 half + l
-#pragma unroll
-        for (int u = 0; u < 32; ++u) E[u] *= E[u];
-#pragma unroll
-        for (int k = 16; k >= 1; k >>= 1) {
-          const bool up = (lane & k) != 0;
-#pragma unroll
-          for (int i = 0; i < k; ++i) {
-            const float send = up ? E[i] : E[i + k];
-            const float keep = up ? E[i + k] : E[i];
-            E[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
-          }
-        }
-        en[qw][32 * half + lane] = E[0];
       }
       sm100::tmem_wait_st();
       sm100::tc_fence_before();
       named_sync(kBarChain, kGroup);
       sm100::tc_fence_after();
-
-      // ---------------------------------------------------------------- S^T master += E'^T G
       if (leader) {
         constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, true);
 #pragma unroll
@@ -500,6 +495,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm100::mma_commit(&bar_c);
       }
+      // sum of E^2 over this warp's 32 lanes for each of the 32 tokens, while the state product runs: after
+      // the butterfly lane l holds token 32 half + l
+#pragma unroll
+      for (int u = 0; u < 32; ++u) E[u] *= E[u];
+#pragma unroll
+      for (int k = 16; k >= 1; k >>= 1) {
+        const bool up = (lane & k) != 0;
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+          const float send = up ? E[i] : E[i + k];
+          const float keep = up ? E[i + k] : E[i];
+          E[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+      }
+      en[qw][32 * half + lane] = E[0];
       // O = diag(A) Q S0 + AT R, while the state product runs (it touches neither column range)
       {
         const bool full = t0 + kC <= L;
@@ -533,27 +543,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!gwait(&bar_c, ph_c)) { aborted = true; break; }  // also: every lane quarter's norms are in
+      ph_c ^= 1;
       if (tid < kC && P.m != nullptr && t0 + tid < L)
         P.m[(size_t)bh * L + t0 + tid] = sqrtf(gn[s][tid]) * sqrtf(en[0][tid] + en[1][tid] + en[2][tid] + en[3][tid]);
-      if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
-      ph_c ^= 1;
 
-      // ---------------------------------------------------------------- state operands of the next chunk
+      // ---------------------------------------------------------------- state operands of the next chunk, and its
+      // S0 product, a half at a time
       if (c + 1 < nchunks) {
         if (!kChainGates && !gwait(&gates_ready[s ^ 1], ((c + 1) >> 1) & 1)) { aborted = true; break; }
+        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
         const float ACn = Aex[s ^ 1][kC - 1];
+        const uint32_t kq_next = kq_addr_of(c + 1);
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
           float x[32];
-          sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
+          const int dk0 = 32 * half + 64 * v;
+          sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + dk0, x);
           sm100::tmem_wait_ld();
-          emit_state(x, v, ACn);
+          emit_state(x, dk0, ACn);
+          sm100::tmem_wait_st();
+          sm100::tc_fence_before();
+          named_sync(kBarChain, kGroup);
+          sm100::tc_fence_after();
+          if (leader) issue_d2(kq_next, v);
         }
-        sm100::tmem_wait_st();
+      } else {
+        sm100::tc_fence_before();
+        named_sync(kBarChain, kGroup);
+        sm100::tc_fence_after();
       }
-      sm100::tc_fence_before();
-      named_sync(kBarChain, kGroup);
-      sm100::tc_fence_after();
       if (leader) {
         sm100::mbar_arrive(&chain_done[s]);
         if (c + NKQ < nchunks) issue_kq(c + NKQ);  // this slot's K, Q are dead
