@@ -382,6 +382,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
       }
+      // ---------------------------------------------------------------- variances of chunk c + 1, while the S0 product runs
+      if (kChainGates && c + 1 < nchunks) {
+        // its scalars were stored before gates_ready of chunk c, its K before the slot's load completed
+        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
+        run_variances(c + 1);
+        if (gw == 4) run_gates(c + 1);
+        named_sync(kBarChain, kGroup);
+        if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
+      }
+
       {
         const uint8_t* vp = Vs + (j / 64) * Lay::V_PANEL;
         uint32_t vv[16];  // V[t][j] for the 32 tokens of this half, as bf16 pairs (t even in the low half)
@@ -420,16 +430,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_sync(kBarChain, kGroup);
       sm100::tc_fence_after();
       if (leader && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
-
-      // ---------------------------------------------------------------- variances of chunk c + 1
-      if (kChainGates && c + 1 < nchunks) {
-        // its scalars were stored before gates_ready of chunk c, its K before the slot's load completed
-        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
-        run_variances(c + 1);
-        if (gw == 4) run_gates(c + 1);
-        named_sync(kBarChain, kGroup);
-        if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
-      }
 
       // ---------------------------------------------------------------- D3^T = R^T [T; AT]^T
       if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
