@@ -81,11 +81,11 @@ _WS_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/chunk_scan_ws.cu",
                "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
                "delta_rule_recurrent_scan_b200/csrc/sm100.cuh"]
 NCU_TRAFFIC = {
-    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "39b1537fb07afebd68394982e597811441d83d3c",
-                         "bytes_per_token": (205.706496e6 + 103.683840e6) / (2 * 16 * 8192),
+    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "ede10530cbb47eeea928d574215cca12a76714e9",
+                         "bytes_per_token": (205.816576e6 + 104.452608e6) / (2 * 16 * 8192),
                          "capture": "profiles/chunk_scan_ws_kernel_kalman_diag_d128.md (B=2 case, scaled)"},
-    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "39b1537fb07afebd68394982e597811441d83d3c",
-                 "bytes_per_token": (205.632256e6 + 104.837632e6) / (2 * 16 * 8192),
+    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "ede10530cbb47eeea928d574215cca12a76714e9",
+                 "bytes_per_token": (205.635072e6 + 104.847872e6) / (2 * 16 * 8192),
                  "capture": "profiles/chunk_scan_ws_kernel_delta_d128.md (B=2 case, scaled)"},
 }
 

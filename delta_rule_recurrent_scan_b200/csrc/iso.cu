@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(kIsoThreads) iso_beta_kernel(IsoArgs p) {
   if (tid == 0) c_carry = p.c[bh];
 
   for (int t0 = 0; t0 < L; t0 += kIsoTile) {
-    // ---- ||k_t||^2 for the tile: LPT lanes per token, 16-byte loads
+    // ---- ||k_t||^2 for the tile: LPT lanes per token, 16-byte loads, several tokens in flight per warp
+#pragma unroll 8
     for (int tb = warp * TPL; tb < kIsoTile; tb += (kIsoThreads / 32) * TPL) {
       const int t = tb + lane / LPT;
       float s = 0.f;
