@@ -8,14 +8,18 @@
 //   delta  g = beta k
 //   diag   p^- = a^2 p + Qn, s = sum p^- k^2 + r, g = p^- k / s,
 //          p <- p^- r / (r + p^- k^2)
+//   iso    c^- = a^2 c + Qn, g = c^- k / (c^- ||k||^2 + r), c <- d_k c^- r / (d_k r + c^- ||k||^2)
 //   e = v - a S^T k,  o = a S^T q + (g . q) e,  S <- a S + g e^T,  m = ||g|| ||e||
 #include "common.cuh"
 #include "kernels.h"
 
 namespace kdn {
 
-template <int DK, int DV, bool kDiag>
+enum DecodeMode : int { kDecDelta = 0, kDecDiag = 1, kDecIso = 2 };
+
+template <int DK, int DV, int MODE>
 __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) decode_kernel(DecodeArgs args) {
+  constexpr bool kDiag = MODE == kDecDiag;
   using Lay = RowBlockLayout<DK, DV>;
   constexpr int NT = Lay::kThreads, CG = Lay::kColGroups, RG = Lay::kRowGroups, RPT = Lay::kRowsPerThread;
   constexpr int DVW = (DV + 31) / 32 * 32;
@@ -64,6 +68,26 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) decode_kerne
         g[i] = pp[i] * kk[i] * inv_s;
         if (c < DK) args.p[(size_t)bh * DK + c] = pp[i] * r / fmaf(pp[i] * kk[i], kk[i], r);
       }
+    } else if constexpr (MODE == kDecIso) {
+      // one uncertainty scalar per head, kept in the p slot
+      const float r = args.r[bh];
+      float kk = 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int c = lane + 32 * i;
+        const float kv = c < DK ? k_s[c] : 0.f;
+        kk = fmaf(kv, kv, kk);
+      }
+      kk = warp_sum(kk);
+      const float cm = fmaf(a * a, args.p[bh], args.qn_scalar);
+      const float beta = cm / fmaf(cm, kk, r);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int c = lane + 32 * i;
+        g[i] = c < DK ? beta * k_s[c] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) args.p[bh] = DK * cm * r / fmaf((float)DK, r, cm * kk);
     } else {
       const float beta = args.beta[bh];
 #pragma unroll
@@ -143,14 +167,16 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) decode_kerne
     default: return cudaErrorInvalidValue;    \
   }
 
-cudaError_t launch_decode(int dk, int dv, bool diag, const DecodeArgs& args, cudaStream_t stream) {
+cudaError_t launch_decode(int dk, int dv, int mode, const DecodeArgs& args, cudaStream_t stream) {
   if (args.BH <= 0) return cudaSuccess;
   KDN_DEC_SWITCH(dk, DK, KDN_DEC_SWITCH(dv, DV, {
     constexpr int NT = RowBlockLayout<DK, DV>::kThreads;
-    if (diag)
-      decode_kernel<DK, DV, true><<<args.BH, NT, 0, stream>>>(args);
+    if (mode == kDecDiag)
+      decode_kernel<DK, DV, kDecDiag><<<args.BH, NT, 0, stream>>>(args);
+    else if (mode == kDecIso)
+      decode_kernel<DK, DV, kDecIso><<<args.BH, NT, 0, stream>>>(args);
     else
-      decode_kernel<DK, DV, false><<<args.BH, NT, 0, stream>>>(args);
+      decode_kernel<DK, DV, kDecDelta><<<args.BH, NT, 0, stream>>>(args);
   }));
   return cudaGetLastError();
 }

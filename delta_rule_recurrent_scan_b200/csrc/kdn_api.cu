@@ -329,8 +329,8 @@ kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* 
 kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype, kdn_dtype out_dtype,
                            const void* q, const void* k, const void* v, const float* beta, const float* a,
                            const float* r, float qn_scalar, float* S, float* p, void* o, float* m, void* stream) {
-  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG)
-    return fail(KDN_ERR_UNSUPPORTED, "decode supports KDN_DELTA and KDN_KALMAN_DIAG");
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_ISO)
+    return fail(KDN_ERR_UNSUPPORTED, "decode supports KDN_DELTA, KDN_KALMAN_DIAG and KDN_KALMAN_ISO");
   kdn_dims d{B, H, 1, dk, dv, 0, in_dtype, out_dtype};
   KDN_TRY(check_dims(&d));
   KDN_TRY(check_ptr(q, "q", 16, false));
@@ -349,8 +349,8 @@ kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kd
   }
   KDN_TRY(use_device_of(S));
   kdn::DecodeArgs args{q, k, v, in_dtype, out_dtype, beta, a, r, qn_scalar, S, p, o, m, B * H};
-  return cuda_status(kdn::launch_decode(dk, dv, variant == KDN_KALMAN_DIAG, args, (cudaStream_t)stream),
-                     "decode launch");
+  const int mode = variant == KDN_KALMAN_DIAG ? 1 : variant == KDN_KALMAN_ISO ? 2 : 0;
+  return cuda_status(kdn::launch_decode(dk, dv, mode, args, (cudaStream_t)stream), "decode launch");
 }
 
 }  // extern "C"

@@ -51,7 +51,7 @@ struct DecodeArgs {
   const float* r;     // diagonal: [BH]
   float qn_scalar;
   float* S;           // [BH, dk, dv]
-  float* p;           // diagonal: [BH, dk]
+  float* p;           // diagonal: [BH, dk]; isotropic: c, [BH]
   void* o;            // [BH, dv]
   float* m;           // [BH] or nullptr
   int BH;
@@ -98,6 +98,7 @@ cudaError_t launch_hola_read_tc(const HolaArgs& args, int BH, cudaStream_t strea
 cudaError_t launch_iso_beta(int dk, const IsoArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_kalman_full_gains(int dk, const GainArgs& args, cudaStream_t stream);
 cudaError_t launch_kalman_diag_gains(int dk, const GainArgs& args, cudaStream_t stream);
-cudaError_t launch_decode(int dk, int dv, bool diag, const DecodeArgs& args, cudaStream_t stream);
+// mode: 0 delta, 1 diagonal Kalman (p = [BH, dk]), 2 isotropic Kalman (p = c, [BH])
+cudaError_t launch_decode(int dk, int dv, int mode, const DecodeArgs& args, cudaStream_t stream);
 
 }  // namespace kdn

@@ -307,8 +307,8 @@ def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, 
 
 def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=0.0, p=None, o=None, m=None, out_dtype=None,
                 stream=None):
-    """One token per head against a resident state.  q, k [B,H,d_k], v [B,H,d_v]; S (and p) updated in place.
-    Returns (o, m)."""
+    """One token per head against a resident state.  q, k [B,H,d_k], v [B,H,d_v]; S (and p: the diagonal
+    variances [B,H,d_k], or for "kalman_iso" the uncertainty scalar [B,H]) updated in place.  Returns (o, m)."""
     if q.dim() != 3:
         raise ValueError("q must be [B, H, d_k]")
     B, H, dk = q.shape
@@ -328,8 +328,8 @@ def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=0.0, p=None, 
     for name, t in (("beta", beta), ("a", a), ("r", r)):
         if t is not None:
             _need(t, name, (B, H), torch.float32, dev)
-    if p is not None:
-        _need(p, "p", (B, H, dk), torch.float32, dev)
+    if p is not None:  # diagonal: p [B,H,d_k]; isotropic: the uncertainty scalar c [B,H]
+        _need(p, "p", (B, H) if variant == "kalman_iso" else (B, H, dk), torch.float32, dev)
     st = lib().kdn_decode_step(VARIANTS[variant], B, H, dk, dv, _DTYPES[q.dtype], _DTYPES[out_dtype], _ptr(q), _ptr(k),
                                _ptr(v), _ptr(beta), _ptr(a), _ptr(r), float(qn), _ptr(S), _ptr(p), _ptr(o), _ptr(m),
                                _stream(stream))

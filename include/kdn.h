@@ -180,9 +180,10 @@ KDN_EXPORT kdn_status kdn_scan_kalman_full_noalloc(const kdn_dims* dims, const v
 
 /* One recurrent token per head against a resident state (constant-memory
  * decoding: Kalman Delta Networks, Abstract).  variant: KDN_DELTA (beta
- * required, p ignored) or KDN_KALMAN_DIAG (r and p required).  q, k [B,H,d_k],
- * v [B,H,d_v], scalars [B,H], o [B,H,d_v], m [B,H] or NULL; S [B,H,d_k,d_v]
- * and p [B,H,d_k] in/out.  Needs no workspace. */
+ * required, p ignored), KDN_KALMAN_DIAG (r and p [B,H,d_k] required) or
+ * KDN_KALMAN_ISO (r required; p is the uncertainty scalar c, [B,H]).  q, k
+ * [B,H,d_k], v [B,H,d_v], scalars [B,H], o [B,H,d_v], m [B,H] or NULL;
+ * S [B,H,d_k,d_v] and p in/out.  Needs no workspace. */
 KDN_EXPORT kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kdn_dtype in_dtype,
                            kdn_dtype out_dtype, const void* q, const void* k, const void* v,
                            const float* beta, const float* a, const float* r, float qn_scalar,

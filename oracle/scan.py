@@ -367,8 +367,9 @@ def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=None, p=None)
 
     Kalman Delta Networks, Abstract (constant-memory decoding with a fixed-size
     recurrent memory).  q, k [..., d_k]; v [..., d_v]; beta, a, r [...] or None;
-    qn a scalar, [...] or None; S [..., d_k, d_v]; p [..., d_k] (diagonal only).
-    ``variant`` is "delta" or "kalman_diag".  Returns o [..., d_v], m [...],
+    qn a scalar, [...] or None; S [..., d_k, d_v]; p [..., d_k] (diagonal) or the
+    uncertainty scalar [...] (isotropic).  ``variant`` is "delta", "kalman_diag" or
+    "kalman_iso".  Returns o [..., d_v], m [...],
     S and (diagonal) p after the token.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -387,4 +388,8 @@ def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=None, p=None)
         qn_t = None if qn is None else (np.broadcast_to(_f64(qn), lead)[..., None])
         res = scan_kalman_diag(tokvec(q), tokvec(k), tokvec(v), tok(r), a=tok(a), qn=qn_t, S0=S, p0=p)
         return {"o": res["o"][..., 0, :], "m": res["m"][..., 0], "S": res["S"], "p": res["p"]}
+    if variant == "kalman_iso":  # p is the uncertainty scalar c [...]
+        qn_t = None if qn is None else (np.broadcast_to(_f64(qn), lead)[..., None])
+        res = scan_kalman_iso(tokvec(q), tokvec(k), tokvec(v), tok(r), a=tok(a), qn=qn_t, S0=S, c0=p)
+        return {"o": res["o"][..., 0, :], "m": res["m"][..., 0], "S": res["S"], "p": res["c"]}
     raise ValueError(f"unknown decode variant {variant!r}")

@@ -186,7 +186,7 @@ def test_full_size_sampled_heads(name):
 # ----------------------------------------------------------------------------- decode
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_iso"])
 def test_decode_steps_equal_scan_and_oracle(variant):
     name = "decode_delta" if variant == "delta" else "decode_diag"
     w = WORKLOADS[name]
@@ -207,8 +207,10 @@ def test_decode_steps_equal_scan_and_oracle(variant):
     assert normwise_err(S, scan["S"]) < SELF_TOL
     ref = run_oracle(variant, xs)
     compare({"o": o, "m": torch.stack(ms, dim=2), "S": S}, ref, TOL["bf16"])
-    if C is not None and variant == "kalman_diag":
+    if variant == "kalman_diag":
         compare({"p": C}, {"p": ref["p"]}, TOL["bf16"])
+    if variant == "kalman_iso":
+        compare({"c": C}, {"c": ref["c"]}, TOL["bf16"])
 
 
 @pytest.mark.parametrize("name", ["decode_delta", "decode_diag"])

@@ -459,7 +459,7 @@ def test_iso_is_the_delta_rule_with_a_variance_driven_beta():
 # ----------------------------------------------------------------------------- decode
 
 
-@pytest.mark.parametrize("variant", ["delta", "kalman_diag"])
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_iso"])
 def test_n_decode_steps_equal_a_scan(variant):
     rng, q, k, v = _case(15, 12, 6, 4, heads=(2, 3))
     beta = rng.random((2, 3, 12))
@@ -467,10 +467,12 @@ def test_n_decode_steps_equal_a_scan(variant):
     r = 0.1 + rng.random((2, 3, 12))
     if variant == "delta":
         ref = scan_delta(q, k, v, beta, a=a)
-    else:
+    elif variant == "kalman_diag":
         ref = scan_kalman_diag(q, k, v, r=r, a=a, qn=1e-3)
+    else:
+        ref = scan_kalman_iso(q, k, v, r=r, a=a, qn=1e-3)
     S = np.zeros((2, 3, 6, 4))
-    p = np.ones((2, 3, 6))
+    p = np.ones((2, 3)) if variant == "kalman_iso" else np.ones((2, 3, 6))
     for t in range(12):
         st = decode_step(variant, q[..., t, :], k[..., t, :], v[..., t, :], S, beta=beta[..., t], a=a[..., t],
                          r=r[..., t], qn=1e-3, p=p)
