@@ -31,6 +31,7 @@
 #include "chunk.h"
 #include "chunk_common.cuh"
 #include "common.cuh"
+#include "mobius.cuh"
 #include "sm100.cuh"
 
 namespace kdn {
@@ -45,7 +46,11 @@ using chunk::named_sync_or;
 using chunk::oct_sum;
 using chunk::store8_split;
 
-enum Var : int { kDelta = 0, kDiag = 1, kFull = 2 };
+enum Var : int { kDelta = 0, kDiag = 1, kFull = 2, kIso = 3 };
+
+// Gains of the form beta_t k_t (the delta rule, and the isotropic Kalman filter whose beta_t the
+// preparation computes from its one uncertainty scalar per head).
+constexpr bool delta_like(int var) { return var == kDelta || var == kIso; }
 
 constexpr int D = 128;
 constexpr int NP = D / 64;                 // 64-wide panels across d
@@ -58,11 +63,11 @@ template <int VAR>
 struct WsLayout {
   static constexpr int KQ_PANEL = 128 * 128;             // [K; Q]: 128 rows x 64 bf16
   static constexpr int KQ_BYTES = NP * KQ_PANEL;
-  static constexpr int NKQ = (VAR == kDelta) ? 3 : 2;    // [K; Q] tiles in flight
+  static constexpr int NKQ = delta_like(VAR) ? 3 : 2;    // [K; Q] tiles in flight
   static constexpr int V_PANEL = 64 * 128;
   static constexpr int V_BYTES = NP * V_PANEL;
   static constexpr int G_PANEL = 64 * 128;
-  static constexpr int G_HALF = (VAR == kDelta) ? 0 : NP * G_PANEL;  // hi or lo of one gain slot
+  static constexpr int G_HALF = delta_like(VAR) ? 0 : NP * G_PANEL;  // hi or lo of one gain slot
   static constexpr int TAT_HALF = 128 * 128;             // [T; AT]: 128 rows x 64 bf16, hi or lo
   static constexpr int SCR_BYTES = 64 * chunk::kLD * 4;  // fp32 [64][68]
 
@@ -74,7 +79,7 @@ struct WsLayout {
   static constexpr int OFF_TF = OFF_NF + SCR_BYTES;
   static constexpr int TOTAL = OFF_TF + SCR_BYTES;
   static constexpr int SMEM = TOTAL + 1024;              // + alignment slack
-  static_assert(VAR == kDelta || 64 * D * 4 == 2 * G_HALF, "a gain slot holds the fp32 gains before their split");
+  static_assert(delta_like(VAR) || 64 * D * 4 == 2 * G_HALF, "a gain slot holds the fp32 gains before their split");
   static_assert(TOTAL <= 216 * 1024, "shared memory budget");
 
   // TMEM columns
@@ -94,7 +99,7 @@ struct Params {
   float qn_scalar;
   const float* gains;  // full Kalman: [BH, L, D] fp32
   float* S;
-  float* p;            // diag: [BH, D]
+  float* p;            // diag: [BH, D]; isotropic: the uncertainty scalar c, [BH]
   void* o;
   float* m;
   int out_dtype;
@@ -142,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float esc[2][kC];                // scale of row t of E in the state update:
                                                             // A_C / A_t (times beta_t for the delta rule)
   __shared__ float en[4][kC];                               // ||e_t||^2 partials per lane quarter
+  __shared__ float knorm[kC];                               // isotropic: ||k_t||^2 of the chunk
   __shared__ uint64_t kq_full[NKQ], v_full, bar_c, bar_p, tat_free;
   __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2], var_done[2];
   __shared__ uint32_t tmem_base;
@@ -232,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ell[sl][lane] = x0, ell[sl][32 + lane] = x1;
     Aex[sl][lane] = __expf(x0), Aex[sl][32 + lane] = __expf(x1);
     const float r0 = __expf(lC - x0), r1 = __expf(lC - x1);  // A_C / A_t without a division
-    esc[sl][lane] = VAR == kDelta ? r0 * sB[sl][lane] : r0;
-    esc[sl][32 + lane] = VAR == kDelta ? r1 * sB[sl][32 + lane] : r1;
+    esc[sl][lane] = delta_like(VAR) ? r0 * sB[sl][lane] : r0;
+    esc[sl][32 + lane] = delta_like(VAR) ? r1 * sB[sl][32 + lane] : r1;
   };
   fetch_scalars(0);
   store_scalars(0);
@@ -480,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks, false);
           const uint32_t al = tmem + Lay::T_D2 + tok_pair_col(ks, true);
-          if (VAR == kDelta) {
+          if (delta_like(VAR)) {
             const uint64_t bk = sm100::smem_desc(kq0 + ks * 2048, Lay::KQ_PANEL, 1024);
             sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bk, id, true);
             sm100::mma_bf16_ts(tmem + Lay::T_SM, al, bk, id, true);
@@ -595,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = pt == 0;             // issues the preparation's products
     bool aborted = false;
     uint32_t ph_p = 0;
+    float c_iso = VAR == kIso ? P.p[bh] : 0.f;  // isotropic: the uncertainty scalar, carried by the gates warp
 
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1, kslot = c % NKQ;
@@ -616,6 +623,59 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) raise_status(P.status, kStatusTimeout);
           aborted = true;
           break;
+        }
+      }
+      // ---------------------------------------------------------------- isotropic: beta of this chunk
+      if (VAR == kIso) {
+        // ||k_t||^2 (eight threads per token, two passes of 32 tokens)
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          const int t = 32 * pass + (pt >> 3), part = pt & 7;
+          float sq = 0.f;
+#pragma unroll
+          for (int pn = 0; pn < NP; ++pn) {
+            float xk[8];
+            load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sq = fmaf(xk[e], xk[e], sq);
+          }
+          sq = oct_sum(sq);
+          if (part == 0) knorm[t] = sq;
+        }
+        named_sync(kBarPrep, kGroup);
+        if (gw == 4) {
+          // The uncertainty scalar's token maps (Kalman Delta Networks, Abstract: Moebius maps, scanned
+          // associatively): two tokens per lane, an inclusive scan over the lanes, then each lane steps its
+          // two tokens exactly from the carried value and writes beta_t over r_t.
+          mobius::Mob mine = mobius::identity();
+          float a2[2], qv[2], rv[2], kk[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = 2 * lane + u;
+            a2[u] = sA[s][t] * sA[s][t], qv[u] = sQ[s][t], rv[u] = sB[s][t], kk[u] = knorm[t];
+            mine = mobius::compose(mobius::iso_token(a2[u], qv[u], kk[u] / (D * rv[u])), mine);
+          }
+          mobius::Mob incl = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const mobius::Mob left = mobius::shfl_up(incl, o);
+            if (lane >= o) incl = mobius::compose(incl, left);
+          }
+          mobius::Mob excl = mobius::shfl_up(incl, 1);
+          if (lane == 0) excl = mobius::identity();
+          float cv = mobius::apply(excl, c_iso);
+          bool bad = false;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const float cm = fmaf(a2[u], cv, qv[u]);
+            const float sden = fmaf(cm, kk[u], rv[u]);
+            bad |= !(sden > 0.f && isfinite(sden) && cm >= 0.f);
+            sB[s][2 * lane + u] = cm / sden;
+            cv = D * cm * rv[u] / fmaf((float)D, rv[u], cm * kk[u]);
+          }
+          if (bad && t0 + 2 * lane < L) raise_status(P.status, kStatusNumeric);
+          c_iso = __shfl_sync(0xffffffffu, cv, 31);
+          __syncwarp();
         }
       }
       // ---------------------------------------------------------------- gates | diagonal variances
@@ -657,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) kv[8 * pn + e] = xk[e];
           }
-          if (VAR == kDelta) {
+          if (delta_like(VAR)) {
             float sq = 0.f;
 #pragma unroll
             for (int e = 0; e < kGD; ++e) sq = fmaf(kv[e], kv[e], sq);
@@ -702,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (part == 0) gn[s][t] = n2;
           }
         }
-        if (VAR != kDelta) {
+        if (!delta_like(VAR)) {
           if (VAR == kDiag) named_sync(kBarPrep, kGroup);
 #pragma unroll
           for (int pass = 0; pass < 2; ++pass) {
@@ -730,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
           const uint64_t a = sm100::smem_desc(kq0 + koff, 16, 1024);
-          if (VAR == kDelta) {
+          if (delta_like(VAR)) {
             sm100::mma_bf16(tmem + Lay::T_D1, a, a, id1, ks > 0);  // G = K (beta enters with Gam)
           } else {
             const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
@@ -770,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int jj = 32 * half + e + u;
-              v4[u] = (jj < i) ? Y[e + u] * __expf(li - ell[s][jj]) * (VAR == kDelta ? sB[s][jj] : 1.f) : 0.f;
+              v4[u] = (jj < i) ? Y[e + u] * __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f) : 0.f;
             }
             *reinterpret_cast<float4*>(Nf + i * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
           }
@@ -783,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int jj = 32 * half + 8 * q8 + e;
-              xa[e] = (jj <= i) ? Y[8 * q8 + e] * __expf(li - ell[s][jj]) * (VAR == kDelta ? sB[s][jj] : 1.f) : 0.f;
+              xa[e] = (jj <= i) ? Y[8 * q8 + e] * __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f) : 0.f;
             }
             store8_split(TAThi, TATlo, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
           }
@@ -858,6 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::tc_fence_after();
       if (leader) sm100::mbar_arrive(&prep_done[s]);
     }
+    if (VAR == kIso && !aborted && gw == 4 && lane == 0) P.p[bh] = c_iso;
   }
 
   sm100::tc_fence_before();
@@ -888,6 +949,10 @@ cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& d, const ChunkA
   p.beta = a.beta, p.a = a.a, p.r = a.r, p.qn = a.qn, p.qn_scalar = a.qn_scalar, p.gains = gains;
   p.S = a.S, p.o = a.o, p.m = a.m, p.out_dtype = a.out_dtype, p.L = a.L, p.status = a.status;
   if (variant == KDN_KALMAN_FULL) return launch_ws_typed<kFull>(tq, tk, tv, p, a.BH, stream);
+  if (variant == KDN_KALMAN_ISO) {
+    p.p = a.P;  // the uncertainty scalar c, [BH]
+    return launch_ws_typed<kIso>(tq, tk, tv, p, a.BH, stream);
+  }
   if (variant == KDN_KALMAN_DIAG) {
     p.p = a.P;
     return launch_ws_typed<kDiag>(tq, tk, tv, p, a.BH, stream);

@@ -17,12 +17,13 @@
 // tokens, a block-wide exclusive scan of those 2x2 products (warp shuffles, then one warp over the warp
 // totals) gives every thread the map from the tile's start to its first token, and each thread then steps
 // its four tokens exactly, writing beta_t.  Products are renormalised so that the lower-right entry is 1
-// (the map is projective), which keeps every entry of a product of non-negative maps in range.
+// (the map is projective).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mobius.cuh"
 
 namespace kdn {
 
@@ -32,32 +33,10 @@ constexpr int kIsoThreads = 512;
 constexpr int kIsoPer = 4;                           // tokens per thread per tile
 constexpr int kIsoTile = kIsoThreads * kIsoPer;      // 2048 tokens
 
-struct Mob {
-  float a, b, c, d;  // [[a, b], [c, d]], d normalised to 1 after every product
-};
-
-// later o earlier (apply `earlier` first), renormalised
-__device__ __forceinline__ Mob compose(const Mob& later, const Mob& earlier) {
-  Mob m;
-  m.a = fmaf(later.a, earlier.a, later.b * earlier.c);
-  m.b = fmaf(later.a, earlier.b, later.b * earlier.d);
-  m.c = fmaf(later.c, earlier.a, later.d * earlier.c);
-  m.d = fmaf(later.c, earlier.b, later.d * earlier.d);
-  const float inv = 1.f / m.d;
-  m.a *= inv, m.b *= inv, m.c *= inv, m.d = 1.f;
-  return m;
-}
-
-__device__ __forceinline__ Mob shfl_up(const Mob& m, int delta) {
-  Mob r;
-  r.a = __shfl_up_sync(0xffffffffu, m.a, delta);
-  r.b = __shfl_up_sync(0xffffffffu, m.b, delta);
-  r.c = __shfl_up_sync(0xffffffffu, m.c, delta);
-  r.d = __shfl_up_sync(0xffffffffu, m.d, delta);
-  return r;
-}
-
-__device__ __forceinline__ Mob identity() { return Mob{1.f, 0.f, 0.f, 1.f}; }
+using mobius::Mob;
+using mobius::compose;
+using mobius::identity;
+using mobius::shfl_up;
 
 template <int DK, bool BF16>
 __global__ void __launch_bounds__(kIsoThreads) iso_beta_kernel(IsoArgs p) {
@@ -118,7 +97,7 @@ __global__ void __launch_bounds__(kIsoThreads) iso_beta_kernel(IsoArgs p) {
       rv[u] = valid ? p.r[ti] : 1.f;
       kk[u] = valid ? knorm[t] : 0.f;
       const float w = kk[u] / (DK * rv[u]);
-      const Mob mt{a2[u], qv[u], w * a2[u], fmaf(w, qv[u], 1.f)};
+      const Mob mt = mobius::iso_token(a2[u], qv[u], w);
       mine = compose(mt, mine);
     }
 

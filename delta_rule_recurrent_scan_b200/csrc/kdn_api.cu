@@ -171,7 +171,8 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
   } else {
     n = 2, name = "seq_scan_kernel";
   }
-  if (variant == KDN_KALMAN_ISO && n > 0) n += 1;
+  if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128))
+    n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself)
   if (launches) *launches = n;
   if (kernel) *kernel = name;
   if (arith) *arith = ar;
@@ -280,6 +281,13 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
   if (!any) return ok();
   const int BH = dims->B * dims->H;
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  if (kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128) {
+    // the d = 128 chunk kernel runs the uncertainty scan in its own preparation: one launch
+    kdn::ChunkArgs ch{};
+    ch.q = q, ch.k = k, ch.v = v, ch.a = a, ch.r = r, ch.qn = qn, ch.qn_scalar = qn_scalar, ch.P = c;
+    ch.S = S, ch.o = o, ch.m = m, ch.out_dtype = dims->out_dtype, ch.BH = BH, ch.L = dims->L, ch.status = status;
+    return cuda_status(kdn::launch_chunk(KDN_KALMAN_ISO, *dims, ch, st), "chunked isotropic scan launch");
+  }
   float* beta = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + kStatusBytes);
   kdn::IsoArgs ia{k, dims->in_dtype, a, r, qn, qn_scalar, c, beta, status, dims->L};
   e = kdn::launch_iso_beta(dims->dk, ia, BH, st);
