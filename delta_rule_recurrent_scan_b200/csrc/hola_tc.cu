@@ -303,9 +303,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
       sm100::tc_fence_after();
       phase ^= 1;
     }
+    int kept = 0;
     if (tid < kRows) {
       const int rank = rank_part[0][tid] + rank_part[1][tid];
-      newpos[tid] = (ics[X][tid] >= 0 && rank < w) ? rank : -1;
+      kept = (ics[X][tid] >= 0 && rank < w) ? 1 : 0;
+      newpos[tid] = kept ? rank : -1;
     }
     {
       float o[32];
@@ -320,8 +322,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
 
     // ---------------------------------------------------------------- merge into rows 0..63 of the other buffer
-    if (tid < 64) mcs[Y][tid] = -INFINITY, ics[Y][tid] = -1;
-    __syncthreads();  // newpos complete
+    const int n_kept = __syncthreads_count(kept);  // also: newpos complete; the kept rows are 0 .. n_kept - 1
     {
       uint8_t* KY = sm + OFF_K + Y * kBuf;
       uint8_t* VY = sm + OFF_V + Y * kBuf;
@@ -335,17 +336,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
       }
     }
-    __syncthreads();
     if (tid < kRows && newpos[tid] >= 0) {
       const int np = newpos[tid];
       mcs[Y][np] = mcs[X][tid], ics[Y][np] = ics[X][tid], rk[Y][np] = rk[X][tid];
     }
-    __syncthreads();
-    if (tid == 0) {
-      int n = 0;
-      for (int c = 0; c < 64; ++c) n += ics[Y][c] >= 0 ? 1 : 0;
-      ncache = n;
-    }
+    if (tid < 64 && tid >= n_kept) mcs[Y][tid] = -INFINITY, ics[Y][tid] = -1;
+    if (tid == 0) ncache = n_kept;
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
