@@ -46,5 +46,8 @@ cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& dims, const Chu
 bool chunk_supported(kdn_variant variant, const kdn_dims& dims);
 void chunk_plan(kdn_variant variant, const kdn_dims& dims, int* launches, const char** kernel, const char** arith);
 cudaError_t launch_chunk(kdn_variant variant, const kdn_dims& dims, const ChunkArgs& args, cudaStream_t stream);
+// The memory (S) side alone; full Kalman reads its per-token gains from ``gains`` ([BH, L, dk] fp32).
+cudaError_t launch_chunk_sside(kdn_variant variant, const kdn_dims& dims, const ChunkArgs& args, const float* gains,
+                               cudaStream_t stream);
 
 }  // namespace kdn

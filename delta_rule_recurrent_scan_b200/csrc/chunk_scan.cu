@@ -753,6 +753,19 @@ void chunk_plan(kdn_variant variant, const kdn_dims& d, int* launches, const cha
 }
 
 cudaError_t launch_chunk(kdn_variant variant, const kdn_dims& d, const ChunkArgs& a, cudaStream_t stream) {
+  if (variant == KDN_KALMAN_FULL) {
+    // covariance side first (chunked Woodbury / LDL): per-token gains into the workspace, then the S side
+    float* gains = reinterpret_cast<float*>(a.workspace);
+    cudaError_t e = launch_kalman_pside(d.dk, a.k, a.a, a.r, a.qn, a.qn_scalar, a.P, gains, a.status, a.BH, a.L, stream);
+    if (e != cudaSuccess) return e;
+    return launch_chunk_sside(variant, d, a, gains, stream);
+  }
+  return launch_chunk_sside(variant, d, a, nullptr, stream);
+}
+
+cudaError_t launch_chunk_sside(kdn_variant variant, const kdn_dims& d, const ChunkArgs& a, const float* gains,
+                               cudaStream_t stream) {
+  if (d.dk == 128) return launch_chunk_ws(variant, d, a, gains, stream);
   const int BH = a.BH;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_impl(&tq, a.q, BH, a.L, d.dk) || !make_tmap_impl(&tk, a.k, BH, a.L, d.dk) ||
@@ -762,15 +775,10 @@ cudaError_t launch_chunk(kdn_variant variant, const kdn_dims& d, const ChunkArgs
   p.beta = a.beta, p.a = a.a, p.r = a.r, p.qn = a.qn, p.qn_scalar = a.qn_scalar;
   p.S = a.S, p.o = a.o, p.m = a.m, p.out_dtype = a.out_dtype, p.L = a.L, p.status = a.status;
   if (variant == KDN_KALMAN_FULL) {
-    // covariance side first (chunked Woodbury / LDL): per-token gains into the workspace, then the S side
-    float* gains = reinterpret_cast<float*>(a.workspace);
-    cudaError_t e = launch_kalman_pside(d.dk, a.k, a.a, a.r, a.qn, a.qn_scalar, a.P, gains, a.status, BH, a.L, stream);
-    if (e != cudaSuccess) return e;
-    if (d.dk == 128) return launch_chunk_ws(variant, d, a, gains, stream);
+    if (gains == nullptr) return cudaErrorInvalidValue;
     p.gains = gains;
     return launch_typed<64, kFull>(tq, tk, tv, p, BH, stream);
   }
-  if (d.dk == 128) return launch_chunk_ws(variant, d, a, nullptr, stream);
   if (variant == KDN_KALMAN_DIAG) {
     p.p = a.P;
     return launch_typed<64, kDiag>(tq, tk, tv, p, BH, stream);

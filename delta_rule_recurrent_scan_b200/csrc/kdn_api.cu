@@ -92,9 +92,66 @@ kdn_status check_dims(const kdn_dims* d) {
 
 size_t gains_bytes(const kdn_dims* d) { return (size_t)d->B * d->H * (size_t)d->L * d->dk * sizeof(float); }
 
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// ---------------------------------------------------------------- segment-parallel scans
+constexpr int kSegTargetCtas = 148;  // one chunk-kernel CTA per SM of a B200
+
+kdn_variant body_of(kdn_variant var) { return var == KDN_KALMAN_ISO ? KDN_DELTA : var; }
+
+// Segments per head for this request (1 = the serial scan).  An explicit request that cannot be served
+// fails; the library choice never does.
+kdn_status resolve_segments(kdn_variant var, const kdn_dims* d, int* P_out) {
+  *P_out = 1;
+  if (d->segments < 0) return fail(KDN_ERR_INVALID_ARG, "segments must be >= 0");
+  if (d->segments == 1 || d->L == 0) return KDN_OK;
+  const bool chunked = kdn::chunk_supported(body_of(var), *d);
+  if (d->segments >= 2) {
+    if (!chunked) return fail(KDN_ERR_UNSUPPORTED, "segments > 1 needs the chunked path (bf16, dk = dv in {64, 128})");
+    if (d->L % d->segments != 0) return fail(KDN_ERR_INVALID_ARG, "segments must divide L");
+    *P_out = d->segments;
+    return KDN_OK;
+  }
+  if (!chunked) return KDN_OK;
+  const long long BH = (long long)d->B * d->H;
+  for (int P = 16; P >= 4; P /= 2)
+    if (BH * P <= kSegTargetCtas && d->L % (64 * P) == 0 && d->L / (64 * P) >= 2) {
+      *P_out = P;
+      return KDN_OK;
+    }
+  return KDN_OK;
+}
+
+// Byte offsets inside the segment area of the workspace.
+struct SegLayout {
+  size_t sz, si, sc, maps, p[3], end;
+};
+
+SegLayout seg_layout(kdn_variant body, const kdn_dims* d, int P) {
+  SegLayout l{};
+  const size_t V = (size_t)d->B * d->H * P;
+  const size_t states = round256(V * d->dk * d->dv * sizeof(float));
+  l.sz = 0, l.si = states, l.sc = 2 * states, l.end = 3 * states;
+  if (body == KDN_KALMAN_DIAG) {
+    l.maps = l.end, l.end += round256(V * d->dk * 4 * sizeof(float));
+    for (int i = 0; i < 3; ++i) l.p[i] = l.end, l.end += round256(V * d->dk * sizeof(float));
+  }
+  return l;
+}
+
+// Start of the segment area: after the status word and the variant's own scratch.
+size_t seg_area_offset(kdn_variant var, const kdn_dims* d) {
+  size_t n = kStatusBytes;
+  if (var == KDN_KALMAN_DIAG || var == KDN_KALMAN_FULL) n += gains_bytes(d);
+  if (var == KDN_KALMAN_ISO) n += (size_t)d->B * d->H * (size_t)d->L * sizeof(float);
+  return round256(n);
+}
+
 kdn_status common_checks(kdn_variant var, const kdn_dims* d, const void* q, const void* k, const void* v,
                          const float* S, const void* o, const float* m, const void* ws, size_t ws_bytes) {
   KDN_TRY(check_dims(d));
+  int P = 1;
+  KDN_TRY(resolve_segments(var, d, &P));
   const bool any = d->L > 0;
   KDN_TRY(check_ptr(S, "S", 16, false));
   KDN_TRY(check_ptr(q, "q", 16, !any));
@@ -113,6 +170,53 @@ kdn_status common_checks(kdn_variant var, const kdn_dims* d, const void* q, cons
 kdn_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return ok();
   return fail(KDN_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// The memory side over P segments per head (the steps are listed with kdn_dims.segments in kdn.h).
+// ``c`` carries the caller's buffers (c.P: diagonal p); ``gains``: full-Kalman per-token gains.
+kdn_status seg_scan(kdn_variant body, const kdn_dims* d, int P, const kdn::ChunkArgs& c, const float* gains,
+                    char* area, cudaStream_t st) {
+  const int BH = c.BH, D = d->dk;
+  const size_t DD = (size_t)D * d->dv;
+  const SegLayout lay = seg_layout(body, d, P);
+  kdn::SegArgs sa{};
+  sa.P = P, sa.L = c.L, sa.k = c.k, sa.in_dtype = d->in_dtype, sa.a = c.a, sa.r = c.r, sa.qn = c.qn;
+  sa.qn_scalar = c.qn_scalar, sa.p0 = c.P, sa.status = c.status;
+  sa.S = c.S;
+  sa.Sz = reinterpret_cast<float*>(area + lay.sz);
+  sa.SI = reinterpret_cast<float*>(area + lay.si);
+  sa.Sc = reinterpret_cast<float*>(area + lay.sc);
+  const bool diag = body == KDN_KALMAN_DIAG;
+  if (diag) {
+    sa.maps = reinterpret_cast<float4*>(area + lay.maps);
+    for (int i = 0; i < 3; ++i) sa.pcopy[i] = reinterpret_cast<float*>(area + lay.p[i]);
+    sa.ncopy = 3;
+    KDN_TRY(cuda_status(kdn::launch_seg_uncertainty(D, sa, BH, st), "segment uncertainty launch"));
+  }
+  KDN_TRY(cuda_status(kdn::launch_seg_init(D, sa, BH, st), "segment start-state launch"));
+  // every segment as a head of its own: [BH, L, d] viewed as [BH P, L / P, d]
+  kdn_dims dv = *d;
+  dv.B = BH * P, dv.H = 1, dv.L = c.L / P, dv.segments = 1;
+  kdn::ChunkArgs v = c;
+  v.BH = BH * P, v.L = c.L / P;
+  // each segment's map S0 -> M S0 + B: runs from S0 = 0 and S0 = I (o is rewritten below, m not written)
+  v.m = nullptr;
+  v.S = sa.Sz, v.P = diag ? sa.pcopy[0] : c.P;
+  KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
+  v.S = sa.SI, v.P = diag ? sa.pcopy[1] : c.P;
+  KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
+  KDN_TRY(cuda_status(kdn::launch_seg_combine(D, sa, BH, st), "segment chaining launch"));
+  // the true scan of every segment from its start state
+  v.m = c.m;
+  v.S = sa.Sc, v.P = diag ? sa.pcopy[2] : c.P;
+  KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
+  // the last segment's end state (and p) is the head's
+  cudaError_t e = cudaMemcpy2DAsync(c.S, DD * sizeof(float), sa.Sc + (size_t)(P - 1) * DD, P * DD * sizeof(float),
+                                    DD * sizeof(float), BH, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && diag)
+    e = cudaMemcpy2DAsync(c.P, D * sizeof(float), sa.pcopy[2] + (size_t)(P - 1) * D, P * D * sizeof(float),
+                          D * sizeof(float), BH, cudaMemcpyDeviceToDevice, st);
+  return cuda_status(e, "copying the final state");
 }
 
 }  // namespace api
@@ -141,15 +245,13 @@ const char* kdn_last_error(void) { return g_last_error.c_str(); }
 size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
   if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
   if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
-  size_t n = kStatusBytes;
-  switch (variant) {
-    case KDN_DELTA: break;
-    case KDN_KALMAN_DIAG:
-    case KDN_KALMAN_FULL: n += gains_bytes(dims); break;
-    case KDN_KALMAN_ISO: n += (size_t)dims->B * dims->H * (size_t)dims->L * sizeof(float); break;
-    default: return 0;
-  }
-  return (n + 255) / 256 * 256;
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_FULL && variant != KDN_KALMAN_ISO)
+    return 0;
+  int P = 1;
+  if (resolve_segments(variant, dims, &P) != KDN_OK) return 0;
+  size_t n = seg_area_offset(variant, dims);
+  if (P > 1) n += seg_layout(body_of(variant), dims, P).end;
+  return round256(n);
 }
 
 kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, const char** kernel,
@@ -171,8 +273,14 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
   } else {
     n = 2, name = "seq_scan_kernel";
   }
-  if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128))
-    n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself)
+  int nseg = 1;
+  KDN_TRY(resolve_segments(variant, dims, &nseg));
+  if (nseg > 1) {
+    // start states, two map runs, chaining, the true run (+ the diagonal uncertainty maps and starts)
+    n = 5 + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 1 : 0);
+  }
+  if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1))
+    n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself on the serial path)
   if (launches) *launches = n;
   if (kernel) *kernel = name;
   if (arith) *arith = ar;
@@ -208,6 +316,11 @@ kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, co
     c.q = q, c.k = k, c.v = v, c.beta = beta, c.a = a, c.S = S, c.o = o, c.m = m;
     c.out_dtype = dims->out_dtype, c.BH = BH, c.L = dims->L;
     c.status = reinterpret_cast<unsigned*>(workspace);
+    int P = 1;
+    KDN_TRY(resolve_segments(KDN_DELTA, dims, &P));
+    if (P > 1)
+      return seg_scan(KDN_DELTA, dims, P, c, nullptr,
+                      reinterpret_cast<char*>(workspace) + seg_area_offset(KDN_DELTA, dims), st);
     return cuda_status(kdn::launch_chunk(KDN_DELTA, *dims, c, st), "chunked delta scan launch");
   }
   kdn::SeqScanArgs s{q, k, v, dims->in_dtype, dims->out_dtype, beta, a, nullptr, S, o, m, BH, dims->L};
@@ -237,6 +350,18 @@ kdn_status kdn::api::kalman_scan(kdn_variant var, const kdn_dims* dims, const vo
     c.q = q, c.k = k, c.v = v, c.a = a, c.r = r, c.qn = qn, c.qn_scalar = qn_scalar, c.S = S, c.o = o, c.m = m;
     c.P = P, c.out_dtype = dims->out_dtype, c.BH = BH, c.L = dims->L, c.status = status;
     c.workspace = reinterpret_cast<char*>(workspace) + kStatusBytes;
+    int nseg = 1;
+    KDN_TRY(resolve_segments(var, dims, &nseg));
+    if (nseg > 1) {
+      float* gains = nullptr;
+      if (var == KDN_KALMAN_FULL) {
+        // the covariance side is one serial pass per head; its gains fix every segment's memory map
+        gains = reinterpret_cast<float*>(c.workspace);
+        KDN_TRY(cuda_status(kdn::launch_kalman_pside(dims->dk, k, a, r, qn, qn_scalar, P, gains, status, BH, dims->L, st),
+                            "Kalman covariance launch"));
+      }
+      return seg_scan(var, dims, nseg, c, gains, reinterpret_cast<char*>(workspace) + seg_area_offset(var, dims), st);
+    }
     return cuda_status(kdn::launch_chunk(var, *dims, c, st), "chunked Kalman scan launch");
   }
   float* gains = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + kStatusBytes);
@@ -281,7 +406,9 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
   if (!any) return ok();
   const int BH = dims->B * dims->H;
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
-  if (kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128) {
+  int nseg = 1;
+  KDN_TRY(resolve_segments(KDN_KALMAN_ISO, dims, &nseg));
+  if (kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1) {
     // the d = 128 chunk kernel runs the uncertainty scan in its own preparation: one launch
     kdn::ChunkArgs ch{};
     ch.q = q, ch.k = k, ch.v = v, ch.a = a, ch.r = r, ch.qn = qn, ch.qn_scalar = qn_scalar, ch.P = c;
@@ -296,6 +423,9 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
     kdn::ChunkArgs ch{};
     ch.q = q, ch.k = k, ch.v = v, ch.beta = beta, ch.a = a, ch.S = S, ch.o = o, ch.m = m;
     ch.out_dtype = dims->out_dtype, ch.BH = BH, ch.L = dims->L, ch.status = status;
+    if (nseg > 1)
+      return seg_scan(KDN_DELTA, dims, nseg, ch, nullptr,
+                      reinterpret_cast<char*>(workspace) + seg_area_offset(KDN_KALMAN_ISO, dims), st);
     return cuda_status(kdn::launch_chunk(KDN_DELTA, *dims, ch, st), "chunked isotropic scan launch");
   }
   kdn::SeqScanArgs sa{q, k, v, dims->in_dtype, dims->out_dtype, beta, a, nullptr, S, o, m, BH, dims->L};

@@ -90,6 +90,33 @@ struct HolaArgs {
   unsigned* status;       // device status word (bounded-wait timeouts)
 };
 
+// Segment-parallel scan (P segments per head): uncertainty maps and starts, start states, chaining.
+struct SegArgs {
+  int P;                  // segments per head (L % P == 0)
+  int L;                  // tokens per head
+  // diagonal-Kalman uncertainty at the segment starts
+  const void* k;          // [BH, L, dk]
+  int in_dtype;
+  const float* a;         // [BH, L] or nullptr
+  const float* r;         // [BH, L]
+  const float* qn;        // [BH, L] or nullptr
+  float qn_scalar;
+  const float* p0;        // [BH, dk] p before the first token
+  float4* maps;           // [BH P, dk] composed map of each segment (slot P - 1 unused)
+  float* pcopy[3];        // [BH P, dk] each: p at every segment start
+  int ncopy;
+  // memory state
+  const float* S;         // [BH, d, d] the caller's start state
+  float* Sz;              // [BH P, d, d] segment end states from S0 = 0
+  float* SI;              // [BH P, d, d] segment end states from S0 = I
+  float* Sc;              // [BH P, d, d] out: the true start state of every segment
+  unsigned* status;
+};
+
+cudaError_t launch_seg_uncertainty(int dk, const SegArgs& args, int BH, cudaStream_t stream);
+cudaError_t launch_seg_init(int d, const SegArgs& args, int BH, cudaStream_t stream);
+cudaError_t launch_seg_combine(int d, const SegArgs& args, int BH, cudaStream_t stream);
+
 cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_t stream);
 cudaError_t launch_hola_read(int dk, int dv, const HolaArgs& args, int BH, cudaStream_t stream);
 // tensor-core variant (bf16, d_k = d_v = 128, blocks of 64); launch_hola_read picks it when it applies

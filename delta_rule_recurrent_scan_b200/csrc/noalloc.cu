@@ -56,6 +56,10 @@ extern "C" kdn_status kdn_scan_kalman_full_noalloc(const kdn_dims* dims, const v
                                                    float* S, float* P, void* o, float* m, void* stream) {
   kdn_status st = kdn::api::check_dims(dims);
   if (st != KDN_OK) return st;
+  // the static array holds the gains of the serial scan: the library's segment choice is turned off
+  kdn_dims d = *dims;
+  if (d.segments == 0) d.segments = 1;
+  dims = &d;
   const size_t need = kdn_workspace_bytes(KDN_KALMAN_FULL, dims);
   if (need > kNoAllocScratchBytes)
     return kdn::api::fail(KDN_ERR_UNSUPPORTED,

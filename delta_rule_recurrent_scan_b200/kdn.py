@@ -37,7 +37,7 @@ class KdnError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int), ("dk", ctypes.c_int),
                 ("dv", ctypes.c_int), ("chunk", ctypes.c_int), ("in_dtype", ctypes.c_int),
-                ("out_dtype", ctypes.c_int)]
+                ("out_dtype", ctypes.c_int), ("segments", ctypes.c_int)]
 
 
 _lib = None
@@ -117,22 +117,22 @@ def _stream(stream):
 
 
 def workspace_bytes(variant: str, B: int, H: int, L: int, dk: int, dv: int, chunk: int = 0,
-                    in_dtype=torch.bfloat16, out_dtype=None) -> int:
-    d = Dims(B, H, L, dk, dv, chunk, _DTYPES[in_dtype], _DTYPES[out_dtype or torch.float32])
+                    in_dtype=torch.bfloat16, out_dtype=None, segments: int = 0) -> int:
+    d = Dims(B, H, L, dk, dv, chunk, _DTYPES[in_dtype], _DTYPES[out_dtype or torch.float32], segments)
     return int(lib().kdn_workspace_bytes(VARIANTS[variant], ctypes.byref(d)))
 
 
 def plan(variant: str, B: int, H: int, L: int, dk: int, dv: int, chunk: int = 0, in_dtype=torch.bfloat16,
-         out_dtype=None) -> dict:
+         out_dtype=None, segments: int = 0) -> dict:
     """The library's own account of the kernels a scan with these sizes runs."""
-    d = Dims(B, H, L, dk, dv, chunk, _DTYPES[in_dtype], _DTYPES[out_dtype or torch.float32])
+    d = Dims(B, H, L, dk, dv, chunk, _DTYPES[in_dtype], _DTYPES[out_dtype or torch.float32], segments)
     n, name, arith = ctypes.c_int(0), ctypes.c_char_p(), ctypes.c_char_p()
     _check(lib().kdn_plan(VARIANTS[variant], ctypes.byref(d), ctypes.byref(n), ctypes.byref(name),
                           ctypes.byref(arith)), "kdn_plan")
     return {"launches": n.value, "kernel": name.value.decode(), "arith": arith.value.decode()}
 
 
-def _scan_common(q, k, v, o, m, S, chunk, out_dtype):
+def _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments=0):
     if q.dim() != 4:
         raise ValueError("q must be [B, H, L, d_k]")
     B, H, L, dk = q.shape
@@ -153,7 +153,7 @@ def _scan_common(q, k, v, o, m, S, chunk, out_dtype):
     if S is None:
         S = torch.zeros(B, H, dk, dv, dtype=torch.float32, device=dev)
     _need(S, "S", (B, H, dk, dv), torch.float32, dev)
-    dims = Dims(B, H, L, dk, dv, chunk, _DTYPES[q.dtype], _DTYPES[out_dtype])
+    dims = Dims(B, H, L, dk, dv, chunk, _DTYPES[q.dtype], _DTYPES[out_dtype], segments)
     return dims, o, m, S
 
 
@@ -166,9 +166,10 @@ def _workspace(variant, dims, workspace, dev):
     return workspace
 
 
-def scan_delta(q, k, v, beta, a=None, S=None, o=None, m=None, workspace=None, chunk=0, out_dtype=None, stream=None):
+def scan_delta(q, k, v, beta, a=None, S=None, o=None, m=None, workspace=None, chunk=0, out_dtype=None, segments=0,
+               stream=None):
     """Gated delta rule scan.  Returns (o, m, S); S is updated in place when given."""
-    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments)
     tok = tuple(q.shape[:3])
     _need(beta, "beta", tok, torch.float32, q.device)
     if a is not None:
@@ -190,9 +191,9 @@ def _qn_args(qn, tok, dev):
 
 
 def scan_kalman_full(q, k, v, r, a=None, qn=None, S=None, P=None, o=None, m=None, workspace=None, chunk=0,
-                     out_dtype=None, stream=None):
+                     out_dtype=None, segments=0, stream=None):
     """Full-covariance Kalman scan.  Returns (o, m, S, P); S and P are updated in place when given."""
-    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments)
     B, H, L, dk = q.shape
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, q.device)
@@ -211,10 +212,10 @@ def scan_kalman_full(q, k, v, r, a=None, qn=None, S=None, P=None, o=None, m=None
 
 
 def scan_kalman_full_noalloc(q, k, v, r, a=None, qn=None, S=None, P=None, o=None, m=None, chunk=0,
-                             out_dtype=None, stream=None):
+                             out_dtype=None, segments=0, stream=None):
     """Full-Kalman scan without a workspace, for callers that cannot allocate one: the library uses a static
     device array (B*H*L*d_k <= 4,194,304; overlapping calls race on it).  Returns (o, m, S, P)."""
-    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments)
     B, H, L, dk = q.shape
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, q.device)
@@ -231,9 +232,9 @@ def scan_kalman_full_noalloc(q, k, v, r, a=None, qn=None, S=None, P=None, o=None
 
 
 def scan_kalman_diag(q, k, v, r, a=None, qn=None, S=None, p=None, o=None, m=None, workspace=None, chunk=0,
-                     out_dtype=None, stream=None):
+                     out_dtype=None, segments=0, stream=None):
     """Diagonal-covariance Kalman scan.  Returns (o, m, S, p); S and p are updated in place when given."""
-    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments)
     B, H, L, dk = q.shape
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, q.device)
@@ -252,10 +253,10 @@ def scan_kalman_diag(q, k, v, r, a=None, qn=None, S=None, p=None, o=None, m=None
 
 
 def scan_kalman_iso(q, k, v, r, a=None, qn=None, S=None, c=None, o=None, m=None, workspace=None, chunk=0,
-                    out_dtype=None, stream=None):
+                    out_dtype=None, segments=0, stream=None):
     """Isotropic-covariance Kalman scan (one uncertainty scalar per head).  Returns (o, m, S, c); S and c
     are updated in place when given."""
-    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype)
+    dims, o, m, S = _scan_common(q, k, v, o, m, S, chunk, out_dtype, segments)
     B, H, L, dk = q.shape
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, q.device)

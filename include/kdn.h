@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define KDN_API_VERSION 1
+#define KDN_API_VERSION 2
 
 #if defined(__GNUC__)
 #define KDN_EXPORT __attribute__((visibility("default")))
@@ -97,7 +97,26 @@ typedef struct kdn_dims {
   int chunk;            /* 0 = library choice; else 16, 32 or 64 tokens per chunk */
   kdn_dtype in_dtype;   /* dtype of q, k, v */
   kdn_dtype out_dtype;  /* dtype of o */
+  int segments;         /* sequence segments per head scanned in parallel:
+                         * 0 = library choice, 1 = one serial pass per head, P >= 2 = P segments
+                         * (L % P == 0; chunked path only, else KDN_ERR_UNSUPPORTED).  See below. */
 } kdn_dims;
+
+/* Segment-parallel scans.  With few heads (B*H well below the GPU's 148 SMs) one CTA per head leaves
+ * most of the GPU idle, and the chunk loop is serial.  The scan functions then cut each head's sequence
+ * into P equal segments (Kalman Delta Networks, Abstract: the uncertainty recurrences of the diagonal
+ * and isotropic variants are Moebius maps and compose associatively; for fixed gains the memory scan is
+ * affine in its start state):
+ *   - diagonal Kalman: each segment composes its per-coordinate uncertainty maps, and the maps are
+ *     chained to get p at every segment start; isotropic: the one-scalar beta prologue runs first;
+ *     full Kalman: the covariance side runs over the whole sequence first (it is not a per-coordinate
+ *     map), giving every token's gain;
+ *   - the chunk kernel runs all segments from S0 = 0 and from S0 = I (giving each segment's map
+ *     S0 -> M S0 + B), one fp32 pass per head chains the segment start states, and a last chunk-kernel
+ *     run from the true start states writes o, m and the final state.
+ * Results equal the serial scan's up to rounding.  The library choice (segments = 0) is P in {16, 8, 4}
+ * (the largest with B*H*P <= 148, L % (64 P) == 0 and at least two chunks per segment), else 1.  The
+ * workspace grows by 3 B*H*P*dk*dv floats (plus 7 B*H*P*dk for the diagonal variant) when P > 1. */
 
 /* Gated delta rule scan (A Hippocampus for Linear Attention, section 3.3
  * Eq. (5)-(6), section 3.5).  beta: write strengths, required.  a: decay gates

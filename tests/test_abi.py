@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.kdn_api_version() == 1
+    assert L.kdn_api_version() == 2
     for code, name in enumerate(["KDN_OK", "KDN_ERR_INVALID_ARG", "KDN_ERR_UNSUPPORTED", "KDN_ERR_CUDA",
                                  "KDN_ERR_NUMERIC", "KDN_ERR_TIMEOUT"]):
         assert L.kdn_status_string(code).decode() == name
@@ -78,6 +78,23 @@ def test_plan_counts_the_isotropic_prologue(L):
         fused = name.value == b"chunk_scan_ws_kernel"
         assert n_iso.value == n_delta.value + (0 if fused else 1)
     assert L.kdn_plan(4, ctypes.byref(kdn.Dims(1, 1, 4, 64, 64, 0, 1, 1)), None, None, None) == kdn.KDN_ERR_INVALID_ARG
+
+
+def test_segment_requests_on_the_host(L):
+    """Segment counts are checked before anything is enqueued: a negative count is invalid, and an explicit
+    split needs the chunked path (bf16 inputs, d_k = d_v in {64, 128}; here fp32 at d = 16)."""
+    for variant in range(4):
+        d = kdn.Dims(1, 1, 64, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32, -1)
+        assert L.kdn_workspace_bytes(variant, ctypes.byref(d)) == 0
+        assert L.kdn_plan(variant, ctypes.byref(d), None, None, None) == kdn.KDN_ERR_INVALID_ARG
+        d = kdn.Dims(1, 1, 64, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32, 2)
+        assert L.kdn_plan(variant, ctypes.byref(d), None, None, None) == kdn.KDN_ERR_UNSUPPORTED
+        assert b"chunked" in L.kdn_last_error()
+        auto = kdn.Dims(1, 1, 64, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32, 0)
+        serial = kdn.Dims(1, 1, 64, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32, 1)
+        assert L.kdn_workspace_bytes(variant, ctypes.byref(auto)) == L.kdn_workspace_bytes(variant, ctypes.byref(serial))
+    d = kdn.Dims(1, 1, 64, 16, 16, 0, kdn.KDN_F32, kdn.KDN_F32, -1)
+    assert _delta(L, d) == kdn.KDN_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():
