@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   __shared__ float sA[2][kC], sR[2][kC], sQ[2][kC];
   __shared__ float ell[kC], Aex[kC], gam[kC];
+  __shared__ float inv_dblk[16];  // 1 / D of the current diagonal block of the LDL
   __shared__ uint64_t bar_k, bar_mma;
   __shared__ uint32_t tmem_base;
 
@@ -311,84 +312,108 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ---------------------------------------------------------------- LDL of the Gram, blocked by 16
     // In place on the lower part of Gf: D on the diagonal, the unit lower factor below it.  Scratch in
     // Lf: the panel rows y = l D (rows 16..63, columns 0..15) and the panel transposed (rows 0..15).
-#pragma unroll 1
-    for (int kb = 0; kb < 4; ++kb) {
-      const int s0 = 16 * kb, s1 = s0 + 16;
-      if (warp == 0) {
-        // diagonal block in registers: lane i < 16 holds row s0 + i; right-looking with shuffles
-        float av[16];
-        const int li = lane & 15;
+    // Look-ahead: after the panel of block kb, warp 0 updates diagonal block kb + 1 and factorises it
+    // while warps 1..7 apply the rest of the trailing update.
+    auto factor_diag = [&](const int s0) {  // warp 0
+      // diagonal block in registers: lane i < 16 holds row s0 + i; right-looking with shuffles
+      float av[16];
+      const int li = lane & 15;
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const float4 v4 = *reinterpret_cast<const float4*>(Gf + (s0 + li) * LD + s0 + j);
-          av[j] = v4.x, av[j + 1] = v4.y, av[j + 2] = v4.z, av[j + 3] = v4.w;
-        }
+      for (int j = 0; j < 16; j += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(Gf + (s0 + li) * LD + s0 + j);
+        av[j] = v4.x, av[j + 1] = v4.y, av[j + 2] = v4.z, av[j + 3] = v4.w;
+      }
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float dp = __shfl_sync(0xffffffffu, av[p], p);
-          const float lp = av[p] * (1.f / dp);
+      for (int p = 0; p < 16; ++p) {
+        // column p of the trailing block, A[s0+j][s0+p] for j >= p (not yet scaled), all shuffles first
+        float cv[16];
 #pragma unroll
-          for (int j = 1; j < 16; ++j) {  // fixed bounds: every register index is a constant
-            const float cj = __shfl_sync(0xffffffffu, av[p], j);  // A[s0+j][s0+p], not yet scaled
-            if (j > p && li > p && j <= li) av[j] = fmaf(-lp, cj, av[j]);
-          }
-          if (li > p) av[p] = lp;
-        }
-        if (lane < 16) {
+        for (int j = p; j < 16; ++j) cv[j] = __shfl_sync(0xffffffffu, av[p], j);
+        const float lp = av[p] * (1.f / cv[p]);
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(Gf + (s0 + li) * LD + s0 + j) = make_float4(av[j], av[j + 1], av[j + 2], av[j + 3]);
-          float dpiv = 0.f;  // av[li] without a dynamic register index
+        for (int j = p + 1; j < 16; ++j)  // fixed bounds: every register index is a constant
+          if (li > p && j <= li) av[j] = fmaf(-lp, cv[j], av[j]);
+        if (li > p) av[p] = lp;
+      }
+      if (lane < 16) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) dpiv = (j == li) ? av[j] : dpiv;
-          if (!(dpiv > 0.f && isfinite(dpiv))) raise_status(P.status, kStatusNumeric);
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(Gf + (s0 + li) * LD + s0 + j) = make_float4(av[j], av[j + 1], av[j + 2], av[j + 3]);
+        float dpiv = 0.f;  // av[li] without a dynamic register index
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dpiv = (j == li) ? av[j] : dpiv;
+        if (!(dpiv > 0.f && isfinite(dpiv))) raise_status(P.status, kStatusNumeric);
+        inv_dblk[li] = 1.f / dpiv;
+      }
+    };
+    auto trailing_strip = [&](const int i, const int j) {  // A[i][j..j+3] -= y_i . l_{j..j+3}
+      float4 acc = *reinterpret_cast<const float4*>(Gf + i * LD + j);
+#pragma unroll
+      for (int cc = 0; cc < 16; cc += 4) {
+        const float4 y4 = *reinterpret_cast<const float4*>(Lf + i * LD + cc);
+        const float yv[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 l4 = *reinterpret_cast<const float4*>(Lf + (cc + u) * LD + j);
+          acc.x = fmaf(-yv[u], l4.x, acc.x), acc.y = fmaf(-yv[u], l4.y, acc.y);
+          acc.z = fmaf(-yv[u], l4.z, acc.z), acc.w = fmaf(-yv[u], l4.w, acc.w);
         }
       }
-      __syncthreads();
-      if (kb < 3) {
-        // panel rows i >= s1: solve y L_kk^T = x, l = y / D
-        const int nr = 64 - s1;
-        if (tid < nr) {
-          const int i = s1 + tid;
-          float y[16];
+      *reinterpret_cast<float4*>(Gf + i * LD + j) = acc;
+    };
+    if (warp == 0) factor_diag(0);
+#pragma unroll 1
+    for (int kb = 0; kb < 3; ++kb) {
+      const int s0 = 16 * kb, s1 = s0 + 16;
+      __syncthreads();  // diagonal block kb factorised, the trailing update of block kb - 1 applied
+      // panel rows i >= s1: solve y L_kk^T = x, l = y / D
+      const int nr = 64 - s1;
+      if (tid < nr) {
+        const int i = s1 + tid;
+        // right-looking forward substitution: once y[cc] is final it updates every later column, so
+        // the dependent chain is one FMA per column
+        float y[16];
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            float v = Gf[i * LD + s0 + cc];
-#pragma unroll
-            for (int m = 0; m < 15; ++m)  // fixed bounds: every register index is a constant
-              if (m < cc) v = fmaf(-y[m], Gf[(s0 + cc) * LD + s0 + m], v);
-            y[cc] = v;
-          }
-#pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const float l = y[cc] / Gf[(s0 + cc) * LD + s0 + cc];
-            Lf[i * LD + cc] = y[cc];
-            Lf[cc * LD + i] = l;  // transposed panel (rows 0..15)
-            Gf[i * LD + s0 + cc] = l;
-          }
+        for (int cc = 0; cc < 16; cc += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(Gf + i * LD + s0 + cc);
+          y[cc] = v4.x, y[cc + 1] = v4.y, y[cc + 2] = v4.z, y[cc + 3] = v4.w;
         }
-        __syncthreads();
-        // trailing update, strips of 4 columns: A[i][j..j+3] -= y_i . l_{j..j+3}
-        for (int idx = tid; idx < nr * (nr / 4); idx += kPThreads) {
-          const int i = s1 + idx / (nr / 4), j = s1 + 4 * (idx % (nr / 4));
-          if (j > i) continue;
-          float4 acc = *reinterpret_cast<const float4*>(Gf + i * LD + j);
 #pragma unroll
-          for (int cc = 0; cc < 16; cc += 4) {
-            const float4 y4 = *reinterpret_cast<const float4*>(Lf + i * LD + cc);
-            const float yv[4] = {y4.x, y4.y, y4.z, y4.w};
+        for (int cc = 0; cc < 15; ++cc) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float4 l4 = *reinterpret_cast<const float4*>(Lf + (cc + u) * LD + j);
-              acc.x = fmaf(-yv[u], l4.x, acc.x), acc.y = fmaf(-yv[u], l4.y, acc.y);
-              acc.z = fmaf(-yv[u], l4.z, acc.z), acc.w = fmaf(-yv[u], l4.w, acc.w);
-            }
-          }
-          *reinterpret_cast<float4*>(Gf + i * LD + j) = acc;
+          for (int c2 = cc + 1; c2 < 16; ++c2) y[c2] = fmaf(-y[cc], Gf[(s0 + c2) * LD + s0 + cc], y[c2]);
         }
-        __syncthreads();
+        float l[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          l[cc] = y[cc] * inv_dblk[cc];
+          Lf[cc * LD + i] = l[cc];  // transposed panel (rows 0..15)
+        }
+#pragma unroll
+        for (int cc = 0; cc < 16; cc += 4) {
+          *reinterpret_cast<float4*>(Lf + i * LD + cc) = make_float4(y[cc], y[cc + 1], y[cc + 2], y[cc + 3]);
+          *reinterpret_cast<float4*>(Gf + i * LD + s0 + cc) = make_float4(l[cc], l[cc + 1], l[cc + 2], l[cc + 3]);
+        }
+      }
+      __syncthreads();  // panel kb in Gf (l) and Lf (y rows, l transposed)
+      if (warp == 0) {
+        // the next diagonal block (rows and columns s1 .. s1 + 15), then its factorisation
+        for (int idx = lane; idx < 64; idx += 32) {
+          const int i = s1 + idx / 4, j = s1 + 4 * (idx % 4);
+          if (j <= i) trailing_strip(i, j);
+        }
+        __syncwarp();
+        factor_diag(s1);
+      } else {
+        // the rows below it, every column strip s1 .. i
+        const int nr2 = 48 - s1, ns = (64 - s1) / 4;
+        for (int idx = tid - 32; idx < nr2 * ns; idx += kPThreads - 32) {
+          const int i = s1 + 16 + idx / ns, j = s1 + 4 * (idx % ns);
+          if (j <= i) trailing_strip(i, j);
+        }
       }
     }
+    __syncthreads();  // the last diagonal block factorised
 
     // ---------------------------------------------------------------- L^-1, then (L^-1 o Gam) as bf16 hi/lo
     chunk::invert_unit_lower_64(Gf, Lf, tid, sync_all);
