@@ -32,6 +32,13 @@ using mobius::Mob;
 
 constexpr int kMapThreads = 512;
 
+// 16-byte asynchronous global -> shared copy (Ampere-style cp.async, cached in L2 only)
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ float load_key(const void* k, size_t i, int dtype) {
   if (dtype == kBF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(k)[i]);
   return reinterpret_cast<const float*>(k)[i];
@@ -110,66 +117,86 @@ __global__ void __launch_bounds__(256) seg_init_kernel(float* Sz, float* SI, int
 }
 
 // Step 3 (d = 64 or 128): S_{s+1} = (SI_s - Sz_s) S_s + Sz_s for one head and a slab of kSlab columns; every
-// S_s (s = 0 .. P-1, S_0 the caller's state) is written to Sc.  M_s = SI_s - Sz_s is staged
-// transposed in shared memory (rows padded by 4 floats) so that each thread reads the 8 rows of its
-// outputs with two 16-byte loads per k.
+// S_s (s = 0 .. P-1, S_0 the caller's state) is written to Sc.  Per segment the CTA stages SI_s and Sz_s in
+// shared memory with asynchronous 16-byte copies (rows padded by 4 floats; every slab of the head reads the
+// same L2-resident rows), then each thread forms one row r of the slab (kCombThreads / D threads per row,
+// kSlab / that many columns each) from its row of M_s and 16-byte broadcast loads of the slab of S_s.
 constexpr int kSlab = 16;
 constexpr int kCombThreads = 256;
 
 template <int D>
+struct CombLayout {
+  static constexpr int RS = D + 4;                               // padded row of the staged SI_s, Sz_s
+  static constexpr size_t SMEM = sizeof(float) * (2 * (size_t)D * RS + (size_t)D * kSlab);
+};
+
+template <int D>
 __global__ void __launch_bounds__(kCombThreads) seg_combine_kernel(SegArgs p) {
-  constexpr int MT = D + 4;                       // padded row of the transposed M
-  constexpr int RPT = D * kSlab / kCombThreads;   // output rows per thread (8 at D = 128)
-  static_assert(RPT % 4 == 0, "two or more 16-byte row groups per thread");
+  constexpr int TPR = kCombThreads / D;          // threads per row: 2 at D = 128, 4 at D = 64
+  constexpr int CPT = kSlab / TPR;               // columns per thread: 8 or 4
+  constexpr int RS = CombLayout<D>::RS;
+  static_assert(CPT % 4 == 0, "whole 16-byte column groups per thread");
   extern __shared__ __align__(16) float sm[];
-  float* Mt = sm;                                 // [D][MT]: Mt[k][r] = M[r][k]
-  float* X = sm + D * MT;                         // [D][kSlab]
+  float* SIs = sm;                               // [D][RS]
+  float* Szs = sm + D * RS;                      // [D][RS]
+  float* X = sm + 2 * D * RS;                    // [D][kSlab]: the slab of S_s
   const int h = blockIdx.y, c0 = blockIdx.x * kSlab;
   const int tid = threadIdx.x;
-  const int c = tid % kSlab, r0 = (tid / kSlab) * RPT;
+  const int r = tid / TPR, cg = (tid % TPR) * CPT;
   const size_t DD = (size_t)D * D;
 
   for (int e = tid; e < D * kSlab; e += kCombThreads) {
-    const int r = e / kSlab, cc = e % kSlab;
-    X[e] = p.S[(size_t)h * DD + (size_t)r * D + c0 + cc];
+    const int rr = e / kSlab, cc = e % kSlab;
+    X[e] = p.S[(size_t)h * DD + (size_t)rr * D + c0 + cc];
   }
   __syncthreads();
   for (int s = 0; s < p.P; ++s) {
     const size_t j = (size_t)h * p.P + s;
-    for (int e = tid; e < D * kSlab; e += kCombThreads) {
-      const int r = e / kSlab, cc = e % kSlab;
-      p.Sc[j * DD + (size_t)r * D + c0 + cc] = X[e];
-    }
-    if (s + 1 == p.P) break;
-    const float* Sz = p.Sz + j * DD;
-    const float* SI = p.SI + j * DD;
-    for (int e = tid; e < D * D; e += kCombThreads) {
-      const int r = e / D, k = e % D;
-      Mt[k * MT + r] = SI[e] - Sz[e];
-    }
-    __syncthreads();
-    float acc[RPT];
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) acc[u] = Sz[(size_t)(r0 + u) * D + c0 + c];
-#pragma unroll 4
-    for (int k = 0; k < D; ++k) {
-      const float x = X[k * kSlab + c];
-      const float4* mr = reinterpret_cast<const float4*>(Mt + k * MT + r0);
-#pragma unroll
-      for (int u4 = 0; u4 < RPT / 4; ++u4) {
-        const float4 m4 = mr[u4];
-        acc[4 * u4 + 0] = fmaf(m4.x, x, acc[4 * u4 + 0]);
-        acc[4 * u4 + 1] = fmaf(m4.y, x, acc[4 * u4 + 1]);
-        acc[4 * u4 + 2] = fmaf(m4.z, x, acc[4 * u4 + 2]);
-        acc[4 * u4 + 3] = fmaf(m4.w, x, acc[4 * u4 + 3]);
+    if (s + 1 < p.P) {
+      const float* SIg = p.SI + j * DD;
+      const float* Szg = p.Sz + j * DD;
+      for (int q = tid; q < D * D / 4; q += kCombThreads) {
+        const int rr = (4 * q) / D, cc = (4 * q) % D;
+        cp_async16(SIs + rr * RS + cc, SIg + 4 * (size_t)q);
+        cp_async16(Szs + rr * RS + cc, Szg + 4 * (size_t)q);
       }
     }
-    __syncthreads();                              // every thread is done with X and Mt
+    for (int e = tid; e < D * kSlab; e += kCombThreads) {
+      const int rr = e / kSlab, cc = e % kSlab;
+      p.Sc[j * DD + (size_t)rr * D + c0 + cc] = X[e];
+    }
+    if (s + 1 == p.P) break;
+    cp_async_wait_all();
+    __syncthreads();                              // SI_s, Sz_s staged
+    float acc[CPT];
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) acc[u] = Szs[r * RS + c0 + cg + u];
+#pragma unroll 4
+    for (int kq = 0; kq < D / 4; ++kq) {
+      const float4 a4 = *reinterpret_cast<const float4*>(SIs + r * RS + 4 * kq);
+      const float4 b4 = *reinterpret_cast<const float4*>(Szs + r * RS + 4 * kq);
+      const float m[4] = {a4.x - b4.x, a4.y - b4.y, a4.z - b4.z, a4.w - b4.w};  // M_s[r][4 kq ..]
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4* xr = reinterpret_cast<const float4*>(X + (4 * kq + e) * kSlab + cg);
+#pragma unroll
+        for (int u4 = 0; u4 < CPT / 4; ++u4) {
+          const float4 x4 = xr[u4];
+          acc[4 * u4 + 0] = fmaf(m[e], x4.x, acc[4 * u4 + 0]);
+          acc[4 * u4 + 1] = fmaf(m[e], x4.y, acc[4 * u4 + 1]);
+          acc[4 * u4 + 2] = fmaf(m[e], x4.z, acc[4 * u4 + 2]);
+          acc[4 * u4 + 3] = fmaf(m[e], x4.w, acc[4 * u4 + 3]);
+        }
+      }
+    }
+    __syncthreads();                              // every thread is done with X, SI_s and Sz_s
     bool bad = false;
 #pragma unroll
-    for (int u = 0; u < RPT; ++u) {
-      X[(r0 + u) * kSlab + c] = acc[u];
-      bad |= !isfinite(acc[u]);
+    for (int u4 = 0; u4 < CPT / 4; ++u4) {
+      *reinterpret_cast<float4*>(X + r * kSlab + cg + 4 * u4) =
+          make_float4(acc[4 * u4], acc[4 * u4 + 1], acc[4 * u4 + 2], acc[4 * u4 + 3]);
+      bad |= !(isfinite(acc[4 * u4]) && isfinite(acc[4 * u4 + 1]) && isfinite(acc[4 * u4 + 2]) &&
+               isfinite(acc[4 * u4 + 3]));
     }
     if (bad) raise_status(p.status, kStatusNumeric);
     __syncthreads();
@@ -178,7 +205,7 @@ __global__ void __launch_bounds__(kCombThreads) seg_combine_kernel(SegArgs p) {
 
 template <int D>
 cudaError_t launch_combine(const SegArgs& p, int BH, cudaStream_t stream) {
-  constexpr size_t smem = sizeof(float) * ((size_t)D * (D + 4) + (size_t)D * kSlab);
+  constexpr size_t smem = CombLayout<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(seg_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   seg_combine_kernel<D><<<dim3(D / kSlab, BH), kCombThreads, smem, stream>>>(p);
