@@ -79,14 +79,25 @@ def decode_bytes(w, in_bytes=2, out_bytes=4) -> int:
 # taken on: a different hash of those files reports null.
 _WS_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/chunk_scan_ws.cu",
                "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
-               "delta_rule_recurrent_scan_b200/csrc/sm100.cuh"]
+               "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
+               "delta_rule_recurrent_scan_b200/csrc/mobius.cuh"]
+_PSIDE_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/pside.cu",
+                  "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
+                  "delta_rule_recurrent_scan_b200/csrc/sm100.cuh"]
+_B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment per head)
 NCU_TRAFFIC = {
-    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "ede10530cbb47eeea928d574215cca12a76714e9",
-                         "bytes_per_token": (205.816576e6 + 104.452608e6) / (2 * 16 * 8192),
-                         "capture": "profiles/chunk_scan_ws_kernel_kalman_diag_d128.md (B=2 case, scaled)"},
-    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "ede10530cbb47eeea928d574215cca12a76714e9",
-                 "bytes_per_token": (205.635072e6 + 104.847872e6) / (2 * 16 * 8192),
-                 "capture": "profiles/chunk_scan_ws_kernel_delta_d128.md (B=2 case, scaled)"},
+    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
+                         "bytes_per_token": (308.443648e6 + 171.383808e6) / _B3,
+                         "capture": "profiles/chunk_scan_ws_kernel_kalman_diag_d128.md (B=3 case, scaled)"},
+    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
+                 "bytes_per_token": (308.621056e6 + 170.472192e6) / _B3,
+                 "capture": "profiles/chunk_scan_ws_kernel_delta_d128.md (B=3 case, scaled)"},
+    "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
+                        "bytes_per_token": (308.480256e6 + 171.998976e6) / _B3,
+                        "capture": "profiles/chunk_scan_ws_kernel_kalman_iso_d128.md (B=3 case, scaled)"},
+    "kalman_full_d128": {"sources": _PSIDE_SOURCES, "sha1": "0bbdf6201df85beaf0b536f88b1722c9cc0b5c8e",
+                         "bytes_per_token": (18.464256e6 + 5.376e3) / (2 * 8 * 4096),
+                         "capture": "profiles/kalman_pside_kernel_kalman_full_d128.md (full workload)"},
 }
 
 
