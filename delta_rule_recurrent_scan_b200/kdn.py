@@ -7,6 +7,11 @@ to fp32: rounding it to bf16 alone costs up to 2^-8 of its magnitude, more than
 the 3e-3 the scan is held to; pass out_dtype=torch.bfloat16 to halve its bytes.  Every step of the scan
 runs in the library's kernels.  There is no fallback: if the library is
 missing or the tensors are not on a CUDA device, the call raises.
+
+Every scan takes ``segments`` (kdn_dims.segments): 0 lets the library cut each
+head's sequence into several segments scanned by separate CTAs when there are
+too few heads to fill the GPU, 1 forces one serial pass per head, P >= 2 asks
+for P segments (P must divide L).  Results agree up to rounding.
 """
 
 from __future__ import annotations
