@@ -289,28 +289,69 @@ def bench_scan(w, steps, warmup, dist_on, rank, world, clocks=None):
 
 
 def bench_e2e(w, steps, warmup, dist_on, rank, world):
-    """Through the public API with host buffers: pinned host inputs -> device, scan, outputs -> host."""
+    """Through the public API with host buffers, as a stream of batches: every step copies its inputs from
+    pinned host memory to the device, scans them and copies o and m back.  Steps are pipelined over three
+    streams with two device buffer sets, so that step i + 1's host-to-device copy runs beside step i's scan
+    and device-to-host copy (the link is full duplex); the time per step is the span of all steps / steps."""
     from delta_rule_recurrent_scan_b200 import kdn
     xd = make_scan_inputs(w, seed=rank, device="cuda")
     host = {k: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
-    dev = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
+    bufs = []
+    for _ in range(2):
+        dev = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
+        fn_dev, outs = scan_closure(w, dev, kdn)
+        bufs.append((dev, fn_dev, outs))
     del xd
-    fn_dev, outs = scan_closure(w, dev, kdn)
-    o_host = torch.empty(outs["o"].shape, dtype=outs["o"].dtype).pin_memory()
-    m_host = torch.empty(outs["m"].shape).pin_memory()
+    o_host = torch.empty(bufs[0][2]["o"].shape, dtype=bufs[0][2]["o"].dtype).pin_memory()
+    m_host = torch.empty(bufs[0][2]["m"].shape).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if isinstance(v, torch.Tensor))
     d2h = o_host.numel() * o_host.element_size() + m_host.numel() * 4
 
-    def step():
-        for k, v in host.items():
-            if isinstance(v, torch.Tensor):
-                dev[k].copy_(v, non_blocking=True)
-        fn_dev()
-        o_host.copy_(outs["o"], non_blocking=True)
-        m_host.copy_(outs["m"], non_blocking=True)
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "comp", "out")}
+    cur = torch.cuda.current_stream()
+    for name in ev:
+        for e in ev[name]:
+            e.record(cur)
 
-    ms = time_device(step, steps, warmup, dist_on)
-    return {"value": w.tokens * world / (ms * 1e-3), "ms": ms, "h2d": h2d, "d2h": d2h}
+    def step(i):
+        b = i % 2
+        dev, fn_dev, outs = bufs[b]
+        s_in.wait_event(ev["comp"][b])       # the scan of step i - 2 has read these inputs
+        with torch.cuda.stream(s_in):
+            for k, v in host.items():
+                if isinstance(v, torch.Tensor):
+                    dev[k].copy_(v, non_blocking=True)
+            ev["in"][b].record(s_in)
+        s_comp.wait_event(ev["in"][b])
+        s_comp.wait_event(ev["out"][b])      # step i - 2's outputs are back on the host
+        with torch.cuda.stream(s_comp):
+            fn_dev()
+            ev["comp"][b].record(s_comp)
+        s_out.wait_event(ev["comp"][b])
+        with torch.cuda.stream(s_out):
+            o_host.copy_(outs["o"], non_blocking=True)
+            m_host.copy_(outs["m"], non_blocking=True)
+            ev["out"][b].record(s_out)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(cur)
+    for st in (s_in, s_comp, s_out):
+        st.wait_event(start)
+    for i in range(steps):
+        step(warmup + i)
+    for st in (s_in, s_comp, s_out):
+        cur.wait_stream(st)
+    end.record(cur)
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    ms = _max_over_ranks(start.elapsed_time(end) / steps, dist_on)
+    return {"value": w.tokens * world / (ms * 1e-3), "ms": ms, "h2d": h2d, "d2h": d2h,
+            "pipelined": "3 streams, 2 device buffer sets: step i + 1's copy-in beside step i's scan and copy-out"}
 
 
 def bench_decode(w, steps, warmup, dist_on, rank, world):
@@ -434,7 +475,7 @@ def main():
     plan = scan_plan(w)
     torch.cuda.empty_cache()
 
-    e2e = None if args.no_e2e else bench_e2e(w, min(args.steps, 5), 3, dist_on, rank, world)
+    e2e = None if args.no_e2e else bench_e2e(w, min(args.steps, 10), 3, dist_on, rank, world)
     torch.cuda.empty_cache()
 
     also = []
@@ -492,7 +533,7 @@ def main():
                          "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events"},
             "e2e": None if e2e is None else {"value": e2e["value"], "unit": "tokens/s",
                                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                                             "ms_per_step": e2e["ms"]},
+                                             "ms_per_step": e2e["ms"], "pipelined": e2e["pipelined"]},
             "gpu_launches": head["launches"],
             "clocks": clocks.summary(),
             "also": also,
