@@ -1,0 +1,101 @@
+"""Float64 reverse-mode derivatives of the gated delta rule scan (training's backward pass).
+
+TEST INFRASTRUCTURE ONLY, like the rest of ``oracle/``: nothing in the product package imports it.
+
+The pages train the layers these scans come from (A Hippocampus for Linear Attention, section 4: models
+pretrained at 340M to 1.3B parameters; Kalman Delta Networks, Abstract: the KDN layers are trained
+end to end), but print no backward pass.  This is the plainest one: the adjoint of the token-by-token
+recurrence of ``oracle.scan.scan_delta``, written out by the chain rule and run backwards in time.
+
+Forward, per head (section 3.3 Eq. (5)-(6) and section 3.5 of the HOLA page):
+
+    e_t = v_t - a_t S_{t-1}^T k_t,   S_t = a_t S_{t-1} + beta_t k_t e_t^T,
+    o_t = S_t^T q_t,                 m_t = beta_t ||k_t|| ||e_t||.
+
+For a scalar loss with upstream gradients dO_t = dLoss/do_t, dm_t = dLoss/dm_t and dS_L = dLoss/dS_L, let
+G_t = dLoss/dS_t (everything that reaches S_t, including through later tokens).  Backwards from t = L:
+
+    G_t     += q_t dO_t^T                         (the read o_t = S_t^T q_t)
+    dq_t     = S_t dO_t
+    de_t     = beta_t G_t^T k_t + dm_t beta_t ||k_t|| e_t / ||e_t||
+    dbeta_t  = k_t^T G_t e_t + dm_t ||k_t|| ||e_t||
+    dk_t     = beta_t G_t e_t + dm_t beta_t ||e_t|| k_t / ||k_t||  -  a_t S_{t-1} de_t
+    dv_t     = de_t
+    da_t     = <G_t, S_{t-1}>  -  k_t^T S_{t-1} de_t
+    G_{t-1}  = a_t G_t  -  a_t k_t de_t^T
+
+and dS_0 = G_0.  The states S_{t-1} are kept from a forward pass (this is the oracle: memory is no object).
+A zero residual or a zero key contributes no surprise gradient (the norm is not differentiable there; the
+one-sided choice 0 is taken).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .scan import _f64, _flatten_inputs, _per_token, _read
+
+__all__ = ["scan_delta_backward"]
+
+
+def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None):
+    """Gradients of the gated delta rule scan.
+
+    Shapes as ``oracle.scan.scan_delta``: q, k [..., L, d_k]; v [..., L, d_v]; beta, a [..., L];
+    S0 [..., d_k, d_v] (None = 0); upstream dO [..., L, d_v], dm [..., L] or None, dS_L [..., d_k, d_v] or
+    None.  Returns a dict of float64 arrays dq, dk, dv, dbeta, da (da is returned even for a=None, as the
+    gradient at a_t = 1) and dS0, each with its input's shape.
+    """
+    lead, n, L, dk, dv, q, k, v = _flatten_inputs(q, k, v)
+    beta = _per_token(beta, n, L, 0.0)
+    a = _per_token(a, n, L, 1.0)
+    dO = _f64(dO).reshape(n, L, dv)
+    dm = _per_token(dm, n, L, 0.0)
+    S = np.zeros((n, dk, dv)) if S0 is None else _f64(S0).reshape(n, dk, dv).copy()
+
+    # forward, keeping every state and residual
+    states = np.zeros((n, L + 1, dk, dv))
+    states[:, 0] = S
+    res = np.zeros((n, L, dv))
+    for t in range(L):
+        kt = k[:, t]
+        S_pred = a[:, t, None, None] * S
+        e = v[:, t] - _read(S_pred, kt)
+        S = S_pred + beta[:, t, None, None] * kt[:, :, None] * e[:, None, :]
+        states[:, t + 1] = S
+        res[:, t] = e
+
+    # backward
+    G = np.zeros((n, dk, dv)) if dS_L is None else _f64(dS_L).reshape(n, dk, dv).copy()
+    dq = np.zeros((n, L, dk))
+    dkk = np.zeros((n, L, dk))
+    dvv = np.zeros((n, L, dv))
+    dbeta = np.zeros((n, L))
+    da = np.zeros((n, L))
+    for t in range(L - 1, -1, -1):
+        kt, qt, e = k[:, t], q[:, t], res[:, t]
+        S_t, S_prev = states[:, t + 1], states[:, t]
+        bt, at = beta[:, t], a[:, t]
+        G = G + qt[:, :, None] * dO[:, t, None, :]
+        dq[:, t] = np.einsum("nij,nj->ni", S_t, dO[:, t])
+        kn = np.linalg.norm(kt, axis=-1)
+        en = np.linalg.norm(e, axis=-1)
+        e_dir = np.where(en[:, None] > 0, e / np.where(en > 0, en, 1.0)[:, None], 0.0)
+        k_dir = np.where(kn[:, None] > 0, kt / np.where(kn > 0, kn, 1.0)[:, None], 0.0)
+        Ge = np.einsum("nij,nj->ni", G, e)                   # G e      (d_k)
+        GTk = _read(G, kt)                                   # G^T k    (d_v)
+        de = bt[:, None] * GTk + (dm[:, t] * bt * kn)[:, None] * e_dir
+        dbeta[:, t] = np.einsum("ni,ni->n", kt, Ge) + dm[:, t] * kn * en
+        dkk[:, t] = bt[:, None] * Ge + (dm[:, t] * bt * en)[:, None] * k_dir
+        dkk[:, t] -= at[:, None] * np.einsum("nij,nj->ni", S_prev, de)
+        dvv[:, t] = de
+        da[:, t] = np.einsum("nij,nij->n", G, S_prev) - np.einsum("ni,nij,nj->n", kt, S_prev, de)
+        G = at[:, None, None] * G - at[:, None, None] * kt[:, :, None] * de[:, None, :]
+    return {
+        "dq": dq.reshape(*lead, L, dk),
+        "dk": dkk.reshape(*lead, L, dk),
+        "dv": dvv.reshape(*lead, L, dv),
+        "dbeta": dbeta.reshape(*lead, L),
+        "da": da.reshape(*lead, L),
+        "dS0": G.reshape(*lead, dk, dv),
+    }

@@ -1,0 +1,89 @@
+"""Pins of the float64 backward of the gated delta rule (oracle/backward.py) — CPU only.
+
+The backward is checked against routes that do not use its reverse recurrence: central finite differences
+of the forward oracle for every input, and the closed form of the scan when nothing is written (beta = 0,
+so S_t = A_t S_0 and every output is linear in S_0 and q).  Shapes use d_k != d_v, q != k, gates below one
+and a non-zero start state, so that a transposed product, a missing decay or a dropped path through the
+residual fails.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import scan_delta
+from oracle.backward import scan_delta_backward
+
+
+def _inputs(seed, heads, L, dk, dv):
+    rng = np.random.default_rng(seed)
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    x = {
+        "q": unit(rng.standard_normal((heads, L, dk))),
+        "k": unit(rng.standard_normal((heads, L, dk))) * (1.0 + 0.3 * rng.random((heads, L, 1))),
+        "v": rng.standard_normal((heads, L, dv)),
+        "beta": 0.2 + 0.7 * rng.random((heads, L)),
+        "a": 0.6 + 0.39 * rng.random((heads, L)),
+        "S0": 0.5 * rng.standard_normal((heads, dk, dv)),
+    }
+    up = {"dO": rng.standard_normal((heads, L, dv)), "dm": rng.standard_normal((heads, L)),
+          "dS_L": rng.standard_normal((heads, dk, dv))}
+    return x, up
+
+
+def _loss(x, up):
+    out = scan_delta(x["q"], x["k"], x["v"], x["beta"], a=x["a"], S0=x["S0"])
+    return float(np.sum(up["dO"] * out["o"]) + np.sum(up["dm"] * out["m"]) + np.sum(up["dS_L"] * out["S"]))
+
+
+@pytest.mark.parametrize("use_dm", [False, True])
+def test_backward_matches_central_differences_for_every_input(use_dm):
+    x, up = _inputs(3, heads=2, L=9, dk=3, dv=4)
+    if not use_dm:
+        up["dm"] = np.zeros_like(up["dm"])
+    g = scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], up["dO"], a=x["a"], S0=x["S0"], dm=up["dm"],
+                            dS_L=up["dS_L"])
+    names = {"q": "dq", "k": "dk", "v": "dv", "beta": "dbeta", "a": "da", "S0": "dS0"}
+    h = 1e-6
+    for name, gname in names.items():
+        num = np.zeros_like(x[name])
+        it = np.nditer(x[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {kk: vv.copy() for kk, vv in x.items()}
+            xm = {kk: vv.copy() for kk, vv in x.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            num[idx] = (_loss(xp, up) - _loss(xm, up)) / (2 * h)
+        scale = np.abs(num).max()
+        assert np.abs(g[gname] - num).max() <= 1e-6 * max(scale, 1.0), (name, np.abs(g[gname] - num).max(), scale)
+
+
+def test_backward_without_writes_is_the_closed_form():
+    """beta = 0: S_t = A_t S_0 with A_t = a_1 ... a_t, so o_t = A_t S_0^T q_t, and
+    dq_t = A_t S_0 dO_t,  dS_0 = sum_t A_t q_t dO_t^T + A_L dS_L,  dv_t = 0,
+    da_t = (1 / a_t) sum_{s >= t} A_s <q_s dO_s^T, S_0> + (A_L / a_t) <dS_L, S_0>."""
+    x, up = _inputs(5, heads=1, L=7, dk=3, dv=2)
+    x["beta"] = np.zeros_like(x["beta"])
+    g = scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], up["dO"], a=x["a"], S0=x["S0"], dS_L=up["dS_L"])
+    a, q, dO, S0, dSL = x["a"][0], x["q"][0], up["dO"][0], x["S0"][0], up["dS_L"][0]
+    A = np.cumprod(a)
+    np.testing.assert_allclose(g["dq"][0], A[:, None] * (dO @ S0.T), rtol=1e-12, atol=1e-14)
+    dS0 = sum(A[t] * np.outer(q[t], dO[t]) for t in range(7)) + A[-1] * dSL
+    np.testing.assert_allclose(g["dS0"][0], dS0, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(g["dv"][0], 0.0, atol=1e-15)
+    read = np.array([A[s] * np.sum(np.outer(q[s], dO[s]) * S0) for s in range(7)])
+    da = np.array([(read[t:].sum() + A[-1] * np.sum(dSL * S0)) / a[t] for t in range(7)])
+    np.testing.assert_allclose(g["da"][0], da, rtol=1e-12, atol=1e-14)
+
+
+def test_backward_of_a_single_token_by_hand():
+    """One token from S_0 = 0 with a = 1: S_1 = beta k v^T, o = beta (q.k) v, so
+    dq = beta (v.dO) k, dv = beta (q.k) dO, dbeta = (q.k)(v.dO), dk = beta (v.dO) q."""
+    rng = np.random.default_rng(7)
+    q, k, v, dO = rng.standard_normal(3), rng.standard_normal(3), rng.standard_normal(2), rng.standard_normal(2)
+    b = 0.7
+    g = scan_delta_backward(q[None], k[None], v[None], np.array([b]), dO[None])
+    np.testing.assert_allclose(g["dq"][0], b * (v @ dO) * k, rtol=1e-13)
+    np.testing.assert_allclose(g["dv"][0], b * (q @ k) * dO, rtol=1e-13)
+    np.testing.assert_allclose(g["dbeta"][0], (q @ k) * (v @ dO), rtol=1e-13)
+    np.testing.assert_allclose(g["dk"][0], b * (v @ dO) * q, rtol=1e-13)
