@@ -1,4 +1,4 @@
-"""Float64 reverse-mode derivatives of the gated delta rule scan (training's backward pass).
+"""Float64 reverse-mode derivatives of the gated delta rule and diagonal-Kalman scans (the backward pass).
 
 TEST INFRASTRUCTURE ONLY, like the rest of ``oracle/``: nothing in the product package imports it.
 
@@ -27,6 +27,18 @@ G_t = dLoss/dS_t (everything that reaches S_t, including through later tokens). 
 and dS_0 = G_0.  The states S_{t-1} are kept from a forward pass (this is the oracle: memory is no object).
 A zero residual or a zero key contributes no surprise gradient (the norm is not differentiable there; the
 one-sided choice 0 is taken).
+
+The diagonal-Kalman variant (Kalman Delta Networks, Abstract; the mean-field reading R3 of
+``oracle.scan``) adds the variance vector p to the state.  Per token
+
+    p^- = a_t^2 p + Qn_t,  s_t = sum_i p^-_i k_ti^2 + r_t,  g_t = p^- o k_t / s_t,
+    p   = p^- r_t / (r_t + p^- o k_t^2),
+
+and the write is S_t = a_t S_{t-1} + g_t e_t^T with m_t = ||g_t|| ||e_t||.  Its backward carries the
+adjoint Pb = dLoss/dp next to G: from g, dp^- = dg o k / s, ds = -(dg . g) / s, dk += dg o p^- / s; from
+the projection p = p^- r / den (den = r + p^- k^2), dp^- += Pb r^2 / den^2, dr += sum Pb (p^- k)^2 / den^2,
+dk -= 2 Pb (p^-)^2 r k / den^2; from s, dp^- += ds k^2, dk += 2 ds p^- k, dr += ds; and through the
+propagation Pb_{t-1} = a_t^2 dp^-, da_t += 2 a_t (dp^- . p_{t-1}), dQn_t = sum dp^-.
 """
 
 from __future__ import annotations
@@ -35,7 +47,7 @@ import numpy as np
 
 from .scan import _f64, _flatten_inputs, _per_token, _read
 
-__all__ = ["scan_delta_backward"]
+__all__ = ["scan_delta_backward", "scan_kalman_diag_backward"]
 
 
 def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None):
@@ -98,4 +110,87 @@ def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None):
         "dbeta": dbeta.reshape(*lead, L),
         "da": da.reshape(*lead, L),
         "dS0": G.reshape(*lead, dk, dv),
+    }
+
+
+def scan_kalman_diag_backward(q, k, v, r, dO, a=None, qn=None, S0=None, p0=None, dm=None, dS_L=None, dp_L=None):
+    """Gradients of the diagonal-Kalman scan (``oracle.scan.scan_kalman_diag``).
+
+    Shapes: q, k [..., L, d_k]; v [..., L, d_v]; r, a, qn [..., L] (a, qn may be None: 1 and 0); S0
+    [..., d_k, d_v]; p0 [..., d_k] (None = 1); upstream dO [..., L, d_v], dm [..., L], dS_L [..., d_k, d_v],
+    dp_L [..., d_k] (each None = 0).  Returns dq, dk, dv, dr, da, dqn (per token), dS0 and dp0.
+    """
+    lead, n, L, dk, dv, q, k, v = _flatten_inputs(q, k, v)
+    r = _per_token(r, n, L, 1.0)
+    a = _per_token(a, n, L, 1.0)
+    qn = _per_token(qn, n, L, 0.0)
+    dO = _f64(dO).reshape(n, L, dv)
+    dm = _per_token(dm, n, L, 0.0)
+    S = np.zeros((n, dk, dv)) if S0 is None else _f64(S0).reshape(n, dk, dv).copy()
+    p = np.ones((n, dk)) if p0 is None else _f64(p0).reshape(n, dk).copy()
+
+    states = np.zeros((n, L + 1, dk, dv))
+    pvec = np.zeros((n, L + 1, dk))
+    states[:, 0], pvec[:, 0] = S, p
+    res, gains, pms, ss = np.zeros((n, L, dv)), np.zeros((n, L, dk)), np.zeros((n, L, dk)), np.zeros((n, L))
+    for t in range(L):
+        kt, at = k[:, t], a[:, t]
+        pm = (at * at)[:, None] * p + qn[:, t, None]
+        st = np.einsum("ni,ni->n", pm, kt * kt) + r[:, t]
+        g = pm * kt / st[:, None]
+        p = pm * r[:, t, None] / (r[:, t, None] + pm * kt * kt)
+        S_pred = at[:, None, None] * S
+        e = v[:, t] - _read(S_pred, kt)
+        S = S_pred + g[:, :, None] * e[:, None, :]
+        states[:, t + 1], pvec[:, t + 1] = S, p
+        res[:, t], gains[:, t], pms[:, t], ss[:, t] = e, g, pm, st
+
+    G = np.zeros((n, dk, dv)) if dS_L is None else _f64(dS_L).reshape(n, dk, dv).copy()
+    Pb = np.zeros((n, dk)) if dp_L is None else _f64(dp_L).reshape(n, dk).copy()
+    dq, dkk, dvv = np.zeros((n, L, dk)), np.zeros((n, L, dk)), np.zeros((n, L, dv))
+    dr, da, dqn = np.zeros((n, L)), np.zeros((n, L)), np.zeros((n, L))
+    for t in range(L - 1, -1, -1):
+        kt, qt, e, g, pm, st = k[:, t], q[:, t], res[:, t], gains[:, t], pms[:, t], ss[:, t]
+        at, rt = a[:, t], r[:, t]
+        S_t, S_prev, p_prev = states[:, t + 1], states[:, t], pvec[:, t]
+        G = G + qt[:, :, None] * dO[:, t, None, :]
+        dq[:, t] = np.einsum("nij,nj->ni", S_t, dO[:, t])
+        gn = np.linalg.norm(g, axis=-1)
+        en = np.linalg.norm(e, axis=-1)
+        e_dir = np.where(en[:, None] > 0, e / np.where(en > 0, en, 1.0)[:, None], 0.0)
+        g_dir = np.where(gn[:, None] > 0, g / np.where(gn > 0, gn, 1.0)[:, None], 0.0)
+        # the write S_t = a S_{t-1} + g e^T and the surprise m_t = ||g|| ||e||
+        de = _read(G, g) + (dm[:, t] * gn)[:, None] * e_dir
+        dg = np.einsum("nij,nj->ni", G, e) + (dm[:, t] * en)[:, None] * g_dir
+        dkt = -at[:, None] * np.einsum("nij,nj->ni", S_prev, de)
+        dvv[:, t] = de
+        da_t = np.einsum("nij,nij->n", G, S_prev) - np.einsum("ni,nij,nj->n", kt, S_prev, de)
+        G = at[:, None, None] * G - at[:, None, None] * kt[:, :, None] * de[:, None, :]
+        # g = p^- o k / s
+        dpm = dg * kt / st[:, None]
+        dkt += dg * pm / st[:, None]
+        ds = -np.einsum("ni,ni->n", dg, g) / st
+        # p = p^- r / (r + p^- k^2)
+        den = rt[:, None] + pm * kt * kt
+        dpm += Pb * rt[:, None] ** 2 / den ** 2
+        dr_t = np.einsum("ni,ni->n", Pb, (pm * kt) ** 2 / den ** 2)
+        dkt -= 2.0 * Pb * pm * pm * rt[:, None] * kt / den ** 2
+        # s = sum p^- k^2 + r
+        dpm += ds[:, None] * kt * kt
+        dkt += 2.0 * ds[:, None] * pm * kt
+        dr_t += ds
+        # p^- = a^2 p + Qn
+        Pb = (at * at)[:, None] * dpm
+        da_t += 2.0 * at * np.einsum("ni,ni->n", dpm, p_prev)
+        dqn[:, t] = dpm.sum(axis=-1)
+        dkk[:, t], dr[:, t], da[:, t] = dkt, dr_t, da_t
+    return {
+        "dq": dq.reshape(*lead, L, dk),
+        "dk": dkk.reshape(*lead, L, dk),
+        "dv": dvv.reshape(*lead, L, dv),
+        "dr": dr.reshape(*lead, L),
+        "da": da.reshape(*lead, L),
+        "dqn": dqn.reshape(*lead, L),
+        "dS0": G.reshape(*lead, dk, dv),
+        "dp0": Pb.reshape(*lead, dk),
     }

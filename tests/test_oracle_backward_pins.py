@@ -1,8 +1,9 @@
-"""Pins of the float64 backward of the gated delta rule (oracle/backward.py) — CPU only.
+"""Pins of the float64 backward of the gated delta rule and diagonal-Kalman scans (oracle/backward.py), CPU.
 
 The backward is checked against routes that do not use its reverse recurrence: central finite differences
-of the forward oracle for every input, and the closed form of the scan when nothing is written (beta = 0,
-so S_t = A_t S_0 and every output is linear in S_0 and q).  Shapes use d_k != d_v, q != k, gates below one
+of the forward oracle for every input, the closed form of the delta scan when nothing is written (beta = 0,
+so S_t = A_t S_0 and every output is linear in S_0 and q), a one-token derivation, and the closed form of
+the diagonal variances at a = 1, Q = 0.  Shapes use d_k != d_v, q != k, gates below one
 and a non-zero start state, so that a transposed product, a missing decay or a dropped path through the
 residual fails.
 """
@@ -10,8 +11,8 @@ residual fails.
 import numpy as np
 import pytest
 
-from oracle import scan_delta
-from oracle.backward import scan_delta_backward
+from oracle import scan_delta, scan_kalman_diag
+from oracle.backward import scan_delta_backward, scan_kalman_diag_backward
 
 
 def _inputs(seed, heads, L, dk, dv):
@@ -87,3 +88,63 @@ def test_backward_of_a_single_token_by_hand():
     np.testing.assert_allclose(g["dv"][0], b * (q @ k) * dO, rtol=1e-13)
     np.testing.assert_allclose(g["dbeta"][0], (q @ k) * (v @ dO), rtol=1e-13)
     np.testing.assert_allclose(g["dk"][0], b * (v @ dO) * q, rtol=1e-13)
+
+
+# ----------------------------------------------------------------------------- diagonal Kalman
+
+
+def _diag_inputs(seed, heads, L, dk, dv):
+    rng = np.random.default_rng(seed)
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    x = {
+        "q": unit(rng.standard_normal((heads, L, dk))),
+        "k": unit(rng.standard_normal((heads, L, dk))) * (1.0 + 0.3 * rng.random((heads, L, 1))),
+        "v": rng.standard_normal((heads, L, dv)),
+        "r": 0.3 + rng.random((heads, L)),
+        "a": 0.6 + 0.39 * rng.random((heads, L)),
+        "qn": 0.05 * rng.random((heads, L)),
+        "S0": 0.5 * rng.standard_normal((heads, dk, dv)),
+        "p0": 0.5 + rng.random((heads, dk)),
+    }
+    up = {"dO": rng.standard_normal((heads, L, dv)), "dm": rng.standard_normal((heads, L)),
+          "dS_L": rng.standard_normal((heads, dk, dv)), "dp_L": rng.standard_normal((heads, dk))}
+    return x, up
+
+
+def _diag_loss(x, up):
+    out = scan_kalman_diag(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S0=x["S0"], p0=x["p0"])
+    return float(np.sum(up["dO"] * out["o"]) + np.sum(up["dm"] * out["m"]) + np.sum(up["dS_L"] * out["S"])
+                 + np.sum(up["dp_L"] * out["p"]))
+
+
+def test_diagonal_kalman_backward_matches_central_differences_for_every_input():
+    x, up = _diag_inputs(11, heads=2, L=8, dk=3, dv=4)
+    g = scan_kalman_diag_backward(x["q"], x["k"], x["v"], x["r"], up["dO"], a=x["a"], qn=x["qn"], S0=x["S0"],
+                                  p0=x["p0"], dm=up["dm"], dS_L=up["dS_L"], dp_L=up["dp_L"])
+    names = {"q": "dq", "k": "dk", "v": "dv", "r": "dr", "a": "da", "qn": "dqn", "S0": "dS0", "p0": "dp0"}
+    h = 1e-6
+    for name, gname in names.items():
+        num = np.zeros_like(x[name])
+        it = np.nditer(x[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {kk: vv.copy() for kk, vv in x.items()}
+            xm = {kk: vv.copy() for kk, vv in x.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            num[idx] = (_diag_loss(xp, up) - _diag_loss(xm, up)) / (2 * h)
+        scale = np.abs(num).max()
+        assert np.abs(g[gname] - num).max() <= 1e-6 * max(scale, 1.0), (name, np.abs(g[gname] - num).max(), scale)
+
+
+def test_diagonal_kalman_backward_of_the_variances_alone():
+    """With only dp_L upstream and a = 1, Q = 0 the variances have the closed form
+    1 / p_L,i = 1 / p_0,i + sum_t k_ti^2 / r_t, so dp0_i = dp_L,i p_L,i^2 / p_0,i^2 and
+    dr_t = sum_i dp_L,i p_L,i^2 k_ti^2 / r_t^2 (S, o and m do not reach the loss)."""
+    x, up = _diag_inputs(13, heads=1, L=6, dk=3, dv=2)
+    zero = np.zeros_like
+    g = scan_kalman_diag_backward(x["q"], x["k"], x["v"], x["r"], zero(up["dO"]), p0=x["p0"], dp_L=up["dp_L"])
+    pL = scan_kalman_diag(x["q"], x["k"], x["v"], x["r"], p0=x["p0"])["p"][0]
+    p0, k, r, dpL = x["p0"][0], x["k"][0], x["r"][0], up["dp_L"][0]
+    np.testing.assert_allclose(g["dp0"][0], dpL * pL ** 2 / p0 ** 2, rtol=1e-12)
+    np.testing.assert_allclose(g["dr"][0], ((dpL * pL ** 2)[None, :] * k ** 2).sum(-1) / r ** 2, rtol=1e-12)
