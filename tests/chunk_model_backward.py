@@ -1,4 +1,4 @@
-"""Float64 NumPy model of the chunked backward of the gated delta rule.
+"""Float64 NumPy model of the chunked backward of the gated delta rule and the diagonal-Kalman scan.
 
 Test infrastructure, like ``tests/chunk_model.py``: it checks the reverse-mode algebra of the chunk form
 against the token-by-token backward oracle (``oracle.backward``) before any kernel exists, so that a
@@ -22,7 +22,9 @@ Backward of the chunk for upstream dO, dm and dS_C, every product a dense matrix
     dG = d(K G^T)^T K + d(Q G^T)^T Q + diag(r) E dS_C^T,  dbeta_j = k_j . dG_j
 and the gate terms collect in log space: dell_i = A_i dA_i + sum_j Gam_ij dGam_ij - sum_i' Gam_i'i dGam_i'i
 - r_i dr_i (plus A_C dA_C + sum_j r_j dr_j at i = n - 1), d log a_m = sum_{i >= m} dell_i, da = d log a / a.
-The chunk's dS0 is the previous chunk's dS_C.
+The chunk's dS0 is the previous chunk's dS_C.  For the diagonal variant G holds the Kalman gains; dG then
+runs back through the per-token variance recursion that made them (sequential within a chunk, as in the
+forward), with the variance adjoint carried from chunk to chunk.
 """
 
 import numpy as np
@@ -34,6 +36,79 @@ def _gates(a_chunk):
     return ell, np.exp(ell), gam
 
 
+def _wy_chunk_backward(Qc, Kc, Vc, G, ac, S0c, dOc, dmc, dS):
+    """Backward of one chunk of the generalised WY form for gains G (rows g_j) and surprise
+    m_j = ||g_j|| ||e_j||.  Returns dQ, dK (through the products only), dV, dG, d log a, dS0."""
+    n, dk = Kc.shape
+    ell, A, gam = _gates(ac)
+    AC = A[-1]
+    rr = AC / A
+    KG, QG = Kc @ G.T, Qc @ G.T
+    N = np.tril(KG * gam, -1)
+    T = np.linalg.inv(np.eye(n) + N)
+    Mm = np.tril(QG * gam)
+    AT = Mm @ T
+    KS, QS = Kc @ S0c, Qc @ S0c
+    R = Vc - A[:, None] * KS
+    E = T @ R
+    W = (G * rr[:, None]).T                                   # d_k x n
+    # S_C = A_C S0 + W E
+    dS0 = AC * dS
+    dAC = np.sum(dS * S0c)
+    dW = dS @ E.T
+    dE = W.T @ dS
+    # surprise m_j = ||g_j|| ||e_j||
+    gn, en = np.linalg.norm(G, axis=1), np.linalg.norm(E, axis=1)
+    dG = np.zeros_like(G)
+    nz = en > 0
+    dE[nz] += (dmc * gn)[nz, None] * E[nz] / en[nz, None]
+    nzg = gn > 0
+    dG[nzg] += (dmc * en)[nzg, None] * G[nzg] / gn[nzg, None]
+    # O = diag(A) Q S0 + AT R
+    dA = np.sum(dOc * QS, axis=1)
+    dQS = A[:, None] * dOc
+    dQc = dQS @ S0c.T
+    dS0 += Qc.T @ dQS
+    dAT = dOc @ R.T
+    dR = AT.T @ dOc
+    # E = T R
+    dR += T.T @ dE
+    dT = dE @ R.T
+    # AT = M T
+    dM = np.tril(dAT @ T.T)
+    dT += Mm.T @ dAT
+    # T = (I + N)^-1
+    dN = np.tril(-T.T @ dT @ T.T, -1)
+    dKG = dN * gam
+    dQG = dM * gam
+    dGam = dN * KG + dM * QG
+    # R = V - diag(A) K S0
+    dVc = dR
+    dA -= np.sum(dR * KS, axis=1)
+    dKS = -A[:, None] * dR
+    dKc = dKS @ S0c.T
+    dS0 += Kc.T @ dKS
+    # K G^T, Q G^T, W = G^T diag(r)
+    dKc += dKG @ G
+    dQc += dQG @ G
+    dG += dKG.T @ Kc + dQG.T @ Qc + rr[:, None] * dW.T
+    drr = np.sum(G * dW.T, axis=1)
+    # gates in log space
+    dell = A * dA + np.sum(gam * dGam, axis=1) - np.sum(gam * dGam, axis=0) - rr * drr
+    dell[-1] += AC * dAC + np.sum(rr * drr)
+    dloga = np.cumsum(dell[::-1])[::-1]
+    return dQc, dKc, dVc, dG, dloga, dS0
+
+
+def _wy_chunk_forward(Kc, Vc, G, ac, S):
+    n = Kc.shape[0]
+    _, A, gam = _gates(ac)
+    N = np.tril((Kc @ G.T) * gam, -1)
+    T = np.linalg.inv(np.eye(n) + N)
+    E = T @ (Vc - A[:, None] * (Kc @ S))
+    return A[-1] * S + (G * (A[-1] / A)[:, None]).T @ E
+
+
 def chunk_delta_backward(q, k, v, beta, a, C, dO, S0=None, dm=None, dS_L=None):
     """One head: q, k [L, dk], v [L, dv], beta, a [L] (a > 0), dO [L, dv], dm [L] or None, dS_L [dk, dv] or
     None.  Returns dq, dk, dv, dbeta, da, dS0 from the chunk form with chunks of C tokens."""
@@ -42,88 +117,80 @@ def chunk_delta_backward(q, k, v, beta, a, C, dO, S0=None, dm=None, dS_L=None):
     dm = np.zeros(L) if dm is None else np.asarray(dm, float)
     S = np.zeros((dk, dv)) if S0 is None else np.array(S0, float)
     chunks = [(c0, min(c0 + C, L)) for c0 in range(0, L, C)]
-    # forward in chunk form, keeping each chunk's start state
     starts = []
     for c0, c1 in chunks:
         starts.append(S.copy())
-        Kc, Vc, bc = k[c0:c1], v[c0:c1], beta[c0:c1]
-        n = c1 - c0
-        _, A, gam = _gates(a[c0:c1])
-        G = bc[:, None] * Kc
-        N = np.tril((Kc @ G.T) * gam, -1)
-        T = np.linalg.inv(np.eye(n) + N)
-        E = T @ (Vc - A[:, None] * (Kc @ S))
-        S = A[-1] * S + (G * (A[-1] / A)[:, None]).T @ E
+        S = _wy_chunk_forward(k[c0:c1], v[c0:c1], beta[c0:c1, None] * k[c0:c1], a[c0:c1], S)
     dS = np.zeros((dk, dv)) if dS_L is None else np.array(dS_L, float)
     dq, dkk, dvv = np.zeros((L, dk)), np.zeros((L, dk)), np.zeros((L, dv))
     dbeta, da = np.zeros(L), np.zeros(L)
     for (c0, c1), S0c in reversed(list(zip(chunks, starts))):
-        Qc, Kc, Vc, bc, ac = q[c0:c1], k[c0:c1], v[c0:c1], beta[c0:c1], a[c0:c1]
-        dOc, dmc = dO[c0:c1], dm[c0:c1]
-        n = c1 - c0
-        ell, A, gam = _gates(ac)
-        AC = A[-1]
-        rr = AC / A
-        G = bc[:, None] * Kc
-        KG, QG = Kc @ G.T, Qc @ G.T
-        N = np.tril(KG * gam, -1)
-        T = np.linalg.inv(np.eye(n) + N)
-        Mm = np.tril(QG * gam)
-        AT = Mm @ T
-        KS, QS = Kc @ S0c, Qc @ S0c
-        R = Vc - A[:, None] * KS
-        E = T @ R
-        W = (G * rr[:, None]).T                               # d_k x n
-        # S_C = A_C S0 + W E
-        dS0 = AC * dS
-        dAC = np.sum(dS * S0c)
-        dW = dS @ E.T
-        dE = W.T @ dS
-        # surprise m_j = beta_j ||k_j|| ||e_j||
-        kn, en = np.linalg.norm(Kc, axis=1), np.linalg.norm(E, axis=1)
-        dKc = np.zeros((n, dk))
-        dbc = dmc * kn * en
-        nz = en > 0
-        dE[nz] += (dmc * bc * kn)[nz, None] * E[nz] / en[nz, None]
-        nzk = kn > 0
-        dKc[nzk] += (dmc * bc * en)[nzk, None] * Kc[nzk] / kn[nzk, None]
-        # O = diag(A) Q S0 + AT R
-        dA = np.sum(dOc * QS, axis=1)
-        dQS = A[:, None] * dOc
-        dQc = dQS @ S0c.T
-        dS0 += Qc.T @ dQS
-        dAT = dOc @ R.T
-        dR = AT.T @ dOc
-        # E = T R
-        dR += T.T @ dE
-        dT = dE @ R.T
-        # AT = M T
-        dM = np.tril(dAT @ T.T)
-        dT += Mm.T @ dAT
-        # T = (I + N)^-1
-        dN = np.tril(-T.T @ dT @ T.T, -1)
-        dKG = dN * gam
-        dQG = dM * gam
-        dGam = dN * KG + dM * QG
-        # R = V - diag(A) K S0
-        dVc = dR
-        dA -= np.sum(dR * KS, axis=1)
-        dKS = -A[:, None] * dR
-        dKc += dKS @ S0c.T
-        dS0 += Kc.T @ dKS
-        # K G^T, Q G^T, W = G^T diag(r), G = diag(beta) K
-        dKc += dKG @ G
-        dQc += dQG @ G
-        dG = dKG.T @ Kc + dQG.T @ Qc + rr[:, None] * dW.T
-        drr = np.sum(G * dW.T, axis=1)
-        dbc += np.sum(Kc * dG, axis=1)
-        dKc += bc[:, None] * dG
-        # gates in log space
-        dell = A * dA + np.sum(gam * dGam, axis=1) - np.sum(gam * dGam, axis=0) - rr * drr
-        dell[-1] += AC * dAC + np.sum(rr * drr)
-        dloga = np.cumsum(dell[::-1])[::-1]
-        dq[c0:c1], dkk[c0:c1], dvv[c0:c1] = dQc, dKc, dVc
-        dbeta[c0:c1] = dbc
-        da[c0:c1] = dloga / ac
-        dS = dS0
+        Kc, bc = k[c0:c1], beta[c0:c1]
+        dQc, dKc, dVc, dG, dloga, dS = _wy_chunk_backward(q[c0:c1], Kc, v[c0:c1], bc[:, None] * Kc, a[c0:c1], S0c,
+                                                          dO[c0:c1], dm[c0:c1], dS)
+        # G = diag(beta) K
+        dq[c0:c1], dvv[c0:c1] = dQc, dVc
+        dkk[c0:c1] = dKc + bc[:, None] * dG
+        dbeta[c0:c1] = np.sum(Kc * dG, axis=1)
+        da[c0:c1] = dloga / a[c0:c1]
     return {"dq": dq, "dk": dkk, "dv": dvv, "dbeta": dbeta, "da": da, "dS0": dS}
+
+
+def chunk_diag_backward(q, k, v, r, a, qn, C, dO, S0=None, p0=None, dm=None, dS_L=None, dp_L=None):
+    """Diagonal Kalman, one head: the chunk backward above for the gains, then the per-token adjoint of
+    the variance recursion that made them (sequential within the chunk, like the forward's variances; the
+    variance adjoint is carried across chunks).  Returns dq, dk, dv, dr, da, dqn, dS0, dp0."""
+    L, dk = k.shape
+    dv = v.shape[1]
+    dm = np.zeros(L) if dm is None else np.asarray(dm, float)
+    S = np.zeros((dk, dv)) if S0 is None else np.array(S0, float)
+    p = np.ones(dk) if p0 is None else np.array(p0, float)
+    chunks = [(c0, min(c0 + C, L)) for c0 in range(0, L, C)]
+    starts, pstarts, gains = [], [], []
+    for c0, c1 in chunks:
+        starts.append(S.copy())
+        pstarts.append(p.copy())
+        G = np.zeros((c1 - c0, dk))
+        for i, t in enumerate(range(c0, c1)):
+            pm = a[t] ** 2 * p + qn[t]
+            G[i] = pm * k[t] / (pm @ (k[t] ** 2) + r[t])
+            p = pm * r[t] / (r[t] + pm * k[t] ** 2)
+        gains.append(G)
+        S = _wy_chunk_forward(k[c0:c1], v[c0:c1], G, a[c0:c1], S)
+    dS = np.zeros((dk, dv)) if dS_L is None else np.array(dS_L, float)
+    Pb = np.zeros(dk) if dp_L is None else np.array(dp_L, float)
+    out = {key: np.zeros(shape) for key, shape in
+           (("dq", (L, dk)), ("dk", (L, dk)), ("dv", (L, dv)), ("dr", L), ("da", L), ("dqn", L))}
+    for ci in range(len(chunks) - 1, -1, -1):
+        c0, c1 = chunks[ci]
+        G = gains[ci]
+        dQc, dKc, dVc, dG, dloga, dS = _wy_chunk_backward(q[c0:c1], k[c0:c1], v[c0:c1], G, a[c0:c1], starts[ci],
+                                                          dO[c0:c1], dm[c0:c1], dS)
+        out["dq"][c0:c1], out["dv"][c0:c1] = dQc, dVc
+        da_c = dloga / a[c0:c1]
+        # the variance recursion of this chunk, replayed to recover p before each token, then reversed
+        pp = [pstarts[ci]]
+        for t in range(c0, c1 - 1):
+            pm = a[t] ** 2 * pp[-1] + qn[t]
+            pp.append(pm * r[t] / (r[t] + pm * k[t] ** 2))
+        for i in range(c1 - c0 - 1, -1, -1):
+            t = c0 + i
+            kt, pprev = k[t], pp[i]
+            pm = a[t] ** 2 * pprev + qn[t]
+            st = pm @ (kt ** 2) + r[t]
+            g = pm * kt / st
+            dg = dG[i]
+            dpm = dg * kt / st
+            dKc[i] += dg * pm / st
+            ds = -(dg @ g) / st
+            den = r[t] + pm * kt ** 2
+            dpm += Pb * r[t] ** 2 / den ** 2 + ds * kt ** 2
+            out["dr"][t] += np.sum(Pb * (pm * kt) ** 2 / den ** 2) + ds
+            dKc[i] += -2.0 * Pb * pm * pm * r[t] * kt / den ** 2 + 2.0 * ds * pm * kt
+            Pb = a[t] ** 2 * dpm
+            da_c[i] += 2.0 * a[t] * (dpm @ pprev)
+            out["dqn"][t] = dpm.sum()
+        out["dk"][c0:c1] = dKc
+        out["da"][c0:c1] = da_c
+    out["dS0"], out["dp0"] = dS, Pb
+    return out
