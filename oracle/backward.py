@@ -39,6 +39,12 @@ adjoint Pb = dLoss/dp next to G: from g, dp^- = dg o k / s, ds = -(dg . g) / s, 
 the projection p = p^- r / den (den = r + p^- k^2), dp^- += Pb r^2 / den^2, dr += sum Pb (p^- k)^2 / den^2,
 dk -= 2 Pb (p^-)^2 r k / den^2; from s, dp^- += ds k^2, dk += 2 ds p^- k, dr += ds; and through the
 propagation Pb_{t-1} = a_t^2 dp^-, da_t += 2 a_t (dp^- . p_{t-1}), dQn_t = sum dp^-.
+
+The isotropic variant (reading R12) carries one scalar c: c^- = a^2 c + Qn, s = c^- ||k||^2 + r,
+g = (c^- / s) k, c = d_k c^- r / (d_k r + c^- ||k||^2); and the full-covariance variant carries P:
+P^- = a^2 P + Qn I, u = P^- k, s = k^T u + r, g = u / s, P = P^- - u u^T / s (the symmetric form the forward
+oracle uses).  Their backwards follow the same pattern: the memory part gives dg, which runs back through
+the gain and the uncertainty update, and the uncertainty adjoint is carried to the previous token.
 """
 
 from __future__ import annotations
@@ -47,7 +53,8 @@ import numpy as np
 
 from .scan import _f64, _flatten_inputs, _per_token, _read
 
-__all__ = ["scan_delta_backward", "scan_kalman_diag_backward"]
+__all__ = ["scan_delta_backward", "scan_kalman_diag_backward", "scan_kalman_iso_backward",
+           "scan_kalman_full_backward"]
 
 
 def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None):
@@ -194,3 +201,148 @@ def scan_kalman_diag_backward(q, k, v, r, dO, a=None, qn=None, S0=None, p0=None,
         "dS0": G.reshape(*lead, dk, dv),
         "dp0": Pb.reshape(*lead, dk),
     }
+
+
+def _memory_step_backward(G, g, e, kt, qt, S_t, S_prev, at, dOt, dmt):
+    """The memory part of one token's backward for a gain g (rows of heads): the read, the write
+    S_t = a S_{t-1} + g e^T, the residual e = v - a S_{t-1}^T k and the surprise ||g|| ||e||.
+    G enters as dLoss/dS_t without the read; returns (G_{t-1}, dq, dv, dk through the residual, da, dg)."""
+    G = G + qt[:, :, None] * dOt[:, None, :]
+    dq = np.einsum("nij,nj->ni", S_t, dOt)
+    gn = np.linalg.norm(g, axis=-1)
+    en = np.linalg.norm(e, axis=-1)
+    e_dir = np.where(en[:, None] > 0, e / np.where(en > 0, en, 1.0)[:, None], 0.0)
+    g_dir = np.where(gn[:, None] > 0, g / np.where(gn > 0, gn, 1.0)[:, None], 0.0)
+    de = _read(G, g) + (dmt * gn)[:, None] * e_dir
+    dg = np.einsum("nij,nj->ni", G, e) + (dmt * en)[:, None] * g_dir
+    dk = -at[:, None] * np.einsum("nij,nj->ni", S_prev, de)
+    da = np.einsum("nij,nij->n", G, S_prev) - np.einsum("ni,nij,nj->n", kt, S_prev, de)
+    G = at[:, None, None] * G - at[:, None, None] * kt[:, :, None] * de[:, None, :]
+    return G, dq, de, dk, da, dg
+
+
+def scan_kalman_iso_backward(q, k, v, r, dO, a=None, qn=None, S0=None, c0=None, dm=None, dS_L=None, dc_L=None):
+    """Gradients of the isotropic-Kalman scan (``oracle.scan.scan_kalman_iso``).  c0 [...] (None = 1) and
+    upstream dc_L [...] (None = 0) are per head.  Returns dq, dk, dv, dr, da, dqn, dS0 and dc0."""
+    lead, n, L, dk, dv, q, k, v = _flatten_inputs(q, k, v)
+    r = _per_token(r, n, L, 1.0)
+    a = _per_token(a, n, L, 1.0)
+    qn = _per_token(qn, n, L, 0.0)
+    dO = _f64(dO).reshape(n, L, dv)
+    dm = _per_token(dm, n, L, 0.0)
+    S = np.zeros((n, dk, dv)) if S0 is None else _f64(S0).reshape(n, dk, dv).copy()
+    c = np.ones(n) if c0 is None else _f64(c0).reshape(n).copy()
+    states, cs = np.zeros((n, L + 1, dk, dv)), np.zeros((n, L + 1))
+    states[:, 0], cs[:, 0] = S, c
+    res, gains = np.zeros((n, L, dv)), np.zeros((n, L, dk))
+    for t in range(L):
+        kt, at = k[:, t], a[:, t]
+        cm = at * at * c + qn[:, t]
+        kk = np.einsum("ni,ni->n", kt, kt)
+        g = (cm / (cm * kk + r[:, t]))[:, None] * kt
+        c = dk * cm * r[:, t] / (dk * r[:, t] + cm * kk)
+        S_pred = at[:, None, None] * S
+        e = v[:, t] - _read(S_pred, kt)
+        S = S_pred + g[:, :, None] * e[:, None, :]
+        states[:, t + 1], cs[:, t + 1], res[:, t], gains[:, t] = S, c, e, g
+    G = np.zeros((n, dk, dv)) if dS_L is None else _f64(dS_L).reshape(n, dk, dv).copy()
+    cb = np.zeros(n) if dc_L is None else _f64(dc_L).reshape(n).copy()
+    out = {key: np.zeros(shape) for key, shape in
+           (("dq", (n, L, dk)), ("dk", (n, L, dk)), ("dv", (n, L, dv)), ("dr", (n, L)), ("da", (n, L)),
+            ("dqn", (n, L)))}
+    for t in range(L - 1, -1, -1):
+        kt, at, rt, c_prev = k[:, t], a[:, t], r[:, t], cs[:, t]
+        G, dq, de, dkt, da_t, dg = _memory_step_backward(G, gains[:, t], res[:, t], kt, q[:, t], states[:, t + 1],
+                                                         states[:, t], at, dO[:, t], dm[:, t])
+        cm = at * at * c_prev + qn[:, t]
+        kk = np.einsum("ni,ni->n", kt, kt)
+        st = cm * kk + rt
+        beta = cm / st
+        # g = beta k, beta = c^- / s, s = c^- kk + r
+        dbeta = np.einsum("ni,ni->n", kt, dg)
+        dkt = dkt + beta[:, None] * dg
+        dcm = dbeta / st
+        ds = -dbeta * cm / st ** 2
+        dcm = dcm + ds * kk
+        dkk = ds * cm
+        dr_t = ds
+        # c = d c^- r / (d r + c^- kk)
+        den = dk * rt + cm * kk
+        dcm = dcm + cb * (dk * rt) ** 2 / den ** 2
+        dr_t = dr_t + cb * dk * cm * cm * kk / den ** 2
+        dkk = dkk - cb * dk * cm * cm * rt / den ** 2
+        dkt = dkt + 2.0 * dkk[:, None] * kt
+        # c^- = a^2 c + Qn
+        cb = at * at * dcm
+        da_t = da_t + 2.0 * at * c_prev * dcm
+        out["dq"][:, t], out["dk"][:, t], out["dv"][:, t] = dq, dkt, de
+        out["dr"][:, t], out["da"][:, t], out["dqn"][:, t] = dr_t, da_t, dcm
+    res_out = {key: val.reshape(*lead, *val.shape[1:]) for key, val in out.items()}
+    res_out["dS0"] = G.reshape(*lead, dk, dv)
+    res_out["dc0"] = cb.reshape(lead)
+    return res_out
+
+
+def scan_kalman_full_backward(q, k, v, r, dO, a=None, qn=None, S0=None, P0=None, dm=None, dS_L=None, dP_L=None):
+    """Gradients of the full-covariance Kalman scan (``oracle.scan.scan_kalman_full``).  P0 [..., d_k, d_k]
+    (None = I), upstream dP_L [..., d_k, d_k] (None = 0).  Returns dq, dk, dv, dr, da, dqn, dS0 and dP0 (the
+    gradient with respect to every entry of P0, as the forward uses it)."""
+    lead, n, L, dk, dv, q, k, v = _flatten_inputs(q, k, v)
+    r = _per_token(r, n, L, 1.0)
+    a = _per_token(a, n, L, 1.0)
+    qn = _per_token(qn, n, L, 0.0)
+    dO = _f64(dO).reshape(n, L, dv)
+    dm = _per_token(dm, n, L, 0.0)
+    eye = np.eye(dk)
+    S = np.zeros((n, dk, dv)) if S0 is None else _f64(S0).reshape(n, dk, dv).copy()
+    P = np.broadcast_to(eye, (n, dk, dk)).copy() if P0 is None else _f64(P0).reshape(n, dk, dk).copy()
+    states, Ps = np.zeros((n, L + 1, dk, dv)), np.zeros((n, L + 1, dk, dk))
+    states[:, 0], Ps[:, 0] = S, P
+    res, gains = np.zeros((n, L, dv)), np.zeros((n, L, dk))
+    for t in range(L):
+        kt, at = k[:, t], a[:, t]
+        Pm = (at * at)[:, None, None] * P + qn[:, t, None, None] * eye
+        u = np.einsum("nij,nj->ni", Pm, kt)
+        st = np.einsum("ni,ni->n", kt, u) + r[:, t]
+        g = u / st[:, None]
+        P = Pm - u[:, :, None] * u[:, None, :] / st[:, None, None]
+        S_pred = at[:, None, None] * S
+        e = v[:, t] - _read(S_pred, kt)
+        S = S_pred + g[:, :, None] * e[:, None, :]
+        states[:, t + 1], Ps[:, t + 1], res[:, t], gains[:, t] = S, P, e, g
+    G = np.zeros((n, dk, dv)) if dS_L is None else _f64(dS_L).reshape(n, dk, dv).copy()
+    Pb = np.zeros((n, dk, dk)) if dP_L is None else _f64(dP_L).reshape(n, dk, dk).copy()
+    out = {key: np.zeros(shape) for key, shape in
+           (("dq", (n, L, dk)), ("dk", (n, L, dk)), ("dv", (n, L, dv)), ("dr", (n, L)), ("da", (n, L)),
+            ("dqn", (n, L)))}
+    for t in range(L - 1, -1, -1):
+        kt, at, rt, P_prev = k[:, t], a[:, t], r[:, t], Ps[:, t]
+        G, dq, de, dkt, da_t, dg = _memory_step_backward(G, gains[:, t], res[:, t], kt, q[:, t], states[:, t + 1],
+                                                         states[:, t], at, dO[:, t], dm[:, t])
+        Pm = (at * at)[:, None, None] * P_prev + qn[:, t, None, None] * eye
+        u = np.einsum("nij,nj->ni", Pm, kt)
+        st = np.einsum("ni,ni->n", kt, u) + rt
+        g = u / st[:, None]
+        # g = u / s
+        du = dg / st[:, None]
+        ds = -np.einsum("ni,ni->n", dg, g) / st
+        # P = P^- - u u^T / s
+        dPm = Pb.copy()
+        du = du - np.einsum("nij,nj->ni", Pb + np.swapaxes(Pb, 1, 2), u) / st[:, None]
+        ds = ds + np.einsum("ni,nij,nj->n", u, Pb, u) / st ** 2
+        # s = k^T u + r
+        dkt = dkt + ds[:, None] * u
+        du = du + ds[:, None] * kt
+        dr_t = ds
+        # u = P^- k
+        dPm = dPm + du[:, :, None] * kt[:, None, :]
+        dkt = dkt + np.einsum("nji,nj->ni", Pm, du)
+        # P^- = a^2 P + Qn I
+        Pb = (at * at)[:, None, None] * dPm
+        da_t = da_t + 2.0 * at * np.einsum("nij,nij->n", dPm, P_prev)
+        out["dq"][:, t], out["dk"][:, t], out["dv"][:, t] = dq, dkt, de
+        out["dr"][:, t], out["da"][:, t], out["dqn"][:, t] = dr_t, da_t, np.trace(dPm, axis1=1, axis2=2)
+    res_out = {key: val.reshape(*lead, *val.shape[1:]) for key, val in out.items()}
+    res_out["dS0"] = G.reshape(*lead, dk, dv)
+    res_out["dP0"] = Pb.reshape(*lead, dk, dk)
+    return res_out

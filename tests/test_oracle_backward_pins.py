@@ -1,4 +1,4 @@
-"""Pins of the float64 backward of the gated delta rule and diagonal-Kalman scans (oracle/backward.py), CPU.
+"""Pins of the float64 backwards of the four scans (oracle/backward.py), CPU only.
 
 The backward is checked against routes that do not use its reverse recurrence: central finite differences
 of the forward oracle for every input, the closed form of the delta scan when nothing is written (beta = 0,
@@ -11,8 +11,9 @@ residual fails.
 import numpy as np
 import pytest
 
-from oracle import scan_delta, scan_kalman_diag
-from oracle.backward import scan_delta_backward, scan_kalman_diag_backward
+from oracle import scan_delta, scan_kalman_diag, scan_kalman_full, scan_kalman_iso
+from oracle.backward import (scan_delta_backward, scan_kalman_diag_backward, scan_kalman_full_backward,
+                             scan_kalman_iso_backward)
 
 
 def _inputs(seed, heads, L, dk, dv):
@@ -148,3 +149,87 @@ def test_diagonal_kalman_backward_of_the_variances_alone():
     p0, k, r, dpL = x["p0"][0], x["k"][0], x["r"][0], up["dp_L"][0]
     np.testing.assert_allclose(g["dp0"][0], dpL * pL ** 2 / p0 ** 2, rtol=1e-12)
     np.testing.assert_allclose(g["dr"][0], ((dpL * pL ** 2)[None, :] * k ** 2).sum(-1) / r ** 2, rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- isotropic and full Kalman
+
+
+def _central_differences(loss, x, names):
+    h = 1e-6
+    out = {}
+    for name in names:
+        num = np.zeros_like(x[name])
+        it = np.nditer(x[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {kk: vv.copy() for kk, vv in x.items()}
+            xm = {kk: vv.copy() for kk, vv in x.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            num[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        out[name] = num
+    return out
+
+
+def _assert_close(g, num, names):
+    for name, gname in names.items():
+        scale = np.abs(num[name]).max()
+        err = np.abs(g[gname] - num[name]).max()
+        assert err <= 1e-6 * max(scale, 1.0), (name, err, scale)
+
+
+def test_isotropic_kalman_backward_matches_central_differences_for_every_input():
+    x, up = _diag_inputs(17, heads=2, L=8, dk=3, dv=4)
+    x["c0"] = 0.5 + np.random.default_rng(18).random(2)
+    del x["p0"]
+    dcL = np.random.default_rng(19).standard_normal(2)
+
+    def loss(xx):
+        out = scan_kalman_iso(xx["q"], xx["k"], xx["v"], xx["r"], a=xx["a"], qn=xx["qn"], S0=xx["S0"], c0=xx["c0"])
+        return float(np.sum(up["dO"] * out["o"]) + np.sum(up["dm"] * out["m"]) + np.sum(up["dS_L"] * out["S"])
+                     + np.sum(dcL * out["c"]))
+
+    g = scan_kalman_iso_backward(x["q"], x["k"], x["v"], x["r"], up["dO"], a=x["a"], qn=x["qn"], S0=x["S0"],
+                                 c0=x["c0"], dm=up["dm"], dS_L=up["dS_L"], dc_L=dcL)
+    names = {"q": "dq", "k": "dk", "v": "dv", "r": "dr", "a": "da", "qn": "dqn", "S0": "dS0", "c0": "dc0"}
+    _assert_close(g, _central_differences(loss, x, names), names)
+
+
+def test_full_kalman_backward_matches_central_differences_for_every_input():
+    x, up = _diag_inputs(21, heads=2, L=7, dk=3, dv=4)
+    rng = np.random.default_rng(22)
+    B = rng.standard_normal((2, 3, 3)) / 3
+    x["P0"] = 0.5 * np.eye(3) + B @ np.swapaxes(B, 1, 2)
+    del x["p0"]
+    dPL = rng.standard_normal((2, 3, 3))
+
+    def loss(xx):
+        out = scan_kalman_full(xx["q"], xx["k"], xx["v"], xx["r"], a=xx["a"], qn=xx["qn"], S0=xx["S0"], P0=xx["P0"])
+        return float(np.sum(up["dO"] * out["o"]) + np.sum(up["dm"] * out["m"]) + np.sum(up["dS_L"] * out["S"])
+                     + np.sum(dPL * out["P"]))
+
+    g = scan_kalman_full_backward(x["q"], x["k"], x["v"], x["r"], up["dO"], a=x["a"], qn=x["qn"], S0=x["S0"],
+                                  P0=x["P0"], dm=up["dm"], dS_L=up["dS_L"], dP_L=dPL)
+    names = {"q": "dq", "k": "dk", "v": "dv", "r": "dr", "a": "da", "qn": "dqn", "S0": "dS0", "P0": "dP0"}
+    _assert_close(g, _central_differences(loss, x, names), names)
+
+
+def test_full_kalman_backward_equals_diagonal_backward_on_one_hot_keys():
+    """One-hot keys and a diagonal P0 keep the full covariance diagonal, and the two filters coincide
+    (a pin of the forwards); their gradients with respect to q, v, r, a, Qn, S0 and the start variances
+    must then coincide as well."""
+    rng = np.random.default_rng(23)
+    L, dk, dv = 9, 4, 3
+    idx = rng.integers(0, dk, L)
+    k = np.eye(dk)[idx][None]
+    q = rng.standard_normal((1, L, dk))
+    v = rng.standard_normal((1, L, dv))
+    r, a, qn = 0.3 + rng.random((1, L)), 0.6 + 0.39 * rng.random((1, L)), 0.05 * rng.random((1, L))
+    S0, p0 = rng.standard_normal((1, dk, dv)), 0.5 + rng.random((1, dk))
+    dO, dm, dSL = rng.standard_normal((1, L, dv)), rng.standard_normal((1, L)), rng.standard_normal((1, dk, dv))
+    gf = scan_kalman_full_backward(q, k, v, r, dO, a=a, qn=qn, S0=S0, P0=p0[:, :, None] * np.eye(dk), dm=dm,
+                                   dS_L=dSL)
+    gd = scan_kalman_diag_backward(q, k, v, r, dO, a=a, qn=qn, S0=S0, p0=p0, dm=dm, dS_L=dSL)
+    for key in ("dq", "dv", "dr", "da", "dqn", "dS0"):
+        np.testing.assert_allclose(gf[key], gd[key], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(np.diagonal(gf["dP0"], axis1=1, axis2=2), gd["dp0"], rtol=1e-10, atol=1e-12)
