@@ -194,3 +194,39 @@ def chunk_diag_backward(q, k, v, r, a, qn, C, dO, S0=None, p0=None, dm=None, dS_
         out["da"][c0:c1] = da_c
     out["dS0"], out["dp0"] = dS, Pb
     return out
+
+
+def chunk_iso_backward(q, k, v, r, a, qn, C, dO, S0=None, c0=1.0, dm=None, dS_L=None, dc_L=0.0):
+    """Isotropic Kalman, one head: the delta chunk backward for beta_t = c^-_t / (c^-_t ||k_t||^2 + r_t), then
+    the per-token adjoint of the uncertainty scalar's recursion.  Returns dq, dk, dv, dr, da, dqn, dS0, dc0."""
+    L, dk = k.shape
+    kk = np.sum(k * k, axis=1)
+    c = float(c0)
+    cprev, beta = np.zeros(L), np.zeros(L)
+    for t in range(L):
+        cprev[t] = c
+        cm = a[t] ** 2 * c + qn[t]
+        beta[t] = cm / (cm * kk[t] + r[t])
+        c = dk * cm * r[t] / (dk * r[t] + cm * kk[t])
+    g = chunk_delta_backward(q, k, v, beta, a, C, dO, S0=S0, dm=dm, dS_L=dS_L)
+    out = {"dq": g["dq"], "dk": g["dk"].copy(), "dv": g["dv"], "da": g["da"].copy(), "dS0": g["dS0"],
+           "dr": np.zeros(L), "dqn": np.zeros(L)}
+    cb = float(dc_L)
+    for t in range(L - 1, -1, -1):
+        cm = a[t] ** 2 * cprev[t] + qn[t]
+        st = cm * kk[t] + r[t]
+        db = g["dbeta"][t]
+        dcm = db / st - db * cm / st ** 2 * kk[t]
+        dkk = -db * cm / st ** 2 * cm
+        dr = -db * cm / st ** 2
+        den = dk * r[t] + cm * kk[t]
+        dcm += cb * (dk * r[t]) ** 2 / den ** 2
+        dr += cb * dk * cm * cm * kk[t] / den ** 2
+        dkk -= cb * dk * cm * cm * r[t] / den ** 2
+        out["dk"][t] += 2.0 * dkk * k[t]
+        out["dr"][t] = dr
+        out["dqn"][t] = dcm
+        out["da"][t] += 2.0 * a[t] * cprev[t] * dcm
+        cb = a[t] ** 2 * dcm
+    out["dc0"] = cb
+    return out

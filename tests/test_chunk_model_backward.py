@@ -46,3 +46,24 @@ def test_chunked_diagonal_backward_equals_token_backward(C):
     for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dp0"):
         scale = max(np.abs(ref[key]).max(), 1e-12)
         assert np.abs(got[key] - ref[key]).max() <= 1e-9 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
+
+
+@pytest.mark.parametrize("C", [1, 16, 64])
+def test_chunked_isotropic_backward_equals_token_backward(C):
+    from chunk_model_backward import chunk_iso_backward
+    from oracle.backward import scan_kalman_iso_backward
+    rng = np.random.default_rng(C + 99)
+    L, dk, dv = 75, 5, 4
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q, k = unit(rng.standard_normal((L, dk))), unit(rng.standard_normal((L, dk)))
+    v = rng.standard_normal((L, dv))
+    r = np.log1p(np.exp(rng.standard_normal(L))) + 0.1
+    a = np.exp(-np.log1p(np.exp(rng.standard_normal(L) - 2.0)))
+    qn = np.full(L, 1e-3)
+    S0 = 0.3 * rng.standard_normal((dk, dv))
+    dO, dm, dSL = rng.standard_normal((L, dv)), rng.standard_normal(L), rng.standard_normal((dk, dv))
+    ref = scan_kalman_iso_backward(q, k, v, r, dO, a=a, qn=qn, S0=S0, c0=0.8, dm=dm, dS_L=dSL, dc_L=0.3)
+    got = chunk_iso_backward(q, k, v, r, a, qn, C, dO, S0=S0, c0=0.8, dm=dm, dS_L=dSL, dc_L=0.3)
+    for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dc0"):
+        scale = max(np.abs(ref[key]).max(), 1e-12)
+        assert np.abs(got[key] - ref[key]).max() <= 1e-9 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
