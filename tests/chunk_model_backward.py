@@ -1,4 +1,4 @@
-"""Float64 NumPy model of the chunked backward of the gated delta rule and the diagonal-Kalman scan.
+"""Float64 NumPy model of the chunked backward of the four scans.
 
 Test infrastructure, like ``tests/chunk_model.py``: it checks the reverse-mode algebra of the chunk form
 against the token-by-token backward oracle (``oracle.backward``) before any kernel exists, so that a
@@ -24,7 +24,12 @@ and the gate terms collect in log space: dell_i = A_i dA_i + sum_j Gam_ij dGam_i
 - r_i dr_i (plus A_C dA_C + sum_j r_j dr_j at i = n - 1), d log a_m = sum_{i >= m} dell_i, da = d log a / a.
 The chunk's dS0 is the previous chunk's dS_C.  For the diagonal variant G holds the Kalman gains; dG then
 runs back through the per-token variance recursion that made them (sequential within a chunk, as in the
-forward), with the variance adjoint carried from chunk to chunk.
+forward), with the variance adjoint carried from chunk to chunk; the isotropic variant runs dbeta back through
+its scalar recursion.  For full Kalman dG runs back through the chunk's covariance side: the rank-n update
+P_C = A_C^2 P0 + gamma_C I - G^T diag(w) G, the gains G = Z / D, Z = (L^-1 o Gam) Bt, the inverse
+(dL = -L^-T dLinv L^-T), the LDL of the innovation Gram (dG = L^-T M L^-1 with
+M = strict_lower(L^T dL D^-1) + diag(dD)), the Gram and Bt = diag(A^2) K P0 + diag(gamma) K; the covariance
+adjoint goes to the previous chunk.
 """
 
 import numpy as np
@@ -229,4 +234,139 @@ def chunk_iso_backward(q, k, v, r, a, qn, C, dO, S0=None, c0=1.0, dm=None, dS_L=
         out["da"][t] += 2.0 * a[t] * cprev[t] * dcm
         cb = a[t] ** 2 * dcm
     out["dc0"] = cb
+    return out
+
+
+def _ldl(G):
+    n = G.shape[0]
+    L = np.eye(n)
+    D = np.zeros(n)
+    A = G.copy()
+    for j in range(n):
+        D[j] = A[j, j]
+        L[j + 1:, j] = A[j + 1:, j] / D[j]
+        A[j + 1:, j + 1:] -= np.outer(L[j + 1:, j], L[j + 1:, j]) * D[j]
+    return L, D
+
+
+def ldl_backward(L, D, dL, dD):
+    """Adjoint of G = L D L^T (L unit lower) as a function of the lower triangle of the symmetric G.
+    With X = L^-1 dG L^-T (symmetric), dD = diag(X) and dL = L strict_lower(X) D^-1, so for upstream dL
+    (strict lower) and dD the matrix M = strict_lower(L^T dL D^-1) + diag(dD) gives dG = L^-T M L^-1 over
+    symmetric perturbations; an entry below the diagonal stands for both of its mirror images."""
+    Li = np.linalg.inv(L)
+    M = np.tril(L.T @ np.tril(dL, -1) / D[None, :], -1) + np.diag(dD)
+    Gb = Li.T @ M @ Li
+    return np.tril(Gb + Gb.T, -1) + np.diag(np.diag(Gb))
+
+
+def chunk_full_backward(q, k, v, r, a, qn, C, dO, S0=None, P0=None, dm=None, dS_L=None, dP_L=None):
+    """Full-covariance Kalman, one head: the WY chunk backward for the gains, then the adjoint of the
+    chunk's covariance side (Gram, LDL, L^-1, Z, the rank-n covariance update), with the covariance adjoint
+    carried from chunk to chunk.  P0 symmetric; returns dq, dk, dv, dr, da, dqn, dS0 and dP0 (symmetric)."""
+    L, dk = k.shape
+    dv = v.shape[1]
+    dm = np.zeros(L) if dm is None else np.asarray(dm, float)
+    S = np.zeros((dk, dv)) if S0 is None else np.array(S0, float)
+    P = np.eye(dk) if P0 is None else np.array(P0, float)
+    eye = np.eye(dk)
+    chunks = [(c0, min(c0 + C, L)) for c0 in range(0, L, C)]
+
+    def cov_forward(Kc, ac, qnc, rc, P):
+        n = Kc.shape[0]
+        ell, A, gam = _gates(ac)
+        gamma = np.zeros(n)
+        gp = 0.0
+        for i in range(n):
+            gp = ac[i] ** 2 * gp + qnc[i]
+            gamma[i] = gp
+        KP = Kc @ P
+        Bt = (A ** 2)[:, None] * KP + gamma[:, None] * Kc
+        Graw = Kc @ Bt.T
+        low = np.tril(Graw * gam) + np.diag(rc)
+        Gs = low + np.tril(low, -1).T
+        Lf, D = _ldl(Gs)
+        Li = np.linalg.inv(Lf)
+        Y = Li * gam
+        Z = Y @ Bt
+        Gm = Z / D[:, None]
+        rr = A[-1] / A
+        w = rr ** 2 * D
+        PC = A[-1] ** 2 * P + gamma[-1] * eye - (Gm.T * w) @ Gm
+        return dict(ell=ell, A=A, gam=gam, gamma=gamma, KP=KP, Bt=Bt, Graw=Graw, Lf=Lf, D=D, Li=Li, Y=Y, Z=Z,
+                    Gm=Gm, rr=rr, w=w, PC=0.5 * (PC + PC.T))
+
+    starts, Pstarts, caches = [], [], []
+    for c0, c1 in chunks:
+        starts.append(S.copy())
+        Pstarts.append(P.copy())
+        cf = cov_forward(k[c0:c1], a[c0:c1], qn[c0:c1], r[c0:c1], P)
+        caches.append(cf)
+        P = cf["PC"]
+        S = _wy_chunk_forward(k[c0:c1], v[c0:c1], cf["Gm"], a[c0:c1], S)
+
+    dS = np.zeros((dk, dv)) if dS_L is None else np.array(dS_L, float)
+    dP = np.zeros((dk, dk)) if dP_L is None else np.array(dP_L, float)
+    out = {key: np.zeros(shape) for key, shape in
+           (("dq", (L, dk)), ("dk", (L, dk)), ("dv", (L, dv)), ("dr", L), ("da", L), ("dqn", L))}
+    for ci in range(len(chunks) - 1, -1, -1):
+        c0, c1 = chunks[ci]
+        cf, P0c = caches[ci], Pstarts[ci]
+        Kc, ac = k[c0:c1], a[c0:c1]
+        n = c1 - c0
+        A, gam, rr, D, Gm = cf["A"], cf["gam"], cf["rr"], cf["D"], cf["Gm"]
+        AC = A[-1]
+        dQc, dKc, dVc, dGm, dloga, dS = _wy_chunk_backward(q[c0:c1], Kc, v[c0:c1], Gm, ac, starts[ci], dO[c0:c1],
+                                                           dm[c0:c1], dS)
+        # P_C = sym(A_C^2 P0 + gamma_C I - Gm^T diag(w) Gm)
+        dPC = 0.5 * (dP + dP.T)
+        dP0 = AC ** 2 * dPC
+        dA = np.zeros(n)
+        dAC = 2.0 * AC * np.sum(dPC * P0c)
+        dgamma = np.zeros(n)
+        dgamma[-1] += np.trace(dPC)
+        dGm -= (cf["w"][:, None] * Gm) @ (dPC + dPC.T)
+        dw = -np.einsum("ji,ik,jk->j", Gm, dPC, Gm)
+        dD = dw * rr ** 2
+        drr = dw * 2.0 * rr * D
+        # Gm = Z / D
+        dZ = dGm / D[:, None]
+        dD -= np.sum(dGm * Gm, axis=1) / D
+        # Z = Y Bt, Y = L^-1 o Gam
+        dY = dZ @ cf["Bt"].T
+        dBt = cf["Y"].T @ dZ
+        dLi = np.tril(dY * gam)
+        dgam = np.tril(dY * cf["Li"])
+        # L^-1 from L
+        dLf = np.tril(-cf["Li"].T @ dLi @ cf["Li"].T, -1)
+        # LDL, then the Gram's lower part: tril(Graw o Gam) + diag(r)
+        dlow = ldl_backward(cf["Lf"], D, dLf, dD)
+        out["dr"][c0:c1] = np.diag(dlow)
+        dGraw = dlow * gam
+        dgam += dlow * cf["Graw"]
+        # Graw = K Bt^T
+        dKc += dGraw @ cf["Bt"]
+        dBt += dGraw.T @ Kc
+        # Bt = diag(A^2) K P0 + diag(gamma) K
+        dKP = (A ** 2)[:, None] * dBt
+        dKc += dKP @ P0c.T + cf["gamma"][:, None] * dBt
+        dP0 += Kc.T @ dKP
+        dA += 2.0 * A * np.sum(dBt * cf["KP"], axis=1)
+        dgamma += np.sum(dBt * Kc, axis=1)
+        # gamma_j = a_j^2 gamma_{j-1} + Qn_j
+        da_c = np.zeros(n)
+        for j in range(n - 1, -1, -1):
+            out["dqn"][c0 + j] = dgamma[j]
+            gprev = cf["gamma"][j - 1] if j > 0 else 0.0
+            da_c[j] += 2.0 * ac[j] * gprev * dgamma[j]
+            if j > 0:
+                dgamma[j - 1] += ac[j] ** 2 * dgamma[j]
+        # gates of the covariance side, in log space
+        dell = A * dA + np.sum(gam * dgam, axis=1) - np.sum(gam * dgam, axis=0) - rr * drr
+        dell[-1] += AC * dAC + np.sum(rr * drr)
+        dloga = dloga + np.cumsum(dell[::-1])[::-1]
+        out["dq"][c0:c1], out["dk"][c0:c1], out["dv"][c0:c1] = dQc, dKc, dVc
+        out["da"][c0:c1] = dloga / ac + da_c
+        dP = dP0
+    out["dS0"], out["dP0"] = dS, 0.5 * (dP + dP.T)
     return out

@@ -67,3 +67,47 @@ def test_chunked_isotropic_backward_equals_token_backward(C):
     for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dc0"):
         scale = max(np.abs(ref[key]).max(), 1e-12)
         assert np.abs(got[key] - ref[key]).max() <= 1e-9 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
+
+
+def test_ldl_adjoint_matches_central_differences():
+    from chunk_model_backward import _ldl, ldl_backward
+    rng = np.random.default_rng(5)
+    n = 6
+    B = rng.standard_normal((n, n))
+    G = B @ B.T + n * np.eye(n)
+    dL, dD = np.tril(rng.standard_normal((n, n)), -1), rng.standard_normal(n)
+    got = ldl_backward(*_ldl(G), dL, dD)
+    h = 1e-6
+    for i in range(n):
+        for j in range(i + 1):
+            E = np.zeros((n, n))
+            E[i, j] = E[j, i] = 1.0  # the lower entry (i, j) stands for both mirror images
+            Lp, Dp = _ldl(G + h * E)
+            Lm, Dm = _ldl(G - h * E)
+            num = (np.sum(dL * (Lp - Lm)) + np.sum(dD * (Dp - Dm))) / (2 * h)
+            assert abs(got[i, j] - num) <= 1e-7 * max(1.0, abs(num)), (i, j, got[i, j], num)
+
+
+@pytest.mark.parametrize("C", [1, 8, 64])
+def test_chunked_full_backward_equals_token_backward(C):
+    from chunk_model_backward import chunk_full_backward
+    from oracle.backward import scan_kalman_full_backward
+    rng = np.random.default_rng(C + 123)
+    L, dk, dv = 70, 5, 4
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q, k = unit(rng.standard_normal((L, dk))), unit(rng.standard_normal((L, dk)))
+    v = rng.standard_normal((L, dv))
+    r = np.log1p(np.exp(rng.standard_normal(L))) + 0.1
+    a = np.exp(-np.log1p(np.exp(rng.standard_normal(L) - 3.0)))
+    qn = np.full(L, 1e-3)
+    B = rng.standard_normal((dk, dk)) / dk
+    S0, P0 = 0.3 * rng.standard_normal((dk, dv)), 0.5 * np.eye(dk) + B @ B.T
+    dO, dm, dSL = rng.standard_normal((L, dv)), rng.standard_normal(L), rng.standard_normal((dk, dv))
+    X = rng.standard_normal((dk, dk))
+    dPL = X + X.T
+    ref = scan_kalman_full_backward(q, k, v, r, dO, a=a, qn=qn, S0=S0, P0=P0, dm=dm, dS_L=dSL, dP_L=dPL)
+    ref["dP0"] = 0.5 * (ref["dP0"] + ref["dP0"].T)
+    got = chunk_full_backward(q, k, v, r, a, qn, C, dO, S0=S0, P0=P0, dm=dm, dS_L=dSL, dP_L=dPL)
+    for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dP0"):
+        scale = max(np.abs(ref[key]).max(), 1e-12)
+        assert np.abs(got[key] - ref[key]).max() <= 1e-8 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
