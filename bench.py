@@ -88,16 +88,16 @@ _B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment pe
 NCU_TRAFFIC = {
     "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
                          "bytes_per_token": (308.443648e6 + 171.383808e6) / _B3,
-                         "capture": "profiles/chunk_scan_ws_kernel_kalman_diag_d128.md (B=3 case, scaled)"},
+                         "capture": "ncu, chunk_scan_ws_kernel<diag> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "gdn_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
                  "bytes_per_token": (308.621056e6 + 170.472192e6) / _B3,
-                 "capture": "profiles/chunk_scan_ws_kernel_delta_d128.md (B=3 case, scaled)"},
+                 "capture": "ncu, chunk_scan_ws_kernel<delta> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
                         "bytes_per_token": (308.480256e6 + 171.998976e6) / _B3,
-                        "capture": "profiles/chunk_scan_ws_kernel_kalman_iso_d128.md (B=3 case, scaled)"},
+                        "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "kalman_full_d128": {"sources": _PSIDE_SOURCES, "sha1": "0bbdf6201df85beaf0b536f88b1722c9cc0b5c8e",
                          "bytes_per_token": (18.464256e6 + 5.376e3) / (2 * 8 * 4096),
-                         "capture": "profiles/kalman_pside_kernel_kalman_full_d128.md (full workload)"},
+                         "capture": "ncu, kalman_pside_kernel at the full workload B=2 H=8 L=4096"},
 }
 
 
@@ -248,13 +248,14 @@ def scan_closure(w, x, kdn):
     o = torch.empty(B, H, w.L, dv, dtype=torch.float32, device=dev)
     m = torch.empty(B, H, w.L, device=dev)
     ws = torch.empty(kdn.workspace_bytes(w.variant, B, H, w.L, dk, dv), dtype=torch.uint8, device=dev)
-    outs = {"o": o, "m": m}
+    outs = {"o": o, "m": m, "S": S}
     if w.variant == "delta":
         def fn():
             kdn.scan_delta(x["q"], x["k"], x["v"], x["beta"], a=x["a"], S=S, o=o, m=m, workspace=ws)
         return fn, outs
     if w.variant == "kalman_full":
         P = torch.eye(dk, device=dev).repeat(B, H, 1, 1)
+        outs["P"] = P
 
         def fn():
             kdn.scan_kalman_full(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, P=P, o=o, m=m,
@@ -262,12 +263,14 @@ def scan_closure(w, x, kdn):
         return fn, outs
     if w.variant == "kalman_iso":
         c = torch.ones(B, H, device=dev)
+        outs["c"] = c
 
         def fn():
             kdn.scan_kalman_iso(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, c=c, o=o, m=m,
                                 workspace=ws)
         return fn, outs
     p = torch.ones(B, H, dk, device=dev)
+    outs["p"] = p
 
     def fn():
         kdn.scan_kalman_diag(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], S=S, p=p, o=o, m=m, workspace=ws)
@@ -288,24 +291,30 @@ def bench_scan(w, steps, warmup, dist_on, rank, world, clocks=None):
     return {"ms": ms, "value": weak_scaling_value(w.tokens, ms, world), "launches": scan_plan(w)["launches"] * steps}
 
 
+# the per-token inputs each variant reads (Qn is a scalar argument)
+E2E_INPUTS = {"delta": ("q", "k", "v", "beta", "a"), "kalman_full": ("q", "k", "v", "a", "r"),
+              "kalman_diag": ("q", "k", "v", "a", "r"), "kalman_iso": ("q", "k", "v", "a", "r")}
+
+
 def bench_e2e(w, steps, warmup, dist_on, rank, world):
-    """Through the public API with host buffers, as a stream of batches: every step copies its inputs from
-    pinned host memory to the device, scans them and copies o and m back.  Steps are pipelined over three
-    streams with two device buffer sets, so that step i + 1's host-to-device copy runs beside step i's scan
-    and device-to-host copy (the link is full duplex); the time per step is the span of all steps / steps."""
+    """Through the public API with host buffers, as a stream of batches: every step copies the inputs its
+    variant reads from pinned host memory to the device, scans them and copies o, m and the final state
+    (S and P, p or c) back.  Steps are pipelined over three streams with two device buffer sets, so that
+    step i + 1's host-to-device copy runs beside step i's scan and device-to-host copy (the link is full
+    duplex); the time per step is the span of all steps / steps."""
     from delta_rule_recurrent_scan_b200 import kdn
     xd = make_scan_inputs(w, seed=rank, device="cuda")
-    host = {k: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
+    keys = E2E_INPUTS[w.variant]
+    host = {k: xd[k].cpu().pin_memory() for k in keys if isinstance(xd[k], torch.Tensor)}
     bufs = []
     for _ in range(2):
         dev = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
         fn_dev, outs = scan_closure(w, dev, kdn)
         bufs.append((dev, fn_dev, outs))
     del xd
-    o_host = torch.empty(bufs[0][2]["o"].shape, dtype=bufs[0][2]["o"].dtype).pin_memory()
-    m_host = torch.empty(bufs[0][2]["m"].shape).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values() if isinstance(v, torch.Tensor))
-    d2h = o_host.numel() * o_host.element_size() + m_host.numel() * 4
+    out_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bufs[0][2].items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
 
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "comp", "out")}
@@ -320,8 +329,7 @@ def bench_e2e(w, steps, warmup, dist_on, rank, world):
         s_in.wait_event(ev["comp"][b])       # the scan of step i - 2 has read these inputs
         with torch.cuda.stream(s_in):
             for k, v in host.items():
-                if isinstance(v, torch.Tensor):
-                    dev[k].copy_(v, non_blocking=True)
+                dev[k].copy_(v, non_blocking=True)
             ev["in"][b].record(s_in)
         s_comp.wait_event(ev["in"][b])
         s_comp.wait_event(ev["out"][b])      # step i - 2's outputs are back on the host
@@ -330,8 +338,8 @@ def bench_e2e(w, steps, warmup, dist_on, rank, world):
             ev["comp"][b].record(s_comp)
         s_out.wait_event(ev["comp"][b])
         with torch.cuda.stream(s_out):
-            o_host.copy_(outs["o"], non_blocking=True)
-            m_host.copy_(outs["m"], non_blocking=True)
+            for k, v in out_host.items():
+                v.copy_(outs[k], non_blocking=True)
             ev["out"][b].record(s_out)
 
     for i in range(warmup):
@@ -351,6 +359,7 @@ def bench_e2e(w, steps, warmup, dist_on, rank, world):
     _barrier(dist_on)
     ms = _max_over_ranks(start.elapsed_time(end) / steps, dist_on)
     return {"value": w.tokens * world / (ms * 1e-3), "ms": ms, "h2d": h2d, "d2h": d2h,
+            "copied": {"in": list(host), "out": list(out_host)},
             "pipelined": "3 streams, 2 device buffer sets: step i + 1's copy-in beside step i's scan and copy-out"}
 
 
@@ -400,16 +409,14 @@ def hola_bytes(w, in_bytes=2) -> int:
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
 
-def cpu_baseline(w, heads=16, seconds_hint=None):
-    """The float64 oracle, as it stands, on a bounded sample: ``heads`` heads over the full sequence."""
-    import numpy as np
-
-    sys.path.insert(0, ROOT)
+def _oracle_head(args):
+    """One head of the workload through the float64 oracle, as it stands (runs in a pool worker).
+    Returns (tokens, seconds of the oracle call alone)."""
+    name, overrides, seed = args
     import oracle
 
-    B = max(1, heads // w.H)
-    H = min(w.H, heads)
-    x = make_scan_inputs(w, seed=0, device="cpu", B=B, H=H)
+    w = WORKLOADS[name].with_(**overrides)
+    x = make_scan_inputs(w, seed=seed, device="cpu", B=1, H=1)
     np_ = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     t0 = time.perf_counter()
     if w.variant == "delta":
@@ -420,12 +427,51 @@ def cpu_baseline(w, heads=16, seconds_hint=None):
         oracle.scan_kalman_iso(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
     else:
         oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
-    dt = time.perf_counter() - t0
-    tokens = B * H * w.L
-    del np
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{B * H} of {w.B * w.H} heads x full L={w.L} ({tokens} tokens, {dt:.1f} s, float64 NumPy, "
-                      f"one thread)"}
+    return w.L, time.perf_counter() - t0
+
+
+def _pool_init():
+    torch.set_num_threads(1)
+    import oracle  # noqa: F401  (import cost outside the timed calls)
+
+
+class OraclePool:
+    """The oracle on every host core: a spawn pool (safe beside a CUDA context) of one single-threaded
+    worker per core in this process's affinity mask; heads are independent, so each worker scans whole
+    heads.  Throughput = the tokens of one round (one head per worker) / the slowest worker's oracle time."""
+
+    def __init__(self):
+        import concurrent.futures
+        import multiprocessing
+
+        self.cores = len(os.sched_getaffinity(0))
+        for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+            os.environ[var] = "1"  # one thread per worker process; the workers cover the cores
+        self.pool = concurrent.futures.ProcessPoolExecutor(
+            max_workers=self.cores, mp_context=multiprocessing.get_context("spawn"), initializer=_pool_init)
+
+    def round(self, w, seed0=0):
+        over = {"B": w.B, "H": w.H}
+        res = list(self.pool.map(_oracle_head, [(w.name, over, seed0 + i) for i in range(self.cores)]))
+        tokens = sum(r[0] for r in res)
+        return tokens, max(r[1] for r in res)
+
+    def close(self):
+        self.pool.shutdown()
+
+
+def cpu_baseline(w):
+    """The float64 oracle, as it stands, on a bounded sample of the workload on all host cores."""
+    pool = OraclePool()
+    try:
+        pool.round(w.with_(L=64), seed0=10_000)  # start the workers (spawn, imports) outside the timing
+        tokens, dt = pool.round(w)
+    finally:
+        pool.close()
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": pool.cores, "kind": "oracle",
+            "sample": f"{pool.cores} of {w.B * w.H} heads x full L={w.L} ({tokens} tokens), one head per worker "
+                      f"on {pool.cores} single-threaded spawn workers (one per core), float64 NumPy, "
+                      f"slowest worker {dt:.2f} s"}
 
 
 # ----------------------------------------------------------------------------- main
@@ -533,7 +579,8 @@ def main():
                          "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events"},
             "e2e": None if e2e is None else {"value": e2e["value"], "unit": "tokens/s",
                                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                                             "ms_per_step": e2e["ms"], "pipelined": e2e["pipelined"]},
+                                             "ms_per_step": e2e["ms"], "copied": e2e["copied"],
+                                             "pipelined": e2e["pipelined"]},
             "gpu_launches": head["launches"],
             "clocks": clocks.summary(),
             "also": also,
@@ -547,46 +594,34 @@ def main():
 
 
 def reference_arm(args, w, rank, world):
-    """The float64 CPU oracle as the reference arm: rank 0 only, bounded sample per step."""
+    """The float64 CPU oracle as the reference arm: rank 0 only; each step is one round of the oracle
+    pool (one head of the workload per host core, full L)."""
     if rank != 0:
         return
-    import numpy as np
-
-    import oracle
-
-    heads, Ls = 2, w.L
-    B, H = 1, heads
-    x = make_scan_inputs(w, seed=0, device="cpu", B=B, H=H, L=Ls)
-    np_ = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-
-    def step():
-        if w.variant == "delta":
-            oracle.scan_delta(np_["q"], np_["k"], np_["v"], np_["beta"], a=np_["a"])
-        elif w.variant == "kalman_full":
-            oracle.scan_kalman_full(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
-        elif w.variant == "kalman_iso":
-            oracle.scan_kalman_iso(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
-        else:
-            oracle.scan_kalman_diag(np_["q"], np_["k"], np_["v"], r=np_["r"], a=np_["a"], qn=np_["qn"])
-
-    for _ in range(min(args.warmup, 1)):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    tokens = B * H * Ls
-    value = tokens / dt
-    sample = f"{B * H} of {w.B * w.H} heads x full L={Ls} per step ({tokens} tokens), float64 NumPy, one thread"
+    pool = OraclePool()
+    try:
+        pool.round(w.with_(L=64), seed0=10_000)  # start the workers outside the timing
+        for i in range(min(args.warmup, 1)):
+            pool.round(w, seed0=100 * (i + 1))
+        total_tokens, total_s = 0, 0.0
+        for i in range(args.steps):
+            tokens, dt = pool.round(w, seed0=i * pool.cores)
+            total_tokens += tokens
+            total_s += dt
+    finally:
+        pool.close()
+    dt = total_s / args.steps
+    value = total_tokens / total_s
+    sample = (f"{pool.cores} of {w.B * w.H} heads x full L={w.L} per step ({total_tokens // args.steps} tokens), "
+              f"one head per single-threaded spawn worker, {pool.cores} workers (one per core), float64 NumPy")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "variant": w.variant, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": pool.cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    del np
     print(json.dumps(line), flush=True)
 
 

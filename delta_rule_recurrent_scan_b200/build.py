@@ -12,6 +12,7 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -58,15 +59,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
     obj_dir = os.path.join(LIB_DIR, "obj")
     os.makedirs(obj_dir, exist_ok=True)
-    objs = []
+    cmds, objs = [], []
     for src in sources():
         name = os.path.basename(src)
         obj = os.path.join(obj_dir, name + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, *PER_FILE_FLAGS.get(name, IEEE_FLAGS), "-I", INCLUDE, "-c", src, "-o", obj]
+        cmds.append([_nvcc(), *NVCC_FLAGS, *PER_FILE_FLAGS.get(name, IEEE_FLAGS), "-I", INCLUDE, "-c", src, "-o", obj])
+        objs.append(obj)
+
+    def compile_one(cmd):
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-        objs.append(obj)
+
+    workers = max(1, min(len(cmds), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=workers) as pool:
+        list(pool.map(compile_one, cmds))
     tmp = LIB + ".tmp"
     link = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
             "-Xcompiler", "-fPIC", "-o", tmp, *objs]

@@ -51,18 +51,18 @@ kdn_status check_ptr(const void* p, const char* name, size_t align, bool allow_n
   return KDN_OK;
 }
 
-// Launch on the device that owns the state buffer (the library links its own
-// CUDA runtime, whose current device need not be the caller's).
-kdn_status use_device_of(const void* p) {
+// Launch on the device that owns the state buffer (the library links its own CUDA runtime, whose
+// current device need not be the caller's); ``guard`` puts the caller's device back on return.
+kdn_status use_device_of(const void* p, DeviceGuard& guard) {
   cudaPointerAttributes attr;
   if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
     cudaGetLastError();
     return fail(KDN_ERR_INVALID_ARG, "cannot query the device of the state buffer");
   }
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess || cur != attr.device) {
-    cudaError_t e = cudaSetDevice(attr.device);
-    if (e != cudaSuccess) return fail(KDN_ERR_CUDA, std::string("cudaSetDevice: ") + cudaGetErrorString(e));
+  const cudaError_t e = static_cast<cudaError_t>(guard.switch_to(attr.device));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(KDN_ERR_CUDA, std::string("cudaSetDevice: ") + cudaGetErrorString(e));
   }
   return KDN_OK;
 }
@@ -148,7 +148,8 @@ size_t seg_area_offset(kdn_variant var, const kdn_dims* d) {
 }
 
 kdn_status common_checks(kdn_variant var, const kdn_dims* d, const void* q, const void* k, const void* v,
-                         const float* S, const void* o, const float* m, const void* ws, size_t ws_bytes) {
+                         const float* S, const void* o, const float* m, const void* ws, size_t ws_bytes,
+                         DeviceGuard& guard) {
   KDN_TRY(check_dims(d));
   int P = 1;
   KDN_TRY(resolve_segments(var, d, &P));
@@ -164,7 +165,7 @@ kdn_status common_checks(kdn_variant var, const kdn_dims* d, const void* q, cons
   if (ws_bytes < need)
     return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(ws_bytes) + " < required " +
                                          std::to_string(need));
-  return use_device_of(S);
+  return use_device_of(S, guard);
 }
 
 kdn_status cuda_status(cudaError_t e, const char* what) {
@@ -289,10 +290,19 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
 
 kdn_status kdn_read_device_status(const void* workspace, int* status_out, void* stream) {
   if (status_out == nullptr) return fail(KDN_ERR_INVALID_ARG, "status_out is NULL");
-  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
-  KDN_TRY(use_device_of(workspace));
+  DeviceGuard guard;
+  const void* word_ptr = workspace;
+  if (workspace == nullptr) {
+    // the no-alloc entry point's status word, in its static array on the current device
+    void* p = nullptr;
+    KDN_TRY(noalloc_scratch_on_current_device(&p));
+    word_ptr = p;
+  } else {
+    KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+    KDN_TRY(use_device_of(workspace, guard));
+  }
   unsigned word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  cudaError_t e = cudaMemcpyAsync(&word, word_ptr, sizeof(word), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "reading the device status");
   *status_out = (word & kdn::kStatusNumeric) ? KDN_ERR_NUMERIC : (word & kdn::kStatusTimeout) ? KDN_ERR_TIMEOUT : KDN_OK;
@@ -302,7 +312,8 @@ kdn_status kdn_read_device_status(const void* workspace, int* status_out, void* 
 kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
                           const float* a, float* S, void* o, float* m, void* workspace, size_t workspace_bytes,
                           void* stream) {
-  KDN_TRY(common_checks(KDN_DELTA, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  DeviceGuard guard;
+  KDN_TRY(common_checks(KDN_DELTA, dims, q, k, v, S, o, m, workspace, workspace_bytes, guard));
   const bool any = dims->L > 0;
   KDN_TRY(check_ptr(beta, "beta", 4, !any));
   KDN_TRY(check_ptr(a, "a", 4, true));
@@ -332,7 +343,8 @@ kdn_status kdn_scan_delta(const kdn_dims* dims, const void* q, const void* k, co
 kdn_status kdn::api::kalman_scan(kdn_variant var, const kdn_dims* dims, const void* q, const void* k, const void* v,
                               const float* a, const float* r, const float* qn, float qn_scalar, float* S, float* P,
                               void* o, float* m, void* workspace, size_t workspace_bytes, void* stream) {
-  KDN_TRY(common_checks(var, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  DeviceGuard guard;
+  KDN_TRY(common_checks(var, dims, q, k, v, S, o, m, workspace, workspace_bytes, guard));
   const bool any = dims->L > 0;
   KDN_TRY(check_ptr(P, var == KDN_KALMAN_FULL ? "P" : "p", var == KDN_KALMAN_FULL ? 16 : 4, false));
   KDN_TRY(check_ptr(r, "r", 4, !any));
@@ -393,7 +405,8 @@ kdn_status kdn_scan_kalman_diag(const kdn_dims* dims, const void* q, const void*
 kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* a,
                                const float* r, const float* qn, float qn_scalar, float* S, float* c, void* o,
                                float* m, void* workspace, size_t workspace_bytes, void* stream) {
-  KDN_TRY(common_checks(KDN_KALMAN_ISO, dims, q, k, v, S, o, m, workspace, workspace_bytes));
+  DeviceGuard guard;
+  KDN_TRY(common_checks(KDN_KALMAN_ISO, dims, q, k, v, S, o, m, workspace, workspace_bytes, guard));
   const bool any = dims->L > 0;
   KDN_TRY(check_ptr(c, "c", 4, false));
   KDN_TRY(check_ptr(r, "r", 4, !any));
@@ -450,7 +463,8 @@ kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* 
   KDN_TRY(check_ptr(cache_idx, "cache_idx", 4, true));
   KDN_TRY(check_ptr(workspace, "workspace", 256, false));
   if (workspace_bytes < kStatusBytes) return fail(KDN_ERR_INVALID_ARG, "workspace_bytes < 256");
-  KDN_TRY(use_device_of(gamma_q));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(gamma_q, guard));
   const int BH = dims->B * dims->H;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
@@ -485,7 +499,8 @@ kdn_status kdn_decode_step(kdn_variant variant, int B, int H, int dk, int dv, kd
     KDN_TRY(check_ptr(p, "p", 4, false));
     if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
   }
-  KDN_TRY(use_device_of(S));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(S, guard));
   kdn::DecodeArgs args{q, k, v, in_dtype, out_dtype, beta, a, r, qn_scalar, S, p, o, m, B * H};
   const int mode = variant == KDN_KALMAN_DIAG ? 1 : variant == KDN_KALMAN_ISO ? 2 : 0;
   return cuda_status(kdn::launch_decode(dk, dv, mode, args, (cudaStream_t)stream), "decode launch");

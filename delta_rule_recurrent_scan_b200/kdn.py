@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_workspace_bytes.argtypes = [i, dims]
     L.kdn_workspace_bytes.restype = sz
     L.kdn_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+    L.kdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    L.kdn_selftest_wait_timeout.restype = ctypes.c_int
     L.kdn_status_string.argtypes = [i]
     L.kdn_status_string.restype = ctypes.c_char_p
     L.kdn_last_error.argtypes = []
@@ -343,9 +345,17 @@ def decode_step(variant, q, k, v, S, beta=None, a=None, r=None, qn=0.0, p=None, 
     return o, m
 
 
-def read_device_status(workspace: torch.Tensor, stream=None) -> int:
-    """Synchronise the stream and return the device status of a scan's workspace (a KDN_* code)."""
+def read_device_status(workspace: torch.Tensor | None, stream=None) -> int:
+    """Synchronise the stream and return the device status of a scan's workspace (a KDN_* code).
+    ``workspace=None`` reads the status word of the no-alloc full-Kalman scan on the current device."""
     out = ctypes.c_int(-1)
     st = lib().kdn_read_device_status(_ptr(workspace), ctypes.byref(out), _stream(stream))
     _check(st, "kdn_read_device_status")
     return out.value
+
+
+def selftest_wait_timeout(workspace: torch.Tensor | None, wait_cycles: int = 100_000, stream=None) -> None:
+    """Run the bounded-wait failure path once on purpose (a wait on an mbarrier nothing arrives at, with
+    nothing in flight): afterwards ``read_device_status(workspace)`` reports KDN_ERR_TIMEOUT."""
+    st = lib().kdn_selftest_wait_timeout(_ptr(workspace), int(wait_cycles), _stream(stream))
+    _check(st, "kdn_selftest_wait_timeout")

@@ -47,6 +47,8 @@
  *   States are updated in place, so consecutive calls continue one scan.
  * Streams.  ``stream`` is a cudaStream_t (NULL = legacy default stream).
  *   Every call only enqueues work on it and returns; nothing synchronises.
+ * Devices.  A call launches on the device that owns its state buffer and
+ *   restores the calling thread's current device before it returns.
  * Errors.  Argument errors return synchronously and enqueue nothing.  A failed
  *   launch returns KDN_ERR_CUDA.  Numeric failures found on the device (a
  *   non-positive or non-finite innovation variance) set the status word in
@@ -186,13 +188,20 @@ KDN_EXPORT kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, c
  *   holds until the process exits.  Limit: B*H*L*d_k <= 4,194,304; larger
  *   requests return KDN_ERR_UNSUPPORTED (kdn_last_error() says why) and
  *   enqueue nothing.
- *   Set-up: the first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   Set-up: on each device the array is reserved when the library's module
+ *   that holds it is loaded, which under CUDA's lazy module loading (the
+ *   default) is the first no-alloc call there, not library load.  A caller
+ *   that reserves device memory at start-up should make that first call
+ *   before it does (an L = 0 call with valid S and P is enough: it enqueues
+ *   only the status-word clear), and before any stream capture.  Each call
+ *   looks the array's device address up again (cudaGetSymbolAddress, with
+ *   the state's device current), so a device reset leaves no stale address.
  *   Sharing: every call, on every stream, uses the same array and leaves its
  *   last contents behind (the status word is cleared at the start of each
- *   call).  Calls whose GPU work overlaps race on it: serialise them.  The
- *   device status word is not readable through this entry point. */
+ *   call).  Calls whose GPU work overlaps race on it: serialise them.
+ *   Status: kdn_read_device_status(NULL, ...) reads this entry point's
+ *   device status word (timeouts, non-positive innovation variances) on the
+ *   calling thread's current device. */
 KDN_EXPORT kdn_status kdn_scan_kalman_full_noalloc(const kdn_dims* dims, const void* q, const void* k, const void* v,
                                                    const float* a, const float* r, const float* qn, float qn_scalar,
                                                    float* S, float* P, void* o, float* m, void* stream);
@@ -214,8 +223,22 @@ KDN_EXPORT size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims)
 
 /* Synchronises ``stream``, then reads the device status word of ``workspace``
  * into *status_out (a kdn_status value: KDN_OK, KDN_ERR_NUMERIC or
- * KDN_ERR_TIMEOUT).  Each scan clears the word when it is enqueued. */
+ * KDN_ERR_TIMEOUT).  Each scan clears the word when it is enqueued.
+ * workspace == NULL reads the word of kdn_scan_kalman_full_noalloc, kept in
+ * its static array on the calling thread's current device. */
 KDN_EXPORT kdn_status kdn_read_device_status(const void* workspace, int* status_out, void* stream);
+
+/* Failure-path self-test (no counterpart on the pages: it checks the
+ * library's own failure detection).  Every wait of the tensor-core kernels
+ * is bounded: on expiry the kernel sets KDN_ERR_TIMEOUT in the status word,
+ * frees its tensor memory and returns.  This launches one small kernel that
+ * takes that path on purpose: it waits on an mbarrier nothing arrives at
+ * (no copy or MMA in flight) for ``wait_cycles`` SM clocks (1 .. 2e9, about
+ * one second at most), then aborts exactly as the scans do.  Afterwards
+ * kdn_read_device_status(workspace, ...) reports KDN_ERR_TIMEOUT.
+ * workspace: >= 256 bytes, 256-byte aligned, or NULL for the no-alloc entry
+ * point's status word on the current device.  Asynchronous on ``stream``. */
+KDN_EXPORT kdn_status kdn_selftest_wait_timeout(void* workspace, long long wait_cycles, void* stream);
 
 /* Which kernels a scan with these dims runs: *launches = kernel launches per
  * call (the status-word clear, a 256-byte memset, not counted), *kernel = name

@@ -108,3 +108,13 @@ def compare(got, ref, tol, heads=None):
     bad = {k_: e for k_, e in errs.items() if not (e <= tol)}
     assert not bad, f"errors above {tol}: {errs}"
     return errs
+
+
+def assert_symmetric_pd(P, tol=TOL["bf16"]):
+    """Every head's returned covariance is symmetric to ``tol`` (normwise) and positive definite
+    (a float64 Cholesky of its symmetric part succeeds)."""
+    P = P.detach().double().cpu().reshape(-1, P.shape[-2], P.shape[-1])
+    asym = (P - P.transpose(1, 2)).flatten(1).abs().amax(1) / P.flatten(1).abs().amax(1)
+    assert float(asym.max()) <= tol, float(asym.max())
+    _, info = torch.linalg.cholesky_ex(0.5 * (P + P.transpose(1, 2)))
+    assert int(info.abs().max()) == 0, "P is not positive definite"

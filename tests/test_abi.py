@@ -18,7 +18,7 @@ def test_every_declared_symbol_is_exported(L):
     names = kdn.exported_names()
     assert {"kdn_scan_delta", "kdn_scan_kalman_full", "kdn_scan_kalman_diag", "kdn_scan_kalman_iso", "kdn_decode_step",
             "kdn_workspace_bytes", "kdn_read_device_status", "kdn_status_string", "kdn_last_error",
-            "kdn_api_version"} <= set(names)
+            "kdn_api_version", "kdn_scan_kalman_full_noalloc", "kdn_selftest_wait_timeout"} <= set(names)
     for n in names:
         assert hasattr(L, n), n
 
@@ -63,7 +63,12 @@ def test_host_validation_without_gpu(L):
     assert b"aligned" in L.kdn_last_error()
     assert L.kdn_decode_step(5, 1, 1, 64, 64, 1, 1, *([None] * 6), 0.0, *([None] * 5)) == kdn.KDN_ERR_UNSUPPORTED
     out = ctypes.c_int(0)
-    assert L.kdn_read_device_status(None, ctypes.byref(out), None) == kdn.KDN_ERR_INVALID_ARG
+    assert L.kdn_read_device_status(ctypes.c_void_p(0x1000), None, None) == kdn.KDN_ERR_INVALID_ARG
+    assert L.kdn_read_device_status(ctypes.c_void_p(0x1004), ctypes.byref(out), None) == kdn.KDN_ERR_INVALID_ARG
+    # the failure-path self-test checks its wait limit before it looks at a device
+    for bad in (0, -1, 3_000_000_000):
+        assert L.kdn_selftest_wait_timeout(None, bad, None) == kdn.KDN_ERR_INVALID_ARG
+        assert b"wait_cycles" in L.kdn_last_error()
 
 
 def test_plan_counts_the_isotropic_prologue(L):

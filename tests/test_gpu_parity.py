@@ -17,7 +17,7 @@ import torch
 import oracle
 from delta_rule_recurrent_scan_b200 import kdn
 from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_decode_inputs, make_scan_inputs
-from parity import TOL, compare, initial_state, normwise_err, run_gpu, run_oracle
+from parity import TOL, assert_symmetric_pd, compare, initial_state, normwise_err, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -119,6 +119,21 @@ def test_tensor_core_path_matches_per_token_path(variant, d):
     compare(fast, run_oracle(variant, x), TOL["bf16"])
 
 
+@pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_results_do_not_depend_on_the_chunk_size(variant, d):
+    """Every chunk size the library accepts (0 = its choice, 16, 32, 64) gives the same scan: to the
+    rounding of the tensor-core splits between chunkings, and to the oracle's tolerance for each."""
+    w = WORKLOADS["gdn_d128"].with_(variant=variant, dk=d, dv=d, qn=1e-3)
+    x = make_scan_inputs(w, seed=15, device=DEV, B=1, H=2, L=333)
+    ref = run_oracle(variant, x)
+    runs = {C: run_gpu(variant, x, chunk=C) for C in (0, 16, 32, 64)}
+    for C, got in runs.items():
+        compare(got, ref, TOL["bf16"])
+        for key in got:
+            assert normwise_err(got[key], runs[64][key]) < 1e-3, (C, key)
+
+
 # ----------------------------------------------------------------------------- edge cases
 
 
@@ -181,6 +196,8 @@ def test_full_size_sampled_heads(name):
     heads = _sample_heads(w.B, w.H)
     ref = run_oracle(w.variant, x, heads=heads)
     compare(got, ref, TOL["bf16"], heads=heads)
+    if w.variant == "kalman_full":
+        assert_symmetric_pd(got["P"])
 
 
 # ----------------------------------------------------------------------------- decode
@@ -239,6 +256,38 @@ def test_decode_full_batch_sampled_heads(name):
     assert normwise_err(got_S, ref["S"]) < TOL["bf16"]
     got_o = torch.stack([o[b, h] for b, h in heads])[None]
     assert normwise_err(got_o.float()[:, :, None], ref["o"][:, :, -1:]) < TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", ["decode_delta", "decode_diag"])
+def test_decode_1024_steps_full_batch_sampled_heads(name):
+    """The decode workload as specified: 1024 one-token calls over the full batch (256 x 32 heads), each
+    step's inputs drawn fresh; three sampled heads are followed by the oracle over all 1024 tokens (o and
+    m at every step, S and p at the end), so that error growth over a long decode would show."""
+    w = WORKLOADS[name]
+    variant, steps = w.variant, w.steps
+    assert steps == 1024
+    S, C = initial_state(variant, w.B, w.H, w.dk, w.dv, DEV)
+    heads = _sample_heads(w.B, w.H, n=3, seed=2)
+    bi = torch.tensor([b for b, _ in heads], device=DEV)
+    hi = torch.tensor([h for _, h in heads], device=DEV)
+    seen = {key: [] for key in ("q", "k", "v", "beta", "a", "r")}
+    outs, ms = [], []
+    for t in range(steps):
+        x = make_decode_inputs(w, steps=1, seed=1000 + t, device=DEV)
+        o, m = kdn.decode_step(variant, x["q"][0], x["k"][0], x["v"][0], S, beta=x["beta"][0], a=x["a"][0],
+                               r=x["r"][0], qn=x["qn"], p=C)
+        for key in seen:
+            seen[key].append(x[key][0][bi, hi])
+        outs.append(o[bi, hi])
+        ms.append(m[bi, hi])
+    # sampled heads as a [1, 3, steps, d] scan for the oracle
+    xs = {key: torch.stack(val, dim=1)[None] for key, val in seen.items()}
+    xs["qn"] = w.qn
+    ref = run_oracle(variant, xs)
+    got = {"o": torch.stack(outs, dim=1)[None], "m": torch.stack(ms, dim=1)[None], "S": S[bi, hi][None]}
+    if variant == "kalman_diag":
+        got["p"] = C[bi, hi][None]
+    compare(got, ref, TOL["bf16"])
 
 
 # ----------------------------------------------------------------------------- status and errors

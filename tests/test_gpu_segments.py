@@ -13,7 +13,7 @@ import torch
 
 from delta_rule_recurrent_scan_b200 import kdn
 from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_scan_inputs
-from parity import TOL, compare, initial_state, run_oracle
+from parity import TOL, assert_symmetric_pd, compare, initial_state, run_oracle
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -71,8 +71,6 @@ VARIANTS = ["delta", "kalman_diag", "kalman_iso", "kalman_full"]
 @pytest.mark.parametrize("d", [64, 128])
 def test_library_choice_splits_few_heads(variant, d):
     """B*H = 2 and L = 1024: the library picks 8 segments of two chunks each."""
-    if variant == "kalman_iso" and d == 64:
-        pytest.skip("covered at d = 128; the isotropic prologue is the same at both sizes")
     w = WORKLOADS["gdn_d128"].with_(variant=variant, dk=d, dv=d, qn=1e-3)
     x = make_scan_inputs(w, seed=11, device=DEV, B=1, H=2, L=1024)
     n = kdn.plan(variant, 1, 2, 1024, d, d)["launches"]
@@ -108,6 +106,7 @@ def test_full_size_kalman_full_layer_uses_segments():
     heads = [(0, 3), (1, 7)]
     ref = run_oracle("kalman_full", x, S0=S0, C0=C0, heads=heads)
     compare(got, ref, TOL["bf16"], heads=heads)
+    assert_symmetric_pd(got["P"])
 
 
 def test_segment_requests_are_validated():
