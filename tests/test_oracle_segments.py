@@ -123,3 +123,75 @@ def test_segmented_scan_equals_the_serial_scan(variant, L, P):
     np.testing.assert_allclose(np.concatenate(o), ref["o"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(np.concatenate(m), ref["m"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(S, ref["S"], rtol=1e-10, atol=1e-12)
+
+
+def _riccati_token_map(a, qn, k, r):
+    """The full-covariance step P -> P^- (I + k k^T P^- / r)^-1 with P^- = a^2 P + Qn I, as the 2d x 2d
+    transfer matrix of the homogeneous pair P = X Y^-1: [X; Y] -> M [X; Y]."""
+    d = k.shape[0]
+    eye = np.eye(d)
+    kk = np.outer(k, k) / r
+    return np.block([[a * a * eye, qn * eye], [a * a * kk, qn * kk + eye]])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_full_covariance_riccati_composes_as_segment_transfer_matrices(seed):
+    """The dense covariance recursion is a matrix Moebius (linear-fractional) map of P (Kalman Delta
+    Networks, Abstract): each token multiplies the homogeneous pair [X; Y] (P = X Y^-1) by a 2d x 2d matrix,
+    so a segment's map is the product of its tokens' matrices, renormalised by any scalar.  Chaining the
+    segment maps from P0 gives the oracle's P at every segment boundary; a wrong block (a instead of a^2,
+    the update's k k^T / r in the upper right, Qn missing from the lower right) fails it."""
+    d, L, seg = 6, 96, 16
+    x = _inputs(seed, L, d)
+    P0 = np.eye(d) * 0.7 + 0.05
+    ref = scan_kalman_full(x["q"], x["k"], x["v"], x["r"], a=x["a"], qn=x["qn"], P0=P0, return_states=True)
+    X, Y = P0.copy(), np.eye(d)
+    for lo in range(0, L, seg):
+        M = np.eye(2 * d)
+        for t in range(lo, lo + seg):
+            M = _riccati_token_map(x["a"][t], x["qn"][t], x["k"][t], x["r"][t]) @ M
+            M = M / np.abs(M).max()
+        XY = M @ np.vstack([X, Y])
+        X, Y = XY[:d], XY[d:]
+        P = X @ np.linalg.inv(Y)
+        np.testing.assert_allclose(P, ref["P_hist"][lo + seg - 1], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(P, P.T, atol=1e-10)
+
+
+def _riccati_chunk_map(a, qn, k, r):
+    """Closed form of the product M_C ... M_1 of a chunk's token transfer matrices.
+
+    M_t = D_t + u_t v_t^T with D_t = [[a_t^2 I, Qn_t I], [0, I]], u_t = [0; k_t], v_t = [a_t^2 k_t; Qn_t k_t] / r_t,
+    so the product is [[alpha I, beta I], [0, I]] + U W^T with alpha = prod a^2, beta = the accumulated
+    process noise, column j of U = [beta_{C,j} k_j; k_j] (beta_{t,j}: the noise accumulated over tokens
+    j+1..t) and W = B (diag(r) - Cs^T)^-1, where column t of B is [alpha_t k_t; beta_t k_t] and
+    Cs_tj = (k_j . k_t) beta_{t,j} for j < t: one triangular solve of the chunk's size."""
+    C, d = k.shape
+    alpha = np.cumprod(a * a)                     # alpha_t
+    beta = np.zeros(C)                            # beta_t = a_t^2 beta_{t-1} + Qn_t
+    for t in range(C):
+        beta[t] = a[t] ** 2 * (beta[t - 1] if t else 0.0) + qn[t]
+    bt = np.zeros((C, C))                         # beta_{t,j}, j <= t (beta_{j,j} = 0)
+    for j in range(C):
+        acc = 0.0
+        for t in range(j + 1, C):
+            acc = a[t] ** 2 * acc + qn[t]
+            bt[t, j] = acc
+    Cs = np.tril((k @ k.T) * bt, -1)
+    Bm = np.vstack([alpha[None, :] * k.T, beta[None, :] * k.T])       # 2d x C
+    W = np.linalg.solve((np.diag(r) - Cs.T).T, Bm.T).T                # B (diag(r) - Cs^T)^-1
+    U = np.vstack([bt[C - 1][None, :] * k.T, k.T])
+    eye = np.eye(d)
+    return np.block([[alpha[-1] * eye, beta[-1] * eye], [0 * eye, eye]]) + U @ W.T
+
+
+@pytest.mark.parametrize("seed", [0, 3])
+def test_riccati_chunk_transfer_matrix_in_closed_form(seed):
+    """The closed form above equals the product of the chunk's token matrices (a chunk-parallel covariance
+    side can build every chunk's map at once and only chain the maps)."""
+    d, C = 5, 12
+    x = _inputs(seed, C, d)
+    M = np.eye(2 * d)
+    for t in range(C):
+        M = _riccati_token_map(x["a"][t], x["qn"][t], x["k"][t], x["r"][t]) @ M
+    np.testing.assert_allclose(_riccati_chunk_map(x["a"], x["qn"], x["k"], x["r"]), M, rtol=1e-11, atol=1e-12)
