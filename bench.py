@@ -401,6 +401,37 @@ def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
     return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": steps}
 
 
+def bench_backward(w, steps, warmup, dist_on, rank, world):
+    """The gated delta rule backward over a layer (upstream dO and dm random; the start state zero)."""
+    from delta_rule_recurrent_scan_b200 import kdn
+    x = make_scan_inputs(w, seed=rank, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(rank + 1)
+    dO = torch.randn(w.B, w.H, w.L, w.dv, device="cuda", generator=g)
+    dm = torch.randn(w.B, w.H, w.L, device="cuda", generator=g)
+    dims = kdn.Dims(w.B, w.H, w.L, w.dk, w.dv, 0, kdn.KDN_BF16, kdn.KDN_F32, 0)
+    ws = torch.empty(int(kdn.lib().kdn_backward_workspace_bytes(0, dims)), dtype=torch.uint8, device="cuda")
+
+    def fn():
+        kdn.scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], dO, a=x["a"], dm=dm, workspace=ws)
+    ms = time_device(fn, steps, warmup, dist_on)
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": 2 * steps}
+
+
+def backward_bytes(w, in_bytes=2) -> int:
+    """q, k, v, beta, a, dO, dm in; dq, dk, dv, dbeta, da out (fp32)."""
+    return w.tokens * ((2 * w.dk + w.dv) * in_bytes + 8 + w.dv * 4 + 4 + (2 * w.dk + w.dv) * 4 + 8)
+
+
+def backward_flops(w, C=32) -> int:
+    """Multiply-adds of the chunked backward (forward recompute included) per token: 8 d^2 + 11 C d, times 2."""
+    d = w.dk
+    return w.tokens * 2 * (8 * d * d + 11 * C * d)
+
+
+FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 fp32 FMA lanes at 1965 MHz
+
+
 def hola_bytes(w, in_bytes=2) -> int:
     """q, k, v in, m in, o^cache out (fp32), the final cache indices."""
     return w.tokens * ((2 * w.dk + w.dv) * in_bytes + 4 + w.dv * 4) + w.B * w.H * 64 * 4
@@ -543,6 +574,15 @@ def main():
         also.append({"workload": "hola_cache_read_d128", "variant": "surprise-cache read (w=64, block 64)",
                      "value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"],
                      "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
+        del r
+        torch.cuda.empty_cache()
+        bw = WORKLOADS["gdn_d128"]
+        r = bench_backward(bw, 2, 1, dist_on, rank, world)
+        also.append({"workload": "gdn_d128_backward", "variant": "delta backward (dq, dk, dv, dbeta, da, dS0)",
+                     "value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"],
+                     "roofline_frac": backward_bytes(bw) / (r["ms"] * 1e-3) / 1e9 / peak,
+                     "fp32_flop_frac": backward_flops(bw) / (r["ms"] * 1e-3) / 1e12 / FP32_CUDA_CORE_TFLOPS,
+                     "arith": "f32 CUDA cores"})
         del r
         torch.cuda.empty_cache()
         for name in DECODE:

@@ -33,9 +33,11 @@ bool make_bf16_tmap(CUtensorMap* tm, const void* base, int BH, int L, int d);
 
 // Covariance side of the full-Kalman scan, chunked (Woodbury / LDL): per-token gains into ``gains``
 // ([BH, L, d] fp32) and P updated in place.  d in {64, 128}, bf16 keys.
+// P_starts (optional): [BH, ceil(nchunks / cps), d, d], the covariance entering every run of cps chunks;
+// every run then walks its chunks in its own CTA (grid BH x runs) and the one holding the last chunk writes P_L.
 cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const float* r, const float* qn,
                                 float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const float* P_starts = nullptr, int cps = 0);
 
 // Warp-specialised chunk kernel for d_k = d_v = 128 (preparation of chunk c + 1 beside the state chain
 // of chunk c).  ``gains``: full-Kalman per-token gains [BH, L, 128] fp32, else unused.

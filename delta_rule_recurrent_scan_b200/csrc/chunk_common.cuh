@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "sm100.cuh"
@@ -22,6 +23,27 @@ __device__ __forceinline__ void store8_split(uint8_t* hi, uint8_t* lo, uint32_t 
   sm100::split2_bf16(x[6], x[7], h.w, l.w);
   *reinterpret_cast<uint4*>(hi + off) = h;
   *reinterpret_cast<uint4*>(lo + off) = l;
+}
+
+// 8 consecutive fp32 values -> fp16, stored as one 16-byte chunk.
+__device__ __forceinline__ void store8_f16(uint8_t* dst, uint32_t off, const float (&x)[8]) {
+  uint4 h;
+  h.x = sm100::pack2_f16(x[0], x[1]);
+  h.y = sm100::pack2_f16(x[2], x[3]);
+  h.z = sm100::pack2_f16(x[4], x[5]);
+  h.w = sm100::pack2_f16(x[6], x[7]);
+  *reinterpret_cast<uint4*>(dst + off) = h;
+}
+
+// 8 consecutive fp16 of a swizzled panel (one 16-byte chunk) as floats.
+__device__ __forceinline__ void load8_f16(const uint8_t* base, uint32_t off, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(base + off);
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h[e]);
+    x[2 * e] = f.x, x[2 * e + 1] = f.y;
+  }
 }
 
 // 8 consecutive bf16 of a swizzled panel (one 16-byte chunk) as floats.

@@ -6,26 +6,35 @@
 // Abstract, for the Kalman gains): with A_i = prod_{m<=i} a_m and Gam_ij = A_i / A_j,
 //
 //   (I + N) E = R,   N = strict_lower((K G^T) o Gam),   R = V - diag(A) K S0,
-//   O = diag(A) Q S0 + AT R,   AT = ((Q G^T) o Gam o lower) T,   T = (I + N)^-1,
+//   O = diag(A) Q S0 + Attn E,   Attn = (Q G^T) o Gam o lower,   T = (I + N)^-1,  E = T R,
 //   S_C = A_C S0 + G^T diag(A_C / A_j) E.
 //
 // Everything that does not involve the state (gates, diagonal variances, gains,
-// N, T, AT) is the "preparation" of a chunk; what does (S0 products, R, E, O,
+// N, Attn, T) is the "preparation" of a chunk; what does (S0 products, R, E, O,
 // the state update) is its "chain".  The CTA runs two groups of 8 warps at once:
 // the preparation group works on chunk c + 1 while the chain group works on
 // chunk c, so the serial part of each chunk is the chain alone.
 //
 // The chain runs transposed, with the d_v index on the TMEM lanes, so that every
 // state-dependent operand lives in tensor memory and enters the products as the
-// A operand (bf16 hi/lo pairs, 2-3 MMAs per product):
+// A operand (fp16 pairs, one MMA per product):
 //
 //   D2^T = S0^T [K; Q]^T         A = S0^T (TMEM)      B = [K; Q] tile    -> (K S0)^T | (Q S0)^T
-//   R^T  = V^T - (K S0)^T diag(A)                      (in place, TMEM)
-//   D3^T = R^T [T; AT]^T         A = R^T (TMEM)       B = [T; AT]         -> E^T | (AT R)^T
+//   E^T  = V^T T^T               A = V^T (smem)       B = T               -> issued before D2 is read
+//        - (K S0)^T (T D_A)^T    A = (K S0)^T (TMEM)  B = -T diag(A)      -> E^T (the innovations)
+//   (Attn E)^T = E^T Attn^T      A = E^T (TMEM)       B = Attn            -> O = diag(A) (Q S0) + Attn E
 //   S_C^T = A_C S0^T + E'^T G    A = E'^T (TMEM)      B = G (or K)        accumulated onto the fp32 master
 //
+// so the residual R = V - diag(A) K S0 is never formed: its V part runs on the tensor cores while the
+// chain converts (K S0)^T, and the decay enters through the preparation's scaled copy of T.  The read-out
+// uses Attn E (= AT R, with Attn = lower((Q G^T) o Gam)), so the preparation never forms AT.
+//
 // and the preparation keeps the row-major products [K; Q] G^T and [T; Attn] T.
-// fp32 state master and accumulators in TMEM; K, Q, V enter exactly as bf16.
+// fp32 state master and accumulators in TMEM.  Every tensor-core operand is fp16: K and Q are
+// converted from bf16 in shared memory when their tile lands (exact in fp16's normal range), the fp32
+// operands (state, (K S0), innovations, gains, T, Attn) are rounded to fp16 once.  A float64 emulation of these
+// roundings over 8192-token layers stays below 6e-4 normwise against the exact scan, inside the 3e-3
+// budget for bf16 inputs, while it halves the tensor work and the conversions of the bf16 hi/lo form.
 #include <cuda.h>
 
 #include "chunk.h"
@@ -40,11 +49,11 @@ namespace {
 
 using chunk::kC;
 using chunk::kWaitCycles;
-using chunk::load8_bf16;
 using chunk::named_sync;
 using chunk::named_sync_or;
 using chunk::oct_sum;
-using chunk::store8_split;
+using chunk::load8_f16;
+using chunk::store8_f16;
 
 enum Var : int { kDelta = 0, kDiag = 1, kFull = 2, kIso = 3 };
 
@@ -61,33 +70,35 @@ constexpr int kGD = D / 8;                 // coordinates per thread in the per-
 
 template <int VAR>
 struct WsLayout {
-  static constexpr int KQ_PANEL = 128 * 128;             // [K; Q]: 128 rows x 64 bf16
+  static constexpr int KQ_PANEL = 128 * 128;             // [K; Q]: 128 rows x 64 (bf16 as loaded, then fp16)
   static constexpr int KQ_BYTES = NP * KQ_PANEL;
   static constexpr int NKQ = delta_like(VAR) ? 3 : 2;    // [K; Q] tiles in flight
   static constexpr int V_PANEL = 64 * 128;
   static constexpr int V_BYTES = NP * V_PANEL;
   static constexpr int G_PANEL = 64 * 128;
-  static constexpr int G_HALF = delta_like(VAR) ? 0 : NP * G_PANEL;  // hi or lo of one gain slot
-  static constexpr int TAT_HALF = 128 * 128;             // [T; AT]: 128 rows x 64 bf16, hi or lo
+  static constexpr int G_HALF = delta_like(VAR) ? 0 : NP * G_PANEL;  // fp16 gains of one slot (first half)
+  static constexpr int TAT_HALF = 128 * 128;             // [T; Attn]: 128 rows x 64 fp16
   static constexpr int SCR_BYTES = 64 * chunk::kLD * 4;  // fp32 [64][68]
 
   static constexpr int OFF_KQ = 0;
   static constexpr int OFF_V = OFF_KQ + NKQ * KQ_BYTES;
-  static constexpr int OFF_G = OFF_V + V_BYTES;          // slot s: hi at 2 s G_HALF, lo at (2 s + 1) G_HALF
-  static constexpr int OFF_TAT = OFF_G + 4 * G_HALF;     // hi, then lo
-  static constexpr int OFF_NF = OFF_TAT + 2 * TAT_HALF;
+  static constexpr int OFF_G = OFF_V + V_BYTES;          // slot s at 2 s G_HALF: fp32 gains, then fp16 in its first half
+  static constexpr int OFF_TAT = OFF_G + 4 * G_HALF;     // [T; Attn]
+  static constexpr int OFF_TAD = OFF_TAT + TAT_HALF;     // -T diag(A) (rows 0..63 used)
+  static constexpr int OFF_NF = OFF_TAD + TAT_HALF;
   static constexpr int OFF_TF = OFF_NF + SCR_BYTES;
   static constexpr int TOTAL = OFF_TF + SCR_BYTES;
   static constexpr int SMEM = TOTAL + 1024;              // + alignment slack
-  static_assert(delta_like(VAR) || 64 * D * 4 == 2 * G_HALF, "a gain slot holds the fp32 gains before their split");
+  static_assert(delta_like(VAR) || 64 * D * 4 == 2 * G_HALF, "a gain slot holds the fp32 gains before their fp16 copy");
   static_assert(TOTAL <= 216 * 1024, "shared memory budget");
 
   // TMEM columns
   static constexpr uint32_t T_SM = 0;    // fp32 S^T master: lane j (d_v), column i (d_k)
-  static constexpr uint32_t T_SA = 128;  // S0^T as bf16 pairs: hi 0..63, lo 64..127; later D3^T = E^T | (AT R)^T
-  static constexpr uint32_t T_D2 = 256;  // 0..63: (K S0)^T, then R^T, then E'^T as pairs; 64..127: (Q S0)^T
-  static constexpr uint32_t T_D1 = 384;  // [K; Q] G^T
-  static constexpr uint32_t T_DT = 448;  // [T; Attn] T
+  static constexpr uint32_t T_SA = 128;  // S0^T as fp16 pairs
+  static constexpr uint32_t T_E = 192;   // E^T
+  static constexpr uint32_t T_D2 = 256;  // 0..63: (K S0)^T, then its fp16 pairs, then E'^T pairs; 64..127: (Q S0)^T
+  static constexpr uint32_t T_AR = 384;  // (Attn E)^T
+  static constexpr uint32_t T_D1 = 448;  // [K; Q] G^T (preparation)
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -115,11 +126,9 @@ __device__ __forceinline__ int gf_pos(int i) {
   return (i & ~63) | (h << 5) | ((((i >> 3) & 7) ^ (h << 2)) << 2) | (i & 3);
 }
 
-// Token column u of a 16-token block of bf16 pairs (hi or lo): TMEM column offset.
-// Thread half h holds tokens 32 h .. 32 h + 31 as 16 hi pair columns at 32 h and 16 lo at 32 h + 16.
-__device__ __forceinline__ uint32_t tok_pair_col(int ks, bool lo) {
-  return 32u * (ks >> 1) + (lo ? 16u : 0u) + 8u * (ks & 1);
-}
+// TMEM column of the fp16 pairs of the 16-token block ks (K step of 16): thread half h holds tokens
+// 32 h .. 32 h + 31 as 16 pair columns at 32 h.
+__device__ __forceinline__ uint32_t tok_pair_col(int ks) { return 32u * (ks >> 1) + 8u * (ks & 1); }
 
 template <int VAR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -130,13 +139,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The diagonal variant's chain runs the gates and variances of chunk c + 1 while it waits for the
   // preparation of chunk c; the other variants' preparation runs its own gates.
   constexpr bool kChainGates = VAR == kDiag;
+  // Who converts each [K; Q] tile from bf16 to fp16 in place: the preparation group for the Kalman
+  // variants, whose chain is the longer group; for the delta-like ones the chain, one chunk ahead.
+  constexpr bool kConvInPrep = !delta_like(VAR);
   constexpr int LD = chunk::kLD;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Vs = sm + Lay::OFF_V;
-  uint8_t* TAThi = sm + Lay::OFF_TAT;
-  uint8_t* TATlo = TAThi + Lay::TAT_HALF;
+  uint8_t* TAThi = sm + Lay::OFF_TAT;  // [T; Attn] as fp16
+  uint8_t* TADs = sm + Lay::OFF_TAD;   // -T diag(A) as fp16 (rows 0..63)
   float* Nf = reinterpret_cast<float*>(sm + Lay::OFF_NF);
   float* Tf = reinterpret_cast<float*>(sm + Lay::OFF_TF);
 
@@ -144,11 +156,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];         // a, beta | r, Qn
   __shared__ float ell[2][kC], gn[2][kC];
   __shared__ __align__(16) float Aex[2][kC];                // A_t
+  __shared__ __align__(16) float gcol[2][kC];               // 1 / A_t (times beta_t for the delta rule), when
+                                                            // the chunk's decay stays above exp(-80)
   __shared__ __align__(16) float esc[2][kC];                // scale of row t of E in the state update:
                                                             // A_C / A_t (times beta_t for the delta rule)
   __shared__ float en[4][kC];                               // ||e_t||^2 partials per lane quarter
   __shared__ float knorm[kC];                               // isotropic: ||k_t||^2 of the chunk
-  __shared__ uint64_t kq_full[NKQ], v_full, bar_c, bar_p, tat_free;
+  __shared__ float pend[VAR == kDiag ? D : 1];              // diagonal: p after the chunk whose variances ran
+  __shared__ uint64_t kq_full[NKQ], kq_conv[NKQ], v_full, bar_c, bar_o, bar_p, tat_free;
   __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2], var_done[2];
   __shared__ uint32_t tmem_base;
 
@@ -172,6 +187,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL + 64 * 128, &tm_q, &kq_full[slot], 64 * pn, cc * kC, bh);
     }
   };
+  // bf16 -> fp16 in place over a [K; Q] slot (2 tensors x 2 panels x 64 rows x 8 chunks of 16 bytes) by the
+  // 256 threads u of one group, made visible to the tensor cores by the fence
+  auto convert_kq = [&](int cc, int u) {
+    uint8_t* KQs = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      uint4* p4 = reinterpret_cast<uint4*>(KQs) + u + kGroup * r;
+      uint4 w = *p4;
+      w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
+      w.z = sm100::bf16x2_to_f16x2(w.z), w.w = sm100::bf16x2_to_f16x2(w.w);
+      *p4 = w;
+    }
+    sm100::fence_async_smem();
+  };
   auto issue_v = [&](int cc) {
     sm100::mbar_arrive_expect_tx(&v_full, NP * 64 * 128);
 #pragma unroll
@@ -183,9 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::prefetch_tmap(&tm_k);
     sm100::prefetch_tmap(&tm_v);
 #pragma unroll
-    for (int i = 0; i < NKQ; ++i) sm100::mbar_init(&kq_full[i], 1);
+    for (int i = 0; i < NKQ; ++i) sm100::mbar_init(&kq_full[i], 1), sm100::mbar_init(&kq_conv[i], 1);
     sm100::mbar_init(&v_full, 1);
     sm100::mbar_init(&bar_c, 1);
+    sm100::mbar_init(&bar_o, 1);
     sm100::mbar_init(&bar_p, 1);
     sm100::mbar_init(&tat_free, 1);
     for (int i = 0; i < 2; ++i) {
@@ -240,6 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float r0 = __expf(lC - x0), r1 = __expf(lC - x1);  // A_C / A_t without a division
     esc[sl][lane] = delta_like(VAR) ? r0 * sB[sl][lane] : r0;
     esc[sl][32 + lane] = delta_like(VAR) ? r1 * sB[sl][32 + lane] : r1;
+    // Gam_ij = A_i (1 / A_j) without an exponential per pair: safe (no overflow) while ell_C >= -80
+    gcol[sl][lane] = __expf(-x0) * (delta_like(VAR) ? sB[sl][lane] : 1.f);
+    gcol[sl][32 + lane] = __expf(-x1) * (delta_like(VAR) ? sB[sl][32 + lane] : 1.f);
   };
   fetch_scalars(0);
   store_scalars(0);
@@ -254,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j = row;                       // d_v index
     const bool leader = tid == 0;            // issues the chain's products and every TMA load
     bool aborted = false;
-    uint32_t ph_c = 0;
+    uint32_t ph_c = 0, ph_o = 0;
     auto gwait = [&](uint64_t* b, uint32_t parity) -> bool {
       bool bad = false;
       if (leader) bad = !sm100::mbar_wait_bounded(b, parity, kWaitCycles);
@@ -267,15 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // x = S[64 half + 32 v .. + 31][j]
     // x = S[dk0 .. dk0 + 31][j]
     auto emit_state = [&](float (&x)[32], int dk0, float scale) {
-      float hw[16], lw[16];
+      float hw[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        uint32_t hu, lu;
-        sm100::split2_bf16(x[2 * e], x[2 * e + 1], hu, lu);
-        hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
-      }
+      for (int e = 0; e < 16; ++e) hw[e] = __uint_as_float(sm100::pack2_f16(x[2 * e], x[2 * e + 1]));
       sm100::tmem_st16(tmem + t_lane + Lay::T_SA + dk0 / 2, hw);
-      sm100::tmem_st16(tmem + t_lane + Lay::T_SA + 64 + dk0 / 2, lw);
 #pragma unroll
       for (int e = 0; e < 32; ++e) x[e] *= scale;
       sm100::tmem_st32(tmem + t_lane + Lay::T_SM + dk0, x);
@@ -283,39 +311,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     // D2^T = S0^T [K; Q]^T, K steps 4 part .. 4 part + 3 (d_k 64 part ..): issued as soon as that half of
     // the S0^T pairs is in tensor memory; the second half commits
     auto issue_d2 = [&](uint32_t kq_addr, int part) {
-      constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t id = sm100::idesc_f16(128, 128, false, false);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int ks = 4 * part + u;
         const uint64_t b = sm100::smem_desc(kq_addr + (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32, 16, 1024);
         sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 8 * ks, b, id, ks > 0);
-        sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 64 + 8 * ks, b, id, true);
       }
       if (part == 1) sm100::mma_commit(&bar_c);
     };
     auto kq_addr_of = [&](int cc) { return sm100::smem_u32(sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES); };
 
-    // Diagonal variances of chunk cc (threads 0..D-1, coordinate i = tid; independent of v and S), run one
-    // chunk ahead while the chain waits for the preparation.  Per coordinate: p^- = a^2 p + Qn,
-    // pk = p^- k, p <- p^- r / (r + pk k), on the homogeneous pair p = x / y (x^- = a^2 x + Qn y,
-    // x <- r x^-, y <- r y + k^2 x^-): three multiply-adds of serial chain per token, the division that
-    // recovers p^- off the chain, and a power-of-two rescale every four tokens that keeps y in [1, 2).
-    // The unnormalised gains pk go, fp32, into the gain slot of chunk cc.
+    // Diagonal variances of chunk cc (independent of v and S), run one chunk ahead while the chain waits for
+    // the preparation.  Per coordinate: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the
+    // homogeneous pair p = x / y: token t maps (x, y) by M_t = [[r a^2, r Qn], [k^2 a^2, k^2 Qn + r]], three
+    // multiply-adds of serial chain per token, the division that recovers p^- off the chain, and a
+    // power-of-two rescale every four tokens that keeps y in [1, 2).  Two threads per coordinate: thread i
+    // runs tokens 0..31 from p, thread D + i runs tokens 32..63 from the product of the first 32 maps
+    // applied to p (the maps compose: Kalman Delta Networks, Abstract, uncertainty recurrences as Moebius
+    // maps), so the serial part is half a chunk.  The unnormalised gains pk go, fp32, into the gain slot of
+    // chunk cc; the value after the chunk goes to pend[i], read by both threads after the group's barrier.
     float pcur = 1.f;
-    if (VAR == kDiag && tid < D) pcur = P.p[(size_t)bh * D + tid];
+    if (VAR == kDiag) pcur = P.p[(size_t)bh * D + (tid & (D - 1))];
     auto run_variances = [&](int cc) {
-      if (VAR == kDiag && tid < D) {
+      if (VAR == kDiag) {
+        const int i = tid & (D - 1), hh = tid / D;  // coordinate, token half (the chain group is 2 D threads)
         const int sl = cc & 1;
-        const uint8_t* Kp = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES + (tid / 64) * Lay::KQ_PANEL;
+        // keys from the chunk's K tile as it landed (bf16): the preparation converts that tile to fp16 only
+        // after these variances are done
+        const uint8_t* Kp = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES + (i / 64) * Lay::KQ_PANEL;
+        auto key = [&](int t) {
+          return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t, i % 64)));
+        };
         float* Gw = reinterpret_cast<float*>(sm + Lay::OFF_G + 2 * sl * Lay::G_HALF);
-        const int gpos = gf_pos(tid);
+        const int gpos = gf_pos(i);
         float x = pcur, y = 1.f;
+        auto rescale = [&]() {
+          const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
+          const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
+          x *= sc, y *= sc;
+        };
+        if (hh == 1) {
+          // (x, y) <- M_31 ... M_0 (x, y), eight maps multiplied out at a time, then applied
 #pragma unroll 1
-        for (int t8 = 0; t8 < kC; t8 += 8) {
+          for (int t8 = 0; t8 < kC / 2; t8 += 8) {
+            float m00 = 1.f, m01 = 0.f, m10 = 0.f, m11 = 1.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float kv = key(t8 + u);
+              const float av = sA[sl][t8 + u], rv = sB[sl][t8 + u], qv = sQ[sl][t8 + u];
+              const float a2 = av * av, k2 = kv * kv;
+              const float b00 = rv * a2, b01 = rv * qv, b10 = k2 * a2, b11 = fmaf(k2, qv, rv);
+              const float n00 = fmaf(b00, m00, b01 * m10), n01 = fmaf(b00, m01, b01 * m11);
+              const float n10 = fmaf(b10, m00, b11 * m10), n11 = fmaf(b10, m01, b11 * m11);
+              m00 = n00, m01 = n01, m10 = n10, m11 = n11;
+            }
+            const float xn = fmaf(m00, x, m01 * y), yn = fmaf(m10, x, m11 * y);
+            x = xn, y = yn;
+            rescale();
+          }
+        }
+#pragma unroll 1
+        for (int t8 = hh * (kC / 2); t8 < (hh + 1) * (kC / 2); t8 += 8) {
           float kk[8], aa[8], rr8[8], qq[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, tid % 64)));
+            kk[u] = key(t8 + u);
             aa[u] = sA[sl][t8 + u], rr8[u] = sB[sl][t8 + u], qq[u] = sQ[sl][t8 + u];
           }
 #pragma unroll
@@ -324,29 +385,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             Gw[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
             x = rr8[u] * xm;
             y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
-            if (u % 4 == 3) {
-              const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
-              const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
-              x *= sc, y *= sc;
-            }
+            if (u % 4 == 3) rescale();
           }
         }
-        pcur = __fdividef(x, y);
+        if (hh == 1) pend[i] = __fdividef(x, y);
       }
     };
 
     float* Sg = P.S + (size_t)bh * D * D;
-    if (kChainGates) {  // gates and variances of chunk 0 (its scalars are in slot 0 already)
+    if (!kConvInPrep) {  // [K; Q] of chunk 0
+      if (!gwait(&kq_full[0], 0)) {
+        aborted = true;
+      } else {
+        convert_kq(0, tid);
+        named_sync(kBarChain, kGroup);
+        if (leader) sm100::mbar_arrive(&kq_conv[0]);
+      }
+    }
+    if (!aborted && kChainGates) {  // gates and variances of chunk 0 (its scalars are in slot 0 already)
       if (!gwait(&kq_full[0], 0)) {
         aborted = true;
       } else {
         run_variances(0);
         if (gw == 4) run_gates(0);
         named_sync(kBarChain, kGroup);
+        if (VAR == kDiag) pcur = pend[tid & (D - 1)];
         if (leader) sm100::mbar_arrive(&var_done[0]);
       }
     }
-    if (aborted || (!kChainGates && !gwait(&gates_ready[0], 0)) || !gwait(&kq_full[0], 0)) {
+    if (aborted || (!kChainGates && !gwait(&gates_ready[0], 0)) || !gwait(&kq_conv[0], 0)) {
       aborted = true;
     } else {
       const float AC0 = Aex[0][kC - 1];
@@ -365,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    const uint32_t tat_hi = sm100::smem_u32(TAThi), tat_lo = sm100::smem_u32(TATlo);
+    const uint32_t tat_hi = sm100::smem_u32(TAThi);
     for (int c = 0; c < nchunks && !aborted; ++c) {
       const int s = c & 1, kslot = c % NKQ;
       const int t0 = c * kC;
@@ -373,13 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // D2^T = S0^T [K; Q]^T of this chunk was issued with its state operands (end of the previous chunk)
 
-      // ---------------------------------------------------------------- R^T = V^T - (K S0)^T diag(A), in place
-      // V and the gates first: the column of V this thread needs is read while the S0 product runs
+      // ---------------------------------------------------------------- V of this chunk to fp16, the gates
       {
         bool bad = false;
         if (leader) {
           bad = !sm100::mbar_wait_bounded(&v_full, c & 1, kWaitCycles) ||
                 !sm100::mbar_wait_bounded(&gates_ready[s], (c >> 1) & 1, kWaitCycles);
+          if (!bad && !kConvInPrep && c + 1 < nchunks)
+            bad = !sm100::mbar_wait_bounded(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1, kWaitCycles);
         }
         bad = named_sync_or(kBarChain, kGroup, bad);
         if (bad) {
@@ -387,116 +455,120 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
+        // 2 panels x 64 rows x 8 chunks of 16 bytes: four chunks per thread (made visible to the MMA by the
+        // fence here and the barrier of the prep_done wait below)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4* p4 = reinterpret_cast<uint4*>(Vs) + tid + kGroup * u;
+          uint4 w = *p4;
+          w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
+          w.z = sm100::bf16x2_to_f16x2(w.z), w.w = sm100::bf16x2_to_f16x2(w.w);
+          *p4 = w;
+        }
+        sm100::fence_async_smem();
+        if (!kConvInPrep && c + 1 < nchunks) {  // [K; Q] of the next chunk, for the preparation
+          convert_kq(c + 1, tid);
+          named_sync(kBarChain, kGroup);
+          if (leader) sm100::mbar_arrive(&kq_conv[(c + 1) % NKQ]);
+        }
       }
       // ---------------------------------------------------------------- variances of chunk c + 1, while the S0 product runs
       if (kChainGates && c + 1 < nchunks) {
-        // its scalars were stored before gates_ready of chunk c, its K before the slot's load completed
+        // its scalars were stored before gates_ready of chunk c; its keys are read before the preparation
+        // converts their tile (that waits for var_done)
         if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
         run_variances(c + 1);
         if (gw == 4) run_gates(c + 1);
         named_sync(kBarChain, kGroup);
+        if (VAR == kDiag) pcur = pend[tid & (D - 1)];
         if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
       }
 
-      {
-        const uint8_t* vp = Vs + (j / 64) * Lay::V_PANEL;
-        uint32_t vv[16];  // V[t][j] for the 32 tokens of this half, as bf16 pairs (t even in the low half)
+      // ---------------------------------------------------------------- E^T = V^T T^T, queued behind the S0 product
+      if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_f16(128, 64, true, false);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int t = 32 * half + 2 * e;
-          const uint32_t v0 = *reinterpret_cast<const uint16_t*>(vp + sm100::sw128(t, j % 64));
-          const uint32_t v1 = *reinterpret_cast<const uint16_t*>(vp + sm100::sw128(t + 1, j % 64));
-          vv[e] = v0 | (v1 << 16);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t a = sm100::smem_desc(sm100::smem_u32(Vs) + ks * 2048, Lay::V_PANEL, 1024);
+          sm100::mma_bf16(tmem + Lay::T_E, a, sm100::smem_desc(tat_hi + ks * 32, 16, 1024), id, ks > 0);
         }
+      }
+
+      // ---------------------------------------------------------------- (K S0)^T to fp16 pairs, in place
+      {
         if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
         ph_c ^= 1;
         float X[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + 32 * half, X);
         sm100::tmem_wait_ld();
-        const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
-        float hw[16], lw[16];
+        float hw[16];
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 av = A4[e4];
-          const float aa[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int e = 2 * e4 + e2;
-            const float v0 = __uint_as_float(vv[e] << 16), v1 = __uint_as_float(vv[e] & 0xffff0000u);
-            uint32_t hu, lu;
-            sm100::split2_bf16(fmaf(-aa[2 * e2], X[2 * e], v0), fmaf(-aa[2 * e2 + 1], X[2 * e + 1], v1), hu, lu);
-            hw[e] = __uint_as_float(hu), lw[e] = __uint_as_float(lu);
-          }
-        }
+        for (int e = 0; e < 16; ++e) hw[e] = __uint_as_float(sm100::pack2_f16(X[2 * e], X[2 * e + 1]));
         sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);
-        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half + 16, lw);
         sm100::tmem_wait_st();
       }
       sm100::tc_fence_before();
       named_sync(kBarChain, kGroup);
       sm100::tc_fence_after();
-      if (leader && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
 
-      // ---------------------------------------------------------------- D3^T = R^T [T; AT]^T
-      if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
+      // ---------------------------------------------------------------- E^T -= (K S0)^T (T diag(A))^T
       if (leader) {
-        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id = sm100::idesc_f16(128, 64, false, false);
+        const uint32_t tad = sm100::smem_u32(TADs);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bh_ = sm100::smem_desc(tat_hi + ks * 32, 16, 1024);
-          const uint64_t bl = sm100::smem_desc(tat_lo + ks * 32, 16, 1024);
-          const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks, false);
-          const uint32_t al = tmem + Lay::T_D2 + tok_pair_col(ks, true);
-          sm100::mma_bf16_ts(tmem + Lay::T_SA, ah, bh_, id, ks > 0);
-          sm100::mma_bf16_ts(tmem + Lay::T_SA, al, bh_, id, true);
-          sm100::mma_bf16_ts(tmem + Lay::T_SA, ah, bl, id, true);
+          const uint32_t a = tmem + Lay::T_D2 + tok_pair_col(ks);
+          sm100::mma_bf16_ts(tmem + Lay::T_E, a, sm100::smem_desc(tad + ks * 32, 16, 1024), id, true);
         }
         sm100::mma_commit(&bar_c);
-        sm100::mma_commit(&tat_free);
       }
       if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
       ph_c ^= 1;
+      if (leader && c + 1 < nchunks) issue_v(c + 1);  // V of this chunk is dead
 
       // ---------------------------------------------------------------- E' pairs; S^T master += E'^T G; ||e||^2
       float E[32];
       {
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_SA + 32 * half, E);
+        sm100::tmem_ld32(tmem + t_lane + Lay::T_E + 32 * half, E);
         sm100::tmem_wait_ld();
         const float4* S4 = reinterpret_cast<const float4*>(&esc[s][32 * half]);
-        float hw[16], lw[16];
+        float hw[16], ew[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 sv = S4[e4];
-          uint32_t hu, lu;
-          sm100::split2_bf16(E[4 * e4] * sv.x, E[4 * e4 + 1] * sv.y, hu, lu);
-          hw[2 * e4] = __uint_as_float(hu), lw[2 * e4] = __uint_as_float(lu);
-          sm100::split2_bf16(E[4 * e4 + 2] * sv.z, E[4 * e4 + 3] * sv.w, hu, lu);
-          hw[2 * e4 + 1] = __uint_as_float(hu), lw[2 * e4 + 1] = __uint_as_float(lu);
+          hw[2 * e4] = __uint_as_float(sm100::pack2_f16(E[4 * e4] * sv.x, E[4 * e4 + 1] * sv.y));
+          hw[2 * e4 + 1] = __uint_as_float(sm100::pack2_f16(E[4 * e4 + 2] * sv.z, E[4 * e4 + 3] * sv.w));
+          ew[2 * e4] = __uint_as_float(sm100::pack2_f16(E[4 * e4], E[4 * e4 + 1]));
+          ew[2 * e4 + 1] = __uint_as_float(sm100::pack2_f16(E[4 * e4 + 2], E[4 * e4 + 3]));
         }
-        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);
-        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half + 16, lw);
+        sm100::tmem_st16(tmem + t_lane + Lay::T_D2 + 32 * half, hw);  // E' pairs, over the dead (K S0) pairs
+        sm100::tmem_st16(tmem + t_lane + Lay::T_E + 32 * half, ew);   // E pairs, in place
       }
       sm100::tmem_wait_st();
       sm100::tc_fence_before();
       named_sync(kBarChain, kGroup);
       sm100::tc_fence_after();
       if (leader) {
-        constexpr uint32_t id = sm100::idesc_bf16(128, 128, false, true);
+        // (Attn E)^T = E^T Attn^T for the read-out first (it frees [T; Attn]), then the state product
+        constexpr uint32_t ido = sm100::idesc_f16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          sm100::mma_bf16_ts(tmem + Lay::T_AR, tmem + Lay::T_E + tok_pair_col(ks),
+                             sm100::smem_desc(tat_hi + 64 * 128 + ks * 32, 16, 1024), ido, ks > 0);
+        sm100::mma_commit(&bar_o);
+        sm100::mma_commit(&tat_free);
+        constexpr uint32_t id = sm100::idesc_f16(128, 128, false, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks, false);
-          const uint32_t al = tmem + Lay::T_D2 + tok_pair_col(ks, true);
+          const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks);
           if (delta_like(VAR)) {
             const uint64_t bk = sm100::smem_desc(kq0 + ks * 2048, Lay::KQ_PANEL, 1024);
             sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bk, id, true);
-            sm100::mma_bf16_ts(tmem + Lay::T_SM, al, bk, id, true);
           } else {
             const uint32_t g0 = sm100::smem_u32(sm + Lay::OFF_G + 2 * s * Lay::G_HALF);
             const uint64_t bgh = sm100::smem_desc(g0 + ks * 2048, Lay::G_PANEL, 1024);
-            const uint64_t bgl = sm100::smem_desc(g0 + Lay::G_HALF + ks * 2048, Lay::G_PANEL, 1024);
             sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bgh, id, true);
-            sm100::mma_bf16_ts(tmem + Lay::T_SM, al, bgh, id, true);
-            sm100::mma_bf16_ts(tmem + Lay::T_SM, ah, bgl, id, true);
           }
         }
         sm100::mma_commit(&bar_c);
@@ -516,7 +588,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       en[qw][32 * half + lane] = E[0];
-      // O = diag(A) Q S0 + AT R, while the state product runs (it touches neither column range)
+      // O = diag(A) Q S0 + Attn E (Attn E = AT R), while the state product runs (it touches neither column range)
+      if (!gwait(&bar_o, ph_o)) { aborted = true; break; }
+      ph_o ^= 1;
       {
         const bool full = t0 + kC <= L;
         const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
@@ -525,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < 2; ++hh) {
           float Y[16], Oi[16];
           sm100::tmem_ld16(tmem + t_lane + Lay::T_D2 + 64 + 32 * half + 16 * hh, Y);
-          sm100::tmem_ld16(tmem + t_lane + Lay::T_SA + 64 + 32 * half + 16 * hh, Oi);
+          sm100::tmem_ld16(tmem + t_lane + Lay::T_AR + 32 * half + 16 * hh, Oi);
           sm100::tmem_wait_ld();
           float ov[16];
 #pragma unroll
@@ -558,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S0 product, a half at a time
       if (c + 1 < nchunks) {
         if (!kChainGates && !gwait(&gates_ready[s ^ 1], ((c + 1) >> 1) & 1)) { aborted = true; break; }
-        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
+        if (!gwait(&kq_conv[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
         const float ACn = Aex[s ^ 1][kC - 1];
         const uint32_t kq_next = kq_addr_of(c + 1);
 #pragma unroll
@@ -609,14 +683,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* KQ = sm + Lay::OFF_KQ + kslot * Lay::KQ_BYTES;
       const uint32_t kq0 = sm100::smem_u32(KQ);
       uint8_t* Ghi = sm + Lay::OFF_G + 2 * s * Lay::G_HALF;
-      uint8_t* Glo = Ghi + Lay::G_HALF;
 
       // ---------------------------------------------------------------- slot s free (chain of c - 2), K, Q of c
       {
         bool bad = false;
         if (leader) {
           if (c >= 2) bad = !sm100::mbar_wait_bounded(&chain_done[s], ((c - 2) >> 1) & 1, kWaitCycles);
-          if (!bad) bad = !sm100::mbar_wait_bounded(&kq_full[kslot], (c / NKQ) & 1, kWaitCycles);
+          if (!bad) bad = !sm100::mbar_wait_bounded(kConvInPrep ? &kq_full[kslot] : &kq_conv[kslot], (c / NKQ) & 1,
+                                                    kWaitCycles);
         }
         bad = named_sync_or(kBarPrep, kGroup, bad);
         if (bad) {
@@ -624,6 +698,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
+      }
+      // ---------------------------------------------------------------- K, Q of this chunk: bf16 -> fp16 in place
+      // (the diagonal variant's chain reads the bf16 keys for its variances first: converted below)
+      if (kConvInPrep && !kChainGates) {
+        convert_kq(c, pt);
+        named_sync(kBarPrep, kGroup);
+        if (leader) sm100::mbar_arrive(&kq_conv[kslot]);
       }
       // ---------------------------------------------------------------- isotropic: beta of this chunk
       if (VAR == kIso) {
@@ -635,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < NP; ++pn) {
             float xk[8];
-            load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
+            load8_f16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
 #pragma unroll
             for (int e = 0; e < 8; ++e) sq = fmaf(xk[e], xk[e], sq);
           }
@@ -696,14 +777,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
+        convert_kq(c, pt);
+        named_sync(kBarPrep, kGroup);
+        if (leader) sm100::mbar_arrive(&kq_conv[kslot]);
       }
 
       // ---------------------------------------------------------------- gains: norms, hi/lo panels (8 threads per token)
       {
         // Thread `part` of token t takes the 16-byte chunk `part` of every 64-wide panel: coordinates
         // 64 pn + 8 part .. + 7, so each group of eight lanes reads and writes one whole 128-byte row.
-        // The diagonal variant normalises the fp32 gains that share the slot with their hi/lo split: all
-        // of them are read before any split is written.
+        // The diagonal variant normalises the fp32 gains that share the slot with their fp16 copy: all
+        // of them are read before any of the copy is written.
         const int part = pt & 7;
         float g[2][kGD];
 #pragma unroll
@@ -713,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < NP; ++pn) {
             float xk[8];
-            load8_bf16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
+            load8_f16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
 #pragma unroll
             for (int e = 0; e < 8; ++e) kv[8 * pn + e] = xk[e];
           }
@@ -772,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float xg[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) xg[e] = g[pass][8 * pn + e];
-              store8_split(Ghi, Glo, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
+              store8_f16(Ghi, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
             }
           }
         }
@@ -784,8 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---------------------------------------------------------------- D1 = [K; Q] G^T
       if (leader) {
-        constexpr uint32_t id1 = sm100::idesc_bf16(128, 64, false, false);
-        const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
+        constexpr uint32_t id1 = sm100::idesc_f16(128, 64, false, false);
+        const uint32_t ghi = sm100::smem_u32(Ghi);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
@@ -795,7 +879,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
             sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + goff, 16, 1024), id1, ks > 0);
-            sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(glo + goff, 16, 1024), id1, true);
           }
         }
         sm100::mma_commit(&bar_p);
@@ -821,37 +904,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         float Y[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * half, Y);
         sm100::tmem_wait_ld();
-        if (qw < 2) {
-          const int i = row;
-          const float li = ell[s][i];
+        // Y_ij (beta_j) Gam_ij: as A_i times the column factor when the chunk's decay allows it, else by
+        // one exponential per pair (chunks with strong resets); the choice is uniform over the chunk
+        const int i = row & 63;
+        const float li = ell[s][i], Ai = Aex[s][i];
+        auto emit = [&](auto gam) {
+          if (qw < 2) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float v4[4];
+            for (int e = 0; e < 32; e += 4) {
+              float v4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int jj = 32 * half + e + u;
-              v4[u] = (jj < i) ? Y[e + u] * __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f) : 0.f;
+              for (int u = 0; u < 4; ++u) {
+                const int jj = 32 * half + e + u;
+                v4[u] = (jj < i) ? Y[e + u] * gam(jj) : 0.f;
+              }
+              *reinterpret_cast<float4*>(Nf + i * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
             }
-            *reinterpret_cast<float4*>(Nf + i * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-          }
-        } else {
-          const int i = row - 64;
-          const float li = ell[s][i];
+          } else {
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            float xa[8];
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float xa[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int jj = 32 * half + 8 * q8 + e;
-              xa[e] = (jj <= i) ? Y[8 * q8 + e] * __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f) : 0.f;
+              for (int e = 0; e < 8; ++e) {
+                const int jj = 32 * half + 8 * q8 + e;
+                xa[e] = (jj <= i) ? Y[8 * q8 + e] * gam(jj) : 0.f;
+              }
+              store8_f16(TAThi, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
             }
-            store8_split(TAThi, TATlo, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
           }
-        }
+        };
+        if (ell[s][kC - 1] >= -80.f)
+          emit([&](int jj) { return Ai * gcol[s][jj]; });
+        else
+          emit([&](int jj) { return __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f); });
       }
       named_sync(kBarPrep, kGroup);
 
-      // ---------------------------------------------------------------- T = (I + N)^-1 into rows 0..63 of [T; AT]
+      // ---------------------------------------------------------------- T = (I + N)^-1 into rows 0..63 of [T; Attn]
       chunk::invert_unit_lower_64(Nf, Tf, pt, [] { named_sync(kBarPrep, kGroup); });
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -860,62 +949,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 lo4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8);
         const float4 hi4 = *reinterpret_cast<const float4*>(Tf + i * LD + 8 * c8 + 4);
         const float tv[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
-        float xt[8];
+        float xt[8], xd[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int jj = 8 * c8 + u;
           xt[u] = (jj < i) ? tv[u] : (jj == i ? 1.f : 0.f);
+          xd[u] = -xt[u] * Aex[s][jj];
         }
-        store8_split(TAThi, TATlo, sm100::sw128_chunk(i, c8), xt);
+        store8_f16(TAThi, sm100::sw128_chunk(i, c8), xt);
+        store8_f16(TADs, sm100::sw128_chunk(i, c8), xd);
       }
       sm100::fence_async_smem();
       sm100::tc_fence_before();
       named_sync(kBarPrep, kGroup);
       sm100::tc_fence_after();
 
-      // ---------------------------------------------------------------- DT = [T; Attn] T  (rows 64..127: AT)
-      if (leader) {
-        constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, true);
-        const uint32_t thi = sm100::smem_u32(TAThi), tlo = sm100::smem_u32(TATlo);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ah = sm100::smem_desc(thi + ks * 32, 16, 1024), al = sm100::smem_desc(tlo + ks * 32, 16, 1024);
-          const uint64_t bh_ = sm100::smem_desc(thi + ks * 2048, 16, 1024), bl = sm100::smem_desc(tlo + ks * 2048, 16, 1024);
-          sm100::mma_bf16(tmem + Lay::T_DT, ah, bh_, id, ks > 0);
-          sm100::mma_bf16(tmem + Lay::T_DT, al, bh_, id, true);
-          sm100::mma_bf16(tmem + Lay::T_DT, ah, bl, id, true);
-        }
-        sm100::mma_commit(&bar_p);
-      }
-      {
-        bool bad = false;
-        if (leader) bad = !sm100::mbar_wait_bounded(&bar_p, ph_p, kWaitCycles);
-        bad = named_sync_or(kBarPrep, kGroup, bad);
-        if (bad) {
-          if (leader) raise_status(P.status, kStatusTimeout);
-          aborted = true;
-          break;
-        }
-        sm100::tc_fence_after();
-        ph_p ^= 1;
-      }
-      if (qw >= 2) {
-        const int i = row - 64;
-        float X[32];
-        sm100::tmem_ld32(tmem + t_lane + Lay::T_DT + 32 * half, X);
-        sm100::tmem_wait_ld();
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          float xa[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xa[e] = X[8 * q8 + e];
-          store8_split(TAThi, TATlo, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
-        }
-      }
-      sm100::fence_async_smem();
-      sm100::tc_fence_before();
-      named_sync(kBarPrep, kGroup);
-      sm100::tc_fence_after();
       if (leader) sm100::mbar_arrive(&prep_done[s]);
     }
     if (VAR == kIso && !aborted && gw == 4 && lane == 0) P.p[bh] = c_iso;

@@ -7,6 +7,7 @@
 
 #include <cstdio>
 #include <string>
+#include <utility>
 
 #include "../../include/kdn.h"
 #include "api_internal.h"
@@ -120,6 +121,13 @@ kdn_status resolve_segments(kdn_variant var, const kdn_dims* d, int* P_out) {
       return KDN_OK;
     }
   return KDN_OK;
+}
+
+// Full Kalman with P segments: the covariance side runs as P runs of chunks (the last one possibly shorter),
+// each from its own start covariance.
+int riccati_run_chunks(const kdn_dims* d, int P) {
+  const int nch = (d->L + 63) / 64;
+  return (nch + P - 1) / P;
 }
 
 // Byte offsets inside the segment area of the workspace.
@@ -252,6 +260,9 @@ size_t kdn_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
   if (resolve_segments(variant, dims, &P) != KDN_OK) return 0;
   size_t n = seg_area_offset(variant, dims);
   if (P > 1) n += seg_layout(body_of(variant), dims, P).end;
+  // few heads, full Kalman: the covariance side runs chunk-parallel from every chunk's start covariance
+  if (P > 1 && variant == KDN_KALMAN_FULL)
+    n = round256(n) + kdn::riccati_scratch_bytes(dims->dk, dims->B * dims->H, dims->L, riccati_run_chunks(dims, P));
   return round256(n);
 }
 
@@ -278,7 +289,7 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
   KDN_TRY(resolve_segments(variant, dims, &nseg));
   if (nseg > 1) {
     // start states, two map runs, chaining, the true run (+ the diagonal uncertainty maps and starts)
-    n = 5 + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 1 : 0);
+    n = 5 + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 4 : 0);
   }
   if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1))
     n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself on the serial path)
@@ -367,9 +378,28 @@ kdn_status kdn::api::kalman_scan(kdn_variant var, const kdn_dims* dims, const vo
     if (nseg > 1) {
       float* gains = nullptr;
       if (var == KDN_KALMAN_FULL) {
-        // the covariance side is one serial pass per head; its gains fix every segment's memory map
+        // the covariance at every chunk start through the chunks' Riccati transfer matrices, then every
+        // chunk's gains at once; the gains fix every segment's memory map
         gains = reinterpret_cast<float*>(c.workspace);
-        KDN_TRY(cuda_status(kdn::launch_kalman_pside(dims->dk, k, a, r, qn, qn_scalar, P, gains, status, BH, dims->L, st),
+        char* area = reinterpret_cast<char*>(workspace) + seg_area_offset(var, dims);
+        char* rs = area + round256(seg_layout(KDN_KALMAN_FULL, dims, nseg).end);
+        const int cps = riccati_run_chunks(dims, nseg), nch = (dims->L + 63) / 64;
+        const size_t chunks = (size_t)BH * nch, runs = (size_t)BH * ((nch + cps - 1) / cps), dk = dims->dk;
+        kdn::RiccatiArgs ra{};
+        ra.k = k, ra.a = a, ra.r = r, ra.qn = qn, ra.qn_scalar = qn_scalar, ra.P0 = P, ra.cps = cps;
+        ra.map_w = reinterpret_cast<float*>(rs);
+        rs += round256(chunks * 64 * 2 * dk * 4);
+        ra.map_u = reinterpret_cast<float*>(rs);
+        rs += round256(chunks * 64 * 4);
+        ra.map_ab = reinterpret_cast<float*>(rs);
+        rs += round256(chunks * 2 * 4);
+        ra.xy = reinterpret_cast<float*>(rs);
+        rs += round256(runs * 2 * dk * dk * 4);
+        ra.P_starts = reinterpret_cast<float*>(rs);
+        ra.status = status, ra.BH = BH, ra.L = dims->L;
+        KDN_TRY(cuda_status(kdn::launch_riccati_starts(dims->dk, ra, st), "Kalman run-start covariance launch"));
+        KDN_TRY(cuda_status(kdn::launch_kalman_pside(dims->dk, k, a, r, qn, qn_scalar, P, gains, status, BH, dims->L, st,
+                                                     ra.P_starts, cps),
                             "Kalman covariance launch"));
       }
       return seg_scan(var, dims, nseg, c, gains, reinterpret_cast<char*>(workspace) + seg_area_offset(var, dims), st);
@@ -443,6 +473,72 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
   }
   kdn::SeqScanArgs sa{q, k, v, dims->in_dtype, dims->out_dtype, beta, a, nullptr, S, o, m, BH, dims->L};
   return cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, sa, st), "isotropic scan launch");
+}
+
+size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
+  if (variant != KDN_DELTA || dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
+  if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
+  const size_t BH = (size_t)dims->B * dims->H, DD = (size_t)dims->dk * dims->dv;
+  const size_t nck = ((size_t)dims->L + kdn::kDeltaBwdChunk - 1) / kdn::kDeltaBwdChunk;
+  return kStatusBytes + round256(BH * DD * 4) + round256(BH * nck * DD * 4) + round256(BH * (size_t)dims->L * 4);
+}
+
+kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
+                                   const float* a, const float* S0, const float* dO, const float* dm, const float* dS_L,
+                                   float* dq, float* dk, float* dv, float* dbeta, float* da, float* dS0,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  KDN_TRY(check_dims(dims));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
+  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
+                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
+                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
+                         std::make_pair((const void*)dv, "dv")})
+    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
+  KDN_TRY(check_ptr(beta, "beta", 4, !any));
+  KDN_TRY(check_ptr(dbeta, "dbeta", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(da, "da", 4, true));
+  KDN_TRY(check_ptr(dm, "dm", 4, true));
+  KDN_TRY(check_ptr(S0, "S0", 16, true));
+  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  const size_t need = kdn_backward_workspace_bytes(KDN_DELTA, dims);
+  if (workspace_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
+                                         std::to_string(need));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(dS0, guard));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BH = (size_t)dims->B * dims->H, L = dims->L, DD = (size_t)dims->dk * dims->dv;
+  const size_t nck = (L + kdn::kDeltaBwdChunk - 1) / kdn::kDeltaBwdChunk;
+  char* ws = reinterpret_cast<char*>(workspace);
+  float* S_work = reinterpret_cast<float*>(ws + kStatusBytes);
+  float* ckpt = reinterpret_cast<float*>(ws + kStatusBytes + round256(BH * DD * 4));
+  float* enorm = reinterpret_cast<float*>(ws + kStatusBytes + round256(BH * DD * 4) + round256(BH * nck * DD * 4));
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "clearing the status word");
+  if (!any) {  // nothing to go back through: dS0 = dS_L
+    e = dS_L != nullptr ? cudaMemcpyAsync(dS0, dS_L, BH * DD * 4, cudaMemcpyDeviceToDevice, st)
+                        : cudaMemsetAsync(dS0, 0, BH * DD * 4, st);
+    return cuda_status(e, "dS0 of an empty sequence");
+  }
+  // the sums over value-column blocks accumulate into zeroed outputs
+  e = cudaMemsetAsync(dq, 0, BH * L * dims->dk * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, BH * L * dims->dk * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, BH * L * 4, st);
+  if (e == cudaSuccess && da != nullptr) e = cudaMemsetAsync(da, 0, BH * L * 4, st);
+  if (e == cudaSuccess)
+    e = S0 != nullptr ? cudaMemcpyAsync(S_work, S0, BH * DD * 4, cudaMemcpyDeviceToDevice, st)
+                      : cudaMemsetAsync(S_work, 0, BH * DD * 4, st);
+  if (e != cudaSuccess) return cuda_status(e, "preparing the backward buffers");
+  // forward again, keeping the state at every chunk start and the residual norms
+  kdn::SeqScanArgs fw{q, k, v, dims->in_dtype, KDN_F32, beta, a, nullptr, S_work, nullptr, nullptr, (int)BH, (int)L};
+  fw.S_ckpt = ckpt, fw.enorm = enorm, fw.ckpt_every = kdn::kDeltaBwdChunk;
+  KDN_TRY(cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, fw, st), "backward: forward checkpoints launch"));
+  kdn::DeltaBwdArgs bw{q, k, v, dims->in_dtype, beta, a, dO, dm, dS_L, ckpt, enorm, dq, dk, dv, dbeta, da, dS0,
+                       (int)BH, (int)L};
+  return cuda_status(kdn::launch_delta_bwd(dims->dk, dims->dv, bw, st), "backward launch");
 }
 
 kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* m,

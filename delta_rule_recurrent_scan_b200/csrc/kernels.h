@@ -18,11 +18,64 @@ struct SeqScanArgs {
   const float* a;      // [BH, L] or nullptr
   const float* gains;  // Kalman: [BH, L, dk] fp32, or nullptr for the delta rule
   float* S;            // [BH, dk, dv]
-  void* o;             // [BH, L, dv]
+  void* o;             // [BH, L, dv], or nullptr (not written)
   float* m;            // [BH, L] or nullptr
   int BH;
   int L;
+  // backward pass support (both optional): the state at the start of every ckpt_every-token chunk,
+  // [BH, ceil(L / ckpt_every), dk, dv], and the residual norms ||e_t||, [BH, L]
+  float* S_ckpt = nullptr;
+  float* enorm = nullptr;
+  int ckpt_every = 64;  // a multiple of 16
 };
+
+// Backward pass of the gated delta rule scan (chunks of 32 tokens).
+struct DeltaBwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_dtype;
+  const float* beta;    // [BH, L]
+  const float* a;       // [BH, L] or nullptr (a_t = 1)
+  const float* dO;      // [BH, L, dv] fp32 upstream gradient of o
+  const float* dm;      // [BH, L] or nullptr
+  const float* dS_L;    // [BH, dk, dv] or nullptr
+  const float* S_ckpt;  // [BH, ceil(L / 32), dk, dv]: the state entering every 32-token chunk
+  const float* enorm;   // [BH, L]: ||e_t|| of the forward
+  float* dq;            // [BH, L, dk], zeroed: accumulated over value-column blocks
+  float* dk;            // [BH, L, dk], zeroed
+  float* dv;            // [BH, L, dv]
+  float* dbeta;         // [BH, L], zeroed
+  float* da;            // [BH, L], zeroed, or nullptr
+  float* dS0;           // [BH, dk, dv]
+  int BH;
+  int L;
+};
+constexpr int kDeltaBwdChunk = 32;
+cudaError_t launch_delta_bwd(int dk, int dv, const DeltaBwdArgs& args, cudaStream_t stream);
+
+// Sequence-parallel covariance side of the full-Kalman scan (chunks of 64 tokens): the covariance entering
+// every run of cps chunks, through the chunks' Riccati transfer matrices.
+struct RiccatiArgs {
+  const void* k;        // [BH, L, d] bf16
+  const float* a;       // [BH, L] or nullptr
+  const float* r;       // [BH, L]
+  const float* qn;      // [BH, L] or nullptr (qn_scalar)
+  float qn_scalar;
+  const float* P0;      // [BH, d, d]
+  float* map_w;         // [BH, nch, 64, 2d] scratch
+  float* map_u;         // [BH, nch, 64] scratch
+  float* map_ab;        // [BH, nch, 2] scratch
+  float* xy;            // [BH, runs, 2d, d] scratch: [X; Y] entering every run
+  float* P_starts;      // [BH, runs, d, d] out: the covariance entering every run
+  unsigned* status;
+  int BH;
+  int L;
+  int cps;              // chunks per run; runs = ceil(nch / cps)
+};
+// Bytes of the scratch above (map_w, map_u, map_ab, xy, P_starts, each 256-byte aligned).
+size_t riccati_scratch_bytes(int d, int BH, int L, int cps);
+cudaError_t launch_riccati_starts(int d, const RiccatiArgs& args, cudaStream_t stream);
 
 // Per-token Kalman gain recursions (covariance side; independent of v and S).
 struct GainArgs {

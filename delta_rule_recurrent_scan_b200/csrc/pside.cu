@@ -69,6 +69,11 @@ struct PParams {
   float* gains;  // [BH, L, D] out
   int L;
   unsigned* status;
+  // nullptr: one CTA per head walks every chunk from P.  Otherwise [BH, ceil(nchunks / cps), D, D], the
+  // covariance entering every run of cps chunks: CTA (head, s) walks chunks [s cps, (s + 1) cps) from it, and
+  // the CTA holding the last chunk writes P_L.
+  const float* P_starts;
+  int cps;
 };
 
 template <int D>
@@ -103,6 +108,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int bh = blockIdx.x;
   const int L = P.L;
   const int nchunks = (L + kC - 1) / kC;
+  const int cb = P.P_starts != nullptr ? blockIdx.y * P.cps : 0;     // chunks [cb, ce) of this CTA
+  const int ce = P.P_starts != nullptr ? min(nchunks, cb + P.cps) : nchunks;
 
   float ra = 1.f, rr = 1.f, rq = 0.f;
   auto fetch_scalars = [&](int cc) {
@@ -129,13 +136,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
     sm100::mbar_init(&bar_k, 1);
     sm100::mbar_init(&bar_mma, 1);
     sm100::fence_mbar_init();
-    issue_k(0);
+    issue_k(cb);
   }
   if (warp == 0) {
     sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
     sm100::tmem_relinquish();
   }
-  fetch_scalars(0);
+  fetch_scalars(cb);
   store_scalars(0);
   sm100::tc_fence_before();
   __syncthreads();
@@ -146,6 +153,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   // ---- covariance: thread (lane row, column half) owns P[row][ch*HALF ..); fp32 master in TMEM
   const bool p_owner = row < D;
   float* Pg = P.P + (size_t)bh * D * D;
+  const float* Pin = P.P_starts != nullptr ? P.P_starts + ((size_t)bh * gridDim.y + blockIdx.y) * D * D : Pg;
   auto write_p_panels = [&](const float* x) {
 #pragma unroll
     for (int u = 0; u < HALF / 8; ++u) {
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       float x[32];
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
-        const float4 v4 = *reinterpret_cast<const float4*>(Pg + (size_t)row * D + ch * HALF + cc + e);
+        const float4 v4 = *reinterpret_cast<const float4*>(Pin + (size_t)row * D + ch * HALF + cc + e);
         x[e] = v4.x, x[e + 1] = v4.y, x[e + 2] = v4.z, x[e + 3] = v4.w;
       }
       sm100::tmem_st32(tmem + t_lane + Lay::T_P + ch * HALF + cc, x);
@@ -199,15 +207,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const uint32_t bhi = sm100::smem_u32(Bhi), blo = sm100::smem_u32(Blo);
   const uint32_t ghi = sm100::smem_u32(Ghi), glo = sm100::smem_u32(Glo);
 
-  for (int c = 0; c < nchunks; ++c) {
+  for (int c = cb; c < ce; ++c) {
     const int t0 = c * kC;
-    const int sb = c & 1;
+    const int sb = (c - cb) & 1;
     const float* a_c = sA[sb];
     const float* r_c = sR[sb];
     const float* q_c = sQ[sb];
 
     // ---------------------------------------------------------------- U = K P0
-    if (!wait_all(&bar_k, c & 1)) { aborted = true; break; }
+    if (!wait_all(&bar_k, (c - cb) & 1)) { aborted = true; break; }
     if (tid == 0) {
       constexpr uint32_t id = sm100::idesc_bf16(128, D, false, true);
 #pragma unroll
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       sm100::mma_commit(&bar_mma);
     }
-    if (c + 1 < nchunks) fetch_scalars(c + 1);
+    if (c + 1 < ce) fetch_scalars(c + 1);
     // ---------------------------------------------------------------- gates and the process-noise prefix
     if (warp == 1) {
       float x0 = a_c[lane], x1 = a_c[32 + lane];
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     if (!wait_all(&bar_mma, mma_phase)) { aborted = true; break; }
     mma_phase ^= 1;
-    if (tid == 0 && c + 1 < nchunks) issue_k(c + 1);  // K of this chunk is dead
+    if (tid == 0 && c + 1 < ce) issue_k(c + 1);  // K of this chunk is dead
 
     // ---------------------------------------------------------------- innovation Gram (lower part)
     if (qw < 2) {
@@ -542,14 +550,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
       }
     }
-    if (c + 1 < nchunks) store_scalars(sb ^ 1);
+    if (c + 1 < ce) store_scalars(sb ^ 1);
     sm100::fence_async_smem();
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
   }
 
-  if (!aborted && p_owner) {
+  if (!aborted && p_owner && ce == nchunks) {
 #pragma unroll
     for (int cc = 0; cc < HALF; cc += 32) {
       float x[32];
@@ -570,7 +578,9 @@ cudaError_t launch_pside_typed(const CUtensorMap& tk, const PParams& p, int BH, 
   using Lay = PLayout<D>;
   cudaError_t e = cudaFuncSetAttribute(kalman_pside_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  kalman_pside_kernel<D><<<BH, kPThreads, Lay::SMEM, stream>>>(tk, p);
+  const int nchunks = (p.L + kC - 1) / kC;
+  const int runs = p.P_starts != nullptr ? (nchunks + p.cps - 1) / p.cps : 1;
+  kalman_pside_kernel<D><<<dim3(BH, runs), kPThreads, Lay::SMEM, stream>>>(tk, p);
   return cudaGetLastError();
 }
 
@@ -578,10 +588,11 @@ cudaError_t launch_pside_typed(const CUtensorMap& tk, const PParams& p, int BH, 
 
 cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const float* r, const float* qn,
                                 float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const float* P_starts, int cps) {
   CUtensorMap tk;
   if (!make_bf16_tmap(&tk, k, BH, L, d)) return cudaErrorInvalidValue;
-  PParams p{a, r, qn, qn_scalar, P, gains, L, status};
+  if (P_starts != nullptr && cps < 1) return cudaErrorInvalidValue;
+  PParams p{a, r, qn, qn_scalar, P, gains, L, status, P_starts, cps};
   if (d == 64) return launch_pside_typed<64>(tk, p, BH, stream);
   if (d == 128) return launch_pside_typed<128>(tk, p, BH, stream);
   return cudaErrorInvalidValue;

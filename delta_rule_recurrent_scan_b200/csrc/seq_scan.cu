@@ -52,8 +52,16 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
     S[i][0] = x.x, S[i][1] = x.y, S[i][2] = x.z, S[i][3] = x.w;
   }
 
+  const int nck = args.S_ckpt != nullptr ? (L + args.ckpt_every - 1) / args.ckpt_every : 0;
   for (int t0 = 0; t0 < L; t0 += kTokBlock) {
     const int nt = min(kTokBlock, L - t0);
+    if (nck > 0 && t0 % args.ckpt_every == 0) {  // the state entering this checkpoint chunk
+      float* Sc = args.S_ckpt + ((size_t)bh * nck + t0 / args.ckpt_every) * DK * DV;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i)
+        *reinterpret_cast<float4*>(Sc + (size_t)(rg + i * RG) * DV + cg * 4) =
+            make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+    }
     __syncthreads();
     for (int idx = tid; idx < nt * DK; idx += NT) {
       const int j = idx / DK, i = idx % DK;
@@ -109,7 +117,8 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
 #pragma unroll
           for (int r = 0; r < RG; ++r) yk += red[r][0][tid], yq += red[r][1][tid];
           e = v_s[j][tid] - a * yk;
-          store_elem(args.o, (tok0 + t0 + j) * DV + tid, fmaf(a, yq, gq_s[j] * e), args.out_dtype);
+          if (args.o != nullptr)
+            store_elem(args.o, (tok0 + t0 + j) * DV + tid, fmaf(a, yq, gq_s[j] * e), args.out_dtype);
           e_s[tid] = e;
         }
         const float es = warp_sum(e * e);
@@ -124,11 +133,12 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
 #pragma unroll
         for (int c = 0; c < 4; ++c) S[i][c] = fmaf(a, S[i][c], gr * e_s[cg * 4 + c]);
       }
-      if (tid == 0 && args.m != nullptr) {
+      if (tid == 0 && (args.m != nullptr || args.enorm != nullptr)) {
         float es = 0.f;
 #pragma unroll
         for (int w = 0; w < DVW / 32; ++w) es += ered[w];
-        args.m[tok0 + t0 + j] = sqrtf(gn_s[j]) * sqrtf(es);
+        if (args.m != nullptr) args.m[tok0 + t0 + j] = sqrtf(gn_s[j]) * sqrtf(es);
+        if (args.enorm != nullptr) args.enorm[tok0 + t0 + j] = sqrtf(es);
       }
     }
   }

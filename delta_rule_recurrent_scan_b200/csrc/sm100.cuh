@@ -11,6 +11,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace kdn {
@@ -107,7 +108,8 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 in, fp32 accumulate); one thread issues.
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 or fp16 inputs as the instruction descriptor says,
+// both of the same type; fp32 accumulate); one thread issues.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          bool accumulate) {
   asm volatile(
@@ -239,6 +241,29 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          | ((b_mn_major ? 1u : 0u) << 16)            // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B and an fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7)                                 // A format: f16
+         | (0u << 10)                                // B format: f16
+         | ((a_mn_major ? 1u : 0u) << 15)            // A major
+         | ((b_mn_major ? 1u : 0u) << 16)            // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Two fp32 values -> one fp16 pair word (first value in the low half), rounded to nearest.
+__device__ __forceinline__ uint32_t pack2_f16(float x0, float x1) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// A bf16 pair word -> the same two values as an fp16 pair word (exact in fp16's normal range; values
+// below it round to fp16 subnormals, values beyond it would become infinities).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t b) {
+  return pack2_f16(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u));
 }
 
 // Two fp32 values -> their bf16 hi parts as one pair word and their bf16 lo parts as another (first

@@ -156,6 +156,38 @@ KDN_EXPORT kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, c
                                float* S, float* c, void* o, float* m,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward pass of the gated delta rule scan (the adjoint of kdn_scan_delta for
+ * training; A Hippocampus for Linear Attention, section 4, and Kalman Delta
+ * Networks, Abstract, train these layers end to end; the pages print no
+ * backward).  Given the forward inputs and the upstream gradients of a scalar
+ * loss, returns its gradients with respect to every input of the scan:
+ *   in   q, k [B,H,L,d_k], v [B,H,L,d_v] (dims->in_dtype); beta, a [B,H,L]
+ *        fp32 (a NULL = 1); S0 [B,H,d_k,d_v] fp32, the state the forward started
+ *        from (NULL = 0; not modified);
+ *        dO [B,H,L,d_v] fp32 = dLoss/do; dm [B,H,L] fp32 = dLoss/dm or NULL;
+ *        dS_L [B,H,d_k,d_v] fp32 = dLoss/dS_L or NULL
+ *   out  dq, dk [B,H,L,d_k], dv [B,H,L,d_v], dbeta [B,H,L], da [B,H,L] (or
+ *        NULL; with a NULL it is the gradient at a = 1), dS0 [B,H,d_k,d_v]:
+ *        all fp32, overwritten.
+ * The surprise m_t = beta_t ||k_t|| ||e_t|| has no gradient where e_t = 0 or
+ * k_t = 0 (the one-sided value 0 is taken).  A gate a_t = 0 is allowed.
+ * Method: the forward is run again, keeping the state at every 32-token
+ * chunk start and ||e_t||, in the workspace; then the chunks are walked
+ * backwards with the state adjoint, every step a product of 32 x 32, 32 x d
+ * or d x d blocks on the fp32 CUDA cores (one CTA per head and block of 32
+ * value columns).  workspace: kdn_backward_workspace_bytes(KDN_DELTA, dims)
+ * bytes (256-byte status word, the states, the norms).  dims->chunk and
+ * dims->out_dtype are ignored.  Asynchronous on ``stream``. */
+KDN_EXPORT kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                              const float* beta, const float* a, const float* S0, const float* dO,
+                                              const float* dm, const float* dS_L, float* dq, float* dk, float* dv,
+                                              float* dbeta, float* da, float* dS0, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace kdn_scan_delta_backward needs (variant KDN_DELTA;
+ * 0 for other variants or invalid dims). */
+KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims);
+
 /* Surprise-cache read (A Hippocampus for Linear Attention, sections 3.3-3.4,
  * Eq. (6)-(7)).  Each head keeps the exact (k, v) of the w tokens with the
  * largest surprise m seen so far (ties: the earlier token); token t of block b

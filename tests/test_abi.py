@@ -107,3 +107,16 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 4, 16)
     with pytest.raises(ValueError, match="CUDA"):
         kdn.scan_delta(q, q, q, torch.zeros(1, 1, 4))
+
+
+def test_backward_host_validation(L):
+    d = kdn.Dims(2, 3, 100, 64, 32, 0, kdn.KDN_BF16, kdn.KDN_F32)
+    n = L.kdn_backward_workspace_bytes(0, ctypes.byref(d))
+    # status word + working state + a state per 32-token chunk + one norm per token
+    assert n >= 256 + 6 * 64 * 32 * 4 * (1 + 4) + 6 * 100 * 4
+    for variant in (1, 2, 3):
+        assert L.kdn_backward_workspace_bytes(variant, ctypes.byref(d)) == 0
+    assert L.kdn_scan_delta_backward(None, *([None] * 15), None, 0, None) == kdn.KDN_ERR_INVALID_ARG
+    # every output pointer is checked before anything is enqueued
+    assert L.kdn_scan_delta_backward(ctypes.byref(d), *([None] * 15), None, 0, None) == kdn.KDN_ERR_INVALID_ARG
+    assert b"dS0" in L.kdn_last_error()

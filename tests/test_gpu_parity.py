@@ -17,11 +17,10 @@ import torch
 import oracle
 from delta_rule_recurrent_scan_b200 import kdn
 from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_decode_inputs, make_scan_inputs
-from parity import TOL, assert_symmetric_pd, compare, initial_state, normwise_err, run_gpu, run_oracle
+from parity import SELF_TOL, TOL, assert_symmetric_pd, compare, initial_state, normwise_err, run_gpu, run_oracle, self_tol
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-SELF_TOL = 1e-4  # two CUDA paths (or two chunkings) of the same scan against each other
 
 
 def _to(x, device):
@@ -220,8 +219,8 @@ def test_decode_steps_equal_scan_and_oracle(variant):
     xs = {k: (v.movedim(0, 2).contiguous() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     scan = run_gpu(variant, xs)
     o = torch.stack(outs, dim=2)
-    assert normwise_err(o.float(), scan["o"].float()) < SELF_TOL
-    assert normwise_err(S, scan["S"]) < SELF_TOL
+    assert normwise_err(o.float(), scan["o"].float()) < self_tol(w.dk)  # the scan takes the d = 128 chunk kernel
+    assert normwise_err(S, scan["S"]) < self_tol(w.dk)
     ref = run_oracle(variant, xs)
     compare({"o": o, "m": torch.stack(ms, dim=2), "S": S}, ref, TOL["bf16"])
     if variant == "kalman_diag":
