@@ -387,12 +387,12 @@ kdn_status kdn::api::kalman_scan(kdn_variant var, const kdn_dims* dims, const vo
         const size_t chunks = (size_t)BH * nch, runs = (size_t)BH * ((nch + cps - 1) / cps), dk = dims->dk;
         kdn::RiccatiArgs ra{};
         ra.k = k, ra.a = a, ra.r = r, ra.qn = qn, ra.qn_scalar = qn_scalar, ra.P0 = P, ra.cps = cps;
-        ra.map_w = reinterpret_cast<float*>(rs);
-        rs += round256(chunks * 64 * 2 * dk * 4);
+        ra.map_g = reinterpret_cast<float*>(rs);
+        rs += round256(chunks * 64 * 64 * 4);
         ra.map_u = reinterpret_cast<float*>(rs);
         rs += round256(chunks * 64 * 4);
         ra.map_ab = reinterpret_cast<float*>(rs);
-        rs += round256(chunks * 2 * 4);
+        rs += round256(chunks * 2 * 64 * 4);
         ra.xy = reinterpret_cast<float*>(rs);
         rs += round256(runs * 2 * dk * dk * 4);
         ra.P_starts = reinterpret_cast<float*>(rs);

@@ -63,9 +63,9 @@ struct RiccatiArgs {
   const float* qn;      // [BH, L] or nullptr (qn_scalar)
   float qn_scalar;
   const float* P0;      // [BH, d, d]
-  float* map_w;         // [BH, nch, 64, 2d] scratch
+  float* map_g;         // [BH, nch, 64, 64] scratch: G^T of every chunk
   float* map_u;         // [BH, nch, 64] scratch
-  float* map_ab;        // [BH, nch, 2] scratch
+  float* map_ab;        // [BH, nch, 64, 2] scratch: alpha_t, beta_t
   float* xy;            // [BH, runs, 2d, d] scratch: [X; Y] entering every run
   float* P_starts;      // [BH, runs, d, d] out: the covariance entering every run
   unsigned* status;
@@ -73,7 +73,7 @@ struct RiccatiArgs {
   int L;
   int cps;              // chunks per run; runs = ceil(nch / cps)
 };
-// Bytes of the scratch above (map_w, map_u, map_ab, xy, P_starts, each 256-byte aligned).
+// Bytes of the scratch above (map_g, map_u, map_ab, xy, P_starts, each 256-byte aligned).
 size_t riccati_scratch_bytes(int d, int BH, int L, int cps);
 cudaError_t launch_riccati_starts(int d, const RiccatiArgs& args, cudaStream_t stream);
 

@@ -1,5 +1,5 @@
-// Sequence-parallel covariance side of the full-Kalman scan: the covariance at every chunk start from
-// composed chunk transfer matrices, so that the chunks' gains can then be computed all at once.
+// Sequence-parallel covariance side of the full-Kalman scan: the covariance at the start of every run of
+// chunks from chained chunk transfer matrices, so that the runs' gains can then be computed all at once.
 //
 // Kalman Delta Networks, Abstract: exact covariance tracking is a dense, state-dependent Riccati
 // recursion that does not map onto GPU-parallel scans, while Moebius maps compose.  The dense recursion
@@ -9,19 +9,23 @@
 // the product of its tokens' matrices.  That product has a closed form: with alpha_t = prod a^2,
 // beta_t = a_t^2 beta_{t-1} + Qn_t, beta_{t,j} the noise accumulated over tokens j+1..t,
 //   M_chunk = [[alpha I, beta I], [0, I]] + U W^T,  U[:, j] = [beta_{C,j} k_j; k_j],
-//   W = B (diag(r) - Cs^T)^-1,  B[:, t] = [alpha_t k_t; beta_t k_t],  Cs_tj = (k_j . k_t) beta_{t,j} (j < t),
-// one C x C triangular solve per chunk.  Three kernels:
-//   riccati_chunk_map_kernel  every chunk's W, U coefficients, alpha and beta, all chunks at once;
-//   riccati_chain_kernel      [X; Y] from [P0; I] through the chunk maps, one CTA per head and block of 16
+//   W = B G,  G = (diag(r) - Cs^T)^-1,  B[:, t] = [alpha_t k_t; beta_t k_t],  Cs_tj = (k_j . k_t) beta_{t,j} (j < t).
+// Applied to [X; Y] without forming W: Z = G^T (diag(alpha_t) K X + diag(beta_t) K Y), then
+// X' = alpha_C X + beta_C Y + K^T diag(beta_{C,j}) Z and Y' = Y + K^T Z.  Three kernels:
+//   riccati_chunk_map_kernel  every chunk's G, U coefficients and per-token alpha, beta, all chunks at
+//                             once; G^T = (diag(r) - Cs)^-1 = diag(1/r) (I - Cs diag(1/r))^-1, a unit lower
+//                             triangular inverse;
+//   riccati_chain_kernel      [X; Y] from [P0; I] through the chunk maps, one CTA per head and block of 8
 //                             columns (the columns of [X; Y] transform independently, and each may be
 //                             rescaled freely: P = X Y^-1 does not change), storing [X; Y] at the start of
 //                             every run of cps chunks;
-//   riccati_extract_kernel    P = X Y^-1 at every run start (LU with partial pivoting of Y^T, then
-//                             P^T = Y^-T X^T by substitution, symmetrised), all runs at once.
+//   riccati_extract_kernel    P = X Y^-1 at every run start: Gauss-Jordan with partial pivoting on
+//                             [Y^T | X^T] held in registers, then symmetrised, all runs at once.
 // The chunked covariance kernel then walks every run from its own start covariance, all runs in parallel.
 #include <cuda_runtime.h>
 
 #include "chunk.h"
+#include "chunk_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,93 +34,123 @@ namespace kdn {
 namespace {
 
 constexpr int kRC = 64;  // tokens per chunk, as the covariance kernel's chunks
+constexpr int kMapThreads = 256;
+
+// Eight bf16 values (one 16-byte load) to floats.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 raw, float* out) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    out[2 * e] = f.x, out[2 * e + 1] = f.y;
+  }
+}
 
 // ---------------------------------------------------------------------------------------- chunk maps
-// W [BH][nch][kRC][2D] (row t: column t of W, i.e. the coefficients of the chunk's t-th rank-1 term),
-// ucoef [BH][nch][kRC] (beta_{C,j}), ab [BH][nch][2] (alpha, beta of the whole chunk).
+// map_g [BH][nch][C][C]: G^T (row t = column t of G), map_u [BH][nch][C]: beta_{C,j},
+// map_ab [BH][nch][C][2]: alpha_t, beta_t.  Only chunks before the last run start are mapped (all full).
 template <int D>
-__global__ void __launch_bounds__(2 * D) riccati_chunk_map_kernel(RiccatiArgs p) {
-  constexpr int NT = 2 * D, C = kRC, LK = D + 1, LC = C + 1;
-  extern __shared__ float msm[];
-  float (*kf)[LK] = reinterpret_cast<float (*)[LK]>(msm);  // [C][LK] the chunk's keys
-  __shared__ float Cs[C][LC];     // (k_j . k_t) beta_{t,j} for j < t
-  __shared__ float sa[C], sr[C], sq[C], salpha[C], sbeta[C];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.x, c = blockIdx.y, L = p.L, nch = (L + C - 1) / C;
-  const int t0 = c * C, n = min(C, L - t0);
-  const size_t tok0 = (size_t)bh * L;
-  const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.k);
+__global__ void __launch_bounds__(kMapThreads) riccati_chunk_map_kernel(RiccatiArgs p) {
+  constexpr int NT = kMapThreads, C = kRC, LK = D + 4, LC = chunk::kLD;
+  static_assert(C == chunk::kC && LK >= LC, "the key buffer is reused for the inverse");
+  extern __shared__ __align__(16) float msm[];
+  float* kf = msm;          // [C][LK] keys, later T = (I - Cs diag(1/r))^-1 with row stride LC
+  float* Cs = kf + C * LK;  // [C][LC]: (k_j . k_t) beta_{t,j} for j < t, then -Cs_tj / r_j
+  __shared__ float sa[C], sr[C], sq[C];
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x, c = blockIdx.y, nch = (p.L + C - 1) / C;
+  const size_t tok0 = (size_t)bh * p.L + (size_t)c * C;
+  const __nv_bfloat16* kg = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok0 * D;
+  const size_t map = (size_t)bh * nch + c;
 
-  for (int idx = tid; idx < C * D; idx += NT) {
-    const int t = idx / D, i = idx % D;
-    kf[t][i] = t < n ? __bfloat162float(kb[(tok0 + t0 + t) * D + i]) : 0.f;
+  for (int idx = tid; idx < C * D / 8; idx += NT) {
+    const int t = idx / (D / 8), i8 = idx % (D / 8);
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(kg + (size_t)t * D + 8 * i8), f);
+    *reinterpret_cast<float4*>(kf + t * LK + 8 * i8) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(kf + t * LK + 8 * i8 + 4) = make_float4(f[4], f[5], f[6], f[7]);
   }
   if (tid < C) {
-    const bool ok = tid < n;
-    const size_t ti = tok0 + t0 + tid;
-    sa[tid] = ok ? (p.a != nullptr ? p.a[ti] : 1.f) : 1.f;
-    sr[tid] = ok ? p.r[ti] : 1.f;
-    sq[tid] = ok ? (p.qn != nullptr ? p.qn[ti] : p.qn_scalar) : 0.f;
+    const size_t ti = tok0 + tid;
+    sa[tid] = p.a != nullptr ? p.a[ti] : 1.f;
+    sr[tid] = p.r[ti];
+    sq[tid] = p.qn != nullptr ? p.qn[ti] : p.qn_scalar;
   }
   __syncthreads();
-  if (warp == 0 && lane == 0) {  // alpha_t, beta_t (64 steps)
+  {  // K K^T: thread (tb, jb) takes rows tb + 16u and jb + 16w (eight consecutive rows per quarter warp)
+    const int tb = tid / 16, jb = tid % 16;
+    float acc[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < D; i += 4) {
+      float4 kt[4], kj[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kt[u] = *reinterpret_cast<const float4*>(kf + (tb + 16 * u) * LK + i);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) kj[w] = *reinterpret_cast<const float4*>(kf + (jb + 16 * w) * LK + i);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          float x = acc[u][w];
+          x = fmaf(kt[u].x, kj[w].x, x);
+          x = fmaf(kt[u].y, kj[w].y, x);
+          x = fmaf(kt[u].z, kj[w].z, x);
+          acc[u][w] = fmaf(kt[u].w, kj[w].w, x);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int t = tb + 16 * u, j = jb + 16 * w;
+        Cs[t * LC + j] = j < t ? acc[u][w] : 0.f;
+      }
+  }
+  __syncthreads();
+  if (tid < C) {  // beta_{t,j} down column j (t > j) and 1 / r_j folded into Cs; beta_{C,j} is the U coefficient
+    const int j = tid;
+    const float nir = -1.f / sr[j];
+    float acc = 0.f;
+    for (int t = j + 1; t < C; ++t) {
+      acc = fmaf(sa[t] * sa[t], acc, sq[t]);
+      Cs[t * LC + j] *= acc * nir;
+    }
+    p.map_u[map * C + j] = acc;
+  } else if (tid == C) {  // alpha_t, beta_t
     float al = 1.f, be = 0.f;
+    float* ab = p.map_ab + map * 2 * C;
     for (int t = 0; t < C; ++t) {
       const float a2 = sa[t] * sa[t];
       al *= a2;
       be = fmaf(a2, be, sq[t]);
-      salpha[t] = al, sbeta[t] = be;
+      ab[2 * t] = al, ab[2 * t + 1] = be;
     }
   }
-  // K K^T into Cs (full), then the noise factors
+  __syncthreads();
+  // T = (I + N)^-1 with N = -Cs diag(1/r) strictly lower; G^T = diag(1/r) T
+  chunk::invert_unit_lower_64(Cs, kf, tid, [] { __syncthreads(); });
+  float* Gt = p.map_g + map * C * C;
   for (int idx = tid; idx < C * C; idx += NT) {
-    const int t = idx / C, j = idx % C;
-    float acc = 0.f;
-    if (j < t) {
-#pragma unroll 8
-      for (int i = 0; i < D; ++i) acc = fmaf(kf[t][i], kf[j][i], acc);
-    }
-    Cs[t][j] = acc;
-  }
-  __syncthreads();
-  float* ucoef = p.map_u + ((size_t)bh * nch + c) * C;
-  if (tid < C) {  // beta_{t,j} down column j (t > j), folded into Cs; beta_{C,j} is the U coefficient
-    const int j = tid;
-    float acc = 0.f;
-    for (int t = j + 1; t < C; ++t) {
-      acc = fmaf(sa[t] * sa[t], acc, sq[t]);
-      Cs[t][j] *= acc;
-    }
-    ucoef[j] = acc;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float* ab = p.map_ab + ((size_t)bh * nch + c) * 2;
-    ab[0] = salpha[C - 1], ab[1] = sbeta[C - 1];
-  }
-  // row rho of W: w_t = (b_t + sum_{j<t} Cs_tj w_j) / r_t, b_t = (alpha_t or beta_t) k_t[rho mod D]
-  {
-    const int rho = tid, i = rho % D;
-    const float* sc = rho < D ? salpha : sbeta;
-    float w[C];
-#pragma unroll
-    for (int t = 0; t < C; ++t) {
-      float acc = sc[t] * kf[t][i];
-#pragma unroll
-      for (int j = 0; j < t; ++j) acc = fmaf(Cs[t][j], w[j], acc);
-      w[t] = acc / sr[t];
-    }
-    float* Wc = p.map_w + ((size_t)bh * nch + c) * C * NT;
-#pragma unroll
-    for (int t = 0; t < C; ++t) Wc[(size_t)t * NT + rho] = w[t];
+    const int t = idx / C, sx = idx % C;
+    Gt[idx] = sx <= t ? kf[t * LC + sx] / sr[t] : 0.f;
   }
 }
 
 // ---------------------------------------------------------------------------------------- the chain
-// [X; Y] (2D x 16 columns of this CTA) from [P0; I] through the chunk maps; xy [BH][runs][2D][D] gets the pair
-// entering every run (every cps-th chunk).  Each chunk's W^T (64 KB at d = 128), keys and U coefficients are
-// copied asynchronously, the next chunk's while the current one is applied.
-constexpr int kRCols = 16, kChainThreads = 512;
+// [X; Y] (2D x 8 columns of this CTA, held transposed) from [P0; I] through the chunk maps; xy [BH][runs][2D][D]
+// gets the pair entering every run (every cps-th chunk).  The next chunk's keys, G^T and coefficients are
+// copied asynchronously while the current chunk is applied.  A chunk, with 256 threads in register blocks:
+//   R = diag(alpha_t) K X + diag(beta_t) K Y   thread: 2 tokens x 2 columns over half of i (pairs summed by shuffle)
+//   Z = G^T R                                   thread: 1 token x 2 columns
+//   X' = alpha_C X + beta_C Y + K^T diag(u) Z,  thread: d/64 rows x 2 columns
+//   Y' = Y + K^T Z
+// Each column of [X; Y] is rescaled by a power of two (exact; X Y^-1 does not change) from the maximum of
+// |Y| over the column one chunk earlier, which needs no extra pass or barrier.
+constexpr int kRCols = 8, kChainThreads = 256;
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
@@ -127,128 +161,280 @@ __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wai
 
 template <int D>
 struct ChainLayout {
-  static constexpr int C = kRC, R2 = 2 * D, NC = kRCols;
-  static constexpr int WS = R2 + 4;  // padded row stride of W^T: rows t, t+1 start 4 banks apart
-  static constexpr int W_FLOATS = C * WS, K_HALVES = C * D;
-  // floats: 2 W^T buffers, 2 U buffers, [X; Y], Z, column scales; then 2 bf16 key buffers
-  static constexpr int OFF_U = 2 * W_FLOATS, OFF_XY = OFF_U + 2 * C, OFF_Z = OFF_XY + R2 * NC, OFF_S = OFF_Z + C * NC;
-  static constexpr int OFF_K = OFF_S + NC;  // in floats, 16-byte aligned below
+  static constexpr int C = kRC, NC = kRCols;
+  static constexpr int LG = C + 4;   // row strides in floats (bf16 for keys), chosen so that the rows a warp
+  static constexpr int LX = D + 4;   // reads together start 4 banks apart
+  static constexpr int LRS = NC + 4;  // R row stride: eight consecutive rows start on distinct bank quads
+  static constexpr int LKB = D + 8;
+  static constexpr int OFF_G = 0;                    // 2 x [C][LG]  G^T
+  static constexpr int OFF_AB = OFF_G + 2 * C * LG;  // 2 x [C][2]   alpha_t, beta_t
+  static constexpr int OFF_U = OFF_AB + 2 * 2 * C;   // 2 x [C]      beta_{C,j}
+  static constexpr int OFF_X = OFF_U + 2 * C;        // [NC][LX]     X^T
+  static constexpr int OFF_Y = OFF_X + NC * LX;      // [NC][LX]     Y^T
+  static constexpr int OFF_R = OFF_Y + NC * LX;      // [C][LRS]     R
+  static constexpr int OFF_Z = OFF_R + C * LRS;      // [C][NC]      Z
+  static constexpr int OFF_ZU = OFF_Z + C * NC;      // [C][NC]      diag(u) Z
+  static constexpr int OFF_S = OFF_ZU + C * NC;      // 2 x [NC]     column maxima of |Y| (by chunk parity)
+  static constexpr int OFF_K = OFF_S + 2 * NC;       // 2 x [C][LKB] bf16 keys
+  static constexpr int K_HALVES = C * LKB;
   static constexpr size_t BYTES = (size_t)OFF_K * 4 + 2 * (size_t)K_HALVES * 2;
-  static_assert(OFF_K % 4 == 0, "key buffers must start 16-byte aligned");
+  static_assert(OFF_AB % 4 == 0 && OFF_U % 4 == 0 && OFF_X % 4 == 0 && OFF_Y % 4 == 0 && OFF_R % 4 == 0 &&
+                    OFF_K % 4 == 0,
+                "16-byte aligned regions");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kChainThreads, 1) riccati_chain_kernel(RiccatiArgs p) {
+__global__ void __launch_bounds__(kChainThreads, 2) riccati_chain_kernel(RiccatiArgs p) {
   using Ly = ChainLayout<D>;
-  constexpr int NT = kChainThreads, C = kRC, R2 = 2 * D, NC = kRCols, WS = Ly::WS;
-  constexpr int PER_Z = C * NC / NT, PER_X = D * NC / NT;
+  constexpr int NT = kChainThreads, C = kRC, NC = kRCols, LG = Ly::LG, LX = Ly::LX, LRS = Ly::LRS, LKB = Ly::LKB;
   extern __shared__ __align__(16) float rsm[];
-  float* XY = rsm + Ly::OFF_XY;  // [R2][NC]
-  float* Z = rsm + Ly::OFF_Z;    // [C][NC]
-  float* scl = rsm + Ly::OFF_S;  // [NC] column maxima, then scales
+  float* Xt = rsm + Ly::OFF_X;
+  float* Yt = rsm + Ly::OFF_Y;
+  float* Rs = rsm + Ly::OFF_R;
+  float* Zs = rsm + Ly::OFF_Z;
+  float* Zu = rsm + Ly::OFF_ZU;
+  float* scl = rsm + Ly::OFF_S;
   __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(rsm + Ly::OFF_K);
   const int tid = threadIdx.x;
-  const int bh = blockIdx.x, col0 = blockIdx.y * NC, L = p.L, nch = (L + C - 1) / C;
+  const int bh = blockIdx.x, col0 = blockIdx.y * NC, nch = (p.L + C - 1) / C;
   const int cps = p.cps, runs = (nch + cps - 1) / cps;
-  const __nv_bfloat16* kg = reinterpret_cast<const __nv_bfloat16*>(p.k) + (size_t)bh * L * D;
-  // chunk c's W^T, U coefficients and keys into buffer c & 1 (chunks before the last run start are full)
+  const __nv_bfloat16* kg = reinterpret_cast<const __nv_bfloat16*>(p.k) + (size_t)bh * p.L * D;
+  // chunk c's G^T, alpha/beta, U coefficients and keys into buffer c & 1 (chunks before the last run are full)
   auto fetch = [&](int c) {
     const int b = c & 1;
-    float* Wd = rsm + b * Ly::W_FLOATS;
-    const float* Wc = p.map_w + ((size_t)bh * nch + c) * C * R2;
-    for (int idx = tid; idx < C * R2 / 4; idx += NT) {
-      const int t = idx / (R2 / 4), q = idx % (R2 / 4);
-      cp_async16(Wd + t * WS + 4 * q, Wc + (size_t)t * R2 + 4 * q);
+    const size_t map = (size_t)bh * nch + c;
+    const float* gsrc = p.map_g + map * C * C;
+    for (int idx = tid; idx < C * C / 4; idx += NT) {
+      const int t = idx / (C / 4), q = idx % (C / 4);
+      cp_async16(rsm + Ly::OFF_G + b * C * LG + t * LG + 4 * q, gsrc + t * C + 4 * q);
     }
-    if (tid < C / 4) cp_async16(rsm + Ly::OFF_U + b * C + 4 * tid, p.map_u + ((size_t)bh * nch + c) * C + 4 * tid);
+    if (tid < 2 * C / 4) cp_async16(rsm + Ly::OFF_AB + b * 2 * C + 4 * tid, p.map_ab + map * 2 * C + 4 * tid);
+    else if (tid < 2 * C / 4 + C / 4) {
+      const int q = tid - 2 * C / 4;
+      cp_async16(rsm + Ly::OFF_U + b * C + 4 * q, p.map_u + map * C + 4 * q);
+    }
     const __nv_bfloat16* kc = kg + (size_t)c * C * D;
-    for (int idx = tid; idx < C * D / 8; idx += NT) cp_async16(kbuf + b * Ly::K_HALVES + 8 * idx, kc + 8 * idx);
+    for (int idx = tid; idx < C * D / 8; idx += NT) {
+      const int t = idx / (D / 8), q = idx % (D / 8);
+      cp_async16(kbuf + b * Ly::K_HALVES + t * LKB + 8 * q, kc + (size_t)t * D + 8 * q);
+    }
     cp_async_commit();
   };
 
-  for (int idx = tid; idx < R2 * NC; idx += NT) {
-    const int rho = idx / NC, cc = idx % NC, col = col0 + cc;
-    XY[idx] = rho < D ? p.P0[((size_t)bh * D + rho) * D + col] : (rho - D == col ? 1.f : 0.f);
+  for (int idx = tid; idx < NC * D; idx += NT) {
+    const int cc = idx / D, i = idx % D;
+    Xt[cc * LX + i] = p.P0[((size_t)bh * D + i) * D + col0 + cc];
+    Yt[cc * LX + i] = i == col0 + cc ? 1.f : 0.f;
   }
-  const int last = (runs - 1) * cps;  // the maps of the chunks past the last run start are not needed
+  if (tid < NC) scl[NC + tid] = 1.f;  // the scale chunk 0 applies: 1
+  const int last = (runs - 1) * cps;  // the chunks past the last run start are not needed
   if (last > 0) fetch(0);
   for (int c = 0; c <= last; ++c) {
     __syncthreads();
     if (c % cps == 0) {
-      float* xyc = p.xy + ((size_t)bh * runs + c / cps) * R2 * D;
-      for (int idx = tid; idx < R2 * NC; idx += NT) xyc[(size_t)(idx / NC) * D + col0 + idx % NC] = XY[idx];
+      float* xyc = p.xy + ((size_t)bh * runs + c / cps) * 2 * D * D;
+      for (int idx = tid; idx < 2 * D * NC; idx += NT) {
+        const int rho = idx / NC, cc = idx % NC;
+        xyc[(size_t)rho * D + col0 + cc] = rho < D ? Xt[cc * LX + rho] : Yt[cc * LX + rho - D];
+      }
     }
     if (c == last) break;
     if (c + 1 < last) fetch(c + 1);
     else cp_async_commit();  // an empty group keeps the wait count uniform
-    const float* ab = p.map_ab + ((size_t)bh * nch + c) * 2;
-    const float alpha = __ldg(ab), beta = __ldg(ab + 1);
-    const float* Ws = rsm + (c & 1) * Ly::W_FLOATS;
+    const float* Gt = rsm + Ly::OFF_G + (c & 1) * C * LG;
+    const float* ab = rsm + Ly::OFF_AB + (c & 1) * 2 * C;
     const float* uc = rsm + Ly::OFF_U + (c & 1) * C;
     const __nv_bfloat16* kf = kbuf + (c & 1) * Ly::K_HALVES;
     cp_async_wait_one();  // this chunk's copies have landed (the next chunk's may still be in flight)
     __syncthreads();
-    // Z = W^T [X; Y]
+    // ---- R = diag(alpha) K X + diag(beta) K Y: thread (token quad tq, column pair cp, i part ip of 4); the
+    // parts hold interleaved i pairs and are summed by shuffles (ip = lane bits 0..1)
+    {
+      const int ip = tid & 3, cp = (tid >> 2) & 3, tq = tid >> 4;
+      const int t0 = 4 * tq, c0 = 2 * cp;
+      float kx[4][2], ky[4][2];
 #pragma unroll
-    for (int u = 0; u < PER_Z; ++u) {
-      const int idx = tid + NT * u, t = idx / NC, cc = idx % NC;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int rho = 0; rho < R2; rho += 4) {
-        const float4 w = *reinterpret_cast<const float4*>(Ws + t * WS + rho);
-        acc = fmaf(w.x, XY[rho * NC + cc], acc);
-        acc = fmaf(w.y, XY[(rho + 1) * NC + cc], acc);
-        acc = fmaf(w.z, XY[(rho + 2) * NC + cc], acc);
-        acc = fmaf(w.w, XY[(rho + 3) * NC + cc], acc);
+      for (int u = 0; u < 4; ++u) kx[u][0] = kx[u][1] = ky[u][0] = ky[u][1] = 0.f;
+#pragma unroll 4
+      for (int i = 2 * ip; i < D; i += 8) {
+        float2 kv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          kv[u] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kf + (t0 + u) * LKB + i));
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const float2 x = *reinterpret_cast<const float2*>(Xt + (c0 + w) * LX + i);
+          const float2 y = *reinterpret_cast<const float2*>(Yt + (c0 + w) * LX + i);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            kx[u][w] = fmaf(kv[u].x, x.x, fmaf(kv[u].y, x.y, kx[u][w]));
+            ky[u][w] = fmaf(kv[u].x, y.x, fmaf(kv[u].y, y.y, ky[u][w]));
+          }
+        }
       }
-      Z[idx] = acc;
-    }
-    __syncthreads();
-    // [X; Y] <- [alpha X + beta Y; Y] + U Z, U[:, t] = [u_t k_t; k_t]
-    float nx[PER_X], ny[PER_X];
 #pragma unroll
-    for (int u = 0; u < PER_X; ++u) {
-      const int idx = tid + NT * u, i = idx / NC, cc = idx % NC;
-      float sx = 0.f, sy = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < C; ++t) {
-        const float kz = __bfloat162float(kf[t * D + i]) * Z[t * NC + cc];
-        sx = fmaf(uc[t], kz, sx);
-        sy += kz;
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          kx[u][w] += __shfl_xor_sync(0xffffffffu, kx[u][w], 1);
+          kx[u][w] += __shfl_xor_sync(0xffffffffu, kx[u][w], 2);
+          ky[u][w] += __shfl_xor_sync(0xffffffffu, ky[u][w], 1);
+          ky[u][w] += __shfl_xor_sync(0xffffffffu, ky[u][w], 2);
+        }
+      // lane ip writes token t0 + ip
+      float rx0 = kx[0][0], rx1 = kx[0][1], ry0 = ky[0][0], ry1 = ky[0][1];
+#pragma unroll
+      for (int u = 1; u < 4; ++u)
+        if (ip == u) rx0 = kx[u][0], rx1 = kx[u][1], ry0 = ky[u][0], ry1 = ky[u][1];
+      const int t = t0 + ip;
+      const float al = ab[2 * t], be = ab[2 * t + 1];
+      *reinterpret_cast<float2*>(Rs + t * LRS + c0) = make_float2(fmaf(al, rx0, be * ry0), fmaf(al, rx1, be * ry1));
+    }
+    if (tid < NC) scl[(c & 1) * NC + tid] = 0.f;  // nobody reads this parity's maxima any more
+    __syncthreads();
+    // ---- Z = G^T R and diag(u) Z: thread (token quad tq, column quad cq, s part sp of 8; sp = lane bits 0..2)
+    {
+      const int sp = tid & 7, cq = (tid >> 3) & 1, tq = tid >> 4, t0 = 4 * tq, c0 = 4 * cq;
+      float z[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) z[u][0] = z[u][1] = z[u][2] = z[u][3] = 0.f;
+#pragma unroll
+      for (int sx = sp; sx < C; sx += 8) {
+        const float4 r4 = *reinterpret_cast<const float4*>(Rs + sx * LRS + c0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float g = Gt[(t0 + u) * LG + sx];
+          z[u][0] = fmaf(g, r4.x, z[u][0]);
+          z[u][1] = fmaf(g, r4.y, z[u][1]);
+          z[u][2] = fmaf(g, r4.z, z[u][2]);
+          z[u][3] = fmaf(g, r4.w, z[u][3]);
+        }
       }
-      const float x = XY[i * NC + cc], y = XY[(D + i) * NC + cc];
-      nx[u] = fmaf(alpha, x, fmaf(beta, y, sx));
-      ny[u] = y + sy;
-    }
-    if (tid < NC) scl[tid] = 0.f;
-    __syncthreads();
 #pragma unroll
-    for (int u = 0; u < PER_X; ++u) {
-      const int idx = tid + NT * u, i = idx / NC, cc = idx % NC;
-      XY[i * NC + cc] = nx[u], XY[(D + i) * NC + cc] = ny[u];
-      atomicMax(reinterpret_cast<int*>(&scl[cc]), __float_as_int(fabsf(ny[u])));  // non-negative floats order as ints
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          z[u][w] += __shfl_xor_sync(0xffffffffu, z[u][w], 1);
+          z[u][w] += __shfl_xor_sync(0xffffffffu, z[u][w], 2);
+          z[u][w] += __shfl_xor_sync(0xffffffffu, z[u][w], 4);
+        }
+      if (sp < 4) {  // lane sp writes token t0 + sp
+        float4 zz = make_float4(z[0][0], z[0][1], z[0][2], z[0][3]);
+#pragma unroll
+        for (int u = 1; u < 4; ++u)
+          if (sp == u) zz = make_float4(z[u][0], z[u][1], z[u][2], z[u][3]);
+        const int t = t0 + sp;
+        const float uu = uc[t];
+        *reinterpret_cast<float4*>(Zs + t * NC + c0) = zz;
+        *reinterpret_cast<float4*>(Zu + t * NC + c0) = make_float4(uu * zz.x, uu * zz.y, uu * zz.z, uu * zz.w);
+      }
     }
     __syncthreads();
-    // rescale each column of [X; Y] by a power of two near 1 / max |Y column| (exact; P = X Y^-1 unchanged)
-    for (int idx = tid; idx < R2 * NC; idx += NT) {
-      const int e = (__float_as_int(scl[idx % NC]) >> 23) & 0xff;
-      XY[idx] *= __int_as_float((254 - min(max(e, 1), 253)) << 23);
+    // ---- X, Y updates and rescale: thread (row quad iq, column quad cq, token part tp of 4; tp = lane bits
+    // 0..1, interleaved tokens), the parts summed by shuffles; lane tp then finishes row i0 + tp
+    {
+      const int tp = tid & 3, cq = (tid >> 2) & 1, iq = tid >> 3, i0 = 4 * iq, c0 = 4 * cq;
+      constexpr int RPT = D / 32;  // row quads per thread: D = 128 -> 1 quad of 4 rows, D = 64 -> rows of 2
+      static_assert(D == 128 || D == 64, "head size");
+      constexpr int NR = D == 128 ? 4 : 2;  // rows per thread
+      const int r0 = D == 128 ? i0 : 2 * iq;
+      float sx[NR][4], sy[NR][4];
+#pragma unroll
+      for (int e = 0; e < NR; ++e)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) sx[e][w] = sy[e][w] = 0.f;
+#pragma unroll 4
+      for (int t = tp; t < C; t += 4) {
+        float kv[NR];
+        if constexpr (NR == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(kf + t * LKB + r0);
+          const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+          const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+          kv[0] = lo.x, kv[1] = lo.y, kv[2] = hi.x, kv[3] = hi.y;
+        } else {
+          const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kf + t * LKB + r0));
+          kv[0] = k2.x, kv[1] = k2.y;
+        }
+        const float4 z = *reinterpret_cast<const float4*>(Zs + t * NC + c0);
+        const float4 zu = *reinterpret_cast<const float4*>(Zu + t * NC + c0);
+        const float zv[4] = {z.x, z.y, z.z, z.w}, zuv[4] = {zu.x, zu.y, zu.z, zu.w};
+#pragma unroll
+        for (int e = 0; e < NR; ++e)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            sx[e][w] = fmaf(kv[e], zuv[w], sx[e][w]);
+            sy[e][w] = fmaf(kv[e], zv[w], sy[e][w]);
+          }
+      }
+#pragma unroll
+      for (int e = 0; e < NR; ++e)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          sx[e][w] += __shfl_xor_sync(0xffffffffu, sx[e][w], 1);
+          sx[e][w] += __shfl_xor_sync(0xffffffffu, sx[e][w], 2);
+          sy[e][w] += __shfl_xor_sync(0xffffffffu, sy[e][w], 1);
+          sy[e][w] += __shfl_xor_sync(0xffffffffu, sy[e][w], 2);
+        }
+      const float alC = ab[2 * (C - 1)], beC = ab[2 * (C - 1) + 1];
+      const float* sprev = scl + ((c + 1) & 1) * NC;  // maxima of the previous chunk (1 before chunk 0)
+      float* snext = scl + (c & 1) * NC;
+      // lane tp finishes row r0 + tp (NR == 4) or, for NR == 2, rows r0 + tp for tp < 2
+      if (tp < NR) {
+        float ax[4], ay[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) ax[w] = sx[0][w], ay[w] = sy[0][w];
+#pragma unroll
+        for (int e = 1; e < NR; ++e)
+          if (tp == e)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) ax[w] = sx[e][w], ay[w] = sy[e][w];
+        const int i = r0 + tp;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int col = c0 + w;
+          const int ex = (__float_as_int(sprev[col]) >> 23) & 0xff;
+          const float f = __int_as_float((254 - min(max(ex, 1), 253)) << 23);
+          const float x = Xt[col * LX + i], y = Yt[col * LX + i];
+          const float yn = f * (y + ay[w]);
+          Xt[col * LX + i] = f * fmaf(alC, x, fmaf(beC, y, ax[w]));
+          Yt[col * LX + i] = yn;
+          atomicMax(reinterpret_cast<int*>(&snext[col]), __float_as_int(fabsf(yn)));  // non-negative floats order as ints
+        }
+      }
+      (void)RPT;
     }
   }
 }
 
 // ---------------------------------------------------------------------------------------- P = X Y^-1
-// At every run start: LU with partial pivoting of Y^T (one warp picks each pivot, swaps and forms the
-// multipliers; every thread updates the trailing block), then P^T = Y^-T X^T by forward and back
-// substitution over the 128 right-hand sides, symmetrised.
-constexpr int kGJThreads = 256;
+// At every run start, Y^T P^T = X^T by Gauss-Jordan elimination with partial pivoting on the augmented
+// [Y^T | X^T] (D x 2D), held in registers: warp w owns rows 8w..8w+7, lane l columns CB l..CB l+CB-1.
+// Pivot rows are not swapped but recorded; once every column is eliminated, the row that was pivot for
+// column k holds row k of P^T in its right half.  P is written symmetrised.
+template <int D>
+struct ExtractLayout {
+  static constexpr int NT = 4 * D, NW = D / 8, CB = D / 16, LP = D + 1;
+  static constexpr int OFF_PROW = D * LP;           // 2 x [2D] normalised pivot row
+  static constexpr int OFF_PCOL = OFF_PROW + 4 * D;  // 2 x [D]  pivot column (the multipliers)
+  static constexpr int OFF_CV = OFF_PCOL + 2 * D;    // 2 x [NW] candidate pivot magnitudes
+  static constexpr int OFF_CR = OFF_CV + 2 * NW;     // 2 x [NW] candidate pivot rows (int)
+  static constexpr int OFF_INV = OFF_CR + 2 * NW;    // [D] column of each pivot row (int)
+  static constexpr size_t BYTES = (size_t)(OFF_INV + D) * 4;
+  static_assert(OFF_PROW % 4 == 0, "16-byte aligned pivot row");
+};
 
 template <int D>
-__global__ void __launch_bounds__(kGJThreads, 1) riccati_extract_kernel(RiccatiArgs p) {
-  constexpr int NT = kGJThreads, LD = D + 1;
-  extern __shared__ float gsm[];
-  float* A = gsm;                   // [D][LD]: Y^T, then its LU factors
-  float* Bm = gsm + D * LD;         // [D][LD]: X^T, then P^T
+__global__ void __launch_bounds__(4 * D, 1) riccati_extract_kernel(RiccatiArgs p) {
+  using Ly = ExtractLayout<D>;
+  constexpr int NT = Ly::NT, NW = Ly::NW, CB = Ly::CB, LP = Ly::LP;
+  extern __shared__ __align__(16) float xsm[];
+  float* Pt = xsm;  // [D][LP]: P^T
+  float* prow = xsm + Ly::OFF_PROW;
+  float* pcol = xsm + Ly::OFF_PCOL;
+  float* cand_v = xsm + Ly::OFF_CV;
+  int* cand_r = reinterpret_cast<int*>(xsm + Ly::OFF_CR);
+  int* invp = reinterpret_cast<int*>(xsm + Ly::OFF_INV);
+  __shared__ int bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x, sg = blockIdx.y, runs = gridDim.y;
   const float* xyc = p.xy + ((size_t)bh * runs + sg) * 2 * D * D;
@@ -257,73 +443,98 @@ __global__ void __launch_bounds__(kGJThreads, 1) riccati_extract_kernel(RiccatiA
     for (int idx = tid; idx < D * D; idx += NT) Pc[idx] = xyc[idx];
     return;
   }
-  for (int idx = tid; idx < D * D; idx += NT) {
-    const int rr = idx / D, cc = idx % D;  // X[rr][cc], Y[rr][cc]
-    Bm[cc * LD + rr] = xyc[(size_t)rr * D + cc];
-    A[cc * LD + rr] = xyc[(size_t)(D + rr) * D + cc];
+  // a[r][c] = [Y^T | X^T][8 warp + r][CB lane + c]; column j < D of the augmented matrix is row j of Y
+  float a[8][CB];
+#pragma unroll
+  for (int c = 0; c < CB; ++c) {
+    const int j = CB * lane + c;
+    const float* src = xyc + (size_t)(j < D ? D + j : j - D) * D + 8 * warp;
+    const float4 lo = *reinterpret_cast<const float4*>(src), hi = *reinterpret_cast<const float4*>(src + 4);
+    a[0][c] = lo.x, a[1][c] = lo.y, a[2][c] = lo.z, a[3][c] = lo.w;
+    a[4][c] = hi.x, a[5][c] = hi.y, a[6][c] = hi.z, a[7][c] = hi.w;
   }
-  __syncthreads();
-  bool singular = false;
-  // --- LU with partial pivoting: A = P L U (rows of A and Bm swapped together)
-  for (int k = 0; k < D; ++k) {
-    if (warp == 0) {
-      float best = -1.f;
-      int bi = k;
-      for (int i = k + lane; i < D; i += 32) {
-        const float v = fabsf(A[i * LD + k]);
-        if (v > best) best = v, bi = i;
+  if (tid == 0) bad = 0;
+  unsigned used = 0;  // rows of this warp already taken as pivots
+  for (int kb = 0; kb < D / CB; ++kb) {
+#pragma unroll
+    for (int cc = 0; cc < CB; ++cc) {
+      const int k = kb * CB + cc, buf = k & 1;
+      if (lane == kb) {  // this lane holds column k for the warp's rows: local pivot candidate, multipliers
+        float best = -1.f;
+        int br = 0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float v = fabsf(a[r][cc]);
+          if (!((used >> r) & 1u) && v > best) best = v, br = r;
+        }
+        cand_v[buf * NW + warp] = best;
+        cand_r[buf * NW + warp] = 8 * warp + br;
+        *reinterpret_cast<float4*>(pcol + buf * D + 8 * warp) = make_float4(a[0][cc], a[1][cc], a[2][cc], a[3][cc]);
+        *reinterpret_cast<float4*>(pcol + buf * D + 8 * warp + 4) = make_float4(a[4][cc], a[5][cc], a[6][cc], a[7][cc]);
       }
+      __syncthreads();
+      // the pivot: largest candidate, the lowest row on ties (every warp reduces the candidates itself)
+      float best = lane < NW ? cand_v[buf * NW + lane] : -2.f;
+      int pr = lane < NW ? cand_r[buf * NW + lane] : 0;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ob > best || (ob == best && oi < bi)) best = ob, bi = oi;
+        const int orr = __shfl_xor_sync(0xffffffffu, pr, o);
+        if (ob > best || (ob == best && orr < pr)) best = ob, pr = orr;
       }
-      if (bi != k)
-        for (int j = lane; j < D; j += 32) {
-          float t = A[k * LD + j];
-          A[k * LD + j] = A[bi * LD + j], A[bi * LD + j] = t;
-          t = Bm[k * LD + j];
-          Bm[k * LD + j] = Bm[bi * LD + j], Bm[bi * LD + j] = t;
-        }
-      __syncwarp();
-      const float piv = A[k * LD + k];
-      singular |= !(fabsf(piv) > 0.f);
-      const float inv = 1.f / piv;
-      for (int i = k + 1 + lane; i < D; i += 32) A[i * LD + k] *= inv;  // multipliers l_ik
+      if (warp == pr / 8) {  // the pivot's warp publishes the normalised pivot row
+        const int rp = pr % 8;
+        float row[CB];
+#pragma unroll
+        for (int c = 0; c < CB; ++c) row[c] = a[0][c];
+#pragma unroll
+        for (int r = 1; r < 8; ++r)
+          if (r == rp)
+#pragma unroll
+            for (int c = 0; c < CB; ++c) row[c] = a[r][c];
+        const float piv = pcol[buf * D + pr];
+        if (lane == 0 && !(fabsf(piv) > 0.f && isfinite(piv))) bad = 1;
+        const float inv = 1.f / piv;
+#pragma unroll
+        for (int c = 0; c < CB; ++c) prow[buf * 2 * D + CB * lane + c] = row[c] * inv;
+        used |= 1u << rp;
+      }
+      if (tid == 0) invp[pr] = k;
+      __syncthreads();
+      float pv[CB], mv[8];
+#pragma unroll
+      for (int c = 0; c < CB; ++c) pv[c] = prow[buf * 2 * D + CB * lane + c];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) mv[r] = pcol[buf * D + 8 * warp + r];
+      if (warp == pr / 8) {  // the pivot row takes the normalised row, the warp's other rows are eliminated
+        const int rp = pr % 8;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < CB; ++c) a[r][c] = r == rp ? pv[c] : fmaf(-mv[r], pv[c], a[r][c]);
+      } else {
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < CB; ++c) a[r][c] = fmaf(-mv[r], pv[c], a[r][c]);
+      }
     }
-    __syncthreads();
-    // trailing update A[i][j] -= l_ik A[k][j] (i, j > k)
-    const int w = D - 1 - k;
-    for (int idx = tid; idx < w * w; idx += NT) {
-      const int i = k + 1 + idx / w, j = k + 1 + idx % w;
-      A[i * LD + j] = fmaf(-A[i * LD + k], A[k * LD + j], A[i * LD + j]);
-    }
-    __syncthreads();
   }
-  // --- forward substitution L Z = Bm (unit lower), then back substitution U P^T = Z; 128 columns in parallel
-  for (int k = 0; k < D - 1; ++k) {
-    for (int idx = tid; idx < (D - 1 - k) * D; idx += NT) {
-      const int i = k + 1 + idx / D, j = idx % D;
-      Bm[i * LD + j] = fmaf(-A[i * LD + k], Bm[k * LD + j], Bm[i * LD + j]);
+  // right half of pivot row p = row invp[p] of P^T
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int k = invp[8 * warp + r];
+#pragma unroll
+    for (int c = 0; c < CB; ++c) {
+      const int j = CB * lane + c;
+      if (j >= D) Pt[k * LP + j - D] = a[r][c];
     }
-    __syncthreads();
   }
-  for (int k = D - 1; k >= 0; --k) {
-    const float inv = 1.f / A[k * LD + k];
-    for (int j = tid; j < D; j += NT) Bm[k * LD + j] *= inv;
-    __syncthreads();
-    for (int idx = tid; idx < k * D; idx += NT) {
-      const int i = idx / D, j = idx % D;
-      Bm[i * LD + j] = fmaf(-A[i * LD + k], Bm[k * LD + j], Bm[i * LD + j]);
-    }
-    __syncthreads();
-  }
-  if (singular && tid == 0) raise_status(p.status, kStatusNumeric);
-  // Bm = P^T; write P symmetrised
+  __syncthreads();
+  if (bad && tid == 0) raise_status(p.status, kStatusNumeric);
   for (int idx = tid; idx < D * D; idx += NT) {
     const int rr = idx / D, cc = idx % D;
-    Pc[idx] = 0.5f * (Bm[cc * LD + rr] + Bm[rr * LD + cc]);
+    Pc[idx] = 0.5f * (Pt[cc * LP + rr] + Pt[rr * LP + cc]);
   }
 }
 
@@ -332,10 +543,10 @@ cudaError_t launch_riccati_typed(const RiccatiArgs& a, cudaStream_t st) {
   const int nch = (a.L + kRC - 1) / kRC, runs = (nch + a.cps - 1) / a.cps, last = (runs - 1) * a.cps;
   cudaError_t e;
   if (last > 0) {  // the maps of the chunks before the last run start
-    const size_t map_smem = (size_t)kRC * (D + 1) * 4;
+    const size_t map_smem = (size_t)kRC * ((D + 4) + (kRC + 4)) * 4;
     e = cudaFuncSetAttribute(riccati_chunk_map_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)map_smem);
     if (e != cudaSuccess) return e;
-    riccati_chunk_map_kernel<D><<<dim3(a.BH, last), 2 * D, map_smem, st>>>(a);
+    riccati_chunk_map_kernel<D><<<dim3(a.BH, last), kMapThreads, map_smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -345,10 +556,10 @@ cudaError_t launch_riccati_typed(const RiccatiArgs& a, cudaStream_t st) {
   riccati_chain_kernel<D><<<dim3(a.BH, D / kRCols), kChainThreads, chain_smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t lu_smem = (size_t)2 * D * (D + 1) * 4;
-  e = cudaFuncSetAttribute(riccati_extract_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lu_smem);
+  const size_t x_smem = ExtractLayout<D>::BYTES;
+  e = cudaFuncSetAttribute(riccati_extract_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)x_smem);
   if (e != cudaSuccess) return e;
-  riccati_extract_kernel<D><<<dim3(a.BH, runs), kGJThreads, lu_smem, st>>>(a);
+  riccati_extract_kernel<D><<<dim3(a.BH, runs), ExtractLayout<D>::NT, x_smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -359,8 +570,8 @@ size_t riccati_scratch_bytes(int d, int BH, int L, int cps) {
   if (cps < 1) return 0;
   const size_t nch = ((size_t)L + kRC - 1) / kRC, chunks = (size_t)BH * nch;
   const size_t runs = (size_t)BH * ((nch + cps - 1) / cps);
-  return r256(chunks * kRC * 2 * d * 4) + r256(chunks * kRC * 4) + r256(chunks * 2 * 4) + r256(runs * 2 * d * d * 4) +
-         r256(runs * d * d * 4);
+  return r256(chunks * kRC * kRC * 4) + r256(chunks * kRC * 4) + r256(chunks * 2 * kRC * 4) +
+         r256(runs * 2 * d * d * 4) + r256(runs * d * d * 4);
 }
 
 cudaError_t launch_riccati_starts(int d, const RiccatiArgs& args, cudaStream_t stream) {

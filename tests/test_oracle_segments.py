@@ -195,3 +195,46 @@ def test_riccati_chunk_transfer_matrix_in_closed_form(seed):
     for t in range(C):
         M = _riccati_token_map(x["a"][t], x["qn"][t], x["k"][t], x["r"][t]) @ M
     np.testing.assert_allclose(_riccati_chunk_map(x["a"], x["qn"], x["k"], x["r"]), M, rtol=1e-11, atol=1e-12)
+
+
+def _riccati_chunk_apply_gform(a, qn, k, r, X, Y):
+    """The chunk map applied to [X; Y] without forming W: with G = (diag(r) - Cs^T)^-1, whose row j follows
+    g_jt = (delta_jt + sum_{m<t} g_jm Cs_tm) / r_t, the rank-C term is U Z with
+    Z = G^T (diag(alpha_t) K X + diag(beta_t) K Y), so that X' = alpha X + beta Y + K^T diag(beta_{C,j}) Z and
+    Y' = Y + K^T Z.  This is the order in which the chain kernel applies a chunk."""
+    C, d = k.shape
+    alpha = np.cumprod(a * a)
+    beta = np.zeros(C)
+    for t in range(C):
+        beta[t] = a[t] ** 2 * (beta[t - 1] if t else 0.0) + qn[t]
+    bt = np.zeros((C, C))
+    for j in range(C):
+        acc = 0.0
+        for t in range(j + 1, C):
+            acc = a[t] ** 2 * acc + qn[t]
+            bt[t, j] = acc
+    Cs = np.tril((k @ k.T) * bt, -1)
+    G = np.zeros((C, C))
+    for j in range(C):          # row j of G by the forward recurrence
+        for t in range(C):
+            G[j, t] = ((1.0 if t == j else 0.0) + G[j, :t] @ Cs[t, :t]) / r[t]
+    R = alpha[:, None] * (k @ X) + beta[:, None] * (k @ Y)
+    Z = G.T @ R
+    u = bt[C - 1]
+    return alpha[-1] * X + beta[-1] * Y + k.T @ (u[:, None] * Z), Y + k.T @ Z
+
+
+@pytest.mark.parametrize("seed", [0, 5])
+def test_riccati_chunk_map_applied_in_g_form(seed):
+    """The G form of a chunk's map (the chain kernel's arithmetic), with G from its row recurrence rather than
+    an inverse, equals the product of the chunk's token transfer matrices applied to [X; Y]."""
+    d, C, n = 5, 12, 4
+    x = _inputs(seed, C, d)
+    rng = np.random.default_rng(seed + 100)
+    X, Y = rng.standard_normal((d, n)), np.eye(d)[:, :n] + 0.1 * rng.standard_normal((d, n))
+    M = np.eye(2 * d)
+    for t in range(C):
+        M = _riccati_token_map(x["a"][t], x["qn"][t], x["k"][t], x["r"][t]) @ M
+    ref = M @ np.vstack([X, Y])
+    Xn, Yn = _riccati_chunk_apply_gform(x["a"], x["qn"], x["k"], x["r"], X, Y)
+    np.testing.assert_allclose(np.vstack([Xn, Yn]), ref, rtol=1e-11, atol=1e-12)
