@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // per-chunk scalars, two slots (chunk c uses slot c & 1)
   __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];         // a, beta | r, Qn
+  __shared__ __align__(16) float4 sVk[VAR == kDiag ? 2 : 1][kC];  // diagonal: (a^2, Qn, r) per token
   __shared__ float ell[2][kC], gn[2][kC];
   __shared__ __align__(16) float Aex[2][kC];                // A_t
   __shared__ __align__(16) float gcol[2][kC];               // 1 / A_t (times beta_t for the delta rule), when
@@ -162,7 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                             // A_C / A_t (times beta_t for the delta rule)
   __shared__ float en[4][kC];                               // ||e_t||^2 partials per lane quarter
   __shared__ float knorm[kC];                               // isotropic: ||k_t||^2 of the chunk
-  __shared__ float pend[VAR == kDiag ? D : 1];              // diagonal: p after the chunk whose variances ran
   __shared__ uint64_t kq_full[NKQ], kq_conv[NKQ], v_full, bar_c, bar_o, bar_p, tat_free;
   __shared__ uint64_t gates_ready[2], prep_done[2], chain_done[2], var_done[2];
   __shared__ uint32_t tmem_base;
@@ -249,7 +249,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto store_scalars = [&](int slot) {
     const int u = tid - kGroup;
-    if (u >= 0 && u < kC) sA[slot][u] = ra, sB[slot][u] = rb, sQ[slot][u] = rq;
+    if (u >= 0 && u < kC) {
+      sA[slot][u] = ra, sB[slot][u] = rb, sQ[slot][u] = rq;
+      if (VAR == kDiag) sVk[slot][u] = make_float4(ra * ra, rq, rb, 0.f);
+    }
   };
   // gates of chunk cc into its slot, by one warp: inclusive prefix sums of log a over the chunk (a gate of 0
   // enters as exp(-60)), A_t, and the state-update row scale A_C / A_t (times beta_t for the delta rule)
@@ -281,6 +284,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = tmem_base;
+
+  // Diagonal variances of chunk cc (independent of v and S), run by the chain one chunk ahead, in its wait
+  // for the preparation.  Per coordinate: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the
+  // homogeneous pair p = x / y: token t maps (x, y) by M_t = [[r a^2, r Qn], [k^2 a^2, k^2 Qn + r]], three
+  // multiply-adds of serial chain per token, the division that recovers p^- off the chain, and a
+  // power-of-two rescale every eight tokens (exact; x / y does not change).  One thread per coordinate steps
+  // all 64 tokens: this phase issues beside the preparation group, and a split of the tokens over threads
+  // (composing the earlier tokens' maps) only adds instructions, while the direct form p <- r p^- / s puts
+  // a division on the serial chain.  The unnormalised gains pk go, fp32, into the gain slot of chunk cc;
+  // p after the chunk stays in the thread.
+  auto run_variances = [&](int cc, int i, float& pcur) {
+    if (VAR == kDiag) {
+      const int sl = cc & 1;
+      // keys from the chunk's K tile as it landed (bf16): the preparation converts that tile to fp16 only
+      // after these variances are done
+      const uint8_t* Kp = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES + (i / 64) * Lay::KQ_PANEL;
+      float* Gw = reinterpret_cast<float*>(sm + Lay::OFF_G + 2 * sl * Lay::G_HALF);
+      const int gpos = gf_pos(i);
+      float x = pcur, y = 1.f;
+#pragma unroll 1
+      for (int t8 = 0; t8 < kC; t8 += 8) {
+        float kk[8];
+        float4 sv[8];  // a^2, Qn, r
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, i % 64)));
+          sv[u] = sVk[sl][t8 + u];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float xm = fmaf(sv[u].x, x, sv[u].y * y);
+          Gw[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
+          x = sv[u].z * xm;
+          y = fmaf(kk[u] * kk[u], xm, sv[u].z * y);
+        }
+        const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
+        const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
+        x *= sc, y *= sc;
+      }
+      pcur = __fdividef(x, y);
+    }
+  };
 
   if (tid < kGroup) {
     // =============================================================================== chain group
@@ -322,76 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto kq_addr_of = [&](int cc) { return sm100::smem_u32(sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES); };
 
-    // Diagonal variances of chunk cc (independent of v and S), run one chunk ahead while the chain waits for
-    // the preparation.  Per coordinate: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the
-    // homogeneous pair p = x / y: token t maps (x, y) by M_t = [[r a^2, r Qn], [k^2 a^2, k^2 Qn + r]], three
-    // multiply-adds of serial chain per token, the division that recovers p^- off the chain, and a
-    // power-of-two rescale every four tokens that keeps y in [1, 2).  Two threads per coordinate: thread i
-    // runs tokens 0..31 from p, thread D + i runs tokens 32..63 from the product of the first 32 maps
-    // applied to p (the maps compose: Kalman Delta Networks, Abstract, uncertainty recurrences as Moebius
-    // maps), so the serial part is half a chunk.  The unnormalised gains pk go, fp32, into the gain slot of
-    // chunk cc; the value after the chunk goes to pend[i], read by both threads after the group's barrier.
-    float pcur = 1.f;
-    if (VAR == kDiag) pcur = P.p[(size_t)bh * D + (tid & (D - 1))];
-    auto run_variances = [&](int cc) {
-      if (VAR == kDiag) {
-        const int i = tid & (D - 1), hh = tid / D;  // coordinate, token half (the chain group is 2 D threads)
-        const int sl = cc & 1;
-        // keys from the chunk's K tile as it landed (bf16): the preparation converts that tile to fp16 only
-        // after these variances are done
-        const uint8_t* Kp = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES + (i / 64) * Lay::KQ_PANEL;
-        auto key = [&](int t) {
-          return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t, i % 64)));
-        };
-        float* Gw = reinterpret_cast<float*>(sm + Lay::OFF_G + 2 * sl * Lay::G_HALF);
-        const int gpos = gf_pos(i);
-        float x = pcur, y = 1.f;
-        auto rescale = [&]() {
-          const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
-          const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
-          x *= sc, y *= sc;
-        };
-        if (hh == 1) {
-          // (x, y) <- M_31 ... M_0 (x, y), eight maps multiplied out at a time, then applied
-#pragma unroll 1
-          for (int t8 = 0; t8 < kC / 2; t8 += 8) {
-            float m00 = 1.f, m01 = 0.f, m10 = 0.f, m11 = 1.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float kv = key(t8 + u);
-              const float av = sA[sl][t8 + u], rv = sB[sl][t8 + u], qv = sQ[sl][t8 + u];
-              const float a2 = av * av, k2 = kv * kv;
-              const float b00 = rv * a2, b01 = rv * qv, b10 = k2 * a2, b11 = fmaf(k2, qv, rv);
-              const float n00 = fmaf(b00, m00, b01 * m10), n01 = fmaf(b00, m01, b01 * m11);
-              const float n10 = fmaf(b10, m00, b11 * m10), n11 = fmaf(b10, m01, b11 * m11);
-              m00 = n00, m01 = n01, m10 = n10, m11 = n11;
-            }
-            const float xn = fmaf(m00, x, m01 * y), yn = fmaf(m10, x, m11 * y);
-            x = xn, y = yn;
-            rescale();
-          }
-        }
-#pragma unroll 1
-        for (int t8 = hh * (kC / 2); t8 < (hh + 1) * (kC / 2); t8 += 8) {
-          float kk[8], aa[8], rr8[8], qq[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            kk[u] = key(t8 + u);
-            aa[u] = sA[sl][t8 + u], rr8[u] = sB[sl][t8 + u], qq[u] = sQ[sl][t8 + u];
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float xm = fmaf(aa[u] * aa[u], x, qq[u] * y);
-            Gw[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
-            x = rr8[u] * xm;
-            y = fmaf(kk[u] * kk[u], xm, rr8[u] * y);
-            if (u % 4 == 3) rescale();
-          }
-        }
-        if (hh == 1) pend[i] = __fdividef(x, y);
-      }
-    };
-
+    // diagonal: p of coordinate tid (threads 0..D-1, warps 0..3, run the variances; warp 4 the gates)
+    const bool var_thread = VAR == kDiag && tid < D;
+    float pcur = var_thread ? P.p[(size_t)bh * D + tid] : 1.f;
     float* Sg = P.S + (size_t)bh * D * D;
     if (!kConvInPrep) {  // [K; Q] of chunk 0
       if (!gwait(&kq_full[0], 0)) {
@@ -406,10 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!gwait(&kq_full[0], 0)) {
         aborted = true;
       } else {
-        run_variances(0);
+        if (var_thread) run_variances(0, tid, pcur);
         if (gw == 4) run_gates(0);
         named_sync(kBarChain, kGroup);
-        if (VAR == kDiag) pcur = pend[tid & (D - 1)];
         if (leader) sm100::mbar_arrive(&var_done[0]);
       }
     }
@@ -477,10 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // its scalars were stored before gates_ready of chunk c; its keys are read before the preparation
         // converts their tile (that waits for var_done)
         if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
-        run_variances(c + 1);
+        if (var_thread) run_variances(c + 1, tid, pcur);
         if (gw == 4) run_gates(c + 1);
         named_sync(kBarChain, kGroup);
-        if (VAR == kDiag) pcur = pend[tid & (D - 1)];
         if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
       }
 
@@ -499,6 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         if (!gwait(&bar_c, ph_c)) { aborted = true; break; }
         ph_c ^= 1;
+        // without the delta rule the state product reads G, not K: this slot's K, Q are dead once the S0
+        // product is (the preparation was done with them before prep_done), so the tile two chunks ahead
+        // loads a whole chain phase earlier than at the chunk's end
+        if (!delta_like(VAR) && leader && c + NKQ < nchunks) issue_kq(c + NKQ);
         float X[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_D2 + 32 * half, X);
         sm100::tmem_wait_ld();
@@ -655,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (leader) {
         sm100::mbar_arrive(&chain_done[s]);
-        if (c + NKQ < nchunks) issue_kq(c + NKQ);  // this slot's K, Q are dead
+        if (delta_like(VAR) && c + NKQ < nchunks) issue_kq(c + NKQ);  // this slot's K, Q are dead
       }
     }
     if (!aborted) {
@@ -667,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 32; ++u) Sg[(size_t)(64 * half + 32 * v + u) * D + j] = x[u];
       }
-      if (VAR == kDiag && tid < D) P.p[(size_t)bh * D + tid] = pcur;
+      if (var_thread) P.p[(size_t)bh * D + tid] = pcur;
     }
   } else {
     // =============================================================================== preparation group
