@@ -43,14 +43,21 @@ constexpr int kBwdThreads = 512;
 constexpr float kLogFloor = -60.f;  // a gate of 0 enters the logs as exp(-60), as in the forward
 
 // C[i][j] (row stride ldc) = alpha * sum_k A(i,k) B(k,j) (+ C[i][j] when acc), for i < M, j < N, with
-// A(i,k) = A[i ai + k ak] and B(k,j) = B[k bk + j bj] in shared memory.  Each thread takes TM x TN
-// outputs per tile.  Ends with a barrier.
+// A(i,k) = A[i ai + k ak] and B(k,j) = B[k bk + j bj] in shared memory (C aliases neither).  Each thread
+// takes a TM x TN register tile (TM + TN loads per TM TN multiply-adds); when the tiles are fewer than the
+// threads, S adjacent lanes share a tile, each summing every S-th k, and their parts are summed by shuffles
+// (TILES S is then a multiple of 32 and at most the block, so every lane of a warp takes part).  Ends with
+// a barrier.
 template <int M, int N, int K, int TM, int TN>
 __device__ __forceinline__ void mm(float* C, int ldc, const float* A, int ai, int ak, const float* B, int bk, int bj,
                                    float alpha, bool acc) {
   static_assert(M % TM == 0 && N % TN == 0, "tile");
   constexpr int NTI = N / TN, TILES = (M / TM) * NTI;
-  for (int tile = threadIdx.x; tile < TILES; tile += kBwdThreads) {
+  constexpr int S0 = kBwdThreads / TILES < 1 ? 1 : kBwdThreads / TILES;
+  constexpr int S = S0 >= 8 && K % 8 == 0 ? 8 : S0 >= 4 && K % 4 == 0 ? 4 : S0 >= 2 && K % 2 == 0 ? 2 : 1;
+  static_assert(S == 1 || (TILES * S % 32 == 0 && TILES * S <= kBwdThreads), "whole warps share the tiles");
+  for (int item = threadIdx.x; item < TILES * S; item += kBwdThreads) {
+    const int sp = item % S, tile = item / S;
     const int i0 = (tile / NTI) * TM, j0 = (tile % NTI) * TN;
     float s[TM][TN];
 #pragma unroll
@@ -58,7 +65,7 @@ __device__ __forceinline__ void mm(float* C, int ldc, const float* A, int ai, in
 #pragma unroll
       for (int w = 0; w < TN; ++w) s[u][w] = 0.f;
 #pragma unroll 4
-    for (int k = 0; k < K; ++k) {
+    for (int k = sp; k < K; k += S) {
       float av[TM], bv[TN];
 #pragma unroll
       for (int u = 0; u < TM; ++u) av[u] = A[(i0 + u) * ai + k * ak];
@@ -70,12 +77,20 @@ __device__ __forceinline__ void mm(float* C, int ldc, const float* A, int ai, in
         for (int w = 0; w < TN; ++w) s[u][w] = fmaf(av[u], bv[w], s[u][w]);
     }
 #pragma unroll
-    for (int u = 0; u < TM; ++u)
+    for (int o = S / 2; o > 0; o >>= 1)
 #pragma unroll
-      for (int w = 0; w < TN; ++w) {
-        float* c = C + (i0 + u) * ldc + j0 + w;
-        *c = acc ? fmaf(alpha, s[u][w], *c) : alpha * s[u][w];
-      }
+      for (int u = 0; u < TM; ++u)
+#pragma unroll
+        for (int w = 0; w < TN; ++w) s[u][w] += __shfl_xor_sync(0xffffffffu, s[u][w], o);
+    if (sp == 0) {
+#pragma unroll
+      for (int u = 0; u < TM; ++u)
+#pragma unroll
+        for (int w = 0; w < TN; ++w) {
+          float* c = C + (i0 + u) * ldc + j0 + w;
+          *c = acc ? fmaf(alpha, s[u][w], *c) : alpha * s[u][w];
+        }
+    }
   }
   __syncthreads();
 }
@@ -241,8 +256,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       Gam[i * LC + j] = j <= i ? __expf(vell[i] - vell[j]) : 0.f;
     }
     // ------------------------------------------------------------------ forward recompute of the chunk
-    mm<C, C, DK, 1, 1>(KG, LC, Kc, LK, 1, Kc, 1, LK, 1.f, false);  // K K^T
-    mm<C, C, DK, 1, 1>(QG, LC, Qc, LK, 1, Kc, 1, LK, 1.f, false);  // Q K^T
+    mm<C, C, DK, 4, 4>(KG, LC, Kc, LK, 1, Kc, 1, LK, 1.f, false);  // K K^T
+    mm<C, C, DK, 4, 4>(QG, LC, Qc, LK, 1, Kc, 1, LK, 1.f, false);  // Q K^T
     for (int idx = tid; idx < C * C; idx += NT) {
       const int i = idx / C, j = idx % C;
       const float kg = KG[i * LC + j] * vb[j], qg = QG[i * LC + j] * vb[j], g = Gam[i * LC + j];
@@ -266,17 +281,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       for (int i = 0; i < C; ++i) Tt[i * LC + cc] = t[i];
     }
     __syncthreads();
-    mm<C, C, C, 1, 1>(AT, LC, Mm, LC, 1, Tt, LC, 1, 1.f, false);
-    mm<C, JB, DK, 1, 1>(KS, LJ, Kc, LK, 1, S0, LJ, 1, 1.f, false);
-    mm<C, JB, DK, 1, 1>(QS, LJ, Qc, LK, 1, S0, LJ, 1, 1.f, false);
+    mm<C, C, C, 2, 2>(AT, LC, Mm, LC, 1, Tt, LC, 1, 1.f, false);
+    mm<C, JB, DK, 4, 4>(KS, LJ, Kc, LK, 1, S0, LJ, 1, 1.f, false);
+    mm<C, JB, DK, 4, 4>(QS, LJ, Qc, LK, 1, S0, LJ, 1, 1.f, false);
     for (int idx = tid; idx < C * JB; idx += NT) {
       const int i = idx / JB, j = idx % JB;
       Rr[i * LJ + j] = Vc[i * LJ + j] - vA[i] * KS[i * LJ + j];
     }
     __syncthreads();
-    mm<C, JB, C, 1, 1>(Ee, LJ, Tt, LC, 1, Rr, LJ, 1, 1.f, false);  // E = T R
+    mm<C, JB, C, 2, 2>(Ee, LJ, Tt, LC, 1, Rr, LJ, 1, 1.f, false);  // E = T R
     // ------------------------------------------------------------------ backward of the chunk
-    mm<C, JB, DK, 1, 1>(dE, LJ, Kc, LK, 1, dS, LJ, 1, 1.f, false);  // K dS
+    mm<C, JB, DK, 4, 4>(dE, LJ, Kc, LK, 1, dS, LJ, 1, 1.f, false);  // K dS
     {
       float acc = 0.f;  // dLoss/dA_C from S_C = A_C S0 + ...: this block's sum of dS o S0
       for (int idx = tid; idx < DK * JB; idx += NT) {
@@ -293,15 +308,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       dE[i * LJ + j] = de;
     }
     __syncthreads();
-    mm<DK, C, JB, 2, 1>(dW, LC, dS, LJ, 1, Ee, 1, LJ, 1.f, false);           // dW = dS E^T
-    mm<C, C, JB, 1, 1>(dAT, LC, dOc, LJ, 1, Rr, 1, LJ, 1.f, false);          // dAT = dO R^T
-    mm<C, JB, C, 1, 1>(dR, LJ, AT, 1, LC, dOc, LJ, 1, 1.f, false);           // dR = AT^T dO
-    mm<C, JB, C, 1, 1>(dR, LJ, Tt, 1, LC, dE, LJ, 1, 1.f, true);             //    + T^T dE
-    mm<C, C, JB, 1, 1>(dT, LC, dE, LJ, 1, Rr, 1, LJ, 1.f, false);           // dT = dE R^T
-    mm<C, C, C, 1, 1>(dT, LC, Mm, 1, LC, dAT, LC, 1, 1.f, true);             //    + M^T dAT
-    mm<C, C, C, 1, 1>(dM, LC, dAT, LC, 1, Tt, 1, LC, 1.f, false);            // dM = dAT T^T (masked below)
-    mm<C, C, C, 1, 1>(dAT, LC, Tt, 1, LC, dT, LC, 1, 1.f, false);            // X = T^T dT (over dAT)
-    mm<C, C, C, 1, 1>(dN, LC, dAT, LC, 1, Tt, 1, LC, -1.f, false);           // dN = -X T^T (masked below)
+    mm<DK, C, JB, 4, 4>(dW, LC, dS, LJ, 1, Ee, 1, LJ, 1.f, false);           // dW = dS E^T
+    mm<C, C, JB, 2, 2>(dAT, LC, dOc, LJ, 1, Rr, 1, LJ, 1.f, false);          // dAT = dO R^T
+    mm<C, JB, C, 2, 2>(dR, LJ, AT, 1, LC, dOc, LJ, 1, 1.f, false);           // dR = AT^T dO
+    mm<C, JB, C, 2, 2>(dR, LJ, Tt, 1, LC, dE, LJ, 1, 1.f, true);             //    + T^T dE
+    mm<C, C, JB, 2, 2>(dT, LC, dE, LJ, 1, Rr, 1, LJ, 1.f, false);           // dT = dE R^T
+    mm<C, C, C, 2, 2>(dT, LC, Mm, 1, LC, dAT, LC, 1, 1.f, true);             //    + M^T dAT
+    mm<C, C, C, 2, 2>(dM, LC, dAT, LC, 1, Tt, 1, LC, 1.f, false);            // dM = dAT T^T (masked below)
+    mm<C, C, C, 2, 2>(dAT, LC, Tt, 1, LC, dT, LC, 1, 1.f, false);            // X = T^T dT (over dAT)
+    mm<C, C, C, 2, 2>(dN, LC, dAT, LC, 1, Tt, 1, LC, -1.f, false);           // dN = -X T^T (masked below)
     for (int idx = tid; idx < C * C; idx += NT) {
       const int i = idx / C, j = idx % C;
       const float dn = j < i ? dN[i * LC + j] : 0.f, dmv = j <= i ? dM[i * LC + j] : 0.f, g = Gam[i * LC + j];
@@ -330,35 +345,76 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
     // dq_ik = sum_j dQS_ij S0_kj + sum_m dQG_im beta_m K_mk
     // dk_ik = sum_j dKS_ij S0_kj + sum_m dKG_im beta_m K_mk + beta_i dG_ik
     // dG_ik = sum_m dKG_mi K_mk + sum_m dQG_mi Q_mk + r_i dW_ki (+ the surprise term, first block)
-    for (int idx = tid; idx < C * DK; idx += NT) {
-      const int i = idx / DK, kk = idx % DK;
-      float dq = 0.f, dk = 0.f, dg = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < JB; ++j) {
-        const float s0 = S0[kk * LJ + j];
-        dq = fmaf(dOc[i * LJ + j], s0, dq);
-        dk = fmaf(dR[i * LJ + j], s0, dk);
-      }
-#pragma unroll 8
-      for (int m = 0; m < C; ++m) {
-        const float km = Kc[m * LK + kk], bk = vb[m] * km;
-        dq = fmaf(dM[i * LC + m], bk, dq);
-        dk = fmaf(dN[i * LC + m], bk, dk);
-        dg = fmaf(dN[m * LC + i], km, dg);
-        dg = fmaf(dM[m * LC + i], Qc[m * LK + kk], dg);
-      }
-      dg = fmaf(vr[i], dW[kk * LC + i], dg);
-      if (first_block && vkn[i] > 0.f) dg = fmaf(vdm[i] * ven[i] / vkn[i], Kc[i * LK + kk], dg);
-      dk = fmaf(vb[i], dg, dk);
-      // dbeta_i = k_i . dG_i: a warp holds 32 consecutive k of one token (two tokens when d_k = 16)
-      float db = Kc[i * LK + kk] * dg;
+    // Thread: tokens i0, i0 + 1 and the four columns kk = kq + (DK / 4) e (a warp reads 32 consecutive
+    // columns of a row at a time).
+    {
+      constexpr int KQ = DK / 4, SEG = KQ < 32 ? KQ : 32;  // lanes that share a token pair
+      for (int item = tid; item < (C / 2) * KQ; item += NT) {
+        const int i0 = 2 * (item / KQ), kq = item % KQ;
+        float dq[2][4], dk[2][4], dg[2][4];
 #pragma unroll
-      for (int o = (DK < 32 ? DK : 32) / 2; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
-      if (lane % (DK < 32 ? DK : 32) == 0) atomicAdd(&vdb[i], db);
-      if (i < n) {
-        const size_t off = (tok0 + t0 + i) * DK + kk;
-        atomicAdd(p.dq + off, dq);
-        atomicAdd(p.dk + off, dk);
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dq[a][e] = dk[a][e] = dg[a][e] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < JB; ++j) {
+          const float o0 = dOc[i0 * LJ + j], o1 = dOc[(i0 + 1) * LJ + j];
+          const float r0 = dR[i0 * LJ + j], r1 = dR[(i0 + 1) * LJ + j];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float s0 = S0[(kq + KQ * e) * LJ + j];
+            dq[0][e] = fmaf(o0, s0, dq[0][e]), dq[1][e] = fmaf(o1, s0, dq[1][e]);
+            dk[0][e] = fmaf(r0, s0, dk[0][e]), dk[1][e] = fmaf(r1, s0, dk[1][e]);
+          }
+        }
+#pragma unroll 4
+        for (int m = 0; m < C; ++m) {
+          const float bm = vb[m];
+          const float qa0 = dM[i0 * LC + m] * bm, qa1 = dM[(i0 + 1) * LC + m] * bm;
+          const float ka0 = dN[i0 * LC + m] * bm, ka1 = dN[(i0 + 1) * LC + m] * bm;
+          const float gk0 = dN[m * LC + i0], gk1 = dN[m * LC + i0 + 1];
+          const float gq0 = dM[m * LC + i0], gq1 = dM[m * LC + i0 + 1];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float km = Kc[m * LK + kq + KQ * e], qm = Qc[m * LK + kq + KQ * e];
+            dq[0][e] = fmaf(qa0, km, dq[0][e]), dq[1][e] = fmaf(qa1, km, dq[1][e]);
+            dk[0][e] = fmaf(ka0, km, dk[0][e]), dk[1][e] = fmaf(ka1, km, dk[1][e]);
+            dg[0][e] = fmaf(gk0, km, fmaf(gq0, qm, dg[0][e]));
+            dg[1][e] = fmaf(gk1, km, fmaf(gq1, qm, dg[1][e]));
+          }
+        }
+        float db[2];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int i = i0 + a;
+          const float sur = first_block && vkn[i] > 0.f ? vdm[i] * ven[i] / vkn[i] : 0.f;
+          db[a] = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kk = kq + KQ * e;
+            const float ki = Kc[i * LK + kk];
+            float g = fmaf(vr[i], dW[kk * LC + i], dg[a][e]);
+            g = fmaf(sur, ki, g);
+            dk[a][e] = fmaf(vb[i], g, dk[a][e]);
+            db[a] = fmaf(ki, g, db[a]);  // dbeta_i = k_i . dG_i
+          }
+          if (i < n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const size_t off = (tok0 + t0 + i) * DK + kq + KQ * e;
+              atomicAdd(p.dq + off, dq[a][e]);
+              atomicAdd(p.dk + off, dk[a][e]);
+            }
+          }
+        }
+        // the token pair's SEG lanes sum their columns' parts (every lane of a warp is here: (C / 2) KQ is a
+        // multiple of 32)
+#pragma unroll
+        for (int o = SEG / 2; o > 0; o >>= 1) {
+          db[0] += __shfl_xor_sync(0xffffffffu, db[0], o);
+          db[1] += __shfl_xor_sync(0xffffffffu, db[1], o);
+        }
+        if (lane % SEG == 0) atomicAdd(&vdb[i0], db[0]), atomicAdd(&vdb[i0 + 1], db[1]);
       }
     }
     // dLoss/dr_j = beta_j sum_k K_jk dW_kj
@@ -404,15 +460,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       }
     }
     // ------------------------------------------------------------------ dS0 = A_C dS + Q^T dQS + K^T dKS, in place
+    // thread: rows kk = kq + (DK / 4) e and columns j0, j0 + 1
     {
+      constexpr int KQ = DK / 4, JP = JB / 2;
       const float AC = vA[C - 1];
-      for (int idx = tid; idx < DK * JB; idx += NT) {
-        const int kk = idx / JB, j = idx % JB;
-        float acc = AC * dS[kk * LJ + j];
-#pragma unroll 8
-        for (int i = 0; i < C; ++i)
-          acc = fmaf(Qc[i * LK + kk], dOc[i * LJ + j], fmaf(Kc[i * LK + kk], dR[i * LJ + j], acc));
-        dS[kk * LJ + j] = acc;
+      for (int item = tid; item < KQ * JP; item += NT) {
+        const int kq = item / JP, jj = 2 * (item % JP);
+        float acc[4][2];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[e][0] = AC * dS[(kq + KQ * e) * LJ + jj];
+          acc[e][1] = AC * dS[(kq + KQ * e) * LJ + jj + 1];
+        }
+#pragma unroll 4
+        for (int i = 0; i < C; ++i) {
+          const float o0 = dOc[i * LJ + jj], o1 = dOc[i * LJ + jj + 1];
+          const float r0 = dR[i * LJ + jj], r1 = dR[i * LJ + jj + 1];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float qv = Qc[i * LK + kq + KQ * e], kv = Kc[i * LK + kq + KQ * e];
+            acc[e][0] = fmaf(qv, o0, fmaf(kv, r0, acc[e][0]));
+            acc[e][1] = fmaf(qv, o1, fmaf(kv, r1, acc[e][1]));
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dS[(kq + KQ * e) * LJ + jj] = acc[e][0];
+          dS[(kq + KQ * e) * LJ + jj + 1] = acc[e][1];
+        }
       }
     }
   }
