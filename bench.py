@@ -81,23 +81,25 @@ _WS_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/chunk_scan_ws.cu",
                "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
                "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
                "delta_rule_recurrent_scan_b200/csrc/mobius.cuh"]
-_PSIDE_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/pside.cu",
-                  "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
-                  "delta_rule_recurrent_scan_b200/csrc/sm100.cuh"]
+_RICCATI_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/riccati.cu",
+                    "delta_rule_recurrent_scan_b200/csrc/chunk_common.cuh",
+                    "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
+                    "delta_rule_recurrent_scan_b200/csrc/common.cuh"]
 _B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment per head)
+_WS_SHA = "94549d85257830a12ddfefcedfdfdaa6908ef443"
 NCU_TRAFFIC = {
-    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
-                         "bytes_per_token": (308.443648e6 + 171.383808e6) / _B3,
+    "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
+                         "bytes_per_token": (308.566272e6 + 171.428096e6) / _B3,
                          "capture": "ncu, chunk_scan_ws_kernel<diag> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "gdn_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
-                 "bytes_per_token": (308.621056e6 + 170.472192e6) / _B3,
+    "gdn_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
+                 "bytes_per_token": (308.382976e6 + 171.018496e6) / _B3,
                  "capture": "ncu, chunk_scan_ws_kernel<delta> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": "4c45c2f9a1e2aa60a36438f975021ae3a7a2114f",
-                        "bytes_per_token": (308.480256e6 + 171.998976e6) / _B3,
+    "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
+                        "bytes_per_token": (308.413952e6 + 170.260480e6) / _B3,
                         "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_full_d128": {"sources": _PSIDE_SOURCES, "sha1": "0bbdf6201df85beaf0b536f88b1722c9cc0b5c8e",
-                         "bytes_per_token": (18.464256e6 + 5.376e3) / (2 * 8 * 4096),
-                         "capture": "ncu, kalman_pside_kernel at the full workload B=2 H=8 L=4096"},
+    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "4a83c95c4b2bec424ca3c3aa8e46b412a0ae6adf",
+                         "bytes_per_token": (31.122432e6 + 1.151488e6) / (2 * 8 * 4096),
+                         "capture": "ncu, riccati_chain_kernel at the full workload B=2 H=8 L=4096"},
 }
 
 
@@ -519,6 +521,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--batch", type=int, default=None, help="override B of the workload (profiling runs)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward of a gated-delta workload (profiling runs): one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -544,6 +548,20 @@ def main():
 
     kdn.lib()  # fail loudly if the library is missing
     peak, peak_kind = measured_peaks()
+    if args.backward_only:
+        if w.variant != "delta":
+            raise SystemExit("--backward-only needs a gated-delta workload")
+        r = bench_backward(w, args.steps, args.warmup, dist_on, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "backward tokens/s (dq, dk, dv, dbeta, da, dS0)", "value": r["value"],
+                              "unit": "tokens/s", "ms_per_step": r["ms"], "steps": args.steps,
+                              "warmup": args.warmup, "gpu_launches": r["launches"],
+                              "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk}}),
+                  flush=True)
+        if dist_on:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     clocks = ClockSampler(local)
     head = bench_scan(w, args.steps, args.warmup, dist_on, rank, world, clocks=clocks)
     ms = head["ms"]

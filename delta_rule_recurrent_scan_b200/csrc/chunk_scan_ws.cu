@@ -27,9 +27,8 @@
 //
 // so the residual R = V - diag(A) K S0 is never formed: its V part runs on the tensor cores while the
 // chain converts (K S0)^T, and the decay enters through the preparation's scaled copy of T.  The read-out
-// uses Attn E (= AT R, with Attn = lower((Q G^T) o Gam)), so the preparation never forms AT.
-//
-// and the preparation keeps the row-major products [K; Q] G^T and [T; Attn] T.
+// uses Attn E (= AT R, with Attn = lower((Q G^T) o Gam)), so the preparation never forms AT; its one
+// product is the row-major [K; Q] G^T.
 // fp32 state master and accumulators in TMEM.  Every tensor-core operand is fp16: K and Q are
 // converted from bf16 in shared memory when their tile lands (exact in fp16's normal range), the fp32
 // operands (state, (K S0), innovations, gains, T, Attn) are rounded to fp16 once.  A float64 emulation of these

@@ -288,8 +288,10 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
   int nseg = 1;
   KDN_TRY(resolve_segments(variant, dims, &nseg));
   if (nseg > 1) {
-    // start states, two map runs, chaining, the true run (+ the diagonal uncertainty maps and starts)
+    // start states, two map runs, chaining, the true run (+ the diagonal uncertainty maps and starts; for
+    // full Kalman the chunk maps, their chain, the run-start covariances and the covariance side)
     n = 5 + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 4 : 0);
+    if (body == KDN_KALMAN_FULL) name = "riccati_chain_kernel", ar = "f32";  // the longest of those launches
   }
   if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1))
     n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself on the serial path)
