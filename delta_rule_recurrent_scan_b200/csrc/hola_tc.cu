@@ -363,6 +363,333 @@ __global__ void __launch_bounds__(kTThreads, 1)
   if (warp == 0) sm100::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------------------- parallel form
+// The cache a block reads depends only on m (section 3.3: the top-w tokens by surprise), not on any read, so
+// it can be fixed for every block first.  hola_cache_select_kernel walks one head's blocks with 128 threads,
+// one per candidate (the cache, then the block's tokens): each candidate's rank is the number of others that
+// come before it (larger m, ties to the earlier token), the first w by rank form the next cache, and the
+// cache read by block b goes to cidx[head][b] in rank order (-1 past its size).  It also writes the final
+// cache's indices, ascending.
+constexpr int kSelThreads = 4 * kRows;  // four lanes per candidate, each comparing every fourth other
+
+__global__ void __launch_bounds__(kSelThreads) hola_cache_select_kernel(HolaArgs p) {
+  __shared__ float cm[kRows];  // candidates: rows 0..63 the cache (rank order), 64..127 the block
+  __shared__ int ci[kRows];
+  __shared__ float nm[64];
+  __shared__ int ni[64];
+  const int tid = threadIdx.x, cand = tid >> 2, part = tid & 3, bh = blockIdx.x, L = p.L, w = p.w;
+  const int nblocks = (L + 63) / 64;
+  const size_t tok0 = (size_t)bh * L;
+  const bool owner = part == 0;  // the lane that stores the candidate's results
+  if (owner && cand < 64) cm[cand] = -INFINITY, ci[cand] = -1;
+  int ncache = 0;
+  float mnext = owner && cand >= 64 && cand - 64 < L ? p.m[tok0 + cand - 64] : -INFINITY;
+  for (int b = 0; b < nblocks; ++b) {
+    if (owner && cand >= 64) {
+      const int t = 64 * b + cand - 64;
+      ci[cand] = t < L ? t : -1;
+      cm[cand] = t < L ? mnext : -INFINITY;
+      const int tn = t + 64;
+      mnext = tn < L ? p.m[tok0 + tn] : -INFINITY;  // the next block's m, in flight during the ranking
+    }
+    __syncthreads();
+    if (owner && cand < 64) p.cidx[((size_t)bh * nblocks + b) * 64 + cand] = ci[cand];
+    const float m0 = cm[cand];
+    const int i0 = ci[cand];
+    int rank = 0;
+#pragma unroll 8
+    for (int c = part; c < kRows; c += 4) rank += (ci[c] >= 0 && before(cm[c], ci[c], m0, i0)) ? 1 : 0;  // 4 banks
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+    const bool kept = owner && i0 >= 0 && rank < w;
+    if (kept) nm[rank] = m0, ni[rank] = i0;
+    ncache = __syncthreads_count(kept);  // also: every read of cm, ci above is done
+    if (owner && cand < 64) {
+      cm[cand] = cand < ncache ? nm[cand] : -INFINITY;
+      ci[cand] = cand < ncache ? ni[cand] : -1;
+    }
+    __syncthreads();
+  }
+  if (p.cache != nullptr && tid < w) {  // the final cache, ascending token indices, -1 past its size
+    const int mine = tid < ncache ? ci[tid] : -1;
+    if (mine >= 0) {
+      int pos = 0;
+      for (int c = 0; c < ncache; ++c) pos += ci[c] < mine ? 1 : 0;
+      p.cache[(size_t)bh * w + pos] = mine;
+    } else {
+      p.cache[(size_t)bh * w + tid] = -1;
+    }
+  }
+}
+
+// hola_read_block_kernel: one CTA per head and run of kBlocksPerCta consecutive blocks, two CTAs per SM.  Each
+// block's q, k, v arrive by TMA, its cache rows by 16-byte cp.async gathers of the token indices chosen above
+// (rows 0..63; empty rows zero), then the same S product, softmax with the sink and P V product as the serial
+// kernel.  While a block is read, the next block's tiles and cache rows are prefetched into L2.
+// The raw queries land in the lo panel: each thread reads its 16-byte chunk there before it writes the lo
+// half of the scaled query to the same address, so the CTA fits twice in an SM's shared memory.
+constexpr int kBlocksPerCta = 4;
+constexpr int PB_K = 0, PB_V = kBuf, PB_H = 2 * kBuf, PB_L = PB_H + kPanel, PB_QS = PB_L;
+constexpr int kPSmem = PB_L + kPanel + 1024;
+
+__device__ __forceinline__ void cp_async16_cg(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
+
+__global__ void __launch_bounds__(kTThreads, 2)
+    hola_read_block_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, HolaArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ float rk[kRows];        // 1 / rms(k) per row (0 for empty rows)
+  __shared__ int crow[64];           // token index of cache row r (-1 = empty)
+  __shared__ float rq[64];
+  __shared__ float gqk[kD];          // gamma_q * gamma_k
+  __shared__ float red[4][64];
+  __shared__ float mxs[64], inv_den[64];
+  __shared__ int ncache;
+  __shared__ uint64_t bar_mma, bar_load;
+  __shared__ uint32_t tmem_base;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qw = warp & 3, half = warp >> 2;
+  const int bh = blockIdx.y, h = bh % p.H;
+  const int L = p.L, nblocks = (L + 63) / 64;
+  const int blk_begin = blockIdx.x * kBlocksPerCta, blk_end = min(nblocks, blk_begin + kBlocksPerCta);
+  const size_t tok0 = (size_t)bh * L;
+  const float sink = p.sink[h];
+  const float inv_sqrt_d = rsqrtf((float)kD);
+  const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+  uint8_t* KB = sm + PB_K;
+  uint8_t* VB = sm + PB_V;
+  const uint8_t* kbytes = reinterpret_cast<const uint8_t*>(p.k);
+  const uint8_t* vbytes = reinterpret_cast<const uint8_t*>(p.v);
+  const uint8_t* qbytes = reinterpret_cast<const uint8_t*>(p.q);
+
+  if (tid == 0) {
+    sm100::prefetch_tmap(&tm_q);
+    sm100::prefetch_tmap(&tm_k);
+    sm100::prefetch_tmap(&tm_v);
+    sm100::mbar_init(&bar_mma, 1);
+    sm100::mbar_init(&bar_load, 1);
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0) {
+    sm100::tmem_alloc(&tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  if (tid < kD) gqk[tid] = p.gamma_q[tid] * p.gamma_k[tid];
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t qh = sm100::smem_u32(sm + PB_H), ql = sm100::smem_u32(sm + PB_L);
+  uint32_t lphase = 0;
+  bool bad = false;
+
+  for (int blk = blk_begin; blk < blk_end && !bad; ++blk) {
+    const int b0 = 64 * blk, nb = min(64, L - b0);
+    if (tid == 0) {  // the block's raw k, v (rows 64..127) and q (the lo panel): six 64 x 64 boxes
+      sm100::mbar_arrive_expect_tx(&bar_load, 3 * kNP * 64 * 128);
+#pragma unroll
+      for (int pn = 0; pn < kNP; ++pn) {
+        sm100::tma_load_3d(KB + pn * kPanel + 64 * 128, &tm_k, &bar_load, 64 * pn, b0, bh);
+        sm100::tma_load_3d(VB + pn * kPanel + 64 * 128, &tm_v, &bar_load, 64 * pn, b0, bh);
+        sm100::tma_load_3d(sm + PB_QS + pn * kQPanel, &tm_q, &bar_load, 64 * pn, b0, bh);
+      }
+    }
+    if (tid < 64) crow[tid] = p.cidx[((size_t)bh * nblocks + blk) * 64 + tid];
+    __syncthreads();
+    // cache rows: 64 rows x (key, value) x 16 chunks of 16 bytes, gathered by token index; empty rows zero
+    for (int e = tid; e < 64 * 2 * 2 * kNP * 8 / 2; e += kTThreads) {
+      const int r = e >> 5, q = e & 31, which = q >> 4, cc = q & 15;
+      uint8_t* dst = (which ? VB : KB) + (cc / 8) * kPanel + sm100::sw128_chunk(r, cc % 8);
+      const int t = crow[r];
+      if (t >= 0) cp_async16_cg(dst, (which ? vbytes : kbytes) + ((tok0 + t) * kD + 8 * cc) * 2);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (blk + 1 < blk_end) {  // the next block's tiles and cache rows into L2, while this block is read
+      const size_t nt = tok0 + 64 * (blk + 1);
+      const uint32_t tile = (uint32_t)min(64, L - 64 * (blk + 1)) * kD * 2;
+      if (tid == 0) prefetch_l2_bulk(qbytes + nt * kD * 2, tile);
+      if (tid == 1) prefetch_l2_bulk(kbytes + nt * kD * 2, tile);
+      if (tid == 2) prefetch_l2_bulk(vbytes + nt * kD * 2, tile);
+      if (tid >= 64 && tid < 128) {
+        const int t = p.cidx[((size_t)bh * nblocks + blk + 1) * 64 + tid - 64];
+        if (t >= 0) {
+          prefetch_l2_bulk(kbytes + (tok0 + t) * kD * 2, kD * 2);
+          prefetch_l2_bulk(vbytes + (tok0 + t) * kD * 2, kD * 2);
+        }
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    {
+      int fail = 0;
+      if (tid == 0) {
+        int n = 0;
+        for (int r = 0; r < 64; ++r) n += crow[r] >= 0 ? 1 : 0;
+        ncache = n;
+        fail = !sm100::mbar_wait_bounded(&bar_load, lphase, kWaitCycles);
+      }
+      bad = __syncthreads_or(fail);
+      lphase ^= 1;
+      if (bad) break;
+    }
+
+    // ---------------------------------------------------------------- scales of k (cache and block rows), scaled q hi/lo
+    {
+      const int i = tid >> 2, part = tid & 3;   // row of each half, quarter of its 16 chunks
+      float kss_c = 0.f, kss = 0.f, qss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = 4 * part + u;             // chunk: elements 8 c .. 8 c + 7
+        const uint4 kc0 = *reinterpret_cast<const uint4*>(KB + (c / 8) * kPanel + sm100::sw128_chunk(i, c % 8));
+        const uint4 kc = *reinterpret_cast<const uint4*>(KB + (c / 8) * kPanel + sm100::sw128_chunk(64 + i, c % 8));
+        const uint4 qc = *reinterpret_cast<const uint4*>(sm + PB_QS + (c / 8) * kQPanel + sm100::sw128_chunk(i, c % 8));
+        const __nv_bfloat162* k0 = reinterpret_cast<const __nv_bfloat162*>(&kc0);
+        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kc);
+        const __nv_bfloat162* qh2 = reinterpret_cast<const __nv_bfloat162*>(&qc);
+        float qs[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 c0 = __bfloat1622float2(k0[e]), kf = __bfloat1622float2(kh[e]), qf = __bfloat1622float2(qh2[e]);
+          kss_c = fmaf(c0.x, c0.x, fmaf(c0.y, c0.y, kss_c));
+          kss = fmaf(kf.x, kf.x, fmaf(kf.y, kf.y, kss));
+          qss = fmaf(qf.x, qf.x, fmaf(qf.y, qf.y, qss));
+          qs[2 * e] = qf.x * gqk[8 * c + 2 * e];
+          qs[2 * e + 1] = qf.y * gqk[8 * c + 2 * e + 1];
+        }
+        store8_split(sm + PB_H, sm + PB_L, (c / 8) * kQPanel + sm100::sw128_chunk(i, c % 8), qs);
+      }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        kss_c += __shfl_xor_sync(0xffffffffu, kss_c, o);
+        kss += __shfl_xor_sync(0xffffffffu, kss, o);
+        qss += __shfl_xor_sync(0xffffffffu, qss, o);
+      }
+      if (part == 0) {
+        rk[i] = crow[i] >= 0 ? rsqrtf(kss_c / kD + 1e-6f) : 0.f;
+        rk[64 + i] = i < nb ? rsqrtf(kss / kD + 1e-6f) : 0.f;
+        rq[i] = rsqrtf(qss / kD + 1e-6f);
+      }
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- S^T = K [q o gamma]^T
+    {
+      int fail = 0;
+      if (tid == 0) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 64, false, false);
+        const uint32_t kb = sm100::smem_u32(KB);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t a = sm100::smem_desc(kb + (ks / 4) * kPanel + (ks % 4) * 32, 16, 1024);
+          const uint32_t boff = (ks / 4) * kQPanel + (ks % 4) * 32;
+          sm100::mma_bf16(tmem + T_S, a, sm100::smem_desc(qh + boff, 16, 1024), id, ks > 0);
+          sm100::mma_bf16(tmem + T_S, a, sm100::smem_desc(ql + boff, 16, 1024), id, true);
+        }
+        sm100::mma_commit(&bar_mma);
+        fail = !sm100::mbar_wait_bounded(&bar_mma, 0, kWaitCycles);
+      }
+      bad = __syncthreads_or(fail);
+      sm100::tc_fence_after();
+      if (bad) break;
+    }
+
+    // ---------------------------------------------------------------- softmax over the keys (lanes) of each query
+    const int j = 32 * qw + lane;             // key row
+    float x[32];
+    {
+      float s2[32];
+      sm100::tmem_ld32(tmem + t_lane + T_S + 32 * half, s2);
+      sm100::tmem_wait_ld();
+      const float kscale = rk[j] * inv_sqrt_d;
+      const int nc = ncache;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int t = 32 * half + u;
+        const bool vis = j < 64 ? j < nc : (j - 64 <= t && j - 64 < nb);
+        x[u] = vis ? s2[u] * kscale * rq[t] : -INFINITY;
+        s2[u] = x[u];
+      }
+      red[qw][32 * half + lane] = butterfly<0>(s2, lane);
+    }
+    __syncthreads();
+    if (tid < 64) mxs[tid] = fmaxf(fmaxf(fmaxf(red[0][tid], red[1][tid]), fmaxf(red[2][tid], red[3][tid])), sink);
+    __syncthreads();
+    {
+      float s2[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        x[u] = __expf(x[u] - mxs[32 * half + u]);  // exp(-inf) = 0 for hidden keys
+        s2[u] = x[u];
+      }
+      red[qw][32 * half + lane] = butterfly<1>(s2, lane);
+    }
+    __syncthreads();
+    if (tid < 64) inv_den[tid] = 1.f / (red[0][tid] + red[1][tid] + red[2][tid] + red[3][tid] + __expf(sink - mxs[tid]));
+    __syncthreads();
+    // P (key rows, query columns) as bf16 hi / lo over the query panels, which the S product no longer reads
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8) {
+      float pv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pv[e] = x[8 * q8 + e] * inv_den[32 * half + 8 * q8 + e];
+      store8_split(sm + PB_H, sm + PB_L, sm100::sw128_chunk(j, 4 * half + q8), pv);
+    }
+    sm100::fence_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+
+    // ---------------------------------------------------------------- O^T = V^T P
+    {
+      int fail = 0;
+      if (tid == 0) {
+        constexpr uint32_t id = sm100::idesc_bf16(128, 64, true, true);
+        const uint32_t vb = sm100::smem_u32(VB);
+#pragma unroll
+        for (int ks = 0; ks < kRows / 16; ++ks) {
+          const uint64_t a = sm100::smem_desc(vb + ks * 2048, kPanel, 1024);
+          sm100::mma_bf16(tmem + T_O, a, sm100::smem_desc(qh + ks * 2048, kPanel, 1024), id, ks > 0);
+          sm100::mma_bf16(tmem + T_O, a, sm100::smem_desc(ql + ks * 2048, kPanel, 1024), id, true);
+        }
+        sm100::mma_commit(&bar_mma);
+        fail = !sm100::mbar_wait_bounded(&bar_mma, 1, kWaitCycles);
+      }
+      bad = __syncthreads_or(fail);
+      sm100::tc_fence_after();
+      if (bad) break;
+    }
+    {
+      float o[32];
+      sm100::tmem_ld32(tmem + t_lane + T_O + 32 * half, o);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int t = 32 * half + u;
+        if (t < nb) p.o[(tok0 + b0 + t) * kD + j] = o[u];
+      }
+    }
+    // the next block's copies overwrite every buffer this one read: all reads done, also by the async proxy
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+  }
+  if (bad && tid == 0) raise_status(p.status, kStatusTimeout);
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) sm100::tmem_dealloc(tmem, kTmemCols);
+}
+
 }  // namespace
 
 bool hola_tc_supported(int dk, int dv, int in_dtype, int block) {
@@ -374,7 +701,20 @@ cudaError_t launch_hola_read_tc(const HolaArgs& p, int BH, cudaStream_t stream) 
   if (!make_bf16_tmap(&tq, p.q, BH, p.L, kD) || !make_bf16_tmap(&tk, p.k, BH, p.L, kD) ||
       !make_bf16_tmap(&tv, p.v, BH, p.L, kD))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(hola_read_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  cudaError_t e;
+  if (p.cidx != nullptr) {  // every block's cache first, then all blocks at once
+    if (p.w < 1 || p.w > 64) return cudaErrorInvalidValue;
+    hola_cache_select_kernel<<<BH, kSelThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(hola_read_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    const int nblocks = (p.L + 63) / 64;
+    hola_read_block_kernel<<<dim3((nblocks + kBlocksPerCta - 1) / kBlocksPerCta, BH), kTThreads, kPSmem, stream>>>(
+        tq, tk, tv, p);
+    return cudaGetLastError();
+  }
+  e = cudaFuncSetAttribute(hola_read_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   hola_read_tc_kernel<<<BH, kTThreads, kSmem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

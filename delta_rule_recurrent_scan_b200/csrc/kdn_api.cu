@@ -543,6 +543,15 @@ kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const vo
   return cuda_status(kdn::launch_delta_bwd(dims->dk, dims->dv, bw, st), "backward launch");
 }
 
+size_t kdn_hola_workspace_bytes(const kdn_dims* dims) {
+  if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
+  const int block = dims->chunk == 0 ? 64 : dims->chunk;
+  size_t n = kStatusBytes;
+  if (kdn::hola_tc_supported(dims->dk, dims->dv, dims->in_dtype, block))  // every block's cache indices
+    n += round256((size_t)dims->B * dims->H * ((dims->L + 63) / 64) * 64 * sizeof(int));
+  return n;
+}
+
 kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* m,
                                const float* gamma_q, const float* gamma_k, const float* sink, int w, float* o_cache,
                                int* cache_idx, void* workspace, size_t workspace_bytes, void* stream) {
@@ -573,6 +582,10 @@ kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* 
   }
   kdn::HolaArgs ha{q, k, v, dims->in_dtype, m, gamma_q, gamma_k, sink, o_cache, cache_idx, dims->H, dims->L, block, w,
                    reinterpret_cast<unsigned*>(workspace)};
+  // with room for every block's cache indices, the tensor-core path reads all blocks at once
+  if (kdn::hola_tc_supported(dims->dk, dims->dv, dims->in_dtype, block) &&
+      workspace_bytes >= kdn_hola_workspace_bytes(dims))
+    ha.cidx = reinterpret_cast<int*>(reinterpret_cast<char*>(workspace) + kStatusBytes);
   return cuda_status(kdn::launch_hola_read(dims->dk, dims->dv, ha, BH, st), "surprise-cache read launch");
 }
 

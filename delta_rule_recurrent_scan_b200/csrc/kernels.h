@@ -141,6 +141,9 @@ struct HolaArgs {
   int block;              // 16, 32 or 64
   int w;                  // 1..64
   unsigned* status;       // device status word (bounded-wait timeouts)
+  // [BH, ceil(L / 64), 64] scratch, or nullptr: the cache token indices each block reads (tensor-core path:
+  // every block's cache is chosen first, then all blocks are read in parallel)
+  int* cidx = nullptr;
 };
 
 // Segment-parallel scan (P segments per head): uncertainty maps and starts, start states, chaining.

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     L.kdn_scan_delta_backward.argtypes = [dims] + [vp] * 16 + [sz, vp]
     L.kdn_scan_delta_backward.restype = ctypes.c_int
+    L.kdn_hola_workspace_bytes.argtypes = [dims]
+    L.kdn_hola_workspace_bytes.restype = sz
     L.kdn_backward_workspace_bytes.argtypes = [i, dims]
     L.kdn_backward_workspace_bytes.restype = sz
     L.kdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
@@ -343,9 +345,10 @@ def hola_cache_read(q, k, v, m, gamma_q, gamma_k, sink, w=64, block=64, o=None, 
     if cache is None:
         cache = torch.empty(B, H, w, dtype=torch.int32, device=dev)
     _need(cache, "cache", (B, H, w), torch.int32, dev)
-    if workspace is None:
-        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
     dims = Dims(B, H, L, dk, dv, block, _DTYPES[q.dtype], KDN_F32)
+    if workspace is None:
+        need = int(lib().kdn_hola_workspace_bytes(ctypes.byref(dims)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     st = lib().kdn_hola_cache_read(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(m), _ptr(gamma_q),
                                    _ptr(gamma_k), _ptr(sink), int(w), _ptr(o), _ptr(cache), _ptr(workspace),
                                    workspace.numel(), _stream(stream))

@@ -202,11 +202,20 @@ KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_di
  * indices of the final cache, ascending, -1 for empty slots, or NULL.  The
  * state-read gate that mixes o_cache into the layer output is the caller's.
  * workspace: >= 256 bytes (the device status word, read with
- * kdn_read_device_status). */
+ * kdn_read_device_status).  For bf16 q, k, v with d_k = d_v = 128 and blocks of
+ * 64, a workspace of kdn_hola_workspace_bytes(dims) also holds the cache
+ * indices of every block: the cache each block reads is chosen first (one
+ * pass over m per head), then all blocks are read at once; with 256 bytes one
+ * CTA per head walks the blocks in order.  Both give the same result. */
 KDN_EXPORT kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v,
                                const float* m, const float* gamma_q, const float* gamma_k, const float* sink,
                                int w, float* o_cache, int* cache_idx, void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/* Bytes of device workspace for kdn_hola_cache_read's parallel form (256 for
+ * the status word, plus B*H*ceil(L/64)*64 int32 cache indices where the
+ * tensor-core path applies); 0 for invalid dims.  Pure host call. */
+KDN_EXPORT size_t kdn_hola_workspace_bytes(const kdn_dims* dims);
 
 /* kdn_scan_kalman_full for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a deployment variant.  Callers that must

@@ -95,3 +95,21 @@ def test_full_layer_sampled_heads_and_tokens():
     gq, gk, sink = _params(128, wl.H, 4)
     tokens = [0, 1, 63, 64, 65, 127, 128, 1000, 4095, 4096, 8190, 8191]
     _check(x, m, gq, gk, sink, 64, 64, TOL["bf16"], tokens=tokens, heads=[(0, 0), (7, 15)])
+
+
+@pytest.mark.parametrize("w,L", [(64, 300), (5, 700), (64, 64), (17, 1)])
+def test_parallel_read_equals_the_block_by_block_walk(w, L):
+    """With room for every block's cache indices the read runs all blocks at once; with the 256-byte status
+    workspace one CTA per head walks them in order.  Same cache indices, o equal to fp32 rounding."""
+    wl = WORKLOADS["gdn_d128"]
+    x = make_scan_inputs(wl, seed=5, device=DEV, B=2, H=3, L=L)
+    m = torch.rand(2, 3, L, device=DEV)
+    m[0, 1, : L // 2] = 0.5  # ties in m: the earlier token wins in both forms
+    gq, gk, sink = _params(128, 3, 2)
+    small = torch.empty(256, dtype=torch.uint8, device=DEV)
+    o_par, c_par = kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=w)
+    o_ser, c_ser = kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=w, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.equal(c_par, c_ser)
+    assert normwise_err(o_par, _np(o_ser)) < 1e-5
+    _check(x, m, gq, gk, sink, w, 64, TOL["bf16"])
