@@ -400,7 +400,9 @@ def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
     def fn():
         kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=cache_w, block=64, o=o, cache=cache)
     ms = time_device(fn, steps, warmup, dist_on)
-    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": steps}
+    # the cache choice and the block reads (bf16, d = 128); one block-by-block kernel elsewhere
+    per_call = 2 if w.dtype == "bf16" and w.dk == 128 and w.dv == 128 else 1
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": per_call * steps}
 
 
 def bench_backward(w, steps, warmup, dist_on, rank, world):
@@ -523,6 +525,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B of the workload (profiling runs)")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward of a gated-delta workload (profiling runs): one JSON line")
+    ap.add_argument("--cache-read-only", action="store_true",
+                    help="time only the surprise-cache read over a workload's shape (profiling runs): one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -548,6 +552,18 @@ def main():
 
     kdn.lib()  # fail loudly if the library is missing
     peak, peak_kind = measured_peaks()
+    if args.cache_read_only:
+        r = bench_hola(w, args.steps, args.warmup, dist_on, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "surprise-cache read tokens/s (w = 64, blocks of 64)", "value": r["value"],
+                              "unit": "tokens/s", "ms_per_step": r["ms"], "steps": args.steps,
+                              "warmup": args.warmup, "gpu_launches": r["launches"],
+                              "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk}}),
+                  flush=True)
+        if dist_on:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.backward_only:
         if w.variant != "delta":
             raise SystemExit("--backward-only needs a gated-delta workload")
