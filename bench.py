@@ -406,7 +406,8 @@ def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
 
 
 def bench_backward(w, steps, warmup, dist_on, rank, world):
-    """The gated delta rule backward over a layer (upstream dO and dm random; the start state zero)."""
+    """The backward over a layer (gated delta rule, or isotropic Kalman: the delta backward with the uncertainty
+    chain around it); upstream dO and dm random, start state zero."""
     from delta_rule_recurrent_scan_b200 import kdn
     x = make_scan_inputs(w, seed=rank, device="cuda")
     g = torch.Generator(device="cuda")
@@ -414,12 +415,17 @@ def bench_backward(w, steps, warmup, dist_on, rank, world):
     dO = torch.randn(w.B, w.H, w.L, w.dv, device="cuda", generator=g)
     dm = torch.randn(w.B, w.H, w.L, device="cuda", generator=g)
     dims = kdn.Dims(w.B, w.H, w.L, w.dk, w.dv, 0, kdn.KDN_BF16, kdn.KDN_F32, 0)
-    ws = torch.empty(int(kdn.lib().kdn_backward_workspace_bytes(0, dims)), dtype=torch.uint8, device="cuda")
+    iso = w.variant == "kalman_iso"
+    ws = torch.empty(int(kdn.lib().kdn_backward_workspace_bytes(3 if iso else 0, dims)), dtype=torch.uint8,
+                     device="cuda")
 
     def fn():
-        kdn.scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], dO, a=x["a"], dm=dm, workspace=ws)
+        if iso:
+            kdn.scan_kalman_iso_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
+        else:
+            kdn.scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], dO, a=x["a"], dm=dm, workspace=ws)
     ms = time_device(fn, steps, warmup, dist_on)
-    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": 2 * steps}
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": (4 if iso else 2) * steps}
 
 
 def backward_bytes(w, in_bytes=2) -> int:
@@ -565,8 +571,8 @@ def main():
             torch.distributed.destroy_process_group()
         return
     if args.backward_only:
-        if w.variant != "delta":
-            raise SystemExit("--backward-only needs a gated-delta workload")
+        if w.variant not in ("delta", "kalman_iso"):
+            raise SystemExit("--backward-only needs a gated-delta or isotropic-Kalman workload")
         r = bench_backward(w, args.steps, args.warmup, dist_on, rank, world)
         if rank == 0:
             print(json.dumps({"metric": "backward tokens/s (dq, dk, dv, dbeta, da, dS0)", "value": r["value"],
@@ -610,15 +616,17 @@ def main():
                      "roofline_frac": ab / (r["ms"] * 1e-3) / 1e9 / peak})
         del r
         torch.cuda.empty_cache()
-        bw = WORKLOADS["gdn_d128"]
-        r = bench_backward(bw, 2, 1, dist_on, rank, world)
-        also.append({"workload": "gdn_d128_backward", "variant": "delta backward (dq, dk, dv, dbeta, da, dS0)",
-                     "value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"],
-                     "roofline_frac": backward_bytes(bw) / (r["ms"] * 1e-3) / 1e9 / peak,
-                     "fp32_flop_frac": backward_flops(bw) / (r["ms"] * 1e-3) / 1e12 / FP32_CUDA_CORE_TFLOPS,
-                     "arith": "f32 CUDA cores"})
-        del r
-        torch.cuda.empty_cache()
+        for bname, bvariant in (("gdn_d128", "delta backward (dq, dk, dv, dbeta, da, dS0)"),
+                                ("kalman_iso_d128", "isotropic Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dc0)")):
+            bw = WORKLOADS[bname]
+            r = bench_backward(bw, 2, 3, dist_on, rank, world)
+            also.append({"workload": bname + "_backward", "variant": bvariant,
+                         "value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"],
+                         "roofline_frac": backward_bytes(bw) / (r["ms"] * 1e-3) / 1e9 / peak,
+                         "fp32_flop_frac": backward_flops(bw) / (r["ms"] * 1e-3) / 1e12 / FP32_CUDA_CORE_TFLOPS,
+                         "arith": "f32 CUDA cores"})
+            del r
+            torch.cuda.empty_cache()
         for name in DECODE:
             dw = WORKLOADS[name]
             r = bench_decode(dw, 64, 8, dist_on, rank, world)

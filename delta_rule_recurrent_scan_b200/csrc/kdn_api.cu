@@ -478,40 +478,24 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
 }
 
 size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
-  if (variant != KDN_DELTA || dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_ISO) return 0;
+  if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
   if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
-  const size_t BH = (size_t)dims->B * dims->H, DD = (size_t)dims->dk * dims->dv;
+  const size_t BH = (size_t)dims->B * dims->H, DD = (size_t)dims->dk * dims->dv, tok = BH * (size_t)dims->L;
   const size_t nck = ((size_t)dims->L + kdn::kDeltaBwdChunk - 1) / kdn::kDeltaBwdChunk;
-  return kStatusBytes + round256(BH * DD * 4) + round256(BH * nck * DD * 4) + round256(BH * (size_t)dims->L * 4);
+  size_t n = kStatusBytes + round256(BH * DD * 4) + round256(BH * nck * DD * 4) + round256(tok * 4);
+  // isotropic: beta, the uncertainty before every token, ||k||^2 and dbeta
+  if (variant == KDN_KALMAN_ISO) n += 4 * round256(tok * 4);
+  return n;
 }
 
-kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
-                                   const float* a, const float* S0, const float* dO, const float* dm, const float* dS_L,
-                                   float* dq, float* dk, float* dv, float* dbeta, float* da, float* dS0,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
-  KDN_TRY(check_dims(dims));
+// The gated-delta backward after validation, on the current device: ``ws`` holds the status word, then
+// the working state, the chunk-start checkpoints and the residual norms (kdn_backward_workspace_bytes).
+kdn_status delta_backward_run(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
+                              const float* a, const float* S0, const float* dO, const float* dm, const float* dS_L,
+                              float* dq, float* dk, float* dv, float* dbeta, float* da, float* dS0, void* workspace,
+                              cudaStream_t st) {
   const bool any = dims->L > 0;
-  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
-  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
-                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
-                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
-                         std::make_pair((const void*)dv, "dv")})
-    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
-  KDN_TRY(check_ptr(beta, "beta", 4, !any));
-  KDN_TRY(check_ptr(dbeta, "dbeta", 4, !any));
-  KDN_TRY(check_ptr(a, "a", 4, true));
-  KDN_TRY(check_ptr(da, "da", 4, true));
-  KDN_TRY(check_ptr(dm, "dm", 4, true));
-  KDN_TRY(check_ptr(S0, "S0", 16, true));
-  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
-  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
-  const size_t need = kdn_backward_workspace_bytes(KDN_DELTA, dims);
-  if (workspace_bytes < need)
-    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
-                                         std::to_string(need));
-  DeviceGuard guard;
-  KDN_TRY(use_device_of(dS0, guard));
-  cudaStream_t st = (cudaStream_t)stream;
   const size_t BH = (size_t)dims->B * dims->H, L = dims->L, DD = (size_t)dims->dk * dims->dv;
   const size_t nck = (L + kdn::kDeltaBwdChunk - 1) / kdn::kDeltaBwdChunk;
   char* ws = reinterpret_cast<char*>(workspace);
@@ -541,6 +525,95 @@ kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const vo
   kdn::DeltaBwdArgs bw{q, k, v, dims->in_dtype, beta, a, dO, dm, dS_L, ckpt, enorm, dq, dk, dv, dbeta, da, dS0,
                        (int)BH, (int)L};
   return cuda_status(kdn::launch_delta_bwd(dims->dk, dims->dv, bw, st), "backward launch");
+}
+
+kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
+                                   const float* a, const float* S0, const float* dO, const float* dm, const float* dS_L,
+                                   float* dq, float* dk, float* dv, float* dbeta, float* da, float* dS0,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  KDN_TRY(check_dims(dims));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
+  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
+                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
+                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
+                         std::make_pair((const void*)dv, "dv")})
+    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
+  KDN_TRY(check_ptr(beta, "beta", 4, !any));
+  KDN_TRY(check_ptr(dbeta, "dbeta", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(da, "da", 4, true));
+  KDN_TRY(check_ptr(dm, "dm", 4, true));
+  KDN_TRY(check_ptr(S0, "S0", 16, true));
+  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  const size_t need = kdn_backward_workspace_bytes(KDN_DELTA, dims);
+  if (workspace_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
+                                         std::to_string(need));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(dS0, guard));
+  cudaStream_t st = (cudaStream_t)stream;
+  return delta_backward_run(dims, q, k, v, beta, a, S0, dO, dm, dS_L, dq, dk, dv, dbeta, da, dS0, workspace, st);
+}
+
+kdn_status kdn_scan_kalman_iso_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                       const float* r, const float* a, const float* qn, float qn_scalar,
+                                       const float* S0, const float* c0, const float* dO, const float* dm,
+                                       const float* dS_L, const float* dc_L, float* dq, float* dk, float* dv,
+                                       float* dr, float* da, float* dqn, float* dS0, float* dc0, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  KDN_TRY(check_dims(dims));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
+  KDN_TRY(check_ptr(dc0, "dc0", 4, false));
+  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
+                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
+                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
+                         std::make_pair((const void*)dv, "dv")})
+    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
+  KDN_TRY(check_ptr(r, "r", 4, !any));
+  KDN_TRY(check_ptr(dr, "dr", 4, !any));
+  KDN_TRY(check_ptr(dqn, "dqn", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(da, "da", 4, true));
+  KDN_TRY(check_ptr(qn, "qn", 4, true));
+  KDN_TRY(check_ptr(dm, "dm", 4, true));
+  KDN_TRY(check_ptr(S0, "S0", 16, true));
+  KDN_TRY(check_ptr(c0, "c0", 4, true));
+  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
+  KDN_TRY(check_ptr(dc_L, "dc_L", 4, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  const size_t need = kdn_backward_workspace_bytes(KDN_KALMAN_ISO, dims);
+  if (workspace_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
+                                         std::to_string(need));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(dS0, guard));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BH = (size_t)dims->B * dims->H, tok = BH * (size_t)dims->L;
+  // the scalar side's arrays sit after the memory backward's part of the workspace
+  kdn_dims dd = *dims;
+  char* iso = reinterpret_cast<char*>(workspace) + kdn_backward_workspace_bytes(KDN_DELTA, &dd);
+  kdn::IsoBwdArgs ia{};
+  ia.k = k, ia.in_dtype = dims->in_dtype, ia.a = a, ia.r = r, ia.qn = qn, ia.qn_scalar = qn_scalar, ia.c0 = c0;
+  ia.beta = reinterpret_cast<float*>(iso);
+  ia.cprev = reinterpret_cast<float*>(iso + round256(tok * 4));
+  ia.knorm2 = reinterpret_cast<float*>(iso + 2 * round256(tok * 4));
+  float* dbeta = reinterpret_cast<float*>(iso + 3 * round256(tok * 4));
+  ia.dbeta = dbeta, ia.dc_L = dc_L, ia.dk = dk, ia.da = da, ia.dr = dr, ia.dqn = dqn, ia.dc0 = dc0;
+  ia.L = dims->L, ia.dk_dim = dims->dk;
+  if (any) KDN_TRY(cuda_status(kdn::launch_iso_forward(ia, (int)BH, st), "isotropic backward: forward chain launch"));
+  // the memory backward with beta_t as an input gives dq, dv, dS0, the key's memory terms, dbeta and the
+  // decay terms of da; the uncertainty chain then adds its key and gate terms
+  KDN_TRY(delta_backward_run(dims, q, k, v, ia.beta, a, S0, dO, dm, dS_L, dq, dk, dv, dbeta, da, dS0, workspace, st));
+  if (!any) {
+    if (dc_L != nullptr)
+      return cuda_status(cudaMemcpyAsync(dc0, dc_L, BH * 4, cudaMemcpyDeviceToDevice, st), "dc0 of an empty sequence");
+    return cuda_status(cudaMemsetAsync(dc0, 0, BH * 4, st), "dc0 of an empty sequence");
+  }
+  return cuda_status(kdn::launch_iso_backward(ia, (int)BH, st), "isotropic backward: uncertainty chain launch");
 }
 
 size_t kdn_hola_workspace_bytes(const kdn_dims* dims) {

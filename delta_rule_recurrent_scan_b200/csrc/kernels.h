@@ -54,6 +54,31 @@ struct DeltaBwdArgs {
 constexpr int kDeltaBwdChunk = 32;
 cudaError_t launch_delta_bwd(int dk, int dv, const DeltaBwdArgs& args, cudaStream_t stream);
 
+// Uncertainty side of the isotropic-Kalman backward (one warp per head).
+struct IsoBwdArgs {
+  const void* k;        // [BH, L, dk]
+  int in_dtype;
+  const float* a;       // [BH, L] or nullptr
+  const float* r;       // [BH, L]
+  const float* qn;      // [BH, L] or nullptr (qn_scalar)
+  float qn_scalar;
+  const float* c0;      // [BH] or nullptr (1)
+  float* beta;          // [BH, L] forward: beta_t
+  float* cprev;         // [BH, L] forward: c before token t
+  float* knorm2;        // [BH, L] forward: ||k_t||^2
+  const float* dbeta;   // [BH, L] backward: dLoss/dbeta_t from the memory backward
+  const float* dc_L;    // [BH] or nullptr: upstream gradient of the final c
+  float* dk;            // [BH, L, dk] in/out: the key terms are added
+  float* da;            // [BH, L] in/out or nullptr: the gate terms are added
+  float* dr;            // [BH, L] out
+  float* dqn;           // [BH, L] out
+  float* dc0;           // [BH] out
+  int L;
+  int dk_dim;           // d_k
+};
+cudaError_t launch_iso_forward(const IsoBwdArgs& args, int BH, cudaStream_t stream);
+cudaError_t launch_iso_backward(const IsoBwdArgs& args, int BH, cudaStream_t stream);
+
 // Sequence-parallel covariance side of the full-Kalman scan (chunks of 64 tokens): the covariance entering
 // every run of cps chunks, through the chunks' Riccati transfer matrices.
 struct RiccatiArgs {

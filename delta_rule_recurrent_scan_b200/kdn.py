@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_delta_backward.restype = ctypes.c_int
     L.kdn_hola_workspace_bytes.argtypes = [dims]
     L.kdn_hola_workspace_bytes.restype = sz
+    L.kdn_scan_kalman_iso_backward.argtypes = [dims, vp, vp, vp, vp, vp, vp, f] + [vp] * 14 + [vp, sz, vp]
+    L.kdn_scan_kalman_iso_backward.restype = ctypes.c_int
     L.kdn_backward_workspace_bytes.argtypes = [i, dims]
     L.kdn_backward_workspace_bytes.restype = sz
     L.kdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
@@ -227,6 +229,45 @@ def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None, 
                                        _ptr(out["dv"]), _ptr(out["dbeta"]), _ptr(out["da"]), _ptr(out["dS0"]),
                                        _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "kdn_scan_delta_backward")
+    return out
+
+
+def scan_kalman_iso_backward(q, k, v, r, dO, a=None, qn=None, S0=None, c0=None, dm=None, dS_L=None, dc_L=None,
+                             workspace=None, stream=None, want_da=True):
+    """Gradients of the isotropic Kalman scan for upstream dO (and dm, dS_L, dc_L).  Returns a dict with dq, dk,
+    dv, dr, da (None if not wanted), dqn (per token), dS0 and dc0, all fp32."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, L, d_k]")
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {q.dtype}")
+    _need(q, "q", (B, H, L, dk), q.dtype)
+    _need(k, "k", (B, H, L, dk), q.dtype, dev)
+    _need(v, "v", (B, H, L, dv), q.dtype, dev)
+    tok = (B, H, L)
+    _need(r, "r", tok, torch.float32, dev)
+    _need(dO, "dO", (B, H, L, dv), torch.float32, dev)
+    for name, t, shape in (("a", a, tok), ("dm", dm, tok), ("S0", S0, (B, H, dk, dv)), ("dS_L", dS_L, (B, H, dk, dv)),
+                           ("c0", c0, (B, H)), ("dc_L", dc_L, (B, H))):
+        if t is not None:
+            _need(t, name, shape, torch.float32, dev)
+    qn_t, qn_s = _qn_args(qn, tok, dev)
+    out = {"dq": torch.empty(B, H, L, dk, device=dev), "dk": torch.empty(B, H, L, dk, device=dev),
+           "dv": torch.empty(B, H, L, dv, device=dev), "dr": torch.empty(B, H, L, device=dev),
+           "da": torch.empty(B, H, L, device=dev) if want_da else None, "dqn": torch.empty(B, H, L, device=dev),
+           "dS0": torch.empty(B, H, dk, dv, device=dev), "dc0": torch.empty(B, H, device=dev)}
+    dims = Dims(B, H, L, dk, dv, 0, _DTYPES[q.dtype], KDN_F32, 0)
+    need = int(lib().kdn_backward_workspace_bytes(VARIANTS["kalman_iso"], ctypes.byref(dims)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib().kdn_scan_kalman_iso_backward(
+        ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(a), _ptr(qn_t), qn_s, _ptr(S0), _ptr(c0),
+        _ptr(dO), _ptr(dm), _ptr(dS_L), _ptr(dc_L), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+        _ptr(out["dr"]), _ptr(out["da"]), _ptr(out["dqn"]), _ptr(out["dS0"]), _ptr(out["dc0"]), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(st, "kdn_scan_kalman_iso_backward")
     return out
 
 

@@ -184,8 +184,28 @@ KDN_EXPORT kdn_status kdn_scan_delta_backward(const kdn_dims* dims, const void* 
                                               float* dbeta, float* da, float* dS0, void* workspace,
                                               size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace kdn_scan_delta_backward needs (variant KDN_DELTA;
- * 0 for other variants or invalid dims). */
+/* Backward of the isotropic Kalman scan (Kalman Delta Networks, Abstract:
+ * Isotropic KDN, one uncertainty scalar per head; the layers are trained end to
+ * end).  The forward is kdn_scan_kalman_iso's: c^- = a^2 c + Qn, the delta-rule
+ * write with beta_t = c^- / (c^- ||k_t||^2 + r_t), c = d_k c^- r / (d_k r +
+ * c^- ||k_t||^2).  For upstream dO (and optional dm, dS_L, dc_L [B,H]) it gives
+ * dq, dk, dv [B,H,L,d] fp32, dr, dqn [B,H,L] (dqn per token: its sum is the
+ * gradient of a scalar Qn), da [B,H,L] (optional), dS0 [B,H,d_k,d_v] and dc0
+ * [B,H].  r [B,H,L]; a, qn (else qn_scalar), S0 (else 0), c0 (else 1)
+ * optional.  Runs the uncertainty chain forward (one warp per head), the
+ * gated-delta backward with that beta (kdn_scan_delta_backward's kernels), and
+ * the uncertainty chain backwards, which adds its key and gate terms.
+ * workspace: kdn_backward_workspace_bytes(KDN_KALMAN_ISO, dims) bytes.
+ * Asynchronous on ``stream``. */
+KDN_EXPORT kdn_status kdn_scan_kalman_iso_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                                   const float* r, const float* a, const float* qn, float qn_scalar,
+                                                   const float* S0, const float* c0, const float* dO, const float* dm,
+                                                   const float* dS_L, const float* dc_L, float* dq, float* dk,
+                                                   float* dv, float* dr, float* da, float* dqn, float* dS0,
+                                                   float* dc0, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace the backward entry points need (KDN_DELTA or
+ * KDN_KALMAN_ISO; 0 for other variants or invalid dims). */
 KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims);
 
 /* Surprise-cache read (A Hippocampus for Linear Attention, sections 3.3-3.4,
