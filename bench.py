@@ -406,8 +406,8 @@ def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
 
 
 def bench_backward(w, steps, warmup, dist_on, rank, world):
-    """The backward over a layer (gated delta rule, or isotropic Kalman: the delta backward with the uncertainty
-    chain around it); upstream dO and dm random, start state zero."""
+    """The backward over a layer (gated delta rule; isotropic or diagonal Kalman: the memory backward with the
+    uncertainty chain around it); upstream dO and dm random, start state zero."""
     from delta_rule_recurrent_scan_b200 import kdn
     x = make_scan_inputs(w, seed=rank, device="cuda")
     g = torch.Generator(device="cuda")
@@ -415,17 +415,18 @@ def bench_backward(w, steps, warmup, dist_on, rank, world):
     dO = torch.randn(w.B, w.H, w.L, w.dv, device="cuda", generator=g)
     dm = torch.randn(w.B, w.H, w.L, device="cuda", generator=g)
     dims = kdn.Dims(w.B, w.H, w.L, w.dk, w.dv, 0, kdn.KDN_BF16, kdn.KDN_F32, 0)
-    iso = w.variant == "kalman_iso"
-    ws = torch.empty(int(kdn.lib().kdn_backward_workspace_bytes(3 if iso else 0, dims)), dtype=torch.uint8,
+    ws = torch.empty(int(kdn.lib().kdn_backward_workspace_bytes(kdn.VARIANTS[w.variant], dims)), dtype=torch.uint8,
                      device="cuda")
 
     def fn():
-        if iso:
+        if w.variant == "kalman_iso":
             kdn.scan_kalman_iso_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
+        elif w.variant == "kalman_diag":
+            kdn.scan_kalman_diag_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
         else:
             kdn.scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], dO, a=x["a"], dm=dm, workspace=ws)
     ms = time_device(fn, steps, warmup, dist_on)
-    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": (4 if iso else 2) * steps}
+    return {"ms": ms, "value": w.tokens * world / (ms * 1e-3), "launches": (2 if w.variant == "delta" else 4) * steps}
 
 
 def backward_bytes(w, in_bytes=2) -> int:
@@ -571,8 +572,8 @@ def main():
             torch.distributed.destroy_process_group()
         return
     if args.backward_only:
-        if w.variant not in ("delta", "kalman_iso"):
-            raise SystemExit("--backward-only needs a gated-delta or isotropic-Kalman workload")
+        if w.variant not in ("delta", "kalman_iso", "kalman_diag"):
+            raise SystemExit("--backward-only needs a gated-delta, isotropic or diagonal Kalman workload")
         r = bench_backward(w, args.steps, args.warmup, dist_on, rank, world)
         if rank == 0:
             print(json.dumps({"metric": "backward tokens/s (dq, dk, dv, dbeta, da, dS0)", "value": r["value"],
@@ -617,7 +618,8 @@ def main():
         del r
         torch.cuda.empty_cache()
         for bname, bvariant in (("gdn_d128", "delta backward (dq, dk, dv, dbeta, da, dS0)"),
-                                ("kalman_iso_d128", "isotropic Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dc0)")):
+                                ("kalman_iso_d128", "isotropic Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dc0)"),
+                                ("kalman_diag_d128", "diagonal Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dp0)")):
             bw = WORKLOADS[bname]
             r = bench_backward(bw, 2, 3, dist_on, rank, world)
             also.append({"workload": bname + "_backward", "variant": bvariant,

@@ -97,7 +97,7 @@ __device__ __forceinline__ void mm(float* C, int ldc, const float* A, int ai, in
 
 // Shared-memory layout of one CTA for JB value columns (floats; every row padded by one so that walks down
 // a column avoid bank conflicts).
-template <int DK, int JB>
+template <int DK, int JB, bool GEN>
 struct BwdSmem {
   static constexpr int LK = DK + 1, LJ = JB + 1, LC = kCB + 1;
   static constexpr int KC = 0;                    // K of the chunk [kCB][LK]
@@ -125,14 +125,17 @@ struct BwdSmem {
   static constexpr int DW = DN + kCB * LC;        // dW = dS E^T [DK][LC]
   static constexpr int VEC = DW + DK * LC;        // per-token vectors of kCB floats (see the kernel)
   static constexpr int NVEC = 12;
-  static constexpr int TOTAL = VEC + NVEC * kCB + 32;
+  static constexpr int GC = VEC + NVEC * kCB + 32; // general gains: the chunk's G [kCB][LK]
+  static constexpr int TOTAL = GC + (GEN ? kCB * LK : 0);
   static constexpr size_t BYTES = TOTAL * sizeof(float);
 };
 
-template <int DK, int DV>
+// GEN: the gains are given per token (g_t, a d_k vector: diagonal Kalman) instead of beta_t k_t, and dG is
+// written instead of dbeta (the key then carries no gain term).
+template <int DK, int DV, bool GEN>
 __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs p) {
   constexpr int JB = DV < kJB ? DV : kJB;
-  using Lay = BwdSmem<DK, JB>;
+  using Lay = BwdSmem<DK, JB, GEN>;
   constexpr int LK = Lay::LK, LJ = Lay::LJ, LC = Lay::LC, C = kCB, NT = kBwdThreads, NW = NT / 32;
   extern __shared__ float sm[];
   float* Kc = sm + Lay::KC;
@@ -166,7 +169,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
   float* vr = vec + 4 * C;     // r = A_C / A
   float* vdm = vec + 5 * C;    // dLoss/dm
   float* ven = vec + 6 * C;    // ||e|| (all columns, from the forward)
-  float* vkn = vec + 7 * C;    // ||k||
+  float* vkn = vec + 7 * C;    // ||k|| (||g|| for given gains)
+  float* Gc = sm + Lay::GC;    // given gains of the chunk (GEN)
   float* vdA = vec + 8 * C;    // dLoss/dA (this block's columns)
   float* vdr = vec + 9 * C;    // dLoss/dr
   float* vdb = vec + 10 * C;   // dbeta
@@ -194,6 +198,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       const size_t off = (tok0 + t0 + i) * DK + kk;
       Kc[i * LK + kk] = ok ? load_elem(p.k, off, p.in_dtype) : 0.f;
       Qc[i * LK + kk] = ok ? load_elem(p.q, off, p.in_dtype) : 0.f;
+      if (GEN) Gc[i * LK + kk] = ok ? p.gains[off] : 0.f;
     }
     for (int idx = tid; idx < C * JB; idx += NT) {
       const int i = idx / JB, j = idx % JB;
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       const size_t ti = tok0 + t0 + i;
       const float a = ok ? (p.a != nullptr ? p.a[ti] : 1.f) : 1.f;
       va[i] = a;
-      vb[i] = ok ? p.beta[ti] : 0.f;
+      vb[i] = GEN ? 1.f : (ok ? p.beta[ti] : 0.f);
       vdm[i] = ok && p.dm != nullptr ? p.dm[ti] : 0.f;
       ven[i] = ok ? p.enorm[ti] : 0.f;
       vdA[i] = 0.f, vdr[i] = 0.f, vdb[i] = 0.f;
@@ -245,8 +250,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       vr[lane] = sa;
     }
     for (int i = warp; i < C; i += NW) {
+      const float* rowv = GEN ? Gc : Kc;
       float sq = 0.f;
-      for (int kk = lane; kk < DK; kk += 32) sq = fmaf(Kc[i * LK + kk], Kc[i * LK + kk], sq);
+      for (int kk = lane; kk < DK; kk += 32) sq = fmaf(rowv[i * LK + kk], rowv[i * LK + kk], sq);
       sq = warp_sum(sq);
       if (lane == 0) vkn[i] = sqrtf(sq);
     }
@@ -256,8 +262,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       Gam[i * LC + j] = j <= i ? __expf(vell[i] - vell[j]) : 0.f;
     }
     // ------------------------------------------------------------------ forward recompute of the chunk
-    mm<C, C, DK, 4, 4>(KG, LC, Kc, LK, 1, Kc, 1, LK, 1.f, false);  // K K^T
-    mm<C, C, DK, 4, 4>(QG, LC, Qc, LK, 1, Kc, 1, LK, 1.f, false);  // Q K^T
+    mm<C, C, DK, 4, 4>(KG, LC, Kc, LK, 1, GEN ? Gc : Kc, 1, LK, 1.f, false);  // K K^T (K G^T)
+    mm<C, C, DK, 4, 4>(QG, LC, Qc, LK, 1, GEN ? Gc : Kc, 1, LK, 1.f, false);  // Q K^T (Q G^T)
     for (int idx = tid; idx < C * C; idx += NT) {
       const int i = idx / C, j = idx % C;
       const float kg = KG[i * LC + j] * vb[j], qg = QG[i * LC + j] * vb[j], g = Gam[i * LC + j];
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
     __syncthreads();
     mm<C, JB, C, 2, 2>(Ee, LJ, Tt, LC, 1, Rr, LJ, 1, 1.f, false);  // E = T R
     // ------------------------------------------------------------------ backward of the chunk
-    mm<C, JB, DK, 4, 4>(dE, LJ, Kc, LK, 1, dS, LJ, 1, 1.f, false);  // K dS
+    mm<C, JB, DK, 4, 4>(dE, LJ, GEN ? Gc : Kc, LK, 1, dS, LJ, 1, 1.f, false);  // K dS (G dS)
     {
       float acc = 0.f;  // dLoss/dA_C from S_C = A_C S0 + ...: this block's sum of dS o S0
       for (int idx = tid; idx < DK * JB; idx += NT) {
@@ -377,8 +383,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float km = Kc[m * LK + kq + KQ * e], qm = Qc[m * LK + kq + KQ * e];
-            dq[0][e] = fmaf(qa0, km, dq[0][e]), dq[1][e] = fmaf(qa1, km, dq[1][e]);
-            dk[0][e] = fmaf(ka0, km, dk[0][e]), dk[1][e] = fmaf(ka1, km, dk[1][e]);
+            const float gm = GEN ? Gc[m * LK + kq + KQ * e] : km;  // the gain row (beta_m enters through bm)
+            dq[0][e] = fmaf(qa0, gm, dq[0][e]), dq[1][e] = fmaf(qa1, gm, dq[1][e]);
+            dk[0][e] = fmaf(ka0, gm, dk[0][e]), dk[1][e] = fmaf(ka1, gm, dk[1][e]);
             dg[0][e] = fmaf(gk0, km, fmaf(gq0, qm, dg[0][e]));
             dg[1][e] = fmaf(gk1, km, fmaf(gq1, qm, dg[1][e]));
           }
@@ -394,9 +401,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
             const int kk = kq + KQ * e;
             const float ki = Kc[i * LK + kk];
             float g = fmaf(vr[i], dW[kk * LC + i], dg[a][e]);
-            g = fmaf(sur, ki, g);
-            dk[a][e] = fmaf(vb[i], g, dk[a][e]);
+            g = fmaf(sur, GEN ? Gc[i * LK + kk] : ki, g);  // the surprise along the gain's direction
+            if (!GEN) dk[a][e] = fmaf(vb[i], g, dk[a][e]);
             db[a] = fmaf(ki, g, db[a]);  // dbeta_i = k_i . dG_i
+            dg[a][e] = g;
           }
           if (i < n) {
 #pragma unroll
@@ -404,6 +412,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
               const size_t off = (tok0 + t0 + i) * DK + kq + KQ * e;
               atomicAdd(p.dq + off, dq[a][e]);
               atomicAdd(p.dk + off, dk[a][e]);
+              if (GEN) atomicAdd(p.dgain + off, dg[a][e]);
             }
           }
         }
@@ -417,10 +426,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
         if (lane % SEG == 0) atomicAdd(&vdb[i0], db[0]), atomicAdd(&vdb[i0 + 1], db[1]);
       }
     }
-    // dLoss/dr_j = beta_j sum_k K_jk dW_kj
+    // dLoss/dr_j = beta_j sum_k K_jk dW_kj (sum_k G_jk dW_kj for given gains)
     for (int j = warp; j < C; j += NW) {
+      const float* rowv = GEN ? Gc : Kc;
       float acc = 0.f;
-      for (int kk = lane; kk < DK; kk += 32) acc = fmaf(Kc[j * LK + kk], dW[kk * LC + j], acc);
+      for (int kk = lane; kk < DK; kk += 32) acc = fmaf(rowv[j * LK + kk], dW[kk * LC + j], acc);
       acc = warp_sum(acc);
       if (lane == 0) vdr[j] = vb[j] * acc;
     }
@@ -456,7 +466,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
       const float da = Aprev * sA + sH + gC * vh[t] + Aprev * gC * vmisc[0];
       if (t < n) {
         if (p.da != nullptr) atomicAdd(p.da + tok0 + t0 + t, da);
-        atomicAdd(p.dbeta + tok0 + t0 + t, vdb[t]);
+        if (!GEN) atomicAdd(p.dbeta + tok0 + t0 + t, vdb[t]);
       }
     }
     // ------------------------------------------------------------------ dS0 = A_C dS + Q^T dQS + K^T dKS, in place
@@ -503,10 +513,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
 template <int DK, int DV>
 cudaError_t launch_delta_bwd_typed(const DeltaBwdArgs& args, cudaStream_t stream) {
   constexpr int JB = DV < kJB ? DV : kJB;
-  const size_t smem = BwdSmem<DK, JB>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(delta_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const dim3 grid(args.BH, DV / JB);
+  if (args.gains != nullptr) {
+    const size_t smem = BwdSmem<DK, JB, true>::BYTES;
+    cudaError_t e =
+        cudaFuncSetAttribute(delta_bwd_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    delta_bwd_kernel<DK, DV, true><<<grid, kBwdThreads, smem, stream>>>(args);
+    return cudaGetLastError();
+  }
+  const size_t smem = BwdSmem<DK, JB, false>::BYTES;
+  cudaError_t e =
+      cudaFuncSetAttribute(delta_bwd_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  delta_bwd_kernel<DK, DV><<<dim3(args.BH, DV / JB), kBwdThreads, smem, stream>>>(args);
+  delta_bwd_kernel<DK, DV, false><<<grid, kBwdThreads, smem, stream>>>(args);
   return cudaGetLastError();
 }
 

@@ -478,7 +478,7 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
 }
 
 size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
-  if (variant != KDN_DELTA && variant != KDN_KALMAN_ISO) return 0;
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_ISO && variant != KDN_KALMAN_DIAG) return 0;
   if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
   if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
   const size_t BH = (size_t)dims->B * dims->H, DD = (size_t)dims->dk * dims->dv, tok = BH * (size_t)dims->L;
@@ -486,6 +486,8 @@ size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
   size_t n = kStatusBytes + round256(BH * DD * 4) + round256(BH * nck * DD * 4) + round256(tok * 4);
   // isotropic: beta, the uncertainty before every token, ||k||^2 and dbeta
   if (variant == KDN_KALMAN_ISO) n += 4 * round256(tok * 4);
+  // diagonal: the gains, p before every token and dG (d_k values per token each)
+  if (variant == KDN_KALMAN_DIAG) n += 3 * round256(tok * dims->dk * 4);
   return n;
 }
 
@@ -494,7 +496,8 @@ size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
 kdn_status delta_backward_run(const kdn_dims* dims, const void* q, const void* k, const void* v, const float* beta,
                               const float* a, const float* S0, const float* dO, const float* dm, const float* dS_L,
                               float* dq, float* dk, float* dv, float* dbeta, float* da, float* dS0, void* workspace,
-                              cudaStream_t st) {
+                              cudaStream_t st, const float* gains = nullptr, float* dgain = nullptr) {
+  // gains != nullptr: the per-token gains are given (diagonal Kalman) and dG goes to dgain; beta, dbeta unused
   const bool any = dims->L > 0;
   const size_t BH = (size_t)dims->B * dims->H, L = dims->L, DD = (size_t)dims->dk * dims->dv;
   const size_t nck = (L + kdn::kDeltaBwdChunk - 1) / kdn::kDeltaBwdChunk;
@@ -512,18 +515,21 @@ kdn_status delta_backward_run(const kdn_dims* dims, const void* q, const void* k
   // the sums over value-column blocks accumulate into zeroed outputs
   e = cudaMemsetAsync(dq, 0, BH * L * dims->dk * 4, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, BH * L * dims->dk * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, BH * L * 4, st);
+  if (e == cudaSuccess)
+    e = gains != nullptr ? cudaMemsetAsync(dgain, 0, BH * L * dims->dk * 4, st) : cudaMemsetAsync(dbeta, 0, BH * L * 4, st);
   if (e == cudaSuccess && da != nullptr) e = cudaMemsetAsync(da, 0, BH * L * 4, st);
   if (e == cudaSuccess)
     e = S0 != nullptr ? cudaMemcpyAsync(S_work, S0, BH * DD * 4, cudaMemcpyDeviceToDevice, st)
                       : cudaMemsetAsync(S_work, 0, BH * DD * 4, st);
   if (e != cudaSuccess) return cuda_status(e, "preparing the backward buffers");
   // forward again, keeping the state at every chunk start and the residual norms
-  kdn::SeqScanArgs fw{q, k, v, dims->in_dtype, KDN_F32, beta, a, nullptr, S_work, nullptr, nullptr, (int)BH, (int)L};
+  kdn::SeqScanArgs fw{q, k, v, dims->in_dtype, KDN_F32, gains != nullptr ? nullptr : beta, a, gains, S_work, nullptr,
+                      nullptr, (int)BH, (int)L};
   fw.S_ckpt = ckpt, fw.enorm = enorm, fw.ckpt_every = kdn::kDeltaBwdChunk;
   KDN_TRY(cuda_status(kdn::launch_seq_scan(dims->dk, dims->dv, fw, st), "backward: forward checkpoints launch"));
   kdn::DeltaBwdArgs bw{q, k, v, dims->in_dtype, beta, a, dO, dm, dS_L, ckpt, enorm, dq, dk, dv, dbeta, da, dS0,
                        (int)BH, (int)L};
+  bw.gains = gains, bw.dgain = dgain;
   return cuda_status(kdn::launch_delta_bwd(dims->dk, dims->dv, bw, st), "backward launch");
 }
 
@@ -614,6 +620,66 @@ kdn_status kdn_scan_kalman_iso_backward(const kdn_dims* dims, const void* q, con
     return cuda_status(cudaMemsetAsync(dc0, 0, BH * 4, st), "dc0 of an empty sequence");
   }
   return cuda_status(kdn::launch_iso_backward(ia, (int)BH, st), "isotropic backward: uncertainty chain launch");
+}
+
+kdn_status kdn_scan_kalman_diag_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                        const float* r, const float* a, const float* qn, float qn_scalar,
+                                        const float* S0, const float* p0, const float* dO, const float* dm,
+                                        const float* dS_L, const float* dp_L, float* dq, float* dk, float* dv,
+                                        float* dr, float* da, float* dqn, float* dS0, float* dp0, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  KDN_TRY(check_dims(dims));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
+  KDN_TRY(check_ptr(dp0, "dp0", 4, false));
+  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
+                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
+                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
+                         std::make_pair((const void*)dv, "dv")})
+    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
+  KDN_TRY(check_ptr(r, "r", 4, !any));
+  KDN_TRY(check_ptr(dr, "dr", 4, !any));
+  KDN_TRY(check_ptr(dqn, "dqn", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(da, "da", 4, true));
+  KDN_TRY(check_ptr(qn, "qn", 4, true));
+  KDN_TRY(check_ptr(dm, "dm", 4, true));
+  KDN_TRY(check_ptr(S0, "S0", 16, true));
+  KDN_TRY(check_ptr(p0, "p0", 4, true));
+  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
+  KDN_TRY(check_ptr(dp_L, "dp_L", 4, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  const size_t need = kdn_backward_workspace_bytes(KDN_KALMAN_DIAG, dims);
+  if (workspace_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
+                                         std::to_string(need));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(dS0, guard));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BH = (size_t)dims->B * dims->H, tok = BH * (size_t)dims->L;
+  kdn_dims dd = *dims;
+  char* side = reinterpret_cast<char*>(workspace) + kdn_backward_workspace_bytes(KDN_DELTA, &dd);
+  kdn::DiagBwdArgs da_args{};
+  da_args.k = k, da_args.in_dtype = dims->in_dtype, da_args.a = a, da_args.r = r, da_args.qn = qn;
+  da_args.qn_scalar = qn_scalar, da_args.p0 = p0;
+  da_args.gains = reinterpret_cast<float*>(side);
+  da_args.pprev = reinterpret_cast<float*>(side + round256(tok * dims->dk * 4));
+  float* dgain = reinterpret_cast<float*>(side + 2 * round256(tok * dims->dk * 4));
+  da_args.dgain = dgain, da_args.dp_L = dp_L, da_args.dk = dk, da_args.da = da, da_args.dr = dr;
+  da_args.dqn = dqn, da_args.dp0 = dp0, da_args.L = dims->L, da_args.dk_dim = dims->dk;
+  if (any) KDN_TRY(cuda_status(kdn::launch_diag_forward(da_args, (int)BH, st), "diagonal backward: forward chain launch"));
+  // the memory backward with the gains as inputs gives dq, dv, dS0, the key's memory terms, dG and the decay
+  // terms of da; the uncertainty chain then adds its key and gate terms
+  KDN_TRY(delta_backward_run(dims, q, k, v, nullptr, a, S0, dO, dm, dS_L, dq, dk, dv, nullptr, da, dS0, workspace, st,
+                             da_args.gains, dgain));
+  if (!any) {
+    if (dp_L != nullptr)
+      return cuda_status(cudaMemcpyAsync(dp0, dp_L, BH * dims->dk * 4, cudaMemcpyDeviceToDevice, st),
+                         "dp0 of an empty sequence");
+    return cuda_status(cudaMemsetAsync(dp0, 0, BH * dims->dk * 4, st), "dp0 of an empty sequence");
+  }
+  return cuda_status(kdn::launch_diag_backward(da_args, (int)BH, st), "diagonal backward: uncertainty chain launch");
 }
 
 size_t kdn_hola_workspace_bytes(const kdn_dims* dims) {

@@ -50,6 +50,10 @@ struct DeltaBwdArgs {
   float* dS0;           // [BH, dk, dv]
   int BH;
   int L;
+  // given gains instead of beta_t k_t (diagonal Kalman): gains [BH, L, dk] in, dgain [BH, L, dk] (zeroed) out;
+  // beta and dbeta are then unused
+  const float* gains = nullptr;
+  float* dgain = nullptr;
 };
 constexpr int kDeltaBwdChunk = 32;
 cudaError_t launch_delta_bwd(int dk, int dv, const DeltaBwdArgs& args, cudaStream_t stream);
@@ -78,6 +82,30 @@ struct IsoBwdArgs {
 };
 cudaError_t launch_iso_forward(const IsoBwdArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_iso_backward(const IsoBwdArgs& args, int BH, cudaStream_t stream);
+
+// Uncertainty side of the diagonal-Kalman backward (one warp per head, lanes over the coordinates).
+struct DiagBwdArgs {
+  const void* k;        // [BH, L, dk]
+  int in_dtype;
+  const float* a;       // [BH, L] or nullptr
+  const float* r;       // [BH, L]
+  const float* qn;      // [BH, L] or nullptr (qn_scalar)
+  float qn_scalar;
+  const float* p0;      // [BH, dk] or nullptr (1)
+  float* gains;         // [BH, L, dk] forward: g_t = p^- o k / s
+  float* pprev;         // [BH, L, dk] forward: p before token t
+  const float* dgain;   // [BH, L, dk] backward: dLoss/dg_t from the memory backward
+  const float* dp_L;    // [BH, dk] or nullptr: upstream gradient of the final p
+  float* dk;            // [BH, L, dk] in/out: the key terms are added
+  float* da;            // [BH, L] in/out or nullptr: the gate terms are added
+  float* dr;            // [BH, L] out
+  float* dqn;           // [BH, L] out
+  float* dp0;           // [BH, dk] out
+  int L;
+  int dk_dim;           // d_k
+};
+cudaError_t launch_diag_forward(const DiagBwdArgs& args, int BH, cudaStream_t stream);
+cudaError_t launch_diag_backward(const DiagBwdArgs& args, int BH, cudaStream_t stream);
 
 // Sequence-parallel covariance side of the full-Kalman scan (chunks of 64 tokens): the covariance entering
 // every run of cps chunks, through the chunks' Riccati transfer matrices.

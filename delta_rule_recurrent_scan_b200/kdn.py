@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_hola_workspace_bytes.restype = sz
     L.kdn_scan_kalman_iso_backward.argtypes = [dims, vp, vp, vp, vp, vp, vp, f] + [vp] * 14 + [vp, sz, vp]
     L.kdn_scan_kalman_iso_backward.restype = ctypes.c_int
+    L.kdn_scan_kalman_diag_backward.argtypes = [dims, vp, vp, vp, vp, vp, vp, f] + [vp] * 14 + [vp, sz, vp]
+    L.kdn_scan_kalman_diag_backward.restype = ctypes.c_int
     L.kdn_backward_workspace_bytes.argtypes = [i, dims]
     L.kdn_backward_workspace_bytes.restype = sz
     L.kdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
@@ -232,10 +234,23 @@ def scan_delta_backward(q, k, v, beta, dO, a=None, S0=None, dm=None, dS_L=None, 
     return out
 
 
+def scan_kalman_diag_backward(q, k, v, r, dO, a=None, qn=None, S0=None, p0=None, dm=None, dS_L=None, dp_L=None,
+                              workspace=None, stream=None, want_da=True):
+    """Gradients of the diagonal Kalman scan for upstream dO (and dm, dS_L, dp_L).  Returns a dict with dq, dk,
+    dv, dr, da (None if not wanted), dqn (per token), dS0 and dp0, all fp32."""
+    return _kalman_backward("kalman_diag", q, k, v, r, dO, a, qn, S0, p0, dm, dS_L, dp_L, workspace, stream, want_da)
+
+
 def scan_kalman_iso_backward(q, k, v, r, dO, a=None, qn=None, S0=None, c0=None, dm=None, dS_L=None, dc_L=None,
                              workspace=None, stream=None, want_da=True):
     """Gradients of the isotropic Kalman scan for upstream dO (and dm, dS_L, dc_L).  Returns a dict with dq, dk,
     dv, dr, da (None if not wanted), dqn (per token), dS0 and dc0, all fp32."""
+    return _kalman_backward("kalman_iso", q, k, v, r, dO, a, qn, S0, c0, dm, dS_L, dc_L, workspace, stream, want_da)
+
+
+def _kalman_backward(variant, q, k, v, r, dO, a, qn, S0, u0, dm, dS_L, du_L, workspace, stream, want_da):
+    """The uncertainty-side backward shared by the isotropic (u = c, one per head) and diagonal (u = p, one per
+    coordinate) variants."""
     if q.dim() != 4:
         raise ValueError("q must be [B, H, L, d_k]")
     B, H, L, dk = q.shape
@@ -249,25 +264,27 @@ def scan_kalman_iso_backward(q, k, v, r, dO, a=None, qn=None, S0=None, c0=None, 
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, dev)
     _need(dO, "dO", (B, H, L, dv), torch.float32, dev)
+    ushape = (B, H) if variant == "kalman_iso" else (B, H, dk)
+    uname = "c" if variant == "kalman_iso" else "p"
     for name, t, shape in (("a", a, tok), ("dm", dm, tok), ("S0", S0, (B, H, dk, dv)), ("dS_L", dS_L, (B, H, dk, dv)),
-                           ("c0", c0, (B, H)), ("dc_L", dc_L, (B, H))):
+                           (uname + "0", u0, ushape), ("d" + uname + "_L", du_L, ushape)):
         if t is not None:
             _need(t, name, shape, torch.float32, dev)
     qn_t, qn_s = _qn_args(qn, tok, dev)
     out = {"dq": torch.empty(B, H, L, dk, device=dev), "dk": torch.empty(B, H, L, dk, device=dev),
            "dv": torch.empty(B, H, L, dv, device=dev), "dr": torch.empty(B, H, L, device=dev),
            "da": torch.empty(B, H, L, device=dev) if want_da else None, "dqn": torch.empty(B, H, L, device=dev),
-           "dS0": torch.empty(B, H, dk, dv, device=dev), "dc0": torch.empty(B, H, device=dev)}
+           "dS0": torch.empty(B, H, dk, dv, device=dev), "d" + uname + "0": torch.empty(*ushape, device=dev)}
     dims = Dims(B, H, L, dk, dv, 0, _DTYPES[q.dtype], KDN_F32, 0)
-    need = int(lib().kdn_backward_workspace_bytes(VARIANTS["kalman_iso"], ctypes.byref(dims)))
+    need = int(lib().kdn_backward_workspace_bytes(VARIANTS[variant], ctypes.byref(dims)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    st = lib().kdn_scan_kalman_iso_backward(
-        ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(a), _ptr(qn_t), qn_s, _ptr(S0), _ptr(c0),
-        _ptr(dO), _ptr(dm), _ptr(dS_L), _ptr(dc_L), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
-        _ptr(out["dr"]), _ptr(out["da"]), _ptr(out["dqn"]), _ptr(out["dS0"]), _ptr(out["dc0"]), _ptr(workspace),
-        workspace.numel(), _stream(stream))
-    _check(st, "kdn_scan_kalman_iso_backward")
+    fn = lib().kdn_scan_kalman_iso_backward if variant == "kalman_iso" else lib().kdn_scan_kalman_diag_backward
+    st = fn(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(a), _ptr(qn_t), qn_s, _ptr(S0), _ptr(u0),
+            _ptr(dO), _ptr(dm), _ptr(dS_L), _ptr(du_L), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+            _ptr(out["dr"]), _ptr(out["da"]), _ptr(out["dqn"]), _ptr(out["dS0"]), _ptr(out["d" + uname + "0"]),
+            _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "kdn_scan_" + variant + "_backward")
     return out
 
 

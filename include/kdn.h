@@ -204,8 +204,26 @@ KDN_EXPORT kdn_status kdn_scan_kalman_iso_backward(const kdn_dims* dims, const v
                                                    float* dv, float* dr, float* da, float* dqn, float* dS0,
                                                    float* dc0, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace the backward entry points need (KDN_DELTA or
- * KDN_KALMAN_ISO; 0 for other variants or invalid dims). */
+/* Backward of the diagonal-Kalman scan (Kalman Delta Networks, Abstract:
+ * mean-field variational Kalman with a diagonal covariance; the layers are
+ * trained end to end).  The forward is kdn_scan_kalman_diag's: p^- = a^2 p + Qn,
+ * s = sum_i p^-_i k_i^2 + r, gain g = p^- o k / s, p = p^- r / (r + p^- o k^2)
+ * per coordinate, the delta-rule memory write with that gain.  Same inputs and
+ * outputs as kdn_scan_kalman_iso_backward with p0, dp_L, dp0 [B,H,d_k] in place
+ * of c0, dc_L, dc0.  Runs the variance chain forward (one warp per head,
+ * storing the gains and the variances), the memory backward with the gains as
+ * inputs (its kernels write dG), and the variance chain backwards, which adds
+ * its key and gate terms.  workspace: kdn_backward_workspace_bytes(
+ * KDN_KALMAN_DIAG, dims) bytes.  Asynchronous on ``stream``. */
+KDN_EXPORT kdn_status kdn_scan_kalman_diag_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                                    const float* r, const float* a, const float* qn, float qn_scalar,
+                                                    const float* S0, const float* p0, const float* dO, const float* dm,
+                                                    const float* dS_L, const float* dp_L, float* dq, float* dk,
+                                                    float* dv, float* dr, float* da, float* dqn, float* dS0,
+                                                    float* dp0, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace the backward entry points need (KDN_DELTA,
+ * KDN_KALMAN_ISO or KDN_KALMAN_DIAG; 0 for full Kalman or invalid dims). */
 KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims);
 
 /* Surprise-cache read (A Hippocampus for Linear Attention, sections 3.3-3.4,

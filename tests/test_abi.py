@@ -114,10 +114,11 @@ def test_backward_host_validation(L):
     n = L.kdn_backward_workspace_bytes(0, ctypes.byref(d))
     # status word + working state + a state per 32-token chunk + one norm per token
     assert n >= 256 + 6 * 64 * 32 * 4 * (1 + 4) + 6 * 100 * 4
-    for variant in (1, 2):
-        assert L.kdn_backward_workspace_bytes(variant, ctypes.byref(d)) == 0
+    assert L.kdn_backward_workspace_bytes(2, ctypes.byref(d)) == 0  # full Kalman has no CUDA backward
     # isotropic: the delta backward's part plus beta, the uncertainty before every token, ||k||^2 and dbeta
     assert L.kdn_backward_workspace_bytes(3, ctypes.byref(d)) >= n + 4 * 6 * 100 * 4
+    # diagonal: plus the gains, the variances before every token and dG
+    assert L.kdn_backward_workspace_bytes(1, ctypes.byref(d)) >= n + 3 * 6 * 100 * 64 * 4
     assert L.kdn_scan_delta_backward(None, *([None] * 15), None, 0, None) == kdn.KDN_ERR_INVALID_ARG
     # every output pointer is checked before anything is enqueued
     assert L.kdn_scan_delta_backward(ctypes.byref(d), *([None] * 15), None, 0, None) == kdn.KDN_ERR_INVALID_ARG
@@ -139,3 +140,11 @@ def test_hola_workspace_covers_every_block_on_the_tensor_core_path(L):
     assert L.kdn_hola_workspace_bytes(ctypes.byref(tc)) >= 256 + 6 * 5 * 64 * 4
     assert L.kdn_hola_workspace_bytes(ctypes.byref(other)) == 256
     assert L.kdn_hola_workspace_bytes(None) == 0
+
+
+def test_diag_backward_host_validation(L):
+    d = kdn.Dims(1, 2, 50, 32, 32, 0, kdn.KDN_BF16, kdn.KDN_F32)
+    args = [None] * 6 + [0.0] + [None] * 14 + [None, 0, None]
+    assert L.kdn_scan_kalman_diag_backward(None, *args) == kdn.KDN_ERR_INVALID_ARG
+    assert L.kdn_scan_kalman_diag_backward(ctypes.byref(d), *args) == kdn.KDN_ERR_INVALID_ARG
+    assert b"dS0" in L.kdn_last_error()
