@@ -576,7 +576,7 @@ def main():
             raise SystemExit("--backward-only needs a gated-delta, isotropic or diagonal Kalman workload")
         r = bench_backward(w, args.steps, args.warmup, dist_on, rank, world)
         if rank == 0:
-            print(json.dumps({"metric": "backward tokens/s (dq, dk, dv, dbeta, da, dS0)", "value": r["value"],
+            print(json.dumps({"metric": f"{w.variant} backward tokens/s (every input gradient)", "value": r["value"],
                               "unit": "tokens/s", "ms_per_step": r["ms"], "steps": args.steps,
                               "warmup": args.warmup, "gpu_launches": r["launches"],
                               "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk}}),
