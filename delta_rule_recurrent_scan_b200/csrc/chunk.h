@@ -19,7 +19,8 @@ struct ChunkArgs {
   float qn_scalar;
   float* S;
   float* P;           // full: [BH, dk, dk]; diagonal: p [BH, dk]
-  void* o;
+  int state_cols;     // columns of a state row: 0 = d_v; 2 d_v = 128 runs the d = 64 chunk kernel on [S | M]
+  void* o;            // or nullptr (no read-out)
   float* m;
   int out_dtype;
   int BH;
@@ -39,8 +40,10 @@ cudaError_t launch_kalman_pside(int d, const void* k, const float* a, const floa
                                 float qn_scalar, float* P, float* gains, unsigned* status, int BH, int L,
                                 cudaStream_t stream, const float* P_starts = nullptr, int cps = 0);
 
-// Warp-specialised chunk kernel for d_k = d_v = 128 (preparation of chunk c + 1 beside the state chain
-// of chunk c).  ``gains``: full-Kalman per-token gains [BH, L, 128] fp32, else unused.
+// Warp-specialised chunk kernel for d_k = d_v = 64 or 128 (preparation of chunk c + 1 beside the state
+// chain of chunk c).  ``gains``: full-Kalman per-token gains [BH, L, d] fp32, else unused.  At d = 64,
+// args.state_cols = 128 carries a [d, 2 d] state [S | M]: the extra columns see zero values (the map's
+// linear part), and o may be nullptr.
 cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& dims, const ChunkArgs& args, const float* gains,
                             cudaStream_t stream);
 

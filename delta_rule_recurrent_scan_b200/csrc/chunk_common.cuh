@@ -60,11 +60,7 @@ __device__ __forceinline__ void load8_bf16(const uint8_t* base, uint32_t off, fl
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-__device__ __forceinline__ void named_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
-// Sum over the 8 consecutive lanes that share a token.
 // Named barrier over ``count`` threads that also ORs a predicate across them.
 __device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
   uint32_t r;
@@ -79,6 +75,7 @@ __device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
   return r != 0;
 }
 
+// Sum over the 8 consecutive lanes that share a token.
 __device__ __forceinline__ float oct_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);
   x += __shfl_xor_sync(0xffffffffu, x, 2);

@@ -1,4 +1,4 @@
-// Warp-specialised chunked scan for d_k = d_v = 128 on the sm_100a tensor cores.
+// Warp-specialised chunked scan for d_k = d_v = 64 or 128 on the sm_100a tensor cores.
 //
 // The chunk algebra is the generalised WY / UT form of the token recurrence
 // S_t = a_t S_{t-1} + g_t e_t^T, e_t = v_t - a_t S_{t-1}^T k_t (A Hippocampus for
@@ -31,9 +31,13 @@
 // product is the row-major [K; Q] G^T.
 // fp32 state master and accumulators in TMEM.  Every tensor-core operand is fp16: K and Q are
 // converted from bf16 in shared memory when their tile lands (exact in fp16's normal range), the fp32
-// operands (state, (K S0), innovations, gains, T, Attn) are rounded to fp16 once.  A float64 emulation of these
-// roundings over 8192-token layers stays below 6e-4 normwise against the exact scan, inside the 3e-3
-// budget for bf16 inputs, while it halves the tensor work and the conversions of the bf16 hi/lo form.
+// operands (state, (K S0), innovations, gains in the state product, T, Attn) are rounded to fp16 once.  A
+// float64 emulation of these roundings over 8192-token layers stays below 6e-4 normwise against the exact
+// scan, inside the 3e-3 budget for bf16 inputs, while it halves the tensor work and the conversions of the
+// bf16 hi/lo form.  The Kalman gains enter [K; Q] G^T as an fp16 hi/lo pair (two products): a read-out
+// q_t . g_s that nearly cancels would otherwise carry the gain's rounding relative to |q| |g| (a 2 %
+// error on one single-token head at d = 64); with the pair, Attn and N are rounded relative to themselves.
+// For the delta-like variants G = K, exact in fp16.
 #include <cuda.h>
 
 #include "chunk.h"
@@ -75,13 +79,13 @@ struct WsLayout {
   static constexpr int V_PANEL = 64 * 128;
   static constexpr int V_BYTES = NP * V_PANEL;
   static constexpr int G_PANEL = 64 * 128;
-  static constexpr int G_HALF = delta_like(VAR) ? 0 : NP * G_PANEL;  // fp16 gains of one slot (first half)
+  static constexpr int G_HALF = delta_like(VAR) ? 0 : NP * G_PANEL;  // fp16 gains of one slot: hi, then lo
   static constexpr int TAT_HALF = 128 * 128;             // [T; Attn]: 128 rows x 64 fp16
   static constexpr int SCR_BYTES = 64 * chunk::kLD * 4;  // fp32 [64][68]
 
   static constexpr int OFF_KQ = 0;
   static constexpr int OFF_V = OFF_KQ + NKQ * KQ_BYTES;
-  static constexpr int OFF_G = OFF_V + V_BYTES;          // slot s at 2 s G_HALF: fp32 gains, then fp16 in its first half
+  static constexpr int OFF_G = OFF_V + V_BYTES;          // slot s at 2 s G_HALF: fp32 gains, then their fp16 hi | lo
   static constexpr int OFF_TAT = OFF_G + 4 * G_HALF;     // [T; Attn]
   static constexpr int OFF_TAD = OFF_TAT + TAT_HALF;     // -T diag(A) (rows 0..63 used)
   static constexpr int OFF_NF = OFF_TAD + TAT_HALF;
@@ -108,9 +112,10 @@ struct Params {
   const float* qn;
   float qn_scalar;
   const float* gains;  // full Kalman: [BH, L, D] fp32
-  float* S;
+  float* S;            // [BH, DT, s_cols]
+  int s_cols;          // DT, or 2 DT = 128 at DT = 64: the state [S | M] whose extra columns see zero values
   float* p;            // diag: [BH, D]; isotropic: the uncertainty scalar c, [BH]
-  void* o;
+  void* o;             // or nullptr
   float* m;
   int out_dtype;
   int L;
@@ -129,12 +134,19 @@ __device__ __forceinline__ int gf_pos(int i) {
 // 32 h .. 32 h + 31 as 16 pair columns at 32 h.
 __device__ __forceinline__ uint32_t tok_pair_col(int ks) { return 32u * (ks >> 1) + 8u * (ks & 1); }
 
-template <int VAR>
+// DT: the head size d_k = d_v (64 or 128).  The tiles and tensor-memory columns are laid out for 128; with
+// DT = 64 the upper 64-wide panels of K, Q and V are zero in shared memory (the products over d_k take
+// half the K steps, the state product half the columns), the d_v lanes 64..127 carry zeros through the
+// chain, and only the true coordinates are read from and written to memory.
+template <int VAR, int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_scan_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, Params P) {
   using Lay = WsLayout<VAR>;
   constexpr int NKQ = Lay::NKQ;
+  static_assert(DT == 64 || DT == D, "head sizes 64 and 128");
+  constexpr int NPT = DT / 64;   // 64-wide panels that hold data
+  constexpr int kGDT = DT / 8;   // true coordinates per thread in the per-token reductions
   // The diagonal variant's chain runs the gates and variances of chunk c + 1 while it waits for the
   // preparation of chunk c; the other variants' preparation runs its own gates.
   constexpr bool kChainGates = VAR == kDiag;
@@ -179,19 +191,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue_kq = [&](int cc) {
     const int slot = cc % NKQ;
     uint8_t* dst = sm + Lay::OFF_KQ + slot * Lay::KQ_BYTES;
-    sm100::mbar_arrive_expect_tx(&kq_full[slot], 2 * NP * 64 * 128);
+    sm100::mbar_arrive_expect_tx(&kq_full[slot], 2 * NPT * 64 * 128);
 #pragma unroll
-    for (int pn = 0; pn < NP; ++pn) {
+    for (int pn = 0; pn < NPT; ++pn) {
       sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL, &tm_k, &kq_full[slot], 64 * pn, cc * kC, bh);
       sm100::tma_load_3d(dst + pn * Lay::KQ_PANEL + 64 * 128, &tm_q, &kq_full[slot], 64 * pn, cc * kC, bh);
     }
   };
-  // bf16 -> fp16 in place over a [K; Q] slot (2 tensors x 2 panels x 64 rows x 8 chunks of 16 bytes) by the
+  // bf16 -> fp16 in place over a [K; Q] slot (2 tensors x NPT panels x 64 rows x 8 chunks of 16 bytes) by the
   // 256 threads u of one group, made visible to the tensor cores by the fence
   auto convert_kq = [&](int cc, int u) {
     uint8_t* KQs = sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
+    for (int r = 0; r < 4 * NPT; ++r) {
       uint4* p4 = reinterpret_cast<uint4*>(KQs) + u + kGroup * r;
       uint4 w = *p4;
       w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
@@ -201,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::fence_async_smem();
   };
   auto issue_v = [&](int cc) {
-    sm100::mbar_arrive_expect_tx(&v_full, NP * 64 * 128);
+    sm100::mbar_arrive_expect_tx(&v_full, NPT * 64 * 128);
 #pragma unroll
-    for (int pn = 0; pn < NP; ++pn) sm100::tma_load_3d(Vs + pn * Lay::V_PANEL, &tm_v, &v_full, 64 * pn, cc * kC, bh);
+    for (int pn = 0; pn < NPT; ++pn) sm100::tma_load_3d(Vs + pn * Lay::V_PANEL, &tm_v, &v_full, 64 * pn, cc * kC, bh);
   };
 
   if (tid == 0) {
@@ -226,6 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::fence_mbar_init();
     for (int cc = 0; cc < NKQ && cc < nchunks; ++cc) issue_kq(cc);
     issue_v(0);
+  }
+  if (DT < D) {  // the upper panels of every [K; Q] slot and of V: zero for the whole launch
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int e = tid; e < NKQ * 1024; e += kThreads)
+      reinterpret_cast<uint4*>(sm + Lay::OFF_KQ + (e / 1024) * Lay::KQ_BYTES + Lay::KQ_PANEL)[e % 1024] = z;
+    for (int e = tid; e < 512; e += kThreads) reinterpret_cast<uint4*>(Vs + Lay::V_PANEL)[e] = z;
+    sm100::fence_async_smem();
   }
   if (warp == 0) {
     sm100::tmem_alloc(&tmem_base, Lay::TMEM_COLS);
@@ -362,14 +381,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t b = sm100::smem_desc(kq_addr + (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32, 16, 1024);
         sm100::mma_bf16_ts(tmem + Lay::T_D2, tmem + Lay::T_SA + 8 * ks, b, id, ks > 0);
       }
-      if (part == 1) sm100::mma_commit(&bar_c);
+      if (part == NPT - 1) sm100::mma_commit(&bar_c);
     };
     auto kq_addr_of = [&](int cc) { return sm100::smem_u32(sm + Lay::OFF_KQ + (cc % NKQ) * Lay::KQ_BYTES); };
 
     // diagonal: p of coordinate tid (threads 0..D-1, warps 0..3, run the variances; warp 4 the gates)
-    const bool var_thread = VAR == kDiag && tid < D;
-    float pcur = var_thread ? P.p[(size_t)bh * D + tid] : 1.f;
-    float* Sg = P.S + (size_t)bh * D * D;
+    const bool var_thread = VAR == kDiag && tid < DT;
+    float pcur = var_thread ? P.p[(size_t)bh * DT + tid] : 1.f;
+    const int SC = P.s_cols;
+    float* Sg = P.S + (size_t)bh * DT * SC;
     if (!kConvInPrep) {  // [K; Q] of chunk 0
       if (!gwait(&kq_full[0], 0)) {
         aborted = true;
@@ -394,11 +414,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       const float AC0 = Aex[0][kC - 1];
 #pragma unroll
-      for (int v = 0; v < 2; ++v) {
+      for (int v = 0; v < NPT; ++v) {
         float x[32];
         const int dk0 = 32 * half + 64 * v;
 #pragma unroll
-        for (int u = 0; u < 32; ++u) x[u] = Sg[(size_t)(dk0 + u) * D + j];
+        for (int u = 0; u < 32; ++u) x[u] = (DT == D || j < SC) ? Sg[(size_t)(dk0 + u) * SC + j] : 0.f;
         emit_state(x, dk0, AC0);
         sm100::tmem_wait_st();
         sm100::tc_fence_before();
@@ -431,10 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
-        // 2 panels x 64 rows x 8 chunks of 16 bytes: four chunks per thread (made visible to the MMA by the
+        // NPT panels x 64 rows x 8 chunks of 16 bytes: 2 NPT chunks per thread (made visible to the MMA by the
         // fence here and the barrier of the prep_done wait below)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2 * NPT; ++u) {
           uint4* p4 = reinterpret_cast<uint4*>(Vs) + tid + kGroup * u;
           uint4 w = *p4;
           w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
@@ -537,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              sm100::smem_desc(tat_hi + 64 * 128 + ks * 32, 16, 1024), ido, ks > 0);
         sm100::mma_commit(&bar_o);
         sm100::mma_commit(&tat_free);
-        constexpr uint32_t id = sm100::idesc_f16(128, 128, false, true);
+        constexpr uint32_t id = sm100::idesc_f16(128, DT, false, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t ah = tmem + Lay::T_D2 + tok_pair_col(ks);
@@ -573,7 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const bool full = t0 + kC <= L;
         const float4* A4 = reinterpret_cast<const float4*>(&Aex[s][32 * half]);
-        const size_t base = ((size_t)bh * L + t0 + 32 * half) * D + j;
+        const size_t base = ((size_t)bh * L + t0 + 32 * half) * DT + j;
+        const bool own = (DT == D || j < DT) && P.o != nullptr;  // a true d_v coordinate (warp-uniform)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float Y[16], Oi[16];
@@ -589,16 +610,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             ov[4 * u4 + 2] = fmaf(av.z, Y[4 * u4 + 2], Oi[4 * u4 + 2]);
             ov[4 * u4 + 3] = fmaf(av.w, Y[4 * u4 + 3], Oi[4 * u4 + 3]);
           }
-          if (P.out_dtype == kF32) {
-            float* op = reinterpret_cast<float*>(P.o) + base + (size_t)(16 * hh) * D;
+          if (!own) {
+          } else if (P.out_dtype == kF32) {
+            float* op = reinterpret_cast<float*>(P.o) + base + (size_t)(16 * hh) * DT;
 #pragma unroll
             for (int u = 0; u < 16; ++u)
-              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * D] = ov[u];
+              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * DT] = ov[u];
           } else {
-            __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(P.o) + base + (size_t)(16 * hh) * D;
+            __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(P.o) + base + (size_t)(16 * hh) * DT;
 #pragma unroll
             for (int u = 0; u < 16; ++u)
-              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * D] = __float2bfloat16_rn(ov[u]);
+              if (full || t0 + 32 * half + 16 * hh + u < L) op[u * DT] = __float2bfloat16_rn(ov[u]);
           }
         }
       }
@@ -615,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float ACn = Aex[s ^ 1][kC - 1];
         const uint32_t kq_next = kq_addr_of(c + 1);
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
+        for (int v = 0; v < NPT; ++v) {
           float x[32];
           const int dk0 = 32 * half + 64 * v;
           sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + dk0, x);
@@ -637,17 +659,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (delta_like(VAR) && c + NKQ < nchunks) issue_kq(c + NKQ);  // this slot's K, Q are dead
       }
     }
-    if (!aborted) {
+    if (!aborted && (DT == D || (half == 0 && j < SC))) {  // warp-uniform: true d_k columns, state lanes
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
         float x[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_SM + 64 * half + 32 * v, x);
         sm100::tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 32; ++u) Sg[(size_t)(64 * half + 32 * v + u) * D + j] = x[u];
+        for (int u = 0; u < 32; ++u) Sg[(size_t)(64 * half + 32 * v + u) * SC + j] = x[u];
       }
-      if (var_thread) P.p[(size_t)bh * D + tid] = pcur;
     }
+    if (!aborted && var_thread) P.p[(size_t)bh * DT + tid] = pcur;
   } else {
     // =============================================================================== preparation group
     const int pt = tid - kGroup;
@@ -693,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = 32 * pass + (pt >> 3), part = pt & 7;
           float sq = 0.f;
 #pragma unroll
-          for (int pn = 0; pn < NP; ++pn) {
+          for (int pn = 0; pn < NPT; ++pn) {
             float xk[8];
             load8_f16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
 #pragma unroll
@@ -713,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 2; ++u) {
             const int t = 2 * lane + u;
             a2[u] = sA[s][t] * sA[s][t], qv[u] = sQ[s][t], rv[u] = sB[s][t], kk[u] = knorm[t];
-            mine = mobius::compose(mobius::iso_token(a2[u], qv[u], kk[u] / (D * rv[u])), mine);
+            mine = mobius::compose(mobius::iso_token(a2[u], qv[u], kk[u] / (DT * rv[u])), mine);
           }
           mobius::Mob incl = mine;
 #pragma unroll
@@ -731,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float sden = fmaf(cm, kk[u], rv[u]);
             bad |= !(sden > 0.f && isfinite(sden) && cm >= 0.f);
             sB[s][2 * lane + u] = cm / sden;
-            cv = D * cm * rv[u] / fmaf((float)D, rv[u], cm * kk[u]);
+            cv = DT * cm * rv[u] / fmaf((float)DT, rv[u], cm * kk[u]);
           }
           if (bad && t0 + 2 * lane < L) raise_status(P.status, kStatusNumeric);
           c_iso = __shfl_sync(0xffffffffu, cv, 31);
@@ -774,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = 32 * pass + (pt >> 3);
           float kv[kGD];
 #pragma unroll
-          for (int pn = 0; pn < NP; ++pn) {
+          for (int pn = 0; pn < NPT; ++pn) {
             float xk[8];
             load8_f16(KQ + pn * Lay::KQ_PANEL, sm100::sw128_chunk(t, part), xk);
 #pragma unroll
@@ -783,14 +805,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (delta_like(VAR)) {
             float sq = 0.f;
 #pragma unroll
-            for (int e = 0; e < kGD; ++e) sq = fmaf(kv[e], kv[e], sq);
+            for (int e = 0; e < kGDT; ++e) sq = fmaf(kv[e], kv[e], sq);
             sq = oct_sum(sq);
             if (part == 0) gn[s][t] = sB[s][t] * sB[s][t] * sq;
           } else {
             if (VAR == kDiag) {
               const float* Gw = reinterpret_cast<const float*>(Ghi);
 #pragma unroll
-              for (int pn = 0; pn < NP; ++pn)
+              for (int pn = 0; pn < NPT; ++pn)
 #pragma unroll
                 for (int hq = 0; hq < 2; ++hq) {
                   const float4 x4 = *reinterpret_cast<const float4*>(Gw + t * D + gf_pos(64 * pn + 8 * part + 4 * hq));
@@ -799,17 +821,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               float sd = 0.f;
 #pragma unroll
-              for (int e = 0; e < kGD; ++e) sd = fmaf(g[pass][e], kv[e], sd);
+              for (int e = 0; e < kGDT; ++e) sd = fmaf(g[pass][e], kv[e], sd);
               sd = oct_sum(sd) + sB[s][t];
               if (part == 0 && !(sd > 0.f && isfinite(sd))) raise_status(P.status, kStatusNumeric);
               const float inv_s = 1.f / sd;
 #pragma unroll
-              for (int e = 0; e < kGD; ++e) g[pass][e] *= inv_s;
+              for (int e = 0; e < kGDT; ++e) g[pass][e] *= inv_s;
             } else {
               const bool valid = t0 + t < L;
-              const float* gp = P.gains + ((size_t)bh * L + t0 + t) * D + 8 * part;
+              const float* gp = P.gains + ((size_t)bh * L + t0 + t) * DT + 8 * part;
 #pragma unroll
-              for (int pn = 0; pn < NP; ++pn)
+              for (int pn = 0; pn < NPT; ++pn)
 #pragma unroll
                 for (int hq = 0; hq < 2; ++hq) {
                   float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -820,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             float n2 = 0.f;
 #pragma unroll
-            for (int e = 0; e < kGD; ++e) n2 = fmaf(g[pass][e], g[pass][e], n2);
+            for (int e = 0; e < kGDT; ++e) n2 = fmaf(g[pass][e], g[pass][e], n2);
             n2 = oct_sum(n2);
             if (part == 0) gn[s][t] = n2;
           }
@@ -831,11 +853,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int pass = 0; pass < 2; ++pass) {
             const int t = 32 * pass + (pt >> 3);
 #pragma unroll
-            for (int pn = 0; pn < NP; ++pn) {
-              float xg[8];
+            for (int pn = 0; pn < NPT; ++pn) {
+              float xg[8], xl[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) xg[e] = g[pass][8 * pn + e];
+              for (int e = 0; e < 8; ++e) {
+                xg[e] = g[pass][8 * pn + e];
+                xl[e] = xg[e] - __half2float(__float2half_rn(xg[e]));
+              }
               store8_f16(Ghi, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xg);
+              store8_f16(Ghi + Lay::G_HALF, pn * Lay::G_PANEL + sm100::sw128_chunk(t, part), xl);
             }
           }
         }
@@ -850,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id1 = sm100::idesc_f16(128, 64, false, false);
         const uint32_t ghi = sm100::smem_u32(Ghi);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
+        for (int ks = 0; ks < DT / 16; ++ks) {
           const uint32_t koff = (ks / 4) * Lay::KQ_PANEL + (ks % 4) * 32;
           const uint64_t a = sm100::smem_desc(kq0 + koff, 16, 1024);
           if (delta_like(VAR)) {
@@ -858,6 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             const uint32_t goff = (ks / 4) * Lay::G_PANEL + (ks % 4) * 32;
             sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + goff, 16, 1024), id1, ks > 0);
+            sm100::mma_bf16(tmem + Lay::T_D1, a, sm100::smem_desc(ghi + Lay::G_HALF + goff, 16, 1024), id1, true);
           }
         }
         sm100::mma_commit(&bar_p);
@@ -953,38 +980,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) sm100::tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
-template <int VAR>
+template <int VAR, int DT>
 cudaError_t launch_ws_typed(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const Params& p, int BH,
                             cudaStream_t stream) {
   using Lay = WsLayout<VAR>;
-  cudaError_t e = cudaFuncSetAttribute(chunk_scan_ws_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(chunk_scan_ws_kernel<VAR, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  chunk_scan_ws_kernel<VAR><<<BH, kThreads, Lay::SMEM, stream>>>(q, k, v, p);
+  chunk_scan_ws_kernel<VAR, DT><<<BH, kThreads, Lay::SMEM, stream>>>(q, k, v, p);
   return cudaGetLastError();
+}
+
+template <int DT>
+cudaError_t launch_ws_dim(kdn_variant variant, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const Params& p, int BH, cudaStream_t stream) {
+  if (variant == KDN_KALMAN_FULL) return launch_ws_typed<kFull, DT>(tq, tk, tv, p, BH, stream);
+  if (variant == KDN_KALMAN_ISO) return launch_ws_typed<kIso, DT>(tq, tk, tv, p, BH, stream);
+  if (variant == KDN_KALMAN_DIAG) return launch_ws_typed<kDiag, DT>(tq, tk, tv, p, BH, stream);
+  return launch_ws_typed<kDelta, DT>(tq, tk, tv, p, BH, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_ws(kdn_variant variant, const kdn_dims& d, const ChunkArgs& a, const float* gains,
                             cudaStream_t stream) {
-  if (d.dk != D || d.dv != D) return cudaErrorInvalidValue;
+  if (d.dk != d.dv || (d.dk != 64 && d.dk != D)) return cudaErrorInvalidValue;
+  if (variant == KDN_KALMAN_FULL && gains == nullptr) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!make_bf16_tmap(&tq, a.q, a.BH, a.L, D) || !make_bf16_tmap(&tk, a.k, a.BH, a.L, D) ||
-      !make_bf16_tmap(&tv, a.v, a.BH, a.L, D))
+  if (!make_bf16_tmap(&tq, a.q, a.BH, a.L, d.dk) || !make_bf16_tmap(&tk, a.k, a.BH, a.L, d.dk) ||
+      !make_bf16_tmap(&tv, a.v, a.BH, a.L, d.dv))
     return cudaErrorInvalidValue;
   Params p{};
   p.beta = a.beta, p.a = a.a, p.r = a.r, p.qn = a.qn, p.qn_scalar = a.qn_scalar, p.gains = gains;
   p.S = a.S, p.o = a.o, p.m = a.m, p.out_dtype = a.out_dtype, p.L = a.L, p.status = a.status;
-  if (variant == KDN_KALMAN_FULL) return launch_ws_typed<kFull>(tq, tk, tv, p, a.BH, stream);
-  if (variant == KDN_KALMAN_ISO) {
-    p.p = a.P;  // the uncertainty scalar c, [BH]
-    return launch_ws_typed<kIso>(tq, tk, tv, p, a.BH, stream);
-  }
-  if (variant == KDN_KALMAN_DIAG) {
-    p.p = a.P;
-    return launch_ws_typed<kDiag>(tq, tk, tv, p, a.BH, stream);
-  }
-  return launch_ws_typed<kDelta>(tq, tk, tv, p, a.BH, stream);
+  p.s_cols = a.state_cols == 0 ? d.dv : a.state_cols;
+  if (p.s_cols != d.dv && !(d.dk == 64 && p.s_cols == 2 * d.dv)) return cudaErrorInvalidValue;
+  // diagonal: the variances, [BH, d]; isotropic: the uncertainty scalar c, [BH]
+  if (variant == KDN_KALMAN_DIAG || variant == KDN_KALMAN_ISO) p.p = a.P;
+  return d.dk == D ? launch_ws_dim<D>(variant, tq, tk, tv, p, a.BH, stream)
+                   : launch_ws_dim<64>(variant, tq, tk, tv, p, a.BH, stream);
 }
 
 }  // namespace kdn

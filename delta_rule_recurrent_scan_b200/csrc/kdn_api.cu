@@ -196,6 +196,8 @@ kdn_status seg_scan(kdn_variant body, const kdn_dims* d, int P, const kdn::Chunk
   sa.SI = reinterpret_cast<float*>(area + lay.si);
   sa.Sc = reinterpret_cast<float*>(area + lay.sc);
   const bool diag = body == KDN_KALMAN_DIAG;
+  // d = 64: B and M from one run on the d x 2d state [S | M] (Sz and SI hold it side by side)
+  sa.aug = D == 64 && d->dv == 64 ? 1 : 0;
   if (diag) {
     sa.maps = reinterpret_cast<float4*>(area + lay.maps);
     for (int i = 0; i < 3; ++i) sa.pcopy[i] = reinterpret_cast<float*>(area + lay.p[i]);
@@ -208,15 +210,20 @@ kdn_status seg_scan(kdn_variant body, const kdn_dims* d, int P, const kdn::Chunk
   dv.B = BH * P, dv.H = 1, dv.L = c.L / P, dv.segments = 1;
   kdn::ChunkArgs v = c;
   v.BH = BH * P, v.L = c.L / P;
-  // each segment's map S0 -> M S0 + B: runs from S0 = 0 and S0 = I (o is rewritten below, m not written)
-  v.m = nullptr;
+  // each segment's map S0 -> M S0 + B: runs from S0 = 0 and S0 = I, or one run from [0 | I] (no read-out
+  // or surprise: o and m are written by the true run below)
+  v.o = nullptr, v.m = nullptr;
   v.S = sa.Sz, v.P = diag ? sa.pcopy[0] : c.P;
+  if (sa.aug) v.state_cols = 2 * d->dv;
   KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
-  v.S = sa.SI, v.P = diag ? sa.pcopy[1] : c.P;
-  KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
+  if (!sa.aug) {
+    v.S = sa.SI, v.P = diag ? sa.pcopy[1] : c.P;
+    KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
+  }
+  v.state_cols = 0;
   KDN_TRY(cuda_status(kdn::launch_seg_combine(D, sa, BH, st), "segment chaining launch"));
   // the true scan of every segment from its start state
-  v.m = c.m;
+  v.o = c.o, v.m = c.m;
   v.S = sa.Sc, v.P = diag ? sa.pcopy[2] : c.P;
   KDN_TRY(cuda_status(kdn::launch_chunk_sside(body, dv, v, gains, st), "segment scan launch"));
   // the last segment's end state (and p) is the head's
@@ -288,13 +295,14 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
   int nseg = 1;
   KDN_TRY(resolve_segments(variant, dims, &nseg));
   if (nseg > 1) {
-    // start states, two map runs, chaining, the true run (+ the diagonal uncertainty maps and starts; for
-    // full Kalman the chunk maps, their chain, the run-start covariances and the covariance side)
-    n = 5 + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 4 : 0);
+    // start states, two map runs (one on [S | M] at d = 64), chaining, the true run (+ the diagonal
+    // uncertainty maps and starts; for full Kalman the chunk maps, their chain, the run-start covariances
+    // and the covariance side)
+    n = (dims->dk == 64 ? 4 : 5) + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 4 : 0);
     if (body == KDN_KALMAN_FULL) name = "riccati_chain_kernel", ar = "f32";  // the longest of those launches
   }
-  if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1))
-    n += 1;  // the beta prologue (at d = 128 the chunk kernel runs it itself on the serial path)
+  if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && nseg == 1))
+    n += 1;  // the beta prologue (the one-segment chunk kernel runs it itself on the serial path)
   if (launches) *launches = n;
   if (kernel) *kernel = name;
   if (arith) *arith = ar;
@@ -453,8 +461,8 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
   int nseg = 1;
   KDN_TRY(resolve_segments(KDN_KALMAN_ISO, dims, &nseg));
-  if (kdn::chunk_supported(KDN_DELTA, *dims) && dims->dk == 128 && nseg == 1) {
-    // the d = 128 chunk kernel runs the uncertainty scan in its own preparation: one launch
+  if (kdn::chunk_supported(KDN_DELTA, *dims) && nseg == 1) {
+    // the chunk kernel runs the uncertainty scan in its own preparation: one launch
     kdn::ChunkArgs ch{};
     ch.q = q, ch.k = k, ch.v = v, ch.a = a, ch.r = r, ch.qn = qn, ch.qn_scalar = qn_scalar, ch.P = c;
     ch.S = S, ch.o = o, ch.m = m, ch.out_dtype = dims->out_dtype, ch.BH = BH, ch.L = dims->L, ch.status = status;

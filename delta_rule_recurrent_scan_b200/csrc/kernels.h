@@ -216,8 +216,9 @@ struct SegArgs {
   int ncopy;
   // memory state
   const float* S;         // [BH, d, d] the caller's start state
-  float* Sz;              // [BH P, d, d] segment end states from S0 = 0
-  float* SI;              // [BH P, d, d] segment end states from S0 = I
+  float* Sz;              // [BH P, d, d] segment end states from S0 = 0 (aug: [BH P, d, 2 d], [B | M])
+  float* SI;              // [BH P, d, d] segment end states from S0 = I (aug: unused)
+  int aug;                // 1: one run on [S | M] from [0 | I] gave B and M side by side
   float* Sc;              // [BH P, d, d] out: the true start state of every segment
   unsigned* status;
 };

@@ -10,7 +10,9 @@
 //   1. (diagonal Kalman) every segment composes its per-coordinate uncertainty maps, and one thread
 //      per coordinate chains them to get p at each segment start;
 //   2. the chunk kernel runs every segment twice in parallel, from S0 = 0 (giving B) and from S0 = I
-//      (giving M + B);
+//      (giving M + B); at d = 64 once instead, on the d x 2d state [S | M] from [0 | I] whose extra
+//      columns see zero values (the columns of the state evolve independently for fixed gains, so
+//      the first block ends at B and the second at M; 2d = 128 fills the chunk kernel's d_v lanes);
 //   3. one pass per head chains S_{s+1} = M_s S_s + B_s across segments, in fp32;
 //   4. the chunk kernel runs every segment once more from its true start state, writing o and m.
 //
@@ -102,6 +104,15 @@ __global__ void __launch_bounds__(DK) seg_prefix_kernel(SegArgs p) {
   if (bad) raise_status(p.status, kStatusNumeric);
 }
 
+// Step 2's start state at d = 64 on [S | M]: [0 | I] ([d][2 d]) for every segment.
+__global__ void __launch_bounds__(256) seg_init_aug_kernel(float* SA, int d) {
+  float* base = SA + (size_t)blockIdx.x * d * 2 * d;
+  for (int u = threadIdx.x; u < 2 * d * d; u += blockDim.x) {
+    const int r = u / (2 * d), c = u % (2 * d);
+    base[u] = (c == d + r) ? 1.f : 0.f;
+  }
+}
+
 // Step 2's start states: S0 = 0 in Sz and S0 = I in SI for every segment (d_k = d_v).
 __global__ void __launch_bounds__(256) seg_init_kernel(float* Sz, float* SI, int d) {
   const size_t base = (size_t)blockIdx.x * d * d;
@@ -116,7 +127,8 @@ __global__ void __launch_bounds__(256) seg_init_kernel(float* Sz, float* SI, int
   }
 }
 
-// Step 3 (d = 64 or 128): S_{s+1} = (SI_s - Sz_s) S_s + Sz_s for one head and a slab of kSlab columns; every
+// Step 3 (d = 64 or 128): S_{s+1} = (SI_s - Sz_s) S_s + Sz_s (at d = 64: M_s S_s + B_s from the run on [S | M])
+// for one head and a slab of kSlab columns; every
 // S_s (s = 0 .. P-1, S_0 the caller's state) is written to Sc.  Per segment the CTA stages SI_s and Sz_s in
 // shared memory with asynchronous 16-byte copies (rows padded by 4 floats; every slab of the head reads the
 // same L2-resident rows), then each thread forms one row r of the slab (kCombThreads / D threads per row,
@@ -153,12 +165,14 @@ __global__ void __launch_bounds__(kCombThreads) seg_combine_kernel(SegArgs p) {
   for (int s = 0; s < p.P; ++s) {
     const size_t j = (size_t)h * p.P + s;
     if (s + 1 < p.P) {
-      const float* SIg = p.SI + j * DD;
-      const float* Szg = p.Sz + j * DD;
+      // rows of SI_s (or M_s) and Sz_s (B_s): [d][d] each, or side by side in rows of 2 d
+      const int ld = p.aug ? 2 * D : D;
+      const float* Szg = p.Sz + j * D * ld;
+      const float* SIg = p.aug ? Szg + D : p.SI + j * DD;
       for (int q = tid; q < D * D / 4; q += kCombThreads) {
         const int rr = (4 * q) / D, cc = (4 * q) % D;
-        cp_async16(SIs + rr * RS + cc, SIg + 4 * (size_t)q);
-        cp_async16(Szs + rr * RS + cc, Szg + 4 * (size_t)q);
+        cp_async16(SIs + rr * RS + cc, SIg + (size_t)rr * ld + cc);
+        cp_async16(Szs + rr * RS + cc, Szg + (size_t)rr * ld + cc);
       }
     }
     for (int e = tid; e < D * kSlab; e += kCombThreads) {
@@ -175,7 +189,8 @@ __global__ void __launch_bounds__(kCombThreads) seg_combine_kernel(SegArgs p) {
     for (int kq = 0; kq < D / 4; ++kq) {
       const float4 a4 = *reinterpret_cast<const float4*>(SIs + r * RS + 4 * kq);
       const float4 b4 = *reinterpret_cast<const float4*>(Szs + r * RS + 4 * kq);
-      const float m[4] = {a4.x - b4.x, a4.y - b4.y, a4.z - b4.z, a4.w - b4.w};  // M_s[r][4 kq ..]
+      const float4 m4 = p.aug ? a4 : make_float4(a4.x - b4.x, a4.y - b4.y, a4.z - b4.z, a4.w - b4.w);
+      const float m[4] = {m4.x, m4.y, m4.z, m4.w};  // M_s[r][4 kq ..]
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float4* xr = reinterpret_cast<const float4*>(X + (4 * kq + e) * kSlab + cg);
@@ -239,7 +254,10 @@ cudaError_t launch_seg_uncertainty(int dk, const SegArgs& p, int BH, cudaStream_
 
 cudaError_t launch_seg_init(int d, const SegArgs& p, int BH, cudaStream_t stream) {
   if (d % 4 != 0) return cudaErrorInvalidValue;
-  seg_init_kernel<<<BH * p.P, 256, 0, stream>>>(p.Sz, p.SI, d);
+  if (p.aug)
+    seg_init_aug_kernel<<<BH * p.P, 256, 0, stream>>>(p.Sz, d);
+  else
+    seg_init_kernel<<<BH * p.P, 256, 0, stream>>>(p.Sz, p.SI, d);
   return cudaGetLastError();
 }
 

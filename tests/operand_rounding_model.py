@@ -1,4 +1,4 @@
-"""Float64 model of the d = 128 chunk kernel's operand roundings.
+"""Float64 model of the chunk kernel's operand roundings (d = 64 and 128).
 
 Test infrastructure: it repeats the chunk form of the scan (the generalised
 WY form: (I + N) E = V - diag(A) K S0, O = diag(A) Q S0 + AT R, S_C = A_C S0 +
@@ -8,7 +8,8 @@ layer length can be measured on the CPU against the exact scan.  It shares no
 code with the oracle or the kernels.
 
 Roundings: ``exact`` (none); ``f16`` (one fp16 value, round to nearest, with
-fp16's range and subnormals: what the kernel does now); ``bf16_pair`` (bf16 hi
+fp16's range and subnormals: what the kernel does now, except that the Kalman
+gains enter K G^T and Q G^T as an fp16 hi + lo pair); ``bf16_pair`` (bf16 hi
 + bf16 lo, about 16 significand bits).
 """
 
@@ -54,10 +55,12 @@ def chunk_scan_rounded(variant, q, k, v, beta, a, r, qn, rounding, C=64):
                 p = pp * r[sl][i] / (r[sl][i] + pp * K[i] ** 2)
             Gr = rnd(G)
             bscale = np.ones(n)
+        # the gains in K G^T and Q G^T: the fp16 pair under f16, else as in the state product
+        Gd = Gr + rnd(G - Gr) if rounding == "f16" and variant != "delta" else Gr
         Kr, Qr = rnd(K), rnd(Q)
-        N = np.tril((Kr @ Gr.T) * gam * bscale[None, :], -1)
+        N = np.tril((Kr @ Gd.T) * gam * bscale[None, :], -1)
         T = np.linalg.inv(np.eye(n) + N)
-        Att = np.tril((Qr @ Gr.T) * gam * bscale[None, :])
+        Att = np.tril((Qr @ Gd.T) * gam * bscale[None, :])
         Tr = rnd(T)
         AT = Att @ Tr
         Sr = rnd(S)

@@ -17,7 +17,7 @@ import torch
 import oracle
 from delta_rule_recurrent_scan_b200 import kdn
 from delta_rule_recurrent_scan_b200.workloads import WORKLOADS, make_decode_inputs, make_scan_inputs
-from parity import SELF_TOL, TOL, assert_symmetric_pd, compare, initial_state, normwise_err, run_gpu, run_oracle, self_tol
+from parity import TOL, assert_symmetric_pd, compare, initial_state, normwise_err, run_gpu, run_oracle, self_tol
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -174,9 +174,9 @@ def test_split_invariance_and_resume(variant):
         out = run_gpu(variant, xs, S=S, C=C)
         parts.append(out)
     o = torch.cat([p["o"] for p in parts], dim=2)
-    # a different chunking rounds differently: the bf16 hi/lo products carry about 2^-16
-    assert normwise_err(o.float(), whole["o"].float()) < SELF_TOL
-    assert normwise_err(S, whole["S"]) < SELF_TOL
+    # a different chunking rounds differently: the fp16 operands carry 2^-11
+    assert normwise_err(o.float(), whole["o"].float()) < self_tol(64)
+    assert normwise_err(S, whole["S"]) < self_tol(64)
 
 
 # ----------------------------------------------------------------------------- full layer-scale workloads
@@ -219,7 +219,7 @@ def test_decode_steps_equal_scan_and_oracle(variant):
     xs = {k: (v.movedim(0, 2).contiguous() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     scan = run_gpu(variant, xs)
     o = torch.stack(outs, dim=2)
-    assert normwise_err(o.float(), scan["o"].float()) < self_tol(w.dk)  # the scan takes the d = 128 chunk kernel
+    assert normwise_err(o.float(), scan["o"].float()) < self_tol(w.dk)  # the scan takes the chunk kernel
     assert normwise_err(S, scan["S"]) < self_tol(w.dk)
     ref = run_oracle(variant, xs)
     compare({"o": o, "m": torch.stack(ms, dim=2), "S": S}, ref, TOL["bf16"])

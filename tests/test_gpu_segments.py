@@ -73,7 +73,7 @@ def test_library_choice_splits_few_heads(variant, d):
     w = WORKLOADS["gdn_d128"].with_(variant=variant, dk=d, dv=d, qn=1e-3)
     x = make_scan_inputs(w, seed=11, device=DEV, B=1, H=2, L=1024)
     n = kdn.plan(variant, 1, 2, 1024, d, d)["launches"]
-    assert n >= 5, n  # the segment-parallel plan
+    assert n >= (4 if d == 64 else 5), n  # the segment-parallel plan (one map run on [S | M] at d = 64)
     _check(variant, x, 0)
 
 
