@@ -153,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Who converts each [K; Q] tile from bf16 to fp16 in place: the preparation group for the Kalman
   // variants, whose chain is the longer group; for the delta-like ones the chain, one chunk ahead.
   constexpr bool kConvInPrep = !delta_like(VAR);
+  // The diagonal variant's preparation writes Attn after its inverse (see the preparation group)
+  constexpr bool kLateAttn = VAR == kDiag;
   constexpr int LD = chunk::kLD;
 
   extern __shared__ uint8_t smem_raw[];
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // per-chunk scalars, two slots (chunk c uses slot c & 1)
   __shared__ float sA[2][kC], sB[2][kC], sQ[2][kC];         // a, beta | r, Qn
-  __shared__ __align__(16) float4 sVk[VAR == kDiag ? 2 : 1][kC];  // diagonal: (a^2, Qn, r) per token
+  __shared__ __align__(16) float4 sVk[VAR == kDiag ? 2 : 1][kC];  // diagonal: (a^2, Qn, 1 / r) per token
   __shared__ float ell[2][kC], gn[2][kC];
   __shared__ __align__(16) float Aex[2][kC];                // A_t
   __shared__ __align__(16) float gcol[2][kC];               // 1 / A_t (times beta_t for the delta rule), when
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int u = tid - kGroup;
     if (u >= 0 && u < kC) {
       sA[slot][u] = ra, sB[slot][u] = rb, sQ[slot][u] = rq;
-      if (VAR == kDiag) sVk[slot][u] = make_float4(ra * ra, rq, rb, 0.f);
+      if (VAR == kDiag) sVk[slot][u] = make_float4(ra * ra, rq, 1.f / rb, 0.f);
     }
   };
   // gates of chunk cc into its slot, by one warp: inclusive prefix sums of log a over the chunk (a gate of 0
@@ -305,9 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Diagonal variances of chunk cc (independent of v and S), run by the chain one chunk ahead, in its wait
   // for the preparation.  Per coordinate: p^- = a^2 p + Qn, pk = p^- k, p <- p^- r / (r + pk k), on the
-  // homogeneous pair p = x / y: token t maps (x, y) by M_t = [[r a^2, r Qn], [k^2 a^2, k^2 Qn + r]], three
-  // multiply-adds of serial chain per token, the division that recovers p^- off the chain, and a
-  // power-of-two rescale every eight tokens (exact; x / y does not change).  One thread per coordinate steps
+  // homogeneous pair p = x / y: token t maps (x, y) by [[a^2, Qn], [w a^2, w Qn + 1]] (w = k^2 / r; the
+  // token's map [[r a^2, r Qn], [k^2 a^2, k^2 Qn + r]] divided by r), i.e. x' = a^2 x + Qn y = p^- y and
+  // y' = y + w x': a multiply and two multiply-adds of serial chain per token; the divisions that recover
+  // the gains p^- k = x' k / y are batched after each four tokens' steps (in-order issue would otherwise
+  // hold the chain behind every reciprocal), and a power-of-two rescale every eight tokens is exact
+  // (x / y does not change).  One thread per coordinate steps
   // all 64 tokens: this phase issues beside the preparation group, and a split of the tokens over threads
   // (composing the earlier tokens' maps) only adds instructions, while the direct form p <- r p^- / s puts
   // a division on the serial chain.  The unnormalised gains pk go, fp32, into the gain slot of chunk cc;
@@ -321,22 +326,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Gw = reinterpret_cast<float*>(sm + Lay::OFF_G + 2 * sl * Lay::G_HALF);
       const int gpos = gf_pos(i);
       float x = pcur, y = 1.f;
+      // keys and (a^2, Qn, 1 / r) of four tokens into registers a group ahead of their use
+      auto load4 = [&](int t4, float (&kq)[4], float4 (&sq)[4]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          kq[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t4 + u, i % 64)));
+          sq[u] = sVk[sl][t4 + u];
+        }
+      };
+      // the serial part of four tokens (two multiply-adds and a multiply each), then their gains: the
+      // reciprocals and stores issue after the chain steps, not between them
+      auto step4 = [&](int t4, const float (&kq)[4], const float4 (&sq)[4]) {
+        float num[4], den[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float xm = fmaf(sq[u].x, x, sq[u].y * y);
+          num[u] = xm * kq[u], den[u] = y;
+          x = xm;
+          y = fmaf(kq[u] * kq[u] * sq[u].z, xm, y);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Gw[(t4 + u) * D + gpos] = __fdividef(num[u], den[u]);
+      };
+      float ka[4], kb[4];
+      float4 va[4], vb[4];
+      load4(0, ka, va);
 #pragma unroll 1
       for (int t8 = 0; t8 < kC; t8 += 8) {
-        float kk[8];
-        float4 sv[8];  // a^2, Qn, r
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          kk[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Kp + sm100::sw128(t8 + u, i % 64)));
-          sv[u] = sVk[sl][t8 + u];
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float xm = fmaf(sv[u].x, x, sv[u].y * y);
-          Gw[(t8 + u) * D + gpos] = __fdividef(xm * kk[u], y);
-          x = sv[u].z * xm;
-          y = fmaf(kk[u] * kk[u], xm, sv[u].z * y);
-        }
+        load4(t8 + 4, kb, vb);
+        step4(t8, ka, va);
+        load4((t8 + 8) & (kC - 1), ka, va);  // (the last one reloads tokens 0..3, unused)
+        step4(t8 + 4, kb, vb);
         const int ey = min((__float_as_int(y) >> 23) & 0xff, 253);
         const float sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey), exact
         x *= sc, y *= sc;
@@ -442,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           bad = !sm100::mbar_wait_bounded(&v_full, c & 1, kWaitCycles) ||
                 !sm100::mbar_wait_bounded(&gates_ready[s], (c >> 1) & 1, kWaitCycles);
-          if (!bad && !kConvInPrep && c + 1 < nchunks)
+          if (!bad && (!kConvInPrep || kChainGates) && c + 1 < nchunks)
             bad = !sm100::mbar_wait_bounded(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1, kWaitCycles);
         }
         bad = named_sync_or(kBarChain, kGroup, bad);
@@ -451,32 +471,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           aborted = true;
           break;
         }
-        // NPT panels x 64 rows x 8 chunks of 16 bytes: 2 NPT chunks per thread (made visible to the MMA by the
-        // fence here and the barrier of the prep_done wait below)
+        // NPT panels x 64 rows x 8 chunks of 16 bytes, in place (made visible to the MMA by the fence here and
+        // the barrier below): the diagonal variant's warps 4..7 convert while warps 0..3 step the variances of
+        // chunk c + 1 and warp 4 runs its gates (its scalars were stored before gates_ready of chunk c; its keys
+        // are read before the preparation converts their tile, which waits for var_done)
+        constexpr int kConvThreads = kChainGates ? kGroup / 2 : kGroup;
+        const int cv = kChainGates ? tid - kGroup / 2 : tid;
+        if (cv >= 0) {
 #pragma unroll
-        for (int u = 0; u < 2 * NPT; ++u) {
-          uint4* p4 = reinterpret_cast<uint4*>(Vs) + tid + kGroup * u;
-          uint4 w = *p4;
-          w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
-          w.z = sm100::bf16x2_to_f16x2(w.z), w.w = sm100::bf16x2_to_f16x2(w.w);
-          *p4 = w;
+          for (int u = 0; u < 2 * NPT * kGroup / kConvThreads; ++u) {
+            uint4* p4 = reinterpret_cast<uint4*>(Vs) + cv + kConvThreads * u;
+            uint4 w = *p4;
+            w.x = sm100::bf16x2_to_f16x2(w.x), w.y = sm100::bf16x2_to_f16x2(w.y);
+            w.z = sm100::bf16x2_to_f16x2(w.z), w.w = sm100::bf16x2_to_f16x2(w.w);
+            *p4 = w;
+          }
+          sm100::fence_async_smem();
         }
-        sm100::fence_async_smem();
-        if (!kConvInPrep && c + 1 < nchunks) {  // [K; Q] of the next chunk, for the preparation
+        if (kChainGates) {
+          if (c + 1 < nchunks) {
+            if (var_thread) run_variances(c + 1, tid, pcur);
+            if (gw == 4) run_gates(c + 1);
+          }
+          named_sync(kBarChain, kGroup);
+          if (leader && c + 1 < nchunks) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
+        } else if (!kConvInPrep && c + 1 < nchunks) {  // [K; Q] of the next chunk, for the preparation
           convert_kq(c + 1, tid);
           named_sync(kBarChain, kGroup);
           if (leader) sm100::mbar_arrive(&kq_conv[(c + 1) % NKQ]);
         }
-      }
-      // ---------------------------------------------------------------- variances of chunk c + 1, while the S0 product runs
-      if (kChainGates && c + 1 < nchunks) {
-        // its scalars were stored before gates_ready of chunk c; its keys are read before the preparation
-        // converts their tile (that waits for var_done)
-        if (!gwait(&kq_full[(c + 1) % NKQ], ((c + 1) / NKQ) & 1)) { aborted = true; break; }
-        if (var_thread) run_variances(c + 1, tid, pcur);
-        if (gw == 4) run_gates(c + 1);
-        named_sync(kBarChain, kGroup);
-        if (leader) sm100::mbar_arrive(&var_done[(c + 1) & 1]);
       }
 
       // ---------------------------------------------------------------- E^T = V^T T^T, queued behind the S0 product
@@ -889,11 +912,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm100::mma_commit(&bar_p);
       }
+      auto prep_wait = [&](uint64_t* b, uint32_t parity) -> bool {
+        bool bad = false;
+        if (leader) bad = !sm100::mbar_wait_bounded(b, parity, kWaitCycles);
+        bad = named_sync_or(kBarPrep, kGroup, bad);
+        if (bad && leader) raise_status(P.status, kStatusTimeout);
+        sm100::tc_fence_after();
+        return !bad;
+      };
       {
         bool bad = false;
         if (leader) {
           bad = !sm100::mbar_wait_bounded(&bar_p, ph_p, kWaitCycles);
-          if (!bad && c >= 1) bad = !sm100::mbar_wait_bounded(&tat_free, (c - 1) & 1, kWaitCycles);
+          if (!bad && !kLateAttn && c >= 1) bad = !sm100::mbar_wait_bounded(&tat_free, (c - 1) & 1, kWaitCycles);
         }
         bad = named_sync_or(kBarPrep, kGroup, bad);
         if (bad) {
@@ -905,49 +936,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         ph_p ^= 1;
       }
 
-      // ---------------------------------------------------------------- N (lanes 0..63) | Attn (lanes 64..127)
-      {
+      // Y_ij (beta_j) Gam_ij from the D1 lanes of this warp: as A_i times the column factor when the chunk's
+      // decay allows it, else by one exponential per pair (chunks with strong resets); the choice is uniform
+      // over the chunk.  N (lanes 0..63) goes to the fp32 scratch, Attn (lanes 64..127) into [T; Attn] once the
+      // chain's read-out product of the previous chunk has released that buffer: at once for the delta-like
+      // variants, whose preparation is the longer group; after the inverse for the diagonal variant, so that its
+      // inverse runs while the chain works on innovations and read-out, not beside the next chunk's variances.
+      const int irow = row & 63;
+      auto emit_d1 = [&](auto store) {
         float Y[32];
         sm100::tmem_ld32(tmem + t_lane + Lay::T_D1 + 32 * half, Y);
         sm100::tmem_wait_ld();
-        // Y_ij (beta_j) Gam_ij: as A_i times the column factor when the chunk's decay allows it, else by
-        // one exponential per pair (chunks with strong resets); the choice is uniform over the chunk
-        const int i = row & 63;
-        const float li = ell[s][i], Ai = Aex[s][i];
-        auto emit = [&](auto gam) {
-          if (qw < 2) {
+        if (ell[s][kC - 1] >= -80.f) {
+          const float Ai = Aex[s][irow];
+          store(Y, [&](int jj) { return Ai * gcol[s][jj]; });
+        } else {
+          const float li = ell[s][irow];
+          store(Y, [&](int jj) { return __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f); });
+        }
+      };
+      auto emit_attn = [&] {
+        emit_d1([&](const float (&Y)[32], auto gam) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              float v4[4];
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float xa[8];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int jj = 32 * half + e + u;
-                v4[u] = (jj < i) ? Y[e + u] * gam(jj) : 0.f;
-              }
-              *reinterpret_cast<float4*>(Nf + i * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+            for (int e = 0; e < 8; ++e) {
+              const int jj = 32 * half + 8 * q8 + e;
+              xa[e] = (jj <= irow) ? Y[8 * q8 + e] * gam(jj) : 0.f;
             }
-          } else {
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-              float xa[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int jj = 32 * half + 8 * q8 + e;
-                xa[e] = (jj <= i) ? Y[8 * q8 + e] * gam(jj) : 0.f;
-              }
-              store8_f16(TAThi, sm100::sw128_chunk(64 + i, 4 * half + q8), xa);
-            }
+            store8_f16(TAThi, sm100::sw128_chunk(64 + irow, 4 * half + q8), xa);
           }
-        };
-        if (ell[s][kC - 1] >= -80.f)
-          emit([&](int jj) { return Ai * gcol[s][jj]; });
-        else
-          emit([&](int jj) { return __expf(li - ell[s][jj]) * (delta_like(VAR) ? sB[s][jj] : 1.f); });
+        });
+      };
+      // ---------------------------------------------------------------- N (lanes 0..63) | Attn (lanes 64..127)
+      if (!kLateAttn && qw >= 2) emit_attn();
+      if (qw < 2) {
+        emit_d1([&](const float (&Y)[32], auto gam) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float v4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int jj = 32 * half + e + u;
+              v4[u] = (jj < irow) ? Y[e + u] * gam(jj) : 0.f;
+            }
+            *reinterpret_cast<float4*>(Nf + irow * LD + 32 * half + e) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+          }
+        });
       }
       named_sync(kBarPrep, kGroup);
 
-      // ---------------------------------------------------------------- T = (I + N)^-1 into rows 0..63 of [T; Attn]
+      // ---------------------------------------------------------------- T = (I + N)^-1 (fp32 scratch)
       chunk::invert_unit_lower_64(Nf, Tf, pt, [] { named_sync(kBarPrep, kGroup); });
+
+      // ---------------------------------------------------------------- [T; Attn] and -T diag(A)
+      if (kLateAttn) {
+        if (c >= 1 && !prep_wait(&tat_free, (c - 1) & 1)) { aborted = true; break; }
+        if (qw >= 2) emit_attn();
+      }
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int e = pt + 256 * hh;
