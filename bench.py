@@ -86,19 +86,19 @@ _RICCATI_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/riccati.cu",
                     "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
                     "delta_rule_recurrent_scan_b200/csrc/common.cuh"]
 _B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment per head)
-_WS_SHA = "94549d85257830a12ddfefcedfdfdaa6908ef443"
+_WS_SHA = "5dcefb7e1efa30da5c9de7ff14c994b0a7163836"
 NCU_TRAFFIC = {
     "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                         "bytes_per_token": (308.566272e6 + 171.428096e6) / _B3,
+                         "bytes_per_token": (308.433408e6 + 172.305664e6) / _B3,
                          "capture": "ncu, chunk_scan_ws_kernel<diag> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "gdn_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                 "bytes_per_token": (308.382976e6 + 171.018496e6) / _B3,
+                 "bytes_per_token": (308.394240e6 + 172.547584e6) / _B3,
                  "capture": "ncu, chunk_scan_ws_kernel<delta> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                        "bytes_per_token": (308.413952e6 + 170.260480e6) / _B3,
+                        "bytes_per_token": (308.401664e6 + 170.171648e6) / _B3,
                         "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "4a83c95c4b2bec424ca3c3aa8e46b412a0ae6adf",
-                         "bytes_per_token": (31.122432e6 + 1.151488e6) / (2 * 8 * 4096),
+    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "cd30a0cc47f438b3b02ed37cc226f50e034ca776",
+                         "bytes_per_token": (31.121920e6 + 1.081856e6) / (2 * 8 * 4096),
                          "capture": "ncu, riccati_chain_kernel at the full workload B=2 H=8 L=4096"},
 }
 
