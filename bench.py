@@ -660,7 +660,11 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(w), "peak_source": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "kernel": plan["kernel"],
-                         "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events"},
+                         "timed": "whole C-ABI call (status-word memset + kernels) with CUDA events",
+                         # the same time against the bytes of a bf16 read-out (the figure the per-token
+                         # byte table of the method's roofline uses; this scan writes o in fp32)
+                         "frac_bf16_o_bytes": algorithmic_bytes(w, out_bytes=2) / (ms * 1e-3) / 1e9 / peak,
+                         "algorithmic_bytes_bf16_o_per_launch": algorithmic_bytes(w, out_bytes=2)},
             "e2e": None if e2e is None else {"value": e2e["value"], "unit": "tokens/s",
                                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                                              "ms_per_step": e2e["ms"], "copied": e2e["copied"],
