@@ -75,6 +75,10 @@ __device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
   return r != 0;
 }
 
+// TMEM column of the fp16 pairs of the 16-token block ks (K step of 16) when thread half h holds tokens
+// 32 h .. 32 h + 31 of a 64-token operand as 16 pair columns at 32 h.
+__device__ __forceinline__ uint32_t tok_pair_col(int ks) { return 32u * (ks >> 1) + 8u * (ks & 1); }
+
 // Sum over the 8 consecutive lanes that share a token.
 __device__ __forceinline__ float oct_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);

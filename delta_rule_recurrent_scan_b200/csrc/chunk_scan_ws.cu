@@ -57,6 +57,7 @@ using chunk::named_sync_or;
 using chunk::oct_sum;
 using chunk::load8_f16;
 using chunk::store8_f16;
+using chunk::tok_pair_col;
 
 enum Var : int { kDelta = 0, kDiag = 1, kFull = 2, kIso = 3 };
 
@@ -129,10 +130,6 @@ __device__ __forceinline__ int gf_pos(int i) {
   const int h = (i >> 2) & 1;
   return (i & ~63) | (h << 5) | ((((i >> 3) & 7) ^ (h << 2)) << 2) | (i & 3);
 }
-
-// TMEM column of the fp16 pairs of the 16-token block ks (K step of 16): thread half h holds tokens
-// 32 h .. 32 h + 31 as 16 pair columns at 32 h.
-__device__ __forceinline__ uint32_t tok_pair_col(int ks) { return 32u * (ks >> 1) + 8u * (ks & 1); }
 
 // DT: the head size d_k = d_v (64 or 128).  The tiles and tensor-memory columns are laid out for 128; with
 // DT = 64 the upper 64-wide panels of K, Q and V are zero in shared memory (the products over d_k take

@@ -299,7 +299,8 @@ kdn_status kdn_plan(kdn_variant variant, const kdn_dims* dims, int* launches, co
     // uncertainty maps and starts; for full Kalman the chunk maps, their chain, the run-start covariances
     // and the covariance side)
     n = (dims->dk == 64 ? 4 : 5) + (body == KDN_KALMAN_DIAG ? 2 : 0) + (body == KDN_KALMAN_FULL ? 4 : 0);
-    if (body == KDN_KALMAN_FULL) name = "riccati_chain_kernel", ar = "f32";  // the longest of those launches
+    if (body == KDN_KALMAN_FULL)  // the longest of those launches (d = 128: on the tensor cores)
+      name = dims->dk == 128 ? "riccati_chain_tc_kernel" : "riccati_chain_kernel", ar = dims->dk == 128 ? "bf16-tc" : "f32";
   }
   if (variant == KDN_KALMAN_ISO && n > 0 && !(kdn::chunk_supported(KDN_DELTA, *dims) && nseg == 1))
     n += 1;  // the beta prologue (the one-segment chunk kernel runs it itself on the serial path)

@@ -406,6 +406,302 @@ __global__ void __launch_bounds__(kChainThreads, 2) riccati_chain_kernel(Riccati
   }
 }
 
+// ---------------------------------------------------------------------------------------- chain on tcgen05
+// d = 128: one CTA per head carries [X^T | Y^T] in tensor memory (lane = column c of [X; Y], fp32 masters
+// X^T and Y^T, their fp16 pairs as the A operands) through the chunk maps with four products per chunk:
+//   R^T  = X^T (diag(alpha) K)^T + Y^T (diag(beta) K)^T      A = X^T, Y^T (TMEM)   B = alpha_t k_t, beta_t k_t
+//   Z^T  = R^T G                                              A = R^T (TMEM)        B = G^T as stored (rows t)
+//   X^T <- alpha_C X^T + beta_C Y^T + Z^T diag(u) K           A = Z^T diag(u)       B = K (d_k contiguous)
+//   Y^T <- Y^T + Z^T K                                        A = Z^T               B = K
+// then every column is rescaled by a power of two (max |Y| of the column in [1, 2); P = X Y^-1 does not
+// change) and the fp16 pairs are formed for the next chunk.  The operands of a chunk (K, alpha K, beta K in
+// fp16, G^T in fp16) are built by a second warp group one chunk ahead, in two slots.  Every operand is
+// rounded to fp16 once (the keys are exact), with fp32 accumulation and fp32 masters; a float64 model of
+// those roundings over a 4096-token head stays near 1e-5 of P.
+constexpr int kTcThreads = 512;  // 256 chain + 256 preparation
+
+struct TcChainLayout {
+  static constexpr int PANEL = 64 * 128;                // 64 rows x 64 fp16
+  static constexpr int OFF_K = 0;                       // K: 2 panels
+  static constexpr int OFF_KA = OFF_K + 2 * PANEL;      // alpha_t k_t
+  static constexpr int OFF_KB = OFF_KA + 2 * PANEL;     // beta_t k_t
+  static constexpr int OFF_G = OFF_KB + 2 * PANEL;      // G^T (row t, columns s): 1 panel
+  static constexpr int SLOT = OFF_G + PANEL;
+  static constexpr int SMEM = 2 * SLOT + 1024;          // + alignment slack
+  // tensor memory columns
+  static constexpr uint32_t T_XM = 0, T_YM = 128, T_XP = 256, T_YP = 320, T_R = 384, T_Z = 448;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) riccati_chain_tc_kernel(RiccatiArgs p) {
+  constexpr int D = 128, C = kRC;
+  using Ly = TcChainLayout;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ float su[2][C], sac[2][2];
+  __shared__ float ymax[2][D];
+  __shared__ uint64_t prep_done[2], chain_done[2], bar_m;
+  __shared__ uint32_t tmem_base;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x, nch = (p.L + C - 1) / C;
+  const int cps = p.cps, runs = (nch + cps - 1) / cps, last = (runs - 1) * cps;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) sm100::mbar_init(&prep_done[i], 1), sm100::mbar_init(&chain_done[i], 1);
+    sm100::mbar_init(&bar_m, 1);
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0) {
+    sm100::tmem_alloc(&tmem_base, 512);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (tid < 256) {
+    // =============================================================== chain: lane c, column half h
+    const int qw = warp & 3, half = warp >> 2, col = 32 * qw + lane;
+    const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+    const bool leader = tid == 0;
+    bool aborted = false;
+    uint32_t ph_m = 0;
+    auto gwait = [&](uint64_t* b, uint32_t parity) -> bool {
+      bool bad = false;
+      if (leader) bad = !sm100::mbar_wait_bounded(b, parity, chunk::kWaitCycles);
+      bad = chunk::named_sync_or(1, 256, bad);
+      if (bad && leader) raise_status(p.status, kStatusTimeout);
+      sm100::tc_fence_after();
+      return !bad;
+    };
+    auto sync_tc = [&] {
+      sm100::tc_fence_before();
+      chunk::named_sync(1, 256);
+      sm100::tc_fence_after();
+    };
+    // fp16 pairs of 64 master columns (elements 64 half ..) of this lane: 32 pair columns at 32 half
+    auto emit_pairs = [&](uint32_t pair_col, const float (&x)[32], int v) {
+      float hw[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) hw[e] = __uint_as_float(sm100::pack2_f16(x[2 * e], x[2 * e + 1]));
+      sm100::tmem_st16(tmem + t_lane + pair_col + 32 * half + 16 * v, hw);
+    };
+    // masters at a run start: X rows then Y rows of this run's [X; Y] (row-major 2D x D)
+    auto store_start = [&](int run) {
+      float* xy = p.xy + ((size_t)bh * runs + run) * 2 * D * D;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          float x[32];
+          sm100::tmem_ld32(tmem + t_lane + (m ? Ly::T_YM : Ly::T_XM) + 64 * half + 32 * v, x);
+          sm100::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) xy[((size_t)m * D + 64 * half + 32 * v + u) * D + col] = x[u];
+        }
+    };
+    // [X; Y] = [P0; I]
+#pragma unroll 1
+    for (int v = 0; v < 2; ++v) {
+      float x[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) x[u] = p.P0[((size_t)bh * D + 64 * half + 32 * v + u) * D + col];
+      sm100::tmem_st32(tmem + t_lane + Ly::T_XM + 64 * half + 32 * v, x);
+      emit_pairs(Ly::T_XP, x, v);
+      sm100::tmem_wait_st();  // (the stores' registers are reused below)
+#pragma unroll
+      for (int u = 0; u < 32; ++u) x[u] = 64 * half + 32 * v + u == col ? 1.f : 0.f;
+      sm100::tmem_st32(tmem + t_lane + Ly::T_YM + 64 * half + 32 * v, x);
+      emit_pairs(Ly::T_YP, x, v);
+      sm100::tmem_wait_st();
+    }
+    sm100::tmem_wait_st();
+    sync_tc();
+
+    for (int c = 0; c < last && !aborted; ++c) {
+      const int s = c & 1;
+      if (c % cps == 0) store_start(c / cps);
+      if (!gwait(&prep_done[s], (c >> 1) & 1)) { aborted = true; break; }
+      const uint32_t slot = sm100::smem_u32(tsm + s * Ly::SLOT);
+      // ---- R^T
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_f16(128, 64, false, false);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t b = slot + (m ? Ly::OFF_KB : Ly::OFF_KA) + (ks / 4) * Ly::PANEL + (ks % 4) * 32;
+            sm100::mma_bf16_ts(tmem + Ly::T_R, tmem + (m ? Ly::T_YP : Ly::T_XP) + 8 * ks,
+                               sm100::smem_desc(b, 16, 1024), id, m > 0 || ks > 0);
+          }
+        sm100::mma_commit(&bar_m);
+      }
+      // ---- X^T <- alpha_C X^T + beta_C Y^T while R^T runs (it reads only the pairs)
+      {
+        const float aC = sac[s][0], bC = sac[s][1];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          float x[16], y[16];
+          sm100::tmem_ld16(tmem + t_lane + Ly::T_XM + 64 * half + 16 * v, x);
+          sm100::tmem_ld16(tmem + t_lane + Ly::T_YM + 64 * half + 16 * v, y);
+          sm100::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) x[u] = fmaf(aC, x[u], bC * y[u]);
+          sm100::tmem_st16(tmem + t_lane + Ly::T_XM + 64 * half + 16 * v, x);
+          sm100::tmem_wait_st();
+        }
+        sm100::tmem_wait_st();
+      }
+      if (!gwait(&bar_m, ph_m)) { aborted = true; break; }
+      ph_m ^= 1;
+      // ---- R^T to fp16 pairs in place (tokens 32 half .. + 31), then Z^T = R^T G
+      {
+        float r[32];
+        sm100::tmem_ld32(tmem + t_lane + Ly::T_R + 32 * half, r);
+        sm100::tmem_wait_ld();
+        float hw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hw[e] = __uint_as_float(sm100::pack2_f16(r[2 * e], r[2 * e + 1]));
+        sm100::tmem_st16(tmem + t_lane + Ly::T_R + 32 * half, hw);
+        sm100::tmem_wait_st();
+      }
+      sync_tc();
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_f16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          sm100::mma_bf16_ts(tmem + Ly::T_Z, tmem + Ly::T_R + chunk::tok_pair_col(ks),
+                             sm100::smem_desc(slot + Ly::OFF_G + ks * 32, 16, 1024), id, ks > 0);
+        sm100::mma_commit(&bar_m);
+      }
+      if (!gwait(&bar_m, ph_m)) { aborted = true; break; }
+      ph_m ^= 1;
+      // ---- Z^T pairs in place, Z^T diag(u) pairs over the dead R^T; then the master updates
+      {
+        float z[32];
+        sm100::tmem_ld32(tmem + t_lane + Ly::T_Z + 32 * half, z);
+        sm100::tmem_wait_ld();
+        float hw[16], hu[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int t = 32 * half + 2 * e;
+          hw[e] = __uint_as_float(sm100::pack2_f16(z[2 * e], z[2 * e + 1]));
+          hu[e] = __uint_as_float(sm100::pack2_f16(z[2 * e] * su[s][t], z[2 * e + 1] * su[s][t + 1]));
+        }
+        sm100::tmem_st16(tmem + t_lane + Ly::T_Z + 32 * half, hw);
+        sm100::tmem_st16(tmem + t_lane + Ly::T_R + 32 * half, hu);
+        sm100::tmem_wait_st();
+      }
+      sync_tc();
+      if (leader) {
+        constexpr uint32_t id = sm100::idesc_f16(128, 128, false, true);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks)
+            sm100::mma_bf16_ts(tmem + (m ? Ly::T_YM : Ly::T_XM), tmem + (m ? Ly::T_Z : Ly::T_R) + chunk::tok_pair_col(ks),
+                               sm100::smem_desc(slot + Ly::OFF_K + ks * 2048, Ly::PANEL, 1024), id, true);
+        sm100::mma_commit(&chain_done[s]);  // the slot's operands are dead once these complete
+        sm100::mma_commit(&bar_m);
+      }
+      if (!gwait(&bar_m, ph_m)) { aborted = true; break; }
+      ph_m ^= 1;
+      // ---- rescale every column by a power of two, and the pairs of the next chunk
+      {
+        float mx = 0.f;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          float y[32];
+          sm100::tmem_ld32(tmem + t_lane + Ly::T_YM + 64 * half + 32 * v, y);
+          sm100::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) mx = fmaxf(mx, fabsf(y[u]));
+        }
+        ymax[half][col] = mx;
+        chunk::named_sync(1, 256);
+        const float m = fmaxf(ymax[0][col], ymax[1][col]);
+        float sc = 1.f;
+        if (m > 0.f && isfinite(m)) {
+          const int ey = min((__float_as_int(m) >> 23) & 0xff, 253);
+          sc = __int_as_float((254 - ey) << 23);  // 2^(127 - ey): max |Y| of the column into [1, 2)
+        } else if (half == 0) {
+          raise_status(p.status, kStatusNumeric);
+        }
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            float x[32];
+            const uint32_t mcol = (mm ? Ly::T_YM : Ly::T_XM) + 64 * half + 32 * v;
+            sm100::tmem_ld32(tmem + t_lane + mcol, x);
+            sm100::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) x[u] *= sc;
+            sm100::tmem_st32(tmem + t_lane + mcol, x);
+            emit_pairs(mm ? Ly::T_YP : Ly::T_XP, x, v);
+            sm100::tmem_wait_st();
+          }
+      }
+      sync_tc();
+    }
+    if (!aborted) store_start(runs - 1);
+  } else {
+    // =============================================================== preparation of chunk c into slot c & 1
+    const int pt = tid - 256;
+    const bool leader = pt == 0;
+    const __nv_bfloat16* kg = reinterpret_cast<const __nv_bfloat16*>(p.k) + (size_t)bh * p.L * D;
+    for (int c = 0; c < last; ++c) {
+      const int s = c & 1;
+      {
+        bool bad = false;
+        if (leader && c >= 2) bad = !sm100::mbar_wait_bounded(&chain_done[s], ((c >> 1) & 1) ^ 1, chunk::kWaitCycles);
+        bad = chunk::named_sync_or(2, 256, bad);
+        if (bad) {
+          if (leader) raise_status(p.status, kStatusTimeout);
+          break;
+        }
+      }
+      uint8_t* sl = tsm + s * Ly::SLOT;
+      const size_t map = (size_t)bh * nch + c;
+      const float* ab = p.map_ab + map * 2 * C;
+      // K, alpha K, beta K: 64 tokens x 16 chunks of 8 keys, four per thread
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int item = pt + 256 * rr, t = item >> 4, q = item & 15;
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(kg + ((size_t)c * C + t) * D + 8 * q), f);
+        const float al = ab[2 * t], be = ab[2 * t + 1];
+        float fa[8], fb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fa[e] = al * f[e], fb[e] = be * f[e];
+        const uint32_t off = (q >> 3) * Ly::PANEL + sm100::sw128_chunk(t, q & 7);
+        chunk::store8_f16(sl + Ly::OFF_K, off, f);
+        chunk::store8_f16(sl + Ly::OFF_KA, off, fa);
+        chunk::store8_f16(sl + Ly::OFF_KB, off, fb);
+      }
+      // G^T rows t: 64 x 8 chunks, two per thread
+      const float* gsrc = p.map_g + map * C * C;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int item = pt + 256 * rr, t = item >> 3, q = item & 7;
+        const float4 g0 = *reinterpret_cast<const float4*>(gsrc + t * C + 8 * q);
+        const float4 g1 = *reinterpret_cast<const float4*>(gsrc + t * C + 8 * q + 4);
+        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        chunk::store8_f16(sl + Ly::OFF_G, sm100::sw128_chunk(t, q), g);
+      }
+      if (pt < C) su[s][pt] = p.map_u[map * C + pt];
+      if (pt == C) sac[s][0] = ab[2 * (C - 1)], sac[s][1] = ab[2 * (C - 1) + 1];
+      sm100::fence_async_smem();
+      chunk::named_sync(2, 256);
+      if (leader) sm100::mbar_arrive(&prep_done[s]);
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) sm100::tmem_dealloc(tmem, 512);
+}
+
 // ---------------------------------------------------------------------------------------- P = X Y^-1
 // At every run start, Y^T P^T = X^T by Gauss-Jordan elimination with partial pivoting on the augmented
 // [Y^T | X^T] (D x 2D), held in registers: warp w owns rows 8w..8w+7, lane l columns CB l..CB l+CB-1.
@@ -550,10 +846,16 @@ cudaError_t launch_riccati_typed(const RiccatiArgs& a, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const size_t chain_smem = ChainLayout<D>::BYTES;
-  e = cudaFuncSetAttribute(riccati_chain_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chain_smem);
-  if (e != cudaSuccess) return e;
-  riccati_chain_kernel<D><<<dim3(a.BH, D / kRCols), kChainThreads, chain_smem, st>>>(a);
+  if constexpr (D == 128) {  // the chain on the tensor cores, one CTA per head
+    e = cudaFuncSetAttribute(riccati_chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TcChainLayout::SMEM);
+    if (e != cudaSuccess) return e;
+    riccati_chain_tc_kernel<<<a.BH, kTcThreads, TcChainLayout::SMEM, st>>>(a);
+  } else {
+    const size_t chain_smem = ChainLayout<D>::BYTES;
+    e = cudaFuncSetAttribute(riccati_chain_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chain_smem);
+    if (e != cudaSuccess) return e;
+    riccati_chain_kernel<D><<<dim3(a.BH, D / kRCols), kChainThreads, chain_smem, st>>>(a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t x_smem = ExtractLayout<D>::BYTES;
