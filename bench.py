@@ -86,7 +86,7 @@ _RICCATI_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/riccati.cu",
                     "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
                     "delta_rule_recurrent_scan_b200/csrc/common.cuh"]
 _B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment per head)
-_WS_SHA = "5dcefb7e1efa30da5c9de7ff14c994b0a7163836"
+_WS_SHA = "f1d52692d9aa476369052689f14393df8bddf887"
 NCU_TRAFFIC = {
     "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
                          "bytes_per_token": (308.433408e6 + 172.305664e6) / _B3,
@@ -97,9 +97,9 @@ NCU_TRAFFIC = {
     "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
                         "bytes_per_token": (308.401664e6 + 170.171648e6) / _B3,
                         "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "cd30a0cc47f438b3b02ed37cc226f50e034ca776",
-                         "bytes_per_token": (31.121920e6 + 1.081856e6) / (2 * 8 * 4096),
-                         "capture": "ncu, riccati_chain_kernel at the full workload B=2 H=8 L=4096"},
+    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "d820f760ed0db550e9296bf73652a633f75682fa",
+                         "bytes_per_token": (31.137024e6 + 0.194560e6) / (2 * 8 * 4096),
+                         "capture": "ncu, riccati_chain_tc_kernel at the full workload B=2 H=8 L=4096"},
 }
 
 
