@@ -148,9 +148,10 @@ def test_empty_sequence_is_a_no_op(variant):
     assert torch.equal(got["S"], S0)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
-def test_single_token_and_degenerate_gates(variant):
-    w = WORKLOADS["gdn_d64"].with_(variant=variant, qn=1e-3)
+def test_single_token_and_degenerate_gates(variant, d):
+    w = WORKLOADS["gdn_d64"].with_(variant=variant, qn=1e-3, dk=d, dv=d)
     x = make_scan_inputs(w, seed=5, device=DEV, B=2, H=2, L=97)
     x["a"][:, :, ::7] = 0.0   # full resets
     x["a"][:, :, 3::11] = 1.0  # no decay
@@ -159,6 +160,24 @@ def test_single_token_and_degenerate_gates(variant):
     compare(run_gpu(variant, x), run_oracle(variant, x), TOL["bf16"])
     x1 = make_scan_inputs(w, seed=6, device=DEV, B=2, H=2, L=1)
     compare(run_gpu(variant, x1), run_oracle(variant, x1), TOL["bf16"])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("variant", ["kalman_diag", "kalman_full"])
+def test_cancelling_single_token_readout(variant, d):
+    """One token per head with q nearly orthogonal to k: o_1 = (q . g) v_1 with q . g about 1e-3 of |q| |g|.
+    The read-out's q . g must then carry the gain's rounding relative to itself, not to |q| |g| (a single fp16
+    rounding of the gains would leave a few per cent here)."""
+    w = WORKLOADS["gdn_d64"].with_(variant=variant, qn=1e-3, dk=d, dv=d)
+    x = make_scan_inputs(w, seed=9, device=DEV, B=1, H=8, L=1)
+    k = x["k"].float()
+    u = torch.randn(k.shape, generator=torch.Generator(device="cpu").manual_seed(10)).to(DEV)
+    u = u - (u * k).sum(-1, keepdim=True) * k  # orthogonal to k
+    q = u / u.norm(dim=-1, keepdim=True) + 1e-3 * k
+    x["q"] = q.to(x["q"].dtype)
+    qk = (x["q"].float() * k).sum(-1).abs().max().item()
+    assert qk < 3e-3, qk  # the bf16 rounding of q keeps q . k small
+    compare(run_gpu(variant, x), run_oracle(variant, x), TOL["bf16"])
 
 
 @pytest.mark.parametrize("variant", ["delta", "kalman_diag", "kalman_full", "kalman_iso"])
