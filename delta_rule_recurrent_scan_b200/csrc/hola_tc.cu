@@ -20,6 +20,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <climits>
+
 #include "chunk.h"
 #include "chunk_common.cuh"
 #include "common.cuh"
@@ -365,56 +367,79 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
 // ---------------------------------------------------------------------------------------- parallel form
 // The cache a block reads depends only on m (section 3.3: the top-w tokens by surprise), not on any read, so
-// it can be fixed for every block first.  hola_cache_select_kernel walks one head's blocks with 128 threads,
-// one per candidate (the cache, then the block's tokens): each candidate's rank is the number of others that
-// come before it (larger m, ties to the earlier token), the first w by rank form the next cache, and the
-// cache read by block b goes to cidx[head][b] in rank order (-1 past its size).  It also writes the final
-// cache's indices, ascending.
-constexpr int kSelThreads = 4 * kRows;  // four lanes per candidate, each comparing every fourth other
+// it can be fixed for every block first.  hola_cache_select_kernel walks one head's blocks with one CTA,
+// keeping the cache as a list in rank order (larger m first, ties to the earlier token: a strict total
+// order).  Per block: the block's 64 candidates are put in rank order among themselves (eight lanes per
+// candidate count the others before it), then the two ordered lists are merged: an element's place in the
+// union is its index in its own list plus the number of elements of the other list before it (a binary
+// search), and the first w places form the next cache.  The cache read by block b goes to cidx[head][b] in
+// rank order (-1 past its size); the final cache's indices are also written, ascending.
+constexpr int kSelThreads = 512;
 
 __global__ void __launch_bounds__(kSelThreads) hola_cache_select_kernel(HolaArgs p) {
-  __shared__ float cm[kRows];  // candidates: rows 0..63 the cache (rank order), 64..127 the block
-  __shared__ int ci[kRows];
-  __shared__ float nm[64];
-  __shared__ int ni[64];
-  const int tid = threadIdx.x, cand = tid >> 2, part = tid & 3, bh = blockIdx.x, L = p.L, w = p.w;
+  __shared__ float cm[2][64];  // the cache in rank order, two buffers
+  __shared__ int ci[2][64];
+  __shared__ float rm[64];     // the block's candidates as they come
+  __shared__ int ri[64];
+  __shared__ float bm[64];     // ... and in rank order
+  __shared__ int bi[64];
+  const int tid = threadIdx.x, bh = blockIdx.x, L = p.L, w = p.w;
   const int nblocks = (L + 63) / 64;
   const size_t tok0 = (size_t)bh * L;
-  const bool owner = part == 0;  // the lane that stores the candidate's results
-  if (owner && cand < 64) cm[cand] = -INFINITY, ci[cand] = -1;
-  int ncache = 0;
-  float mnext = owner && cand >= 64 && cand - 64 < L ? p.m[tok0 + cand - 64] : -INFINITY;
+  int ncache = 0, cur = 0;
+  float mnext = tid < 64 && tid < L ? p.m[tok0 + tid] : -INFINITY;  // the next block's m, in flight
   for (int b = 0; b < nblocks; ++b) {
-    if (owner && cand >= 64) {
-      const int t = 64 * b + cand - 64;
-      ci[cand] = t < L ? t : -1;
-      cm[cand] = t < L ? mnext : -INFINITY;
-      const int tn = t + 64;
-      mnext = tn < L ? p.m[tok0 + tn] : -INFINITY;  // the next block's m, in flight during the ranking
+    const int nv = min(64, L - 64 * b);  // valid tokens of the block (the others sort last)
+    if (tid < 64) {
+      rm[tid] = tid < nv ? mnext : -INFINITY;
+      ri[tid] = tid < nv ? 64 * b + tid : INT_MAX;
+      const int tn = 64 * (b + 1) + tid;
+      mnext = tn < L ? p.m[tok0 + tn] : -INFINITY;
+    } else if (tid < 128) {  // the cache block b reads
+      const int r = tid - 64;
+      p.cidx[((size_t)bh * nblocks + b) * 64 + r] = r < ncache ? ci[cur][r] : -1;
     }
     __syncthreads();
-    if (owner && cand < 64) p.cidx[((size_t)bh * nblocks + b) * 64 + cand] = ci[cand];
-    const float m0 = cm[cand];
-    const int i0 = ci[cand];
-    int rank = 0;
-#pragma unroll 8
-    for (int c = part; c < kRows; c += 4) rank += (ci[c] >= 0 && before(cm[c], ci[c], m0, i0)) ? 1 : 0;  // 4 banks
-    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
-    const bool kept = owner && i0 >= 0 && rank < w;
-    if (kept) nm[rank] = m0, ni[rank] = i0;
-    ncache = __syncthreads_count(kept);  // also: every read of cm, ci above is done
-    if (owner && cand < 64) {
-      cm[cand] = cand < ncache ? nm[cand] : -INFINITY;
-      ci[cand] = cand < ncache ? ni[cand] : -1;
+    {
+      const int cand = tid >> 3, part = tid & 7;
+      const float m0 = rm[cand];
+      const int i0 = ri[cand];
+      int rank = 0;
+#pragma unroll
+      for (int c = part; c < 64; c += 8) rank += before(rm[c], ri[c], m0, i0) ? 1 : 0;
+      rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+      rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+      rank += __shfl_xor_sync(0xffffffffu, rank, 4);
+      if (part == 0) bm[rank] = m0, bi[rank] = i0;
     }
+    __syncthreads();
+    if (tid < 128) {  // warps 0..1: the cache's elements, warps 2..3: the block's
+      const bool from_cache = tid < 64;
+      const int k = tid & 63;
+      if (k < (from_cache ? ncache : nv)) {
+        const float mx = from_cache ? cm[cur][k] : bm[k];
+        const int ix = from_cache ? ci[cur][k] : bi[k];
+        const float* om = from_cache ? bm : cm[cur];
+        const int* oi = from_cache ? bi : ci[cur];
+        int lo = 0, hi = from_cache ? nv : ncache;  // the other list's elements before this one: a prefix
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (before(om[mid], oi[mid], mx, ix)) lo = mid + 1;
+          else hi = mid;
+        }
+        const int pos = k + lo;
+        if (pos < w) cm[cur ^ 1][pos] = mx, ci[cur ^ 1][pos] = ix;
+      }
+    }
+    ncache = min(w, ncache + nv);
+    cur ^= 1;
     __syncthreads();
   }
   if (p.cache != nullptr && tid < w) {  // the final cache, ascending token indices, -1 past its size
-    const int mine = tid < ncache ? ci[tid] : -1;
+    const int mine = tid < ncache ? ci[cur][tid] : -1;
     if (mine >= 0) {
       int pos = 0;
-      for (int c = 0; c < ncache; ++c) pos += ci[c] < mine ? 1 : 0;
+      for (int c = 0; c < ncache; ++c) pos += ci[cur][c] < mine ? 1 : 0;
       p.cache[(size_t)bh * w + pos] = mine;
     } else {
       p.cache[(size_t)bh * w + tid] = -1;
