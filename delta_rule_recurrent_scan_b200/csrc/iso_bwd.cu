@@ -136,77 +136,160 @@ __global__ void __launch_bounds__(32) iso_backward_kernel(IsoBwdArgs p) {
   if (lane == 0) p.dc0[bh] = cb;
 }
 
+// N sums across the warp at once: the shuffle stages of the N values interleave.
+template <int N>
+__device__ __forceinline__ void warp_sum_n(float (&x)[N]) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i], o);
+}
+
+// Asynchronous global -> shared copies for the input rings of the chain kernels below.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Rows of n floats-or-bf16 (e bytes each, n e a multiple of 16) from global to shared, by the 32 lanes.
+__device__ __forceinline__ void copy_rows(void* dst, const void* src, int bytes, int lane) {
+  for (int c = lane; c < bytes / 16; c += 32)
+    cp_async16(static_cast<uint8_t*>(dst) + 16 * c, static_cast<const uint8_t*>(src) + 16 * c);
+}
+
+__device__ __forceinline__ float smem_elem(const uint8_t* base, int idx, int dtype) {
+  return dtype == kBF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx])
+                        : reinterpret_cast<const float*>(base)[idx];
+}
+
+// Only p is serial in t (p_{t+1} = p^-_t r_t / (r_t + p^-_t k_t^2) per coordinate); the coupled sum s_t of each
+// token depends on p^-_t but nothing serial depends on s_t.  So each batch steps the per-coordinate chain over
+// its kTB tokens first, then reduces the kTB sums at once, then writes the gains.  The inputs arrive through a
+// ring of kStages batches in shared memory, copied asynchronously kStages - 1 batches ahead (one warp per
+// head has nothing else to hide the load latency with).
+constexpr int kStages = 4;
+
 template <int NPL>
 __global__ void __launch_bounds__(32) diag_forward_kernel(DiagBwdArgs p) {
+  constexpr int KB = kTB * 128 * 4;  // key bytes of a stage (at most fp32 keys of d_k = 128)
+  __shared__ __align__(16) uint8_t ks[kStages][KB];
+  __shared__ float sa[kStages][kTB], sr[kStages][kTB], sq[kStages][kTB];
   const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
+  const int es = p.in_dtype == kBF16 ? 2 : 4;
   const size_t tok0 = (size_t)bh * L;
+  const int nbt = (L + kTB - 1) / kTB;
+  auto issue = [&](int bt) {
+    if (bt < nbt) {
+      const int t0 = bt * kTB, nb = min(kTB, L - t0), st = bt % kStages;
+      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane);
+      if (lane < nb) {
+        const size_t ti = tok0 + t0 + lane;
+        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        cp_async4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+      }
+    }
+    cp_async_commit();  // (an empty group past the end keeps the wait count uniform)
+  };
+  for (int bt = 0; bt < kStages - 1; ++bt) issue(bt);
   float pv[NPL];
 #pragma unroll
   for (int e = 0; e < NPL; ++e) {
     const int i = lane + 32 * e;
     pv[e] = i < D ? (p.p0 != nullptr ? p.p0[(size_t)bh * D + i] : 1.f) : 0.f;
   }
-  for (int t0 = 0; t0 < L; t0 += kTB) {
-    const int nb = min(kTB, L - t0);
-    float sa = 1.f, sr = 1.f, sq = 0.f;
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      sa = p.a != nullptr ? p.a[ti] : 1.f, sr = p.r[ti], sq = p.qn != nullptr ? p.qn[ti] : p.qn_scalar;
-    }
-    float kv[kTB][NPL];
+  for (int bt = 0; bt < nbt; ++bt) {
+    issue(bt + kStages - 1);
+    cp_async_wait<kStages - 1>();  // this batch has landed
+    __syncwarp();
+    const int st = bt % kStages, t0 = bt * kTB, nb = min(kTB, L - t0);
+    float pm[kTB][NPL], kv[kTB][NPL], sum[kTB];
 #pragma unroll
-    for (int u = 0; u < kTB; ++u)
+    for (int u = 0; u < kTB; ++u) {  // the serial chain (tokens past the end: a = 1, Qn = 0, k = 0 keep p)
+      const bool ok = u < nb;
+      const float at = ok ? sa[st][u] : 1.f, rt = ok ? sr[st][u] : 1.f, qt = ok ? sq[st][u] : 0.f;
+      sum[u] = 0.f;
 #pragma unroll
       for (int e = 0; e < NPL; ++e) {
         const int i = lane + 32 * e;
-        kv[u][e] = u < nb && i < D ? load_elem(p.k, (tok0 + t0 + u) * D + i, p.in_dtype) : 0.f;
+        kv[u][e] = ok && i < D ? smem_elem(ks[st], u * D + i, p.in_dtype) : 0.f;
+        if (ok && i < D) p.pprev[(tok0 + t0 + u) * D + i] = pv[e];
+        pm[u][e] = fmaf(at * at, pv[e], qt);
+        const float pk = pm[u][e] * kv[u][e];
+        sum[u] = fmaf(pk, kv[u][e], sum[u]);
+        pv[e] = __fdividef(pm[u][e] * rt, fmaf(pk, kv[u][e], rt));
       }
+    }
+    warp_sum_n(sum);
 #pragma unroll
     for (int u = 0; u < kTB; ++u) {
       if (u >= nb) break;
-      const float at = __shfl_sync(0xffffffffu, sa, u), rt = __shfl_sync(0xffffffffu, sr, u);
-      const float qt = __shfl_sync(0xffffffffu, sq, u);
-      float pm[NPL], sum = 0.f;
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) {
-        pm[e] = fmaf(at * at, pv[e], qt);
-        sum = fmaf(pm[e] * kv[u][e], kv[u][e], sum);
-      }
-      const float is = 1.f / (warp_sum(sum) + rt);
-      const size_t ti = tok0 + t0 + u;
+      const float is = __fdividef(1.f, sum[u] + sr[st][u]);
 #pragma unroll
       for (int e = 0; e < NPL; ++e) {
         const int i = lane + 32 * e;
-        if (i < D) {
-          p.gains[ti * D + i] = pm[e] * kv[u][e] * is;
-          p.pprev[ti * D + i] = pv[e];
-        }
-        pv[e] = pm[e] * rt / fmaf(pm[e] * kv[u][e], kv[u][e], rt);
+        if (i < D) p.gains[(tok0 + t0 + u) * D + i] = pm[u][e] * kv[u][e] * is;
       }
     }
+    __syncwarp();  // every lane is done with this stage before it is refilled
   }
+  cp_async_wait<0>();
 }
 
+// The adjoint pb of p is the only serial quantity backwards: pb_{t-1} = a_t^2 (c1 + pb_t c2) per coordinate,
+// with c1 = dG k / s + ds k^2 and c2 = r^2 / den^2 fixed by the token's own inputs.  Each batch first forms
+// p^- and reduces its TB sums s and dG . g at once (ds = -(dG . g) / s), then steps pb through the batch,
+// collecting the per-token parts of dr, da and dQn, and reduces those at once.  The inputs arrive through a
+// ring of kStages batches in shared memory, copied kStages - 1 batches ahead of the (backward) walk.
 template <int NPL>
 __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
-  constexpr int TB = 4;  // tokens per batch (four d_k vectors per token stay in registers)
+  constexpr int TB = 4;                    // tokens per batch
+  constexpr int RB = TB * 128 * 4;         // bytes of one array's rows in a stage
+  __shared__ __align__(16) uint8_t ks[kStages][RB];
+  __shared__ __align__(16) float spp[kStages][TB * 128], sdg[kStages][TB * 128], sdk[kStages][TB * 128];
+  __shared__ float sa[kStages][TB], sr[kStages][TB], sq[kStages][TB], sda[kStages][TB];
   const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
+  const int es = p.in_dtype == kBF16 ? 2 : 4;
   const size_t tok0 = (size_t)bh * L;
+  const int nbatch = (L + TB - 1) / TB;
+  // batches in walk order: k-th is batch nbatch - 1 - k
+  auto issue = [&](int k) {
+    if (k < nbatch) {
+      const int bi = nbatch - 1 - k, t0 = bi * TB, nb = min(TB, L - t0), st = k % kStages;
+      const size_t row0 = (tok0 + t0) * D;
+      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane);
+      copy_rows(spp[st], p.pprev + row0, nb * D * 4, lane);
+      copy_rows(sdg[st], p.dgain + row0, nb * D * 4, lane);
+      copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane);
+      if (lane < nb) {
+        const size_t ti = tok0 + t0 + lane;
+        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        cp_async4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        if (p.da != nullptr) cp_async4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
+      }
+    }
+    cp_async_commit();
+  };
+  for (int k = 0; k < kStages - 1; ++k) issue(k);
   float pb[NPL];
 #pragma unroll
   for (int e = 0; e < NPL; ++e) {
     const int i = lane + 32 * e;
     pb[e] = i < D && p.dp_L != nullptr ? p.dp_L[(size_t)bh * D + i] : 0.f;
   }
-  const int nbatch = (L + TB - 1) / TB;
-  for (int bi = nbatch - 1; bi >= 0; --bi) {
-    const int t0 = bi * TB, nb = min(TB, L - t0);
-    float sa = 1.f, sr = 1.f, sq = 0.f, sda = 0.f;
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      sa = p.a != nullptr ? p.a[ti] : 1.f, sr = p.r[ti], sq = p.qn != nullptr ? p.qn[ti] : p.qn_scalar;
-      if (p.da != nullptr) sda = p.da[ti];
-    }
+  for (int k = 0; k < nbatch; ++k) {
+    issue(k + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const int st = k % kStages, bi = nbatch - 1 - k, t0 = bi * TB, nb = min(TB, L - t0);
     float kv[TB][NPL], pp[TB][NPL], dg[TB][NPL], dko[TB][NPL];
 #pragma unroll
     for (int u = 0; u < TB; ++u)
@@ -214,47 +297,70 @@ __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
       for (int e = 0; e < NPL; ++e) {
         const int i = lane + 32 * e;
         const bool ok = u < nb && i < D;
-        const size_t off = (tok0 + t0 + u) * D + i;
-        kv[u][e] = ok ? load_elem(p.k, off, p.in_dtype) : 0.f;
-        pp[u][e] = ok ? p.pprev[off] : 0.f;
-        dg[u][e] = ok ? p.dgain[off] : 0.f;
-        dko[u][e] = ok ? p.dk[off] : 0.f;
+        kv[u][e] = ok ? smem_elem(ks[st], u * D + i, p.in_dtype) : 0.f;
+        pp[u][e] = ok ? spp[st][u * D + i] : 0.f;
+        dg[u][e] = ok ? sdg[st][u * D + i] : 0.f;
+        dko[u][e] = ok ? sdk[st][u * D + i] : 0.f;
       }
-    float dr_mine = 0.f, dqn_mine = 0.f, da_mine = sda;
+    // ---- p^-, s and ds of every token of the batch (nothing serial in them)
+    float at[TB], rt[TB], pm[TB][NPL], red[2 * TB];
+#pragma unroll
+    for (int u = 0; u < TB; ++u) {
+      const bool ok = u < nb;
+      at[u] = ok ? sa[st][u] : 1.f, rt[u] = ok ? sr[st][u] : 1.f;
+      const float qt = ok ? sq[st][u] : 0.f;
+      red[u] = 0.f;
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        const int i = lane + 32 * e;
+        pm[u][e] = i < D ? fmaf(at[u] * at[u], pp[u][e], qt) : 0.f;
+        red[u] = fmaf(pm[u][e] * kv[u][e], kv[u][e], red[u]);
+      }
+    }
+    {
+      float s4[TB];
+#pragma unroll
+      for (int u = 0; u < TB; ++u) s4[u] = red[u];
+      warp_sum_n(s4);
+#pragma unroll
+      for (int u = 0; u < TB; ++u) red[u] = __fdividef(1.f, s4[u] + rt[u]);  // 1 / s
+    }
+    {
+      float g4[TB];
+#pragma unroll
+      for (int u = 0; u < TB; ++u) {
+        g4[u] = 0.f;
+#pragma unroll
+        for (int e = 0; e < NPL; ++e) g4[u] = fmaf(dg[u][e], pm[u][e] * kv[u][e] * red[u], g4[u]);
+      }
+      warp_sum_n(g4);
+#pragma unroll
+      for (int u = 0; u < TB; ++u) red[TB + u] = -g4[u] * red[u];  // ds
+    }
+    // ---- the serial adjoint through the batch, newest token first
+    float drp[TB], dap[TB], dqp[TB];
 #pragma unroll
     for (int u = TB - 1; u >= 0; --u) {
-      const float at = __shfl_sync(0xffffffffu, sa, u), rt = __shfl_sync(0xffffffffu, sr, u);
-      const float qt = __shfl_sync(0xffffffffu, sq, u);
+      drp[u] = dap[u] = dqp[u] = 0.f;
       if (u >= nb) continue;  // uniform over the warp
-      float pm[NPL], sum = 0.f;
+      const float is = red[u], ds = red[TB + u], r = rt[u];
 #pragma unroll
       for (int e = 0; e < NPL; ++e) {
         const int i = lane + 32 * e;
-        pm[e] = i < D ? fmaf(at * at, pp[u][e], qt) : 0.f;
-        sum = fmaf(pm[e] * kv[u][e], kv[u][e], sum);
-      }
-      const float is = 1.f / (warp_sum(sum) + rt);
-      float dgg = 0.f;  // dG . g
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) dgg = fmaf(dg[u][e], pm[e] * kv[u][e] * is, dgg);
-      const float ds = -warp_sum(dgg) * is;
-      float drp = 0.f, dap = 0.f, dqp = 0.f;
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) {
-        const int i = lane + 32 * e;
-        const float k1 = kv[u][e], m1 = pm[e];
-        const float den = fmaf(m1 * k1, k1, rt), id2 = 1.f / (den * den);
-        float dpm = dg[u][e] * k1 * is + pb[e] * rt * rt * id2 + ds * k1 * k1;
-        dko[u][e] += dg[u][e] * m1 * is - 2.f * pb[e] * m1 * m1 * rt * k1 * id2 + 2.f * ds * m1 * k1;
-        drp = fmaf(pb[e] * (m1 * k1) * (m1 * k1), id2, drp);
+        const float k1 = kv[u][e], m1 = pm[u][e];
+        const float den = fmaf(m1 * k1, k1, r), id2 = __fdividef(1.f, den * den);
+        float dpm = fmaf(pb[e], r * r * id2, fmaf(dg[u][e] * k1, is, ds * k1 * k1));
+        dko[u][e] += dg[u][e] * m1 * is - 2.f * pb[e] * m1 * m1 * r * k1 * id2 + 2.f * ds * m1 * k1;
+        drp[u] = fmaf(pb[e] * (m1 * k1) * (m1 * k1), id2, drp[u]);
         if (i >= D) dpm = 0.f;
-        dap = fmaf(dpm, pp[u][e], dap);
-        dqp += dpm;
-        pb[e] = at * at * dpm;
+        dap[u] = fmaf(dpm, pp[u][e], dap[u]);
+        dqp[u] += dpm;
+        pb[e] = at[u] * at[u] * dpm;
       }
-      const float dr = warp_sum(drp) + ds, dav = warp_sum(dap), dqv = warp_sum(dqp);
-      if (lane == u) dr_mine = dr, dqn_mine = dqv, da_mine += 2.f * at * dav;
     }
+    warp_sum_n(drp);
+    warp_sum_n(dap);
+    warp_sum_n(dqp);
 #pragma unroll
     for (int u = 0; u < TB; ++u)
 #pragma unroll
@@ -262,12 +368,18 @@ __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
         const int i = lane + 32 * e;
         if (u < nb && i < D) p.dk[(tok0 + t0 + u) * D + i] = dko[u][e];
       }
+    float dr_mine = 0.f, dqn_mine = 0.f, da_mine = lane < nb ? sda[st][lane] : 0.f;
+#pragma unroll
+    for (int u = 0; u < TB; ++u)
+      if (lane == u) dr_mine = drp[u] + red[TB + u], dqn_mine = dqp[u], da_mine += 2.f * at[u] * dap[u];
     if (lane < nb) {
       const size_t ti = tok0 + t0 + lane;
       p.dr[ti] = dr_mine, p.dqn[ti] = dqn_mine;
       if (p.da != nullptr) p.da[ti] = da_mine;
     }
+    __syncwarp();  // every lane is done with this stage before it is refilled
   }
+  cp_async_wait<0>();
 #pragma unroll
   for (int e = 0; e < NPL; ++e) {
     const int i = lane + 32 * e;
