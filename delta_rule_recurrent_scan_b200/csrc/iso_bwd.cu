@@ -28,122 +28,11 @@ namespace kdn {
 
 namespace {
 
-// The chains are serial in t and bound by load latency, so each warp loads a batch of kTB tokens at once
-// (lane u < kTB the scalars of token t0 + u, every lane its coordinates of all kTB keys) and then steps
-// through the batch in registers.
+// The chains are serial in t and one warp per head has nothing else to hide load latency with: each kernel
+// takes its inputs in batches of tokens through a ring of kStages batches in shared memory, copied
+// asynchronously kStages - 1 batches ahead of the walk, and steps through a batch in registers.
 constexpr int kTB = 8;
-
-template <int NPL>
-__global__ void __launch_bounds__(32) iso_forward_kernel(IsoBwdArgs p) {
-  const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
-  const size_t tok0 = (size_t)bh * L;
-  float c = p.c0 != nullptr ? p.c0[bh] : 1.f;
-  for (int t0 = 0; t0 < L; t0 += kTB) {
-    const int nb = min(kTB, L - t0);
-    float sa = 1.f, sr = 1.f, sq = 0.f;
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      sa = p.a != nullptr ? p.a[ti] : 1.f, sr = p.r[ti], sq = p.qn != nullptr ? p.qn[ti] : p.qn_scalar;
-    }
-    float kk[kTB];
-#pragma unroll
-    for (int u = 0; u < kTB; ++u) {
-      float acc = 0.f;
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) {
-        const int i = lane + 32 * e;
-        const float x = u < nb && i < D ? load_elem(p.k, (tok0 + t0 + u) * D + i, p.in_dtype) : 0.f;
-        acc = fmaf(x, x, acc);
-      }
-      kk[u] = acc;
-    }
-#pragma unroll
-    for (int u = 0; u < kTB; ++u) kk[u] = warp_sum(kk[u]);
-    float beta_mine = 0.f, c_mine = 0.f, kk_mine = 0.f;
-#pragma unroll
-    for (int u = 0; u < kTB; ++u) {
-      const float at = __shfl_sync(0xffffffffu, sa, u), rt = __shfl_sync(0xffffffffu, sr, u);
-      const float qt = __shfl_sync(0xffffffffu, sq, u);
-      const float cm = fmaf(at * at, c, qt);
-      if (lane == u) beta_mine = cm / fmaf(cm, kk[u], rt), c_mine = c, kk_mine = kk[u];
-      if (u < nb) c = (float)D * cm * rt / fmaf((float)D, rt, cm * kk[u]);
-    }
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      p.beta[ti] = beta_mine, p.cprev[ti] = c_mine, p.knorm2[ti] = kk_mine;
-    }
-  }
-}
-
-template <int NPL>
-__global__ void __launch_bounds__(32) iso_backward_kernel(IsoBwdArgs p) {
-  const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
-  const size_t tok0 = (size_t)bh * L;
-  float cb = p.dc_L != nullptr ? p.dc_L[bh] : 0.f;
-  const float fd = (float)D;
-  const int nbatch = (L + kTB - 1) / kTB;
-  for (int bi = nbatch - 1; bi >= 0; --bi) {
-    const int t0 = bi * kTB, nb = min(kTB, L - t0);
-    float sa = 1.f, sr = 1.f, sq = 0.f, sc = 0.f, skk = 0.f, sdb = 0.f, sda = 0.f;
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      sa = p.a != nullptr ? p.a[ti] : 1.f, sr = p.r[ti], sq = p.qn != nullptr ? p.qn[ti] : p.qn_scalar;
-      sc = p.cprev[ti], skk = p.knorm2[ti], sdb = p.dbeta[ti];
-      if (p.da != nullptr) sda = p.da[ti];
-    }
-    float kv[kTB][NPL], dko[kTB][NPL];  // the batch's keys and key gradients, loaded at once
-#pragma unroll
-    for (int u = 0; u < kTB; ++u)
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) {
-        const int i = lane + 32 * e;
-        const bool ok = u < nb && i < D;
-        const size_t off = (tok0 + t0 + u) * D + i;
-        kv[u][e] = ok ? load_elem(p.k, off, p.in_dtype) : 0.f;
-        dko[u][e] = ok ? p.dk[off] : 0.f;
-      }
-    float dr_mine = 0.f, dqn_mine = 0.f, da_mine = sda, dkk_b[kTB];
-#pragma unroll
-    for (int u = kTB - 1; u >= 0; --u) {
-      const float at = __shfl_sync(0xffffffffu, sa, u), rt = __shfl_sync(0xffffffffu, sr, u);
-      const float qt = __shfl_sync(0xffffffffu, sq, u), c = __shfl_sync(0xffffffffu, sc, u);
-      const float kk = __shfl_sync(0xffffffffu, skk, u), db = __shfl_sync(0xffffffffu, sdb, u);
-      dkk_b[u] = 0.f;
-      if (u < nb) {
-        const float cm = fmaf(at * at, c, qt);
-        const float st = fmaf(cm, kk, rt), den = fmaf(fd, rt, cm * kk);
-        const float is2 = 1.f / (st * st), id2 = 1.f / (den * den);
-        const float dcm = db / st - db * cm * kk * is2 + cb * (fd * rt) * (fd * rt) * id2;
-        const float dr = -db * cm * is2 + cb * fd * cm * cm * kk * id2;
-        dkk_b[u] = -db * cm * cm * is2 - cb * fd * cm * cm * rt * id2;
-        if (lane == u) dr_mine = dr, dqn_mine = dcm, da_mine += 2.f * at * c * dcm;
-        cb = at * at * dcm;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kTB; ++u)
-#pragma unroll
-      for (int e = 0; e < NPL; ++e) {
-        const int i = lane + 32 * e;
-        if (u < nb && i < D) p.dk[(tok0 + t0 + u) * D + i] = fmaf(2.f * dkk_b[u], kv[u][e], dko[u][e]);
-      }
-    if (lane < nb) {
-      const size_t ti = tok0 + t0 + lane;
-      p.dr[ti] = dr_mine, p.dqn[ti] = dqn_mine;
-      if (p.da != nullptr) p.da[ti] = da_mine;
-    }
-  }
-  if (lane == 0) p.dc0[bh] = cb;
-}
-
-// N sums across the warp at once: the shuffle stages of the N values interleave.
-template <int N>
-__device__ __forceinline__ void warp_sum_n(float (&x)[N]) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int i = 0; i < N; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i], o);
-}
+constexpr int kStages = 4;
 
 // Asynchronous global -> shared copies for the input rings of the chain kernels below.
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
@@ -169,12 +58,153 @@ __device__ __forceinline__ float smem_elem(const uint8_t* base, int idx, int dty
                         : reinterpret_cast<const float*>(base)[idx];
 }
 
+// N sums across the warp at once: the shuffle stages of the N values interleave.
+template <int N>
+__device__ __forceinline__ void warp_sum_n(float (&x)[N]) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i], o);
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(32) iso_forward_kernel(IsoBwdArgs p) {
+  constexpr int KB = kTB * 128 * 4;
+  __shared__ __align__(16) uint8_t ks[kStages][KB];
+  __shared__ float sa[kStages][kTB], sr[kStages][kTB], sq[kStages][kTB];
+  const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
+  const int es = p.in_dtype == kBF16 ? 2 : 4;
+  const size_t tok0 = (size_t)bh * L;
+  const int nbt = (L + kTB - 1) / kTB;
+  auto issue = [&](int bt) {
+    if (bt < nbt) {
+      const int t0 = bt * kTB, nb = min(kTB, L - t0), st = bt % kStages;
+      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane);
+      if (lane < nb) {
+        const size_t ti = tok0 + t0 + lane;
+        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        cp_async4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+      }
+    }
+    cp_async_commit();
+  };
+  for (int bt = 0; bt < kStages - 1; ++bt) issue(bt);
+  float c = p.c0 != nullptr ? p.c0[bh] : 1.f;
+  for (int bt = 0; bt < nbt; ++bt) {
+    issue(bt + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const int st = bt % kStages, t0 = bt * kTB, nb = min(kTB, L - t0);
+    float kk[kTB];
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        const int i = lane + 32 * e;
+        const float x = u < nb && i < D ? smem_elem(ks[st], u * D + i, p.in_dtype) : 0.f;
+        acc = fmaf(x, x, acc);
+      }
+      kk[u] = acc;
+    }
+    warp_sum_n(kk);
+    float beta_mine = 0.f, c_mine = 0.f, kk_mine = 0.f;
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) {
+      if (u >= nb) break;
+      const float at = sa[st][u], rt = sr[st][u], qt = sq[st][u];
+      const float cm = fmaf(at * at, c, qt);
+      if (lane == u) beta_mine = cm / fmaf(cm, kk[u], rt), c_mine = c, kk_mine = kk[u];
+      c = (float)D * cm * rt / fmaf((float)D, rt, cm * kk[u]);
+    }
+    if (lane < nb) {
+      const size_t ti = tok0 + t0 + lane;
+      p.beta[ti] = beta_mine, p.cprev[ti] = c_mine, p.knorm2[ti] = kk_mine;
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(32) iso_backward_kernel(IsoBwdArgs p) {
+  constexpr int KB = kTB * 128 * 4;
+  __shared__ __align__(16) uint8_t ks[kStages][KB];
+  __shared__ __align__(16) float sdk[kStages][kTB * 128];
+  __shared__ float sa[kStages][kTB], sr[kStages][kTB], sq[kStages][kTB], sc[kStages][kTB], skk[kStages][kTB],
+      sdb[kStages][kTB], sda[kStages][kTB];
+  const int bh = blockIdx.x, lane = threadIdx.x, L = p.L, D = p.dk_dim;
+  const int es = p.in_dtype == kBF16 ? 2 : 4;
+  const size_t tok0 = (size_t)bh * L;
+  const float fd = (float)D;
+  const int nbatch = (L + kTB - 1) / kTB;
+  auto issue = [&](int k) {  // the k-th batch of the backward walk
+    if (k < nbatch) {
+      const int bi = nbatch - 1 - k, t0 = bi * kTB, nb = min(kTB, L - t0), st = k % kStages;
+      const size_t row0 = (tok0 + t0) * D;
+      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane);
+      copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane);
+      if (lane < nb) {
+        const size_t ti = tok0 + t0 + lane;
+        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        cp_async4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        cp_async4(&sc[st][lane], p.cprev + ti);
+        cp_async4(&skk[st][lane], p.knorm2 + ti);
+        cp_async4(&sdb[st][lane], p.dbeta + ti);
+        if (p.da != nullptr) cp_async4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
+      }
+    }
+    cp_async_commit();
+  };
+  for (int k = 0; k < kStages - 1; ++k) issue(k);
+  float cb = p.dc_L != nullptr ? p.dc_L[bh] : 0.f;
+  for (int k = 0; k < nbatch; ++k) {
+    issue(k + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const int st = k % kStages, bi = nbatch - 1 - k, t0 = bi * kTB, nb = min(kTB, L - t0);
+    float dr_mine = 0.f, dqn_mine = 0.f, da_mine = lane < nb ? sda[st][lane] : 0.f, dkk_b[kTB];
+#pragma unroll
+    for (int u = kTB - 1; u >= 0; --u) {
+      dkk_b[u] = 0.f;
+      if (u < nb) {
+        const float at = sa[st][u], rt = sr[st][u], qt = sq[st][u], c = sc[st][u], kk = skk[st][u], db = sdb[st][u];
+        const float cm = fmaf(at * at, c, qt);
+        const float stv = fmaf(cm, kk, rt), den = fmaf(fd, rt, cm * kk);
+        const float is2 = 1.f / (stv * stv), id2 = 1.f / (den * den);
+        const float dcm = db / stv - db * cm * kk * is2 + cb * (fd * rt) * (fd * rt) * id2;
+        const float dr = -db * cm * is2 + cb * fd * cm * cm * kk * id2;
+        dkk_b[u] = -db * cm * cm * is2 - cb * fd * cm * cm * rt * id2;
+        if (lane == u) dr_mine = dr, dqn_mine = dcm, da_mine += 2.f * at * c * dcm;
+        cb = at * at * dcm;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTB; ++u)
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        const int i = lane + 32 * e;
+        if (u < nb && i < D)
+          p.dk[(tok0 + t0 + u) * D + i] =
+              fmaf(2.f * dkk_b[u], smem_elem(ks[st], u * D + i, p.in_dtype), sdk[st][u * D + i]);
+      }
+    if (lane < nb) {
+      const size_t ti = tok0 + t0 + lane;
+      p.dr[ti] = dr_mine, p.dqn[ti] = dqn_mine;
+      if (p.da != nullptr) p.da[ti] = da_mine;
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  if (lane == 0) p.dc0[bh] = cb;
+}
+
 // Only p is serial in t (p_{t+1} = p^-_t r_t / (r_t + p^-_t k_t^2) per coordinate); the coupled sum s_t of each
 // token depends on p^-_t but nothing serial depends on s_t.  So each batch steps the per-coordinate chain over
-// its kTB tokens first, then reduces the kTB sums at once, then writes the gains.  The inputs arrive through a
-// ring of kStages batches in shared memory, copied asynchronously kStages - 1 batches ahead (one warp per
-// head has nothing else to hide the load latency with).
-constexpr int kStages = 4;
+// its kTB tokens first, then reduces the kTB sums at once, then writes the gains.  The inputs arrive through
+// the ring of kStages batches.
 
 template <int NPL>
 __global__ void __launch_bounds__(32) diag_forward_kernel(DiagBwdArgs p) {
