@@ -32,6 +32,24 @@ __device__ __forceinline__ void store_elem(void* p, size_t i, float x, int dtype
     reinterpret_cast<float*>(p)[i] = x;
 }
 
+// Asynchronous global -> shared copies (Ampere-style cp.async) for input rings.
+__device__ __forceinline__ void async_copy16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void async_copy4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// ``bytes`` (a multiple of 16, both addresses 16-byte aligned) by the threads t = 0, stride, 2 stride, ...
+__device__ __forceinline__ void async_copy_rows(void* dst, const void* src, int bytes, int t, int stride) {
+  for (int c = t; c < bytes / 16; c += stride)
+    async_copy16(static_cast<uint8_t*>(dst) + 16 * c, static_cast<const uint8_t*>(src) + 16 * c);
+}
+
 __device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
   if (status != nullptr) atomicOr(status, bits);
 }

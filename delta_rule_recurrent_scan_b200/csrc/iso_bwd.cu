@@ -34,25 +34,6 @@ namespace {
 constexpr int kTB = 8;
 constexpr int kStages = 4;
 
-// Asynchronous global -> shared copies for the input rings of the chain kernels below.
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-               "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-               "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Rows of n floats-or-bf16 (e bytes each, n e a multiple of 16) from global to shared, by the 32 lanes.
-__device__ __forceinline__ void copy_rows(void* dst, const void* src, int bytes, int lane) {
-  for (int c = lane; c < bytes / 16; c += 32)
-    cp_async16(static_cast<uint8_t*>(dst) + 16 * c, static_cast<const uint8_t*>(src) + 16 * c);
-}
-
 __device__ __forceinline__ float smem_elem(const uint8_t* base, int idx, int dtype) {
   return dtype == kBF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx])
                         : reinterpret_cast<const float*>(base)[idx];
@@ -79,21 +60,21 @@ __global__ void __launch_bounds__(32) iso_forward_kernel(IsoBwdArgs p) {
   auto issue = [&](int bt) {
     if (bt < nbt) {
       const int t0 = bt * kTB, nb = min(kTB, L - t0), st = bt % kStages;
-      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane);
+      async_copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane, 32);
       if (lane < nb) {
         const size_t ti = tok0 + t0 + lane;
-        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
-        cp_async4(&sr[st][lane], p.r + ti);
-        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        if (p.a != nullptr) async_copy4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        async_copy4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) async_copy4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
       }
     }
-    cp_async_commit();
+    async_commit();
   };
   for (int bt = 0; bt < kStages - 1; ++bt) issue(bt);
   float c = p.c0 != nullptr ? p.c0[bh] : 1.f;
   for (int bt = 0; bt < nbt; ++bt) {
     issue(bt + kStages - 1);
-    cp_async_wait<kStages - 1>();
+    async_wait<kStages - 1>();
     __syncwarp();
     const int st = bt % kStages, t0 = bt * kTB, nb = min(kTB, L - t0);
     float kk[kTB];
@@ -124,7 +105,7 @@ __global__ void __launch_bounds__(32) iso_forward_kernel(IsoBwdArgs p) {
     }
     __syncwarp();
   }
-  cp_async_wait<0>();
+  async_wait<0>();
 }
 
 template <int NPL>
@@ -143,26 +124,26 @@ __global__ void __launch_bounds__(32) iso_backward_kernel(IsoBwdArgs p) {
     if (k < nbatch) {
       const int bi = nbatch - 1 - k, t0 = bi * kTB, nb = min(kTB, L - t0), st = k % kStages;
       const size_t row0 = (tok0 + t0) * D;
-      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane);
-      copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane);
+      async_copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane, 32);
+      async_copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane, 32);
       if (lane < nb) {
         const size_t ti = tok0 + t0 + lane;
-        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
-        cp_async4(&sr[st][lane], p.r + ti);
-        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
-        cp_async4(&sc[st][lane], p.cprev + ti);
-        cp_async4(&skk[st][lane], p.knorm2 + ti);
-        cp_async4(&sdb[st][lane], p.dbeta + ti);
-        if (p.da != nullptr) cp_async4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
+        if (p.a != nullptr) async_copy4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        async_copy4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) async_copy4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        async_copy4(&sc[st][lane], p.cprev + ti);
+        async_copy4(&skk[st][lane], p.knorm2 + ti);
+        async_copy4(&sdb[st][lane], p.dbeta + ti);
+        if (p.da != nullptr) async_copy4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
       }
     }
-    cp_async_commit();
+    async_commit();
   };
   for (int k = 0; k < kStages - 1; ++k) issue(k);
   float cb = p.dc_L != nullptr ? p.dc_L[bh] : 0.f;
   for (int k = 0; k < nbatch; ++k) {
     issue(k + kStages - 1);
-    cp_async_wait<kStages - 1>();
+    async_wait<kStages - 1>();
     __syncwarp();
     const int st = k % kStages, bi = nbatch - 1 - k, t0 = bi * kTB, nb = min(kTB, L - t0);
     float dr_mine = 0.f, dqn_mine = 0.f, da_mine = lane < nb ? sda[st][lane] : 0.f, dkk_b[kTB];
@@ -197,7 +178,7 @@ __global__ void __launch_bounds__(32) iso_backward_kernel(IsoBwdArgs p) {
     }
     __syncwarp();
   }
-  cp_async_wait<0>();
+  async_wait<0>();
   if (lane == 0) p.dc0[bh] = cb;
 }
 
@@ -218,15 +199,15 @@ __global__ void __launch_bounds__(32) diag_forward_kernel(DiagBwdArgs p) {
   auto issue = [&](int bt) {
     if (bt < nbt) {
       const int t0 = bt * kTB, nb = min(kTB, L - t0), st = bt % kStages;
-      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane);
+      async_copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + (tok0 + t0) * D * es, nb * D * es, lane, 32);
       if (lane < nb) {
         const size_t ti = tok0 + t0 + lane;
-        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
-        cp_async4(&sr[st][lane], p.r + ti);
-        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        if (p.a != nullptr) async_copy4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        async_copy4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) async_copy4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
       }
     }
-    cp_async_commit();  // (an empty group past the end keeps the wait count uniform)
+    async_commit();  // (an empty group past the end keeps the wait count uniform)
   };
   for (int bt = 0; bt < kStages - 1; ++bt) issue(bt);
   float pv[NPL];
@@ -237,7 +218,7 @@ __global__ void __launch_bounds__(32) diag_forward_kernel(DiagBwdArgs p) {
   }
   for (int bt = 0; bt < nbt; ++bt) {
     issue(bt + kStages - 1);
-    cp_async_wait<kStages - 1>();  // this batch has landed
+    async_wait<kStages - 1>();  // this batch has landed
     __syncwarp();
     const int st = bt % kStages, t0 = bt * kTB, nb = min(kTB, L - t0);
     float pm[kTB][NPL], kv[kTB][NPL], sum[kTB];
@@ -270,7 +251,7 @@ __global__ void __launch_bounds__(32) diag_forward_kernel(DiagBwdArgs p) {
     }
     __syncwarp();  // every lane is done with this stage before it is refilled
   }
-  cp_async_wait<0>();
+  async_wait<0>();
 }
 
 // The adjoint pb of p is the only serial quantity backwards: pb_{t-1} = a_t^2 (c1 + pb_t c2) per coordinate,
@@ -294,19 +275,19 @@ __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
     if (k < nbatch) {
       const int bi = nbatch - 1 - k, t0 = bi * TB, nb = min(TB, L - t0), st = k % kStages;
       const size_t row0 = (tok0 + t0) * D;
-      copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane);
-      copy_rows(spp[st], p.pprev + row0, nb * D * 4, lane);
-      copy_rows(sdg[st], p.dgain + row0, nb * D * 4, lane);
-      copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane);
+      async_copy_rows(ks[st], static_cast<const uint8_t*>(p.k) + row0 * es, nb * D * es, lane, 32);
+      async_copy_rows(spp[st], p.pprev + row0, nb * D * 4, lane, 32);
+      async_copy_rows(sdg[st], p.dgain + row0, nb * D * 4, lane, 32);
+      async_copy_rows(sdk[st], p.dk + row0, nb * D * 4, lane, 32);
       if (lane < nb) {
         const size_t ti = tok0 + t0 + lane;
-        if (p.a != nullptr) cp_async4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
-        cp_async4(&sr[st][lane], p.r + ti);
-        if (p.qn != nullptr) cp_async4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
-        if (p.da != nullptr) cp_async4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
+        if (p.a != nullptr) async_copy4(&sa[st][lane], p.a + ti); else sa[st][lane] = 1.f;
+        async_copy4(&sr[st][lane], p.r + ti);
+        if (p.qn != nullptr) async_copy4(&sq[st][lane], p.qn + ti); else sq[st][lane] = p.qn_scalar;
+        if (p.da != nullptr) async_copy4(&sda[st][lane], p.da + ti); else sda[st][lane] = 0.f;
       }
     }
-    cp_async_commit();
+    async_commit();
   };
   for (int k = 0; k < kStages - 1; ++k) issue(k);
   float pb[NPL];
@@ -317,7 +298,7 @@ __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
   }
   for (int k = 0; k < nbatch; ++k) {
     issue(k + kStages - 1);
-    cp_async_wait<kStages - 1>();
+    async_wait<kStages - 1>();
     __syncwarp();
     const int st = k % kStages, bi = nbatch - 1 - k, t0 = bi * TB, nb = min(TB, L - t0);
     float kv[TB][NPL], pp[TB][NPL], dg[TB][NPL], dko[TB][NPL];
@@ -409,7 +390,7 @@ __global__ void __launch_bounds__(32) diag_backward_kernel(DiagBwdArgs p) {
     }
     __syncwarp();  // every lane is done with this stage before it is refilled
   }
-  cp_async_wait<0>();
+  async_wait<0>();
 #pragma unroll
   for (int e = 0; e < NPL; ++e) {
     const int i = lane + 32 * e;

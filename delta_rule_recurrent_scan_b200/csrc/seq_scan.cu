@@ -23,6 +23,16 @@ namespace kdn {
 
 constexpr int kTokBlock = 16;  // tokens staged in shared memory at a time
 
+// Raw inputs of one token block in shared memory (the per-token kernel's two-stage ring, copied
+// asynchronously one block ahead): k, q ([16][DK], bf16 or fp32 as given), v ([16][DV]), gains ([16][DK] fp32,
+// Kalman), a and beta ([16] each).  Sized for fp32 inputs.
+template <int DK, int DV, bool kGains>
+struct RawStage {
+  static constexpr int K = 0, Q = K + kTokBlock * DK * 4, V = Q + kTokBlock * DK * 4, G = V + kTokBlock * DV * 4;
+  static constexpr int A = G + (kGains ? kTokBlock * DK * 4 : 0), B = A + kTokBlock * 4;
+  static constexpr int BYTES = B + kTokBlock * 4;
+};
+
 template <int DK, int DV, bool kGainsFromWs>
 __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_kernel(SeqScanArgs args) {
   using Lay = RowBlockLayout<DK, DV>;
@@ -52,9 +62,34 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
     S[i][0] = x.x, S[i][1] = x.y, S[i][2] = x.z, S[i][3] = x.w;
   }
 
+  // the raw inputs of block b + 1 are copied while block b runs
+  using RS = RawStage<DK, DV, kGainsFromWs>;
+  extern __shared__ __align__(16) uint8_t raw[];
+  const int es = args.in_dtype == kBF16 ? 2 : 4;
+  const int nblk = (L + kTokBlock - 1) / kTokBlock;
+  auto issue = [&](int blk) {
+    if (blk < nblk) {
+      const int t0 = blk * kTokBlock, nt = min(kTokBlock, L - t0);
+      uint8_t* st = raw + (blk & 1) * RS::BYTES;
+      async_copy_rows(st + RS::K, static_cast<const uint8_t*>(args.k) + (tok0 + t0) * DK * es, nt * DK * es, tid, NT);
+      async_copy_rows(st + RS::Q, static_cast<const uint8_t*>(args.q) + (tok0 + t0) * DK * es, nt * DK * es, tid, NT);
+      async_copy_rows(st + RS::V, static_cast<const uint8_t*>(args.v) + (tok0 + t0) * DV * es, nt * DV * es, tid, NT);
+      if constexpr (kGainsFromWs) async_copy_rows(st + RS::G, args.gains + (tok0 + t0) * DK, nt * DK * 4, tid, NT);
+      if (tid < nt) {
+        float* sa_ = reinterpret_cast<float*>(st + RS::A);
+        float* sb_ = reinterpret_cast<float*>(st + RS::B);
+        if (args.a != nullptr) async_copy4(sa_ + tid, args.a + tok0 + t0 + tid); else sa_[tid] = 1.f;
+        if (!kGainsFromWs) async_copy4(sb_ + tid, args.beta + tok0 + t0 + tid); else sb_[tid] = 0.f;
+      }
+    }
+    async_commit();
+  };
+  issue(0);
+
   const int nck = args.S_ckpt != nullptr ? (L + args.ckpt_every - 1) / args.ckpt_every : 0;
   for (int t0 = 0; t0 < L; t0 += kTokBlock) {
     const int nt = min(kTokBlock, L - t0);
+    const int blk = t0 / kTokBlock;
     if (nck > 0 && t0 % args.ckpt_every == 0) {  // the state entering this checkpoint chunk
       float* Sc = args.S_ckpt + ((size_t)bh * nck + t0 / args.ckpt_every) * DK * DV;
 #pragma unroll
@@ -62,21 +97,26 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
         *reinterpret_cast<float4*>(Sc + (size_t)(rg + i * RG) * DV + cg * 4) =
             make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
     }
-    __syncthreads();
-    for (int idx = tid; idx < nt * DK; idx += NT) {
-      const int j = idx / DK, i = idx % DK;
-      const size_t off = (tok0 + t0 + j) * DK + i;
-      k_s[j][i] = load_elem(args.k, off, args.in_dtype);
-      q_s[j][i] = load_elem(args.q, off, args.in_dtype);
-      if constexpr (kGainsFromWs) g_s[j][i] = args.gains[off];
-    }
-    for (int idx = tid; idx < nt * DV; idx += NT) {
-      const int j = idx / DV, i = idx % DV;
-      v_s[j][i] = load_elem(args.v, (tok0 + t0 + j) * DV + i, args.in_dtype);
-    }
-    for (int j = tid; j < nt; j += NT) {
-      a_s[j] = args.a ? args.a[tok0 + t0 + j] : 1.f;
-      b_s[j] = kGainsFromWs ? 0.f : args.beta[tok0 + t0 + j];
+    issue(blk + 1);
+    async_wait<1>();
+    __syncthreads();  // this block's raw inputs are in; the previous block's staged floats are no longer read
+    {
+      const uint8_t* st = raw + (blk & 1) * RS::BYTES;
+      auto elem = [&](int off, int idx) {
+        return args.in_dtype == kBF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(st + off)[idx])
+                                      : reinterpret_cast<const float*>(st + off)[idx];
+      };
+      for (int idx = tid; idx < nt * DK; idx += NT) {
+        const int j = idx / DK, i = idx % DK;
+        k_s[j][i] = elem(RS::K, idx);
+        q_s[j][i] = elem(RS::Q, idx);
+        if constexpr (kGainsFromWs) g_s[j][i] = reinterpret_cast<const float*>(st + RS::G)[idx];
+      }
+      for (int idx = tid; idx < nt * DV; idx += NT) v_s[idx / DV][idx % DV] = elem(RS::V, idx);
+      for (int j = tid; j < nt; j += NT) {
+        a_s[j] = reinterpret_cast<const float*>(st + RS::A)[j];
+        b_s[j] = reinterpret_cast<const float*>(st + RS::B)[j];
+      }
     }
     __syncthreads();
     for (int j = warp; j < nt; j += NW) {
@@ -142,6 +182,7 @@ __global__ void __launch_bounds__(RowBlockLayout<DK, DV>::kThreads) seq_scan_ker
       }
     }
   }
+  async_wait<0>();
 #pragma unroll
   for (int i = 0; i < RPT; ++i)
     *reinterpret_cast<float4*>(Sg + (size_t)(rg + i * RG) * DV + cg * 4) = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
@@ -306,10 +347,17 @@ cudaError_t launch_seq_scan(int dk, int dv, const SeqScanArgs& args, cudaStream_
   if (args.BH <= 0 || args.L <= 0) return cudaSuccess;
   KDN_DIMS_SWITCH(dk, DK, KDN_DIMS_SWITCH(dv, DV, {
     constexpr int NT = RowBlockLayout<DK, DV>::kThreads;
-    if (args.gains != nullptr)
-      seq_scan_kernel<DK, DV, true><<<args.BH, NT, 0, stream>>>(args);
-    else
-      seq_scan_kernel<DK, DV, false><<<args.BH, NT, 0, stream>>>(args);
+    if (args.gains != nullptr) {
+      constexpr int smem = 2 * RawStage<DK, DV, true>::BYTES;
+      cudaError_t e = cudaFuncSetAttribute(seq_scan_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      seq_scan_kernel<DK, DV, true><<<args.BH, NT, smem, stream>>>(args);
+    } else {
+      constexpr int smem = 2 * RawStage<DK, DV, false>::BYTES;
+      cudaError_t e = cudaFuncSetAttribute(seq_scan_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      seq_scan_kernel<DK, DV, false><<<args.BH, NT, smem, stream>>>(args);
+    }
   }));
   return cudaGetLastError();
 }
