@@ -126,7 +126,13 @@ struct BwdSmem {
   static constexpr int VEC = DW + DK * LC;        // per-token vectors of kCB floats (see the kernel)
   static constexpr int NVEC = 12;
   static constexpr int GC = VEC + NVEC * kCB + 32; // general gains: the chunk's G [kCB][LK]
-  static constexpr int TOTAL = GC + (GEN ? kCB * LK : 0);
+  static constexpr int RAW = (GC + (GEN ? kCB * LK : 0) + 3) / 4 * 4;  // the next chunk's inputs as copied
+  // raw stage (in floats from RAW): K, Q [kCB][DK] and V [kCB][JB] as bf16 (fp32 inputs are read directly),
+  // dO [kCB][JB], S0 [DK][JB], then a, beta, dm and ||e|| [kCB] each
+  static constexpr int RK = 0, RQ = RK + kCB * DK / 2, RV = RQ + kCB * DK / 2, RO = RV + kCB * JB / 2;
+  static constexpr int RS = RO + kCB * JB;
+  static constexpr int RA = RS + DK * JB, RB = RA + kCB, RM = RB + kCB, RE = RM + kCB, RAW_FLOATS = RE + kCB;
+  static constexpr int TOTAL = RAW + RAW_FLOATS;
   static constexpr size_t BYTES = TOTAL * sizeof(float);
 };
 
@@ -188,42 +194,80 @@ __global__ void __launch_bounds__(kBwdThreads, 1) delta_bwd_kernel(DeltaBwdArgs 
     dS[kk * LJ + j] = p.dS_L != nullptr ? p.dS_L[((size_t)bh * DK + kk) * DV + j0 + j] : 0.f;
   }
 
+  // The inputs of chunk c - 1 are copied asynchronously into the raw stage while chunk c is worked on (the
+  // walk is backwards); each chunk starts by spreading its stage into the padded working layouts.
+  float* raw = sm + Lay::RAW;
+  const bool raw_in = p.in_dtype == kBF16;  // bf16 keys, queries, values go through the stage
+  auto issue = [&](int cc) {
+    if (cc >= 0) {
+      const int u0 = cc * C, nn = min(C, L - u0);
+      const int och = JB * 4 / 16;  // 16-byte pieces of one fp32 row's column block
+      if (raw_in) {
+        const uint8_t* kb = static_cast<const uint8_t*>(p.k) + (tok0 + u0) * DK * 2;
+        const uint8_t* qb = static_cast<const uint8_t*>(p.q) + (tok0 + u0) * DK * 2;
+        async_copy_rows(raw + Lay::RK, kb, nn * DK * 2, tid, NT);
+        async_copy_rows(raw + Lay::RQ, qb, nn * DK * 2, tid, NT);
+        const int vch = JB * 2 / 16;
+        for (int idx = tid; idx < nn * vch; idx += NT) {
+          const int i = idx / vch, q = idx % vch;
+          async_copy16(reinterpret_cast<uint8_t*>(raw + Lay::RV) + (size_t)i * JB * 2 + 16 * q,
+                       static_cast<const uint8_t*>(p.v) + ((tok0 + u0 + i) * DV + j0) * 2 + 16 * q);
+        }
+      }
+      for (int idx = tid; idx < nn * och; idx += NT) {
+        const int i = idx / och, q = idx % och;
+        async_copy16(raw + Lay::RO + i * JB + 4 * q, p.dO + (tok0 + u0 + i) * DV + j0 + 4 * q);
+      }
+      for (int idx = tid; idx < DK * och; idx += NT) {
+        const int kk = idx / och, q = idx % och;
+        async_copy16(raw + Lay::RS + kk * JB + 4 * q, p.S_ckpt + (((size_t)bh * nck + cc) * DK + kk) * DV + j0 + 4 * q);
+      }
+      if (tid < nn) {
+        const size_t ti = tok0 + u0 + tid;
+        if (p.a != nullptr) async_copy4(raw + Lay::RA + tid, p.a + ti); else raw[Lay::RA + tid] = 1.f;
+        if (!GEN) async_copy4(raw + Lay::RB + tid, p.beta + ti); else raw[Lay::RB + tid] = 1.f;
+        if (p.dm != nullptr) async_copy4(raw + Lay::RM + tid, p.dm + ti); else raw[Lay::RM + tid] = 0.f;
+        async_copy4(raw + Lay::RE + tid, p.enorm + ti);
+      }
+    }
+    async_commit();
+  };
+  auto raw_bf16 = [&](int off, int idx) { return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw + off)[idx]); };
+  issue(nck - 1);
+
   for (int c = nck - 1; c >= 0; --c) {
     const int t0 = c * C, n = min(C, L - t0);
-    __syncthreads();  // the previous chunk is done with every buffer
+    async_wait<0>();
+    __syncthreads();  // this chunk's inputs are in, and the previous chunk is done with every buffer
     // ------------------------------------------------------------------ inputs of the chunk (zero past L)
     for (int idx = tid; idx < C * DK; idx += NT) {
       const int i = idx / DK, kk = idx % DK;
       const bool ok = i < n;
       const size_t off = (tok0 + t0 + i) * DK + kk;
-      Kc[i * LK + kk] = ok ? load_elem(p.k, off, p.in_dtype) : 0.f;
-      Qc[i * LK + kk] = ok ? load_elem(p.q, off, p.in_dtype) : 0.f;
+      Kc[i * LK + kk] = ok ? (raw_in ? raw_bf16(Lay::RK, idx) : load_elem(p.k, off, p.in_dtype)) : 0.f;
+      Qc[i * LK + kk] = ok ? (raw_in ? raw_bf16(Lay::RQ, idx) : load_elem(p.q, off, p.in_dtype)) : 0.f;
       if (GEN) Gc[i * LK + kk] = ok ? p.gains[off] : 0.f;
     }
     for (int idx = tid; idx < C * JB; idx += NT) {
       const int i = idx / JB, j = idx % JB;
       const bool ok = i < n;
-      const size_t off = (tok0 + t0 + i) * DV + j0 + j;
-      Vc[i * LJ + j] = ok ? load_elem(p.v, off, p.in_dtype) : 0.f;
-      dOc[i * LJ + j] = ok ? p.dO[off] : 0.f;
+      Vc[i * LJ + j] = ok ? (raw_in ? raw_bf16(Lay::RV, idx) : load_elem(p.v, (tok0 + t0 + i) * DV + j0 + j, p.in_dtype))
+                          : 0.f;
+      dOc[i * LJ + j] = ok ? raw[Lay::RO + idx] : 0.f;
     }
-    for (int idx = tid; idx < DK * JB; idx += NT) {
-      const int kk = idx / JB, j = idx % JB;
-      S0[kk * LJ + j] = p.S_ckpt[(((size_t)bh * nck + c) * DK + kk) * DV + j0 + j];
-    }
+    for (int idx = tid; idx < DK * JB; idx += NT) S0[(idx / JB) * LJ + idx % JB] = raw[Lay::RS + idx];
     if (tid < C) {
       const int i = tid;
       const bool ok = i < n;
-      const size_t ti = tok0 + t0 + i;
-      const float a = ok ? (p.a != nullptr ? p.a[ti] : 1.f) : 1.f;
-      va[i] = a;
-      vb[i] = GEN ? 1.f : (ok ? p.beta[ti] : 0.f);
-      vdm[i] = ok && p.dm != nullptr ? p.dm[ti] : 0.f;
-      ven[i] = ok ? p.enorm[ti] : 0.f;
+      va[i] = ok ? raw[Lay::RA + i] : 1.f;
+      vb[i] = GEN ? 1.f : (ok ? raw[Lay::RB + i] : 0.f);
+      vdm[i] = ok ? raw[Lay::RM + i] : 0.f;
+      ven[i] = ok ? raw[Lay::RE + i] : 0.f;
       vdA[i] = 0.f, vdr[i] = 0.f, vdb[i] = 0.f;
     }
     if (tid == 0) vmisc[0] = 0.f;
     __syncthreads();
+    issue(c - 1);  // the stage is free again
     // ------------------------------------------------------------------ gates (warp 0), key norms (all warps)
     if (warp == 0) {
       // ell (for the ratios Gam_ij = exp(ell_i - ell_j), a gate of 0 floored at e^-60 there), and A_i, r_j as
