@@ -114,8 +114,9 @@ typedef struct kdn_dims {
  *     full Kalman: the covariance side runs over the whole sequence first (it is not a per-coordinate
  *     map), giving every token's gain;
  *   - the chunk kernel runs all segments from S0 = 0 and from S0 = I (giving each segment's map
- *     S0 -> M S0 + B), one fp32 pass per head chains the segment start states, and a last chunk-kernel
- *     run from the true start states writes o, m and the final state.
+ *     S0 -> M S0 + B; at d = 64 one run on the d x 2d state [S | M] from [0 | I] gives both), one fp32
+ *     pass per head chains the segment start states, and a last chunk-kernel run from the true start
+ *     states writes o, m and the final state.
  * Results equal the serial scan's up to rounding.  The library choice (segments = 0) is P in {16, 8, 4}
  * (the largest with B*H*P <= 148, L % (64 P) == 0 and at least two chunks per segment), else 1.  The
  * workspace grows by 3 B*H*P*dk*dv floats (plus 7 B*H*P*dk for the diagonal variant) when P > 1. */
