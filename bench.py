@@ -97,7 +97,7 @@ NCU_TRAFFIC = {
     "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
                         "bytes_per_token": (308.401664e6 + 170.171648e6) / _B3,
                         "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "d820f760ed0db550e9296bf73652a633f75682fa",
+    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "957f2e01392f7d5107da534f246864810121e84f",
                          "bytes_per_token": (31.137024e6 + 0.194560e6) / (2 * 8 * 4096),
                          "capture": "ncu, riccati_chain_tc_kernel at the full workload B=2 H=8 L=4096"},
 }
