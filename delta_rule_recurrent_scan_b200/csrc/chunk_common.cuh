@@ -87,6 +87,58 @@ __device__ __forceinline__ float oct_sum(float x) {
   return x;
 }
 
+// One m16n8k8 warp-level tensor-core product with tf32 operands and fp32 accumulation: d += a b.  The
+// operands are fp32 bit patterns, of which the unit reads the sign, exponent and 10 leading mantissa bits.
+// Fragments, with g = lane / 4 and t = lane % 4: a = A[g][t], A[g + 8][t], A[g][t + 4], A[g + 8][t + 4];
+// b = B[t][g], B[t + 4][g]; d = D[g][2 t], D[g][2 t + 1], D[g + 8][2 t], D[g + 8][2 t + 1].
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// x = hi + lo with hi the leading 19 bits (sign, exponent, 10 mantissa bits) and lo = x - hi exactly.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = __float_as_uint(x) & 0xffffe000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+// acc = A B for one 16 x 8 tile over KS steps of 8 along k (from k0): A points at the tile's row 0, B at
+// its column 0, both fp32 row-major with row stride kLD in shared memory.  Every operand is split as
+// hi + lo and the product taken as hi hi + (hi lo + lo hi): the dropped lo lo term and the tf32 reading of
+// lo leave about 2^-20 of |A| |B|, against 2^-11 for a single tf32 product.  Run by a whole warp.
+template <int KS>
+__device__ __forceinline__ void tile_mma_x3(const float* A, const float* B, int k0, float (&acc)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float hh[4] = {0.f, 0.f, 0.f, 0.f}, cr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s = 0; s < KS; ++s) {
+    const int k = k0 + 8 * s;
+    const float av[4] = {A[g * kLD + k + t], A[(g + 8) * kLD + k + t], A[g * kLD + k + t + 4],
+                         A[(g + 8) * kLD + k + t + 4]};
+    const float bv[2] = {B[(k + t) * kLD + g], B[(k + t + 4) * kLD + g]};
+    uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) split_tf32(av[e], ah[e], al[e]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) split_tf32(bv[e], bh[e], bl[e]);
+    mma_tf32_16x8x8(hh, ah, bh);
+    mma_tf32_16x8x8(cr, ah, bl);
+    mma_tf32_16x8x8(cr, al, bh);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] = hh[e] + cr[e];
+}
+
+// scale * acc into the 16 x 8 tile at D (row stride kLD), in the fragment layout of mma_tf32_16x8x8.
+__device__ __forceinline__ void store_tile(float* D, const float (&acc)[4], float scale) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2*>(D + g * kLD + 2 * t) = make_float2(scale * acc[0], scale * acc[1]);
+  *reinterpret_cast<float2*>(D + (g + 8) * kLD + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
+}
+
 // T = (I + N)^-1 for a 64 x 64 strictly lower N (fp32, row stride kLD; only the strict lower part of N
 // is read).  T's lower part is written to Tf (its unit diagonal and the zeros above it inside the 16 x 16
 // diagonal blocks too); the other upper blocks of Tf are scratch.  Run by the 256 threads gt = 0..255 of
@@ -94,7 +146,10 @@ __device__ __forceinline__ float oct_sum(float x) {
 //   (1) diagonal blocks T_bb = (I + N_bb)^-1 by forward substitution, one thread per column;
 //   (2) 16 -> 32: T_{b+1,b} = -T_{b+1,b+1} (N_{b+1,b} T_bb) for b = 0, 2;
 //   (3) 32 -> 64: T_{[23],[01]} = -T_{[23],[23]} (N_{[23],[01]} T_{[01],[01]}),
-// the block form of the inverse of [[X, 0], [Y, Z]] at each doubling.
+// the block form of the inverse of [[X, 0], [Y, Z]] at each doubling.  The products of (2) and (3) run as
+// warp-level tf32 tensor-core products split three ways (tile_mma_x3), one 16 x 8 output tile per warp: the
+// tiles are too small for a tcgen05 round trip through shared and tensor memory, and on the fp32 pipe half the
+// group waited on the other half's 32-term dot products.
 template <class Sync>
 __device__ __forceinline__ void invert_unit_lower_64(const float* Nf, float* Tf, int gt, Sync sync) {
   constexpr int LD = kLD;
@@ -122,99 +177,49 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* Nf, float* Tf,
     for (int i = 0; i < 16; ++i) Tb[i * LD + cc] = t[i];
   }
   sync();
-  // (2) pairs (a, b) = (1, 0), (3, 2): M = N_ab T_bb parked in the upper block (b, a), then T_ab = -T_aa M
+  // (2) pairs (a, b) = (1, 0), (3, 2): M = N_ab T_bb parked in the upper block (b, a), then T_ab = -T_aa M;
+  // warps 0..3 take pair w / 2, columns 8 (w % 2) ..
+  const int w = gt >> 5;
   {
-    const int pr = gt >> 6, i = (gt >> 2) & 15, jq = gt & 3;
+    const int pr = w >> 1, n0 = 8 * (w & 1);
     const int a = 2 * pr + 1, b = 2 * pr;
-    if (gt < 128) {
-      float nv[16];
-#pragma unroll
-      for (int l = 0; l < 16; l += 4) {
-        const float4 n4 = *reinterpret_cast<const float4*>(Nf + (16 * a + i) * LD + 16 * b + l);
-        nv[l] = n4.x, nv[l + 1] = n4.y, nv[l + 2] = n4.z, nv[l + 3] = n4.w;
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * b + k) * LD + 16 * b + 4 * jq);
-        acc.x = fmaf(nv[k], t4.x, acc.x), acc.y = fmaf(nv[k], t4.y, acc.y);
-        acc.z = fmaf(nv[k], t4.z, acc.z), acc.w = fmaf(nv[k], t4.w, acc.w);
-      }
-      *reinterpret_cast<float4*>(Tf + (16 * b + i) * LD + 16 * a + 4 * jq) = acc;
+    if (w < 4) {
+      float acc[4];
+      tile_mma_x3<2>(Nf + (16 * a) * LD + 16 * b, Tf + (16 * b) * LD + 16 * b + n0, 0, acc);
+      store_tile(Tf + (16 * b) * LD + 16 * a + n0, acc, 1.f);
     }
     sync();
-    if (gt < 128) {
-      float tv[16];
-#pragma unroll
-      for (int l = 0; l < 16; l += 4) {
-        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (16 * a + i) * LD + 16 * a + l);
-        tv[l] = t4.x, tv[l + 1] = t4.y, tv[l + 2] = t4.z, tv[l + 3] = t4.w;
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float4 m4 = *reinterpret_cast<const float4*>(Tf + (16 * b + k) * LD + 16 * a + 4 * jq);
-        acc.x = fmaf(tv[k], m4.x, acc.x), acc.y = fmaf(tv[k], m4.y, acc.y);
-        acc.z = fmaf(tv[k], m4.z, acc.z), acc.w = fmaf(tv[k], m4.w, acc.w);
-      }
-      *reinterpret_cast<float4*>(Tf + (16 * a + i) * LD + 16 * b + 4 * jq) =
-          make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    if (w < 4) {
+      float acc[4];
+      tile_mma_x3<2>(Tf + (16 * a) * LD + 16 * a, Tf + (16 * b) * LD + 16 * a + n0, 0, acc);
+      store_tile(Tf + (16 * a) * LD + 16 * b + n0, acc, -1.f);
     }
     sync();
   }
   // (3) X = N_{[23],[01]} T_{[01],[01]} parked in rows 0..31, columns 32..63; then the lower-left 32 x 32
-  // block of T = -T_{[23],[23]} X.  Threads 0..127 each take rows {r, r + 16} x four columns (register
-  // tiles halve the shared-memory reads of the broadcast operand); warps take uniform column ranges.
+  // block of T = -T_{[23],[23]} X.  Warp w < 8 takes rows 16 (w / 4) .., columns 8 (w % 4) .. of each product.
+  // Blocks that hold parked products instead of zeros are skipped: T_{[01],[01]} rows 0..15 past column 15
+  // (M of the pair (1, 0)), and T_{[23],[23]} rows 32..47 past column 47 (M of the pair (3, 2)).
   {
-    const int u = gt & 127;
-    if (gt < 128) {
-      const int jh = u >> 6, r = (u >> 2) & 15, j0 = 16 * jh + 4 * (u & 3);
-      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-#pragma unroll
-      for (int kb = 0; kb < 32; kb += 4) {
-        if (kb < 16 * jh) continue;  // T_{[01],[01]}[k][j] = 0 for k < 16 <= j
-        const float4 na = *reinterpret_cast<const float4*>(Nf + (32 + r) * LD + kb);
-        const float4 nb = *reinterpret_cast<const float4*>(Nf + (48 + r) * LD + kb);
-        const float n0[4] = {na.x, na.y, na.z, na.w}, n1[4] = {nb.x, nb.y, nb.z, nb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 t4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + j0);
-          acc0.x = fmaf(n0[e], t4.x, acc0.x), acc0.y = fmaf(n0[e], t4.y, acc0.y);
-          acc0.z = fmaf(n0[e], t4.z, acc0.z), acc0.w = fmaf(n0[e], t4.w, acc0.w);
-          acc1.x = fmaf(n1[e], t4.x, acc1.x), acc1.y = fmaf(n1[e], t4.y, acc1.y);
-          acc1.z = fmaf(n1[e], t4.z, acc1.z), acc1.w = fmaf(n1[e], t4.w, acc1.w);
-        }
+    const int mt = (w >> 2) & 1, n0 = 8 * (w & 3);
+    if (w < 8) {
+      float acc[4];
+      if (n0 >= 16) {
+        tile_mma_x3<2>(Nf + (32 + 16 * mt) * LD + 16, Tf + 16 * LD + n0, 0, acc);
+      } else {
+        tile_mma_x3<4>(Nf + (32 + 16 * mt) * LD, Tf + n0, 0, acc);
       }
-      *reinterpret_cast<float4*>(Tf + r * LD + 32 + j0) = acc0;
-      *reinterpret_cast<float4*>(Tf + (16 + r) * LD + 32 + j0) = acc1;
+      store_tile(Tf + (16 * mt) * LD + 32 + n0, acc, 1.f);
     }
     sync();
-    if (gt < 128) {
-      const int r = u >> 3, j0 = 4 * (u & 7);
-      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-#pragma unroll
-      for (int kb = 0; kb < 32; kb += 4) {
-        // row r of T_{[23],[23]} is zero past column 15; row 16 + r runs to column 31
-        float t0v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (kb < 16) {
-          const float4 ta = *reinterpret_cast<const float4*>(Tf + (32 + r) * LD + 32 + kb);
-          t0v[0] = ta.x, t0v[1] = ta.y, t0v[2] = ta.z, t0v[3] = ta.w;
-        }
-        const float4 tb = *reinterpret_cast<const float4*>(Tf + (48 + r) * LD + 32 + kb);
-        const float t1v[4] = {tb.x, tb.y, tb.z, tb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 x4 = *reinterpret_cast<const float4*>(Tf + (kb + e) * LD + 32 + j0);
-          if (kb < 16) {
-            acc0.x = fmaf(t0v[e], x4.x, acc0.x), acc0.y = fmaf(t0v[e], x4.y, acc0.y);
-            acc0.z = fmaf(t0v[e], x4.z, acc0.z), acc0.w = fmaf(t0v[e], x4.w, acc0.w);
-          }
-          acc1.x = fmaf(t1v[e], x4.x, acc1.x), acc1.y = fmaf(t1v[e], x4.y, acc1.y);
-          acc1.z = fmaf(t1v[e], x4.z, acc1.z), acc1.w = fmaf(t1v[e], x4.w, acc1.w);
-        }
+    if (w < 8) {
+      float acc[4];
+      if (mt == 0) {
+        tile_mma_x3<2>(Tf + 32 * LD + 32, Tf + 32 + n0, 0, acc);
+      } else {
+        tile_mma_x3<4>(Tf + 48 * LD + 32, Tf + 32 + n0, 0, acc);
       }
-      *reinterpret_cast<float4*>(Tf + (32 + r) * LD + j0) = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
-      *reinterpret_cast<float4*>(Tf + (48 + r) * LD + j0) = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
+      store_tile(Tf + (32 + 16 * mt) * LD + n0, acc, -1.f);
     }
     sync();
   }
