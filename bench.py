@@ -86,18 +86,18 @@ _RICCATI_SOURCES = ["delta_rule_recurrent_scan_b200/csrc/riccati.cu",
                     "delta_rule_recurrent_scan_b200/csrc/sm100.cuh",
                     "delta_rule_recurrent_scan_b200/csrc/common.cuh"]
 _B3 = 3 * 16 * 8192  # tokens of the reduced capture (B = 3 keeps one segment per head)
-_WS_SHA = "f1d52692d9aa476369052689f14393df8bddf887"
+_WS_SHA = "913c18f440d3d0df7e31a9fe0288d4cc5e0a0097"
 NCU_TRAFFIC = {
     "kalman_diag_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                         "bytes_per_token": (308.433408e6 + 172.305664e6) / _B3,
+                         "bytes_per_token": (308.486912e6 + 170.518272e6) / _B3,
                          "capture": "ncu, chunk_scan_ws_kernel<diag> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "gdn_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                 "bytes_per_token": (308.394240e6 + 172.547584e6) / _B3,
+                 "bytes_per_token": (308.391680e6 + 170.423808e6) / _B3,
                  "capture": "ncu, chunk_scan_ws_kernel<delta> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
     "kalman_iso_d128": {"sources": _WS_SOURCES, "sha1": _WS_SHA,
-                        "bytes_per_token": (308.401664e6 + 170.171648e6) / _B3,
+                        "bytes_per_token": (308.401664e6 + 172.895488e6) / _B3,
                         "capture": "ncu, chunk_scan_ws_kernel<iso> at B=3 H=16 L=8192, per-token bytes scaled to the launch"},
-    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "957f2e01392f7d5107da534f246864810121e84f",
+    "kalman_full_d128": {"sources": _RICCATI_SOURCES, "sha1": "c3a61774284b0bdb56eeaa3f4bd8987e544152b7",
                          "bytes_per_token": (31.137024e6 + 0.194560e6) / (2 * 8 * 4096),
                          "capture": "ncu, riccati_chain_tc_kernel at the full workload B=2 H=8 L=4096"},
 }
