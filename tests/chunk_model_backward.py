@@ -370,3 +370,54 @@ def chunk_full_backward(q, k, v, r, a, qn, C, dO, S0=None, P0=None, dm=None, dS_
         dP = dP0
     out["dS0"], out["dP0"] = dS, 0.5 * (dP + dP.T)
     return out
+
+
+def full_cov_backward_tokens(k, r, a, qn, P0, dg, dP_L=None, block=64):
+    """Full-covariance Kalman, one head: the covariance side of the backward token by token, as the CUDA
+    kernels take it, for the gains' upstream gradient dg [L, d_k] from the memory backward.
+
+    The forward P^- = a^2 P + Qn I, u = P^- k, s = k^T u + r, g = u / s, P <- P^- - u u^T / s keeps P at every
+    block start; the backward recomputes each block's P, u, s from its checkpoint and walks it in reverse.
+    Instead of the covariance adjoint Pb it carries M = Pb + Pb^T, which is enough while P is symmetric:
+    (Pb + Pb^T) u = M u, u^T Pb u = u^T M u / 2, <Pb, P> = <M, P> / 2, tr Pb = tr M / 2, and
+    Pb <- a^2 (Pb + du k^T) becomes the symmetric M <- a^2 (M + du k^T + k du^T).  Returns the covariance
+    side's key and gate terms (dk, da: to be added to the memory backward's), dr, dqn and dP0 = M_0 / 2, the
+    gradient with respect to a symmetric P0."""
+    L, d = k.shape
+    eye = np.eye(d)
+    P = np.array(P0, float)
+    ckpt = []
+    for t in range(L):
+        if t % block == 0:
+            ckpt.append(P.copy())
+        Pm = a[t] ** 2 * P + qn[t] * eye
+        u = Pm @ k[t]
+        P = Pm - np.outer(u, u) / (k[t] @ u + r[t])
+    M = np.zeros((d, d)) if dP_L is None else np.array(dP_L, float) + np.array(dP_L, float).T
+    trM = np.trace(M)
+    out = {key: np.zeros(shape) for key, shape in (("dk", (L, d)), ("da", L), ("dr", L), ("dqn", L))}
+    for b in range(len(ckpt) - 1, -1, -1):
+        t0, t1 = b * block, min(L, (b + 1) * block)
+        P = ckpt[b].copy()
+        Pp, U, S = [], [], []
+        for t in range(t0, t1):
+            Pp.append(P)
+            Pm = a[t] ** 2 * P + qn[t] * eye
+            u = Pm @ k[t]
+            s = k[t] @ u + r[t]
+            U.append(u)
+            S.append(s)
+            P = Pm - np.outer(u, u) / s
+        for t in range(t1 - 1, t0 - 1, -1):
+            Pprev, u, s, kt = Pp[t - t0], U[t - t0], S[t - t0], k[t]
+            Mu, Pk = M @ u, Pprev @ kt
+            ds = (-(dg[t] @ u) + 0.5 * (u @ Mu)) / s ** 2
+            du = (dg[t] - Mu) / s + ds * kt
+            out["dk"][t] = ds * u + a[t] ** 2 * (Pprev @ du) + qn[t] * du
+            out["da"][t] = 2.0 * a[t] * (0.5 * np.sum(M * Pprev) + du @ Pk)
+            out["dqn"][t] = 0.5 * trM + du @ kt
+            out["dr"][t] = ds
+            M = a[t] ** 2 * (M + np.outer(du, kt) + np.outer(kt, du))
+            trM = a[t] ** 2 * (trM + 2.0 * (du @ kt))
+    out["dP0"] = 0.5 * M
+    return out

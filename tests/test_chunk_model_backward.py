@@ -111,3 +111,51 @@ def test_chunked_full_backward_equals_token_backward(C):
     for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dP0"):
         scale = max(np.abs(ref[key]).max(), 1e-12)
         assert np.abs(got[key] - ref[key]).max() <= 1e-8 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
+
+
+@pytest.mark.parametrize("block", [1, 5, 64])
+def test_full_cov_backward_tokens_with_memory_step_equals_token_backward(block):
+    """The covariance side the full-Kalman backward kernels run (carried M = Pb + Pb^T, blocks recomputed
+    from checkpoints), fed with the oracle's memory step for dg, gives the oracle's gradients."""
+    from chunk_model_backward import full_cov_backward_tokens
+    from oracle.backward import _memory_step_backward, scan_kalman_full_backward
+    rng = np.random.default_rng(block + 7)
+    L, dk, dv = 23, 6, 4
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q, k = unit(rng.standard_normal((L, dk))), unit(rng.standard_normal((L, dk)))
+    v = rng.standard_normal((L, dv))
+    r = np.log1p(np.exp(rng.standard_normal(L))) + 0.1
+    a = np.exp(-np.log1p(np.exp(rng.standard_normal(L) - 3.0)))
+    a[4] = 0.0
+    qn = 1e-3 + 1e-2 * rng.random(L)
+    B = rng.standard_normal((dk, dk)) / dk
+    S0, P0 = 0.3 * rng.standard_normal((dk, dv)), 0.5 * np.eye(dk) + B @ B.T
+    dO, dm, dSL = rng.standard_normal((L, dv)), rng.standard_normal(L), rng.standard_normal((dk, dv))
+    dPL = rng.standard_normal((dk, dk))  # not symmetric: the carried M symmetrises it
+    ref = scan_kalman_full_backward(q, k, v, r, dO, a=a, qn=qn, S0=S0, P0=P0, dm=dm, dS_L=dSL, dP_L=dPL)
+    # forward, then the memory backward with the gains as given inputs (its dg feeds the covariance side)
+    S, P, states, gains, res = S0.copy(), P0.copy(), [S0.copy()], [], []
+    for t in range(L):
+        Pm = a[t] ** 2 * P + qn[t] * np.eye(dk)
+        u = Pm @ k[t]
+        s = k[t] @ u + r[t]
+        g = u / s
+        P = Pm - np.outer(u, u) / s
+        e = v[t] - a[t] * S.T @ k[t]
+        S = a[t] * S + np.outer(g, e)
+        states.append(S.copy()), gains.append(g), res.append(e)
+    G = dSL[None].copy()
+    dg = np.zeros((L, dk))
+    mem = {key: np.zeros(shape) for key, shape in (("dq", (L, dk)), ("dk", (L, dk)), ("dv", (L, dv)), ("da", L))}
+    for t in range(L - 1, -1, -1):
+        G, dq, de, dkt, da_t, dgt = _memory_step_backward(G, gains[t][None], res[t][None], k[t][None], q[t][None],
+                                                         states[t + 1][None], states[t][None], a[t:t + 1],
+                                                         dO[t][None], dm[t:t + 1])
+        mem["dq"][t], mem["dk"][t], mem["dv"][t], mem["da"][t], dg[t] = dq[0], dkt[0], de[0], da_t[0], dgt[0]
+    cov = full_cov_backward_tokens(k, r, a, qn, P0, dg, dP_L=dPL, block=block)
+    got = {"dq": mem["dq"], "dv": mem["dv"], "dk": mem["dk"] + cov["dk"], "da": mem["da"] + cov["da"],
+           "dr": cov["dr"], "dqn": cov["dqn"], "dS0": G[0], "dP0": cov["dP0"]}
+    ref["dP0"] = 0.5 * (ref["dP0"] + ref["dP0"].T)
+    for key in ("dq", "dk", "dv", "dr", "da", "dqn", "dS0", "dP0"):
+        scale = max(np.abs(ref[key]).max(), 1e-12)
+        assert np.abs(got[key] - ref[key]).max() <= 1e-9 * scale, (key, np.abs(got[key] - ref[key]).max(), scale)
