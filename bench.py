@@ -406,8 +406,8 @@ def bench_hola(w, steps, warmup, dist_on, rank, world, cache_w=64):
 
 
 def bench_backward(w, steps, warmup, dist_on, rank, world):
-    """The backward over a layer (gated delta rule; isotropic or diagonal Kalman: the memory backward with the
-    uncertainty chain around it); upstream dO and dm random, start state zero."""
+    """The backward over a layer (gated delta rule; isotropic, diagonal or full Kalman: the memory backward with
+    the uncertainty chain around it); upstream dO and dm random, start state zero."""
     from delta_rule_recurrent_scan_b200 import kdn
     x = make_scan_inputs(w, seed=rank, device="cuda")
     g = torch.Generator(device="cuda")
@@ -423,6 +423,8 @@ def bench_backward(w, steps, warmup, dist_on, rank, world):
             kdn.scan_kalman_iso_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
         elif w.variant == "kalman_diag":
             kdn.scan_kalman_diag_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
+        elif w.variant == "kalman_full":
+            kdn.scan_kalman_full_backward(x["q"], x["k"], x["v"], x["r"], dO, a=x["a"], qn=x["qn"], dm=dm, workspace=ws)
         else:
             kdn.scan_delta_backward(x["q"], x["k"], x["v"], x["beta"], dO, a=x["a"], dm=dm, workspace=ws)
     ms = time_device(fn, steps, warmup, dist_on)
@@ -435,9 +437,11 @@ def backward_bytes(w, in_bytes=2) -> int:
 
 
 def backward_flops(w, C=32) -> int:
-    """Multiply-adds of the chunked backward (forward recompute included) per token: 8 d^2 + 11 C d, times 2."""
+    """Multiply-adds of the chunked backward (forward recompute included) per token: 8 d^2 + 11 C d, times 2; the
+    full-covariance side adds 10 d^2 (forward and block recompute: a matrix-vector product and a rank-1 update each;
+    backward: four matrix-vector products and the rank-2 update of the adjoint)."""
     d = w.dk
-    return w.tokens * 2 * (8 * d * d + 11 * C * d)
+    return w.tokens * 2 * (8 * d * d + 11 * C * d + (10 * d * d if w.variant == "kalman_full" else 0))
 
 
 FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 fp32 FMA lanes at 1965 MHz
@@ -531,7 +535,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--batch", type=int, default=None, help="override B of the workload (profiling runs)")
     ap.add_argument("--backward-only", action="store_true",
-                    help="time only the backward of a gated-delta workload (profiling runs): one JSON line")
+                    help="time only the backward of a gated-delta or Kalman workload (profiling runs): one JSON line")
     ap.add_argument("--cache-read-only", action="store_true",
                     help="time only the surprise-cache read over a workload's shape (profiling runs): one JSON line")
     args = ap.parse_args()
@@ -572,8 +576,8 @@ def main():
             torch.distributed.destroy_process_group()
         return
     if args.backward_only:
-        if w.variant not in ("delta", "kalman_iso", "kalman_diag"):
-            raise SystemExit("--backward-only needs a gated-delta, isotropic or diagonal Kalman workload")
+        if w.variant not in ("delta", "kalman_iso", "kalman_diag", "kalman_full"):
+            raise SystemExit("--backward-only needs a gated-delta or Kalman workload")
         r = bench_backward(w, args.steps, args.warmup, dist_on, rank, world)
         if rank == 0:
             print(json.dumps({"metric": f"{w.variant} backward tokens/s (every input gradient)", "value": r["value"],
@@ -619,7 +623,8 @@ def main():
         torch.cuda.empty_cache()
         for bname, bvariant in (("gdn_d128", "delta backward (dq, dk, dv, dbeta, da, dS0)"),
                                 ("kalman_iso_d128", "isotropic Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dc0)"),
-                                ("kalman_diag_d128", "diagonal Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dp0)")):
+                                ("kalman_diag_d128", "diagonal Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dp0)"),
+                                ("kalman_full_d128", "full Kalman backward (dq, dk, dv, dr, da, dqn, dS0, dP0)")):
             bw = WORKLOADS[bname]
             r = bench_backward(bw, 2, 3, dist_on, rank, world)
             also.append({"workload": bname + "_backward", "variant": bvariant,

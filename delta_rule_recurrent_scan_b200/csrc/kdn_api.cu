@@ -487,7 +487,8 @@ kdn_status kdn_scan_kalman_iso(const kdn_dims* dims, const void* q, const void* 
 }
 
 size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
-  if (variant != KDN_DELTA && variant != KDN_KALMAN_ISO && variant != KDN_KALMAN_DIAG) return 0;
+  if (variant != KDN_DELTA && variant != KDN_KALMAN_ISO && variant != KDN_KALMAN_DIAG && variant != KDN_KALMAN_FULL)
+    return 0;
   if (dims == nullptr || dims->B < 1 || dims->H < 1 || dims->L < 0) return 0;
   if (!supported_dim(dims->dk) || !supported_dim(dims->dv)) return 0;
   const size_t BH = (size_t)dims->B * dims->H, DD = (size_t)dims->dk * dims->dv, tok = BH * (size_t)dims->L;
@@ -497,6 +498,9 @@ size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims) {
   if (variant == KDN_KALMAN_ISO) n += 4 * round256(tok * 4);
   // diagonal: the gains, p before every token and dG (d_k values per token each)
   if (variant == KDN_KALMAN_DIAG) n += 3 * round256(tok * dims->dk * 4);
+  // full: the gains and dG, then P at every 32-token block start and one block's P before every token per head
+  if (variant == KDN_KALMAN_FULL)
+    n += 2 * round256(tok * dims->dk * 4) + kdn::full_backward_scratch_bytes((int)BH, dims->L, dims->dk);
   return n;
 }
 
@@ -689,6 +693,61 @@ kdn_status kdn_scan_kalman_diag_backward(const kdn_dims* dims, const void* q, co
     return cuda_status(cudaMemsetAsync(dp0, 0, BH * dims->dk * 4, st), "dp0 of an empty sequence");
   }
   return cuda_status(kdn::launch_diag_backward(da_args, (int)BH, st), "diagonal backward: uncertainty chain launch");
+}
+
+kdn_status kdn_scan_kalman_full_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                        const float* r, const float* a, const float* qn, float qn_scalar,
+                                        const float* S0, const float* P0, const float* dO, const float* dm,
+                                        const float* dS_L, const float* dP_L, float* dq, float* dk, float* dv,
+                                        float* dr, float* da, float* dqn, float* dS0, float* dP0, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  KDN_TRY(check_dims(dims));
+  const bool any = dims->L > 0;
+  KDN_TRY(check_ptr(dS0, "dS0", 16, false));
+  KDN_TRY(check_ptr(dP0, "dP0", 16, false));
+  for (const auto& pr : {std::make_pair((const void*)q, "q"), std::make_pair((const void*)k, "k"),
+                         std::make_pair((const void*)v, "v"), std::make_pair((const void*)dO, "dO"),
+                         std::make_pair((const void*)dq, "dq"), std::make_pair((const void*)dk, "dk"),
+                         std::make_pair((const void*)dv, "dv")})
+    KDN_TRY(check_ptr(pr.first, pr.second, 16, !any));
+  KDN_TRY(check_ptr(r, "r", 4, !any));
+  KDN_TRY(check_ptr(dr, "dr", 4, !any));
+  KDN_TRY(check_ptr(dqn, "dqn", 4, !any));
+  KDN_TRY(check_ptr(a, "a", 4, true));
+  KDN_TRY(check_ptr(da, "da", 4, true));
+  KDN_TRY(check_ptr(qn, "qn", 4, true));
+  KDN_TRY(check_ptr(dm, "dm", 4, true));
+  KDN_TRY(check_ptr(S0, "S0", 16, true));
+  KDN_TRY(check_ptr(P0, "P0", 16, true));
+  KDN_TRY(check_ptr(dS_L, "dS_L", 16, true));
+  KDN_TRY(check_ptr(dP_L, "dP_L", 16, true));
+  KDN_TRY(check_ptr(workspace, "workspace", 256, false));
+  if (!(qn_scalar >= 0.f)) return fail(KDN_ERR_INVALID_ARG, "qn_scalar must be >= 0");
+  const size_t need = kdn_backward_workspace_bytes(KDN_KALMAN_FULL, dims);
+  if (workspace_bytes < need)
+    return fail(KDN_ERR_INVALID_ARG, "workspace_bytes " + std::to_string(workspace_bytes) + " < required " +
+                                         std::to_string(need));
+  DeviceGuard guard;
+  KDN_TRY(use_device_of(dS0, guard));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BH = (size_t)dims->B * dims->H, tok = BH * (size_t)dims->L;
+  kdn_dims dd = *dims;
+  char* side = reinterpret_cast<char*>(workspace) + kdn_backward_workspace_bytes(KDN_DELTA, &dd);
+  kdn::FullBwdArgs fa{};
+  fa.k = k, fa.in_dtype = dims->in_dtype, fa.a = a, fa.r = r, fa.qn = qn, fa.qn_scalar = qn_scalar, fa.P0 = P0;
+  fa.gains = reinterpret_cast<float*>(side);
+  float* dgain = reinterpret_cast<float*>(side + round256(tok * dims->dk * 4));
+  fa.dgain = dgain, fa.dP_L = dP_L, fa.dk = dk, fa.da = da, fa.dr = dr, fa.dqn = dqn, fa.dP0 = dP0;
+  fa.status = reinterpret_cast<unsigned*>(workspace), fa.L = dims->L, fa.d = dims->dk;
+  kdn::full_backward_bind_scratch(fa, side + 2 * round256(tok * dims->dk * 4), (int)BH);
+  if (any)
+    KDN_TRY(cuda_status(kdn::launch_full_cov_forward(fa, (int)BH, st), "full-Kalman backward: covariance forward launch"));
+  // the memory backward with the gains as inputs (it clears the status word first) gives dq, dv, dS0, the key's
+  // memory terms, dG and the decay terms of da; the covariance side then adds its key and gate terms and
+  // writes dr, dQn and dP0 (for an empty sequence: dP0 = the symmetric part of dP_L)
+  KDN_TRY(delta_backward_run(dims, q, k, v, nullptr, a, S0, dO, dm, dS_L, dq, dk, dv, nullptr, da, dS0, workspace, st,
+                             fa.gains, dgain));
+  return cuda_status(kdn::launch_full_cov_backward(fa, (int)BH, st), "full-Kalman backward: covariance chain launch");
 }
 
 size_t kdn_hola_workspace_bytes(const kdn_dims* dims) {

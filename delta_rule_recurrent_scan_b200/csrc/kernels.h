@@ -107,6 +107,35 @@ struct DiagBwdArgs {
 cudaError_t launch_diag_forward(const DiagBwdArgs& args, int BH, cudaStream_t stream);
 cudaError_t launch_diag_backward(const DiagBwdArgs& args, int BH, cudaStream_t stream);
 
+// Covariance side of the full-Kalman backward: the forward keeps the per-token gains and P at every 32-token
+// block start; the backward recomputes each block and walks it in reverse with M = Pb + Pb^T.
+struct FullBwdArgs {
+  const void* k;        // [BH, L, d]
+  int in_dtype;
+  const float* a;       // [BH, L] or nullptr
+  const float* r;       // [BH, L]
+  const float* qn;      // [BH, L] or nullptr (qn_scalar)
+  float qn_scalar;
+  const float* P0;      // [BH, d, d] or nullptr (I)
+  float* gains;         // [BH, L, d] forward: g_t = u_t / s_t
+  float* ckpt;          // scratch [BH, nblk, d, d]: P at every block start (thread order)
+  float* scr_P;         // scratch [BH, 32, d, d]: P before every token of the block being walked
+  const float* dgain;   // [BH, L, d] backward: dLoss/dg_t from the memory backward
+  const float* dP_L;    // [BH, d, d] or nullptr: upstream gradient of the final P
+  float* dk;            // [BH, L, d] in/out: the key terms are added
+  float* da;            // [BH, L] in/out or nullptr: the gate terms are added
+  float* dr;            // [BH, L] out
+  float* dqn;           // [BH, L] out
+  float* dP0;           // [BH, d, d] out: the gradient for a symmetric P0
+  unsigned* status;     // the call's status word (a non-positive or non-finite s)
+  int L;
+  int d;                // d_k: 16, 32, 64 or 128
+};
+size_t full_backward_scratch_bytes(int BH, int L, int d);
+void full_backward_bind_scratch(FullBwdArgs& args, void* scratch, int BH);
+cudaError_t launch_full_cov_forward(const FullBwdArgs& args, int BH, cudaStream_t stream);
+cudaError_t launch_full_cov_backward(const FullBwdArgs& args, int BH, cudaStream_t stream);
+
 // Sequence-parallel covariance side of the full-Kalman scan (chunks of 64 tokens): the covariance entering
 // every run of cps chunks, through the chunks' Riccati transfer matrices.
 struct RiccatiArgs {

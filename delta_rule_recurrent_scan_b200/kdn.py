@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
     L.kdn_scan_kalman_iso_backward.restype = ctypes.c_int
     L.kdn_scan_kalman_diag_backward.argtypes = [dims, vp, vp, vp, vp, vp, vp, f] + [vp] * 14 + [vp, sz, vp]
     L.kdn_scan_kalman_diag_backward.restype = ctypes.c_int
+    L.kdn_scan_kalman_full_backward.argtypes = [dims, vp, vp, vp, vp, vp, vp, f] + [vp] * 14 + [vp, sz, vp]
+    L.kdn_scan_kalman_full_backward.restype = ctypes.c_int
     L.kdn_backward_workspace_bytes.argtypes = [i, dims]
     L.kdn_backward_workspace_bytes.restype = sz
     L.kdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
@@ -248,9 +250,16 @@ def scan_kalman_iso_backward(q, k, v, r, dO, a=None, qn=None, S0=None, c0=None, 
     return _kalman_backward("kalman_iso", q, k, v, r, dO, a, qn, S0, c0, dm, dS_L, dc_L, workspace, stream, want_da)
 
 
+def scan_kalman_full_backward(q, k, v, r, dO, a=None, qn=None, S0=None, P0=None, dm=None, dS_L=None, dP_L=None,
+                              workspace=None, stream=None, want_da=True):
+    """Gradients of the full-covariance Kalman scan for upstream dO (and dm, dS_L, dP_L).  Returns a dict with dq,
+    dk, dv, dr, da (None if not wanted), dqn (per token), dS0 and dP0 (the gradient for a symmetric P0), all fp32."""
+    return _kalman_backward("kalman_full", q, k, v, r, dO, a, qn, S0, P0, dm, dS_L, dP_L, workspace, stream, want_da)
+
+
 def _kalman_backward(variant, q, k, v, r, dO, a, qn, S0, u0, dm, dS_L, du_L, workspace, stream, want_da):
-    """The uncertainty-side backward shared by the isotropic (u = c, one per head) and diagonal (u = p, one per
-    coordinate) variants."""
+    """The uncertainty-side backward shared by the isotropic (u = c, one per head), diagonal (u = p, one per
+    coordinate) and full (u = P, d_k x d_k per head) variants."""
     if q.dim() != 4:
         raise ValueError("q must be [B, H, L, d_k]")
     B, H, L, dk = q.shape
@@ -264,8 +273,8 @@ def _kalman_backward(variant, q, k, v, r, dO, a, qn, S0, u0, dm, dS_L, du_L, wor
     tok = (B, H, L)
     _need(r, "r", tok, torch.float32, dev)
     _need(dO, "dO", (B, H, L, dv), torch.float32, dev)
-    ushape = (B, H) if variant == "kalman_iso" else (B, H, dk)
-    uname = "c" if variant == "kalman_iso" else "p"
+    ushape = {"kalman_iso": (B, H), "kalman_diag": (B, H, dk), "kalman_full": (B, H, dk, dk)}[variant]
+    uname = {"kalman_iso": "c", "kalman_diag": "p", "kalman_full": "P"}[variant]
     for name, t, shape in (("a", a, tok), ("dm", dm, tok), ("S0", S0, (B, H, dk, dv)), ("dS_L", dS_L, (B, H, dk, dv)),
                            (uname + "0", u0, ushape), ("d" + uname + "_L", du_L, ushape)):
         if t is not None:
@@ -279,7 +288,8 @@ def _kalman_backward(variant, q, k, v, r, dO, a, qn, S0, u0, dm, dS_L, du_L, wor
     need = int(lib().kdn_backward_workspace_bytes(VARIANTS[variant], ctypes.byref(dims)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    fn = lib().kdn_scan_kalman_iso_backward if variant == "kalman_iso" else lib().kdn_scan_kalman_diag_backward
+    fn = {"kalman_iso": lib().kdn_scan_kalman_iso_backward, "kalman_diag": lib().kdn_scan_kalman_diag_backward,
+          "kalman_full": lib().kdn_scan_kalman_full_backward}[variant]
     st = fn(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(a), _ptr(qn_t), qn_s, _ptr(S0), _ptr(u0),
             _ptr(dO), _ptr(dm), _ptr(dS_L), _ptr(du_L), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
             _ptr(out["dr"]), _ptr(out["da"]), _ptr(out["dqn"]), _ptr(out["dS0"]), _ptr(out["d" + uname + "0"]),

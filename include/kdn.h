@@ -223,8 +223,32 @@ KDN_EXPORT kdn_status kdn_scan_kalman_diag_backward(const kdn_dims* dims, const 
                                                     float* dv, float* dr, float* da, float* dqn, float* dS0,
                                                     float* dp0, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward of the full-covariance Kalman scan (Kalman Delta Networks, Abstract:
+ * the dense Riccati recursion of the memory's uncertainty; the layers are
+ * trained end to end).  The forward is kdn_scan_kalman_full's: P^- = a^2 P +
+ * Qn I, u = P^- k, s = k^T u + r, gain g = u / s, P = P^- - u u^T / s, the
+ * delta-rule memory write with that gain.  Same inputs and outputs as
+ * kdn_scan_kalman_diag_backward with P0 (NULL = I), dP_L (NULL = 0) and dP0
+ * [B,H,d_k,d_k] fp32 in place of p0, dp_L, dp0.  P0 must be symmetric, as the
+ * forward requires; dP0 is the gradient with respect to a symmetric P0, i.e.
+ * the symmetric part of the entrywise derivative (for an empty sequence the
+ * symmetric part of dP_L).  Runs the covariance chain forward (one CTA of 4 d_k
+ * threads per head, storing the gains and P at every 32-token block start),
+ * the memory backward with the gains as inputs (its kernels write dG), and the
+ * covariance chain backwards (each block's P recomputed from its checkpoint,
+ * the adjoint carried as its symmetric sum), which adds its key and gate terms.
+ * A non-positive or non-finite s raises KDN_ERR_NUMERIC in the status word.
+ * workspace: kdn_backward_workspace_bytes(KDN_KALMAN_FULL, dims) bytes.
+ * Asynchronous on ``stream``. */
+KDN_EXPORT kdn_status kdn_scan_kalman_full_backward(const kdn_dims* dims, const void* q, const void* k, const void* v,
+                                                    const float* r, const float* a, const float* qn, float qn_scalar,
+                                                    const float* S0, const float* P0, const float* dO, const float* dm,
+                                                    const float* dS_L, const float* dP_L, float* dq, float* dk,
+                                                    float* dv, float* dr, float* da, float* dqn, float* dS0,
+                                                    float* dP0, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace the backward entry points need (KDN_DELTA,
- * KDN_KALMAN_ISO or KDN_KALMAN_DIAG; 0 for full Kalman or invalid dims). */
+ * KDN_KALMAN_ISO, KDN_KALMAN_DIAG or KDN_KALMAN_FULL; 0 for invalid dims). */
 KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_dims* dims);
 
 /* Surprise-cache read (A Hippocampus for Linear Attention, sections 3.3-3.4,

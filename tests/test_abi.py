@@ -114,7 +114,8 @@ def test_backward_host_validation(L):
     n = L.kdn_backward_workspace_bytes(0, ctypes.byref(d))
     # status word + working state + a state per 32-token chunk + one norm per token
     assert n >= 256 + 6 * 64 * 32 * 4 * (1 + 4) + 6 * 100 * 4
-    assert L.kdn_backward_workspace_bytes(2, ctypes.byref(d)) == 0  # full Kalman has no CUDA backward
+    # full Kalman: plus the gains and dG, P at every 32-token block start (4 blocks) and one block's P per token
+    assert L.kdn_backward_workspace_bytes(2, ctypes.byref(d)) >= n + 2 * 6 * 100 * 64 * 4 + 6 * (4 + 32) * 64 * 64 * 4
     # isotropic: the delta backward's part plus beta, the uncertainty before every token, ||k||^2 and dbeta
     assert L.kdn_backward_workspace_bytes(3, ctypes.byref(d)) >= n + 4 * 6 * 100 * 4
     # diagonal: plus the gains, the variances before every token and dG
@@ -140,6 +141,16 @@ def test_hola_workspace_covers_every_block_on_the_tensor_core_path(L):
     assert L.kdn_hola_workspace_bytes(ctypes.byref(tc)) >= 256 + 6 * 5 * 64 * 4
     assert L.kdn_hola_workspace_bytes(ctypes.byref(other)) == 256
     assert L.kdn_hola_workspace_bytes(None) == 0
+
+
+def test_full_backward_host_validation(L):
+    d = kdn.Dims(1, 2, 50, 32, 32, 0, kdn.KDN_BF16, kdn.KDN_F32)
+    args = [None] * 6 + [0.0] + [None] * 14 + [None, 0, None]
+    assert L.kdn_scan_kalman_full_backward(None, *args) == kdn.KDN_ERR_INVALID_ARG
+    assert L.kdn_scan_kalman_full_backward(ctypes.byref(d), *args) == kdn.KDN_ERR_INVALID_ARG
+    assert b"dS0" in L.kdn_last_error()
+    bad = kdn.Dims(1, 2, 50, 48, 32, 0, kdn.KDN_BF16, kdn.KDN_F32)  # d_k outside 16, 32, 64, 128
+    assert L.kdn_backward_workspace_bytes(2, ctypes.byref(bad)) == 0
 
 
 def test_diag_backward_host_validation(L):
