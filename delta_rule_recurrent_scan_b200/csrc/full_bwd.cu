@@ -11,10 +11,11 @@
 //   M <- a^2 (M + du k^T + k du^T)            (dP0 = M_0 / 2, the gradient for a symmetric P0).
 // One CTA of 4 d threads per head: thread (i, q) = (tid / 4, tid % 4) holds row i of P (and of M) at the d/4
 // columns 16 m + 4 q + e (e < 4), so a matrix-vector product is d/4 multiply-adds per thread and a reduction
-// over four lanes, and the four threads of a row read a broadcast vector as four adjacent float4 (one
-// shared-memory wavefront; columns q d/4 .. of each thread would fall on one bank four times over).  Both kernels go through the tokens in blocks of kFB, each block's inputs staged
-// in shared memory before it is walked (the forward loads the next block into registers while it walks the
-// current one), so no global load sits on a token's serial path.  The forward keeps P at every block start;
+// over four lanes, and the four threads of a row read a broadcast vector as four adjacent float4, free of
+// bank conflicts (with columns q d/4 .. per thread the four quarters would sit on the same banks).  Both
+// kernels go through the tokens in blocks of kFB, each block's inputs staged in shared memory before it is
+// walked (the forward loads the next block into registers while it walks the current one), so no global
+// load sits on a token's serial path.  The forward keeps P at every block start;
 // the backward recomputes each block's P before every token (to global scratch, in the threads' own float4
 // order; u and s stay in shared memory), then walks the block in reverse with that P streamed back through a
 // two-slot cp.async buffer, each thread copying and reading only its own slots.
