@@ -450,7 +450,8 @@ __global__ void __launch_bounds__(kSelThreads) hola_cache_select_kernel(HolaArgs
 // hola_read_block_kernel: one CTA per head and run of kBlocksPerCta consecutive blocks, two CTAs per SM.  Each
 // block's q, k, v arrive by TMA, its cache rows by 16-byte cp.async gathers of the token indices chosen above
 // (rows 0..63; empty rows zero), then the same S product, softmax with the sink and P V product as the serial
-// kernel.  While a block is read, the next block's tiles and cache rows are prefetched into L2.
+// kernel.  (An L2 prefetch of the next block's tiles and cache rows while a block was read cost 6 %: the
+// cache rows repeat from block to block and are mostly in L2 already.)
 // The raw queries land in the lo panel: each thread reads its 16-byte chunk there before it writes the lo
 // half of the scaled query to the same address, so the CTA fits twice in an SM's shared memory.
 constexpr int kBlocksPerCta = 4;
@@ -460,9 +461,6 @@ constexpr int kPSmem = PB_L + kPanel + 1024;
 __device__ __forceinline__ void cp_async16_cg(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void prefetch_l2_bulk(const void* gmem, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
 }
 
 __global__ void __launch_bounds__(kTThreads, 2)
@@ -493,7 +491,6 @@ __global__ void __launch_bounds__(kTThreads, 2)
   uint8_t* VB = sm + PB_V;
   const uint8_t* kbytes = reinterpret_cast<const uint8_t*>(p.k);
   const uint8_t* vbytes = reinterpret_cast<const uint8_t*>(p.v);
-  const uint8_t* qbytes = reinterpret_cast<const uint8_t*>(p.q);
 
   if (tid == 0) {
     sm100::prefetch_tmap(&tm_q);
@@ -538,20 +535,6 @@ __global__ void __launch_bounds__(kTThreads, 2)
       else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    if (blk + 1 < blk_end) {  // the next block's tiles and cache rows into L2, while this block is read
-      const size_t nt = tok0 + 64 * (blk + 1);
-      const uint32_t tile = (uint32_t)min(64, L - 64 * (blk + 1)) * kD * 2;
-      if (tid == 0) prefetch_l2_bulk(qbytes + nt * kD * 2, tile);
-      if (tid == 1) prefetch_l2_bulk(kbytes + nt * kD * 2, tile);
-      if (tid == 2) prefetch_l2_bulk(vbytes + nt * kD * 2, tile);
-      if (tid >= 64 && tid < 128) {
-        const int t = p.cidx[((size_t)bh * nblocks + blk + 1) * 64 + tid - 64];
-        if (t >= 0) {
-          prefetch_l2_bulk(kbytes + (tok0 + t) * kD * 2, kD * 2);
-          prefetch_l2_bulk(vbytes + (tok0 + t) * kD * 2, kD * 2);
-        }
-      }
-    }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     {
       int fail = 0;
