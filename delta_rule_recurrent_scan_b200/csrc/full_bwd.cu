@@ -9,16 +9,16 @@
 //   ds = (-(dg . u) + u^T M u / 2) / s^2,   du = (dg - M u) / s + ds k,
 //   dk += ds u + P^- du,   dr = ds,   dQn = tr(M) / 2 + du . k,   da += 2 a (<M, P> / 2 + du . P k),
 //   M <- a^2 (M + du k^T + k du^T)            (dP0 = M_0 / 2, the gradient for a symmetric P0).
-// One CTA of 4 d threads per head: thread (i, q) = (tid / 4, tid % 4) holds row i of P (and of M) at the d/4
-// columns 16 m + 4 q + e (e < 4), so a matrix-vector product is d/4 multiply-adds per thread and a reduction
-// over four lanes, and the four threads of a row read a broadcast vector as four adjacent float4, free of
-// bank conflicts (with columns q d/4 .. per thread the four quarters would sit on the same banks).  Both
+// One CTA of 4 d threads per head, in row groups of G = 4 R threads: thread g of group n holds rows
+// n R .. n R + R - 1 of P (and of M) at the d / G columns 4 G m + 4 g + e (e < 4); R = 2 from d = 32 on (1 at
+// d = 16), so that each broadcast vector is read as d / (4 G) float4 per thread, G adjacent float4 per group
+// (free of bank conflicts), and a matrix-vector product ends in a reduction over the group's lanes.  Both
 // kernels go through the tokens in blocks of kFB, each block's inputs staged in shared memory before it is
 // walked (the forward loads the next block into registers while it walks the current one), so no global
-// load sits on a token's serial path.  The forward keeps P at every block start;
-// the backward recomputes each block's P before every token (to global scratch, in the threads' own float4
-// order; u and s stay in shared memory), then walks the block in reverse with that P streamed back through a
-// two-slot cp.async buffer, each thread copying and reading only its own slots.
+// load sits on a token's serial path.  The forward keeps P at every block start; the backward recomputes
+// each block's P before every token (to global scratch, in the threads' own float4 order; u and s stay in
+// shared memory), then walks the block in reverse with that P streamed back through a two-slot cp.async
+// buffer, each thread copying and reading only its own slots.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -32,7 +32,10 @@ constexpr int kFB = 32;  // tokens per block: inputs staged per block, P checkpo
 
 template <int D>
 struct FullBwdShape {
-  static constexpr int NT = 4 * D, NW = NT / 32, CW = D / 4, NV = CW / 4;  // NV float4 per thread per matrix
+  // R rows of P per thread (two from d = 32 on, so that a broadcast vector is read half as often), G = 4 R
+  // threads per row group, CW columns per row and thread
+  static constexpr int NT = 4 * D, NW = NT / 32, R = D >= 32 ? 2 : 1, G = 4 * R, CW = D / G, NM = CW / 4;
+  static constexpr int NV = R * CW / 4;     // float4 per thread per matrix
   static constexpr int KPT = kFB * D / NT;  // block elements per thread when a [kFB, D] block is staged
 };
 
@@ -42,10 +45,13 @@ __device__ __forceinline__ float4* slot(float* base, int m, int tid) {
   return reinterpret_cast<float4*>(base) + (size_t)m * FullBwdShape<D>::NT + tid;
 }
 
-// Column of register j of thread quarter q, and that thread's float4 m of a d-vector in shared memory.
-__device__ __forceinline__ int colof(int q, int j) { return 16 * (j >> 2) + 4 * q + (j & 3); }
-__device__ __forceinline__ float4 vec4(const float* v, int m, int q) {
-  return reinterpret_cast<const float4*>(v)[4 * m + q];
+// Column of register j of thread g of its row group, and that thread's float4 m of a d-vector in shared
+// memory: the G threads of a group read G adjacent float4, free of bank conflicts.
+template <int G>
+__device__ __forceinline__ int colof(int g, int j) { return 4 * G * (j >> 2) + 4 * g + (j & 3); }
+template <int G>
+__device__ __forceinline__ float4 vec4(const float* v, int m, int g) {
+  return reinterpret_cast<const float4*>(v)[G * m + g];
 }
 
 // Sum of the NW warp partials v[0 .. NW) (16-byte aligned; NW = 2, 4, 8 or 16), in a short tree.
@@ -64,45 +70,67 @@ __device__ __forceinline__ float sum_parts(const float* v) {
   }
 }
 
-// One forward token of P held by the calling thread: P <- P^- - u u^T / s.  kv holds the token's key (fp32),
-// us receives u (it is also this token's broadcast slot), part the warp partial sums.  Returns u_i and s;
-// one __syncthreads.
+// Sum over the G lanes of a row group.
+template <int G>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int o = 1; o < G; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// One forward token of P held by the calling thread (rows r0 .. r0 + R - 1): P <- P^- - u u^T / s.  kv holds the
+// token's key (fp32), us receives u (it is also this token's broadcast slot), part the warp partial sums.
+// Returns u of the thread's rows and s; one __syncthreads.
 template <int D>
 __device__ __forceinline__ void cov_step(float (&Pr)[D / 4], const float* kv, float* us, float* part, float at,
-                                         float rt, float qt, int tid, unsigned* status, float& ui, float& s) {
+                                         float rt, float qt, int tid, unsigned* status,
+                                         float (&ui)[FullBwdShape<D>::R], float& s) {
   using Sh = FullBwdShape<D>;
-  const int i = tid >> 2, q = tid & 3, lane = tid & 31, warp = tid >> 5;
+  constexpr int R = Sh::R, G = Sh::G, CW = Sh::CW;
+  const int g = tid % G, r0 = (tid / G) * R, lane = tid & 31, warp = tid >> 5;
   const float a2 = at * at;
-  float d4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums keep the dependent chain d / 16 long
+  float d4[R][4];  // four partial sums per row keep the dependent chains short
 #pragma unroll
-  for (int m = 0; m < Sh::NV; ++m) {
-    const float4 k4 = vec4(kv, m, q);
+  for (int r = 0; r < R; ++r) d4[r][0] = d4[r][1] = d4[r][2] = d4[r][3] = 0.f;
+#pragma unroll
+  for (int m = 0; m < Sh::NM; ++m) {
+    const float4 k4 = vec4<G>(kv, m, g);
     const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 4 * m + e;
-      Pr[j] = fmaf(a2, Pr[j], colof(q, j) == i ? qt : 0.f);
-      d4[e] = fmaf(Pr[j], kk[e], d4[e]);
-    }
-  }
-  float dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
-  dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-  dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-  ui = dot;
-  float ku = (tid & 3) == 0 ? kv[i] * ui : 0.f;
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) ku += __shfl_xor_sync(0xffffffffu, ku, o);
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * m + e, x = r * CW + j;
+        Pr[x] = fmaf(a2, Pr[x], colof<G>(g, j) == r0 + r ? qt : 0.f);
+        d4[r][e] = fmaf(Pr[x], kk[e], d4[r][e]);
+      }
+  }
+  float ku = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    ui[r] = group_sum<G>((d4[r][0] + d4[r][1]) + (d4[r][2] + d4[r][3]));
+    if (g == 0) ku = fmaf(kv[r0 + r], ui[r], ku);
+  }
+#pragma unroll
+  for (int o = G; o < 32; o <<= 1) ku += __shfl_xor_sync(0xffffffffu, ku, o);
   if (lane == 0) part[warp] = ku;
-  if ((tid & 3) == 0) us[i] = ui;
+  if (g == 0)
+#pragma unroll
+    for (int r = 0; r < R; ++r) us[r0 + r] = ui[r];
   __syncthreads();
   s = rt + sum_parts<Sh::NW>(part);
   if (tid == 0 && status != nullptr && !(s > 0.f && isfinite(s))) raise_status(status, kStatusNumeric);
-  const float f = ui / s;
+  float f[R];
 #pragma unroll
-  for (int m = 0; m < Sh::NV; ++m) {
-    const float4 u4 = vec4(us, m, q);
-    Pr[4 * m] = fmaf(-f, u4.x, Pr[4 * m]), Pr[4 * m + 1] = fmaf(-f, u4.y, Pr[4 * m + 1]);
-    Pr[4 * m + 2] = fmaf(-f, u4.z, Pr[4 * m + 2]), Pr[4 * m + 3] = fmaf(-f, u4.w, Pr[4 * m + 3]);
+  for (int r = 0; r < R; ++r) f[r] = ui[r] / s;
+#pragma unroll
+  for (int m = 0; m < Sh::NM; ++m) {
+    const float4 u4 = vec4<G>(us, m, g);
+    const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Pr[r * CW + 4 * m + e] = fmaf(-f[r], uu[e], Pr[r * CW + 4 * m + e]);
   }
 }
 
@@ -125,14 +153,19 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_forward_kernel(FullBwdArgs 
   __shared__ __align__(16) float kf[2][kFB][D];
   __shared__ float sa[2][kFB], sr[2][kFB], sq[2][kFB];
   __shared__ __align__(16) float us[2][D], part[2][Sh::NW];
+  constexpr int R = Sh::R, G = Sh::G, CW = Sh::CW;
   const int tid = threadIdx.x, bh = blockIdx.x, L = p.L;
-  const int i = tid >> 2, q = tid & 3;
+  const int g = tid % G, r0 = (tid / G) * R;
   const size_t tok0 = (size_t)bh * L;
   const int nblk = (L + kFB - 1) / kFB;
-  float Pr[Sh::CW];
+  float Pr[R * CW];
 #pragma unroll
-  for (int j = 0; j < Sh::CW; ++j)
-    Pr[j] = p.P0 != nullptr ? p.P0[((size_t)bh * D + i) * D + colof(q, j)] : (colof(q, j) == i ? 1.f : 0.f);
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < CW; ++j) {
+      const int row = r0 + r, c = colof<G>(g, j);
+      Pr[r * CW + j] = p.P0 != nullptr ? p.P0[((size_t)bh * D + row) * D + c] : (c == row ? 1.f : 0.f);
+    }
   // the next block's keys and scalars travel in registers while the current block is walked
   float kr[Sh::KPT];
   float ra = 1.f, rr = 1.f, rq = 0.f;
@@ -160,9 +193,11 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_forward_kernel(FullBwdArgs 
     for (int m = 0; m < Sh::NV; ++m)
       *slot<D>(ck, m, tid) = make_float4(Pr[4 * m], Pr[4 * m + 1], Pr[4 * m + 2], Pr[4 * m + 3]);
     for (int tt = 0; tt < n; ++tt) {
-      float ui, s;
+      float ui[R], s;
       cov_step<D>(Pr, kf[b][tt], us[tt & 1], part[tt & 1], sa[b][tt], sr[b][tt], sq[b][tt], tid, nullptr, ui, s);
-      if ((tid & 3) == 0) p.gains[(tok0 + t0 + tt) * D + i] = ui / s;  // (the backward's recompute checks s)
+      if (g == 0)  // (the backward's recompute checks s)
+#pragma unroll
+        for (int r = 0; r < R; ++r) p.gains[(tok0 + t0 + tt) * D + r0 + r] = ui[r] / s;
     }
     if (blk + 1 < nblk) {
       stash(b ^ 1);  // the other buffer was last read in block blk - 1, before this block's barriers
@@ -175,7 +210,7 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_forward_kernel(FullBwdArgs 
 template <int D>
 __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs p) {
   using Sh = FullBwdShape<D>;
-  constexpr int CW = Sh::CW, NV = Sh::NV, NW = Sh::NW;
+  constexpr int R = Sh::R, G = Sh::G, CW = Sh::CW, NV = Sh::NV, NW = Sh::NW;
   // dynamic: [2][D * D] P before the token (thread order) | keys | u | dG | dk in, [kFB][D] fp32 each
   extern __shared__ __align__(16) float dyn[];
   float* pbuf = dyn;
@@ -187,22 +222,25 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
   __shared__ __align__(16) float dus[2][D];
   __shared__ __align__(16) float part[2][3][NW], part2[2][2][NW], rpart[2][NW];
   const int tid = threadIdx.x, bh = blockIdx.x, L = p.L, lane = tid & 31, warp = tid >> 5;
-  const int i = tid >> 2, q = tid & 3;
-  const bool row_lead = q == 0;
+  const int g = tid % G, r0 = (tid / G) * R;
+  const bool row_lead = g == 0;
   const size_t tok0 = (size_t)bh * L;
   const int nblk = (L + kFB - 1) / kFB;
   float* scrP = p.scr_P + (size_t)bh * kFB * D * D;
 
   // M = dP_L + dP_L^T, and its trace
-  float Mr[CW];
+  float Mr[R * CW];
   float tr = 0.f;
 #pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const size_t base = (size_t)bh * D * D;
-    const int c = colof(q, j);
-    Mr[j] = p.dP_L != nullptr ? p.dP_L[base + (size_t)i * D + c] + p.dP_L[base + (size_t)c * D + i] : 0.f;
-    if (c == i) tr = Mr[j];
-  }
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < CW; ++j) {
+      const size_t base = (size_t)bh * D * D;
+      const int row = r0 + r, c = colof<G>(g, j);
+      Mr[r * CW + j] =
+          p.dP_L != nullptr ? p.dP_L[base + (size_t)row * D + c] + p.dP_L[base + (size_t)c * D + row] : 0.f;
+      if (c == row) tr += Mr[r * CW + j];
+    }
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
   if (lane == 0) rpart[0][warp] = tr;
@@ -236,7 +274,7 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
     // ---------------------------------------------------------------- recompute the block's P, u, s
     {
       const float* ck = p.ckpt + ((size_t)bh * nblk + blk) * D * D;
-      float Pr[CW];
+      float Pr[R * CW];
 #pragma unroll
       for (int m = 0; m < NV; ++m) {
         const float4 x = *slot<D>(const_cast<float*>(ck), m, tid);
@@ -249,7 +287,7 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
 #pragma unroll
         for (int m = 0; m < NV; ++m)
           *slot<D>(sp, m, tid) = make_float4(Pr[4 * m], Pr[4 * m + 1], Pr[4 * m + 2], Pr[4 * m + 3]);
-        float ui, s;
+        float ui[R], s;
         cov_step<D>(Pr, kf[tt], ub[tt], rpart[tt & 1], sa[tt], sr[tt], sq[tt], tid, p.status, ui, s);
         if (tid == 0) ss[tt] = s;
       }
@@ -268,7 +306,7 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
       const int b = tt & 1;
       const size_t ti = tok0 + t0 + tt;
       async_wait<0>();
-      float Pp[CW];
+      float Pp[R * CW];
 #pragma unroll
       for (int m = 0; m < NV; ++m) {
         const float4 x = *slot<D>(pbuf + b * D * D, m, tid);
@@ -276,28 +314,36 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
       }
       if (tt > 0) fetch_P(tt - 1);
       const float at = sa[tt], qt = sq[tt], s = ss[tt], a2 = at * at, inv = 1.f / s;
-      const float ui = ub[tt][i], ki = kf[tt][i], dgi = gb[tt][i];
-      float mu4[4] = {0.f, 0.f, 0.f, 0.f}, pk4[4] = {0.f, 0.f, 0.f, 0.f}, mp4[4] = {0.f, 0.f, 0.f, 0.f};
+      float ui[R], ki[R], dgi[R];
 #pragma unroll
-      for (int m = 0; m < NV; ++m) {
-        const float4 u4 = vec4(ub[tt], m, q), k4 = vec4(kf[tt], m, q);
+      for (int r = 0; r < R; ++r) ui[r] = ub[tt][r0 + r], ki[r] = kf[tt][r0 + r], dgi[r] = gb[tt][r0 + r];
+      float mu4[R][4], pk4[R][4], mp4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mu4[r][e] = pk4[r][e] = 0.f;
+#pragma unroll
+      for (int m = 0; m < Sh::NM; ++m) {
+        const float4 u4 = vec4<G>(ub[tt], m, g), k4 = vec4<G>(kf[tt], m, g);
         const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 4 * m + e;
-          mu4[e] = fmaf(Mr[j], uu[e], mu4[e]);
-          pk4[e] = fmaf(Pp[j], kk[e], pk4[e]);
-          mp4[e] = fmaf(Mr[j], Pp[j], mp4[e]);
-        }
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int x = r * CW + 4 * m + e;
+            mu4[r][e] = fmaf(Mr[x], uu[e], mu4[r][e]);
+            pk4[r][e] = fmaf(Pp[x], kk[e], pk4[r][e]);
+            mp4[e] = fmaf(Mr[x], Pp[x], mp4[e]);
+          }
       }
-      float Mu = (mu4[0] + mu4[1]) + (mu4[2] + mu4[3]), Pk = (pk4[0] + pk4[1]) + (pk4[2] + pk4[3]);
-      const float MP = (mp4[0] + mp4[1]) + (mp4[2] + mp4[3]);
-      Mu += __shfl_xor_sync(0xffffffffu, Mu, 1);
-      Mu += __shfl_xor_sync(0xffffffffu, Mu, 2);
-      Pk += __shfl_xor_sync(0xffffffffu, Pk, 1);
-      Pk += __shfl_xor_sync(0xffffffffu, Pk, 2);
-      // every lane of a row holds u_i and the reduced Mu, so the row terms take each lane's quarter
-      float x0 = 0.25f * dgi * ui, x1 = 0.25f * ui * Mu, x2 = MP;
+      float Mu[R], Pk[R], x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        Mu[r] = group_sum<G>((mu4[r][0] + mu4[r][1]) + (mu4[r][2] + mu4[r][3]));
+        Pk[r] = group_sum<G>((pk4[r][0] + pk4[r][1]) + (pk4[r][2] + pk4[r][3]));
+        if (row_lead) x0 = fmaf(dgi[r], ui[r], x0), x1 = fmaf(ui[r], Mu[r], x1);
+      }
+      float x2 = (mp4[0] + mp4[1]) + (mp4[2] + mp4[3]);
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         x0 += __shfl_xor_sync(0xffffffffu, x0, o);
@@ -308,47 +354,58 @@ __global__ void __launch_bounds__(4 * D, 1) full_cov_backward_kernel(FullBwdArgs
       __syncthreads();
       const float dgu = sum_parts<NW>(part[b][0]), uMu = sum_parts<NW>(part[b][1]), MPs = sum_parts<NW>(part[b][2]);
       const float ds = (0.5f * uMu - dgu) * inv * inv;
-      const float dui = (dgi - Mu) * inv + ds * ki;
-      if (row_lead) dus[b][i] = dui;
-      float y0 = row_lead ? dui * Pk : 0.f, y1 = row_lead ? dui * ki : 0.f;
+      float dui[R], y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
+      for (int r = 0; r < R; ++r) {
+        dui[r] = (dgi[r] - Mu[r]) * inv + ds * ki[r];
+        if (row_lead) {
+          dus[b][r0 + r] = dui[r];
+          y0 = fmaf(dui[r], Pk[r], y0), y1 = fmaf(dui[r], ki[r], y1);
+        }
+      }
+#pragma unroll
+      for (int o = G; o < 32; o <<= 1) {
         y0 += __shfl_xor_sync(0xffffffffu, y0, o);
         y1 += __shfl_xor_sync(0xffffffffu, y1, o);
       }
       if (lane == 0) part2[b][0][warp] = y0, part2[b][1][warp] = y1;
       __syncthreads();
       const float duPk = sum_parts<NW>(part2[b][0]), duk = sum_parts<NW>(part2[b][1]);
-      float pd4[4] = {0.f, 0.f, 0.f, 0.f};
+      // P du and the update of M in one pass over this thread's columns of du and k
+      float pd4[R][4];
 #pragma unroll
-      for (int m = 0; m < NV; ++m) {
-        const float4 d4 = vec4(dus[b], m, q);
-        pd4[0] = fmaf(Pp[4 * m], d4.x, pd4[0]), pd4[1] = fmaf(Pp[4 * m + 1], d4.y, pd4[1]);
-        pd4[2] = fmaf(Pp[4 * m + 2], d4.z, pd4[2]), pd4[3] = fmaf(Pp[4 * m + 3], d4.w, pd4[3]);
+      for (int r = 0; r < R; ++r) pd4[r][0] = pd4[r][1] = pd4[r][2] = pd4[r][3] = 0.f;
+#pragma unroll
+      for (int m = 0; m < Sh::NM; ++m) {
+        const float4 k4 = vec4<G>(kf[tt], m, g), d4 = vec4<G>(dus[b], m, g);
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int x = r * CW + 4 * m + e;
+            pd4[r][e] = fmaf(Pp[x], dd[e], pd4[r][e]);
+            Mr[x] = a2 * (Mr[x] + fmaf(dui[r], kk[e], ki[r] * dd[e]));
+          }
       }
-      float Pdu = (pd4[0] + pd4[1]) + (pd4[2] + pd4[3]);
-      Pdu += __shfl_xor_sync(0xffffffffu, Pdu, 1);
-      Pdu += __shfl_xor_sync(0xffffffffu, Pdu, 2);
-      if (row_lead) p.dk[ti * D + i] = dkb[tt][i] + ds * ui + a2 * Pdu + qt * dui;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float Pdu = group_sum<G>((pd4[r][0] + pd4[r][1]) + (pd4[r][2] + pd4[r][3]));
+        if (row_lead) p.dk[ti * D + r0 + r] = dkb[tt][r0 + r] + ds * ui[r] + a2 * Pdu + qt * dui[r];
+      }
       if (tid == 0) {
         p.dr[ti] = ds;
         p.dqn[ti] = 0.5f * trM + duk;
         if (p.da != nullptr) p.da[ti] = sda[tt] + 2.f * at * (0.5f * MPs + duPk);
-      }
-#pragma unroll
-      for (int m = 0; m < NV; ++m) {
-        const float4 k4 = vec4(kf[tt], m, q), d4 = vec4(dus[b], m, q);
-        Mr[4 * m] = a2 * (Mr[4 * m] + fmaf(dui, k4.x, ki * d4.x));
-        Mr[4 * m + 1] = a2 * (Mr[4 * m + 1] + fmaf(dui, k4.y, ki * d4.y));
-        Mr[4 * m + 2] = a2 * (Mr[4 * m + 2] + fmaf(dui, k4.z, ki * d4.z));
-        Mr[4 * m + 3] = a2 * (Mr[4 * m + 3] + fmaf(dui, k4.w, ki * d4.w));
       }
       trM = a2 * (trM + 2.f * duk);
     }
     __syncthreads();  // the block's buffers are free for the next block
   }
 #pragma unroll
-  for (int j = 0; j < CW; ++j) p.dP0[((size_t)bh * D + i) * D + colof(q, j)] = 0.5f * Mr[j];
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < CW; ++j) p.dP0[((size_t)bh * D + r0 + r) * D + colof<G>(g, j)] = 0.5f * Mr[r * CW + j];
 }
 
 template <int D>
