@@ -447,6 +447,109 @@ __global__ void __launch_bounds__(kSelThreads) hola_cache_select_kernel(HolaArgs
   }
 }
 
+// hola_cache_scan_kernel: the same caches by a log-depth scan instead of the walk.  The cache block b reads is
+// the top w of blocks 0 .. b - 1, and the top w of a union of disjoint sets is the top w of the union of their
+// top w, so the lists combine associatively: an inclusive scan over the blocks (Hillis-Steele: at distance
+// d = 1, 2, 4, .. each block's list is merged with that of the block d before it) gives at block b the top w of
+// blocks 0 .. b, i.e. the cache of block b + 1.  An entry is one 64-bit key, larger first in rank order: m
+// mapped to an order-preserving unsigned word above INT_MAX - token (the rank order of `before`: larger m
+// first, ties to the earlier token; -0 is taken as +0), and the padding past a list's size is key 0 below every
+// token.  Every list is 64 keys in rank order, held by one warp as two keys per lane (positions lane and
+// lane + 32) and ordered by bitonic networks over the lanes: a block's own candidates by a full sort, a merge
+// of lists A and B as the bitonic sequence C_i = max(A_i, B_63-i) (exactly the 64 first of A u B) followed by
+// six half-cleaner stages.  Positions from w on are cleared to the padding.  One CTA of kScanThreads per head;
+// the lists are double-buffered in shared memory (2 x blocks x 64 keys), hence at most kScanMaxBlocks blocks.
+constexpr int kScanThreads = 1024;
+constexpr int kScanMaxBlocks = 192;
+
+__host__ __device__ constexpr size_t scan_smem_bytes(int nblocks) { return (size_t)nblocks * 2 * 64 * 8; }
+
+__device__ __forceinline__ unsigned long long rank_key(float m, int token) {
+  uint32_t u = __float_as_uint(m + 0.f);  // (-0 + 0 = +0)
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(0x7fffffff - token);
+}
+__device__ __forceinline__ int key_token(unsigned long long key) {
+  return key == 0ull ? -1 : 0x7fffffff - static_cast<int>(static_cast<uint32_t>(key));
+}
+
+// Bitonic stages j = jstart, jstart / 2, .., 1 of sub-sequence size k over the two keys at positions lane (x0)
+// and lane + 32 (x1): the lower position of each pair (pos, pos ^ j) keeps the larger key where the
+// sub-sequence runs in rank order (pos & k clear, or k = 64), the smaller one elsewhere.
+__device__ __forceinline__ void bitonic_stages(unsigned long long& x0, unsigned long long& x1, int k, int jstart,
+                                               int lane) {
+  for (int j = jstart; j >= 1; j >>= 1) {
+    unsigned long long y0, y1;
+    if (j == 32) {
+      y0 = x1, y1 = x0;
+    } else {
+      y0 = __shfl_xor_sync(0xffffffffu, x0, j);
+      y1 = __shfl_xor_sync(0xffffffffu, x1, j);
+    }
+    const int p0 = lane, p1 = lane + 32;
+    const bool w0 = ((p0 & j) == 0) == ((p0 & k) == 0 || k == 64);  // this position keeps the larger key
+    const bool w1 = ((p1 & j) == 0) == ((p1 & k) == 0 || k == 64);
+    x0 = (w0 == (y0 > x0)) ? y0 : x0;
+    x1 = (w1 == (y1 > x1)) ? y1 : x1;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) hola_cache_scan_kernel(HolaArgs p) {
+  extern __shared__ __align__(16) uint8_t scan_raw[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, bh = blockIdx.x, L = p.L, w = p.w;
+  constexpr int kWarps = kScanThreads / 32;
+  const int nblocks = (L + 63) / 64;
+  const size_t tok0 = (size_t)bh * L;
+  unsigned long long* lk = reinterpret_cast<unsigned long long*>(scan_raw);  // [2][nblocks][64] keys
+  auto at = [&](int buf, int b, int pos) -> unsigned long long& { return lk[(buf * nblocks + b) * 64 + pos]; };
+  auto put = [&](int buf, int b, unsigned long long x0, unsigned long long x1) {  // positions from w on: padding
+    at(buf, b, lane) = lane < w ? x0 : 0ull;
+    at(buf, b, lane + 32) = lane + 32 < w ? x1 : 0ull;
+  };
+  // each block's own candidates, sorted into rank order
+  for (int b = warp; b < nblocks; b += kWarps) {
+    const int t0 = 64 * b + lane, t1 = t0 + 32;
+    unsigned long long x0 = t0 < L ? rank_key(p.m[tok0 + t0], t0) : 0ull;
+    unsigned long long x1 = t1 < L ? rank_key(p.m[tok0 + t1], t1) : 0ull;
+    for (int k = 2; k <= 64; k <<= 1) bitonic_stages(x0, x1, k, k / 2, lane);
+    put(0, b, x0, x1);
+  }
+  __syncthreads();
+  int cur = 0;
+  for (int d = 1; d < nblocks; d <<= 1) {
+    for (int b = warp; b < nblocks; b += kWarps) {
+      unsigned long long x0 = at(cur, b, lane), x1 = at(cur, b, lane + 32);
+      if (b >= d) {  // C_i = max(A_i, B_63-i): A block b's list, B the list d blocks before
+        x0 = max(x0, at(cur, b - d, 63 - lane));
+        x1 = max(x1, at(cur, b - d, 31 - lane));
+        bitonic_stages(x0, x1, 64, 32, lane);
+      }
+      put(cur ^ 1, b, x0, x1);
+    }
+    cur ^= 1;
+    __syncthreads();
+  }
+  // block b reads the top w of blocks 0 .. b - 1, in rank order, -1 past its size
+  for (int e = tid; e < nblocks * 64; e += kScanThreads) {
+    const int b = e >> 6, r = e & 63;
+    p.cidx[((size_t)bh * nblocks + b) * 64 + r] = b > 0 ? key_token(at(cur, b - 1, r)) : -1;
+  }
+  if (p.cache != nullptr && tid < w) {  // the final cache, ascending token indices, -1 past its size
+    const int last = nblocks - 1;
+    const int mine = key_token(at(cur, last, tid));
+    if (mine >= 0) {
+      int pos = 0;
+      for (int c = 0; c < w; ++c) {
+        const int o = key_token(at(cur, last, c));
+        pos += (o >= 0 && o < mine) ? 1 : 0;
+      }
+      p.cache[(size_t)bh * w + pos] = mine;
+    } else {
+      p.cache[(size_t)bh * w + tid] = -1;
+    }
+  }
+}
+
 // hola_read_block_kernel: one CTA per head and run of kBlocksPerCta consecutive blocks, two CTAs per SM.  Each
 // block's q, k, v arrive by TMA, its cache rows by 16-byte cp.async gathers of the token indices chosen above
 // (rows 0..63; empty rows zero), then the same S product, softmax with the sink and P V product as the serial
@@ -712,7 +815,15 @@ cudaError_t launch_hola_read_tc(const HolaArgs& p, int BH, cudaStream_t stream) 
   cudaError_t e;
   if (p.cidx != nullptr) {  // every block's cache first, then all blocks at once
     if (p.w < 1 || p.w > 64) return cudaErrorInvalidValue;
-    hola_cache_select_kernel<<<BH, kSelThreads, 0, stream>>>(p);
+    const int nb = (p.L + 63) / 64;
+    if (nb <= kScanMaxBlocks) {
+      const size_t sb = scan_smem_bytes(nb);
+      e = cudaFuncSetAttribute(hola_cache_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+      if (e != cudaSuccess) return e;
+      hola_cache_scan_kernel<<<BH, kScanThreads, sb, stream>>>(p);
+    } else {
+      hola_cache_select_kernel<<<BH, kSelThreads, 0, stream>>>(p);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(hola_read_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);

@@ -113,3 +113,21 @@ def test_parallel_read_equals_the_block_by_block_walk(w, L):
     assert torch.equal(c_par, c_ser)
     assert normwise_err(o_par, _np(o_ser)) < 1e-5
     _check(x, m, gq, gk, sink, w, 64, TOL["bf16"])
+
+
+@pytest.mark.parametrize("w,L", [(64, 64 * 192), (9, 64 * 193 - 5)])
+def test_cache_scan_limit_and_the_walk_beyond_it(w, L):
+    """Up to 192 blocks every block's cache comes from the log-depth scan over the blocks' ranked lists,
+    beyond that from the serial walk over the blocks; both must give the caches (and o) of the block-by-block
+    read, ties in m included."""
+    wl = WORKLOADS["gdn_d128"]
+    x = make_scan_inputs(wl, seed=6, device=DEV, B=1, H=2, L=L)
+    m = torch.rand(1, 2, L, device=DEV)
+    m[0, 1, : L // 3] = 0.25
+    gq, gk, sink = _params(128, 2, 3)
+    small = torch.empty(256, dtype=torch.uint8, device=DEV)
+    o_par, c_par = kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=w)
+    o_ser, c_ser = kdn.hola_cache_read(x["q"], x["k"], x["v"], m, gq, gk, sink, w=w, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.equal(c_par, c_ser)
+    assert normwise_err(o_par, _np(o_ser)) < 1e-5
