@@ -267,9 +267,11 @@ KDN_EXPORT size_t kdn_backward_workspace_bytes(kdn_variant variant, const kdn_di
  * workspace: >= 256 bytes (the device status word, read with
  * kdn_read_device_status).  For bf16 q, k, v with d_k = d_v = 128 and blocks of
  * 64, a workspace of kdn_hola_workspace_bytes(dims) also holds the cache
- * indices of every block: the cache each block reads is chosen first (one
- * pass over m per head), then all blocks are read at once; with 256 bytes one
- * CTA per head walks the blocks in order.  Both give the same result. */
+ * indices of every block: the cache each block reads is chosen first (from m
+ * alone: up to 192 blocks by a log-depth scan of the blocks' ranked top-w
+ * lists, beyond that by one pass over the blocks per head), then all blocks
+ * are read at once; with 256 bytes one CTA per head walks the blocks in order.
+ * All give the same caches; m must not hold NaN. */
 KDN_EXPORT kdn_status kdn_hola_cache_read(const kdn_dims* dims, const void* q, const void* k, const void* v,
                                const float* m, const float* gamma_q, const float* gamma_k, const float* sink,
                                int w, float* o_cache, int* cache_idx, void* workspace, size_t workspace_bytes,
